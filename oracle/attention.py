@@ -1,0 +1,119 @@
+"""Unbiased inner-product scores and one-pass decode attention over the
+compressed cache.
+
+Test infrastructure only (see oracle/__init__.py).
+
+Score of query q against a compressed key (the audit's
+``TurboQuantProd.attention_score``, "turboquant/audit_claims.py" AUDIT 3,
+AUDIT 5, AUDIT 6; the query is rotated once and the estimate is corrected by
+the 1-bit QJL term, "TurboQuant" explainer, troisinh.com, "Ý tưởng cốt lõi"
+and "Giới hạn cần biết": the query rotation happens every step):
+
+    q~ = Pi q,  s^ = S q
+    score = nk16 * ( <q~, c[idx]> + kappa * rn16 * <s^, 2 sign - 1> ),
+    kappa = sqrt(pi/2) / d.
+
+By orthogonality <q~, c> = <q, Pi^T c> and <s^, sigma> = <q, S^T sigma>,
+so the score equals <q, k_hat> for the explicit reconstruction.
+
+Decode attention ("03. Results & Benchmarks", turboquant_cutile, "Latency
+Benchmarks": score, QJL correction, online softmax and V accumulation in one
+pass): for query head hq with KV head h = hq // G (consecutive grouping),
+logits = score / sqrt(d) over the len_b cached tokens (no mask), softmax,
+out = sum_n p_n v_hat_n with v_hat the group-dequantized values.  Reading: the
+output is float32-sized; the oracle works in float64.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .quant import dequantize_keys, dequantize_values, kappa
+
+
+def rotate_query(q: np.ndarray, pi: np.ndarray, s: np.ndarray):
+    """(Pi q, S q) for q [..., d]."""
+    q = np.asarray(q, np.float64)
+    return q @ np.asarray(pi, np.float64).T, q @ np.asarray(s, np.float64).T
+
+
+def qjl_term(sh: np.ndarray, sign, rn, d: int):
+    """QJL correction kappa * rn * <S q, 2 sign - 1> for sign bits [..., d]
+    and residual norm(s) rn; an unbiased estimate of <q, r>."""
+    sigma = 2.0 * np.asarray(sign, np.float64) - 1.0
+    return kappa(d) * np.asarray(rn, np.float64) * (sigma @ np.asarray(sh, np.float64))
+
+
+def score_keys(q: np.ndarray, idx, sign, nk16, rn16, pi, s, centroids) -> np.ndarray:
+    """Scores of one query [d] against n compressed keys -> [n]."""
+    q = np.asarray(q, np.float64)
+    d = q.shape[-1]
+    qt, sh = rotate_query(q, pi, s)
+    c = np.asarray(centroids, np.float64)[idx]            # [n, d]
+    mse = c @ qt
+    return np.asarray(nk16, np.float64) * (mse + qjl_term(sh, sign, rn16, d))
+
+
+def softmax_average(logits: np.ndarray, vhat: np.ndarray) -> np.ndarray:
+    """sum_n softmax(logits)_n vhat_n, max-subtracted, float64."""
+    m = np.max(logits)
+    p = np.exp(logits - m)
+    p = p / np.sum(p)
+    return p @ vhat
+
+
+def decode_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
+                        softmax_scale: float | None = None) -> np.ndarray:
+    """Decode attention for one sequence.
+
+    q   [H_q, d] query
+    rec logical cache fields of the sequence's cached tokens, each with a
+        leading [N, H_kv] (idx, sign, codes: [N, H_kv, d]; nk16, rn16:
+        [N, H_kv]; scale16, zero16: [N, H_kv, d/group])
+    Returns out [H_q, d] float64.
+    """
+    q = np.asarray(q, np.float64)
+    hq, d = q.shape
+    n, hkv = rec["nk16"].shape
+    if n == 0:
+        raise ValueError("decode needs at least one cached token")
+    g = hq // hkv
+    scale = 1.0 / np.sqrt(d) if softmax_scale is None else softmax_scale
+    out = np.zeros((hq, d))
+    for h in range(hkv):
+        vhat = dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
+                                 rec["zero16"][:, h], group)
+        for j in range(g):
+            qh = h * g + j
+            sc = score_keys(q[qh], rec["idx"][:, h], rec["sign"][:, h],
+                            rec["nk16"][:, h], rec["rn16"][:, h], pi, s, centroids)
+            out[qh] = softmax_average(sc * scale, vhat)
+    return out
+
+
+def brute_force_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids,
+                             group: int, softmax_scale: float | None = None) -> np.ndarray:
+    """softmax(K_hat q / sqrt d) V_hat over explicitly dequantized K and V
+    (the dequantize-then-matmul pattern of the audit's hybrid path, AUDIT 4)."""
+    q = np.asarray(q, np.float64)
+    hq, d = q.shape
+    n, hkv = rec["nk16"].shape
+    g = hq // hkv
+    scale = 1.0 / np.sqrt(d) if softmax_scale is None else softmax_scale
+    out = np.zeros((hq, d))
+    for h in range(hkv):
+        khat = dequantize_keys(rec["idx"][:, h], rec["sign"][:, h], rec["nk16"][:, h],
+                               rec["rn16"][:, h], pi, s, centroids)
+        vhat = dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
+                                 rec["zero16"][:, h], group)
+        for j in range(g):
+            qh = h * g + j
+            logits = (khat @ q[qh]) * scale
+            w = np.exp(logits - logits.max())
+            out[qh] = (w / w.sum()) @ vhat
+    return out
+
+
+def stack_heads(recs: list) -> dict:
+    """Combine per-head logical records (each [N, ...]) into [N, H_kv, ...]."""
+    return {k: np.stack([r[k] for r in recs], axis=1) for k in recs[0]}

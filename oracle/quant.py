@@ -1,0 +1,144 @@
+"""TurboQuant-prod key encoding and group quantization of values.
+
+Test infrastructure only (see oracle/__init__.py).
+
+Keys ("TurboQuant" explainer, troisinh.com, "Ý tưởng cốt lõi" and "Tại sao nó
+hoạt động"; "turboquant/audit_claims.py", AUDIT 1, AUDIT 5, AUDIT 6):
+  1. keep the norm nk = ||k||; work on the unit vector u = k / nk (the
+     distortion bound is stated for unit-norm vectors, AUDIT 5);
+  2. rotate: y = Pi u;
+  3. bucketize every coordinate against the Lloyd-Max decision boundaries:
+     idx_j = #{ i : t_i < y_j }   (a value on a boundary goes to the lower
+     cell; reading);
+  4. residual in the original space: r = u - Pi^T c, c_j = centroids[idx_j];
+  5. 1-bit QJL sketch of the residual: s_j = [ (S r)_j >= 0 ] (an exact zero
+     counts as +1; reading) and rn = ||r||;
+  6. store nk and rn as fp16, round-to-nearest-even (reading: fp16 norms make
+     the audit's 5.1x record accounting come out exactly; see accounting.py).
+  A zero key stores nk = rn = 0 and all-zero codes and signs.
+
+Values ("turboquant/audit_claims.py", AUDIT 1: ``value_bits``,
+``value_group_size``): asymmetric min/max quantization per group of
+``group`` contiguous channels of one token's head vector, no rotation.
+Reading: fp16 scale and zero per group, codes by round-half-even then clamp.
+Because these floating-point steps decide integers (the codes), the oracle
+takes them in float32, the precision the kernel uses, step by step:
+  mn, mx      = min, max of the group (exact)
+  zero16      = fp16(mn)
+  scale16     = fp16( f32( f32(mx - mn) / f32(2^vb - 1) ) )
+  code        = clamp( rint( f32( f32(v - zero16) / scale16 ) ), 0, 2^vb - 1 ),
+                0 when scale16 == 0
+  dequantized = code * scale16 + zero16
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def kappa(d: int) -> float:
+    """QJL estimator constant sqrt(pi/2) / m with m = d sketch rows."""
+    return math.sqrt(math.pi / 2.0) / d
+
+
+def fp16(x) -> np.ndarray:
+    """Round to fp16, nearest-even, returned as float64 values."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def bucketize(y: np.ndarray, boundaries: np.ndarray) -> np.ndarray:
+    """idx = number of boundaries strictly below y (ties go to the lower cell)."""
+    return np.searchsorted(np.asarray(boundaries, np.float64), y, side="left")
+
+
+def encode_keys(keys: np.ndarray, pi: np.ndarray, s: np.ndarray,
+                centroids: np.ndarray, boundaries: np.ndarray) -> dict:
+    """Encode a batch of key vectors [n, d] (any float dtype).
+
+    Returns a dict of logical fields:
+      idx   [n, d] int   Lloyd-Max cell indices
+      sign  [n, d] uint8 QJL sign bits (1 means +1)
+      nk16  [n]   fp16-rounded key norms (float64)
+      rn16  [n]   fp16-rounded residual norms (float64)
+      y     [n, d] rotated unit coordinates (float64, for boundary bands)
+      z     [n, d] S r (float64, for sign bands)
+      nk, rn [n]   unrounded norms
+    """
+    x = np.asarray(keys, dtype=np.float64)
+    pi = np.asarray(pi, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    cent = np.asarray(centroids, dtype=np.float64)
+    n, d = x.shape
+    nk = np.sqrt(np.sum(x * x, axis=1))
+    zero = nk == 0.0
+    u = np.where(zero[:, None], 0.0, x / np.where(zero, 1.0, nk)[:, None])
+    y = u @ pi.T                         # y = Pi u, row by row
+    idx = bucketize(y, boundaries)
+    c = cent[idx]
+    r = u - c @ pi                       # r = u - Pi^T c, row by row
+    rn = np.sqrt(np.sum(r * r, axis=1))
+    z = r @ s.T                          # z = S r, row by row
+    sign = (z >= 0.0).astype(np.uint8)
+    idx[zero] = 0
+    sign[zero] = 0
+    rn = np.where(zero, 0.0, rn)
+    return {"idx": idx, "sign": sign, "nk16": fp16(nk), "rn16": fp16(rn),
+            "y": y, "z": z, "nk": nk, "rn": rn}
+
+
+def encode_values(values: np.ndarray, value_bits: int, group: int) -> dict:
+    """Group-quantize value vectors [n, d].  Returns codes [n, d] int,
+    scale16 / zero16 [n, d/group] (float64 holding fp16 values) and the
+    float32 code coordinate t [n, d] (for half-integer bands)."""
+    v = np.asarray(values, dtype=np.float32)
+    n, d = v.shape
+    if d % group:
+        raise ValueError("d must be a multiple of the group size")
+    ng = d // group
+    vg = v.reshape(n, ng, group)
+    mn = vg.min(axis=2)
+    mx = vg.max(axis=2)
+    levels = np.float32(2 ** value_bits - 1)
+    zero16 = mn.astype(np.float16)
+    diff = (mx - mn).astype(np.float32)              # f32 subtraction
+    s32 = (diff / levels).astype(np.float32)         # f32 division
+    scale16 = s32.astype(np.float16)
+    z32 = zero16.astype(np.float32)[:, :, None]
+    sc32 = scale16.astype(np.float32)[:, :, None]
+    num = (vg - z32).astype(np.float32)              # f32 subtraction
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (num / sc32).astype(np.float32)          # f32 division
+    codes = np.clip(np.rint(t), 0, 2 ** value_bits - 1)
+    codes = np.where(sc32 == 0, 0, codes).astype(np.int64)
+    t = np.where(sc32 == 0, 0.0, t)
+    return {"codes": codes.reshape(n, d),
+            "scale16": scale16.astype(np.float64),
+            "zero16": zero16.astype(np.float64),
+            "t": t.reshape(n, d).astype(np.float64)}
+
+
+def dequantize_values(codes: np.ndarray, scale16: np.ndarray,
+                      zero16: np.ndarray, group: int) -> np.ndarray:
+    """v_hat = code * scale16 + zero16, per group, float64 [n, d]."""
+    codes = np.asarray(codes, np.float64)
+    n, d = codes.shape
+    sc = np.repeat(np.asarray(scale16, np.float64), group, axis=1)
+    ze = np.repeat(np.asarray(zero16, np.float64), group, axis=1)
+    return codes * sc + ze
+
+
+def dequantize_keys(idx: np.ndarray, sign: np.ndarray, nk16: np.ndarray,
+                    rn16: np.ndarray, pi: np.ndarray, s: np.ndarray,
+                    centroids: np.ndarray) -> np.ndarray:
+    """Explicit reconstruction k_hat = nk * (Pi^T c + kappa * rn * S^T (2s - 1))
+    [n, d] float64 (the audit's ``quantizer.dequantize(prod_q)``, AUDIT 2)."""
+    pi = np.asarray(pi, np.float64)
+    s = np.asarray(s, np.float64)
+    d = pi.shape[0]
+    c = np.asarray(centroids, np.float64)[idx]
+    sigma = 2.0 * np.asarray(sign, np.float64) - 1.0
+    mse = c @ pi                          # Pi^T c, row by row
+    qjl = sigma @ s                       # S^T sigma, row by row
+    return nk16[:, None] * (mse + kappa(d) * rn16[:, None] * qjl)
