@@ -1,0 +1,504 @@
+#!/usr/bin/env python3
+"""Benchmark: TurboQuant-prod compressed-KV decode on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batched|llama8b|qwen15b_16384|longctx]
+
+A step is one pass of the whole hot path over one batch: quantize-append of
+one new token per sequence (all KV heads) followed by one decode-attention
+step (query rotation, split-K one-pass attention over the compressed cache,
+combine).  The default workload is the batched decode case (batch 32,
+H_kv=8, H_q=32, d=128, ragged lengths uniform in [16384, 32768], 3-bit keys,
+2-bit values): the cache read per step (~630 MB) is larger than the 126 MB
+L2, so no flush is needed between steps.
+
+Multi-GPU (``torchrun --nproc-per-node N``): every rank holds its own batch
+(weak scaling, no data-path collective); the time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle (test infrastructure) on
+the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from kv_cache_quantization_turboquantprod_b200 import tq, workloads  # noqa: E402
+
+METRIC = "decode attn ctx-tokens/s & HBM GB/s vs ~8 TB/s; quantize Mvec/s (1 B200)"
+UNIT = "ctx-tokens/s"
+DECODE_SRC = os.path.join(ROOT, "kv_cache_quantization_turboquantprod_b200", "csrc")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _source_hash(files):
+    h = hashlib.sha256()
+    for f in sorted(files):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _decode_kernel_files():
+    return [os.path.join(DECODE_SRC, f) for f in sorted(os.listdir(DECODE_SRC))
+            if f.startswith("decode") or f in ("tq_common.cuh", "tq_kernels.h")]
+
+
+def _traffic_from_profile(kernel_hash):
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, if it was taken on this exact source; else None."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("source_hash") == kernel_hash:
+            return d
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.4)
+
+    def stop(self):
+        if self.proc is None:
+            return
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def _fill_cache(wl, layer, cache, device):
+    """Quantize-append every sequence's synthetic K/V (8192-token chunks)."""
+    nchunks = (wl.capacity + workloads.TOKEN_CHUNK - 1) // workloads.TOKEN_CHUNK
+    lens = [0] * wl.batch
+    for c in range(nchunks):
+        t0 = c * workloads.TOKEN_CHUNK
+        nnew = [max(0, min(wl.lengths[b] - t0, workloads.TOKEN_CHUNK)) for b in range(wl.batch)]
+        if max(nnew) == 0:
+            break
+        T = max(nnew)
+        ks, vs = [], []
+        for b in range(wl.batch):
+            k, v = workloads.kv_chunk(wl, b, c, device)
+            ks.append(k[:T])
+            vs.append(v[:T])
+        k = torch.stack(ks).contiguous()
+        v = torch.stack(vs).contiguous()
+        tq.tq_quantize_append(layer, cache, k, v, lens, nnew)
+        lens = [lens[b] + nnew[b] for b in range(wl.batch)]
+        del k, v, ks, vs
+    torch.cuda.synchronize()
+    return lens
+
+
+def run_ours(args, rank, world, device):
+    wl = workloads.by_name(args.workload)
+    _, pi32, s32 = workloads.layer_matrices(wl)
+    layer = tq.Layer(pi32, s32, wl.key_bits, wl.value_bits, device=device)
+    cache = tq.CompressedCache(layer, wl.batch, wl.h_kv, wl.capacity, device=device)
+    lengths = list(wl.lengths)
+    # leave one free slot per sequence for the per-step append
+    lengths = [min(n, wl.capacity - 1) for n in lengths]
+    wl_fill = workloads.scaled(wl, lengths=tuple(lengths), capacity=wl.capacity)
+    _fill_cache(wl_fill, layer, cache, device)
+
+    B, HQ, D, HKV = wl.batch, wl.h_q, wl.d, wl.h_kv
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1234 + rank)
+    dt = torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32
+    q = torch.randn((B, HQ, D), generator=gen, device=device).to(dt)
+    k_new = torch.randn((B, 1, HKV, D), generator=gen, device=device).to(dt)
+    v_new = torch.randn((B, 1, HKV, D), generator=gen, device=device).to(dt)
+    len_after = torch.tensor([n + 1 for n in lengths], dtype=torch.int32, device=device)
+    max_len = max(lengths) + 1
+    ws = tq.workspace_for(layer, cache, HQ, max_len, device=device)
+    out = torch.empty((B, HQ, D), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 1 + 3
+
+    def step(ev_pair=None):
+        tq.tq_quantize_append(layer, cache, k_new, v_new, lengths)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        tq.tq_decode_attention(layer, cache, q, len_after, max_len, out, ws)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", device.index or 0)))
+    if rank == 0:
+        sampler.start()
+    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(dec_events[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_events) / args.steps
+
+    # end to end through the public API with host buffers (pinned), H2D of the
+    # step's inputs and D2H of its output inside the timed region
+    q_h = q.cpu().pin_memory()
+    k_h = k_new.cpu().pin_memory()
+    v_h = v_new.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        tq.tq_quantize_append(layer, cache, k_d, v_d, lengths)
+        tq.tq_decode_attention(layer, cache, q_d, len_after, max_len, out, ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    ctx_tokens_step = float(sum(n + 1 for n in lengths))
+    rec_bytes = layer.record_bytes()
+    dec_bytes = ctx_tokens_step * HKV * rec_bytes
+
+    times = torch.tensor([elapsed_ms, e2e_ms, dec_ms], dtype=torch.float64, device=device)
+    toks = torch.tensor([ctx_tokens_step, dec_bytes], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(toks, op=torch.distributed.ReduceOp.SUM)
+    elapsed_ms, e2e_ms, dec_ms = times.tolist()
+    ctx_all, dec_bytes_all = toks.tolist()
+    if rank != 0:
+        return None
+
+    value = ctx_all * args.steps / (elapsed_ms / 1e3)
+    e2e_value = ctx_all * args.steps / (e2e_ms / 1e3)
+    peak, peak_kind = _peaks()
+    achieved = (dec_bytes_all / world) / (dec_ms / 1e3) / 1e9
+    khash = _source_hash(_decode_kernel_files())
+    prof = _traffic_from_profile(khash)
+    traffic = None
+    if prof is not None:
+        traffic = prof.get("dram_bytes_per_launch_scaled")
+    clocks = sampler.summary()
+    cpu = cpu_baseline(wl, pi32, s32, args) if (rank == 0 and world == 1 and not args.no_cpu) else None
+    h2d = q.numel() * q.element_size() + k_new.numel() * k_new.element_size() * 2
+    d2h = out.numel() * out.element_size()
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; bf16 K/V/q with lognormal channel scales and outlier channels; no model weights)",
+        "config": {
+            "workload": wl.name,
+            "batch_per_gpu": B, "h_kv": HKV, "h_q": HQ, "d": D,
+            "key_bits": wl.key_bits, "value_bits": wl.value_bits, "group": wl.group,
+            "capacity": wl.capacity, "ctx_tokens_per_step_per_gpu": ctx_tokens_step,
+            "lengths": "ragged uniform [16384, 32768]" if wl.name == "batched" else list(wl.lengths),
+            "step": "quantize-append 1 token/sequence + decode (qprep, split-K, combine)",
+            "l2": "no flush: each step streams the whole compressed cache (> 126 MB L2)",
+            "parallelism": f"dp{world} (independent batches per GPU)",
+        },
+        "decode_gbs": dec_bytes_all / world / (dec_ms / 1e3) / 1e9,
+        "decode_ms": dec_ms,
+        "record_bytes": rec_bytes,
+        "roofline": {
+            "kernel": "tq_decode_attention (qprep + split-K + combine, timed as one call)",
+            "bound": "hbm",
+            "achieved": achieved,
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": dec_bytes_all / world,
+        },
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if args.quantize and world == 1:
+        line["quantize"] = bench_quantize(args, device)
+    return line
+
+
+def bench_quantize(args, device):
+    """Quantize-append Mvec/s on one 8192-token chunk of the long-context
+    workload (batch 4, H_kv=8, 3+1-bit keys, 2-bit values)."""
+    wl = workloads.longctx()
+    _, pi32, s32 = workloads.layer_matrices(wl)
+    layer = tq.Layer(pi32, s32, wl.key_bits, wl.value_bits, device=device)
+    cap = 2 * workloads.TOKEN_CHUNK
+    cache = tq.CompressedCache(layer, wl.batch, wl.h_kv, cap, device=device)
+    ks, vs = [], []
+    for b in range(wl.batch):
+        k, v = workloads.kv_chunk(wl, b, 0, device)
+        ks.append(k)
+        vs.append(v)
+    k = torch.stack(ks).contiguous()
+    v = torch.stack(vs).contiguous()
+    lens = [workloads.TOKEN_CHUNK] * wl.batch
+    for _ in range(3):
+        tq.tq_quantize_append(layer, cache, k, v, lens)
+    torch.cuda.synchronize()
+    n = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        tq.tq_quantize_append(layer, cache, k, v, lens)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    vecs = wl.batch * workloads.TOKEN_CHUNK * wl.h_kv
+    in_bytes = k.numel() * k.element_size() * 2
+    out_bytes = vecs * layer.record_bytes()
+    return {"workload": "longctx chunk (4 x 8192 tokens x 8 heads, bf16)",
+            "ms_per_chunk": ms, "mvec_s": vecs / (ms / 1e3) / 1e6,
+            "gbs": (in_bytes + out_bytes) / (ms / 1e3) / 1e9,
+            "useful_tflops": vecs * 3 * 2 * 128 * 128 / (ms / 1e3) / 1e12}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(wl, pi32, s32, pairs, max_tokens):
+    """Prepare oracle-encoded records for sampled (b, h) pairs (not timed)."""
+    from oracle import attention, codebook, quant  # test infrastructure
+    pi = pi32.astype(np.float64)
+    s = s32.astype(np.float64)
+    cent, bnd, _ = codebook.lloyd_max_gaussian(wl.key_bits - 1, wl.d)
+    samples = []
+    for (b, h) in pairs:
+        n = min(wl.lengths[b], max_tokens)
+        k, v = workloads.kv_tokens(wl, b, 0, n, device="cpu")
+        ke = quant.encode_keys(k[:, h].float().numpy(), pi, s, cent, bnd)
+        ve = quant.encode_values(v[:, h].float().numpy(), wl.value_bits, wl.group)
+        rec = {"idx": ke["idx"][:, None], "sign": ke["sign"][:, None],
+               "nk16": ke["nk16"][:, None], "rn16": ke["rn16"][:, None],
+               "codes": ve["codes"][:, None], "scale16": ve["scale16"][:, None],
+               "zero16": ve["zero16"][:, None]}
+        q = workloads.queries(wl, 0, device="cpu")[b, h * wl.gqa:(h + 1) * wl.gqa].float().numpy()
+        samples.append((q, rec, n))
+    return samples, (pi, s, cent, attention)
+
+
+def _oracle_decode_samples(samples, consts, group):
+    pi, s, cent, attention = consts
+    for q, rec, _ in samples:
+        attention.decode_one_sequence(q, rec, pi, s, cent, group)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return None
+
+
+def cpu_baseline(wl, pi32, s32, args, budget_s=10.0):
+    """Time the oracle's decode on host cores over a bounded sample of the
+    workload: (b, h) pairs, each with all G query heads of that KV head."""
+    rng = np.random.default_rng(0)
+    pairs = [(int(rng.integers(wl.batch)), int(rng.integers(wl.h_kv))) for _ in range(64)]
+    max_tokens = 8192
+    samples, consts = _oracle_sample(wl, pi32, s32, pairs[:2], max_tokens)
+    t0 = time.perf_counter()
+    done_tokens = 0.0
+    i = 0
+    while True:
+        _oracle_decode_samples(samples, consts, wl.group)
+        done_tokens += sum(n for _, _, n in samples)
+        i += 1
+        if time.perf_counter() - t0 > budget_s or i >= 50:
+            break
+    dt = time.perf_counter() - t0
+    # a ctx-token covers all H_kv heads: a (b, h) pair's n tokens are n / H_kv ctx-tokens
+    value = done_tokens / wl.h_kv / dt
+    return {"value": value, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+            "blas_threads": _blas_threads(), "kind": "oracle",
+            "sample": f"oracle decode of 2 (sequence, KV head) pairs x {max_tokens} tokens "
+                      f"x {wl.gqa} query heads, repeated {i}x ({dt:.1f} s); "
+                      f"ctx-tokens counted as tokens / H_kv"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = workloads.by_name(args.workload)
+    _, pi32, s32 = workloads.layer_matrices(wl)
+    rng = np.random.default_rng(1)
+    pairs = [(int(rng.integers(wl.batch)), int(rng.integers(wl.h_kv))) for _ in range(4)]
+    max_tokens = 4096
+    samples, consts = _oracle_sample(wl, pi32, s32, pairs[:1], max_tokens)
+    for _ in range(args.warmup):
+        _oracle_decode_samples(samples, consts, wl.group)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_decode_samples(samples, consts, wl.group)
+    dt = time.perf_counter() - t0
+    tokens = sum(n for _, _, n in samples) * args.steps / wl.h_kv
+    value = tokens / dt
+    sample = (f"each step: oracle decode of 1 (sequence, KV head) pair x {max_tokens} tokens x "
+              f"{wl.gqa} query heads of the {wl.name} workload; ctx-tokens = tokens / H_kv")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
+                             "cores": len(os.sched_getaffinity(0)), "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="batched")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-quantize", dest="quantize", action="store_false",
+                    help="skip the quantize-append Mvec/s measurement")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=device)
+    tq.load()
+    try:
+        line = run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

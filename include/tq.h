@@ -1,0 +1,224 @@
+/*
+ * tq.h -- C ABI of the TurboQuant-prod compressed KV-cache library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (the pages' statement of the method):
+ *
+ *  - Keys ("TurboQuant" explainer, troisinh.com, "Ý tưởng cốt lõi";
+ *    "turboquant/audit_claims.py", AUDIT 1 and AUDIT 5): each key head
+ *    vector k is normalised, u = k / ||k||, rotated by a fixed random
+ *    orthogonal Pi, and every rotated coordinate is bucketized against a
+ *    (key_bits - 1)-bit Lloyd-Max codebook fitted to N(0, 1/d).  The
+ *    residual r = u - Pi^T c (c the centroids of the chosen cells) is kept
+ *    as 1-bit QJL signs sign(S r) plus ||r||.  ||k|| and ||r|| are stored
+ *    as fp16.
+ *  - Values (AUDIT 1: value_bits, value_group_size): asymmetric min/max
+ *    quantization per group of 32 channels with fp16 scale and zero.
+ *  - Decode ("03. Results & Benchmarks", turboquant_cutile, "Latency
+ *    Benchmarks"): one pass over the compressed cache with the query
+ *    rotated once (Pi q, S q); each score is the centroid-lookup inner
+ *    product scaled by ||k|| plus the unbiased QJL correction
+ *    ||k|| * ||r|| * sqrt(pi/2)/d * <S q, 2 sign - 1>; then softmax and the
+ *    group-dequantized value accumulation.  Split-K over the sequence with a
+ *    separate combine step.
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller owns every buffer and the stream.  The library
+ *    allocates no memory, never synchronises, and keeps no state beyond a
+ *    cached per-device SM count.
+ *  - Pointers documented as "device" must be device (or managed) memory of
+ *    the current CUDA device; "host" pointers are read before the call
+ *    returns.
+ *  - Errors: arguments are validated on the host before any launch; a bad
+ *    argument returns a status and launches nothing.  A launch failure
+ *    returns TQ_ERR_CUDA (from cudaGetLastError).  Kernels never trap; an
+ *    asynchronous fault surfaces at the caller's next synchronisation.
+ *  - Calls are asynchronous on `stream` and re-entrant.  Calls that write
+ *    the same cache region (or the same workspace) must be ordered by the
+ *    caller.
+ *  - Only d = 128 and group = 32 are built; other values return
+ *    TQ_ERR_UNSUPPORTED.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *tq_stream_t;
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad alignment */
+  TQ_ERR_UNSUPPORTED = 2,      /* d, group, bit width or dtype not built */
+  TQ_ERR_CAPACITY = 3,         /* len + n_new > capacity, batch too large */
+  TQ_ERR_WORKSPACE = 4,        /* workspace missing or too small */
+  TQ_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
+  TQ_ERR_INTERNAL = 6
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* Tokens per cache tile; capacity must be a multiple of it. */
+#define TQ_TILE_TOKENS 128
+/* Largest batch tq_quantize_append takes (its lengths travel as kernel
+ * parameters). */
+#define TQ_MAX_BATCH 1024
+
+/* Human-readable name of a status code (static string). */
+TQ_API const char *tq_status_string(tq_status s);
+
+/*
+ * tq_make_codebook -- host only, deterministic.
+ *
+ * Lloyd-Max scalar quantizer for N(0, 1/d) with 2^mse_bits levels: the
+ * MSE-optimal codebook for a rotated coordinate (explainer, "Ý tưởng cốt
+ * lõi" and "Tại sao nó hoạt động"; the audit's mse_quantizer keeps
+ * centroids and decision boundaries, AUDIT 1).  Lloyd's iteration
+ * (boundary = midpoint of neighbouring centroids, centroid = conditional
+ * mean of its cell) in double precision until no centroid moves by more
+ * than 1e-14 / sqrt(d).
+ *
+ *   mse_bits    1..4
+ *   d           > 0
+ *   centroids   host, [2^mse_bits] doubles, written ascending
+ *   boundaries  host, [2^mse_bits - 1] doubles, written ascending
+ * Returns TQ_ERR_INVALID_ARGUMENT for a null pointer, TQ_ERR_UNSUPPORTED
+ * for mse_bits outside 1..4 or d < 1.
+ */
+TQ_API tq_status tq_make_codebook(int mse_bits, int d, double *centroids,
+                           double *boundaries);
+
+/* Constants of one layer.  All pointers: device, fp32, read-only, owned by
+ * the caller, alive for the duration of every call that uses them. */
+typedef struct {
+  int d;          /* head dimension; 128 */
+  int key_bits;   /* 2..4 total key bits: key_bits - 1 Lloyd-Max bits + 1 QJL bit */
+  int value_bits; /* 2..4 */
+  int group;      /* value quantization group; 32 */
+  const float *pi;         /* [d][d] row-major: Pi, y = Pi u */
+  const float *s;          /* [d][d] row-major: S, QJL sketch of r is S r */
+  const float *centroids;  /* [2^(key_bits-1)] ascending */
+  const float *boundaries; /* [2^(key_bits-1) - 1] ascending decision boundaries */
+} tq_params;
+
+/*
+ * One layer's compressed cache: a single caller-owned device buffer.
+ *
+ * Layout (the pages fix none; this is the library's):
+ *  - For every sequence b and KV head h (b-major, then h), capacity/128
+ *    tiles of 128 tokens; tile (b, h, t) starts at byte
+ *    ((b * h_kv + h) * (capacity / 128) + t) * tile_bytes.
+ *  - A tile holds, in order, for its 128 token slots:
+ *      1. key code bit-planes: (key_bits - 1) planes, each [128][d/8] bytes;
+ *         plane p holds bit p of each coordinate's Lloyd-Max cell index;
+ *      2. QJL sign plane [128][d/8]; bit 1 means sign +1 ((S r)_j >= 0);
+ *      3. value code bit-planes: value_bits planes, [128][d/8] each;
+ *      4. norms [128] x {||k||, ||r||}, two little-endian fp16 per token;
+ *      5. value groups [128][d/group] x {scale, zero}, two fp16 each.
+ *    In a plane row, byte i bit k (LSB first) is coordinate 8 i + k.
+ *  - Record bytes per (token, KV head) R = (key_bits + value_bits) d/8 + 4
+ *    + 4 d/group (100 bytes for 3-bit keys and 2-bit values at d = 128);
+ *    tile_bytes = 128 R.
+ *  - data must be 256-byte aligned.  Slots beyond a sequence's length may
+ *    hold anything; they are never read by decode.
+ */
+typedef struct {
+  int batch;    /* sequences */
+  int h_kv;     /* KV heads */
+  int capacity; /* token slots per sequence, multiple of 128 */
+  void *data;   /* device, tq_cache_bytes() bytes */
+} tq_cache;
+
+/* Bytes per (token, KV head) record R, or 0 for unsupported params. */
+TQ_API size_t tq_record_bytes(const tq_params *p);
+
+/* Bytes of a cache buffer for the given shape, or 0 for bad arguments. */
+TQ_API size_t tq_cache_bytes(const tq_params *p, int batch, int h_kv, int capacity);
+
+/*
+ * tq_quantize_append -- compress T new tokens of every sequence and write
+ * them at the end of the sequence (the store's append_chunk(k, v),
+ * "turboquant/audit_claims.py", AUDIT 1).
+ *
+ *   k, v        device, [batch][T][h_kv][d] contiguous, `dtype` (F32 or
+ *               BF16), 16-byte aligned
+ *   T           tokens per sequence in k and v (>= 0; 0 is a no-op)
+ *   len_host    host, [batch]: current length of each sequence; token t of
+ *               sequence b is written at position len_host[b] + t
+ *   n_new_host  host, [batch] or NULL: tokens of sequence b to take
+ *               (<= T); NULL takes all T for every sequence
+ * The caller advances its lengths afterwards; the library keeps none.
+ * Errors: TQ_ERR_CAPACITY if len + n_new > capacity for any sequence or
+ * batch > TQ_MAX_BATCH; TQ_ERR_INVALID_ARGUMENT for null pointers,
+ * negative sizes or misalignment; TQ_ERR_UNSUPPORTED for params.
+ * A zero key stores ||k|| = ||r|| = 0 with all-zero codes and signs.
+ * Norms above the fp16 range (65504) are not representable (unsupported).
+ */
+TQ_API tq_status tq_quantize_append(const tq_params *p, const tq_cache *c,
+                             const void *k, const void *v, tq_dtype dtype,
+                             int T, const int32_t *len_host,
+                             const int32_t *n_new_host, tq_stream_t stream);
+
+/*
+ * Workspace bytes tq_decode_attention needs for these shapes (the rotated
+ * queries and the split-K partial softmax states).  0 for bad arguments.
+ */
+TQ_API size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c,
+                                int h_q, int max_len);
+
+/*
+ * tq_decode_attention -- one decode step of attention over the compressed
+ * cache, in one pass over the packed records, split over the sequence
+ * (split-K) and merged by a log-sum-exp combine.
+ *
+ *   q              device, [batch][h_q][d], q_dtype (F32 or BF16)
+ *   h_q            query heads; a multiple of h_kv; query head hq reads KV
+ *                  head hq / (h_q / h_kv)
+ *   len_dev        device, [batch] int32: cached tokens of each sequence;
+ *                  a sequence with length 0 gets a zero output row
+ *   max_len        host: an upper bound of every len_dev[b] (used to size
+ *                  the split grid), 0 <= max_len <= capacity; tokens at or
+ *                  beyond max_len are not read
+ *   softmax_scale  logits = score * softmax_scale (1/sqrt(d) is the
+ *                  standard choice); must be finite
+ *   out            device, [batch][h_q][d] fp32
+ *   workspace      device, >= tq_decode_workspace_size(p, c, h_q, max_len)
+ *                  bytes, 256-byte aligned; contents need no initialisation
+ * Errors: TQ_ERR_WORKSPACE if the workspace is missing or too small;
+ * TQ_ERR_INVALID_ARGUMENT / TQ_ERR_UNSUPPORTED as for the other calls.
+ */
+TQ_API tq_status tq_decode_attention(const tq_params *p, const tq_cache *c,
+                              const void *q, tq_dtype q_dtype, int h_q,
+                              const int32_t *len_dev, int max_len,
+                              float softmax_scale, float *out, void *workspace,
+                              size_t workspace_bytes, tq_stream_t stream);
+
+/*
+ * tq_dequantize -- explicit reconstruction of cached tokens [start,
+ * start + count) of sequence b (the audit's quantizer.dequantize(prod_q),
+ * AUDIT 2):  k_hat = ||k|| (Pi^T c + sqrt(pi/2)/d ||r|| S^T (2 sign - 1)),
+ * v_hat = code * scale + zero.  Off the decode path; for tests and tools.
+ *
+ *   k_out, v_out  device, [count][h_kv][d] fp32 each
+ */
+TQ_API tq_status tq_dequantize(const tq_params *p, const tq_cache *c, int b,
+                        int start, int count, float *k_out, float *v_out,
+                        tq_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* TQ_H_ */

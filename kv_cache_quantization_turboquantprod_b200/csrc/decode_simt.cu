@@ -1,0 +1,217 @@
+// Decode attention over the compressed cache, SIMT form: qprep (rotate the
+// query once), split-K one-pass attention, log-sum-exp combine.
+//
+// Score of a cached key ("turboquant/audit_claims.py" attention_score,
+// AUDIT 3/5/6; "TurboQuant" explainer, troisinh.com, "Ý tưởng cốt lõi"):
+//   score = ||k|| * ( <Pi q, c[idx]> + sqrt(pi/2)/d * ||r|| * <S q, 2 sign - 1> )
+// One pass per split ("03. Results & Benchmarks", turboquant_cutile,
+// "Latency Benchmarks": score, QJL correction, online softmax and V
+// accumulation in one pass): logits = score * softmax_scale, online softmax
+// (base 2), acc += p * (code * scale + zero).
+#include <math.h>
+
+#include "tq_common.cuh"
+#include "tq_kernels.h"
+
+namespace tq {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxG = 8;
+
+// ---------------------------------------------------------------------------
+// qprep: qrot[b][hq][0][:] = Pi q, qrot[b][hq][1][:] = S q   (fp32)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qprep_kernel(DecodeArgs a) {
+  const int bh = blockIdx.x;  // b * h_q + hq
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float qv[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) qv[m] = load_elem(a.q, a.q_dtype, (size_t)bh * kD + lane + 32 * m);
+  float *dst = a.qrot + (size_t)bh * 2 * kD;
+  for (int o = warp; o < 2 * kD; o += 8) {
+    const float *row = (o < kD) ? (a.pi + (size_t)o * kD) : (a.s + (size_t)(o - kD) * kD);
+    float acc = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc = fmaf(row[lane + 32 * m], qv[m], acc);
+    acc = warp_sum(acc);
+    if (lane == 0) dst[o] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split-K: one CTA per (split, h_kv, b); 4 warps stride over the split's
+// tokens; a lane owns 4 consecutive dims (one nibble of every plane row).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = a.h_q / a.h_kv;
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  const float kappa = qjl_kappa();
+  const float scale2 = a.softmax_scale * kLog2e;
+
+  __shared__ float cent[16];
+  __shared__ float sm_m[4][kMaxG], sm_l[4][kMaxG];
+  __shared__ float sm_acc[4][kMaxG][kD];
+  if (threadIdx.x < (1 << L.mb)) cent[threadIdx.x] = a.centroids[threadIdx.x];
+
+  float qt[kMaxG][4], sh[kMaxG][4], acc[kMaxG][4], mrun[kMaxG], lrun[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    mrun[g] = -INFINITY;
+    lrun[g] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[g][k] = 0.f;
+      if (g < G) {
+        const float *src = a.qrot + ((size_t)b * a.h_q + h * G + g) * 2 * kD;
+        qt[g][k] = src[4 * lane + k];
+        sh[g][k] = src[kD + 4 * lane + k];
+      } else {
+        qt[g][k] = sh[g][k] = 0.f;
+      }
+    }
+  }
+  __syncthreads();
+
+  int len = a.len[b];
+  len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
+  const int t0 = s * a.tiles_per_split * kTile;
+  const int t1 = min(len, (s + 1) * a.tiles_per_split * kTile);
+  const int byte = lane >> 1, shift = (lane & 1) * 4;
+  const int grp = lane >> 3;
+
+  for (int n = t0 + warp; n < t1; n += 4) {
+    const uint8_t *tp = tile_ptr(const_cast<void *>(a.data), L, a.h_kv, a.ntiles, b, h, n / kTile);
+    const int slot = n % kTile;
+    int idx[4] = {0, 0, 0, 0};
+    for (int p = 0; p < L.mb; ++p) {
+      const int nib = (tp[L.kplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> shift) & 0xF;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) idx[k] |= ((nib >> k) & 1) << p;
+    }
+    const int snib = (tp[L.signs + slot * kRowBytes + byte] >> shift) & 0xF;
+    int code[4] = {0, 0, 0, 0};
+    for (int p = 0; p < L.vb; ++p) {
+      const int nib = (tp[L.vplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> shift) & 0xF;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) code[k] |= ((nib >> k) & 1) << p;
+    }
+    const __half2 nr = *reinterpret_cast<const __half2 *>(tp + L.norms + slot * 4);
+    const float nk = __low2float(nr), rn = __high2float(nr);
+    const __half2 sz = *reinterpret_cast<const __half2 *>(tp + L.vsz + (slot * kGroups + grp) * 4);
+    const float vs = __low2float(sz), vz = __high2float(sz);
+    float c[4], sg[4], vh[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      c[k] = cent[idx[k]];
+      sg[k] = ((snib >> k) & 1) ? 1.f : -1.f;
+      vh[k] = fmaf((float)code[k], vs, vz);
+    }
+    const float krn = kappa * rn;
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g >= G) break;
+      float mse = 0.f, qjl = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mse = fmaf(qt[g][k], c[k], mse);
+        qjl = fmaf(sh[g][k], sg[k], qjl);
+      }
+      const float part = warp_sum(fmaf(krn, qjl, mse));
+      const float l2 = nk * part * scale2;
+      const float mnew = fmaxf(mrun[g], l2);
+      const float corr = exp2f(mrun[g] - mnew);
+      const float p = exp2f(l2 - mnew);
+      lrun[g] = fmaf(lrun[g], corr, p);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[g][k] = fmaf(acc[g][k], corr, p * vh[k]);
+      mrun[g] = mnew;
+    }
+  }
+
+  // merge the 4 warps' states
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    if (g >= G) break;
+    if (lane == 0) { sm_m[warp][g] = mrun[g]; sm_l[warp][g] = lrun[g]; }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sm_acc[warp][g][4 * lane + k] = acc[g][k];
+  }
+  __syncthreads();
+  const int j = threadIdx.x;  // one dim per thread
+  for (int g = 0; g < G; ++g) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w][g]);
+    float Lsum = 0.f, A = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float f = exp2f(sm_m[w][g] - M);
+        Lsum = fmaf(sm_l[w][g], f, Lsum);
+        A = fmaf(sm_acc[w][g][j], f, A);
+      }
+    }
+    float *dst = a.part + (((size_t)b * a.h_q + h * G + g) * a.nsplit + s) * (kD + 2);
+    dst[j] = A;
+    if (j == 0) { dst[kD] = M; dst[kD + 1] = Lsum; }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// combine: out[b][hq][:] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
+  const int bh = blockIdx.x;
+  const int j = threadIdx.x;
+  const float *src = a.part + (size_t)bh * a.nsplit * (kD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, src[s * (kD + 2) + kD]);
+  float num = 0.f, den = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < a.nsplit; ++s) {
+      const float f = exp2f(src[s * (kD + 2) + kD] - M);
+      num = fmaf(src[s * (kD + 2) + j], f, num);
+      den = fmaf(src[s * (kD + 2) + kD + 1], f, den);
+    }
+  }
+  a.out[(size_t)bh * kD + j] = den > 0.f ? num / den : 0.f;
+}
+
+}  // namespace
+
+DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms) {
+  DecodePlan P;
+  const int ntile = (max_len + kTile - 1) / kTile;
+  const long long units = (long long)batch * h_kv;
+  const long long target = 4LL * num_sms;
+  long long ns = (target + units - 1) / units;
+  ns = std::max(1LL, std::min(ns, (long long)std::max(ntile, 1)));
+  int tps = ntile > 0 ? (int)((ntile + ns - 1) / ns) : 0;
+  int nsplit = tps > 0 ? (ntile + tps - 1) / tps : 1;
+  P.nsplit = nsplit;
+  P.tiles_per_split = tps;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  P.qrot_bytes = al((size_t)batch * h_q * 2 * kD * sizeof(float));
+  P.part_bytes = al((size_t)batch * h_q * nsplit * (kD + 2) * sizeof(float));
+  P.total_bytes = P.qrot_bytes + P.part_bytes;
+  return P;
+}
+
+cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream) {
+  const int bhq = a.batch * a.h_q;
+  qprep_kernel<<<bhq, 256, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nsplit, a.h_kv, a.batch);
+  decode_splitk_simt_kernel<<<grid, 128, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  combine_kernel<<<bhq, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,56 @@
+// Explicit reconstruction of cached tokens (the audit's
+// quantizer.dequantize(prod_q), "turboquant/audit_claims.py", AUDIT 2):
+//   k_hat = ||k|| * (Pi^T c + sqrt(pi/2)/d * ||r|| * S^T (2 sign - 1))
+//   v_hat = code * scale + zero
+// One CTA per (token, KV head); thread j produces output coordinate j by
+// walking column j of Pi and S (coalesced across threads).
+#include "tq_common.cuh"
+#include "tq_kernels.h"
+
+namespace tq {
+
+namespace {
+
+__global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
+  const int i = blockIdx.x;   // token offset in [0, count)
+  const int h = blockIdx.y;
+  const int j = threadIdx.x;
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  const int n = a.start + i;
+  const uint8_t *tp = tile_ptr(const_cast<void *>(a.data), L, a.h_kv, a.ntiles, a.b, h, n / kTile);
+  const int slot = n % kTile;
+  __shared__ float c[kD], sg[kD];
+  const int byte = j >> 3, bit = j & 7;
+  int idx = 0;
+  for (int p = 0; p < L.mb; ++p)
+    idx |= ((tp[L.kplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> bit) & 1) << p;
+  const int sbit = (tp[L.signs + slot * kRowBytes + byte] >> bit) & 1;
+  int code = 0;
+  for (int p = 0; p < L.vb; ++p)
+    code |= ((tp[L.vplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> bit) & 1) << p;
+  c[j] = a.centroids[idx];
+  sg[j] = sbit ? 1.f : -1.f;
+  __syncthreads();
+  const __half2 nr = *reinterpret_cast<const __half2 *>(tp + L.norms + slot * 4);
+  const float nk = __low2float(nr), rn = __high2float(nr);
+  float mse = 0.f, qjl = 0.f;
+  for (int r = 0; r < kD; ++r) {
+    mse = fmaf(a.pi[(size_t)r * kD + j], c[r], mse);
+    qjl = fmaf(a.s[(size_t)r * kD + j], sg[r], qjl);
+  }
+  const size_t o = ((size_t)i * a.h_kv + h) * kD + j;
+  a.k_out[o] = nk * fmaf(qjl_kappa() * rn, qjl, mse);
+  const __half2 sz = *reinterpret_cast<const __half2 *>(tp + L.vsz + (slot * kGroups + j / kGroup) * 4);
+  a.v_out[o] = fmaf((float)code, __low2float(sz), __high2float(sz));
+}
+
+}  // namespace
+
+cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t stream) {
+  if (a.count <= 0) return cudaSuccess;
+  dim3 grid(a.count, a.h_kv);
+  dequantize_kernel<<<grid, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,271 @@
+// quantize_append, SIMT form: TurboQuant-prod key encoding and value group
+// quantization of new tokens, written straight into the tiled cache.
+//
+// Keys ("TurboQuant" explainer, troisinh.com, "Ý tưởng cốt lõi";
+// "turboquant/audit_claims.py", AUDIT 1 / AUDIT 5): u = k/||k||, y = Pi u,
+// idx = #{boundaries < y}, r = u - Pi^T c, signs = [S r >= 0], ||r||.
+// Values (AUDIT 1, value_bits / value_group_size): per 32-channel group
+// min/max, fp16 zero = min, fp16 scale = (max-min)/(2^vb - 1) computed in
+// fp32, code = clamp(rint((v - zero)/scale)).
+//
+// A persistent CTA keeps Pi and S in shared memory (rows padded to 129
+// floats so both row- and column-direction walks are bank-conflict free) and
+// encodes 16 vectors per pass: three 128x128 mat-vecs per vector (Pi u,
+// Pi^T c, S r) in fp32 with exact fp32 accumulation order per output.
+#include "tq_common.cuh"
+#include "tq_kernels.h"
+
+namespace tq {
+
+namespace {
+
+constexpr int kNV = 16;              // vectors per pass
+constexpr int kThreads = 256;
+constexpr int kPad = kD + 1;         // padded row stride of Pi / S in smem
+constexpr int kMatFloats = kD * kPad;
+
+struct QuantSmem {
+  float pi[kMatFloats];
+  float s[kMatFloats];
+  float u[kNV][kD];
+  float c[kNV][kD];
+  float r[kNV][kD];
+  float rn2[kNV][4];
+  float nk[kNV];
+  float cent[16];
+  float bnd[16];
+};
+
+__device__ __forceinline__ void vec_coords(const AppendArgs &a, long long id, int &b,
+                                           int &t, int &h, bool &valid) {
+  const long long per_b = (long long)a.T * a.h_kv;
+  const long long total = (long long)a.batch * per_b;
+  valid = id < total;
+  if (!valid) { b = t = h = 0; return; }
+  b = (int)(id / per_b);
+  long long rem = id - (long long)b * per_b;
+  t = (int)(rem / a.h_kv);
+  h = (int)(rem - (long long)t * a.h_kv);
+  valid = t < a.nnew[b];
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  QuantSmem &S = *reinterpret_cast<QuantSmem *>(smem_raw);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  const int ncent = 1 << L.mb;
+
+  for (int i = tid; i < kD * kD; i += kThreads) {
+    const int r = i / kD, cc = i % kD;
+    S.pi[r * kPad + cc] = a.pi[i];
+    S.s[r * kPad + cc] = a.s[i];
+  }
+  if (tid < ncent) S.cent[tid] = a.centroids[tid];
+  if (tid < ncent - 1) S.bnd[tid] = a.boundaries[tid];
+  __syncthreads();
+
+  const long long total = (long long)a.batch * a.T * a.h_kv;
+  const long long nchunks = (total + kNV - 1) / kNV;
+  const float vlevels = (float)((1 << a.value_bits) - 1);
+
+  for (long long chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
+    const long long id0 = chunk * kNV;
+
+    // ---- phase 0: load, normalise keys; quantize values ----------------
+    for (int vi = warp; vi < kNV; vi += kThreads / 32) {
+      int b, t, h;
+      bool valid;
+      vec_coords(a, id0 + vi, b, t, h, valid);
+      float x[4];
+      float ss = 0.f;
+      const size_t base = valid ? ((((size_t)b * a.T + t) * a.h_kv + h) * kD) : 0;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        x[m] = valid ? load_elem(a.k, a.dtype, base + lane + 32 * m) : 0.f;
+        ss = fmaf(x[m], x[m], ss);
+      }
+      ss = warp_sum(ss);
+      const float nk = sqrtf(ss);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) S.u[vi][lane + 32 * m] = nk > 0.f ? __fdiv_rn(x[m], nk) : 0.f;
+      if (lane == 0) S.nk[vi] = nk;
+
+      if (valid) {
+        const int pos = a.lens[b] + t;
+        uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
+        const int slot = pos % kTile;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float vv = load_elem(a.v, a.dtype, base + lane + 32 * m);
+          const float mn = warp_min(vv);
+          const float mx = warp_max(vv);
+          const __half zero16 = __float2half_rn(mn);
+          const float s32 = __fdiv_rn(__fsub_rn(mx, mn), vlevels);
+          const __half scale16 = __float2half_rn(s32);
+          const float z32 = __half2float(zero16);
+          const float sc32 = __half2float(scale16);
+          int code = 0;
+          if (sc32 != 0.f) {
+            float tq = rintf(__fdiv_rn(__fsub_rn(vv, z32), sc32));
+            tq = fminf(fmaxf(tq, 0.f), vlevels);
+            code = (int)tq;
+          }
+          for (int p = 0; p < L.vb; ++p) {
+            const unsigned word = __ballot_sync(0xffffffffu, (code >> p) & 1);
+            if (lane == 0)
+              *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * kPlaneBytes +
+                                            slot * kRowBytes + 4 * m) = word;
+          }
+          if (lane == 0) {
+            __half2 sz = __halves2half2(scale16, zero16);
+            *reinterpret_cast<__half2 *>(tile + L.vsz + (slot * kGroups + m) * 4) = sz;
+          }
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- phase 1: y = Pi u, bucketize, pack code planes ------------------
+    {
+      const int i = tid & (kD - 1);
+      const int v0 = (tid >> 7) * (kNV / 2);
+      float acc[kNV / 2];
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) acc[v] = 0.f;
+      for (int j = 0; j < kD; j += 4) {
+        const float w0 = S.pi[i * kPad + j], w1 = S.pi[i * kPad + j + 1];
+        const float w2 = S.pi[i * kPad + j + 2], w3 = S.pi[i * kPad + j + 3];
+#pragma unroll
+        for (int v = 0; v < kNV / 2; ++v) {
+          const float4 uu = *reinterpret_cast<const float4 *>(&S.u[v0 + v][j]);
+          acc[v] = fmaf(w0, uu.x, acc[v]);
+          acc[v] = fmaf(w1, uu.y, acc[v]);
+          acc[v] = fmaf(w2, uu.z, acc[v]);
+          acc[v] = fmaf(w3, uu.w, acc[v]);
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) {
+        const int vi = v0 + v;
+        int b, t, h;
+        bool valid;
+        vec_coords(a, id0 + vi, b, t, h, valid);
+        int idx = 0;
+        for (int q = 0; q < ncent - 1; ++q) idx += (S.bnd[q] < acc[v]) ? 1 : 0;
+        const bool zero = !(S.nk[vi] > 0.f);
+        if (zero) idx = 0;
+        S.c[vi][i] = zero ? 0.f : S.cent[idx];
+        if (valid) {
+          const int pos = a.lens[b] + t;
+          uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
+          const int slot = pos % kTile;
+          for (int p = 0; p < L.mb; ++p) {
+            const unsigned word = __ballot_sync(0xffffffffu, (idx >> p) & 1);
+            if (lane == 0)
+              *reinterpret_cast<uint32_t *>(tile + L.kplanes + p * kPlaneBytes +
+                                            slot * kRowBytes + 4 * (i >> 5)) = word;
+          }
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- phase 2: r = u - Pi^T c, partial ||r||^2 -------------------------
+    {
+      const int j = tid & (kD - 1);
+      const int v0 = (tid >> 7) * (kNV / 2);
+      float acc[kNV / 2];
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) acc[v] = 0.f;
+      for (int i = 0; i < kD; i += 4) {
+        const float w0 = S.pi[i * kPad + j], w1 = S.pi[(i + 1) * kPad + j];
+        const float w2 = S.pi[(i + 2) * kPad + j], w3 = S.pi[(i + 3) * kPad + j];
+#pragma unroll
+        for (int v = 0; v < kNV / 2; ++v) {
+          const float4 cc = *reinterpret_cast<const float4 *>(&S.c[v0 + v][i]);
+          acc[v] = fmaf(w0, cc.x, acc[v]);
+          acc[v] = fmaf(w1, cc.y, acc[v]);
+          acc[v] = fmaf(w2, cc.z, acc[v]);
+          acc[v] = fmaf(w3, cc.w, acc[v]);
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) {
+        const int vi = v0 + v;
+        const float rr = S.u[vi][j] - acc[v];
+        S.r[vi][j] = rr;
+        const float part = warp_sum(rr * rr);
+        if (lane == 0) S.rn2[vi][(j >> 5)] = part;
+      }
+    }
+    __syncthreads();
+
+    // ---- phase 3: z = S r, sign plane, norms ------------------------------
+    {
+      const int i = tid & (kD - 1);
+      const int v0 = (tid >> 7) * (kNV / 2);
+      float acc[kNV / 2];
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) acc[v] = 0.f;
+      for (int j = 0; j < kD; j += 4) {
+        const float w0 = S.s[i * kPad + j], w1 = S.s[i * kPad + j + 1];
+        const float w2 = S.s[i * kPad + j + 2], w3 = S.s[i * kPad + j + 3];
+#pragma unroll
+        for (int v = 0; v < kNV / 2; ++v) {
+          const float4 rr = *reinterpret_cast<const float4 *>(&S.r[v0 + v][j]);
+          acc[v] = fmaf(w0, rr.x, acc[v]);
+          acc[v] = fmaf(w1, rr.y, acc[v]);
+          acc[v] = fmaf(w2, rr.z, acc[v]);
+          acc[v] = fmaf(w3, rr.w, acc[v]);
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) {
+        const int vi = v0 + v;
+        int b, t, h;
+        bool valid;
+        vec_coords(a, id0 + vi, b, t, h, valid);
+        const bool zero = !(S.nk[vi] > 0.f);
+        const int bit = (!zero && acc[v] >= 0.f) ? 1 : 0;
+        const unsigned word = __ballot_sync(0xffffffffu, bit);
+        if (valid) {
+          const int pos = a.lens[b] + t;
+          uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
+          const int slot = pos % kTile;
+          if (lane == 0)
+            *reinterpret_cast<uint32_t *>(tile + L.signs + slot * kRowBytes + 4 * (i >> 5)) = word;
+          if (i == 0) {
+            const float rn = zero ? 0.f
+                                  : sqrtf(S.rn2[vi][0] + S.rn2[vi][1] + S.rn2[vi][2] + S.rn2[vi][3]);
+            __half2 nr = __halves2half2(__float2half_rn(S.nk[vi]), __float2half_rn(rn));
+            *reinterpret_cast<__half2 *>(tile + L.norms + slot * 4) = nr;
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t quantize_simt_smem_bytes() { return sizeof(QuantSmem); }
+
+cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream) {
+  const size_t smem = sizeof(QuantSmem);
+  cudaError_t e = cudaFuncSetAttribute(quantize_append_simt_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)a.batch * a.T * a.h_kv;
+  const long long nchunks = (total + kNV - 1) / kNV;
+  const int grid = (int)std::min<long long>(nchunks, (long long)num_sms);
+  if (grid <= 0) return cudaSuccess;
+  quantize_append_simt_kernel<<<grid, kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,79 @@
+// Shared device-side definitions for the TurboQuant-prod kernels: the cache
+// tile layout (documented in include/tq.h) and small helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr int kD = 128;            // head dimension built
+constexpr int kGroup = 32;         // value group
+constexpr int kGroups = kD / kGroup;
+constexpr int kTile = TQ_TILE_TOKENS;
+constexpr int kRowBytes = kD / 8;  // one bit-plane row of a token
+constexpr int kPlaneBytes = kTile * kRowBytes;  // 2048
+
+// Byte offsets of the sections inside one tile.
+struct TileLayout {
+  int mb;          // Lloyd-Max bits (key_bits - 1)
+  int vb;          // value bits
+  int kplanes;     // offset of key planes
+  int signs;       // offset of the sign plane
+  int vplanes;     // offset of value planes
+  int norms;       // offset of {||k||, ||r||} fp16 pairs
+  int vsz;         // offset of {scale, zero} fp16 pairs
+  int tile_bytes;  // bytes of one tile
+
+  __host__ __device__ static TileLayout make(int key_bits, int value_bits) {
+    TileLayout L;
+    L.mb = key_bits - 1;
+    L.vb = value_bits;
+    L.kplanes = 0;
+    L.signs = L.mb * kPlaneBytes;
+    L.vplanes = L.signs + kPlaneBytes;
+    L.norms = L.vplanes + L.vb * kPlaneBytes;
+    L.vsz = L.norms + kTile * 4;
+    L.tile_bytes = L.vsz + kTile * 4 * kGroups;
+    return L;
+  }
+  __host__ __device__ int record_bytes() const { return tile_bytes / kTile; }
+};
+
+// Base pointer of tile t of (b, h).
+__device__ __forceinline__ uint8_t *tile_ptr(void *data, const TileLayout &L,
+                                             int h_kv, int ntiles, int b, int h,
+                                             int t) {
+  size_t idx = ((size_t)b * h_kv + h) * (size_t)ntiles + (size_t)t;
+  return reinterpret_cast<uint8_t *>(data) + idx * (size_t)L.tile_bytes;
+}
+
+__device__ __forceinline__ float load_elem(const void *p, tq_dtype dt, size_t i) {
+  if (dt == TQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+  return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_min(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// QJL constant sqrt(pi/2) / d.
+__host__ __device__ constexpr float qjl_kappa() { return 1.2533141373155003f / kD; }
+
+}  // namespace tq

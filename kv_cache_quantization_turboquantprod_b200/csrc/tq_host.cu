@@ -1,0 +1,216 @@
+// C-ABI entry points (include/tq.h): host-side validation, the Lloyd-Max
+// codebook, workspace planning and kernel launches.  Nothing here allocates
+// device memory or synchronises.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+#include <cmath>
+#include <vector>
+
+#include "tq_common.cuh"
+#include "tq_kernels.h"
+
+namespace {
+
+using tq::kD;
+using tq::kGroup;
+using tq::kTile;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];  // 0 = not yet queried
+
+// SM count of the current device (cached per device).
+cudaError_t current_sm_count(int *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices) {
+    int v = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (v > 0) { *out = v; return cudaSuccess; }
+  }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(sms, std::memory_order_relaxed);
+  *out = sms;
+  return cudaSuccess;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+tq_status check_params(const tq_params *p) {
+  if (!p) return TQ_ERR_INVALID_ARGUMENT;
+  if (p->d != kD || p->group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if (p->key_bits < 2 || p->key_bits > 4) return TQ_ERR_UNSUPPORTED;
+  if (p->value_bits < 2 || p->value_bits > 4) return TQ_ERR_UNSUPPORTED;
+  if (!p->pi || !p->s || !p->centroids || !p->boundaries) return TQ_ERR_INVALID_ARGUMENT;
+  return TQ_OK;
+}
+
+tq_status check_cache(const tq_cache *c) {
+  if (!c || !c->data) return TQ_ERR_INVALID_ARGUMENT;
+  if (c->batch < 1 || c->h_kv < 1 || c->capacity < kTile || c->capacity % kTile)
+    return TQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(c->data, 256)) return TQ_ERR_INVALID_ARGUMENT;
+  return TQ_OK;
+}
+
+bool dtype_ok(tq_dtype d) { return d == TQ_F32 || d == TQ_BF16; }
+
+double phi(double x) { return std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI); }
+
+// P(a < Z <= b), Z standard normal; infinite ends allowed.
+double normal_mass(double a, double b) {
+  const double fa = std::isinf(a) ? (a < 0 ? 0.0 : 1.0) : 0.5 * std::erfc(-a / std::sqrt(2.0));
+  const double fb = std::isinf(b) ? (b < 0 ? 0.0 : 1.0) : 0.5 * std::erfc(-b / std::sqrt(2.0));
+  return fb - fa;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_ARGUMENT: return "TQ_ERR_INVALID_ARGUMENT";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+    case TQ_ERR_CAPACITY: return "TQ_ERR_CAPACITY";
+    case TQ_ERR_WORKSPACE: return "TQ_ERR_WORKSPACE";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+    case TQ_ERR_INTERNAL: return "TQ_ERR_INTERNAL";
+  }
+  return "TQ_UNKNOWN_STATUS";
+}
+
+tq_status tq_make_codebook(int mse_bits, int d, double *centroids, double *boundaries) {
+  if (!centroids || (!boundaries && mse_bits > 0)) return TQ_ERR_INVALID_ARGUMENT;
+  if (mse_bits < 1 || mse_bits > 4 || d < 1) return TQ_ERR_UNSUPPORTED;
+  const int levels = 1 << mse_bits;
+  const double sigma = 1.0 / std::sqrt((double)d);
+  // Lloyd's iteration: cell boundaries at midpoints, centroids at the
+  // conditional means of N(0, sigma^2) over the cells.
+  std::vector<double> c(levels), t(levels - 1), cn(levels);
+  for (int i = 0; i < levels; ++i) c[i] = sigma * (-2.0 + 4.0 * i / (levels - 1));
+  for (int it = 0; it < 100000; ++it) {
+    for (int i = 0; i + 1 < levels; ++i) t[i] = 0.5 * (c[i] + c[i + 1]);
+    double delta = 0.0;
+    for (int i = 0; i < levels; ++i) {
+      const double a = (i == 0) ? -INFINITY : t[i - 1] / sigma;
+      const double b = (i == levels - 1) ? INFINITY : t[i] / sigma;
+      const double pa = std::isinf(a) ? 0.0 : phi(a);
+      const double pb = std::isinf(b) ? 0.0 : phi(b);
+      cn[i] = sigma * (pa - pb) / normal_mass(a, b);
+      delta = std::fmax(delta, std::fabs(cn[i] - c[i]));
+    }
+    c.swap(cn);
+    if (delta < 1e-14 * sigma) break;
+  }
+  for (int i = 0; i + 1 < levels; ++i) t[i] = 0.5 * (c[i] + c[i + 1]);
+  for (int i = 0; i < levels; ++i) centroids[i] = c[i];
+  for (int i = 0; i + 1 < levels; ++i) boundaries[i] = t[i];
+  return TQ_OK;
+}
+
+size_t tq_record_bytes(const tq_params *p) {
+  if (check_params(p) != TQ_OK) return 0;
+  return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits).record_bytes();
+}
+
+size_t tq_cache_bytes(const tq_params *p, int batch, int h_kv, int capacity) {
+  if (check_params(p) != TQ_OK) return 0;
+  if (batch < 1 || h_kv < 1 || capacity < kTile || capacity % kTile) return 0;
+  const tq::TileLayout L = tq::TileLayout::make(p->key_bits, p->value_bits);
+  return (size_t)batch * h_kv * (size_t)(capacity / kTile) * (size_t)L.tile_bytes;
+}
+
+tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *k,
+                             const void *v, tq_dtype dtype, int T, const int32_t *len_host,
+                             const int32_t *n_new_host, tq_stream_t stream) {
+  tq_status st = check_params(p);
+  if (st != TQ_OK) return st;
+  if ((st = check_cache(c)) != TQ_OK) return st;
+  if (!dtype_ok(dtype)) return TQ_ERR_UNSUPPORTED;
+  if (T < 0 || !len_host) return TQ_ERR_INVALID_ARGUMENT;
+  if (c->batch > TQ_MAX_BATCH) return TQ_ERR_CAPACITY;
+  if (T == 0) return TQ_OK;
+  if (!k || !v || !aligned(k, 16) || !aligned(v, 16)) return TQ_ERR_INVALID_ARGUMENT;
+  tq::AppendArgs a;
+  memset(&a, 0, sizeof(a));
+  for (int b = 0; b < c->batch; ++b) {
+    const int len = len_host[b];
+    const int nn = n_new_host ? n_new_host[b] : T;
+    if (len < 0 || nn < 0 || nn > T) return TQ_ERR_INVALID_ARGUMENT;
+    if ((long long)len + nn > c->capacity) return TQ_ERR_CAPACITY;
+    a.lens[b] = len;
+    a.nnew[b] = nn;
+  }
+  a.pi = p->pi; a.s = p->s; a.centroids = p->centroids; a.boundaries = p->boundaries;
+  a.data = c->data; a.k = k; a.v = v;
+  a.batch = c->batch; a.h_kv = c->h_kv; a.ntiles = c->capacity / kTile; a.T = T;
+  a.key_bits = p->key_bits; a.value_bits = p->value_bits; a.dtype = dtype;
+  int sms = 0;
+  if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
+  if (tq::launch_quantize_simt(a, sms, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
+size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, int max_len) {
+  if (check_params(p) != TQ_OK || check_cache(c) != TQ_OK) return 0;
+  if (h_q < c->h_kv || h_q % c->h_kv || max_len < 0 || max_len > c->capacity) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != cudaSuccess) return 0;
+  return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms).total_bytes;
+}
+
+tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void *q,
+                              tq_dtype q_dtype, int h_q, const int32_t *len_dev, int max_len,
+                              float softmax_scale, float *out, void *workspace,
+                              size_t workspace_bytes, tq_stream_t stream) {
+  tq_status st = check_params(p);
+  if (st != TQ_OK) return st;
+  if ((st = check_cache(c)) != TQ_OK) return st;
+  if (!dtype_ok(q_dtype)) return TQ_ERR_UNSUPPORTED;
+  if (!q || !len_dev || !out) return TQ_ERR_INVALID_ARGUMENT;
+  if (h_q < c->h_kv || h_q % c->h_kv) return TQ_ERR_INVALID_ARGUMENT;
+  if (h_q / c->h_kv > 8) return TQ_ERR_UNSUPPORTED;
+  if (max_len < 0 || max_len > c->capacity) return TQ_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(softmax_scale)) return TQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(len_dev, 4)) return TQ_ERR_INVALID_ARGUMENT;
+  if (!workspace || !aligned(workspace, 256)) return TQ_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
+  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms);
+  if (workspace_bytes < P.total_bytes) return TQ_ERR_WORKSPACE;
+  tq::DecodeArgs a;
+  a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
+  a.data = c->data; a.q = q; a.q_dtype = q_dtype; a.len = len_dev;
+  a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q; a.ntiles = c->capacity / kTile;
+  a.max_len = max_len; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
+  a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
+  a.qrot = reinterpret_cast<float *>(workspace);
+  a.part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + P.qrot_bytes);
+  a.out = out;
+  if (tq::launch_decode_simt(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
+tq_status tq_dequantize(const tq_params *p, const tq_cache *c, int b, int start, int count,
+                        float *k_out, float *v_out, tq_stream_t stream) {
+  tq_status st = check_params(p);
+  if (st != TQ_OK) return st;
+  if ((st = check_cache(c)) != TQ_OK) return st;
+  if (b < 0 || b >= c->batch || start < 0 || count < 0) return TQ_ERR_INVALID_ARGUMENT;
+  if ((long long)start + count > c->capacity) return TQ_ERR_INVALID_ARGUMENT;
+  if (count == 0) return TQ_OK;
+  if (!k_out || !v_out || !aligned(k_out, 4) || !aligned(v_out, 4)) return TQ_ERR_INVALID_ARGUMENT;
+  tq::DequantArgs a;
+  a.pi = p->pi; a.s = p->s; a.centroids = p->centroids; a.data = c->data;
+  a.h_kv = c->h_kv; a.ntiles = c->capacity / kTile; a.b = b; a.start = start; a.count = count;
+  a.key_bits = p->key_bits; a.value_bits = p->value_bits; a.k_out = k_out; a.v_out = v_out;
+  if (tq::launch_dequantize(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// Internal launch interface between the C-ABI host layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "tq.h"
+
+namespace tq {
+
+// Arguments of one quantize_append launch.  Passed by value as a
+// __grid_constant__ kernel parameter (8 KB of per-sequence lengths; CUDA
+// 12.1+ allows kernel parameters up to 32764 bytes).
+struct AppendArgs {
+  const float *pi, *s, *centroids, *boundaries;
+  void *data;
+  const void *k, *v;
+  int batch, h_kv, ntiles, T;
+  int key_bits, value_bits;
+  tq_dtype dtype;
+  int lens[TQ_MAX_BATCH];
+  int nnew[TQ_MAX_BATCH];
+};
+
+// Split-K plan of one decode call (host-computed, identical in the
+// workspace-size query and the launch).
+struct DecodePlan {
+  int nsplit;          // splits per (b, h_kv)
+  int tiles_per_split; // 128-token tiles per split
+  size_t qrot_bytes;   // [B][H_q][2][d] fp32
+  size_t part_bytes;   // [B][H_q][nsplit][d + 2] fp32 (acc, m, l)
+  size_t total_bytes;
+};
+
+struct DecodeArgs {
+  const float *pi, *s, *centroids;
+  const void *data;
+  const void *q;
+  tq_dtype q_dtype;
+  const int32_t *len;
+  int batch, h_kv, h_q, ntiles, max_len;
+  int key_bits, value_bits;
+  float softmax_scale;
+  int nsplit, tiles_per_split;
+  float *qrot;   // workspace: [B][H_q][2][d]
+  float *part;   // workspace: [B][H_q][nsplit][d+2]
+  float *out;    // [B][H_q][d]
+};
+
+struct DequantArgs {
+  const float *pi, *s, *centroids;
+  const void *data;
+  int h_kv, ntiles, b, start, count;
+  int key_bits, value_bits;
+  float *k_out, *v_out;
+};
+
+DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms);
+
+cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t stream);
+
+}  // namespace tq

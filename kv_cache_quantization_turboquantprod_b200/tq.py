@@ -1,0 +1,229 @@
+"""Thin Python binding of the C-ABI library libtq.so (include/tq.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory (``tensor.data_ptr()``) and the
+stream (``torch.cuda.current_stream().cuda_stream``).  Function names match
+the C entry points.  There is no fallback: if libtq.so is missing, loading
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK = 0
+STATUS = {0: "TQ_OK", 1: "TQ_ERR_INVALID_ARGUMENT", 2: "TQ_ERR_UNSUPPORTED",
+          3: "TQ_ERR_CAPACITY", 4: "TQ_ERR_WORKSPACE", 5: "TQ_ERR_CUDA",
+          6: "TQ_ERR_INTERNAL"}
+TQ_F32, TQ_BF16 = 0, 1
+TILE_TOKENS = 128
+MAX_BATCH = 1024
+
+# Every function include/tq.h declares.
+EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_bytes",
+           "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
+           "tq_dequantize")
+
+
+class TQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("key_bits", ctypes.c_int),
+                ("value_bits", ctypes.c_int), ("group", ctypes.c_int),
+                ("pi", ctypes.c_void_p), ("s", ctypes.c_void_p),
+                ("centroids", ctypes.c_void_p), ("boundaries", ctypes.c_void_p)]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("h_kv", ctypes.c_int),
+                ("capacity", ctypes.c_int), ("data", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libtq.so (once) and declare its prototypes."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} not built; run python -m kv_cache_quantization_turboquantprod_b200.build")
+    lib = ctypes.CDLL(p)
+    P, C = ctypes.POINTER(Params), ctypes.POINTER(Cache)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.tq_status_string.restype = ctypes.c_char_p
+    lib.tq_status_string.argtypes = [ci]
+    lib.tq_make_codebook.restype = ci
+    lib.tq_make_codebook.argtypes = [ci, ci, ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(ctypes.c_double)]
+    lib.tq_record_bytes.restype = sz
+    lib.tq_record_bytes.argtypes = [P]
+    lib.tq_cache_bytes.restype = sz
+    lib.tq_cache_bytes.argtypes = [P, ci, ci, ci]
+    lib.tq_quantize_append.restype = ci
+    lib.tq_quantize_append.argtypes = [P, C, vp, vp, ci, ci, i32p, i32p, vp]
+    lib.tq_decode_workspace_size.restype = sz
+    lib.tq_decode_workspace_size.argtypes = [P, C, ci, ci]
+    lib.tq_decode_attention.restype = ci
+    lib.tq_decode_attention.argtypes = [P, C, vp, ci, ci, vp, ci, ctypes.c_float, vp, vp, sz, vp]
+    lib.tq_dequantize.restype = ci
+    lib.tq_dequantize.argtypes = [P, C, ci, ci, ci, vp, vp, vp]
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(fn: str, st: int) -> None:
+    if st != TQ_OK:
+        raise TQError(fn, st)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TQ_F32
+    if t.dtype == torch.bfloat16:
+        return TQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _i32_array(xs):
+    arr = (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+    return arr
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def tq_status_string(status: int) -> str:
+    return load().tq_status_string(int(status)).decode()
+
+
+def tq_make_codebook(mse_bits: int, d: int):
+    """Host-only Lloyd-Max codebook: (centroids [2^b], boundaries [2^b - 1]) as
+    Python float lists."""
+    n = 1 << mse_bits if 1 <= mse_bits <= 4 else 1
+    c = (ctypes.c_double * n)()
+    b = (ctypes.c_double * max(n - 1, 1))()
+    _check("tq_make_codebook", load().tq_make_codebook(mse_bits, d, c, b))
+    return list(c), list(b)[: n - 1]
+
+
+class Layer:
+    """Device-resident constants of one layer (Pi, S, codebook) packaged as
+    the C struct tq_params.  Holds references to the tensors it points to."""
+
+    def __init__(self, pi, s, key_bits: int, value_bits: int, group: int = 32,
+                 device="cuda"):
+        d = int(pi.shape[0])
+        cent, bnd = tq_make_codebook(key_bits - 1, d)
+        self.pi = torch.as_tensor(pi, dtype=torch.float32).contiguous().to(device)
+        self.s = torch.as_tensor(s, dtype=torch.float32).contiguous().to(device)
+        self.centroids = torch.tensor(cent, dtype=torch.float32, device=device)
+        self.boundaries = torch.tensor(bnd if bnd else [0.0], dtype=torch.float32, device=device)
+        self.codebook = (cent, bnd)
+        self.params = Params(d, key_bits, value_bits, group, self.pi.data_ptr(),
+                             self.s.data_ptr(), self.centroids.data_ptr(),
+                             self.boundaries.data_ptr())
+
+    @property
+    def d(self):
+        return self.params.d
+
+    def record_bytes(self) -> int:
+        return int(load().tq_record_bytes(ctypes.byref(self.params)))
+
+
+class CompressedCache:
+    """A caller-owned cache buffer (torch uint8 tensor) as the C struct
+    tq_cache."""
+
+    def __init__(self, layer: Layer, batch: int, h_kv: int, capacity: int,
+                 device="cuda", zero: bool = False):
+        n = tq_cache_bytes(layer, batch, h_kv, capacity)
+        if n == 0:
+            raise TQError("tq_cache_bytes", 1)
+        alloc = torch.zeros if zero else torch.empty
+        self.buffer = alloc(n, dtype=torch.uint8, device=device)
+        self.cache = Cache(batch, h_kv, capacity, self.buffer.data_ptr())
+        self.batch, self.h_kv, self.capacity = batch, h_kv, capacity
+
+
+def tq_record_bytes(layer: Layer) -> int:
+    return int(load().tq_record_bytes(ctypes.byref(layer.params)))
+
+
+def tq_cache_bytes(layer: Layer, batch: int, h_kv: int, capacity: int) -> int:
+    return int(load().tq_cache_bytes(ctypes.byref(layer.params), batch, h_kv, capacity))
+
+
+def tq_quantize_append(layer: Layer, cache: CompressedCache, k: torch.Tensor,
+                       v: torch.Tensor, len_host, n_new_host=None, stream=None) -> None:
+    """k, v: [B, T, H_kv, d] device tensors (fp32 or bf16, contiguous)."""
+    if k.dtype != v.dtype:
+        raise TypeError("k and v must share a dtype")
+    if not (k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("k and v must be contiguous")
+    T = int(k.shape[1]) if k.dim() == 4 else 0
+    lens = _i32_array(len_host)
+    nn = _i32_array(n_new_host) if n_new_host is not None else None
+    st = load().tq_quantize_append(ctypes.byref(layer.params), ctypes.byref(cache.cache),
+                                   k.data_ptr(), v.data_ptr(), _dtype_code(k), T, lens,
+                                   nn, _stream(stream))
+    _check("tq_quantize_append", st)
+
+
+def tq_decode_workspace_size(layer: Layer, cache: CompressedCache, h_q: int, max_len: int) -> int:
+    return int(load().tq_decode_workspace_size(ctypes.byref(layer.params),
+                                               ctypes.byref(cache.cache), h_q, max_len))
+
+
+def tq_decode_attention(layer: Layer, cache: CompressedCache, q: torch.Tensor,
+                        len_dev: torch.Tensor, max_len: int, out: torch.Tensor,
+                        workspace: torch.Tensor, softmax_scale: float | None = None,
+                        stream=None) -> None:
+    """q [B, H_q, d] (fp32/bf16), len_dev [B] int32 device, out [B, H_q, d]
+    fp32, workspace a uint8 device tensor."""
+    if len_dev.dtype != torch.int32:
+        raise TypeError("len_dev must be int32")
+    scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().tq_decode_attention(ctypes.byref(layer.params), ctypes.byref(cache.cache),
+                                    q.data_ptr(), _dtype_code(q), int(q.shape[1]),
+                                    len_dev.data_ptr(), int(max_len), scale, out.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream(stream))
+    _check("tq_decode_attention", st)
+
+
+def tq_dequantize(layer: Layer, cache: CompressedCache, b: int, start: int, count: int,
+                  k_out: torch.Tensor, v_out: torch.Tensor, stream=None) -> None:
+    st = load().tq_dequantize(ctypes.byref(layer.params), ctypes.byref(cache.cache), b, start,
+                              count, k_out.data_ptr(), v_out.data_ptr(), _stream(stream))
+    _check("tq_dequantize", st)
+
+
+def workspace_for(layer: Layer, cache: CompressedCache, h_q: int, max_len: int,
+                  device="cuda") -> torch.Tensor:
+    n = tq_decode_workspace_size(layer, cache, h_q, max_len)
+    if n == 0:
+        raise TQError("tq_decode_workspace_size", 1)
+    return torch.empty(n, dtype=torch.uint8, device=device)

@@ -1,0 +1,138 @@
+"""Helpers shared by the GPU parity tests: run the oracle on the same seeded
+inputs, read the library's cache bytes back with the oracle's layout reader,
+and compare with the bands and tolerances the parity bar fixes.
+
+Parity bar:
+* key codes and sign bits bit-exact except coordinates within 1e-6 of a
+  decision boundary (|y - t| < 1e-6, oracle y) or of zero (|S r| < 1e-6);
+  the band count is reported and must be <= 1e-4 of all coordinates;
+* value codes, scales and zeros bit-exact everywhere (both sides take the
+  float32 steps in the same order; bf16 inputs put many values exactly on
+  half-integer code boundaries, so the band |t - (k + 1/2)| < 1e-6 is only
+  counted, not excluded);
+* norms and attention outputs within 1e-3 relative: per row,
+  max |gpu - oracle| / max |oracle|.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from kv_cache_quantization_turboquantprod_b200 import tq, workloads
+from oracle import attention, codebook, layout, quant
+
+BAND = 1e-6
+BAND_FRACTION_MAX = 1e-4
+REL_TOL = 1e-3
+
+
+class OracleLayer:
+    """The oracle's view of one layer: the same Pi (float32 values), S and a
+    codebook from the oracle's own Lloyd-Max."""
+
+    def __init__(self, pi32: np.ndarray, s32: np.ndarray, key_bits: int, value_bits: int,
+                 group: int = 32):
+        self.pi = np.asarray(pi32, np.float64)
+        self.s = np.asarray(s32, np.float64)
+        self.key_bits, self.value_bits, self.group = key_bits, value_bits, group
+        self.cent, self.bnd, _ = codebook.lloyd_max_gaussian(key_bits - 1, self.pi.shape[0])
+
+    def encode(self, k: np.ndarray, v: np.ndarray):
+        ke = quant.encode_keys(k, self.pi, self.s, self.cent, self.bnd)
+        ve = quant.encode_values(v, self.value_bits, self.group)
+        return ke, ve
+
+
+def gpu_layer(pi32, s32, key_bits, value_bits, device="cuda"):
+    return tq.Layer(pi32, s32, key_bits, value_bits, device=device)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy()
+
+
+def compare_records(spec: layout.CacheSpec, buf: np.ndarray, b: int, h: int, pos0: int,
+                    ke: dict, ve: dict, stats: dict | None = None) -> dict:
+    """Compare the library's records of tokens [pos0, pos0+n) of (b, h) with
+    the oracle's encoding (ke, ve of n vectors).  Raises AssertionError on a
+    mismatch outside the bands; returns accumulated band statistics."""
+    n = len(ke["nk16"])
+    got = spec.read(buf, b, h, pos0, n)
+    stats = stats if stats is not None else {"coords": 0, "code_band": 0, "sign_band": 0,
+                                             "value_band": 0, "max_norm_rel": 0.0}
+    bnd = np.asarray(codebook.lloyd_max_gaussian(spec.key_bits - 1, spec.d)[1])
+    # codes: band where y is within 1e-6 of a boundary
+    near = np.zeros_like(ke["y"], dtype=bool)
+    for t in bnd:
+        near |= np.abs(ke["y"] - t) < BAND
+    zero = ke["nk"] == 0
+    near[zero] = False
+    bad = (got["idx"] != ke["idx"]) & ~near
+    assert not bad.any(), f"code mismatch outside band at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
+    snear = np.abs(ke["z"]) < BAND
+    snear[zero] = False
+    bad = (got["sign"] != ke["sign"]) & ~snear
+    assert not bad.any(), f"sign mismatch outside band at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
+    t = ve["t"]
+    vnear = np.abs(t - np.floor(t) - 0.5) < BAND
+    # value codes are decided by the same float32 steps on both sides: exact
+    # everywhere, half-integer ties included (the band is only counted)
+    bad = got["codes"] != ve["codes"]
+    assert not bad.any(), f"value code mismatch at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
+    assert np.array_equal(got["scale16"], ve["scale16"]), "value scale mismatch"
+    assert np.array_equal(got["zero16"], ve["zero16"]), "value zero mismatch"
+    for key in ("nk16", "rn16"):
+        ref = ke[key]
+        rel = np.abs(got[key] - ref) / np.maximum(np.abs(ref), 1e-30)
+        rel[(ref == 0) & (got[key] == 0)] = 0.0
+        assert rel.max(initial=0.0) <= REL_TOL, f"{key} rel err {rel.max()}"
+        stats["max_norm_rel"] = max(stats["max_norm_rel"], float(rel.max(initial=0.0)))
+    stats["coords"] += n * spec.d
+    stats["code_band"] += int(near.sum())
+    stats["sign_band"] += int(snear.sum())
+    stats["value_band"] += int(vnear.sum())
+    return stats
+
+
+def check_band_fraction(stats: dict) -> None:
+    for key in ("code_band", "sign_band"):
+        frac = stats[key] / max(stats["coords"], 1)
+        assert frac <= BAND_FRACTION_MAX, f"{key} fraction {frac}"
+
+
+def row_rel_err(got: np.ndarray, ref: np.ndarray) -> float:
+    """max over rows of max|got - ref| / max|ref| (rows = last axis)."""
+    g = got.reshape(-1, got.shape[-1])
+    r = ref.reshape(-1, ref.shape[-1])
+    num = np.abs(g - r).max(axis=1)
+    den = np.abs(r).max(axis=1)
+    rel = np.where(den > 0, num / np.maximum(den, 1e-300), num)
+    return float(rel.max(initial=0.0))
+
+
+def oracle_records_for(layer: OracleLayer, k: np.ndarray, v: np.ndarray):
+    """Encode [n, H_kv, d] keys/values head by head; returns per-head lists."""
+    kes, ves = [], []
+    for h in range(k.shape[1]):
+        ke, ve = layer.encode(k[:, h], v[:, h])
+        kes.append(ke)
+        ves.append(ve)
+    return kes, ves
+
+
+def logical(ke: dict, ve: dict) -> dict:
+    return {"idx": ke["idx"], "sign": ke["sign"], "nk16": ke["nk16"], "rn16": ke["rn16"],
+            "codes": ve["codes"], "scale16": ve["scale16"], "zero16": ve["zero16"]}
+
+
+def oracle_decode(layer: OracleLayer, q: np.ndarray, kes: list, ves: list, length: int,
+                  start: int = 0) -> np.ndarray:
+    """Oracle decode for one sequence from per-head encodings, using tokens
+    [start, start + length) of the encodings."""
+    recs = []
+    for ke, ve in zip(kes, ves):
+        r = logical(ke, ve)
+        recs.append({k2: v2[start:start + length] for k2, v2 in r.items()})
+    rec = attention.stack_heads(recs)
+    return attention.decode_one_sequence(q, rec, layer.pi, layer.s, layer.cent, layer.group)

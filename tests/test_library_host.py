@@ -1,0 +1,149 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+* libtq.so loads and exports every function include/tq.h declares.
+* The library's host Lloyd-Max codebook (its own C++ implementation) agrees
+  with the oracle's.
+* Argument validation returns the documented status before any launch.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from kv_cache_quantization_turboquantprod_b200 import tq
+from oracle import codebook
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    return sorted(set(re.findall(r"TQ_API\s+[\w\s\*]*?\b(tq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared_functions() == sorted(tq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tq.load()
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {tq.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (tq_\w+)", out))
+    assert set(_declared_functions()) <= exported
+    # nothing else of ours leaks out of the library
+    assert {s for s in exported if s.startswith("tq")} == set(_declared_functions())
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("d", [64, 128])
+def test_host_codebook_matches_oracle(bits, d):
+    c, b = tq.tq_make_codebook(bits, d)
+    oc, ob, _ = codebook.lloyd_max_gaussian(bits, d)
+    assert np.allclose(c, oc, rtol=0, atol=1e-13)
+    assert np.allclose(b, ob, rtol=0, atol=1e-13)
+
+
+def test_codebook_argument_errors():
+    lib = tq.load()
+    buf = (ctypes.c_double * 16)()
+    assert lib.tq_make_codebook(0, 128, buf, buf) == 2
+    assert lib.tq_make_codebook(5, 128, buf, buf) == 2
+    assert lib.tq_make_codebook(2, 0, buf, buf) == 2
+    assert lib.tq_make_codebook(2, 128, None, buf) == 1
+
+
+def test_status_strings():
+    for code, name in tq.STATUS.items():
+        assert tq.tq_status_string(code) == name
+
+
+def _params(d=128, kb=3, vb=2, g=32, ptr=256):
+    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr)
+
+
+def test_record_and_cache_bytes():
+    lib = tq.load()
+    P = _params()
+    assert lib.tq_record_bytes(ctypes.byref(P)) == 100
+    assert lib.tq_record_bytes(ctypes.byref(_params(kb=4))) == 116
+    assert lib.tq_record_bytes(ctypes.byref(_params(vb=3))) == 116
+    assert lib.tq_cache_bytes(ctypes.byref(P), 2, 8, 256) == 2 * 8 * 2 * 12800
+    assert lib.tq_cache_bytes(ctypes.byref(P), 2, 8, 200) == 0     # not a tile multiple
+    assert lib.tq_record_bytes(ctypes.byref(_params(d=64))) == 0
+    assert lib.tq_record_bytes(ctypes.byref(_params(g=16))) == 0
+    assert lib.tq_record_bytes(ctypes.byref(_params(kb=5))) == 0
+
+
+def test_append_validation_before_launch():
+    """Every error below is detected on the host; nothing touches a GPU."""
+    lib = tq.load()
+    P = _params()
+    C = tq.Cache(2, 8, 256, 1 << 20)
+    lens = (ctypes.c_int32 * 2)(0, 250)
+    k = v = 1 << 21
+    f = lib.tq_quantize_append
+    assert f(None, ctypes.byref(C), k, v, 1, 4, lens, None, None) == 1
+    assert f(ctypes.byref(_params(d=64)), ctypes.byref(C), k, v, 1, 4, lens, None, None) == 2
+    assert f(ctypes.byref(P), None, k, v, 1, 4, lens, None, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 7, 4, lens, None, None) == 2   # dtype
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, -1, lens, None, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, 4, None, None, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), None, v, 1, 4, lens, None, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), k + 2, v, 1, 4, lens, None, None) == 1  # align
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, 7, lens, None, None) == 3   # 250+7>256
+    nn = (ctypes.c_int32 * 2)(4, 9)
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, 8, lens, nn, None) == 1     # 9 > T
+    nn = (ctypes.c_int32 * 2)(4, 7)
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, 8, lens, nn, None) == 3
+    bad = (ctypes.c_int32 * 2)(-1, 0)
+    assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, 4, bad, None, None) == 1
+    Cmis = tq.Cache(2, 8, 256, (1 << 20) + 16)                                     # data align
+    assert f(ctypes.byref(P), ctypes.byref(Cmis), k, v, 1, 4, lens, None, None) == 1
+    Cbig = tq.Cache(tq.MAX_BATCH + 1, 1, 128, 1 << 20)
+    big = (ctypes.c_int32 * (tq.MAX_BATCH + 1))()
+    assert f(ctypes.byref(P), ctypes.byref(Cbig), k, v, 1, 4, big, None, None) == 3
+    # T = 0 is a no-op that succeeds without launching
+    assert f(ctypes.byref(P), ctypes.byref(C), None, None, 1, 0, lens, None, None) == 0
+
+
+def test_decode_validation_before_launch():
+    lib = tq.load()
+    P = _params()
+    C = tq.Cache(2, 8, 256, 1 << 20)
+    f = lib.tq_decode_attention
+    q, ln, out, ws = 1 << 22, 1 << 23, 1 << 24, 1 << 25
+    args = lambda **kw: [kw.get("p", ctypes.byref(P)), kw.get("c", ctypes.byref(C)),
+                         kw.get("q", q), kw.get("dt", 1), kw.get("hq", 32), kw.get("ln", ln),
+                         kw.get("ml", 256), kw.get("sc", 0.088), kw.get("out", out),
+                         kw.get("ws", ws), kw.get("wsb", 1 << 20), None]
+    assert f(*args(p=None)) == 1
+    assert f(*args(q=None)) == 1
+    assert f(*args(ln=None)) == 1
+    assert f(*args(out=None)) == 1
+    assert f(*args(hq=12)) == 1           # not a multiple of h_kv
+    assert f(*args(hq=4)) == 1            # fewer than h_kv
+    assert f(*args(hq=80)) == 2           # G = 10 not built
+    assert f(*args(ml=257)) == 1          # beyond capacity
+    assert f(*args(ml=-1)) == 1
+    assert f(*args(sc=float("inf"))) == 1
+    assert f(*args(ws=None)) == 4
+    assert f(*args(ws=ws + 8)) == 4       # workspace alignment
+    assert f(*args(dt=3)) == 2
+
+
+def test_dequantize_validation_before_launch():
+    lib = tq.load()
+    P = _params()
+    C = tq.Cache(2, 8, 256, 1 << 20)
+    f = lib.tq_dequantize
+    o = 1 << 22
+    assert f(ctypes.byref(P), ctypes.byref(C), 2, 0, 1, o, o, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), 0, 200, 57, o, o, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), 0, -1, 1, o, o, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), 0, 0, 1, None, o, None) == 1
+    assert f(ctypes.byref(P), ctypes.byref(C), 0, 0, 0, None, None, None) == 0
