@@ -205,6 +205,43 @@ TQ_API tq_status tq_decode_attention(const tq_params *p, const tq_cache *c,
                               float softmax_scale, float *out, void *workspace,
                               size_t workspace_bytes, tq_stream_t stream);
 
+/* Size of the fixed device scratch tq_decode_attention_noalloc uses. */
+#define TQ_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * tq_decode_attention_noalloc -- tq_decode_attention for callers that cannot
+ * provide a workspace.  The pages have no counterpart of this call; it
+ * exists for users of this library.
+ *
+ * Some callers cannot allocate device memory for the library: a plain C host
+ * that links only libtq and owns no device allocator, a decode loop that must
+ * not call cudaMalloc (it can synchronise the whole device and stall other
+ * streams), or an engine that reserved all free device memory for its own
+ * pool at start-up.  This entry point takes the same arguments as
+ * tq_decode_attention minus the workspace and allocates nothing: its scratch
+ * (rotated queries and split-K partial states) is one fixed array of
+ * TQ_NOALLOC_SCRATCH_BYTES (8 MiB) in device memory, reserved in every GPU
+ * that loads the library until the process exits.
+ *
+ *  - A call whose scratch need (tq_decode_workspace_size for the same
+ *    shapes) exceeds TQ_NOALLOC_SCRATCH_BYTES returns TQ_ERR_WORKSPACE and
+ *    launches nothing.
+ *  - The first call on a device looks up the array's device address with
+ *    that device current and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the previous call's contents
+ *    (nothing in it needs clearing: every byte the kernels read is written
+ *    earlier in the same call).  Calls that overlap on the GPU -- on
+ *    different streams, or from different host threads without ordering --
+ *    race on the array and produce wrong results; order them.
+ * Other errors as for tq_decode_attention.
+ */
+TQ_API tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_cache *c,
+                                             const void *q, tq_dtype q_dtype, int h_q,
+                                             const int32_t *len_dev, int max_len,
+                                             float softmax_scale, float *out,
+                                             tq_stream_t stream);
+
 /*
  * tq_dequantize -- explicit reconstruction of cached tokens [start,
  * start + count) of sequence b (the audit's quantizer.dequantize(prod_q),

@@ -28,7 +28,8 @@ MAX_BATCH = 1024
 # Every function include/tq.h declares.
 EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_bytes",
            "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
-           "tq_dequantize")
+           "tq_dequantize", "tq_decode_attention_noalloc")
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class TQError(RuntimeError):
@@ -79,6 +80,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_decode_workspace_size.argtypes = [P, C, ci, ci]
     lib.tq_decode_attention.restype = ci
     lib.tq_decode_attention.argtypes = [P, C, vp, ci, ci, vp, ci, ctypes.c_float, vp, vp, sz, vp]
+    lib.tq_decode_attention_noalloc.restype = ci
+    lib.tq_decode_attention_noalloc.argtypes = [P, C, vp, ci, ci, vp, ci, ctypes.c_float, vp, vp]
     lib.tq_dequantize.restype = ci
     lib.tq_dequantize.argtypes = [P, C, ci, ci, ci, vp, vp, vp]
     if path is None:
@@ -212,6 +215,21 @@ def tq_decode_attention(layer: Layer, cache: CompressedCache, q: torch.Tensor,
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream))
     _check("tq_decode_attention", st)
+
+
+def tq_decode_attention_noalloc(layer: Layer, cache: CompressedCache, q: torch.Tensor,
+                                len_dev: torch.Tensor, max_len: int, out: torch.Tensor,
+                                softmax_scale: float | None = None, stream=None) -> None:
+    """Decode attention for callers that cannot allocate a workspace: the
+    scratch is the library's fixed 8 MiB device array (see include/tq.h)."""
+    if len_dev.dtype != torch.int32:
+        raise TypeError("len_dev must be int32")
+    scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().tq_decode_attention_noalloc(ctypes.byref(layer.params), ctypes.byref(cache.cache),
+                                            q.data_ptr(), _dtype_code(q), int(q.shape[1]),
+                                            len_dev.data_ptr(), int(max_len), scale,
+                                            out.data_ptr(), _stream(stream))
+    _check("tq_decode_attention_noalloc", st)
 
 
 def tq_dequantize(layer: Layer, cache: CompressedCache, b: int, start: int, count: int,
