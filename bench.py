@@ -162,8 +162,22 @@ def _fill_cache(wl, layer, cache, device):
     return lens
 
 
+def aggregate_across_ranks(times, counts, world, device):
+    """Max over ranks of the times, sum over ranks of the work counts (weak
+    scaling: every rank processes its own batch).  Identity for one rank."""
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    c = torch.tensor(counts, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(c, op=torch.distributed.ReduceOp.SUM)
+    return t.tolist(), c.tolist()
+
+
 def run_ours(args, rank, world, device):
     wl = workloads.by_name(args.workload)
+    if args.batch:
+        wl = workloads.scaled(wl, batch=args.batch, capacity=wl.capacity,
+                              name=f"{wl.name}_b{args.batch}")
     _, pi32, s32 = workloads.layer_matrices(wl)
     layer = tq.Layer(pi32, s32, wl.key_bits, wl.value_bits, device=device)
     cache = tq.CompressedCache(layer, wl.batch, wl.h_kv, wl.capacity, device=device)
@@ -254,13 +268,8 @@ def run_ours(args, rank, world, device):
     rec_bytes = layer.record_bytes()
     dec_bytes = ctx_tokens_step * HKV * rec_bytes
 
-    times = torch.tensor([elapsed_ms, e2e_ms, dec_ms], dtype=torch.float64, device=device)
-    toks = torch.tensor([ctx_tokens_step, dec_bytes], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-        torch.distributed.all_reduce(toks, op=torch.distributed.ReduceOp.SUM)
-    elapsed_ms, e2e_ms, dec_ms = times.tolist()
-    ctx_all, dec_bytes_all = toks.tolist()
+    (elapsed_ms, e2e_ms, dec_ms), (ctx_all, dec_bytes_all) = aggregate_across_ranks(
+        [elapsed_ms, e2e_ms, dec_ms], [ctx_tokens_step, dec_bytes], world, device)
     if rank != 0:
         return None
 
@@ -465,6 +474,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batched")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="use the first N sequences of the workload (profiling)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-quantize", dest="quantize", action="store_false",
                     help="skip the quantize-append Mvec/s measurement")

@@ -82,7 +82,7 @@ extern "C" tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_ca
     return TQ_ERR_INVALID_ARGUMENT;
   const int sms = sm_count_current();
   if (sms <= 0) return TQ_ERR_CUDA;
-  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms);
+  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits);
   if (P.total_bytes > kNoAllocScratchBytes) return TQ_ERR_WORKSPACE;
   void *scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess || scratch == nullptr) return TQ_ERR_CUDA;
@@ -92,11 +92,11 @@ extern "C" tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_ca
   a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q; a.ntiles = c->capacity / tq::kTile;
   a.max_len = max_len; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
   a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
-  a.qrot = reinterpret_cast<float *>(scratch);
-  a.part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + P.qrot_bytes);
+  a.num_sms = sms;
+  tq::bind_workspace(a, P, scratch);
   a.out = out;
   // Every byte of the scratch that the kernels read is written earlier in the
   // same call, so nothing needs clearing between calls.
-  if (tq::launch_decode_simt(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (tq::launch_decode(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }

@@ -25,6 +25,7 @@ constexpr int kMaxG = 8;
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) qprep_kernel(DecodeArgs a) {
   const int bh = blockIdx.x;  // b * h_q + hq
+  if (bh == 0 && threadIdx.x == 0 && a.status) *a.status = 0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float qv[4];
 #pragma unroll
@@ -183,7 +184,8 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
 
 }  // namespace
 
-DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms) {
+DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms,
+                            int key_bits, int value_bits) {
   DecodePlan P;
   const int ntile = (max_len + kTile - 1) / kTile;
   const long long units = (long long)batch * h_kv;
@@ -195,10 +197,34 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   P.nsplit = nsplit;
   P.tiles_per_split = tps;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  P.status_bytes = 256;
   P.qrot_bytes = al((size_t)batch * h_q * 2 * kD * sizeof(float));
   P.part_bytes = al((size_t)batch * h_q * nsplit * (kD + 2) * sizeof(float));
-  P.total_bytes = P.qrot_bytes + P.part_bytes;
+  const int G = h_q / h_kv;
+  P.qblock_bytes = decode_tc_supported(key_bits, value_bits, G) ? decode_tc_qblock_bytes(key_bits, G) : 0;
+  P.total_bytes = P.status_bytes + P.qrot_bytes + P.part_bytes + al((size_t)batch * h_kv * P.qblock_bytes);
   return P;
+}
+
+void bind_workspace(DecodeArgs &a, const DecodePlan &P, void *workspace) {
+  uint8_t *w = reinterpret_cast<uint8_t *>(workspace);
+  a.status = reinterpret_cast<int *>(w);
+  a.qrot = reinterpret_cast<float *>(w + P.status_bytes);
+  a.part = reinterpret_cast<float *>(w + P.status_bytes + P.qrot_bytes);
+  a.qblocks = w + P.status_bytes + P.qrot_bytes + P.part_bytes;
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
+  if (!decode_tc_supported(a.key_bits, a.value_bits, a.h_q / a.h_kv))
+    return launch_decode_simt(a, stream);
+  const int bhq = a.batch * a.h_q;
+  // the status word is cleared here; the query blocks are built inside
+  cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  e = launch_decode_tc(a, stream);
+  if (e != cudaSuccess) return e;
+  combine_kernel<<<bhq, 128, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream) {

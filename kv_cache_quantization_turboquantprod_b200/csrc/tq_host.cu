@@ -161,7 +161,7 @@ size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, 
   if (h_q < c->h_kv || h_q % c->h_kv || max_len < 0 || max_len > c->capacity) return 0;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return 0;
-  return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms).total_bytes;
+  return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits).total_bytes;
 }
 
 tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void *q,
@@ -181,7 +181,7 @@ tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void 
   if (!workspace || !aligned(workspace, 256)) return TQ_ERR_WORKSPACE;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
-  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms);
+  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits);
   if (workspace_bytes < P.total_bytes) return TQ_ERR_WORKSPACE;
   tq::DecodeArgs a;
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
@@ -189,10 +189,10 @@ tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void 
   a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q; a.ntiles = c->capacity / kTile;
   a.max_len = max_len; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
   a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
-  a.qrot = reinterpret_cast<float *>(workspace);
-  a.part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + P.qrot_bytes);
+  a.num_sms = sms;
+  tq::bind_workspace(a, P, workspace);
   a.out = out;
-  if (tq::launch_decode_simt(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (tq::launch_decode(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }
 

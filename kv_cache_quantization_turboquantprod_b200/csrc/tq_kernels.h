@@ -30,8 +30,10 @@ struct AppendArgs {
 struct DecodePlan {
   int nsplit;          // splits per (b, h_kv)
   int tiles_per_split; // 128-token tiles per split
+  size_t status_bytes; // status word (nonzero: a kernel gave up on a bounded wait)
   size_t qrot_bytes;   // [B][H_q][2][d] fp32
   size_t part_bytes;   // [B][H_q][nsplit][d + 2] fp32 (acc, m, l)
+  size_t qblock_bytes; // per (b, h_kv) query block of the tensor-core kernel (0: SIMT path)
   size_t total_bytes;
 };
 
@@ -45,8 +47,11 @@ struct DecodeArgs {
   int key_bits, value_bits;
   float softmax_scale;
   int nsplit, tiles_per_split;
+  int *status;   // workspace: status word, cleared by qprep
   float *qrot;   // workspace: [B][H_q][2][d]
   float *part;   // workspace: [B][H_q][nsplit][d+2]
+  uint8_t *qblocks;  // workspace: [B][H_kv] query blocks (tensor-core path)
+  int num_sms;
   float *out;    // [B][H_q][d]
 };
 
@@ -58,10 +63,19 @@ struct DequantArgs {
   float *k_out, *v_out;
 };
 
-DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms);
+DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms,
+                            int key_bits, int value_bits);
 
 cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
+// Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
+bool decode_tc_supported(int key_bits, int value_bits, int gqa);
+size_t decode_tc_qblock_bytes(int key_bits, int gqa);
+cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
+// qprep -> split-K (tensor-core kernel where built, SIMT otherwise) -> combine
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+// Fill DecodeArgs' workspace pointers from a plan.
+void bind_workspace(DecodeArgs &a, const DecodePlan &P, void *workspace);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t stream);
 
 }  // namespace tq

@@ -294,3 +294,21 @@ def test_end_to_end_quantize_then_decode(name):
     err = pu.row_rel_err(out[0].cpu().numpy(), ref)
     print(name, "end-to-end row rel err", err)
     assert err <= 5e-3
+
+
+@pytest.mark.parametrize("kb,vb", [(2, 2), (4, 2), (3, 4), (4, 3)])
+def test_decode_bit_widths(kb, vb):
+    """1-, 2- and 3-bit Lloyd-Max keys and 2-4-bit values at GQA 4 (tensor-core
+    kernel where built, the general SIMT kernel otherwise)."""
+    import dataclasses
+    lengths = (700, 256)
+    wl = dataclasses.replace(workloads.llama8b(), batch=2, key_bits=kb, value_bits=vb,
+                             lengths=lengths, capacity=768, name=f"dec_bits{kb}{vb}")
+    glayer, olayer, spec = _setup(wl)
+    buf, encs = _oracle_cache(wl, olayer, spec, lengths)
+    q = workloads.queries(wl, 0)
+    got = _run_decode(glayer, wl, buf, list(lengths), q)
+    for b in range(wl.batch):
+        kes, ves = encs[b]
+        ref = pu.oracle_decode(olayer, q[b].float().numpy(), kes, ves, lengths[b])
+        assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (kb, vb, b)
