@@ -124,7 +124,10 @@ typedef struct {
  *      1. key code bit-planes: (key_bits - 1) planes, each [128][d/8] bytes;
  *         plane p holds bit p of each coordinate's Lloyd-Max cell index;
  *      2. QJL sign plane [128][d/8]; bit 1 means sign +1 ((S r)_j >= 0);
- *      3. value code bit-planes: value_bits planes, [128][d/8] each;
+ *      3. value codes: for value_bits = 2, packed codes [128][d/4] bytes,
+ *         byte i holding channels 4i .. 4i+3 (channel 4i + m in bits 2m and
+ *         2m+1); for value_bits = 3 or 4, value_bits bit-planes [128][d/8]
+ *         each, plane p holding bit p of each code;
  *      4. norms [128] x {||k||, ||r||}, two little-endian fp16 per token;
  *      5. value groups [128][d/group] x {scale, zero}, two fp16 each.
  *    In a plane row, byte i bit k (LSB first) is coordinate 8 i + k.

@@ -95,10 +95,16 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
     }
     const int snib = (tp[L.signs + slot * kRowBytes + byte] >> shift) & 0xF;
     int code[4] = {0, 0, 0, 0};
-    for (int p = 0; p < L.vb; ++p) {
-      const int nib = (tp[L.vplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> shift) & 0xF;
+    if (L.vb == 2) {
+      const int pk = tp[L.vplanes + slot * kPackedRowBytes + lane];  // channels 4 lane .. 4 lane + 3
 #pragma unroll
-      for (int k = 0; k < 4; ++k) code[k] |= ((nib >> k) & 1) << p;
+      for (int k = 0; k < 4; ++k) code[k] = (pk >> (2 * k)) & 3;
+    } else {
+      for (int p = 0; p < L.vb; ++p) {
+        const int nib = (tp[L.vplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> shift) & 0xF;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) code[k] |= ((nib >> k) & 1) << p;
+      }
     }
     const __half2 nr = *reinterpret_cast<const __half2 *>(tp + L.norms + slot * 4);
     const float nk = __low2float(nr), rn = __high2float(nr);

@@ -18,9 +18,11 @@
 //     as four signed base-128 fixed-point limbs; s32 accumulation is exact;
 //     the centroid lookup is exact because c(idx) is multilinear in the code
 //     bits (2-bit codes) or a sum of threshold planes (3-bit codes);
-//   * values: D[channel, (group, head, byte)] = A_v[channel, plane bits x
-//     tokens] x B_p[tokens, (p * scale_g as 22-bit fixed point) << plane];
-//     the 2^k weight of each operand row is undone per output channel.
+//   * values: D[channel, (group, head, byte)] = A_v[channel, codes x tokens]
+//     x B_p[tokens, p * scale_g as 22-bit fixed point]; 2-bit codes are
+//     stored packed, so one mask (w & (0x03030303 << 2m)) yields code * 4^m
+//     operands; wider codes are bit-planes whose B_p copies carry 2^plane.
+//     The 4^m (or 2^k) weight of each operand row is undone per channel.
 // Per 128-token tile the record bytes arrive by one 1-D bulk copy (TMA
 // engine) into a ring of shared-memory stages.
 //
@@ -95,10 +97,14 @@ struct Cfg {
   static constexpr int OFF_V = (MB + 1) * 2048;
   static constexpr int OFF_NORMS = (MB + 1 + VB) * 2048;
   static constexpr int OFF_VSZ = OFF_NORMS + 512;
-  static constexpr int AV_BYTES = VB * 128 * 128;       // [128 channels] x [VB*128 K]
-  static constexpr int BP_BYTES = VB * 128 * NPV;       // [VB*128 K] x [NPV]
+  // value operands: 2-bit values are stored packed (one operand byte per
+  // channel holds code * 4^m); wider values are bit-planes (one operand each)
+  static constexpr bool PACKED_V = (VB == 2);
+  static constexpr int VOPS = PACKED_V ? 1 : VB;
+  static constexpr int AV_BYTES = VOPS * 128 * 128;     // [128 channels] x [VOPS*128 K]
+  static constexpr int BP_BYTES = VOPS * 128 * NPV;     // [VOPS*128 K] x [NPV]
   static constexpr int BQ_BYTES = (NP + 1) * 128 * NS;  // [(NP+1)*128 K] x [NS]
-  static constexpr int SBO_V = VB * 2048;               // MN-major stride of 16-byte chunks
+  static constexpr int SBO_V = VOPS * 2048;             // MN-major stride of 16-byte chunks
   static constexpr int LBO_Q = (NS / 8) * 128;          // K-major stride of 16-byte K chunks
   static constexpr int QBLOCK = BQ_BYTES + kQConstBytes;  // per (sequence, KV head)
   static constexpr int FIXED = 2 * AV_BYTES + 2 * BP_BYTES + QBLOCK + 4096;
@@ -275,11 +281,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ------------------------------------------
+    // Descriptors are built once; an instruction's operand offsets are
+    // compile-time constants added to the 16-byte-unit address field.
     if (lane == 0) {
       const uint32_t id_s = idesc_i8(128, C::NS, false, true, false, false);
       const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
       const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
       const bool skip3 = Q.skip_product_plane != 0;
+      const uint64_t dq0 = smem_desc(S.bq, C::LBO_Q, 128);
+      const uint64_t dav[2] = {smem_desc(S.av[0], 128, C::SBO_V), smem_desc(S.av[1], 128, C::SBO_V)};
+      const uint64_t dbp[2] = {smem_desc(S.bp[0], 128, C::SBO_V), smem_desc(S.bp[1], 128, C::SBO_V)};
       int last_s = -1, last_p = -1;
       for (int i = 0; qok && i <= ntile; ++i) {
         if (i < ntile) {
@@ -290,20 +301,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           const uint32_t a_base = tbase + C::COL_AK + (i % C::AKB) * C::AK_COLS;
           const uint32_t d_mse = tbase + C::COL_DS + kb * 2 * C::NS;
           const uint32_t d_qjl = d_mse + C::NS;
-          int first = 1;
+#pragma unroll
           for (int p = 0; p < C::NP; ++p) {
             if (MB == 2 && p == 2 && skip3) continue;
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const int ins = p * 4 + kk;
-              mma_i8_ts(d_mse, a_base + ins * 8,
-                        smem_desc(S.bq + 2 * ins * C::LBO_Q, C::LBO_Q, 128), id_s, first ? 0u : 1u);
-              first = 0;
+              mma_i8_ts(d_mse, a_base + ins * 8, dq0 + (uint64_t)((2 * ins * C::LBO_Q) >> 4), id_s,
+                        ins ? 1u : 0u);
             }
           }
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const int ins = C::NP * 4 + kk;
-            mma_i8_ts(d_qjl, a_base + ins * 8, smem_desc(S.bq + 2 * ins * C::LBO_Q, C::LBO_Q, 128),
-                      id_s, kk ? 1u : 0u);
+            mma_i8_ts(d_qjl, a_base + ins * 8, dq0 + (uint64_t)((2 * ins * C::LBO_Q) >> 4), id_s,
+                      kk ? 1u : 0u);
           }
           mma_commit(&S.s_ready[kb]);
           last_s = i;
@@ -315,9 +327,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           if (jt >= 2 && !wait_bar(&S.pv_free[pb], ((jt - 2) >> 1) & 1, &S.abort_flag, status)) break;
           tc_fence_after();
           const uint32_t d_pv = tbase + C::COL_DPV + pb * C::NPV;
-          for (int ins = 0; ins < C::VB * 4; ++ins)
-            mma_i8_ss(d_pv, smem_desc(S.av[pb] + 512 * ins, 128, C::SBO_V),
-                      smem_desc(S.bp[pb] + 512 * ins, 128, C::SBO_V), id_p, ins ? 1u : 0u);
+          const uint64_t da = dav[pb], db = dbp[pb];
+#pragma unroll
+          for (int ins = 0; ins < C::VOPS * 4; ++ins)
+            mma_i8_ss(d_pv, da + (uint64_t)(32 * ins), db + (uint64_t)(32 * ins), id_p, ins ? 1u : 0u);
           mma_commit(&S.pv_done[pb]);
           last_p = jt;
         }
@@ -377,8 +390,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     const int q4 = warp & 3;
     const int t = 32 * q4 + lane;  // token slot for expansion; M slot for PV
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    const int kk = (t & 31) >> 2;  // mask index of this M slot
-    const int chan = 32 * q4 + 8 * (t & 3) + kk;
+    // channel of this M slot and the 2^kk weight its operand bytes carry
+    const int kk = C::PACKED_V ? 2 * ((t >> 2) & 3) : (t & 31) >> 2;
+    const int chan = C::PACKED_V ? 16 * (t >> 4) + 4 * (t & 3) + ((t >> 2) & 3)
+                                 : 32 * q4 + 8 * (t & 3) + kk;
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = 0.f;
@@ -387,24 +402,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         const int s = i % C::STAGES, vb = i & 1;
         if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
         const uint8_t *st = S.stage[s];
-        uint4 vp[VB];
-#pragma unroll
-        for (int p = 0; p < VB; ++p)
-          vp[p] = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[s]);
         uint8_t *av = S.av[vb];
+        if constexpr (C::PACKED_V) {
+          // packed row: word w holds channels 16w .. 16w+15; mask m keeps
+          // channel 16w + 4i + m in byte i as code * 4^m (M slot 16w + 4m + i)
+          const uint4 v0 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes);
+          const uint4 v1 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes + 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.empty[s]);
+          const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          uint8_t *row = av + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
-        for (int p = 0; p < VB; ++p) {
-          const uint32_t vw[4] = {vp[p].x, vp[p].y, vp[p].z, vp[p].w};
-          uint8_t *row = av + p * 2048 + (t >> 3) * 128 + (t & 7) * 16;
+          for (int w = 0; w < 8; ++w)
+            *reinterpret_cast<uint4 *>(row + w * C::SBO_V) =
+                make_uint4(vw[w] & 0x03030303u, vw[w] & 0x0C0C0C0Cu, vw[w] & 0x30303030u,
+                           vw[w] & 0xC0C0C0C0u);
+        } else {
+          uint4 vp[VB];
 #pragma unroll
-          for (int m16 = 0; m16 < 8; ++m16) {
-            const uint32_t word = vw[m16 >> 1];
-            const int k0 = (m16 & 1) * 4;
-            *reinterpret_cast<uint4 *>(row + m16 * C::SBO_V) =
-                make_uint4(word & (0x01010101u << k0), word & (0x01010101u << (k0 + 1)),
-                           word & (0x01010101u << (k0 + 2)), word & (0x01010101u << (k0 + 3)));
+          for (int p = 0; p < VB; ++p)
+            vp[p] = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.empty[s]);
+#pragma unroll
+          for (int p = 0; p < VB; ++p) {
+            const uint32_t vw[4] = {vp[p].x, vp[p].y, vp[p].z, vp[p].w};
+            uint8_t *row = av + p * 2048 + (t >> 3) * 128 + (t & 7) * 16;
+#pragma unroll
+            for (int m16 = 0; m16 < 8; ++m16) {
+              const uint32_t word = vw[m16 >> 1];
+              const int k0 = (m16 & 1) * 4;
+              *reinterpret_cast<uint4 *>(row + m16 * C::SBO_V) =
+                  make_uint4(word & (0x01010101u << k0), word & (0x01010101u << (k0 + 1)),
+                             word & (0x01010101u << (k0 + 2)), word & (0x01010101u << (k0 + 3)));
+            }
           }
         }
         fence_proxy_async_smem();
@@ -561,13 +592,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       if (jt >= 2 && !wait_bar(&S.pv_free[pb], ((jt - 2) >> 1) & 1, &S.abort_flag, status)) break;
       uint8_t *bp = S.bp[pb];
 #pragma unroll
-      for (int p = 0; p < VB; ++p) {
-        // n = group * 4G + head * 4 + byte: one u32 per (group, head)
+      for (int p = 0; p < C::VOPS; ++p) {
+        // n = group * 4G + head * 4 + byte: one u32 per (group, head); the
+        // operand of bit-plane p carries the plane weight 2^p
         uint32_t wv[4 * G];
 #pragma unroll
         for (int gg = 0; gg < 4; ++gg)
 #pragma unroll
-          for (int g = 0; g < G; ++g) wv[gg * G + g] = X[g][gg] << p;
+          for (int g = 0; g < G; ++g) wv[gg * G + g] = C::PACKED_V ? X[g][gg] : (X[g][gg] << p);
         uint8_t *row = bp + p * 2048 + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
         for (int c = 0; c < G; ++c)

@@ -25,9 +25,7 @@ __global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
   for (int p = 0; p < L.mb; ++p)
     idx |= ((tp[L.kplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> bit) & 1) << p;
   const int sbit = (tp[L.signs + slot * kRowBytes + byte] >> bit) & 1;
-  int code = 0;
-  for (int p = 0; p < L.vb; ++p)
-    code |= ((tp[L.vplanes + p * kPlaneBytes + slot * kRowBytes + byte] >> bit) & 1) << p;
+  const int code = value_code(tp, L, slot, j);
   c[j] = a.centroids[idx];
   sg[j] = sbit ? 1.f : -1.f;
   __syncthreads();

@@ -114,11 +114,22 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
             tq = fminf(fmaxf(tq, 0.f), vlevels);
             code = (int)tq;
           }
-          for (int p = 0; p < L.vb; ++p) {
-            const unsigned word = __ballot_sync(0xffffffffu, (code >> p) & 1);
-            if (lane == 0)
-              *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * kPlaneBytes +
-                                            slot * kRowBytes + 4 * m) = word;
+          if (L.vb == 2) {
+            // packed codes: channel 4i + m' of a row in bits 2m', 2m'+1 of byte i
+            const unsigned lo = __ballot_sync(0xffffffffu, code & 1);
+            const unsigned hi = __ballot_sync(0xffffffffu, (code >> 1) & 1);
+            if (lane == 0) {
+              uint32_t *dst = reinterpret_cast<uint32_t *>(tile + L.vplanes + slot * kPackedRowBytes + 8 * m);
+              dst[0] = spread_bits16(lo & 0xFFFFu) | (spread_bits16(hi & 0xFFFFu) << 1);
+              dst[1] = spread_bits16(lo >> 16) | (spread_bits16(hi >> 16) << 1);
+            }
+          } else {
+            for (int p = 0; p < L.vb; ++p) {
+              const unsigned word = __ballot_sync(0xffffffffu, (code >> p) & 1);
+              if (lane == 0)
+                *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * kPlaneBytes +
+                                              slot * kRowBytes + 4 * m) = word;
+            }
           }
           if (lane == 0) {
             __half2 sz = __halves2half2(scale16, zero16);

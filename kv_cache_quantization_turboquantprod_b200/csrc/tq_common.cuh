@@ -17,6 +17,7 @@ constexpr int kGroups = kD / kGroup;
 constexpr int kTile = TQ_TILE_TOKENS;
 constexpr int kRowBytes = kD / 8;  // one bit-plane row of a token
 constexpr int kPlaneBytes = kTile * kRowBytes;  // 2048
+constexpr int kPackedRowBytes = kD / 4;         // packed 2-bit value codes of a token
 
 // Byte offsets of the sections inside one tile.
 struct TileLayout {
@@ -52,9 +53,29 @@ __device__ __forceinline__ uint8_t *tile_ptr(void *data, const TileLayout &L,
   return reinterpret_cast<uint8_t *>(data) + idx * (size_t)L.tile_bytes;
 }
 
+// Value code of channel j of token slot `slot`: packed 2-bit codes (channel
+// 4i + m in bits 2m, 2m+1 of byte i) for 2-bit values, bit-planes otherwise.
+__device__ __forceinline__ int value_code(const uint8_t *tile, const TileLayout &L, int slot, int j) {
+  if (L.vb == 2) return (tile[L.vplanes + slot * kPackedRowBytes + (j >> 2)] >> (2 * (j & 3))) & 3;
+  int code = 0;
+  for (int p = 0; p < L.vb; ++p)
+    code |= ((tile[L.vplanes + p * kPlaneBytes + slot * kRowBytes + (j >> 3)] >> (j & 7)) & 1) << p;
+  return code;
+}
+
 __device__ __forceinline__ float load_elem(const void *p, tq_dtype dt, size_t i) {
   if (dt == TQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
   return reinterpret_cast<const float *>(p)[i];
+}
+
+// Bits 0..15 of x moved to the even positions 0, 2, .., 30.
+__device__ __forceinline__ uint32_t spread_bits16(uint32_t x) {
+  x &= 0xFFFFu;
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  x = (x | (x << 1)) & 0x55555555u;
+  return x;
 }
 
 __device__ __forceinline__ float warp_sum(float x) {

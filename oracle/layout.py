@@ -13,7 +13,10 @@ The pages do not fix a layout (reading).  The spec:
     1. key code bit-planes: mb planes (mb = key_bits - 1); plane p is
        [128 tokens][d/8 bytes] and holds bit p of every Lloyd-Max index;
     2. the QJL sign plane: [128][d/8], bit = 1 for sign +1;
-    3. value code bit-planes: vb planes, [128][d/8] each, bit p of the code;
+    3. value codes: for 2-bit values, packed codes [128 tokens][d/4 bytes],
+       byte i holding channels 4i .. 4i+3, channel 4i + m in bits 2m, 2m+1;
+       for 3- and 4-bit values, vb bit-planes [128][d/8] each (bit p of the
+       code);
     4. norms: [128] x (nk, rn) as two little-endian fp16 (4 bytes a token);
     5. value scale/zero: [128][d/group] x (scale, zero) as two fp16.
 * Inside a plane row, byte i, bit k (LSB = 0) holds coordinate 8 i + k.
@@ -68,6 +71,20 @@ def _bits_to_plane_row(bits: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint16) * weights).sum(axis=-1).astype(np.uint8)
 
 
+def _codes_to_packed2_row(codes: np.ndarray) -> np.ndarray:
+    """[..., d] codes in 0..3 -> [..., d/4] bytes, channel 4i+m at bits 2m, 2m+1."""
+    c = np.asarray(codes, np.uint16).reshape(*codes.shape[:-1], -1, 4)
+    weights = (1 << (2 * np.arange(4))).astype(np.uint16)
+    return (c * weights).sum(axis=-1).astype(np.uint8)
+
+
+def _packed2_row_to_codes(rows: np.ndarray, d: int) -> np.ndarray:
+    r = np.asarray(rows, np.uint8)
+    m = (2 * np.arange(4)).astype(np.uint8)
+    c = (r[..., :, None] >> m) & 3
+    return c.reshape(*r.shape[:-1], d)
+
+
 def _plane_row_to_bits(rows: np.ndarray, d: int) -> np.ndarray:
     r = np.asarray(rows, np.uint8)
     k = np.arange(8, dtype=np.uint8)
@@ -108,9 +125,13 @@ class CacheSpec:
         o = base + self.off["signs"] + slot * rowb
         buf[o:o + rowb] = _bits_to_plane_row(keyrec["sign"][i])
         codes = valrec["codes"][i]
-        for p in range(self.value_bits):
-            o = base + self.off["vplanes"] + p * plane + slot * rowb
-            buf[o:o + rowb] = _bits_to_plane_row((codes >> p) & 1)
+        if self.value_bits == 2:
+            o = base + self.off["vplanes"] + slot * (d // 4)
+            buf[o:o + d // 4] = _codes_to_packed2_row(codes)
+        else:
+            for p in range(self.value_bits):
+                o = base + self.off["vplanes"] + p * plane + slot * rowb
+                buf[o:o + rowb] = _bits_to_plane_row((codes >> p) & 1)
         o = base + self.off["norms"] + slot * 4
         buf[o:o + 4] = np.array([keyrec["nk16"][i], keyrec["rn16"][i]],
                                 np.float16).view(np.uint8)
@@ -140,9 +161,12 @@ class CacheSpec:
                 _bits_to_plane_row((idx >> p) & 1))
         put(base + self.off["signs"] + slot * rowb, _bits_to_plane_row(keyrec["sign"]))
         codes = np.asarray(valrec["codes"])
-        for p in range(self.value_bits):
-            put(base + self.off["vplanes"] + p * plane + slot * rowb,
-                _bits_to_plane_row((codes >> p) & 1))
+        if self.value_bits == 2:
+            put(base + self.off["vplanes"] + slot * (d // 4), _codes_to_packed2_row(codes))
+        else:
+            for p in range(self.value_bits):
+                put(base + self.off["vplanes"] + p * plane + slot * rowb,
+                    _bits_to_plane_row((codes >> p) & 1))
         nr = np.stack([keyrec["nk16"], keyrec["rn16"]], axis=1).astype(np.float16)
         put(base + self.off["norms"] + slot * 4, nr.view(np.uint8).reshape(n, 4))
         sz = np.stack([valrec["scale16"], valrec["zero16"]], axis=2).astype(np.float16)
@@ -170,9 +194,13 @@ class CacheSpec:
             idx |= _plane_row_to_bits(rows, d).astype(np.int64) << p
         sign = _plane_row_to_bits(get(base + self.off["signs"] + slot * rowb, rowb), d)
         codes = np.zeros((count, d), np.int64)
-        for p in range(self.value_bits):
-            rows = get(base + self.off["vplanes"] + p * plane + slot * rowb, rowb)
-            codes |= _plane_row_to_bits(rows, d).astype(np.int64) << p
+        if self.value_bits == 2:
+            rows = get(base + self.off["vplanes"] + slot * (d // 4), d // 4)
+            codes = _packed2_row_to_codes(rows, d).astype(np.int64)
+        else:
+            for p in range(self.value_bits):
+                rows = get(base + self.off["vplanes"] + p * plane + slot * rowb, rowb)
+                codes |= _plane_row_to_bits(rows, d).astype(np.int64) << p
         nr = get(base + self.off["norms"] + slot * 4, 4).copy().view(np.float16)
         nr = nr.astype(np.float64).reshape(count, 2)
         sz = get(base + self.off["vsz"] + slot * 4 * ng, 4 * ng).copy().view(np.float16)
@@ -204,9 +232,13 @@ class CacheSpec:
                 idx[i] |= _plane_row_to_bits(buf[o:o + rowb], d).astype(np.int64) << p
             o = base + self.off["signs"] + slot * rowb
             sign[i] = _plane_row_to_bits(buf[o:o + rowb], d)
-            for p in range(self.value_bits):
-                o = base + self.off["vplanes"] + p * plane + slot * rowb
-                codes[i] |= _plane_row_to_bits(buf[o:o + rowb], d).astype(np.int64) << p
+            if self.value_bits == 2:
+                o = base + self.off["vplanes"] + slot * (d // 4)
+                codes[i] = _packed2_row_to_codes(buf[o:o + d // 4], d)
+            else:
+                for p in range(self.value_bits):
+                    o = base + self.off["vplanes"] + p * plane + slot * rowb
+                    codes[i] |= _plane_row_to_bits(buf[o:o + rowb], d).astype(np.int64) << p
             o = base + self.off["norms"] + slot * 4
             nr = buf[o:o + 4].copy().view(np.float16).astype(np.float64)
             nk[i], rn[i] = nr[0], nr[1]

@@ -31,7 +31,7 @@ def test_single_bit_positions_by_hand():
     kr, vr = _blank(1)
     kr["idx"][0, 13] = 2          # bit 1 of coordinate 13 -> plane 1, byte 1, bit 5
     kr["sign"][0, 127] = 1        # byte 15, bit 7
-    vr["codes"][0, 64] = 1        # value plane 0, byte 8, bit 0
+    vr["codes"][0, 65] = 2        # 2-bit values packed: byte 16, bits 2-3 -> 0b1000
     kr["nk16"][0] = 1.0           # fp16 0x3C00
     kr["rn16"][0] = -2.0          # fp16 0xC000
     vr["scale16"][0, 3] = 0.5     # fp16 0x3800, group 3 scale
@@ -42,7 +42,7 @@ def test_single_bit_positions_by_hand():
     slot = 2
     assert buf[base + 1 * 2048 + slot * 16 + 1] == 1 << 5
     assert buf[base + 2 * 2048 + slot * 16 + 15] == 1 << 7
-    assert buf[base + 3 * 2048 + slot * 16 + 8] == 1
+    assert buf[base + 3 * 2048 + slot * 32 + 16] == 0b1000
     norms = base + 5 * 2048 + slot * 4
     assert list(buf[norms:norms + 4]) == [0x00, 0x3C, 0x00, 0xC0]
     vsz = base + 5 * 2048 + 512 + slot * 16 + 3 * 4
@@ -80,3 +80,16 @@ def test_roundtrip_and_readers_agree():
         for i in range(n):
             spec.write(buf2, 1, 0, 50 + i, kr, vr, i)
         assert np.array_equal(buf, buf2)
+
+
+def test_three_bit_values_stay_bit_planes():
+    spec = layout.CacheSpec(batch=1, h_kv=1, capacity=128, d=128, key_bits=3,
+                            value_bits=3, group=32)
+    buf = spec.empty()
+    kr, vr = _blank(1)
+    vr["codes"][0, 64] = 5        # 0b101 -> planes 0 and 2, byte 8, bit 0
+    spec.write(buf, 0, 0, 1, kr, vr, 0)
+    vbase = 3 * 2048              # after 2 key planes and the sign plane
+    assert buf[vbase + 0 * 2048 + 1 * 16 + 8] == 1
+    assert buf[vbase + 1 * 2048 + 1 * 16 + 8] == 0
+    assert buf[vbase + 2 * 2048 + 1 * 16 + 8] == 1
