@@ -1,5 +1,5 @@
 // Decode attention over the compressed cache on the 5th-generation tensor
-// cores (tcgen05, kind::i8), one CTA per (split, KV head, sequence).
+// cores (tcgen05), one CTA per (split, KV head, sequence).
 //
 // What it computes is the one-pass decode of "03. Results & Benchmarks"
 // (turboquant_cutile, "Latency Benchmarks": score, QJL correction, online
@@ -10,32 +10,40 @@
 // How.  Decode is HBM-bound on the packed records, but a SIMT
 // implementation cannot retire a 128-coordinate dot product per (token,
 // query head) inside the ~20 issue slots per record that full bandwidth
-// allows.  The bit-planes are therefore fed to the tensor cores as exact
-// 0/2^k integer operands: one LOP3 (w & (0x01010101 << k)) turns a 32-bit
-// plane word into four u8 operands, and
-//   * scores: D[token, (head, limb)] = A_k[token, plane bits] x B_q, where
-//     B_q holds the rotated query (times the plane weight, divided by 2^k)
-//     as four signed base-128 fixed-point limbs; s32 accumulation is exact;
-//     the centroid lookup is exact because c(idx) is multilinear in the code
-//     bits (2-bit codes) or a sum of threshold planes (3-bit codes);
-//   * values: D[channel, (group, head, byte)] = A_v[channel, codes x tokens]
-//     x B_p[tokens, p * scale_g as 22-bit fixed point]; 2-bit codes are
-//     stored packed, so one mask (w & (0x03030303 << 2m)) yields code * 4^m
-//     operands; wider codes are bit-planes whose B_p copies carry 2^plane.
-//     The 4^m (or 2^k) weight of each operand row is undone per channel.
+// allows, so both contractions run on the tensor cores with exact operands.
+//
+//   Scores (kind::mxf4, K = 64 per instruction, unit block scales).  Write
+//   the code bits of coordinate j as spins s_k = 2 b_k - 1.  Any codebook
+//   of 2^m levels is a multilinear polynomial in the spins (its Walsh
+//   expansion), c(idx) = a_0 + sum_S a_S prod_{k in S} s_k, and for the
+//   symmetric Lloyd-Max codebooks only the odd subsets S survive (1, 2 and
+//   4 planes at m = 1, 2, 3).  Each subset's spin product and the QJL sign
+//   (2 sign - 1 is a spin too) become +-1 e2m1 operands, four per byte
+//   operation; the query side B holds a_S Pi q (and S q) as balanced base-9
+//   digits in [-4, 4], all exact in e2m1, so every product and the f32
+//   accumulation of a 128-coordinate tile is exact.  The limbs are combined
+//   per (token, head) in the epilogue.
+//   Values (kind::i8): D[channel, (group, head, byte)] = A_v[channel, code
+//   bytes x tokens] x B_p[tokens, p * scale_g as 22-bit fixed point].  Two-
+//   bit codes are stored packed, so one mask (w & (0x03030303 << 2m))
+//   yields code * 4^m operands; wider codes are assembled from their bit-
+//   planes into one code byte.  The 4^m weight of each row is undone per
+//   channel.
 // Per 128-token tile the record bytes arrive by one 1-D bulk copy (TMA
 // engine) into a ring of shared-memory stages.
 //
-// Warp roles (448 threads; each SM sub-partition gets one warp of each
-// worker group, so the three per-token instruction streams overlap):
-//   warp 0       bulk-copy producer; allocates / frees tensor memory
-//   warp 1       single-thread MMA issuer (tcgen05.mma + commit)
-//   warps 2-5    key group: key bit-planes -> A_k operand in tensor memory
-//   warps 6-9    value group: V bit-planes -> A_v (MN-major, shared memory);
-//                PV epilogue and the per-channel accumulators
-//   warps 10-13  softmax group: score epilogue, online softmax (tile max by
-//                warp redux + an mbarrier exchange), the P' operand, running
-//                l and zero-point sums
+// Warp roles (576 threads; each SM sub-partition gets one warp of each
+// worker group):
+//   warp 0        bulk-copy producer; allocates / frees tensor memory
+//   warp 1        MMA issuer (one elected lane issues), polling the score
+//                 and PV queues so neither blocks the other
+//   warps 2-5     key group: code bits -> spin planes (shared memory)
+//   warps 6-9     value group: codes -> A_v (MN-major, shared memory); PV
+//                 epilogue and the per-channel accumulators
+//   warps 10-17   two softmax groups taking alternate tiles, each with its
+//                 own running max / sum (merged at the end like two splits):
+//                 score epilogue, tile max by warp redux + an mbarrier
+//                 exchange, the P' operand, running l and zero-point sums
 // Every mbarrier wait is bounded (2 s); on timeout the CTA sets the status word in
 // the workspace, stops, waits for its own copies and MMAs and frees TMEM.
 #include <math.h>
@@ -50,77 +58,92 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 448;
+constexpr int kTcThreads = 576;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kTmemCols = 512;
+constexpr int kColSF = 448;         // 64 columns of 1.0 block scales (ue8m0 0x7F)
+constexpr int kPlaneBytes4 = 128 * 64;  // one e2m1 operand plane: 128 rows x 128 coordinates
 
 // 2^n for n in [-126, 127]
 __device__ __forceinline__ float exp2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
 // floor(log2(x)) for a positive normal float
 __device__ __forceinline__ int ilog2f(float x) { return (int)((__float_as_uint(x) >> 23) & 0xFF) - 127; }
 
-// Score constants that follow B_q in a query block (floats): cm[8] (c_0 sum
-// q~), csum[8] (sum s^), coef_m[8][2], coef_s[8][2] (limb weights), then the
-// skip flag of the product plane (int).
+// balanced base-9 digits per query coordinate: 8 (|X| < 2^24.3), or 6 when
+// eight do not fit the tensor-memory budget (8 query heads per KV head)
+__host__ __device__ constexpr int limbs_for(int G) { return G <= 6 ? 8 : 6; }
+// floor(log2((9^L - 1) / 2)): the largest |X| is below 2^(this + 1)
+__host__ __device__ constexpr int xbits_for(int L) {
+  long long x = 1;
+  for (int l = 0; l < L; ++l) x *= 9;
+  x = (x - 1) / 2;
+  int e = 0;
+  while ((x >> (e + 1)) != 0) ++e;
+  return e;
+}
+__host__ __device__ constexpr int score_n(int G) { return ((limbs_for(G) * G + 15) / 16) * 16; }
+// all non-empty code-bit subsets + the sign plane
+__host__ __device__ constexpr int max_planes(int MB) { return (1 << MB); }
+
+// Score constants that follow B_q in a query block.
 constexpr int kQConstBytes = 256;
 struct QConst {
-  float cm[8];
-  float csum[8];
-  float coef_m[8][2];
-  float coef_s[8][2];
-  int skip_product_plane;
+  float cm[8];      // a_0 * sum_j q~_j
+  float inv_m[8];   // 2^-F of the MSE limbs
+  float inv_s[8];   // 2^-F of the QJL limbs
+  int n_mse;        // active subset planes (1 .. 2^m - 1)
+  int subset[7];    // their code-bit masks
 };
 static_assert(sizeof(QConst) <= kQConstBytes, "query constants");
+
+__host__ __device__ constexpr size_t qblock_bytes_for(int MB, int G) {
+  return (size_t)max_planes(MB) * 64 * score_n(G) + kQConstBytes;
+}
 
 template <int MB_, int VB_, int G_>
 struct Cfg {
   static constexpr int MB = MB_, VB = VB_, G = G_;
-  // operand planes of the MSE term: b0 (1 bit); b0, b1, b0&b1 (2 bits,
-  // multilinear, exact for any 4-level codebook); [idx >= l], l = 1..7
-  // (3 bits, threshold planes)
-  static constexpr int NP = MB == 1 ? 1 : (MB == 2 ? 3 : 7);
-  static constexpr int AK_COLS = (NP + 1) * 32;          // one A_k buffer
-  static constexpr int NS = ((4 * G + 15) / 16) * 16;   // score N per accumulator
+  // MSE planes of a symmetric codebook (the odd code-bit subsets)
+  static constexpr int NSYM = MB == 1 ? 1 : (MB == 2 ? 2 : 4);
+  static constexpr int L = limbs_for(G);
+  static constexpr int NS = score_n(G);                 // score N per accumulator
   static constexpr int NPV = 16 * G;                    // PV N: 4 groups x G heads x 4 bytes
-  static constexpr int DS_COLS = 4 * NS;                // 2 buffers x (mse, qjl)
-  static constexpr int DPV_COLS = 2 * NPV;              // 2 buffers
-  static constexpr int AKB = (2 * AK_COLS + DS_COLS + DPV_COLS <= 512) ? 2 : 1;
-  static constexpr int COL_AK = 0;
-  static constexpr int COL_DS = AKB * AK_COLS;
-  static constexpr int COL_DPV = COL_DS + DS_COLS;
-  static constexpr int COLS_USED = COL_DPV + DPV_COLS;
-  static constexpr int TMEM_COLS =
-      COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
-                                                    : COLS_USED <= 256 ? 256 : 512;
+  static constexpr int NPL = max_planes(MB);            // operand planes, upper bound
+  // A_k plane slots: two buffers of up to NPL planes (at m = 3 two buffers
+  // of the 5 planes a symmetric codebook needs; one buffer otherwise)
+  static constexpr int AK_SLOTS = MB == 3 ? 10 : 2 * NPL;
+  static constexpr int COL_DS = 0;                      // 2 buffers x (mse, qjl)
+  static constexpr int COL_DPV = 4 * NS;                // 2 buffers
+  static constexpr int BQ_PLANE = 64 * NS;              // e2m1 [NS][128]
+  static constexpr int BQ_BYTES = NPL * BQ_PLANE;
+  static constexpr int QBLOCK = BQ_BYTES + kQConstBytes;
   static constexpr int REC = (MB + 1 + VB) * 16 + 20;
   static constexpr int TILE_BYTES = 128 * REC;
   static constexpr int OFF_SIGNS = MB * 2048;
   static constexpr int OFF_V = (MB + 1) * 2048;
   static constexpr int OFF_NORMS = (MB + 1 + VB) * 2048;
   static constexpr int OFF_VSZ = OFF_NORMS + 512;
-  // value operands: 2-bit values are stored packed (one operand byte per
-  // channel holds code * 4^m); wider values are bit-planes (one operand each)
   static constexpr bool PACKED_V = (VB == 2);
-  static constexpr int VOPS = PACKED_V ? 1 : VB;
-  static constexpr int AV_BYTES = VOPS * 128 * 128;     // [128 channels] x [VOPS*128 K]
-  static constexpr int BP_BYTES = VOPS * 128 * NPV;     // [VOPS*128 K] x [NPV]
-  static constexpr int BQ_BYTES = (NP + 1) * 128 * NS;  // [(NP+1)*128 K] x [NS]
-  static constexpr int SBO_V = VOPS * 2048;             // MN-major stride of 16-byte chunks
-  static constexpr int LBO_Q = (NS / 8) * 128;          // K-major stride of 16-byte K chunks
-  static constexpr int QBLOCK = BQ_BYTES + kQConstBytes;  // per (sequence, KV head)
-  static constexpr int FIXED = 2 * AV_BYTES + 2 * BP_BYTES + QBLOCK + 4096;
+  static constexpr int AV_BYTES = 128 * 128;            // [128 channel slots] x [128 tokens]
+  static constexpr int BP_BYTES = 128 * NPV;            // [128 tokens] x [NPV]
+  static constexpr int SBO_V = 2048;                    // MN-major stride of 16-byte chunks
+  static constexpr int FIXED = AK_SLOTS * kPlaneBytes4 + 2 * AV_BYTES + 2 * BP_BYTES + QBLOCK + 4096;
   static constexpr int STAGES_FIT = (220 * 1024 - FIXED) / TILE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static_assert(COLS_USED <= 512, "tensor memory budget");
+  static_assert(COL_DPV + 2 * NPV <= kColSF, "tensor memory budget");
   static_assert(STAGES >= 2, "shared memory budget");
   static_assert(TILE_BYTES % 16 == 0, "bulk copy size");
+  static_assert(QBLOCK == (int)qblock_bytes_for(MB, G), "query block size");
+  static_assert(2 * L * ((G + 1) / 2) <= NS && (2 * L) % 4 == 0, "score limb loads");
 };
 
 template <class C>
 struct TcSmem {
   alignas(128) uint8_t stage[C::STAGES][C::TILE_BYTES];
+  alignas(128) uint8_t ak[C::AK_SLOTS][kPlaneBytes4];
   alignas(128) uint8_t av[2][C::AV_BYTES];
   alignas(128) uint8_t bp[2][C::BP_BYTES];
-  alignas(128) uint8_t bq[C::BQ_BYTES + kQConstBytes];  // B_q operand + score constants
+  alignas(128) uint8_t bq[C::QBLOCK];  // B_q operand + score constants
   uint64_t full[C::STAGES];
   uint64_t empty[C::STAGES];
   uint64_t ak_ready[2], s_ready[2], s_free[2], av_ready[2], p_ready[2], pv_done[2], pv_free[2];
@@ -128,11 +151,12 @@ struct TcSmem {
   uint64_t q_full;
   uint32_t tmem_base;
   volatile int abort_flag;
-  uint32_t red[2][4][C::G + 1];
+  uint32_t red[2][2][4][C::G + 1];  // [softmax group][slot][warp][head | value scale]
   float alpha[2][C::G];
   float pscale[2];
-  float zsum[4][C::G][4];
-  float lsum[4][C::G];
+  float fin_m[2][C::G];
+  float lsum[2][4][C::G];
+  float zsum[2][4][C::G][4];
 };
 
 // Bounded wait (2 s of wall time) that also gives up when another role has
@@ -151,22 +175,37 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   return false;
 }
 
-// Operand plane `op` of the MSE term for one 32-bit word of each bit-plane.
-template <int MB>
-__device__ __forceinline__ uint32_t mse_plane_word(int op, const uint32_t (&bw)[3]) {
-  if (MB == 1) return bw[0];
-  if (MB == 2) return op == 0 ? bw[0] : (op == 1 ? bw[1] : (bw[0] & bw[1]));
-  // MB == 3: threshold planes [idx >= op + 1]
-  const uint32_t b0 = bw[0], b1 = bw[1], b2 = bw[2];
-  switch (op) {
-    case 0: return b0 | b1 | b2;
-    case 1: return b1 | b2;
-    case 2: return b2 | (b1 & b0);
-    case 3: return b2;
-    case 4: return b2 & (b1 | b0);
-    case 5: return b2 & b1;
-    default: return b2 & b1 & b0;
-  }
+// Spin word of code-bit subset S over 32 coordinates: bit set <=> the
+// product of the spins 2 b_k - 1, k in S, is +1 (an even number of zero bits).
+__device__ __forceinline__ uint32_t subset_word(int S, uint32_t b0, uint32_t b1, uint32_t b2) {
+  uint32_t x = ((S & 1) ? b0 : 0u) ^ ((S & 2) ? b1 : 0u) ^ ((S & 4) ? b2 : 0u);
+  return (__popc(S) & 1) ? x : ~x;
+}
+
+// Four e2m1 operand words of one 32-coordinate spin word w: word k, nibble n
+// is coordinate 4n + k: +1.0 (0x2) where the bit is set, -1.0 (0xA) where not.
+__device__ __forceinline__ uint4 spin_nibbles(uint32_t w) {
+  const uint32_t nw = ~w;
+  return make_uint4(0x22222222u | ((nw << 3) & 0x88888888u), 0x22222222u | ((nw << 2) & 0x88888888u),
+                    0x22222222u | ((nw << 1) & 0x88888888u), 0x22222222u | (nw & 0x88888888u));
+}
+
+// Score MMAs of one tile with a compile-time plane count: planes 0..NPM-1
+// accumulate the MSE term, plane NPM (the signs) the QJL term; two K = 64
+// halves per plane.
+template <int NPM, int NS, int BQ_PLANE>
+__device__ __forceinline__ void issue_scores(bool leader, uint64_t da, uint64_t dbq, uint32_t d_mse,
+                                             uint32_t d_qjl, uint32_t id_s, uint32_t sf) {
+#pragma unroll
+  for (int p = 0; p <= NPM; ++p)
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint64_t a_d = da + (uint64_t)((p * kPlaneBytes4 + m * 4096) >> 4);
+      const uint64_t b_d = dbq + (uint64_t)((p * BQ_PLANE + m * 32 * NS) >> 4);
+      const uint32_t d = p < NPM ? d_mse : d_qjl;
+      const uint32_t acc = (p < NPM) ? ((p | m) ? 1u : 0u) : (m ? 1u : 0u);
+      if (leader) mma_mxf4_ss(d, a_d, b_d, id_s, sf, sf, acc);
+    }
 }
 
 template <int N>
@@ -201,6 +240,15 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
 #pragma unroll
     for (int x = 0; x < 4; ++x) r[c + x] = t[x];
   }
+}
+
+// sum_l 9^l D_l over one head's limbs (f32 columns)
+template <int L>
+__device__ __forceinline__ float combine_limbs(const uint32_t *d) {
+  float h = __uint_as_float(d[L - 1]);
+#pragma unroll
+  for (int l = L - 2; l >= 0; --l) h = fmaf(h, 9.f, __uint_as_float(d[l]));
+  return h;
 }
 
 template <int MB, int VB, int G>
@@ -247,7 +295,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&S.tmem_base, C::TMEM_COLS);
+  if (warp == 0) tmem_alloc(&S.tmem_base, kTmemCols);
 
   const uint8_t *tiles = reinterpret_cast<const uint8_t *>(a.data) +
                          (((size_t)b * a.h_kv + h) * a.ntiles + tile0) * (size_t)C::TILE_BYTES;
@@ -281,106 +329,152 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ------------------------------------------
-    // Descriptors are built once; an instruction's operand offsets are
-    // compile-time constants added to the 16-byte-unit address field.
-    if (lane == 0) {
-      const uint32_t id_s = idesc_i8(128, C::NS, false, true, false, false);
-      const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
-      const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
-      const bool skip3 = Q.skip_product_plane != 0;
-      const uint64_t dq0 = smem_desc(S.bq, C::LBO_Q, 128);
-      const uint64_t dav[2] = {smem_desc(S.av[0], 128, C::SBO_V), smem_desc(S.av[1], 128, C::SBO_V)};
-      const uint64_t dbp[2] = {smem_desc(S.bp[0], 128, C::SBO_V), smem_desc(S.bp[1], 128, C::SBO_V)};
-      int last_s = -1, last_p = -1;
-      for (int i = 0; qok && i <= ntile; ++i) {
-        if (i < ntile) {
-          const int kb = i & 1;
-          if (!wait_bar(&S.ak_ready[kb], (i >> 1) & 1, &S.abort_flag, status)) break;
-          if (i >= 2 && !wait_bar(&S.s_free[kb], ((i - 2) >> 1) & 1, &S.abort_flag, status)) break;
-          tc_fence_after();
-          const uint32_t a_base = tbase + C::COL_AK + (i % C::AKB) * C::AK_COLS;
-          const uint32_t d_mse = tbase + C::COL_DS + kb * 2 * C::NS;
-          const uint32_t d_qjl = d_mse + C::NS;
+    // The whole warp runs the loop, so queue tests and descriptor arithmetic
+    // stay warp-uniform; one elected lane issues each tcgen05 instruction.
+    // It polls both queues (score of tile is, PV of tile ip) with
+    // non-blocking tests and issues whichever is ready.
+    const bool leader = elect_one();
+    const uint32_t id_s = idesc_mxf4(128, C::NS);
+    const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
+    const uint32_t sf = tbase + kColSF;
+    const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
+    const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
+    const int akb = (2 * npl <= C::AK_SLOTS) ? 2 : 1;
+    const uint64_t dak = smem_desc(S.ak[0], 2048, 128);
+    const uint64_t dbq = smem_desc(S.bq, C::NS * 16, 128);
+    const uint64_t dav0 = smem_desc(S.av[0], 128, C::SBO_V), dbp0 = smem_desc(S.bp[0], 128, C::SBO_V);
+    int is = 0, ip = 0;
+    uint32_t idle = 0;
+    uint64_t t_idle = 0;
+    while (qok && ip < ntile) {
+      bool progress = false;
+      bool rs = is < ntile && mbar_test(&S.ak_ready[is & 1], (is >> 1) & 1) &&
+                (is < 2 || mbar_test(&S.s_free[is & 1], ((is - 2) >> 1) & 1));
+      rs = __shfl_sync(0xffffffffu, rs, 0);
+      if (rs) {
+        tc_fence_after();
+        const uint32_t d_mse = tbase + C::COL_DS + (is & 1) * 2 * C::NS;
+        const uint32_t d_qjl = d_mse + C::NS;
+        if (nm == C::NSYM) {
+          // symmetric codebook: plane count and buffer offsets are
+          // compile-time, so the descriptors stay in uniform registers
+          const uint64_t da = dak + (uint64_t)(((is & 1) * (C::NSYM + 1) * kPlaneBytes4) >> 4);
+          issue_scores<C::NSYM, C::NS, C::BQ_PLANE>(leader, da, dbq, d_mse, d_qjl, id_s, sf);
+        } else {
+        const uint64_t da = dak + (uint64_t)(((akb == 2 ? (is & 1) : 0) * npl * kPlaneBytes4) >> 4);
+        for (int p = 0; p < nm; ++p) {
 #pragma unroll
-          for (int p = 0; p < C::NP; ++p) {
-            if (MB == 2 && p == 2 && skip3) continue;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int ins = p * 4 + kk;
-              mma_i8_ts(d_mse, a_base + ins * 8, dq0 + (uint64_t)((2 * ins * C::LBO_Q) >> 4), id_s,
-                        ins ? 1u : 0u);
-            }
+          for (int m = 0; m < 2; ++m) {
+            const uint64_t a_d = da + (uint64_t)((p * kPlaneBytes4 + m * 4096) >> 4);
+            const uint64_t b_d = dbq + (uint64_t)((p * C::BQ_PLANE + m * 32 * C::NS) >> 4);
+            if (leader) mma_mxf4_ss(d_mse, a_d, b_d, id_s, sf, sf, (p | m) ? 1u : 0u);
           }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int ins = C::NP * 4 + kk;
-            mma_i8_ts(d_qjl, a_base + ins * 8, dq0 + (uint64_t)((2 * ins * C::LBO_Q) >> 4), id_s,
-                      kk ? 1u : 0u);
-          }
-          mma_commit(&S.s_ready[kb]);
-          last_s = i;
         }
-        if (i >= 1) {
-          const int jt = i - 1, pb = jt & 1;
-          if (!wait_bar(&S.p_ready[pb], (jt >> 1) & 1, &S.abort_flag, status)) break;
-          if (!wait_bar(&S.av_ready[pb], (jt >> 1) & 1, &S.abort_flag, status)) break;
-          if (jt >= 2 && !wait_bar(&S.pv_free[pb], ((jt - 2) >> 1) & 1, &S.abort_flag, status)) break;
-          tc_fence_after();
-          const uint32_t d_pv = tbase + C::COL_DPV + pb * C::NPV;
-          const uint64_t da = dav[pb], db = dbp[pb];
 #pragma unroll
-          for (int ins = 0; ins < C::VOPS * 4; ++ins)
-            mma_i8_ss(d_pv, da + (uint64_t)(32 * ins), db + (uint64_t)(32 * ins), id_p, ins ? 1u : 0u);
-          mma_commit(&S.pv_done[pb]);
-          last_p = jt;
+        for (int m = 0; m < 2; ++m) {
+          const uint64_t a_d = da + (uint64_t)((nm * kPlaneBytes4 + m * 4096) >> 4);
+          const uint64_t b_d = dbq + (uint64_t)((nm * C::BQ_PLANE + m * 32 * C::NS) >> 4);
+          if (leader) mma_mxf4_ss(d_qjl, a_d, b_d, id_s, sf, sf, m ? 1u : 0u);
+        }
+        }
+        if (leader) mma_commit(&S.s_ready[is & 1]);
+        __syncwarp();
+        ++is;
+        progress = true;
+      }
+      bool rp = ip < is && mbar_test(&S.p_ready[ip & 1], (ip >> 1) & 1) &&
+                mbar_test(&S.av_ready[ip & 1], (ip >> 1) & 1) &&
+                (ip < 2 || mbar_test(&S.pv_free[ip & 1], ((ip - 2) >> 1) & 1));
+      rp = __shfl_sync(0xffffffffu, rp, 0);
+      if (rp) {
+        tc_fence_after();
+        const int pb = ip & 1;
+        const uint32_t d_pv = tbase + C::COL_DPV + pb * C::NPV;
+        const uint64_t da = dav0 + (uint64_t)((pb * C::AV_BYTES) >> 4);
+        const uint64_t db = dbp0 + (uint64_t)((pb * C::BP_BYTES) >> 4);
+#pragma unroll
+        for (int ins = 0; ins < 4; ++ins)
+          if (leader) mma_i8_ss(d_pv, da + (uint64_t)(32 * ins), db + (uint64_t)(32 * ins), id_p, ins ? 1u : 0u);
+        if (leader) mma_commit(&S.pv_done[pb]);
+        __syncwarp();
+        ++ip;
+        progress = true;
+      }
+      if (progress) {
+        idle = 0;
+        t_idle = 0;
+      } else if ((++idle & 15u) != 0) {
+        __nanosleep(32);  // yield the issue slots of this sub-partition
+      } else {  // the clock is read rarely
+        if (S.abort_flag) break;
+        const uint64_t now = globaltimer_ns();
+        if (t_idle == 0) {
+          t_idle = now;
+        } else if (now - t_idle > 2000000000ull) {
+          if (leader) {
+            S.abort_flag = 1;
+            atomicOr(status, 1);
+          }
+          break;
         }
       }
-      // never leave with an MMA in flight
-      if (last_s >= 0) mbar_wait(&S.s_ready[last_s & 1], (last_s >> 1) & 1);
-      if (last_p >= 0) mbar_wait(&S.pv_done[last_p & 1], (last_p >> 1) & 1);
     }
+    // never leave with an MMA in flight
+    if (is > 0) mbar_wait(&S.s_ready[(is - 1) & 1], ((is - 1) >> 1) & 1);
+    if (ip > 0) mbar_wait(&S.pv_done[(ip - 1) & 1], ((ip - 1) >> 1) & 1);
   } else if (warp < 6) {
-    // ---------------- key group: A_k expansion ----------------------------
+    // ---------------- key group: spin planes ------------------------------
     const int q4 = warp & 3;
-    const int t = 32 * q4 + lane;  // token slot == TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+    const int t = 32 * q4 + lane;  // token slot == operand row
+    {  // unit block scales for every scaled MMA of this CTA
+      uint32_t r[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) r[x] = 0x7F7F7F7Fu;
+      tmem_st32(tbase + ((uint32_t)(32 * q4) << 16) + kColSF, r);
+      tmem_st32(tbase + ((uint32_t)(32 * q4) << 16) + kColSF + 32, r);
+      tmem_wait_st();
+    }
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
-    const bool skip3 = Q.skip_product_plane != 0;
+    const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
+    const int akb = (2 * npl <= C::AK_SLOTS) ? 2 : 1;
+    int subs[7];
+#pragma unroll
+    for (int p = 0; p < 7; ++p) subs[p] = (qok && p < nm) ? Q.subset[p] : 0;
+    uint8_t *const rowbase = &S.ak[0][0] + (t >> 3) * 128 + (t & 7) * 16;
     for (int i = 0; qok && i < ntile; ++i) {
       const int s = i % C::STAGES;
       if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
-      // the A_k buffer of tile i was last read by the score MMA of tile i - AKB
-      if (i >= C::AKB) {
-        const int prev = i - C::AKB;
+      // the A_k buffer of tile i was last read by the score MMA of tile i - akb
+      if (i >= akb) {
+        const int prev = i - akb;
         if (!wait_bar(&S.s_ready[prev & 1], (prev >> 1) & 1, &S.abort_flag, status)) break;
       }
       const uint8_t *st = S.stage[s];
-      uint32_t bw[4][3];
+      uint32_t bw[3][4];
 #pragma unroll
-      for (int p = 0; p < MB; ++p) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(st + p * kPlaneBytes + t * kRowBytes);
-        bw[0][p] = v.x; bw[1][p] = v.y; bw[2][p] = v.z; bw[3][p] = v.w;
+      for (int p = 0; p < 3; ++p) {
+        if (p < MB) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(st + p * kPlaneBytes + t * kRowBytes);
+          bw[p][0] = v.x; bw[p][1] = v.y; bw[p][2] = v.z; bw[p][3] = v.w;
+        } else {
+          bw[p][0] = bw[p][1] = bw[p][2] = bw[p][3] = 0u;
+        }
       }
-#pragma unroll
-      for (int p = MB; p < 3; ++p) bw[0][p] = bw[1][p] = bw[2][p] = bw[3][p] = 0u;
       const uint4 sv = *reinterpret_cast<const uint4 *>(st + C::OFF_SIGNS + t * kRowBytes);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[s]);
       const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-      const uint32_t a_base = tbase + lane_off + C::COL_AK + (i % C::AKB) * C::AK_COLS;
+      uint8_t *row = rowbase + (akb == 2 ? (i & 1) : 0) * npl * kPlaneBytes4;
 #pragma unroll
-      for (int op = 0; op <= C::NP; ++op) {
-        if (MB == 2 && op == 2 && skip3) continue;
-        uint32_t r[32];
+      for (int p = 0; p < 8; ++p) {
+        if (p > nm) break;
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
-          const uint32_t word = (op < C::NP) ? mse_plane_word<MB>(op, bw[wd]) : sw[wd];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) r[wd * 8 + k] = word & (0x01010101u << k);
+          const uint32_t w = (p < nm) ? subset_word(subs[p < 7 ? p : 6], bw[0][wd], bw[1][wd], bw[2][wd]) : sw[wd];
+          *reinterpret_cast<uint4 *>(row + p * kPlaneBytes4 + wd * 2048) = spin_nibbles(w);
         }
-        tmem_st32(a_base + op * 32, r);
       }
-      tmem_wait_st();
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.ak_ready[i & 1]);
@@ -390,19 +484,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     const int q4 = warp & 3;
     const int t = 32 * q4 + lane;  // token slot for expansion; M slot for PV
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    // channel of this M slot and the 2^kk weight its operand bytes carry
-    const int kk = C::PACKED_V ? 2 * ((t >> 2) & 3) : (t & 31) >> 2;
+    // channel of this M slot and the 4^m weight its operand bytes carry
+    const int kk = C::PACKED_V ? 2 * ((t >> 2) & 3) : 0;
     const int chan = C::PACKED_V ? 16 * (t >> 4) + 4 * (t & 3) + ((t >> 2) & 3)
-                                 : 32 * q4 + 8 * (t & 3) + kk;
-    float acc[G];
+                                 : 32 * (t >> 5) + 8 * (t & 3) + 4 * ((t >> 4) & 1) + ((t >> 2) & 3);
+    float acc[2][G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.f;
+    for (int g = 0; g < G; ++g) acc[0][g] = acc[1][g] = 0.f;
     for (int i = 0; i <= ntile; ++i) {
       if (i < ntile) {
         const int s = i % C::STAGES, vb = i & 1;
         if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
         const uint8_t *st = S.stage[s];
-        uint8_t *av = S.av[vb];
+        uint8_t *row = S.av[vb] + (t >> 3) * 128 + (t & 7) * 16;
         if constexpr (C::PACKED_V) {
           // packed row: word w holds channels 16w .. 16w+15; mask m keeps
           // channel 16w + 4i + m in byte i as code * 4^m (M slot 16w + 4m + i)
@@ -411,31 +505,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.empty[s]);
           const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-          uint8_t *row = av + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
           for (int w = 0; w < 8; ++w)
             *reinterpret_cast<uint4 *>(row + w * C::SBO_V) =
                 make_uint4(vw[w] & 0x03030303u, vw[w] & 0x0C0C0C0Cu, vw[w] & 0x30303030u,
                            vw[w] & 0xC0C0C0C0u);
         } else {
-          uint4 vp[VB];
+          // bit-planes: u32 x of chunk m16 holds, in byte i, the code of
+          // channel 32 (m16 / 2) + 8 i + 4 (m16 % 2) + x (M slot 16 m16 + 4 x + i)
+          uint32_t vp[VB][4];
 #pragma unroll
-          for (int p = 0; p < VB; ++p)
-            vp[p] = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
+          for (int p = 0; p < VB; ++p) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
+            vp[p][0] = v.x; vp[p][1] = v.y; vp[p][2] = v.z; vp[p][3] = v.w;
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.empty[s]);
 #pragma unroll
-          for (int p = 0; p < VB; ++p) {
-            const uint32_t vw[4] = {vp[p].x, vp[p].y, vp[p].z, vp[p].w};
-            uint8_t *row = av + p * 2048 + (t >> 3) * 128 + (t & 7) * 16;
+          for (int m16 = 0; m16 < 8; ++m16) {
+            uint32_t o[4];
 #pragma unroll
-            for (int m16 = 0; m16 < 8; ++m16) {
-              const uint32_t word = vw[m16 >> 1];
-              const int k0 = (m16 & 1) * 4;
-              *reinterpret_cast<uint4 *>(row + m16 * C::SBO_V) =
-                  make_uint4(word & (0x01010101u << k0), word & (0x01010101u << (k0 + 1)),
-                             word & (0x01010101u << (k0 + 2)), word & (0x01010101u << (k0 + 3)));
+            for (int x = 0; x < 4; ++x) {
+              const int k = 4 * (m16 & 1) + x;
+              uint32_t c = 0;
+#pragma unroll
+              for (int p = 0; p < VB; ++p) c |= ((vp[p][m16 >> 1] >> k) & 0x01010101u) << p;
+              o[x] = c;
             }
+            *reinterpret_cast<uint4 *>(row + m16 * C::SBO_V) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
         fence_proxy_async_smem();
@@ -462,21 +559,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           const float v = fmaf(16777216.f, (float)d[4 * g + 3],
                                fmaf(65536.f, (float)d[4 * g + 2],
                                     fmaf(256.f, (float)d[4 * g + 1], (float)d[4 * g])));
-          acc[g] = fmaf(acc[g], alpha[g], v * sc);
+          acc[pb][g] = fmaf(acc[pb][g], alpha[g], v * sc);
         }
       }
     }
-    named_bar_sync(3, 256);  // the softmax group's zero-point sums are in smem
-    // unnormalised partial output: sum_t p_t (code * scale + zero)
+    named_bar_sync(3, 384);  // the softmax groups' states are in shared memory
+    // merge the two softmax states; unnormalised partial output
+    // sum_t p_t (code * scale + zero)
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float z = 0.f;
+      const float m0 = S.fin_m[0][g], m1 = S.fin_m[1][g];
+      const float mm = fmaxf(m0, m1);
+      const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mm);
+      const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mm);
+      float z0 = 0.f, z1 = 0.f, l0 = 0.f, l1 = 0.f;
 #pragma unroll
-      for (int wq = 0; wq < 4; ++wq) z += S.zsum[wq][g][q4];
-      part_row(g)[chan] = acc[g] + z;
+      for (int wq = 0; wq < 4; ++wq) {
+        z0 += S.zsum[0][wq][g][q4];
+        z1 += S.zsum[1][wq][g][q4];
+        l0 += S.lsum[0][wq][g];
+        l1 += S.lsum[1][wq][g];
+      }
+      float *pr = part_row(g);
+      pr[chan] = (acc[0][g] + z0) * f0 + (acc[1][g] + z1) * f1;
+      if (t == 0) {
+        // m (log2 units, as the SIMT path) and l of the split
+        pr[kD] = mm;
+        pr[kD + 1] = l0 * f0 + l1 * f1;
+      }
     }
   } else {
-    // ---------------- softmax group ----------------------------------------
+    // ---------------- softmax groups ---------------------------------------
+    const int grp = (warp - 10) >> 2;  // takes tiles grp, grp + 2, ...
     const int q4 = warp & 3;
     const int t = 32 * q4 + lane;  // token slot == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
@@ -491,18 +605,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       for (int gg = 0; gg < 4; ++gg) zs[g][gg] = 0.f;
     }
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
-    for (int jt = 0; qok && jt < ntile; ++jt) {
-      const int kb = jt & 1, pb = jt & 1, s = jt % C::STAGES;
+    for (int jt = grp; qok && jt < ntile; jt += 2) {
+      const int kb = grp, pb = grp, s = jt % C::STAGES, n = jt >> 1;
       if (!wait_bar(&S.full[s], (jt / C::STAGES) & 1, &S.abort_flag, status)) break;
-      if (!wait_bar(&S.s_ready[kb], (jt >> 1) & 1, &S.abort_flag, status)) break;
+      if (!wait_bar(&S.s_ready[kb], n & 1, &S.abort_flag, status)) break;
       tc_fence_after();
-      uint32_t dm[4 * G], dq[4 * G];
+      float mse[G], qjl[G];
       {
+        // two heads' limbs per load keep the register footprint small
         const uint32_t base = tbase + lane_off + C::COL_DS + kb * 2 * C::NS;
-        tmem_ld_cols<4 * G>(base, dm);
-        tmem_ld_cols<4 * G>(base + C::NS, dq);
+#pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          constexpr int W = 2 * C::L;
+          uint32_t d[W];  // an odd last head reads padding columns
+          tmem_ld_cols<W>(base + g * C::L, d);
+          tmem_wait_ld();
+          mse[g] = fmaf(Q.inv_m[g], combine_limbs<C::L>(d), Q.cm[g]);
+          if (g + 1 < G) mse[g + 1] = fmaf(Q.inv_m[g + 1], combine_limbs<C::L>(d + C::L), Q.cm[g + 1]);
+        }
+#pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          constexpr int W = 2 * C::L;
+          uint32_t d[W];  // an odd last head reads padding columns
+          tmem_ld_cols<W>(base + C::NS + g * C::L, d);
+          tmem_wait_ld();
+          qjl[g] = Q.inv_s[g] * combine_limbs<C::L>(d);
+          if (g + 1 < G) qjl[g + 1] = Q.inv_s[g + 1] * combine_limbs<C::L>(d + C::L);
+        }
       }
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.s_free[kb]);
@@ -527,44 +657,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       float lg[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const int am = (int)dm[4 * g] + 128 * (int)dm[4 * g + 1];
-        const int bm = (int)dm[4 * g + 2] + 128 * (int)dm[4 * g + 3];
-        const int as = (int)dq[4 * g] + 128 * (int)dq[4 * g + 1];
-        const int bs = (int)dq[4 * g + 2] + 128 * (int)dq[4 * g + 3];
-        const float mse = fmaf(Q.coef_m[g][1], (float)bm, fmaf(Q.coef_m[g][0], (float)am, Q.cm[g]));
-        const float qjl =
-            fmaf(Q.coef_s[g][1], (float)bs, fmaf(Q.coef_s[g][0], (float)as, -Q.csum[g]));
-        const float score = nk * fmaf(krn, qjl, mse);
+        const float score = nk * fmaf(krn, qjl[g], mse[g]);
         lg[g] = valid ? score * scale2 : -INFINITY;
       }
       // tile maxima (logits per head, value scale) over the 128 tokens
+      uint32_t(&red)[4][G + 1] = S.red[grp][n & 1];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const uint32_t u = __reduce_max_sync(0xffffffffu, float_to_ordered(lg[g]));
-        if (lane == 0) S.red[pb][q4][g] = u;
+        if (lane == 0) red[q4][g] = u;
       }
       {
         const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(msc));
-        if (lane == 0) S.red[pb][q4][G] = u;
+        if (lane == 0) red[q4][G] = u;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.red_bar[pb]);
-      if (!wait_bar(&S.red_bar[pb], (jt >> 1) & 1, &S.abort_flag, status)) break;
+      if (lane == 0) mbar_arrive(&S.red_bar[grp]);
+      if (!wait_bar(&S.red_bar[grp], n & 1, &S.abort_flag, status)) break;
       float alpha[G];
       bool changed = false;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        uint32_t u = S.red[pb][0][g];
+        uint32_t u = red[0][g];
 #pragma unroll
-        for (int wq = 1; wq < 4; ++wq) u = max(u, S.red[pb][wq][g]);
+        for (int wq = 1; wq < 4; ++wq) u = max(u, red[wq][g]);
         const float mnew = fmaxf(mrun[g], ordered_to_float(u));
         alpha[g] = exp2f(mrun[g] - mnew);
         changed |= (mnew != mrun[g]);
         mrun[g] = mnew;
       }
-      uint32_t us = S.red[pb][0][G];
+      uint32_t us = red[0][G];
 #pragma unroll
-      for (int wq = 1; wq < 4; ++wq) us = max(us, S.red[pb][wq][G]);
+      for (int wq = 1; wq < 4; ++wq) us = max(us, red[wq][G]);
       const float mscale = __uint_as_float(us);
       if (changed) {
 #pragma unroll
@@ -577,34 +701,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       // p * scale <= mscale < 2^(e+1); fixed point with values < 2^21
       const int F = mscale > 0.f ? 20 - ilog2f(mscale) : 0;
       const float fscale = mscale > 0.f ? exp2i(F) : 0.f;
-      uint32_t X[G][4];
+      float p[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float p = valid ? exp2f(lg[g] - mrun[g]) : 0.f;
-        lsum[g] += p;
+        p[g] = valid ? exp2f(lg[g] - mrun[g]) : 0.f;
+        lsum[g] += p[g];
 #pragma unroll
-        for (int gg = 0; gg < 4; ++gg) {
-          zs[g][gg] = fmaf(p, vze[gg], zs[g][gg]);
-          X[g][gg] = __float_as_uint(fmaf(p * vsc[gg], fscale, 12582912.f)) & 0x3FFFFFu;
-        }
+        for (int gg = 0; gg < 4; ++gg) zs[g][gg] = fmaf(p[g], vze[gg], zs[g][gg]);
       }
-      // P' operand of tile j: wait until the PV of tile j-2 has been read
-      if (jt >= 2 && !wait_bar(&S.pv_free[pb], ((jt - 2) >> 1) & 1, &S.abort_flag, status)) break;
-      uint8_t *bp = S.bp[pb];
+      // P' operand of tile jt: wait until the PV of tile jt-2 has been read
+      if (jt >= 2 && !wait_bar(&S.pv_free[pb], (n - 1) & 1, &S.abort_flag, status)) break;
+      // column n = group * 4G + head * 4 + byte: one u32 per (group, head),
+      // 22-bit fixed point p * scale * 2^F
+      uint8_t *row = S.bp[pb] + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
-      for (int p = 0; p < C::VOPS; ++p) {
-        // n = group * 4G + head * 4 + byte: one u32 per (group, head); the
-        // operand of bit-plane p carries the plane weight 2^p
-        uint32_t wv[4 * G];
+      for (int c = 0; c < G; ++c) {
+        uint32_t w4[4];
 #pragma unroll
-        for (int gg = 0; gg < 4; ++gg)
-#pragma unroll
-          for (int g = 0; g < G; ++g) wv[gg * G + g] = C::PACKED_V ? X[g][gg] : (X[g][gg] << p);
-        uint8_t *row = bp + p * 2048 + (t >> 3) * 128 + (t & 7) * 16;
-#pragma unroll
-        for (int c = 0; c < G; ++c)
-          *reinterpret_cast<uint4 *>(row + c * C::SBO_V) =
-              make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+        for (int x = 0; x < 4; ++x) {
+          const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
+          w4[x] = __float_as_uint(fmaf(p[g] * vsc[gg], fscale, 12582912.f)) & 0x3FFFFFu;
+        }
+        *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
       if (t == 0) {
 #pragma unroll
@@ -615,36 +733,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.p_ready[pb]);
     }
-    // reduce l and the zero-point sums over the 128 tokens
+    // l and the zero-point sums over this group's tokens, and its max
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float l = warp_sum(lsum[g]);
-      if (lane == 0) S.lsum[q4][g] = l;
+      if (lane == 0) S.lsum[grp][q4][g] = l;
 #pragma unroll
       for (int gg = 0; gg < 4; ++gg) {
         const float z = warp_sum(zs[g][gg]);
-        if (lane == 0) S.zsum[q4][g][gg] = z;
+        if (lane == 0) S.zsum[grp][q4][g][gg] = z;
       }
+      if (t == 0) S.fin_m[grp][g] = mrun[g];
     }
-    named_bar_sync(3, 256);  // publish to the value group
-    if (t == 0) {
-      // m (log2 units, as the SIMT path) and l of the split
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float l = 0.f;
-#pragma unroll
-        for (int wq = 0; wq < 4; ++wq) l += S.lsum[wq][g];
-        part_row(g)[kD] = mrun[g];
-        part_row(g)[kD + 1] = l;
-      }
-    }
+    named_bar_sync(3, 384);  // publish to the value group
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tbase, C::TMEM_COLS);
+    tmem_dealloc(tbase, kTmemCols);
     tmem_relinquish();
   }
 }
@@ -652,19 +760,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 
 // ---------------------------------------------------------------------------
 // Query blocks: for every (sequence, KV head) the score MMA's B operand
-// (B_q in its shared-memory byte layout) and the score constants, built once
-// per decode call.  A persistent CTA keeps Pi and S in shared memory (rows
-// padded to 129 floats) and rotates the G query heads of each unit:
-// q~ = Pi q, s^ = S q (fp32), then writes
-//   B_q[kappa][head * 4 + limb] = limb of round(w_p q~_j 2^(F - k)) or of
-//   round(2 s^_j 2^(F - k)), kappa <-> (plane p, word wd, mask k, byte i),
-//   j = 32 wd + 8 i + k, four signed base-128 limbs,
-// with F per head chosen so every operand stays below 2^26.
+// (e2m1, in its shared-memory byte layout) and the score constants, built
+// once per decode call.  A persistent CTA keeps Pi and S in shared memory
+// (rows padded to 129 floats) and rotates the G query heads of each unit:
+// q~ = Pi q, s^ = S q (fp32).  Plane P < n_mse holds a_S q~ for the P-th
+// active code-bit subset S (Walsh coefficient a_S of the codebook), the last
+// plane holds s^; each value is rounded to X = round(x 2^F), F per head so
+// |X| <= (9^L - 1) / 2, and written as L balanced base-9 digits.
+// Coordinate j sits at K-chunk j / 32, word j % 4, nibble (j % 32) / 4, the
+// same places the key group's spin words put it.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1_digit(int d) {
+  const int m = d < 0 ? -d : d;
+  const uint32_t code = m == 0 ? 0u : (m == 1 ? 2u : (m == 2 ? 4u : (m == 3 ? 5u : 6u)));
+  return code | (d < 0 ? 8u : 0u);
+}
+
 template <int MB, int VB, int G>
 __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ DecodeArgs a) {
   using C = Cfg<MB, VB, G>;
+  constexpr int L = C::L;
   constexpr int kPadQ = kD + 1;
+  constexpr int NC = 1 << MB;
   extern __shared__ __align__(16) float qsm[];
   float *mat = qsm;                         // [256][129]: rows of Pi then S
   float *qv = mat + 2 * kD * kPadQ;         // [G][128]
@@ -677,23 +794,42 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     const int r = i / kD, c = i % kD;
     mat[r * kPadQ + c] = (r < kD) ? a.pi[i] : a.s[i - kD * kD];
   }
-  float cent[8];
+  for (int i = tid; i < C::QBLOCK / 4; i += 256) reinterpret_cast<uint32_t *>(blk)[i] = 0u;
+  // Walsh coefficients of the codebook, idx paired with its complement so
+  // that a symmetric codebook gives exact zeros for the even subsets
+  float cent[NC];
 #pragma unroll
-  for (int i = 0; i < (1 << MB); ++i) cent[i] = a.centroids[i];
-  float w[C::NP];
-  if (MB == 1) {
-    w[0] = cent[1] - cent[0];
-  } else if (MB == 2) {
-    w[0] = cent[1] - cent[0];
-    w[1] = cent[2] - cent[0];
-    w[2] = cent[3] - cent[2] - cent[1] + cent[0];
-  } else {
+  for (int i = 0; i < NC; ++i) cent[i] = a.centroids[i];
+  float wal[NC];
 #pragma unroll
-    for (int l = 0; l < C::NP; ++l) w[l] = cent[l + 1] - cent[l];
+  for (int S = 0; S < NC; ++S) {
+    float acc = 0.f;
+    const bool even = (__popc(S) & 1) == 0;
+#pragma unroll
+    for (int idx = 0; idx < NC / 2; ++idx) {
+      const float pr = (__popc(~idx & S) & 1) ? -1.f : 1.f;  // prod of spins over S
+      const float pair = even ? cent[idx] + cent[NC - 1 - idx] : cent[idx] - cent[NC - 1 - idx];
+      acc = fmaf(pr, pair, acc);
+    }
+    wal[S] = acc / (float)NC;
   }
+  int nm = 0, subs[7];
+  float wts[7];
   float wmax = 0.f;
 #pragma unroll
-  for (int p = 0; p < C::NP; ++p) wmax = fmaxf(wmax, fabsf(w[p]));
+  for (int S = 1; S < NC; ++S) {
+    if (wal[S] != 0.f) {
+      subs[nm] = S;
+      wts[nm] = wal[S];
+      ++nm;
+      wmax = fmaxf(wmax, fabsf(wal[S]));
+    }
+  }
+  if (nm == 0) {  // degenerate codebook: one all-zero plane
+    subs[0] = 1;
+    wts[0] = 0.f;
+    nm = 1;
+  }
   QConst *qc = reinterpret_cast<QConst *>(blk + C::BQ_BYTES);
   __syncthreads();
 
@@ -717,67 +853,70 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
       for (int g = 0; g < G; ++g) rot[g * 2 * kD + o] = acc[g];
     }
     __syncthreads();
-    // per head: sum q~, max |q~|, sum s^, max |s^|
+    // per head: sum q~, max |q~|, max |s^|
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int j = tid & (kD - 1);
       const float x = rot[g * 2 * kD + (tid < kD ? 0 : kD) + j];
       const float sm = warp_sum(x), mx = warp_max(fabsf(x));
       if (lane == 0) {
-        red[(warp * G + g) * 4 + (tid < kD ? 0 : 2)] = sm;
-        red[(warp * G + g) * 4 + (tid < kD ? 1 : 3)] = mx;
+        red[(warp * G + g) * 4 + 0] = sm;
+        red[(warp * G + g) * 4 + 1] = mx;
       }
     }
     __syncthreads();
+    constexpr int emax = xbits_for(L);
     int fm[G], fs[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float sq = 0.f, mq = 0.f, ss = 0.f, ms = 0.f;
+      float sq = 0.f, mq = 0.f, ms = 0.f;
       for (int wq = 0; wq < 4; ++wq) {        // warps 0-3 hold q~, 4-7 hold s^
         sq += red[(wq * G + g) * 4 + 0];
         mq = fmaxf(mq, red[(wq * G + g) * 4 + 1]);
-        ss += red[((wq + 4) * G + g) * 4 + 2];
-        ms = fmaxf(ms, red[((wq + 4) * G + g) * 4 + 3]);
+        ms = fmaxf(ms, red[((wq + 4) * G + g) * 4 + 1]);
       }
-      const float bm = wmax * mq, bs = 2.f * ms;
-      fm[g] = bm > 0.f ? 25 - ilogbf(bm) : 0;
-      fs[g] = bs > 0.f ? 25 - ilogbf(bs) : 0;
+      const float bm = wmax * mq;
+      fm[g] = bm > 0.f ? emax - 1 - ilogbf(bm) : 0;
+      fs[g] = ms > 0.f ? emax - 1 - ilogbf(ms) : 0;
       if (tid == 0) {
-        qc->cm[g] = cent[0] * sq;
-        qc->csum[g] = ss;
-        // limbs combine as (D0 + 128 D1) 2^-F + (D2 + 128 D3) 2^(14-F)
-        qc->coef_m[g][0] = ldexpf(1.f, -fm[g]);
-        qc->coef_m[g][1] = ldexpf(1.f, 14 - fm[g]);
-        qc->coef_s[g][0] = ldexpf(1.f, -fs[g]);
-        qc->coef_s[g][1] = ldexpf(1.f, 14 - fs[g]);
+        qc->cm[g] = wal[0] * sq;
+        qc->inv_m[g] = ldexpf(1.f, -fm[g]);
+        qc->inv_s[g] = ldexpf(1.f, -fs[g]);
       }
     }
-    if (tid == 0) qc->skip_product_plane = (MB == 2 && w[2] == 0.f) ? 1 : 0;
-    for (int kappa = tid; kappa < (C::NP + 1) * 128; kappa += 256) {
-      const int p = kappa >> 7, rem = kappa & 127;
-      const int col = rem >> 2, bi = rem & 3;
-      const int wd = col >> 3, k = col & 7;
-      const int coord = 32 * wd + 8 * bi + k;
-      uint8_t *dst0 = blk + (kappa >> 4) * C::LBO_Q + (kappa & 15);
-      for (int n = 4 * G; n < C::NS; ++n) dst0[(n >> 3) * 128 + (n & 7) * 16] = 0;
+    if (tid == 0) {
+      qc->n_mse = nm;
+      for (int p = 0; p < 7; ++p) qc->subset[p] = p < nm ? subs[p] : 0;
+    }
+    // one item = one byte position (plane, chunk wd, word k, byte m): the
+    // coordinates 32 wd + 8 m + k (low nibble) and that + 4 (high nibble)
+    for (int item = tid; item < (nm + 1) * 64; item += 256) {
+      const int P = item >> 6, wd = (item >> 4) & 3, k = (item >> 2) & 3, m = item & 3;
+      const int jlo = 32 * wd + 8 * m + k, jhi = jlo + 4;
+      uint8_t *dst0 = blk + P * C::BQ_PLANE + wd * (C::NS * 16) + 4 * k + m;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float x;
+        float xl, xh;
         int F;
-        if (p < C::NP) {
-          x = w[p] * rot[g * 2 * kD + coord];
+        if (P < nm) {
+          xl = wts[P] * rot[g * 2 * kD + jlo];
+          xh = wts[P] * rot[g * 2 * kD + jhi];
           F = fm[g];
         } else {
-          x = 2.f * rot[g * 2 * kD + kD + coord];
+          xl = rot[g * 2 * kD + kD + jlo];
+          xh = rot[g * 2 * kD + kD + jhi];
           F = fs[g];
         }
-        int X = __float2int_rn(ldexpf(x, F - k));
+        int Xl = __float2int_rn(ldexpf(xl, F)), Xh = __float2int_rn(ldexpf(xh, F));
 #pragma unroll
-        for (int l = 0; l < 4; ++l) {
-          const int dgt = (l < 3) ? (((X + 64) & 127) - 64) : X;
-          X = (X - dgt) >> 7;
-          const int n = g * 4 + l;
-          dst0[(n >> 3) * 128 + (n & 7) * 16] = (uint8_t)(int8_t)dgt;
+        for (int l = 0; l < L; ++l) {
+          int dl = Xl % 9, dh = Xh % 9;
+          dl = dl > 4 ? dl - 9 : (dl < -4 ? dl + 9 : dl);
+          dh = dh > 4 ? dh - 9 : (dh < -4 ? dh + 9 : dh);
+          Xl = (Xl - dl) / 9;
+          Xh = (Xh - dh) / 9;
+          const int ncol = g * L + l;
+          dst0[(ncol >> 3) * 128 + (ncol & 7) * 16] = (uint8_t)(e2m1_digit(dl) | (e2m1_digit(dh) << 4));
         }
       }
     }
@@ -819,12 +958,7 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
-size_t decode_tc_qblock_bytes(int key_bits, int G) {
-  const int mb = key_bits - 1;
-  const int np = mb == 1 ? 1 : (mb == 2 ? 3 : 7);
-  const int ns = ((4 * G + 15) / 16) * 16;
-  return (size_t)(np + 1) * 128 * ns + kQConstBytes;
-}
+size_t decode_tc_qblock_bytes(int key_bits, int G) { return qblock_bytes_for(key_bits - 1, G); }
 
 bool decode_tc_supported(int key_bits, int value_bits, int G) {
   const int mb = key_bits - 1;

@@ -312,3 +312,49 @@ def test_decode_bit_widths(kb, vb):
         kes, ves = encs[b]
         ref = pu.oracle_decode(olayer, q[b].float().numpy(), kes, ves, lengths[b])
         assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (kb, vb, b)
+
+
+@pytest.mark.parametrize("h_kv,h_q", [(2, 2), (2, 4), (2, 8), (1, 8)])
+def test_decode_ragged_packed_values_gqa(h_kv, h_q):
+    """2-bit packed values (the tensor-core kernel) at GQA 1, 2, 4 and 8, with
+    lengths 1, a tile minus one, a tile plus one, a partial last tile and an
+    empty sequence."""
+    import dataclasses
+    lengths = (1, 127, 129, 300, 0)
+    wl = dataclasses.replace(workloads.llama8b(), batch=5, h_kv=h_kv, h_q=h_q, lengths=lengths,
+                             capacity=384, name=f"ragged_packed_{h_kv}_{h_q}")
+    glayer, olayer, spec = _setup(wl)
+    buf, encs = _oracle_cache(wl, olayer, spec, lengths)
+    q = workloads.queries(wl, 0)
+    got = _run_decode(glayer, wl, buf, list(lengths), q)
+    for b in range(wl.batch):
+        if lengths[b] == 0:
+            assert np.all(got[b] == 0.0)
+            continue
+        kes, ves = encs[b]
+        ref = pu.oracle_decode(olayer, q[b].float().numpy(), kes, ves, lengths[b])
+        assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (h_kv, h_q, b)
+
+
+@pytest.mark.parametrize("kb", [2, 3, 4])
+def test_decode_asymmetric_codebook(kb):
+    """A caller-supplied codebook that is not symmetric about zero (shifted and
+    stretched Lloyd-Max levels): decode must use every level as given, so the
+    constant and even-order terms of its expansion in the code bits matter."""
+    import dataclasses
+    lengths = (700, 256)
+    wl = dataclasses.replace(workloads.llama8b(), batch=2, key_bits=kb, lengths=lengths,
+                             capacity=768, name=f"asym{kb}")
+    glayer, olayer, spec = _setup(wl)
+    buf, encs = _oracle_cache(wl, olayer, spec, lengths)
+    n = len(olayer.cent)
+    cent = np.asarray(olayer.cent, np.float64) * (1.0 + 0.1 * np.arange(n) / n) + 0.02
+    cent = np.asarray(cent.astype(np.float32), np.float64)
+    olayer.cent = cent
+    glayer.centroids.copy_(torch.tensor(cent, dtype=torch.float32))
+    q = workloads.queries(wl, 0)
+    got = _run_decode(glayer, wl, buf, list(lengths), q)
+    for b in range(wl.batch):
+        kes, ves = encs[b]
+        ref = pu.oracle_decode(olayer, q[b].float().numpy(), kes, ves, lengths[b])
+        assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (kb, b)
