@@ -68,24 +68,42 @@ def encode_keys(keys: np.ndarray, pi: np.ndarray, s: np.ndarray,
     """
     x = np.asarray(keys, dtype=np.float64)
     pi = np.asarray(pi, dtype=np.float64)
-    s = np.asarray(s, dtype=np.float64)
-    cent = np.asarray(centroids, dtype=np.float64)
     n, d = x.shape
     nk = np.sqrt(np.sum(x * x, axis=1))
     zero = nk == 0.0
     u = np.where(zero[:, None], 0.0, x / np.where(zero, 1.0, nk)[:, None])
     y = u @ pi.T                         # y = Pi u, row by row
     idx = bucketize(y, boundaries)
-    c = cent[idx]
-    r = u - c @ pi                       # r = u - Pi^T c, row by row
-    rn = np.sqrt(np.sum(r * r, axis=1))
-    z = r @ s.T                          # z = S r, row by row
-    sign = (z >= 0.0).astype(np.uint8)
+    res = residual_sketch(u, idx, pi, s, centroids)
     idx[zero] = 0
+    sign, rn = res["sign"], res["rn"]
     sign[zero] = 0
     rn = np.where(zero, 0.0, rn)
     return {"idx": idx, "sign": sign, "nk16": fp16(nk), "rn16": fp16(rn),
-            "y": y, "z": z, "nk": nk, "rn": rn}
+            "y": y, "z": res["z"], "nk": nk, "rn": rn}
+
+
+def unit_keys(keys: np.ndarray) -> np.ndarray:
+    """Step 1 alone: u = k / ||k|| (0 for a zero key), float64."""
+    x = np.asarray(keys, dtype=np.float64)
+    nk = np.sqrt(np.sum(x * x, axis=1))
+    return np.where((nk == 0.0)[:, None], 0.0, x / np.where(nk == 0.0, 1.0, nk)[:, None])
+
+
+def residual_sketch(u: np.ndarray, idx: np.ndarray, pi: np.ndarray, s: np.ndarray,
+                    centroids: np.ndarray) -> dict:
+    """Steps 4 and 5 for given cells: r = u - Pi^T c[idx], rn = ||r||,
+    z = S r, sign = [z >= 0].  The residual and its sketch are functions of
+    the chosen cells, so a coordinate that lies on a decision boundary (where
+    either cell is a correct bucketization) determines them through the cell
+    actually chosen."""
+    pi = np.asarray(pi, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    c = np.asarray(centroids, dtype=np.float64)[idx]
+    r = np.asarray(u, dtype=np.float64) - c @ pi     # r = u - Pi^T c, row by row
+    z = r @ s.T                                      # z = S r, row by row
+    return {"r": r, "rn": np.sqrt(np.sum(r * r, axis=1)), "z": z,
+            "sign": (z >= 0.0).astype(np.uint8)}
 
 
 def encode_values(values: np.ndarray, value_bits: int, group: int) -> dict:

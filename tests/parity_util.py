@@ -53,10 +53,13 @@ def to_np(t: torch.Tensor) -> np.ndarray:
 
 
 def compare_records(spec: layout.CacheSpec, buf: np.ndarray, b: int, h: int, pos0: int,
-                    ke: dict, ve: dict, stats: dict | None = None) -> dict:
+                    ke: dict, ve: dict, stats: dict | None = None, layer=None,
+                    keys: np.ndarray | None = None) -> dict:
     """Compare the library's records of tokens [pos0, pos0+n) of (b, h) with
     the oracle's encoding (ke, ve of n vectors).  Raises AssertionError on a
-    mismatch outside the bands; returns accumulated band statistics."""
+    mismatch outside the bands; returns accumulated band statistics.
+    layer / keys (the oracle layer and the n key vectors) let a vector whose
+    banded code took the other cell be checked against that cell's residual."""
     n = len(ke["nk16"])
     got = spec.read(buf, b, h, pos0, n)
     stats = stats if stats is not None else {"coords": 0, "code_band": 0, "sign_band": 0,
@@ -70,10 +73,25 @@ def compare_records(spec: layout.CacheSpec, buf: np.ndarray, b: int, h: int, pos
     near[zero] = False
     bad = (got["idx"] != ke["idx"]) & ~near
     assert not bad.any(), f"code mismatch outside band at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
-    snear = np.abs(ke["z"]) < BAND
+    if layer is not None:
+        layer_pi, layer_s, layer_cent = layer.pi, layer.s, layer.cent
+    elif (got["idx"] != ke["idx"]).any():
+        raise AssertionError("banded code mismatch: pass layer= and keys= to check its residual")
+    # a vector whose banded code went to the other cell has the residual,
+    # signs and ||r|| of the cell the library chose: take those from the
+    # oracle's steps 4-5 on the library's codes
+    z_ref, sign_ref, rn16_ref = ke["z"], ke["sign"], ke["rn16"]
+    alt = np.flatnonzero((got["idx"] != ke["idx"]).any(axis=1) & ~zero)
+    if alt.size:
+        res = quant.residual_sketch(quant.unit_keys(keys[alt]), got["idx"][alt], layer_pi, layer_s,
+                                    layer_cent)
+        z_ref, sign_ref, rn16_ref = z_ref.copy(), sign_ref.copy(), rn16_ref.copy()
+        z_ref[alt], sign_ref[alt], rn16_ref[alt] = res["z"], res["sign"], quant.fp16(res["rn"])
+    snear = np.abs(z_ref) < BAND
     snear[zero] = False
-    bad = (got["sign"] != ke["sign"]) & ~snear
+    bad = (got["sign"] != sign_ref) & ~snear
     assert not bad.any(), f"sign mismatch outside band at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
+    stats["alt_cell_vectors"] = stats.get("alt_cell_vectors", 0) + int(alt.size)
     t = ve["t"]
     vnear = np.abs(t - np.floor(t) - 0.5) < BAND
     # value codes are decided by the same float32 steps on both sides: exact
@@ -83,7 +101,7 @@ def compare_records(spec: layout.CacheSpec, buf: np.ndarray, b: int, h: int, pos
     assert np.array_equal(got["scale16"], ve["scale16"]), "value scale mismatch"
     assert np.array_equal(got["zero16"], ve["zero16"]), "value zero mismatch"
     for key in ("nk16", "rn16"):
-        ref = ke[key]
+        ref = ke[key] if key == "nk16" else rn16_ref
         rel = np.abs(got[key] - ref) / np.maximum(np.abs(ref), 1e-30)
         rel[(ref == 0) & (got[key] == 0)] = 0.0
         assert rel.max(initial=0.0) <= REL_TOL, f"{key} rel err {rel.max()}"
