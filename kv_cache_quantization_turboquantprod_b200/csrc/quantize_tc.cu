@@ -1,0 +1,558 @@
+// quantize_append on the 5th-generation tensor cores (tcgen05 kind::f16):
+// the TurboQuant-prod key encoding of "TurboQuant" explainer (troisinh.com,
+// "Ý tưởng cốt lõi") and "turboquant/audit_claims.py" (AUDIT 1 / AUDIT 5),
+// with the three d x d products of every key vector as tensor-core GEMMs
+// over 128-vector tiles and everything else fused in their epilogues:
+//   GEMM1  Y = K Pi^T            y = Y / ||k||, bucketize -> codes, c = c[idx]
+//   GEMM2  P = C Pi              r = u - P (= u - Pi^T c), ||r||
+//   GEMM3  Z = R S^T             signs = [z >= 0]
+// Values are group-quantized (per 32 channels, fp16 scale/zero) by the
+// loader warps on the way in.
+//
+// Precision.  A bf16 key is exact in fp16 once scaled per vector by 2^s
+// (largest |k| 2^s in [2^14, 2^15)); Pi, S, the centroids and the residual
+// are split into fp16 hi + lo parts (scaled so no part is subnormal where it
+// matters), and each product takes the three significant hi/lo terms with
+// f32 accumulation: about 22 bits per operand, the error of an fp32 mat-vec.
+//
+// Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
+// record section a tile writes is one contiguous run of the cache.
+//
+// Warp roles (416 threads):
+//   warp 0        MMA issuer (one elected lane), polling both epilogue groups
+//   warps 1-4     loader: K rows -> scaled fp16 A operand + norms in shared
+//                 memory; V rows -> codes, scales, zeros straight to the cache
+//   warps 5-8     epilogue group 0 (even tiles)   | thread = tile row = TMEM
+//   warps 9-12    epilogue group 1 (odd tiles)    | lane; 256 TMEM columns each
+// Every mbarrier wait is bounded (2 s); on timeout the CTA raises its abort
+// flag, stops, lets its own MMAs finish and frees TMEM.
+#include <math.h>
+
+#include "sm100.cuh"
+#include "tq_common.cuh"
+#include "tq_kernels.h"
+
+namespace tq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kQtThreads = 416;
+constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
+constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
+constexpr float kSScale = 256.f;       // S parts x 2^8
+constexpr float kCScale = 65536.f;     // centroid parts x 2^16
+constexpr float kRScale = 8192.f;      // residual parts x 2^13
+
+// byte offset of element (row, col) of a 128 x 128 fp16 matrix in the
+// canonical no-swizzle layout: 8 x 8 blocks, block (row / 8, col / 8) at
+// (col / 8) * 2048 + (row / 8) * 128.  Read K-major (K = col) with
+// LBO 2048 / SBO 128, or MN-major (K = row, N = col) with LBO 128 / SBO 2048.
+__host__ __device__ constexpr int blk_off(int row, int col) {
+  return (col >> 3) * 2048 + (row >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2;
+}
+
+struct QtSmem {
+  alignas(1024) uint8_t pi[2][kMat16];  // Pi x 2^10: hi, lo
+  alignas(1024) uint8_t s[2][kMat16];   // S x 2^8: hi, lo
+  alignas(1024) uint8_t a1[2][kMat16];  // K rows x 2^s (fp16), one per epilogue group
+  float nk[2][128];
+  int sh[2][128];
+  float cent[8];
+  float bnd[8];
+  uint64_t a1_full[2], a1_free[2], d1_full[2], a2_full[2], d2_full[2], a3_full[2], d3_full[2],
+      d_free[2];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+struct TileInfo {
+  int b, h, t0, nrow;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const AppendArgs &a, int gt) {
+  // batch b owns tiles [tstart[b], tstart[b + 1])
+  int lo = 0, hi = a.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.tstart[mid] <= gt) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.b = lo;
+  const int rem = gt - a.tstart[lo];
+  const int ntb = (a.nnew[lo] + 127) >> 7;
+  ti.h = rem / ntb;
+  const int tb = rem - ti.h * ntb;
+  ti.t0 = tb * 128;
+  ti.nrow = min(128, a.nnew[lo] - ti.t0);
+  return ti;
+}
+
+__device__ __forceinline__ bool qwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > 2000000000ull) break;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo_elem, float hi_elem) {
+  const __half2 h = __floats2half2_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// hi + lo fp16 parts of x (already scaled)
+__device__ __forceinline__ void split16(float x, float &hi, float &lo) {
+  hi = __half2float(__float2half_rn(x));
+  lo = x - hi;
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid_constant__ AppendArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  QtSmem &S = *reinterpret_cast<QtSmem *>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  constexpr int ncent = 1 << MB;
+  const int nlocal = a.total_tiles > (int)blockIdx.x
+                         ? (a.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                         : 0;
+
+  // ---- setup: split Pi and S into fp16 parts, barriers, TMEM -------------
+  for (int e = tid; e < 128 * 128; e += kQtThreads) {
+    const int i = e >> 7, j = e & 127;
+    float hi, lo;
+    split16(a.pi[e] * kPiScale, hi, lo);
+    *reinterpret_cast<__half *>(S.pi[0] + blk_off(i, j)) = __float2half_rn(hi);
+    *reinterpret_cast<__half *>(S.pi[1] + blk_off(i, j)) = __float2half_rn(lo);
+    split16(a.s[e] * kSScale, hi, lo);
+    *reinterpret_cast<__half *>(S.s[0] + blk_off(i, j)) = __float2half_rn(hi);
+    *reinterpret_cast<__half *>(S.s[1] + blk_off(i, j)) = __float2half_rn(lo);
+  }
+  if (tid < ncent) S.cent[tid] = a.centroids[tid];
+  if (tid < ncent - 1) S.bnd[tid] = a.boundaries[tid];
+  if (tid == 0) {
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&S.a1_full[g], 4);
+      mbar_init(&S.a1_free[g], 4);
+      mbar_init(&S.d1_full[g], 1);
+      mbar_init(&S.a2_full[g], 4);
+      mbar_init(&S.d2_full[g], 1);
+      mbar_init(&S.a3_full[g], 4);
+      mbar_init(&S.d3_full[g], 1);
+      mbar_init(&S.d_free[g], 4);
+    }
+    S.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&S.tmem_base, 512);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = S.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- MMA issuer ------------------------------------------
+    const bool leader = elect_one();
+    const uint32_t id1 = idesc_f16(128, 128, false, false);
+    const uint32_t id2 = idesc_f16(128, 128, false, true);
+    const uint64_t dpk[2] = {smem_desc(S.pi[0], 2048, 128), smem_desc(S.pi[1], 2048, 128)};
+    const uint64_t dpm[2] = {smem_desc(S.pi[0], 128, 2048), smem_desc(S.pi[1], 128, 2048)};
+    const uint64_t dsk[2] = {smem_desc(S.s[0], 2048, 128), smem_desc(S.s[1], 2048, 128)};
+    const uint64_t da1[2] = {smem_desc(S.a1[0], 2048, 128), smem_desc(S.a1[1], 2048, 128)};
+    int tile[2] = {0, 1}, stage[2] = {0, 0};
+    uint64_t *last_bar[2] = {nullptr, nullptr};
+    uint32_t last_ph[2] = {0u, 0u};
+    uint32_t idle = 0;
+    uint64_t t_idle = 0;
+    while (tile[0] < nlocal || tile[1] < nlocal) {
+      bool progress = false;
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int i = tile[g];
+        if (i >= nlocal) continue;
+        const uint32_t ph = (i >> 1) & 1;
+        const uint32_t d = tbase + g * 256, aop = d + 128;
+        bool ready;
+        if (stage[g] == 0)
+          ready = mbar_test(&S.a1_full[g], ph) && (i < 2 || mbar_test(&S.d_free[g], ph ^ 1));
+        else if (stage[g] == 1)
+          ready = mbar_test(&S.a2_full[g], ph);
+        else
+          ready = mbar_test(&S.a3_full[g], ph);
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (!ready) continue;
+        tc_fence_after();
+        if (stage[g] == 0) {  // Y = K Pi^T: (K)(Pi_hi + Pi_lo)
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              if (leader)
+                mma_f16_ss(d, da1[g] + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4),
+                           id1, (pr | ks) ? 1u : 0u);
+          if (leader) mma_commit(&S.d1_full[g]);
+          last_bar[g] = &S.d1_full[g];
+        } else if (stage[g] == 1) {  // P = C Pi: C_hi Pi_hi + C_hi Pi_lo + C_lo Pi_hi
+#pragma unroll
+          for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              if (leader)
+                mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks, dpm[pr == 1 ? 1 : 0] + (uint64_t)(16 * ks), id2,
+                           (pr | ks) ? 1u : 0u);
+          if (leader) mma_commit(&S.d2_full[g]);
+          last_bar[g] = &S.d2_full[g];
+        } else {  // Z = R S^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
+#pragma unroll
+          for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              if (leader)
+                mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks,
+                           dsk[pr == 1 ? 1 : 0] + (uint64_t)((ks * 4096) >> 4), id1, (pr | ks) ? 1u : 0u);
+          if (leader) mma_commit(&S.d3_full[g]);
+          last_bar[g] = &S.d3_full[g];
+        }
+        last_ph[g] = ph;
+        __syncwarp();
+        if (++stage[g] == 3) {
+          stage[g] = 0;
+          tile[g] += 2;
+        }
+        progress = true;
+      }
+      if (progress) {
+        idle = 0;
+        t_idle = 0;
+      } else if ((++idle & 15u) != 0) {
+        __nanosleep(64);
+      } else {
+        if (S.abort_flag) break;
+        const uint64_t now = globaltimer_ns();
+        if (t_idle == 0) {
+          t_idle = now;
+        } else if (now - t_idle > 2000000000ull) {
+          S.abort_flag = 1;
+          break;
+        }
+      }
+    }
+    // never leave with an MMA in flight: the last commit of each group
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+      if (last_bar[g]) mbar_wait(last_bar[g], last_ph[g]);
+  } else if (warp <= 4) {
+    // ---------------- loader -----------------------------------------------
+    // A warp takes 8 rows at a time (one 8-row group of the operand): lane
+    // (row rr = lane / 4, channel quarter q = lane % 4) holds channels
+    // 32q .. 32q + 31 -- one value group.  Both rows are fetched before
+    // either is used.
+    const int w = warp - 1, rr = lane >> 2, q = lane & 3;
+    const float vlevels = (float)((1 << a.value_bits) - 1);
+    for (int i = 0; i < nlocal; ++i) {
+      const int g = i & 1;
+      if (i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag)) break;
+      const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
+      uint8_t *a1 = S.a1[g];
+#pragma unroll 1
+      for (int pass = 0; pass < 4; ++pass) {
+        const int r = 32 * pass + 8 * w + rr;
+        const bool valid = r < ti.nrow;
+        const int t = ti.t0 + r;
+        const size_t base = valid ? ((((size_t)ti.b * a.T + t) * a.h_kv + ti.h) * kD + 32 * q) : 0;
+        uint4 kr[4], vr[4];
+        {
+          const uint4 *ks = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + base);
+          const uint4 *vs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v) + base);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            kr[c] = valid ? ks[c] : make_uint4(0u, 0u, 0u, 0u);
+            vr[c] = valid ? vs[c] : make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        // ---- key: norm, per-vector scale, fp16 operand ----
+        float ss = 0.f, mx = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[c]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(p2[e]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float nk = sqrtf(ss);
+        const int sh = mx > 0.f ? min(14 - ilogbf(mx), 127) : 0;
+        const float f2 = __uint_as_float((uint32_t)(sh + 127) << 23);  // 2^sh
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[c]);
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(p2[e]);
+            o[e] = pack_h2(f.x * f2, f.y * f2);
+          }
+          *reinterpret_cast<uint4 *>(a1 + blk_off(r, 32 * q + 8 * c)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (q == 0) {
+          S.nk[g][r] = nk;
+          S.sh[g][r] = sh;
+        }
+        // ---- values: this lane's 32 channels are one group ----
+        if (valid) {
+          float mn = INFINITY, mxv = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[c]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(p2[e]);
+              mn = fminf(mn, fminf(f.x, f.y));
+              mxv = fmaxf(mxv, fmaxf(f.x, f.y));
+            }
+          }
+          const __half zero16 = __float2half_rn(mn);
+          const __half scale16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxv, mn), vlevels));
+          const float z32 = __half2float(zero16), sc32 = __half2float(scale16);
+          const float rsc = sc32 != 0.f ? 1.f / sc32 : 0.f;
+          const int pos = a.lens[ti.b] + t;
+          uint8_t *tp = tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile);
+          const int slot = pos % kTile;
+          uint32_t w2[2] = {0u, 0u}, wp[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[c]);
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2) {
+              const int e = 8 * c + e2;
+              const float2 f = __bfloat1622float2(p2[e2 >> 1]);
+              const float x = (e2 & 1) ? f.y : f.x;
+              // the code is rint((v - zero) / scale) with an exactly rounded
+              // quotient; the reciprocal product is within 2 ulp of it, so it
+              // decides the code unless it sits next to a half-integer
+              const float num = __fsub_rn(x, z32);
+              float tq = num * rsc;
+              const float fr = tq - floorf(tq);
+              if (fabsf(fr - 0.5f) < 1e-5f) tq = __fdiv_rn(num, sc32);
+              tq = fminf(fmaxf(rintf(tq), 0.f), vlevels);
+              const uint32_t code = sc32 != 0.f ? (uint32_t)tq : 0u;
+              w2[e >> 4] |= (code & 3u) << (2 * (e & 15));
+#pragma unroll
+              for (int p = 0; p < 4; ++p) wp[p] |= ((code >> p) & 1u) << e;
+            }
+          }
+          if (L.vb == 2) {
+            *reinterpret_cast<uint2 *>(tp + L.vplanes + slot * kPackedRowBytes + 8 * q) = make_uint2(w2[0], w2[1]);
+          } else {
+            for (int p = 0; p < L.vb; ++p)
+              *reinterpret_cast<uint32_t *>(tp + L.vplanes + p * kPlaneBytes + slot * kRowBytes + 4 * q) = wp[p];
+          }
+          *reinterpret_cast<__half2 *>(tp + L.vsz + (slot * kGroups + q) * 4) = __halves2half2(scale16, zero16);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a1_full[g]);
+    }
+  } else {
+    // ---------------- epilogue groups --------------------------------------
+    const int g = (warp - 5) >> 2;
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;  // tile row == TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+    const uint32_t dcol = tbase + lane_off + g * 256, acol = dcol + 128;
+    const uint8_t *a1 = S.a1[g];
+    constexpr int NB = (1 << MB) - 1;
+    float bnd[NB], cent[NB + 1];
+#pragma unroll
+    for (int x = 0; x < NB; ++x) bnd[x] = S.bnd[x];
+#pragma unroll
+    for (int x = 0; x <= NB; ++x) cent[x] = S.cent[x] * kCScale;
+    for (int i = g; i < nlocal; i += 2) {
+      const uint32_t ph = (i >> 1) & 1;
+      const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
+      const bool valid = r < ti.nrow;
+      const int pos = a.lens[ti.b] + ti.t0 + r;
+      uint8_t *tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
+      const int slot = pos % kTile;
+      if (!qwait(&S.d1_full[g], ph, &S.abort_flag)) break;
+      tc_fence_after();
+      const float nk = S.nk[g][r];
+      const int sh = S.sh[g][r];
+      const bool zero = !(nk > 0.f);
+      const float rnk = zero ? 0.f : 1.f / nk;
+      const float inv1 = ldexpf(rnk, -(sh + 10));  // y = Y 2^-(s+10) / ||k||
+      const float inv2 = ldexpf(rnk, -sh);         // u = K 2^-s / ||k||
+      // ---- E1: y = Pi u, codes, centroid operand C (16 columns at a time) ----
+      uint32_t planes[3][4];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t d[16];
+        tmem_ld16(dcol + 16 * c, d);
+        tmem_wait_ld();
+        uint32_t hw[8], lw[8];
+        uint32_t pw[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float cv[2];
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const float y = __uint_as_float(d[e + x]) * inv1;
+            int idx = 0;
+#pragma unroll
+            for (int qq = 0; qq < NB; ++qq) idx += (bnd[qq] < y) ? 1 : 0;
+            if (zero) idx = 0;
+#pragma unroll
+            for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
+            float cc = cent[0];
+#pragma unroll
+            for (int qq = 1; qq <= NB; ++qq) cc = (idx == qq) ? cent[qq] : cc;
+            cv[x] = zero ? 0.f : cc;
+          }
+          float h0, l0, h1, l1;
+          split16(cv[0], h0, l0);
+          split16(cv[1], h1, l1);
+          hw[e >> 1] = pack_h2(h0, h1);
+          lw[e >> 1] = pack_h2(l0, l1);
+        }
+        tmem_st8(acol + 8 * c, hw);
+        tmem_st8(acol + 64 + 8 * c, lw);
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          if (c & 1) planes[p][c >> 1] |= pw[p] << 16;
+          else planes[p][c >> 1] = pw[p];
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a2_full[g]);
+      if (valid)
+#pragma unroll
+        for (int p = 0; p < MB; ++p)
+          *reinterpret_cast<uint4 *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes) =
+              make_uint4(planes[p][0], planes[p][1], planes[p][2], planes[p][3]);
+      // ---- E2: r = u - Pi^T c, ||r||, residual operand R ----
+      if (!qwait(&S.d2_full[g], ph, &S.abort_flag)) break;
+      tc_fence_after();
+      float rr = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t d[16];
+        tmem_ld16(dcol + 16 * c, d);
+        tmem_wait_ld();
+        uint32_t hw[8], lw[8];
+#pragma unroll
+        for (int c8 = 0; c8 < 2; ++c8) {
+          const uint4 kv = *reinterpret_cast<const uint4 *>(a1 + blk_off(r, 16 * c + 8 * c8));
+          const __half2 *kh = reinterpret_cast<const __half2 *>(&kv);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 kf = __half22float2(kh[e2]);
+            const int e = 8 * c8 + 2 * e2;
+            const float r0 = zero ? 0.f : kf.x * inv2 - __uint_as_float(d[e]) * 1.4901161193847656e-08f;
+            const float r1 = zero ? 0.f : kf.y * inv2 - __uint_as_float(d[e + 1]) * 1.4901161193847656e-08f;
+            rr = fmaf(r0, r0, rr);
+            rr = fmaf(r1, r1, rr);
+            float h0, l0, h1, l1;
+            split16(r0 * kRScale, h0, l0);
+            split16(r1 * kRScale, h1, l1);
+            hw[4 * c8 + e2] = pack_h2(h0, h1);
+            lw[4 * c8 + e2] = pack_h2(l0, l1);
+          }
+        }
+        tmem_st8(acol + 8 * c, hw);
+        tmem_st8(acol + 64 + 8 * c, lw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&S.a3_full[g]);
+        mbar_arrive(&S.a1_free[g]);
+      }
+      // ---- E3: signs of z = S r, norms ----
+      if (!qwait(&S.d3_full[g], ph, &S.abort_flag)) break;
+      tc_fence_after();
+      uint32_t sw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t d[16];
+        tmem_ld16(dcol + 16 * c, d);
+        tmem_wait_ld();
+        uint32_t wv = 0u;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) wv |= (__uint_as_float(d[e]) >= 0.f ? 1u : 0u) << e;
+        sw[c >> 1] |= (zero ? 0u : wv) << (16 * (c & 1));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.d_free[g]);
+      if (valid) {
+        *reinterpret_cast<uint4 *>(tp + L.signs + slot * kRowBytes) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+        const float rn = zero ? 0.f : sqrtf(rr);
+        *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) =
+            __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+    tmem_relinquish();
+  }
+}
+
+template <int MB>
+cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
+  const size_t smem = sizeof(QtSmem);
+  static_assert(sizeof(QtSmem) <= 227 * 1024, "shared memory per CTA");
+  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  quantize_tc_kernel<MB><<<grid, kQtThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool quantize_tc_supported(const AppendArgs &a) {
+  return a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 && a.value_bits >= 2 &&
+         a.value_bits <= 4 && a.T >= 64;
+}
+
+cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream) {
+  int total = 0;
+  for (int b = 0; b < a.batch; ++b) {
+    a.tstart[b] = total;
+    total += a.h_kv * ((a.nnew[b] + 127) / 128);
+  }
+  a.tstart[a.batch] = total;
+  a.total_tiles = total;
+  if (total == 0) return cudaSuccess;
+  const int grid = total < num_sms ? total : num_sms;
+  switch (a.key_bits - 1) {
+    case 1: return launch_qt<1>(a, grid, stream);
+    case 2: return launch_qt<2>(a, grid, stream);
+    case 3: return launch_qt<3>(a, grid, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace tq

@@ -152,7 +152,9 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
   a.key_bits = p->key_bits; a.value_bits = p->value_bits; a.dtype = dtype;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
-  if (tq::launch_quantize_simt(a, sms, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  const cudaError_t e = tq::quantize_tc_supported(a) ? tq::launch_quantize_tc(a, sms, (cudaStream_t)stream)
+                                                    : tq::launch_quantize_simt(a, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }
 

@@ -12,8 +12,8 @@
 namespace tq {
 
 // Arguments of one quantize_append launch.  Passed by value as a
-// __grid_constant__ kernel parameter (8 KB of per-sequence lengths; CUDA
-// 12.1+ allows kernel parameters up to 32764 bytes).
+// __grid_constant__ kernel parameter (12 KB of per-sequence lengths and tile
+// offsets; CUDA 12.1+ allows kernel parameters up to 32764 bytes).
 struct AppendArgs {
   const float *pi, *s, *centroids, *boundaries;
   void *data;
@@ -23,6 +23,10 @@ struct AppendArgs {
   tq_dtype dtype;
   int lens[TQ_MAX_BATCH];
   int nnew[TQ_MAX_BATCH];
+  // tensor-core path: 128-token tiles per (sequence, head); sequence b owns
+  // tiles [tstart[b], tstart[b + 1])
+  int tstart[TQ_MAX_BATCH + 1];
+  int total_tiles;
 };
 
 // Split-K plan of one decode call (host-computed, identical in the
@@ -67,6 +71,9 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
                             int key_bits, int value_bits);
 
 cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream);
+// Tensor-core quantize-append (bf16 K/V, appends of 64+ tokens).
+bool quantize_tc_supported(const AppendArgs &a);
+cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 // Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
 bool decode_tc_supported(int key_bits, int value_bits, int gqa);

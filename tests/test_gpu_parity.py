@@ -64,6 +64,7 @@ def _append_all(glayer, cache, wl, chunks, device_tensors):
     ("tiny", [(0, 256)]),
     ("tiny", [(0, 100), (100, 101), (101, 256)]),      # ragged tails, mid-tile starts
     ("llama8b", [(0, 4096)]),
+    ("llama8b", [(0, 40), (40, 1000), (1000, 4096)]),  # short append (SIMT), then tiles mid-way
 ])
 def test_quantize_append_parity(name, chunks):
     wl = workloads.by_name(name)
@@ -82,7 +83,7 @@ def test_quantize_append_parity(name, chunks):
         v = dev[b][1].float().cpu().numpy()
         for h in range(wl.h_kv):
             ke, ve = olayer.encode(k[:, h], v[:, h])
-            stats = pu.compare_records(spec, buf, b, h, 0, ke, ve, stats)
+            stats = pu.compare_records(spec, buf, b, h, 0, ke, ve, stats, olayer, k[:, h])
     pu.check_band_fraction(stats)
     print(name, chunks, stats)
 
@@ -112,7 +113,7 @@ def test_quantize_append_ragged_batch_and_zero_key():
         vv = v[b, :nnew[b]].float().numpy()
         for h in range(wl.h_kv):
             ke, ve = olayer.encode(kk[:, h], vv[:, h])
-            stats = pu.compare_records(spec, buf, b, h, lens0[b], ke, ve, stats)
+            stats = pu.compare_records(spec, buf, b, h, lens0[b], ke, ve, stats, olayer, kk[:, h])
         # slots before lens0 and after lens0 + nnew stay untouched (zeroed buffer)
         if lens0[b] > 0:
             assert not spec.read(buf, b, 0, 0, lens0[b])["nk16"].any()
@@ -138,8 +139,34 @@ def test_quantize_append_bit_widths(kb, vb):
     stats = None
     for h in range(wl.h_kv):
         ke, ve = olayer.encode(k[:, h].numpy(), v[:, h].numpy())
-        stats = pu.compare_records(spec, buf, 0, h, 0, ke, ve, stats)
+        stats = pu.compare_records(spec, buf, 0, h, 0, ke, ve, stats, olayer, k[:, h].numpy())
     pu.check_band_fraction(stats)
+
+
+@pytest.mark.parametrize("kb,vb", [(2, 2), (4, 2), (3, 3), (4, 4)])
+def test_quantize_append_bit_widths_bf16_tiles(kb, vb):
+    """bf16 appends of 300 tokens (the tensor-core kernel) at every key and
+    value width, into a sequence that already holds 77 tokens."""
+    import dataclasses
+    wl = dataclasses.replace(workloads.llama8b(), batch=2, key_bits=kb, value_bits=vb,
+                             capacity=384, lengths=(377, 377), name=f"tcbits{kb}{vb}")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, 2, wl.h_kv, 384, zero=True)
+    T = 300
+    k = torch.stack([workloads.kv_tokens(wl, b, 0, T)[0] for b in range(2)])
+    v = torch.stack([workloads.kv_tokens(wl, b, 0, T)[1] for b in range(2)])
+    tq.tq_quantize_append(glayer, cache, k.to(DEV).contiguous(), v.to(DEV).contiguous(), [77, 0],
+                          [T, 250])
+    torch.cuda.synchronize()
+    buf = cache.buffer.cpu().numpy()
+    stats = None
+    for b, (start, n) in enumerate([(77, T), (0, 250)]):
+        for h in range(wl.h_kv):
+            ke, ve = olayer.encode(k[b, :n, h].float().numpy(), v[b, :n, h].float().numpy())
+            stats = pu.compare_records(spec, buf, b, h, start, ke, ve, stats, olayer,
+                                       k[b, :n, h].float().numpy())
+    pu.check_band_fraction(stats)
+    print(kb, vb, stats)
 
 
 # ---------------------------------------------------------------------------
