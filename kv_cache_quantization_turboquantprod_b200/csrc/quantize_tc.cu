@@ -60,7 +60,8 @@ struct QtSmem {
   float nk[2][128];
   int sh[2][128];
   float cent[8];
-  float bnd[8];
+  float bnd[8];                  // ascending, padded with +inf
+  uint32_t cpair[2][64];         // packed fp16 (hi, lo) parts of c[i0], c[i1] x 2^16, index i0 | i1 << 3
   uint64_t a1_full[2], a1_free[2], d1_full[2], a2_full[2], d2_full[2], a3_full[2], d3_full[2],
       d_free[2];
   uint32_t tmem_base;
@@ -135,7 +136,15 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     *reinterpret_cast<__half *>(S.s[1] + blk_off(i, j)) = __float2half_rn(lo);
   }
   if (tid < ncent) S.cent[tid] = a.centroids[tid];
-  if (tid < ncent - 1) S.bnd[tid] = a.boundaries[tid];
+  if (tid < 8) S.bnd[tid] = tid < ncent - 1 ? a.boundaries[tid] : INFINITY;
+  if (tid < 64) {
+    const int i0 = tid & 7, i1 = tid >> 3;
+    float h0 = 0.f, l0 = 0.f, h1 = 0.f, l1 = 0.f;
+    if (i0 < ncent) split16(a.centroids[i0] * kCScale, h0, l0);
+    if (i1 < ncent) split16(a.centroids[i1] * kCScale, h1, l1);
+    S.cpair[0][tid] = pack_h2(h0, h1);
+    S.cpair[1][tid] = pack_h2(l0, l1);
+  }
   if (tid == 0) {
     for (int g = 0; g < 2; ++g) {
       mbar_init(&S.a1_full[g], 4);
@@ -256,27 +265,44 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     // either is used.
     const int w = warp - 1, rr = lane >> 2, q = lane & 3;
     const float vlevels = (float)((1 << a.value_bits) - 1);
+    // rows of step u = 4 i + pass; the next step's rows are fetched while
+    // this step's are converted
+    auto fetch = [&](int u, uint4 (&kr)[4], uint4 (&vr)[4]) {
+      const int i = u >> 2, pass = u & 3;
+      bool valid = i < nlocal;
+      size_t base = 0;
+      if (valid) {
+        const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
+        const int r = 32 * pass + 8 * w + rr;
+        valid = r < ti.nrow;
+        base = ((((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD + 32 * q);
+      }
+      const uint4 *ks = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + base);
+      const uint4 *vs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v) + base);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        kr[c] = valid ? ks[c] : make_uint4(0u, 0u, 0u, 0u);
+        vr[c] = valid ? vs[c] : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    uint4 kr[4], vr[4];
+    fetch(0, kr, vr);
     for (int i = 0; i < nlocal; ++i) {
       const int g = i & 1;
-      if (i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag)) break;
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
       uint8_t *a1 = S.a1[g];
+      bool stop = false;
 #pragma unroll 1
       for (int pass = 0; pass < 4; ++pass) {
+        uint4 kn[4], vn[4];
+        fetch(4 * i + pass + 1, kn, vn);
+        if (pass == 0 && i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag)) {
+          stop = true;
+          break;
+        }
         const int r = 32 * pass + 8 * w + rr;
         const bool valid = r < ti.nrow;
         const int t = ti.t0 + r;
-        const size_t base = valid ? ((((size_t)ti.b * a.T + t) * a.h_kv + ti.h) * kD + 32 * q) : 0;
-        uint4 kr[4], vr[4];
-        {
-          const uint4 *ks = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + base);
-          const uint4 *vs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v) + base);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            kr[c] = valid ? ks[c] : make_uint4(0u, 0u, 0u, 0u);
-            vr[c] = valid ? vs[c] : make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
         // ---- key: norm, per-vector scale, fp16 operand ----
         float ss = 0.f, mx = 0.f;
 #pragma unroll
@@ -332,38 +358,58 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           const int pos = a.lens[ti.b] + t;
           uint8_t *tp = tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile);
           const int slot = pos % kTile;
-          uint32_t w2[2] = {0u, 0u}, wp[4] = {0u, 0u, 0u, 0u};
+          // code = clamp(rint((v - zero) / scale)) with an exactly rounded
+          // quotient.  The reciprocal product is within 2 ulp of it, so it
+          // decides the code unless it sits next to a half-integer; those
+          // (rare) elements are redone with the exact division afterwards.
+          uint32_t codes[4] = {0u, 0u, 0u, 0u};  // 4 bits per element, 8 per word
+          uint32_t fix = 0u;
+          if (sc32 != 0.f) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[c]);
+            for (int c = 0; c < 4; ++c) {
+              const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[c]);
 #pragma unroll
-            for (int e2 = 0; e2 < 8; ++e2) {
-              const int e = 8 * c + e2;
-              const float2 f = __bfloat1622float2(p2[e2 >> 1]);
-              const float x = (e2 & 1) ? f.y : f.x;
-              // the code is rint((v - zero) / scale) with an exactly rounded
-              // quotient; the reciprocal product is within 2 ulp of it, so it
-              // decides the code unless it sits next to a half-integer
-              const float num = __fsub_rn(x, z32);
-              float tq = num * rsc;
-              const float fr = tq - floorf(tq);
-              if (fabsf(fr - 0.5f) < 1e-5f) tq = __fdiv_rn(num, sc32);
-              tq = fminf(fmaxf(rintf(tq), 0.f), vlevels);
-              const uint32_t code = sc32 != 0.f ? (uint32_t)tq : 0u;
-              w2[e >> 4] |= (code & 3u) << (2 * (e & 15));
-#pragma unroll
-              for (int p = 0; p < 4; ++p) wp[p] |= ((code >> p) & 1u) << e;
+              for (int e2 = 0; e2 < 8; ++e2) {
+                const float2 f = __bfloat1622float2(p2[e2 >> 1]);
+                const float tq = __fsub_rn((e2 & 1) ? f.y : f.x, z32) * rsc;
+                const float fr = tq - floorf(tq);
+                fix |= (fabsf(fr - 0.5f) < 1e-5f ? 1u : 0u) << (8 * c + e2);
+                codes[c] |= (uint32_t)fminf(fmaxf(rintf(tq), 0.f), vlevels) << (4 * e2);
+              }
+            }
+            const __nv_bfloat16 *vrow = reinterpret_cast<const __nv_bfloat16 *>(a.v) +
+                                        ((((size_t)ti.b * a.T + t) * a.h_kv + ti.h) * kD + 32 * q);
+            while (fix) {
+              const int e = __ffs(fix) - 1;
+              fix &= fix - 1;
+              const float tq = __fdiv_rn(__fsub_rn(__bfloat162float(vrow[e]), z32), sc32);
+              const uint32_t code = (uint32_t)fminf(fmaxf(rintf(tq), 0.f), vlevels);
+              codes[e >> 3] = (codes[e >> 3] & ~(15u << (4 * (e & 7)))) | (code << (4 * (e & 7)));
             }
           }
           if (L.vb == 2) {
+            // channel 4i + m of the group in bits 2m, 2m+1 of byte i
+            uint32_t w2[2] = {0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w2[e >> 4] |= ((codes[e >> 3] >> (4 * (e & 7))) & 3u) << (2 * (e & 15));
             *reinterpret_cast<uint2 *>(tp + L.vplanes + slot * kPackedRowBytes + 8 * q) = make_uint2(w2[0], w2[1]);
           } else {
-            for (int p = 0; p < L.vb; ++p)
-              *reinterpret_cast<uint32_t *>(tp + L.vplanes + p * kPlaneBytes + slot * kRowBytes + 4 * q) = wp[p];
+            for (int p = 0; p < L.vb; ++p) {
+              uint32_t wp = 0u;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) wp |= ((codes[e >> 3] >> (4 * (e & 7) + p)) & 1u) << e;
+              *reinterpret_cast<uint32_t *>(tp + L.vplanes + p * kPlaneBytes + slot * kRowBytes + 4 * q) = wp;
+            }
           }
           *reinterpret_cast<__half2 *>(tp + L.vsz + (slot * kGroups + q) * 4) = __halves2half2(scale16, zero16);
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          kr[c] = kn[c];
+          vr[c] = vn[c];
+        }
       }
+      if (stop) break;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.a1_full[g]);
@@ -376,12 +422,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const uint32_t dcol = tbase + lane_off + g * 256, acol = dcol + 128;
     const uint8_t *a1 = S.a1[g];
-    constexpr int NB = (1 << MB) - 1;
-    float bnd[NB], cent[NB + 1];
-#pragma unroll
-    for (int x = 0; x < NB; ++x) bnd[x] = S.bnd[x];
-#pragma unroll
-    for (int x = 0; x <= NB; ++x) cent[x] = S.cent[x] * kCScale;
+    constexpr int NC = 1 << MB;
     for (int i = g; i < nlocal; i += 2) {
       const uint32_t ph = (i >> 1) & 1;
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
@@ -397,37 +438,35 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       const float rnk = zero ? 0.f : 1.f / nk;
       const float inv1 = ldexpf(rnk, -(sh + 10));  // y = Y 2^-(s+10) / ||k||
       const float inv2 = ldexpf(rnk, -sh);         // u = K 2^-s / ||k||
-      // ---- E1: y = Pi u, codes, centroid operand C (16 columns at a time) ----
+      // ---- E1: y = Pi u, codes, centroid operand C (16 columns at a time,
+      // the next chunk's TMEM load in flight while this one is processed) ----
       uint32_t planes[3][4];
+      uint32_t dA[16], dB[16];
+      tmem_ld16(dcol, dA);
+      tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        uint32_t d[16];
-        tmem_ld16(dcol + 16 * c, d);
-        tmem_wait_ld();
+        uint32_t(&d)[16] = (c & 1) ? dB : dA;
+        if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
         uint32_t hw[8], lw[8];
         uint32_t pw[3] = {0u, 0u, 0u};
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          float cv[2];
+          int ix[2];
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             const float y = __uint_as_float(d[e + x]) * inv1;
-            int idx = 0;
+            int idx = 0;  // #{boundaries < y}, binary search
 #pragma unroll
-            for (int qq = 0; qq < NB; ++qq) idx += (bnd[qq] < y) ? 1 : 0;
-            if (zero) idx = 0;
+            for (int step = NC / 2; step >= 1; step >>= 1) idx += (S.bnd[idx + step - 1] < y) ? step : 0;
+            idx = zero ? 0 : idx;
 #pragma unroll
             for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
-            float cc = cent[0];
-#pragma unroll
-            for (int qq = 1; qq <= NB; ++qq) cc = (idx == qq) ? cent[qq] : cc;
-            cv[x] = zero ? 0.f : cc;
+            ix[x] = idx;
           }
-          float h0, l0, h1, l1;
-          split16(cv[0], h0, l0);
-          split16(cv[1], h1, l1);
-          hw[e >> 1] = pack_h2(h0, h1);
-          lw[e >> 1] = pack_h2(l0, l1);
+          const int pi2 = ix[0] | (ix[1] << 3);
+          hw[e >> 1] = zero ? 0u : S.cpair[0][pi2];
+          lw[e >> 1] = zero ? 0u : S.cpair[1][pi2];
         }
         tmem_st8(acol + 8 * c, hw);
         tmem_st8(acol + 64 + 8 * c, lw);
@@ -436,6 +475,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           if (c & 1) planes[p][c >> 1] |= pw[p] << 16;
           else planes[p][c >> 1] = pw[p];
         }
+        if (c < 7) tmem_wait_ld();
       }
       tmem_wait_st();
       tc_fence_before();
@@ -449,12 +489,14 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       // ---- E2: r = u - Pi^T c, ||r||, residual operand R ----
       if (!qwait(&S.d2_full[g], ph, &S.abort_flag)) break;
       tc_fence_after();
-      float rr = 0.f;
+      float rr = 0.f;  // ||r||^2 x 2^26
+      const float inv2r = inv2 * kRScale;
+      tmem_ld16(dcol, dA);
+      tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        uint32_t d[16];
-        tmem_ld16(dcol + 16 * c, d);
-        tmem_wait_ld();
+        uint32_t(&d)[16] = (c & 1) ? dB : dA;
+        if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
         uint32_t hw[8], lw[8];
 #pragma unroll
         for (int c8 = 0; c8 < 2; ++c8) {
@@ -464,19 +506,21 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           for (int e2 = 0; e2 < 4; ++e2) {
             const float2 kf = __half22float2(kh[e2]);
             const int e = 8 * c8 + 2 * e2;
-            const float r0 = zero ? 0.f : kf.x * inv2 - __uint_as_float(d[e]) * 1.4901161193847656e-08f;
-            const float r1 = zero ? 0.f : kf.y * inv2 - __uint_as_float(d[e + 1]) * 1.4901161193847656e-08f;
-            rr = fmaf(r0, r0, rr);
-            rr = fmaf(r1, r1, rr);
-            float h0, l0, h1, l1;
-            split16(r0 * kRScale, h0, l0);
-            split16(r1 * kRScale, h1, l1);
-            hw[4 * c8 + e2] = pack_h2(h0, h1);
-            lw[4 * c8 + e2] = pack_h2(l0, l1);
+            // r x 2^13 = u 2^13 - (Pi^T c) 2^13, with D = (Pi^T c) 2^26
+            const float s0 = zero ? 0.f : fmaf(__uint_as_float(d[e]), -1.220703125e-04f, kf.x * inv2r);
+            const float s1 = zero ? 0.f : fmaf(__uint_as_float(d[e + 1]), -1.220703125e-04f, kf.y * inv2r);
+            rr = fmaf(s0, s0, rr);
+            rr = fmaf(s1, s1, rr);
+            const __half2 hh = __floats2half2_rn(s0, s1);
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(s0 - hf.x, s1 - hf.y);
+            hw[4 * c8 + e2] = *reinterpret_cast<const uint32_t *>(&hh);
+            lw[4 * c8 + e2] = *reinterpret_cast<const uint32_t *>(&ll);
           }
         }
         tmem_st8(acol + 8 * c, hw);
         tmem_st8(acol + 64 + 8 * c, lw);
+        if (c < 7) tmem_wait_ld();
       }
       tmem_wait_st();
       tc_fence_before();
@@ -489,22 +533,24 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       if (!qwait(&S.d3_full[g], ph, &S.abort_flag)) break;
       tc_fence_after();
       uint32_t sw[4] = {0u, 0u, 0u, 0u};
+      tmem_ld16(dcol, dA);
+      tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        uint32_t d[16];
-        tmem_ld16(dcol + 16 * c, d);
-        tmem_wait_ld();
+        uint32_t(&d)[16] = (c & 1) ? dB : dA;
+        if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
         uint32_t wv = 0u;
 #pragma unroll
         for (int e = 0; e < 16; ++e) wv |= (__uint_as_float(d[e]) >= 0.f ? 1u : 0u) << e;
         sw[c >> 1] |= (zero ? 0u : wv) << (16 * (c & 1));
+        if (c < 7) tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.d_free[g]);
       if (valid) {
         *reinterpret_cast<uint4 *>(tp + L.signs + slot * kRowBytes) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-        const float rn = zero ? 0.f : sqrtf(rr);
+        const float rn = zero ? 0.f : sqrtf(rr) * (1.f / kRScale);
         *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) =
             __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
       }
