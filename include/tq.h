@@ -107,8 +107,8 @@ typedef struct {
   int key_bits;   /* 2..4 total key bits: key_bits - 1 Lloyd-Max bits + 1 QJL bit */
   int value_bits; /* 2..4 */
   int group;      /* value quantization group; 32 */
-  const float *pi;         /* [d][d] row-major: Pi, y = Pi u */
-  const float *s;          /* [d][d] row-major: S, QJL sketch of r is S r */
+  const float *pi;         /* [d][d] row-major: Pi, y = Pi u; 16-byte aligned */
+  const float *s;          /* [d][d] row-major: S, QJL sketch of r is S r; 16-byte aligned */
   const float *centroids;  /* [2^(key_bits-1)] ascending */
   const float *boundaries; /* [2^(key_bits-1) - 1] ascending decision boundaries */
 } tq_params;

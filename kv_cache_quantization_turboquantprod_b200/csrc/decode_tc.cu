@@ -790,10 +790,8 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   uint8_t *blk = reinterpret_cast<uint8_t *>(red + 8 * G * 4);  // QBLOCK staging
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  for (int i = tid; i < 2 * kD * kD; i += 256) {
-    const int r = i / kD, c = i % kD;
-    mat[r * kPadQ + c] = (r < kD) ? a.pi[i] : a.s[i - kD * kD];
-  }
+  stage_matrix(mat, kPadQ, a.pi, tid, 256);
+  stage_matrix(mat + kD * kPadQ, kPadQ, a.s, tid, 256);
   for (int i = tid; i < C::QBLOCK / 4; i += 256) reinterpret_cast<uint32_t *>(blk)[i] = 0u;
   // Walsh coefficients of the codebook, idx paired with its complement so
   // that a symmetric codebook gives exact zeros for the even subsets

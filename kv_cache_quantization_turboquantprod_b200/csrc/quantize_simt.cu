@@ -59,11 +59,8 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
   const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
   const int ncent = 1 << L.mb;
 
-  for (int i = tid; i < kD * kD; i += kThreads) {
-    const int r = i / kD, cc = i % kD;
-    S.pi[r * kPad + cc] = a.pi[i];
-    S.s[r * kPad + cc] = a.s[i];
-  }
+  stage_matrix(S.pi, kPad, a.pi, tid, kThreads);
+  stage_matrix(S.s, kPad, a.s, tid, kThreads);
   if (tid < ncent) S.cent[tid] = a.centroids[tid];
   if (tid < ncent - 1) S.bnd[tid] = a.boundaries[tid];
   __syncthreads();

@@ -125,15 +125,32 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                          : 0;
 
   // ---- setup: split Pi and S into fp16 parts, barriers, TMEM -------------
-  for (int e = tid; e < 128 * 128; e += kQtThreads) {
-    const int i = e >> 7, j = e & 127;
-    float hi, lo;
-    split16(a.pi[e] * kPiScale, hi, lo);
-    *reinterpret_cast<__half *>(S.pi[0] + blk_off(i, j)) = __float2half_rn(hi);
-    *reinterpret_cast<__half *>(S.pi[1] + blk_off(i, j)) = __float2half_rn(lo);
-    split16(a.s[e] * kSScale, hi, lo);
-    *reinterpret_cast<__half *>(S.s[0] + blk_off(i, j)) = __float2half_rn(hi);
-    *reinterpret_cast<__half *>(S.s[1] + blk_off(i, j)) = __float2half_rn(lo);
+  // eight elements (one 16-byte block row) per item, both matrices' loads
+  // issued before any is used
+  for (int it = tid; it < 128 * 16; it += kQtThreads) {
+    const int i = it >> 4, j0 = (it & 15) * 8;
+    const float4 *pp = reinterpret_cast<const float4 *>(a.pi + i * 128 + j0);
+    const float4 *sp = reinterpret_cast<const float4 *>(a.s + i * 128 + j0);
+    const float4 p0 = pp[0], p1 = pp[1], s0 = sp[0], s1 = sp[1];
+    const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    uint32_t ph[4], pl[4], sh2[4], sl[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float h0, l0, h1, l1;
+      split16(pv[2 * e] * kPiScale, h0, l0);
+      split16(pv[2 * e + 1] * kPiScale, h1, l1);
+      ph[e] = pack_h2(h0, h1);
+      pl[e] = pack_h2(l0, l1);
+      split16(sv[2 * e] * kSScale, h0, l0);
+      split16(sv[2 * e + 1] * kSScale, h1, l1);
+      sh2[e] = pack_h2(h0, h1);
+      sl[e] = pack_h2(l0, l1);
+    }
+    *reinterpret_cast<uint4 *>(S.pi[0] + blk_off(i, j0)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+    *reinterpret_cast<uint4 *>(S.pi[1] + blk_off(i, j0)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    *reinterpret_cast<uint4 *>(S.s[0] + blk_off(i, j0)) = make_uint4(sh2[0], sh2[1], sh2[2], sh2[3]);
+    *reinterpret_cast<uint4 *>(S.s[1] + blk_off(i, j0)) = make_uint4(sl[0], sl[1], sl[2], sl[3]);
   }
   if (tid < ncent) S.cent[tid] = a.centroids[tid];
   if (tid < 8) S.bnd[tid] = tid < ncent - 1 ? a.boundaries[tid] : INFINITY;

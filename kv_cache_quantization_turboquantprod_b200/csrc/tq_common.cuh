@@ -94,6 +94,33 @@ __device__ __forceinline__ float warp_min(float x) {
   return x;
 }
 
+// Copy a row-major kD x kD fp32 matrix (16-byte aligned) into shared memory
+// with a row stride of `pad` floats.  Eight 16-byte loads per thread are in
+// flight at a time, so staging is bandwidth- rather than latency-bound.
+__device__ __forceinline__ void stage_matrix(float *dst, int pad, const float *src, int tid, int nthr) {
+  const float4 *s4 = reinterpret_cast<const float4 *>(src);
+  constexpr int kN4 = kD * kD / 4;
+  for (int base = tid; base < kN4; base += 8 * nthr) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * nthr;
+      v[u] = i < kN4 ? s4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * nthr;
+      if (i < kN4) {
+        float *d = dst + ((4 * i) / kD) * pad + (4 * i) % kD;
+        d[0] = v[u].x;
+        d[1] = v[u].y;
+        d[2] = v[u].z;
+        d[3] = v[u].w;
+      }
+    }
+  }
+}
+
 // QJL constant sqrt(pi/2) / d.
 __host__ __device__ constexpr float qjl_kappa() { return 1.2533141373155003f / kD; }
 

@@ -45,6 +45,7 @@ tq_status check_params(const tq_params *p) {
   if (p->key_bits < 2 || p->key_bits > 4) return TQ_ERR_UNSUPPORTED;
   if (p->value_bits < 2 || p->value_bits > 4) return TQ_ERR_UNSUPPORTED;
   if (!p->pi || !p->s || !p->centroids || !p->boundaries) return TQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(p->pi, 16) || !aligned(p->s, 16)) return TQ_ERR_INVALID_ARGUMENT;
   return TQ_OK;
 }
 

@@ -77,6 +77,11 @@ def test_record_and_cache_bytes():
     assert lib.tq_record_bytes(ctypes.byref(_params(d=64))) == 0
     assert lib.tq_record_bytes(ctypes.byref(_params(g=16))) == 0
     assert lib.tq_record_bytes(ctypes.byref(_params(kb=5))) == 0
+    # Pi and S must be 16-byte aligned (the kernels stage them with 16-byte loads)
+    misaligned = tq.Params(128, 3, 2, 32, 264, 256, 256, 256)
+    assert lib.tq_record_bytes(ctypes.byref(misaligned)) == 0
+    misaligned = tq.Params(128, 3, 2, 32, 256, 260, 256, 256)
+    assert lib.tq_record_bytes(ctypes.byref(misaligned)) == 0
 
 
 def test_append_validation_before_launch():
