@@ -305,7 +305,7 @@ def run_ours(args, rank, world, device):
             "key_bits": wl.key_bits, "value_bits": wl.value_bits, "group": wl.group,
             "capacity": wl.capacity, "ctx_tokens_per_step_per_gpu": ctx_tokens_step,
             "lengths": "ragged uniform [16384, 32768]" if wl.name == "batched" else list(wl.lengths),
-            "step": "quantize-append 1 token/sequence + decode (qprep, split-K, combine)",
+            "step": "quantize-append 1 token/sequence + decode (query blocks, split-K, combine)",
             "l2": "no flush: each step streams the whole compressed cache (> 126 MB L2)",
             "parallelism": f"dp{world} (independent batches per GPU)",
         },
@@ -313,7 +313,7 @@ def run_ours(args, rank, world, device):
         "decode_ms": dec_ms,
         "record_bytes": rec_bytes,
         "roofline": {
-            "kernel": "tq_decode_attention (qprep + split-K + combine, timed as one call)",
+            "kernel": "tq_decode_attention (query blocks + split-K + combine, timed as one call)",
             "bound": "hbm",
             "achieved": achieved,
             "peak": peak,
