@@ -12,17 +12,18 @@
 // query head) inside the ~20 issue slots per record that full bandwidth
 // allows, so both contractions run on the tensor cores with exact operands.
 //
-//   Scores (kind::mxf4, K = 64 per instruction, unit block scales).  Write
-//   the code bits of coordinate j as spins s_k = 2 b_k - 1.  Any codebook
-//   of 2^m levels is a multilinear polynomial in the spins (its Walsh
-//   expansion), c(idx) = a_0 + sum_S a_S prod_{k in S} s_k, and for the
-//   symmetric Lloyd-Max codebooks only the odd subsets S survive (1, 2 and
-//   4 planes at m = 1, 2, 3).  Each subset's spin product and the QJL sign
-//   (2 sign - 1 is a spin too) become +-1 e2m1 operands, four per byte
-//   operation; the query side B holds a_S Pi q (and S q) as balanced base-9
-//   digits in [-4, 4], all exact in e2m1, so every product and the f32
-//   accumulation of a 128-coordinate tile is exact.  The limbs are combined
-//   per (token, head) in the epilogue.
+//   Scores (kind::i8, A from tensor memory).  Write the code bits of
+//   coordinate j as spins s_k = 2 b_k - 1.  Any codebook of 2^m levels is a
+//   multilinear polynomial in the spins (its Walsh expansion),
+//   c(idx) = a_0 + sum_S a_S prod_{k in S} s_k, and for the symmetric
+//   Lloyd-Max codebooks only the odd subsets S survive (1, 2 and 4 planes at
+//   m = 1, 2, 3).  A spin is 2 bit - 1, so each subset plane and the QJL sign
+//   plane enter as 0/1 bits (the -1 halves are per-head constants).  One LOP3
+//   (w & (0x01010101 << k)) turns a 32-bit plane word into four u8 operands
+//   of weight 2^k; the key group stores them straight into tensor memory, so
+//   the score operands never touch shared memory.  The query side B holds
+//   2 a_S Pi q / 2^k (and 2 S q / 2^k) in four signed base-128 limbs; the s32
+//   accumulation is exact and the limbs are combined per (token, head).
 //   Values (kind::i8): D[channel, (group, head, byte)] = A_v[channel, code
 //   bytes x tokens] x B_p[tokens, p * scale_g as 22-bit fixed point].  Two-
 //   bit codes are stored packed, so one mask (w & (0x03030303 << 2m))
@@ -37,7 +38,7 @@
 //   warp 0        bulk-copy producer; allocates / frees tensor memory
 //   warp 1        MMA issuer (one elected lane issues), polling the score
 //                 and PV queues so neither blocks the other
-//   warps 2-5     key group: code bits -> spin planes (shared memory)
+//   warps 2-5     key group: code-bit / sign planes -> u8 operands in tensor memory
 //   warps 6-9     value group: codes -> A_v (MN-major, shared memory); PV
 //                 epilogue and the per-channel accumulators
 //   warps 10-17   two softmax groups taking alternate tiles, each with its
@@ -61,43 +62,32 @@ using namespace sm100;
 constexpr int kTcThreads = 576;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTmemCols = 512;
-constexpr int kColSF = 448;         // 64 columns of 1.0 block scales (ue8m0 0x7F)
-constexpr int kPlaneBytes4 = 128 * 64;  // one e2m1 operand plane: 128 rows x 128 coordinates
+constexpr int kPlaneCols = 32;  // one u8 operand plane: 128 coordinates per row = 32 TMEM columns
 
 // 2^n for n in [-126, 127]
 __device__ __forceinline__ float exp2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
 // floor(log2(x)) for a positive normal float
 __device__ __forceinline__ int ilog2f(float x) { return (int)((__float_as_uint(x) >> 23) & 0xFF) - 127; }
 
-// balanced base-9 digits per query coordinate: 8 (|X| < 2^24.3), or 6 when
-// eight do not fit the tensor-memory budget (8 query heads per KV head)
-__host__ __device__ constexpr int limbs_for(int G) { return G <= 6 ? 8 : 6; }
-// floor(log2((9^L - 1) / 2)): the largest |X| is below 2^(this + 1)
-__host__ __device__ constexpr int xbits_for(int L) {
-  long long x = 1;
-  for (int l = 0; l < L; ++l) x *= 9;
-  x = (x - 1) / 2;
-  int e = 0;
-  while ((x >> (e + 1)) != 0) ++e;
-  return e;
-}
-__host__ __device__ constexpr int score_n(int G) { return ((limbs_for(G) * G + 15) / 16) * 16; }
+// score N per accumulator: 4 limbs per query head
+__host__ __device__ constexpr int score_n(int G) { return ((4 * G + 15) / 16) * 16; }
 // all non-empty code-bit subsets + the sign plane
 __host__ __device__ constexpr int max_planes(int MB) { return (1 << MB); }
 
 // Score constants that follow B_q in a query block.
 constexpr int kQConstBytes = 256;
 struct QConst {
-  float cm[8];      // a_0 * sum_j q~_j
-  float inv_m[8];   // 2^-F of the MSE limbs
-  float inv_s[8];   // 2^-F of the QJL limbs
-  int n_mse;        // active subset planes (1 .. 2^m - 1)
-  int subset[7];    // their code-bit masks
+  float cm[8];         // (a_0 - sum of the active a_S) * sum_j q~_j
+  float csum[8];       // sum_j s^_j
+  float coef_m[8][2];  // limb weights of the MSE term: 2^-F, 2^(14-F)
+  float coef_s[8][2];  // limb weights of the QJL term
+  int n_mse;           // active subset planes (1 .. 2^m - 1)
+  int subset[7];       // their code-bit masks
 };
 static_assert(sizeof(QConst) <= kQConstBytes, "query constants");
 
 __host__ __device__ constexpr size_t qblock_bytes_for(int MB, int G) {
-  return (size_t)max_planes(MB) * 64 * score_n(G) + kQConstBytes;
+  return (size_t)max_planes(MB) * 128 * score_n(G) + kQConstBytes;
 }
 
 template <int MB_, int VB_, int G_>
@@ -105,16 +95,15 @@ struct Cfg {
   static constexpr int MB = MB_, VB = VB_, G = G_;
   // MSE planes of a symmetric codebook (the odd code-bit subsets)
   static constexpr int NSYM = MB == 1 ? 1 : (MB == 2 ? 2 : 4);
-  static constexpr int L = limbs_for(G);
   static constexpr int NS = score_n(G);                 // score N per accumulator
   static constexpr int NPV = 16 * G;                    // PV N: 4 groups x G heads x 4 bytes
   static constexpr int NPL = max_planes(MB);            // operand planes, upper bound
-  // A_k plane slots: two buffers of up to NPL planes (at m = 3 two buffers
-  // of the 5 planes a symmetric codebook needs; one buffer otherwise)
-  static constexpr int AK_SLOTS = MB == 3 ? 10 : 2 * NPL;
-  static constexpr int COL_DS = 0;                      // 2 buffers x (mse, qjl)
-  static constexpr int COL_DPV = 4 * NS;                // 2 buffers
-  static constexpr int BQ_PLANE = 64 * NS;              // e2m1 [NS][128]
+  // tensor memory: A_k planes | D_s (2 buffers x (mse, qjl)) | D_pv (2 buffers)
+  static constexpr int AK_COLS = kTmemCols - 4 * NS - 2 * NPV;
+  static constexpr int COL_DS = AK_COLS;
+  static constexpr int COL_DPV = COL_DS + 4 * NS;
+  static constexpr int LBO_Q = (NS / 8) * 128;          // K-major stride of 16-byte K chunks
+  static constexpr int BQ_PLANE = 128 * NS;             // u8/s8 [128 K] x [NS]
   static constexpr int BQ_BYTES = NPL * BQ_PLANE;
   static constexpr int QBLOCK = BQ_BYTES + kQConstBytes;
   static constexpr int REC = (MB + 1 + VB) * 16 + 20;
@@ -127,20 +116,18 @@ struct Cfg {
   static constexpr int AV_BYTES = 128 * 128;            // [128 channel slots] x [128 tokens]
   static constexpr int BP_BYTES = 128 * NPV;            // [128 tokens] x [NPV]
   static constexpr int SBO_V = 2048;                    // MN-major stride of 16-byte chunks
-  static constexpr int FIXED = AK_SLOTS * kPlaneBytes4 + 2 * AV_BYTES + 2 * BP_BYTES + QBLOCK + 4096;
+  static constexpr int FIXED = 2 * AV_BYTES + 2 * BP_BYTES + QBLOCK + 4096;
   static constexpr int STAGES_FIT = (220 * 1024 - FIXED) / TILE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static_assert(COL_DPV + 2 * NPV <= kColSF, "tensor memory budget");
+  static_assert(NPL * kPlaneCols <= AK_COLS, "tensor memory budget");
   static_assert(STAGES >= 2, "shared memory budget");
   static_assert(TILE_BYTES % 16 == 0, "bulk copy size");
   static_assert(QBLOCK == (int)qblock_bytes_for(MB, G), "query block size");
-  static_assert(2 * L * ((G + 1) / 2) <= NS && (2 * L) % 4 == 0, "score limb loads");
 };
 
 template <class C>
 struct TcSmem {
   alignas(128) uint8_t stage[C::STAGES][C::TILE_BYTES];
-  alignas(128) uint8_t ak[C::AK_SLOTS][kPlaneBytes4];
   alignas(128) uint8_t av[2][C::AV_BYTES];
   alignas(128) uint8_t bp[2][C::BP_BYTES];
   alignas(128) uint8_t bq[C::QBLOCK];  // B_q operand + score constants
@@ -182,29 +169,32 @@ __device__ __forceinline__ uint32_t subset_word(int S, uint32_t b0, uint32_t b1,
   return (__popc(S) & 1) ? x : ~x;
 }
 
-// Four e2m1 operand words of one 32-coordinate spin word w: word k, nibble n
-// is coordinate 4n + k: +1.0 (0x2) where the bit is set, -1.0 (0xA) where not.
-__device__ __forceinline__ uint4 spin_nibbles(uint32_t w) {
-  const uint32_t nw = ~w;
-  return make_uint4(0x22222222u | ((nw << 3) & 0x88888888u), 0x22222222u | ((nw << 2) & 0x88888888u),
-                    0x22222222u | ((nw << 1) & 0x88888888u), 0x22222222u | (nw & 0x88888888u));
+// Eight u8 operand words of one 32-coordinate bit word w: word k, byte i is
+// coordinate 8i + k with weight 2^(k mod 4) (bits 4..7 are taken from w >> 4
+// so no operand byte exceeds 8).
+__device__ __forceinline__ void plane_operands(uint32_t w, uint32_t *o) {
+  const uint32_t w4 = w >> 4;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    o[k] = w & (0x01010101u << k);
+    o[4 + k] = w4 & (0x01010101u << k);
+  }
 }
 
 // Score MMAs of one tile with a compile-time plane count: planes 0..NPM-1
-// accumulate the MSE term, plane NPM (the signs) the QJL term; two K = 64
-// halves per plane.
-template <int NPM, int NS, int BQ_PLANE>
-__device__ __forceinline__ void issue_scores(bool leader, uint64_t da, uint64_t dbq, uint32_t d_mse,
-                                             uint32_t d_qjl, uint32_t id_s, uint32_t sf) {
+// accumulate the MSE term, plane NPM (the signs) the QJL term; four K = 32
+// steps per plane.
+template <int NPM, int LBO_Q, int BQ_PLANE>
+__device__ __forceinline__ void issue_scores(bool leader, uint32_t a_base, uint64_t dbq, uint32_t d_mse,
+                                             uint32_t d_qjl, uint32_t id_s) {
 #pragma unroll
   for (int p = 0; p <= NPM; ++p)
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const uint64_t a_d = da + (uint64_t)((p * kPlaneBytes4 + m * 4096) >> 4);
-      const uint64_t b_d = dbq + (uint64_t)((p * BQ_PLANE + m * 32 * NS) >> 4);
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t b_d = dbq + (uint64_t)((p * BQ_PLANE + kk * 2 * LBO_Q) >> 4);
       const uint32_t d = p < NPM ? d_mse : d_qjl;
-      const uint32_t acc = (p < NPM) ? ((p | m) ? 1u : 0u) : (m ? 1u : 0u);
-      if (leader) mma_mxf4_ss(d, a_d, b_d, id_s, sf, sf, acc);
+      const uint32_t acc = (p < NPM) ? ((p | kk) ? 1u : 0u) : (kk ? 1u : 0u);
+      if (leader) mma_i8_ts(d, a_base + p * kPlaneCols + 8 * kk, b_d, id_s, acc);
     }
 }
 
@@ -240,15 +230,6 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
 #pragma unroll
     for (int x = 0; x < 4; ++x) r[c + x] = t[x];
   }
-}
-
-// sum_l 9^l D_l over one head's limbs (f32 columns)
-template <int L>
-__device__ __forceinline__ float combine_limbs(const uint32_t *d) {
-  float h = __uint_as_float(d[L - 1]);
-#pragma unroll
-  for (int l = L - 2; l >= 0; --l) h = fmaf(h, 9.f, __uint_as_float(d[l]));
-  return h;
 }
 
 template <int MB, int VB, int G>
@@ -334,14 +315,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // It polls both queues (score of tile is, PV of tile ip) with
     // non-blocking tests and issues whichever is ready.
     const bool leader = elect_one();
-    const uint32_t id_s = idesc_mxf4(128, C::NS);
+    const uint32_t id_s = idesc_i8(128, C::NS, false, true, false, false);
     const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
-    const uint32_t sf = tbase + kColSF;
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
     const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
-    const int akb = (2 * npl <= C::AK_SLOTS) ? 2 : 1;
-    const uint64_t dak = smem_desc(S.ak[0], 2048, 128);
-    const uint64_t dbq = smem_desc(S.bq, C::NS * 16, 128);
+    const int akb = (2 * npl * kPlaneCols <= C::AK_COLS) ? 2 : 1;
+    const uint64_t dbq = smem_desc(S.bq, C::LBO_Q, 128);
     const uint64_t dav0 = smem_desc(S.av[0], 128, C::SBO_V), dbp0 = smem_desc(S.bp[0], 128, C::SBO_V);
     int is = 0, ip = 0;
     uint32_t idle = 0;
@@ -355,27 +334,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         tc_fence_after();
         const uint32_t d_mse = tbase + C::COL_DS + (is & 1) * 2 * C::NS;
         const uint32_t d_qjl = d_mse + C::NS;
-        if (nm == C::NSYM) {
+        if (nm == C::NSYM && 2 * (C::NSYM + 1) * kPlaneCols <= C::AK_COLS) {
           // symmetric codebook: plane count and buffer offsets are
           // compile-time, so the descriptors stay in uniform registers
-          const uint64_t da = dak + (uint64_t)(((is & 1) * (C::NSYM + 1) * kPlaneBytes4) >> 4);
-          issue_scores<C::NSYM, C::NS, C::BQ_PLANE>(leader, da, dbq, d_mse, d_qjl, id_s, sf);
+          issue_scores<C::NSYM, C::LBO_Q, C::BQ_PLANE>(
+              leader, tbase + (is & 1) * (C::NSYM + 1) * kPlaneCols, dbq, d_mse, d_qjl, id_s);
         } else {
-        const uint64_t da = dak + (uint64_t)(((akb == 2 ? (is & 1) : 0) * npl * kPlaneBytes4) >> 4);
-        for (int p = 0; p < nm; ++p) {
+          const uint32_t a_base = tbase + (akb == 2 ? (is & 1) : 0) * npl * kPlaneCols;
+          for (int p = 0; p < npl; ++p) {
 #pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const uint64_t a_d = da + (uint64_t)((p * kPlaneBytes4 + m * 4096) >> 4);
-            const uint64_t b_d = dbq + (uint64_t)((p * C::BQ_PLANE + m * 32 * C::NS) >> 4);
-            if (leader) mma_mxf4_ss(d_mse, a_d, b_d, id_s, sf, sf, (p | m) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t b_d = dbq + (uint64_t)((p * C::BQ_PLANE + kk * 2 * C::LBO_Q) >> 4);
+              const uint32_t acc = (p < nm) ? ((p | kk) ? 1u : 0u) : (kk ? 1u : 0u);
+              if (leader) mma_i8_ts(p < nm ? d_mse : d_qjl, a_base + p * kPlaneCols + 8 * kk, b_d, id_s, acc);
+            }
           }
-        }
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const uint64_t a_d = da + (uint64_t)((nm * kPlaneBytes4 + m * 4096) >> 4);
-          const uint64_t b_d = dbq + (uint64_t)((nm * C::BQ_PLANE + m * 32 * C::NS) >> 4);
-          if (leader) mma_mxf4_ss(d_qjl, a_d, b_d, id_s, sf, sf, m ? 1u : 0u);
-        }
         }
         if (leader) mma_commit(&S.s_ready[is & 1]);
         __syncwarp();
@@ -423,24 +396,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     if (is > 0) mbar_wait(&S.s_ready[(is - 1) & 1], ((is - 1) >> 1) & 1);
     if (ip > 0) mbar_wait(&S.pv_done[(ip - 1) & 1], ((ip - 1) >> 1) & 1);
   } else if (warp < 6) {
-    // ---------------- key group: spin planes ------------------------------
+    // ---------------- key group: plane operands -> tensor memory ----------
     const int q4 = warp & 3;
-    const int t = 32 * q4 + lane;  // token slot == operand row
-    {  // unit block scales for every scaled MMA of this CTA
-      uint32_t r[32];
-#pragma unroll
-      for (int x = 0; x < 32; ++x) r[x] = 0x7F7F7F7Fu;
-      tmem_st32(tbase + ((uint32_t)(32 * q4) << 16) + kColSF, r);
-      tmem_st32(tbase + ((uint32_t)(32 * q4) << 16) + kColSF + 32, r);
-      tmem_wait_st();
-    }
+    const int t = 32 * q4 + lane;  // token slot == TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
     const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
-    const int akb = (2 * npl <= C::AK_SLOTS) ? 2 : 1;
+    const int akb = (2 * npl * kPlaneCols <= C::AK_COLS) ? 2 : 1;
     int subs[7];
 #pragma unroll
     for (int p = 0; p < 7; ++p) subs[p] = (qok && p < nm) ? Q.subset[p] : 0;
-    uint8_t *const rowbase = &S.ak[0][0] + (t >> 3) * 128 + (t & 7) * 16;
     for (int i = 0; qok && i < ntile; ++i) {
       const int s = i % C::STAGES;
       if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
@@ -464,17 +429,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[s]);
       const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-      uint8_t *row = rowbase + (akb == 2 ? (i & 1) : 0) * npl * kPlaneBytes4;
+      const uint32_t a_base = tbase + lane_off + (akb == 2 ? (i & 1) : 0) * npl * kPlaneCols;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
         if (p > nm) break;
+        uint32_t r[32];
 #pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          const uint32_t w = (p < nm) ? subset_word(subs[p < 7 ? p : 6], bw[0][wd], bw[1][wd], bw[2][wd]) : sw[wd];
-          *reinterpret_cast<uint4 *>(row + p * kPlaneBytes4 + wd * 2048) = spin_nibbles(w);
-        }
+        for (int wd = 0; wd < 4; ++wd)
+          plane_operands((p < nm) ? subset_word(subs[p < 7 ? p : 6], bw[0][wd], bw[1][wd], bw[2][wd]) : sw[wd],
+                         r + 8 * wd);
+        tmem_st32(a_base + p * kPlaneCols, r);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.ak_ready[i & 1]);
@@ -612,25 +578,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       tc_fence_after();
       float mse[G], qjl[G];
       {
-        // two heads' limbs per load keep the register footprint small
+        // limbs combine as (D0 + 128 D1) 2^-F + (D2 + 128 D3) 2^(14-F)
         const uint32_t base = tbase + lane_off + C::COL_DS + kb * 2 * C::NS;
+        uint32_t d[4 * G];
+        tmem_ld_cols<4 * G>(base, d);
+        tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; g += 2) {
-          constexpr int W = 2 * C::L;
-          uint32_t d[W];  // an odd last head reads padding columns
-          tmem_ld_cols<W>(base + g * C::L, d);
-          tmem_wait_ld();
-          mse[g] = fmaf(Q.inv_m[g], combine_limbs<C::L>(d), Q.cm[g]);
-          if (g + 1 < G) mse[g + 1] = fmaf(Q.inv_m[g + 1], combine_limbs<C::L>(d + C::L), Q.cm[g + 1]);
+        for (int g = 0; g < G; ++g) {
+          const int am = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
+          const int bm = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
+          mse[g] = fmaf(Q.coef_m[g][1], (float)bm, fmaf(Q.coef_m[g][0], (float)am, Q.cm[g]));
         }
+        tmem_ld_cols<4 * G>(base + C::NS, d);
+        tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; g += 2) {
-          constexpr int W = 2 * C::L;
-          uint32_t d[W];  // an odd last head reads padding columns
-          tmem_ld_cols<W>(base + C::NS + g * C::L, d);
-          tmem_wait_ld();
-          qjl[g] = Q.inv_s[g] * combine_limbs<C::L>(d);
-          if (g + 1 < G) qjl[g + 1] = Q.inv_s[g + 1] * combine_limbs<C::L>(d + C::L);
+        for (int g = 0; g < G; ++g) {
+          const int as = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
+          const int bs = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
+          qjl[g] = fmaf(Q.coef_s[g][1], (float)bs, fmaf(Q.coef_s[g][0], (float)as, -Q.csum[g]));
         }
       }
       tc_fence_before();
@@ -760,26 +725,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 
 // ---------------------------------------------------------------------------
 // Query blocks: for every (sequence, KV head) the score MMA's B operand
-// (e2m1, in its shared-memory byte layout) and the score constants, built
-// once per decode call.  A persistent CTA keeps Pi and S in shared memory
-// (rows padded to 129 floats) and rotates the G query heads of each unit:
-// q~ = Pi q, s^ = S q (fp32).  Plane P < n_mse holds a_S q~ for the P-th
+// (s8, in its shared-memory byte layout) and the score constants, built once
+// per decode call.  A persistent CTA keeps Pi and S in shared memory (rows
+// padded to 129 floats) and rotates the G query heads of each unit:
+// q~ = Pi q, s^ = S q (fp32).  Plane P < n_mse holds 2 a_S q~ for the P-th
 // active code-bit subset S (Walsh coefficient a_S of the codebook), the last
-// plane holds s^; each value is rounded to X = round(x 2^F), F per head so
-// |X| <= (9^L - 1) / 2, and written as L balanced base-9 digits.
-// Coordinate j sits at K-chunk j / 32, word j % 4, nibble (j % 32) / 4, the
-// same places the key group's spin words put it.
+// plane holds 2 s^.  K byte kappa of a plane is operand byte i of TMEM column
+// c = kappa / 4, i.e. coordinate j = 32 (c / 8) + 8 i + (c % 8) with weight
+// 2^((c % 8) mod 4), so it holds X = round(x_j 2^(F - weight exponent)) as
+// four signed base-128 limbs; F per head keeps |X| < 2^26.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t e2m1_digit(int d) {
-  const int m = d < 0 ? -d : d;
-  const uint32_t code = m == 0 ? 0u : (m == 1 ? 2u : (m == 2 ? 4u : (m == 3 ? 5u : 6u)));
-  return code | (d < 0 ? 8u : 0u);
-}
-
 template <int MB, int VB, int G>
 __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ DecodeArgs a) {
   using C = Cfg<MB, VB, G>;
-  constexpr int L = C::L;
   constexpr int kPadQ = kD + 1;
   constexpr int NC = 1 << MB;
   extern __shared__ __align__(16) float qsm[];
@@ -813,7 +771,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   }
   int nm = 0, subs[7];
   float wts[7];
-  float wmax = 0.f;
+  float wmax = 0.f, wsum = 0.f;
 #pragma unroll
   for (int S = 1; S < NC; ++S) {
     if (wal[S] != 0.f) {
@@ -821,6 +779,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
       wts[nm] = wal[S];
       ++nm;
       wmax = fmaxf(wmax, fabsf(wal[S]));
+      wsum += wal[S];
     }
   }
   if (nm == 0) {  // degenerate codebook: one all-zero plane
@@ -851,7 +810,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
       for (int g = 0; g < G; ++g) rot[g * 2 * kD + o] = acc[g];
     }
     __syncthreads();
-    // per head: sum q~, max |q~|, max |s^|
+    // per head: sum and max |.| of q~ (warps 0-3) and s^ (warps 4-7)
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int j = tid & (kD - 1);
@@ -863,58 +822,57 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
       }
     }
     __syncthreads();
-    constexpr int emax = xbits_for(L);
     int fm[G], fs[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float sq = 0.f, mq = 0.f, ms = 0.f;
-      for (int wq = 0; wq < 4; ++wq) {        // warps 0-3 hold q~, 4-7 hold s^
+      float sq = 0.f, mq = 0.f, ss = 0.f, ms = 0.f;
+      for (int wq = 0; wq < 4; ++wq) {
         sq += red[(wq * G + g) * 4 + 0];
         mq = fmaxf(mq, red[(wq * G + g) * 4 + 1]);
+        ss += red[((wq + 4) * G + g) * 4 + 0];
         ms = fmaxf(ms, red[((wq + 4) * G + g) * 4 + 1]);
       }
-      const float bm = wmax * mq;
-      fm[g] = bm > 0.f ? emax - 1 - ilogbf(bm) : 0;
-      fs[g] = ms > 0.f ? emax - 1 - ilogbf(ms) : 0;
+      const float bm = 2.f * wmax * mq, bs = 2.f * ms;
+      fm[g] = bm > 0.f ? 25 - ilogbf(bm) : 0;
+      fs[g] = bs > 0.f ? 25 - ilogbf(bs) : 0;
       if (tid == 0) {
-        qc->cm[g] = wal[0] * sq;
-        qc->inv_m[g] = ldexpf(1.f, -fm[g]);
-        qc->inv_s[g] = ldexpf(1.f, -fs[g]);
+        // spins are 2 bit - 1: the -1 halves are constants per head
+        qc->cm[g] = (wal[0] - wsum) * sq;
+        qc->csum[g] = ss;
+        qc->coef_m[g][0] = ldexpf(1.f, -fm[g]);
+        qc->coef_m[g][1] = ldexpf(1.f, 14 - fm[g]);
+        qc->coef_s[g][0] = ldexpf(1.f, -fs[g]);
+        qc->coef_s[g][1] = ldexpf(1.f, 14 - fs[g]);
       }
     }
     if (tid == 0) {
       qc->n_mse = nm;
       for (int p = 0; p < 7; ++p) qc->subset[p] = p < nm ? subs[p] : 0;
     }
-    // one item = one byte position (plane, chunk wd, word k, byte m): the
-    // coordinates 32 wd + 8 m + k (low nibble) and that + 4 (high nibble)
-    for (int item = tid; item < (nm + 1) * 64; item += 256) {
-      const int P = item >> 6, wd = (item >> 4) & 3, k = (item >> 2) & 3, m = item & 3;
-      const int jlo = 32 * wd + 8 * m + k, jhi = jlo + 4;
-      uint8_t *dst0 = blk + P * C::BQ_PLANE + wd * (C::NS * 16) + 4 * k + m;
+    for (int kappa = tid; kappa < (nm + 1) * 128; kappa += 256) {
+      const int P = kappa >> 7, rem = kappa & 127;
+      const int col = rem >> 2, bi = rem & 3;
+      const int wd = col >> 3, k = col & 7, kw = k & 3;
+      const int coord = 32 * wd + 8 * bi + k;
+      uint8_t *dst0 = blk + P * C::BQ_PLANE + (rem >> 4) * C::LBO_Q + (rem & 15);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float xl, xh;
+        float x;
         int F;
         if (P < nm) {
-          xl = wts[P] * rot[g * 2 * kD + jlo];
-          xh = wts[P] * rot[g * 2 * kD + jhi];
+          x = 2.f * wts[P] * rot[g * 2 * kD + coord];
           F = fm[g];
         } else {
-          xl = rot[g * 2 * kD + kD + jlo];
-          xh = rot[g * 2 * kD + kD + jhi];
+          x = 2.f * rot[g * 2 * kD + kD + coord];
           F = fs[g];
         }
-        int Xl = __float2int_rn(ldexpf(xl, F)), Xh = __float2int_rn(ldexpf(xh, F));
+        int X = __float2int_rn(ldexpf(x, F - kw));
 #pragma unroll
-        for (int l = 0; l < L; ++l) {
-          int dl = Xl % 9, dh = Xh % 9;
-          dl = dl > 4 ? dl - 9 : (dl < -4 ? dl + 9 : dl);
-          dh = dh > 4 ? dh - 9 : (dh < -4 ? dh + 9 : dh);
-          Xl = (Xl - dl) / 9;
-          Xh = (Xh - dh) / 9;
-          const int ncol = g * L + l;
-          dst0[(ncol >> 3) * 128 + (ncol & 7) * 16] = (uint8_t)(e2m1_digit(dl) | (e2m1_digit(dh) << 4));
+        for (int l = 0; l < 4; ++l) {
+          const int dgt = (l < 3) ? (((X + 64) & 127) - 64) : X;
+          X = (X - dgt) >> 7;
+          const int n = g * 4 + l;
+          dst0[(n >> 3) * 128 + (n & 7) * 16] = (uint8_t)(int8_t)dgt;
         }
       }
     }
