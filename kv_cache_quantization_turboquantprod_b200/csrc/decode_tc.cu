@@ -98,8 +98,18 @@ struct Cfg {
   static constexpr int NS = score_n(G);                 // score N per accumulator
   static constexpr int NPV = 16 * G;                    // PV N: 4 groups x G heads x 4 bytes
   static constexpr int NPL = max_planes(MB);            // operand planes, upper bound
-  // tensor memory: A_k planes | D_s (2 buffers x (mse, qjl)) | D_pv (2 buffers)
-  static constexpr int AK_COLS = kTmemCols - 4 * NS - 2 * NPV;
+  // tensor memory: A_k planes | D_s (2 buffers x (mse, qjl)) | D_pv (NR buffers).
+  // The P.V ring (A_v, B_p, D_pv) is 3 deep when three A_k buffers of a
+  // symmetric codebook's planes still fit, else 2; A_k takes what is left.
+  static constexpr int NR =
+      (4 * NS + 3 * NPV + 3 * (NSYM + 1) * kPlaneCols <= kTmemCols) ? 3 : 2;
+  static constexpr int AK_COLS = kTmemCols - 4 * NS - NR * NPV;
+  // A_k ring depth for a codebook with npl planes (1 or 2; a third buffer
+  // measured slower: it lets the key group run ahead of the other roles)
+  __host__ __device__ static constexpr int ak_ring(int npl) {
+    return AK_COLS / (npl * kPlaneCols) >= 2 ? 2 : 1;
+  }
+  static constexpr int NAK_SYM = ak_ring(NSYM + 1);
   static constexpr int COL_DS = AK_COLS;
   static constexpr int COL_DPV = COL_DS + 4 * NS;
   static constexpr int LBO_Q = (NS / 8) * 128;          // K-major stride of 16-byte K chunks
@@ -116,7 +126,7 @@ struct Cfg {
   static constexpr int AV_BYTES = 128 * 128;            // [128 channel slots] x [128 tokens]
   static constexpr int BP_BYTES = 128 * NPV;            // [128 tokens] x [NPV]
   static constexpr int SBO_V = 2048;                    // MN-major stride of 16-byte chunks
-  static constexpr int FIXED = 2 * AV_BYTES + 2 * BP_BYTES + QBLOCK + 4096;
+  static constexpr int FIXED = NR * AV_BYTES + NR * BP_BYTES + QBLOCK + 4096;
   static constexpr int STAGES_FIT = (220 * 1024 - FIXED) / TILE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static_assert(NPL * kPlaneCols <= AK_COLS, "tensor memory budget");
@@ -128,19 +138,20 @@ struct Cfg {
 template <class C>
 struct TcSmem {
   alignas(128) uint8_t stage[C::STAGES][C::TILE_BYTES];
-  alignas(128) uint8_t av[2][C::AV_BYTES];
-  alignas(128) uint8_t bp[2][C::BP_BYTES];
+  alignas(128) uint8_t av[C::NR][C::AV_BYTES];
+  alignas(128) uint8_t bp[C::NR][C::BP_BYTES];
   alignas(128) uint8_t bq[C::QBLOCK];  // B_q operand + score constants
   uint64_t full[C::STAGES];
   uint64_t empty[C::STAGES];
-  uint64_t ak_ready[2], s_ready[2], s_free[2], av_ready[2], p_ready[2], pv_done[2], pv_free[2];
+  uint64_t ak_ready[2], s_ready[2], s_free[2];
+  uint64_t av_ready[C::NR], p_ready[C::NR], pv_done[C::NR], pv_free[C::NR];
   uint64_t red_bar[2];
   uint64_t q_full;
   uint32_t tmem_base;
   volatile int abort_flag;
-  uint32_t red[2][2][4][C::G + 1];  // [softmax group][slot][warp][head | value scale]
-  float alpha[2][C::G];
-  float pscale[2];
+  alignas(16) float red[2][2][C::G + 1][4];  // [softmax group][slot][head | value scale][warp]
+  float alpha[C::NR][C::G];
+  float pscale[C::NR];
   float fin_m[2][C::G];
   float lsum[2][4][C::G];
   float zsum[2][4][C::G][4];
@@ -153,7 +164,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // the abort flag and the clock are checked every 16 tries: a waiting
+    // warp then costs its sub-partition almost no issue slots
+#pragma unroll 1
+    for (int r = 0; r < 16; ++r)
+      if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > 2000000000ull) break;
   }
@@ -262,15 +277,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 12);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&S.ak_ready[i], 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.ak_ready[i], 4);
       mbar_init(&S.s_ready[i], 1);
       mbar_init(&S.s_free[i], 4);
+      mbar_init(&S.red_bar[i], 4);
+    }
+    for (int i = 0; i < C::NR; ++i) {
       mbar_init(&S.av_ready[i], 4);
       mbar_init(&S.p_ready[i], 4);
       mbar_init(&S.pv_done[i], 1);
       mbar_init(&S.pv_free[i], 4);
-      mbar_init(&S.red_bar[i], 4);
     }
     mbar_init(&S.q_full, 1);
     S.abort_flag = 0;
@@ -319,7 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
     const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
-    const int akb = (2 * npl * kPlaneCols <= C::AK_COLS) ? 2 : 1;
+    const int akb = C::ak_ring(npl);
     const uint64_t dbq = smem_desc(S.bq, C::LBO_Q, 128);
     const uint64_t dav0 = smem_desc(S.av[0], 128, C::SBO_V), dbp0 = smem_desc(S.bp[0], 128, C::SBO_V);
     int is = 0, ip = 0;
@@ -327,20 +344,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     uint64_t t_idle = 0;
     while (qok && ip < ntile) {
       bool progress = false;
-      bool rs = is < ntile && mbar_test(&S.ak_ready[is & 1], (is >> 1) & 1) &&
+      const int ab = akb == 2 ? (is & 1) : 0;
+      const uint32_t aph = akb == 2 ? ((is >> 1) & 1) : (is & 1);
+      bool rs = is < ntile && mbar_test(&S.ak_ready[ab], aph) &&
                 (is < 2 || mbar_test(&S.s_free[is & 1], ((is - 2) >> 1) & 1));
       rs = __shfl_sync(0xffffffffu, rs, 0);
       if (rs) {
         tc_fence_after();
         const uint32_t d_mse = tbase + C::COL_DS + (is & 1) * 2 * C::NS;
         const uint32_t d_qjl = d_mse + C::NS;
-        if (nm == C::NSYM && 2 * (C::NSYM + 1) * kPlaneCols <= C::AK_COLS) {
+        if (nm == C::NSYM) {
           // symmetric codebook: plane count and buffer offsets are
           // compile-time, so the descriptors stay in uniform registers
           issue_scores<C::NSYM, C::LBO_Q, C::BQ_PLANE>(
-              leader, tbase + (is & 1) * (C::NSYM + 1) * kPlaneCols, dbq, d_mse, d_qjl, id_s);
+              leader, tbase + (C::NAK_SYM == 2 ? (is & 1) : 0) * (C::NSYM + 1) * kPlaneCols, dbq, d_mse,
+              d_qjl, id_s);
         } else {
-          const uint32_t a_base = tbase + (akb == 2 ? (is & 1) : 0) * npl * kPlaneCols;
+          const uint32_t a_base = tbase + ab * npl * kPlaneCols;
           for (int p = 0; p < npl; ++p) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -355,13 +375,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         ++is;
         progress = true;
       }
-      bool rp = ip < is && mbar_test(&S.p_ready[ip & 1], (ip >> 1) & 1) &&
-                mbar_test(&S.av_ready[ip & 1], (ip >> 1) & 1) &&
-                (ip < 2 || mbar_test(&S.pv_free[ip & 1], ((ip - 2) >> 1) & 1));
+      const int rb = ip % C::NR;
+      const uint32_t rph = (ip / C::NR) & 1;
+      bool rp = ip < is && mbar_test(&S.p_ready[rb], rph) && mbar_test(&S.av_ready[rb], rph) &&
+                (ip < C::NR || mbar_test(&S.pv_free[rb], rph ^ 1));
       rp = __shfl_sync(0xffffffffu, rp, 0);
       if (rp) {
         tc_fence_after();
-        const int pb = ip & 1;
+        const int pb = rb;
         const uint32_t d_pv = tbase + C::COL_DPV + pb * C::NPV;
         const uint64_t da = dav0 + (uint64_t)((pb * C::AV_BYTES) >> 4);
         const uint64_t db = dbp0 + (uint64_t)((pb * C::BP_BYTES) >> 4);
@@ -394,28 +415,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     }
     // never leave with an MMA in flight
     if (is > 0) mbar_wait(&S.s_ready[(is - 1) & 1], ((is - 1) >> 1) & 1);
-    if (ip > 0) mbar_wait(&S.pv_done[(ip - 1) & 1], ((ip - 1) >> 1) & 1);
+    if (ip > 0) mbar_wait(&S.pv_done[(ip - 1) % C::NR], ((ip - 1) / C::NR) & 1);
   } else if (warp < 6) {
     // ---------------- key group: plane operands -> tensor memory ----------
+    // The next tile's plane words are fetched while this tile's tensor-memory
+    // stores drain.
     const int q4 = warp & 3;
     const int t = 32 * q4 + lane;  // token slot == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
     const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
-    const int akb = (2 * npl * kPlaneCols <= C::AK_COLS) ? 2 : 1;
+    const int akb = C::ak_ring(npl);
     int subs[7];
 #pragma unroll
     for (int p = 0; p < 7; ++p) subs[p] = (qok && p < nm) ? Q.subset[p] : 0;
-    for (int i = 0; qok && i < ntile; ++i) {
+    uint32_t bw[3][4], sw[4];
+    auto fetch = [&](int i) -> bool {
       const int s = i % C::STAGES;
-      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
-      // the A_k buffer of tile i was last read by the score MMA of tile i - akb
-      if (i >= akb) {
-        const int prev = i - akb;
-        if (!wait_bar(&S.s_ready[prev & 1], (prev >> 1) & 1, &S.abort_flag, status)) break;
-      }
+      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) return false;
       const uint8_t *st = S.stage[s];
-      uint32_t bw[3][4];
 #pragma unroll
       for (int p = 0; p < 3; ++p) {
         if (p < MB) {
@@ -426,10 +444,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         }
       }
       const uint4 sv = *reinterpret_cast<const uint4 *>(st + C::OFF_SIGNS + t * kRowBytes);
+      sw[0] = sv.x; sw[1] = sv.y; sw[2] = sv.z; sw[3] = sv.w;
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[s]);
-      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-      const uint32_t a_base = tbase + lane_off + (akb == 2 ? (i & 1) : 0) * npl * kPlaneCols;
+      return true;
+    };
+    bool ok = qok && fetch(0);
+    for (int i = 0; ok && i < ntile; ++i) {
+      // the A_k buffer of tile i was last read by the score MMA of tile i - akb
+      if (i >= akb) {
+        const int prev = i - akb;
+        if (!wait_bar(&S.s_ready[prev & 1], (prev >> 1) & 1, &S.abort_flag, status)) break;
+      }
+      const int ab = akb == 2 ? (i & 1) : 0;
+      const uint32_t a_base = tbase + lane_off + ab * npl * kPlaneCols;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
         if (p > nm) break;
@@ -440,10 +468,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
                          r + 8 * wd);
         tmem_st32(a_base + p * kPlaneCols, r);
       }
+      const bool next = (i + 1 < ntile) ? fetch(i + 1) : true;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.ak_ready[i & 1]);
+      if (lane == 0) mbar_arrive(&S.ak_ready[ab]);
+      ok = next;
     }
   } else if (warp < 10) {
     // ---------------- value group ------------------------------------------
@@ -457,20 +487,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     float acc[2][G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[0][g] = acc[1][g] = 0.f;
+    // value words of the next tile are fetched before this tile's PV result
+    // is waited for
+    constexpr int NVW = C::PACKED_V ? 8 : 4 * VB;
+    uint32_t vw[NVW];
+    auto fetch = [&](int i) -> bool {
+      const int s = i % C::STAGES;
+      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) return false;
+      const uint8_t *st = S.stage[s];
+      if constexpr (C::PACKED_V) {
+        const uint4 v0 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes);
+        const uint4 v1 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes + 16);
+        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+        vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+      } else {
+#pragma unroll
+        for (int p = 0; p < VB; ++p) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
+          vw[4 * p] = v.x; vw[4 * p + 1] = v.y; vw[4 * p + 2] = v.z; vw[4 * p + 3] = v.w;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[s]);
+      return true;
+    };
+    bool have = ntile > 0 && fetch(0);
     for (int i = 0; i <= ntile; ++i) {
       if (i < ntile) {
-        const int s = i % C::STAGES, vb = i & 1;
-        if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
-        const uint8_t *st = S.stage[s];
+        if (!have) break;
+        const int vb = i % C::NR;
         uint8_t *row = S.av[vb] + (t >> 3) * 128 + (t & 7) * 16;
         if constexpr (C::PACKED_V) {
           // packed row: word w holds channels 16w .. 16w+15; mask m keeps
           // channel 16w + 4i + m in byte i as code * 4^m (M slot 16w + 4m + i)
-          const uint4 v0 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes);
-          const uint4 v1 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes + 16);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.empty[s]);
-          const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
           for (int w = 0; w < 8; ++w)
             *reinterpret_cast<uint4 *>(row + w * C::SBO_V) =
@@ -479,14 +528,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         } else {
           // bit-planes: u32 x of chunk m16 holds, in byte i, the code of
           // channel 32 (m16 / 2) + 8 i + 4 (m16 % 2) + x (M slot 16 m16 + 4 x + i)
-          uint32_t vp[VB][4];
-#pragma unroll
-          for (int p = 0; p < VB; ++p) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
-            vp[p][0] = v.x; vp[p][1] = v.y; vp[p][2] = v.z; vp[p][3] = v.w;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.empty[s]);
 #pragma unroll
           for (int m16 = 0; m16 < 8; ++m16) {
             uint32_t o[4];
@@ -495,7 +536,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
               const int k = 4 * (m16 & 1) + x;
               uint32_t c = 0;
 #pragma unroll
-              for (int p = 0; p < VB; ++p) c |= ((vp[p][m16 >> 1] >> k) & 0x01010101u) << p;
+              for (int p = 0; p < VB; ++p) c |= ((vw[4 * p + (m16 >> 1)] >> k) & 0x01010101u) << p;
               o[x] = c;
             }
             *reinterpret_cast<uint4 *>(row + m16 * C::SBO_V) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -504,11 +545,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.av_ready[vb]);
+        have = (i + 1 < ntile) ? fetch(i + 1) : true;
       }
       if (i >= 1) {
-        const int jt = i - 1, pb = jt & 1;
-        if (!wait_bar(&S.pv_done[pb], (jt >> 1) & 1, &S.abort_flag, status)) break;
-        if (!wait_bar(&S.p_ready[pb], (jt >> 1) & 1, &S.abort_flag, status)) break;
+        const int jt = i - 1, pb = jt % C::NR, sg = jt & 1;
+        const uint32_t rph = (jt / C::NR) & 1;
+        if (!wait_bar(&S.pv_done[pb], rph, &S.abort_flag, status)) break;
+        if (!wait_bar(&S.p_ready[pb], rph, &S.abort_flag, status)) break;
         tc_fence_after();
         uint32_t d[4 * G];
         tmem_ld_cols<4 * G>(tbase + lane_off + C::COL_DPV + pb * C::NPV + q4 * 4 * G, d);
@@ -525,7 +568,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           const float v = fmaf(16777216.f, (float)d[4 * g + 3],
                                fmaf(65536.f, (float)d[4 * g + 2],
                                     fmaf(256.f, (float)d[4 * g + 1], (float)d[4 * g])));
-          acc[pb][g] = fmaf(acc[pb][g], alpha[g], v * sc);
+          acc[sg][g] = fmaf(acc[sg][g], alpha[g], v * sc);
         }
       }
     }
@@ -571,8 +614,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       for (int gg = 0; gg < 4; ++gg) zs[g][gg] = 0.f;
     }
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
+    // score constants of this (sequence, KV head): in registers up to GQA 4
+    constexpr bool kRegConst = G <= 4;
+    float qcm[G], qcs[G], qfm[G], qfs[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (kRegConst) {
+        qcm[g] = Q.cm[g];
+        qcs[g] = -Q.csum[g];
+        qfm[g] = Q.coef_m[g][0];
+        qfs[g] = Q.coef_s[g][0];
+      }
+    }
     for (int jt = grp; qok && jt < ntile; jt += 2) {
-      const int kb = grp, pb = grp, s = jt % C::STAGES, n = jt >> 1;
+      const int kb = grp, pb = jt % C::NR, s = jt % C::STAGES, n = jt >> 1;
       if (!wait_bar(&S.full[s], (jt / C::STAGES) & 1, &S.abort_flag, status)) break;
       if (!wait_bar(&S.s_ready[kb], n & 1, &S.abort_flag, status)) break;
       tc_fence_after();
@@ -587,7 +642,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         for (int g = 0; g < G; ++g) {
           const int am = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
           const int bm = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
-          mse[g] = fmaf(Q.coef_m[g][1], (float)bm, fmaf(Q.coef_m[g][0], (float)am, Q.cm[g]));
+          const float fm = kRegConst ? qfm[g] : Q.coef_m[g][0];
+          mse[g] = fmaf(fm * 16384.f, (float)bm, fmaf(fm, (float)am, kRegConst ? qcm[g] : Q.cm[g]));
         }
         tmem_ld_cols<4 * G>(base + C::NS, d);
         tmem_wait_ld();
@@ -595,7 +651,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         for (int g = 0; g < G; ++g) {
           const int as = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
           const int bs = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
-          qjl[g] = fmaf(Q.coef_s[g][1], (float)bs, fmaf(Q.coef_s[g][0], (float)as, -Q.csum[g]));
+          const float fs = kRegConst ? qfs[g] : Q.coef_s[g][0];
+          qjl[g] = fmaf(fs * 16384.f, (float)bs, fmaf(fs, (float)as, kRegConst ? qcs[g] : -Q.csum[g]));
         }
       }
       tc_fence_before();
@@ -626,15 +683,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         lg[g] = valid ? score * scale2 : -INFINITY;
       }
       // tile maxima (logits per head, value scale) over the 128 tokens
-      uint32_t(&red)[4][G + 1] = S.red[grp][n & 1];
+      float(&red)[G + 1][4] = S.red[grp][n & 1];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const uint32_t u = __reduce_max_sync(0xffffffffu, float_to_ordered(lg[g]));
-        if (lane == 0) red[q4][g] = u;
+        const float u = redux_max_f32(lg[g]);
+        if (lane == 0) red[g][q4] = u;
       }
       {
-        const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(msc));
-        if (lane == 0) red[q4][G] = u;
+        const float u = redux_max_f32(msc);
+        if (lane == 0) red[G][q4] = u;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.red_bar[grp]);
@@ -643,18 +700,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       bool changed = false;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        uint32_t u = red[0][g];
-#pragma unroll
-        for (int wq = 1; wq < 4; ++wq) u = max(u, red[wq][g]);
-        const float mnew = fmaxf(mrun[g], ordered_to_float(u));
+        const float4 r4 = *reinterpret_cast<const float4 *>(red[g]);
+        const float mnew = fmaxf(mrun[g], fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
         alpha[g] = exp2f(mrun[g] - mnew);
         changed |= (mnew != mrun[g]);
         mrun[g] = mnew;
       }
-      uint32_t us = red[0][G];
-#pragma unroll
-      for (int wq = 1; wq < 4; ++wq) us = max(us, red[wq][G]);
-      const float mscale = __uint_as_float(us);
+      const float4 rs = *reinterpret_cast<const float4 *>(red[G]);
+      const float mscale = fmaxf(fmaxf(rs.x, rs.y), fmaxf(rs.z, rs.w));
       if (changed) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -666,6 +719,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       // p * scale <= mscale < 2^(e+1); fixed point with values < 2^21
       const int F = mscale > 0.f ? 20 - ilog2f(mscale) : 0;
       const float fscale = mscale > 0.f ? exp2i(F) : 0.f;
+      float vscf[4];
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) vscf[gg] = vsc[gg] * fscale;  // exact: power-of-two scale
       float p[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -674,8 +730,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
         for (int gg = 0; gg < 4; ++gg) zs[g][gg] = fmaf(p[g], vze[gg], zs[g][gg]);
       }
-      // P' operand of tile jt: wait until the PV of tile jt-2 has been read
-      if (jt >= 2 && !wait_bar(&S.pv_free[pb], (n - 1) & 1, &S.abort_flag, status)) break;
+      // P' operand of tile jt: wait until the PV of tile jt - NR has been read
+      if (jt >= C::NR && !wait_bar(&S.pv_free[pb], ((jt / C::NR) & 1) ^ 1, &S.abort_flag, status)) break;
       // column n = group * 4G + head * 4 + byte: one u32 per (group, head),
       // 22-bit fixed point p * scale * 2^F
       uint8_t *row = S.bp[pb] + (t >> 3) * 128 + (t & 7) * 16;
@@ -685,7 +741,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
-          w4[x] = __float_as_uint(fmaf(p[g] * vsc[gg], fscale, 12582912.f)) & 0x3FFFFFu;
+          w4[x] = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
         }
         *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }

@@ -94,7 +94,10 @@ __device__ __forceinline__ bool qwait(uint64_t *bar, uint32_t parity, volatile i
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // abort flag and clock every 16 tries: a waiting warp costs few issue slots
+#pragma unroll 1
+    for (int r = 0; r < 16; ++r)
+      if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > 2000000000ull) break;
   }

@@ -215,6 +215,13 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Warp-wide maximum of a float (sm_100a floating-point redux).
+__device__ __forceinline__ float redux_max_f32(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Order-preserving map of floats to unsigned (for integer max reductions).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
   const uint32_t b = __float_as_uint(f);
