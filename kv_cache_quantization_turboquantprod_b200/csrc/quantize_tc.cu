@@ -62,6 +62,7 @@ struct QtSmem {
   float cent[8];
   float bnd[8];                  // ascending, padded with +inf
   uint32_t cpair[2][64];         // packed fp16 (hi, lo) parts of c[i0], c[i1] x 2^16, index i0 | i1 << 3
+  int sym;                       // boundaries exactly antisymmetric (b[i] == -b[nb - 1 - i])
   uint64_t a1_full[2], a1_free[2], d1_full[2], a2_full[2], d2_full[2], a3_full[2], d3_full[2],
       d_free[2];
   uint32_t tmem_base;
@@ -157,6 +158,11 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   }
   if (tid < ncent) S.cent[tid] = a.centroids[tid];
   if (tid < 8) S.bnd[tid] = tid < ncent - 1 ? a.boundaries[tid] : INFINITY;
+  if (tid == 0) {
+    int sym = 1;
+    for (int i = 0; i < ncent - 1; ++i) sym &= (a.boundaries[i] == -a.boundaries[ncent - 2 - i]) ? 1 : 0;
+    S.sym = sym;
+  }
   if (tid < 64) {
     const int i0 = tid & 7, i1 = tid >> 3;
     float h0 = 0.f, l0 = 0.f, h1 = 0.f, l1 = 0.f;
@@ -385,16 +391,22 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           uint32_t codes[4] = {0u, 0u, 0u, 0u};  // 4 bits per element, 8 per word
           uint32_t fix = 0u;
           if (sc32 != 0.f) {
+            const int ilev = (int)vlevels;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[c]);
+              const uint32_t *w2v = reinterpret_cast<const uint32_t *>(&vr[c]);
 #pragma unroll
               for (int e2 = 0; e2 < 8; ++e2) {
-                const float2 f = __bfloat1622float2(p2[e2 >> 1]);
-                const float tq = __fsub_rn((e2 & 1) ? f.y : f.x, z32) * rsc;
-                const float fr = tq - floorf(tq);
-                fix |= (fabsf(fr - 0.5f) < 1e-5f ? 1u : 0u) << (8 * c + e2);
-                codes[c] |= (uint32_t)fminf(fmaxf(rintf(tq), 0.f), vlevels) << (4 * e2);
+                const uint32_t wb = w2v[e2 >> 1];  // two bf16
+                const float x = __uint_as_float((e2 & 1) ? (wb & 0xFFFF0000u) : (wb << 16));
+                // t stays within [-1, levels + 1] (fp16 zero/scale rounding);
+                // rint by the 1.5 * 2^23 magic add, integer clamp
+                const float tq = fminf(fmaxf(__fsub_rn(x, z32) * rsc, -1.f), vlevels + 1.f);
+                const float r = tq + 12582912.f;
+                const float rq = r - 12582912.f;
+                fix |= (fabsf(tq - rq) > 0.5f - 1e-5f ? 1u : 0u) << (8 * c + e2);
+                const int code = min(max(__float_as_int(r) - 0x4B400000, 0), ilev);
+                codes[c] |= (uint32_t)code << (4 * e2);
               }
             }
             const __nv_bfloat16 *vrow = reinterpret_cast<const __nv_bfloat16 *>(a.v) +
@@ -443,6 +455,14 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     const uint32_t dcol = tbase + lane_off + g * 256, acol = dcol + 128;
     const uint8_t *a1 = S.a1[g];
     constexpr int NC = 1 << MB;
+    // upper half of a symmetric codebook's boundaries, for the compare-count
+    // bucketize: idx = NC/2 + #{ub < |y|} (y > 0) or NC/2 - 1 - #{ub < |y|}
+    // (y <= 0), equal to #{b < y} except at exact ties (inside the band)
+    constexpr int NU = NC / 2 - 1 > 0 ? NC / 2 - 1 : 1;
+    float ub[NU];
+#pragma unroll
+    for (int k = 0; k < NU; ++k) ub[k] = (k < NC / 2 - 1) ? S.bnd[NC / 2 + k] : INFINITY;
+    const bool sym = S.sym != 0;
     for (int i = g; i < nlocal; i += 2) {
       const uint32_t ph = (i >> 1) & 1;
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
@@ -476,9 +496,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             const float y = __uint_as_float(d[e + x]) * inv1;
-            int idx = 0;  // #{boundaries < y}, binary search
+            int idx;  // #{boundaries < y}
+            if (sym) {
+              const float ay = fabsf(y);
+              int cnt = 0;
 #pragma unroll
-            for (int step = NC / 2; step >= 1; step >>= 1) idx += (S.bnd[idx + step - 1] < y) ? step : 0;
+              for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
+              idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
+            } else {  // binary search
+              idx = 0;
+#pragma unroll
+              for (int step = NC / 2; step >= 1; step >>= 1) idx += (S.bnd[idx + step - 1] < y) ? step : 0;
+            }
             idx = zero ? 0 : idx;
 #pragma unroll
             for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
