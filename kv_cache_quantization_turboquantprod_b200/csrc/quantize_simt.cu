@@ -19,11 +19,13 @@ namespace tq {
 
 namespace {
 
-constexpr int kNV = 16;              // vectors per pass
+// vectors per pass: 16 for large appends, 2 for small ones (decode steps),
+// so a 1-token append over B x H_kv heads still spreads over many SMs
 constexpr int kThreads = 256;
 constexpr int kPad = kD + 1;         // padded row stride of Pi / S in smem
 constexpr int kMatFloats = kD * kPad;
 
+template <int kNV>
 struct QuantSmem {
   float pi[kMatFloats];
   float s[kMatFloats];
@@ -49,10 +51,11 @@ __device__ __forceinline__ void vec_coords(const AppendArgs &a, long long id, in
   valid = t < a.nnew[b];
 }
 
+template <int kNV>
 __global__ void __launch_bounds__(kThreads, 1)
 quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  QuantSmem &S = *reinterpret_cast<QuantSmem *>(smem_raw);
+  QuantSmem<kNV> &S = *reinterpret_cast<QuantSmem<kNV> *>(smem_raw);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -259,21 +262,25 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
   }
 }
 
-}  // namespace
-
-size_t quantize_simt_smem_bytes() { return sizeof(QuantSmem); }
-
-cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream) {
-  const size_t smem = sizeof(QuantSmem);
-  cudaError_t e = cudaFuncSetAttribute(quantize_append_simt_kernel,
+template <int kNV>
+cudaError_t launch_simt_nv(const AppendArgs &a, int num_sms, cudaStream_t stream) {
+  const size_t smem = sizeof(QuantSmem<kNV>);
+  cudaError_t e = cudaFuncSetAttribute(quantize_append_simt_kernel<kNV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long total = (long long)a.batch * a.T * a.h_kv;
   const long long nchunks = (total + kNV - 1) / kNV;
   const int grid = (int)std::min<long long>(nchunks, (long long)num_sms);
   if (grid <= 0) return cudaSuccess;
-  quantize_append_simt_kernel<<<grid, kThreads, smem, stream>>>(a);
+  quantize_append_simt_kernel<kNV><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream) {
+  const long long total = (long long)a.batch * a.T * a.h_kv;
+  return total <= 2LL * num_sms ? launch_simt_nv<2>(a, num_sms, stream) : launch_simt_nv<16>(a, num_sms, stream);
 }
 
 }  // namespace tq
