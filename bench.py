@@ -329,9 +329,38 @@ def run_ours(args, rank, world, device):
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
+    if world == 1:
+        line["window"] = bench_window(layer, cache, q, len_after, max_len, out, ws, wl, device,
+                                      dec_bytes_all, dec_ms)
     if args.quantize and world == 1:
         line["quantize"] = bench_quantize(args, device)
     return line
+
+
+def bench_window(layer, cache, q, len_dev, max_len, out, ws, wl, device, dec_bytes, dec_ms):
+    """The same decode call with a full 128-token exact window (bf16 K and V)
+    per sequence merged into the softmax: time and the window's cost."""
+    B, HKV, D = wl.batch, wl.h_kv, wl.d
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4321)
+    wk = torch.randn((B, HKV, 128, D), generator=gen, device=device).to(torch.bfloat16)
+    wv = torch.randn((B, HKV, 128, D), generator=gen, device=device).to(torch.bfloat16)
+    wlen = torch.full((B,), 128, dtype=torch.int32, device=device)
+    for _ in range(3):
+        tq.tq_decode_attention_window(layer, cache, q, len_dev, max_len, wk, wv, wlen, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 20
+    e0.record()
+    for _ in range(n):
+        tq.tq_decode_attention_window(layer, cache, q, len_dev, max_len, wk, wv, wlen, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    win_bytes = B * HKV * 128 * D * 2 * 2
+    return {"win_cap": 128, "decode_ms": ms, "decode_ms_without_window": dec_ms,
+            "gbs": (dec_bytes + win_bytes) / (ms / 1e3) / 1e9,
+            "window_bytes": win_bytes}
 
 
 def bench_quantize(args, device):

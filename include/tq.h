@@ -208,6 +208,33 @@ TQ_API tq_status tq_decode_attention(const tq_params *p, const tq_cache *c,
                               float softmax_scale, float *out, void *workspace,
                               size_t workspace_bytes, tq_stream_t stream);
 
+/*
+ * tq_decode_attention_window -- tq_decode_attention over the compressed
+ * cache plus a window of recent tokens kept exactly, merged into the same
+ * softmax ("turboquant/audit_claims.py", AUDIT 1: the store keeps a ring
+ * buffer of the 128 most recent tokens in bf16 next to the compressed
+ * history).  Window tokens contribute exact scores q.k * softmax_scale and
+ * exact values; the result equals one softmax over both sets.
+ *
+ *   win_k, win_v   device, [batch][h_kv][win_cap][d], win_dtype (F32 or
+ *                  BF16), 16-byte aligned; slot order is free (attention
+ *                  does not depend on it)
+ *   win_len_dev    device, [batch] int32: valid window slots 0..win_cap of
+ *                  each sequence (values outside are clamped)
+ *   win_cap        host, 1 <= win_cap <= 128
+ * The other arguments are tq_decode_attention's, with the same workspace
+ * size.  A sequence with no compressed tokens and no window tokens gets a
+ * zero output row.
+ */
+TQ_API tq_status tq_decode_attention_window(const tq_params *p, const tq_cache *c,
+                                     const void *q, tq_dtype q_dtype, int h_q,
+                                     const int32_t *len_dev, int max_len,
+                                     const void *win_k, const void *win_v,
+                                     tq_dtype win_dtype, const int32_t *win_len_dev,
+                                     int win_cap, float softmax_scale, float *out,
+                                     void *workspace, size_t workspace_bytes,
+                                     tq_stream_t stream);
+
 /* Size of the fixed device scratch tq_decode_attention_noalloc uses. */
 #define TQ_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 

@@ -92,6 +92,8 @@ extern "C" tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_ca
   a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q; a.ntiles = c->capacity / tq::kTile;
   a.max_len = max_len; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
   a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
+  a.part_stride = P.nsplit;
+  a.win_k = nullptr; a.win_v = nullptr; a.win_dtype = TQ_BF16; a.win_len = nullptr; a.win_cap = 0;
   a.num_sms = sms;
   tq::bind_workspace(a, P, scratch);
   a.out = out;

@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
         A = fmaf(sm_acc[w][g][j], f, A);
       }
     }
-    float *dst = a.part + (((size_t)b * a.h_q + h * G + g) * a.nsplit + s) * (kD + 2);
+    float *dst = a.part + (((size_t)b * a.h_q + h * G + g) * a.part_stride + s) * (kD + 2);
     dst[j] = A;
     if (j == 0) { dst[kD] = M; dst[kD + 1] = Lsum; }
   }
@@ -174,18 +174,106 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
 __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
   const int bh = blockIdx.x;
   const int j = threadIdx.x;
-  const float *src = a.part + (size_t)bh * a.nsplit * (kD + 2);
+  const float *src = a.part + (size_t)bh * a.part_stride * (kD + 2);
   float M = -INFINITY;
-  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, src[s * (kD + 2) + kD]);
+  for (int s = 0; s < a.part_stride; ++s) M = fmaxf(M, src[s * (kD + 2) + kD]);
   float num = 0.f, den = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < a.nsplit; ++s) {
+    for (int s = 0; s < a.part_stride; ++s) {
       const float f = exp2f(src[s * (kD + 2) + kD] - M);
       num = fmaf(src[s * (kD + 2) + j], f, num);
       den = fmaf(src[s * (kD + 2) + kD + 1], f, den);
     }
   }
   a.out[(size_t)bh * kD + j] = den > 0.f ? num / den : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// Recent-token window: exact attention of the G query heads of (b, h_kv)
+// over win_len[b] window tokens, written as partial slot nsplit (acc, m in
+// log2 units, l), so the combine merges it with the compressed splits.
+// One CTA per (h_kv, b); thread t scores window slot t, thread j then sums
+// dimension j over the slots.
+// ---------------------------------------------------------------------------
+template <int G>
+__global__ void __launch_bounds__(128) window_kernel(DecodeArgs a) {
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  __shared__ float qs[G][kD];
+  __shared__ float ps[G][kTile];
+  __shared__ float red[G][4];
+  int wl = a.win_len[b];
+  wl = wl < 0 ? 0 : (wl > a.win_cap ? a.win_cap : wl);
+  for (int i = t; i < G * kD; i += 128)
+    qs[i / kD][i % kD] = load_elem(a.q, a.q_dtype, ((size_t)b * a.h_q + (size_t)h * G) * kD + i);
+  __syncthreads();
+  const size_t row0 = ((size_t)b * a.h_kv + h) * (size_t)a.win_cap;
+  const float scale2 = a.softmax_scale * 1.4426950408889634f;
+  float lg[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) lg[g] = -INFINITY;
+  if (t < wl) {
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.f;
+    for (int j = 0; j < kD; ++j) {
+      const float k = load_elem(a.win_k, a.win_dtype, (row0 + t) * kD + j);
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = fmaf(qs[g][j], k, acc[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) lg[g] = acc[g] * scale2;
+  }
+  const int warp = t >> 5, lane = t & 31;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float m = warp_max(lg[g]);
+    if (lane == 0) red[g][warp] = m;
+  }
+  __syncthreads();
+  float mx[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    mx[g] = fmaxf(fmaxf(red[g][0], red[g][1]), fmaxf(red[g][2], red[g][3]));
+    ps[g][t] = (t < wl) ? exp2f(lg[g] - mx[g]) : 0.f;
+  }
+  __syncthreads();
+  // thread t now sums dimension t over the window slots
+  float num[G], den[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) num[g] = den[g] = 0.f;
+  for (int i = 0; i < wl; ++i) {
+    const float v = load_elem(a.win_v, a.win_dtype, (row0 + i) * kD + t);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      num[g] = fmaf(ps[g][i], v, num[g]);
+      den[g] += ps[g][i];
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float *dst = a.part + (((size_t)b * a.h_q + (size_t)h * G + g) * a.part_stride + a.nsplit) * (kD + 2);
+    dst[t] = num[g];
+    if (t == 0) {
+      dst[kD] = wl > 0 ? mx[g] : -INFINITY;
+      dst[kD + 1] = den[g];
+    }
+  }
+}
+
+cudaError_t launch_window(const DecodeArgs &a, cudaStream_t stream) {
+  const dim3 grid(a.h_kv, a.batch);
+  switch (a.h_q / a.h_kv) {
+    case 1: window_kernel<1><<<grid, 128, 0, stream>>>(a); break;
+    case 2: window_kernel<2><<<grid, 128, 0, stream>>>(a); break;
+    case 3: window_kernel<3><<<grid, 128, 0, stream>>>(a); break;
+    case 4: window_kernel<4><<<grid, 128, 0, stream>>>(a); break;
+    case 5: window_kernel<5><<<grid, 128, 0, stream>>>(a); break;
+    case 6: window_kernel<6><<<grid, 128, 0, stream>>>(a); break;
+    case 7: window_kernel<7><<<grid, 128, 0, stream>>>(a); break;
+    case 8: window_kernel<8><<<grid, 128, 0, stream>>>(a); break;
+    default: return cudaErrorNotSupported;
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -205,7 +293,7 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   P.status_bytes = 256;
   P.qrot_bytes = al((size_t)batch * h_q * 2 * kD * sizeof(float));
-  P.part_bytes = al((size_t)batch * h_q * nsplit * (kD + 2) * sizeof(float));
+  P.part_bytes = al((size_t)batch * h_q * (nsplit + 1) * (kD + 2) * sizeof(float));
   const int G = h_q / h_kv;
   P.qblock_bytes = decode_tc_supported(key_bits, value_bits, G) ? decode_tc_qblock_bytes(key_bits, G) : 0;
   P.total_bytes = P.status_bytes + P.qrot_bytes + P.part_bytes + al((size_t)batch * h_kv * P.qblock_bytes);
@@ -229,6 +317,10 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = launch_decode_tc(a, stream);
   if (e != cudaSuccess) return e;
+  if (a.win_k) {
+    e = launch_window(a, stream);
+    if (e != cudaSuccess) return e;
+  }
   combine_kernel<<<bhq, 128, 0, stream>>>(a);
   return cudaGetLastError();
 }
@@ -242,6 +334,10 @@ cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream) {
   decode_splitk_simt_kernel<<<grid, 128, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.win_k) {
+    e = launch_window(a, stream);
+    if (e != cudaSuccess) return e;
+  }
   combine_kernel<<<bhq, 128, 0, stream>>>(a);
   return cudaGetLastError();
 }

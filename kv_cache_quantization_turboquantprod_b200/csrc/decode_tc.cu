@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   const int t_end = min(len, (split + 1) * a.tiles_per_split * kTile);
   const int ntile = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
   auto part_row = [&](int g) {
-    return a.part + (((size_t)b * a.h_q + (size_t)h * G + g) * a.nsplit + split) * (kD + 2);
+    return a.part + (((size_t)b * a.h_q + (size_t)h * G + g) * a.part_stride + split) * (kD + 2);
   };
   if (ntile == 0) {  // empty split: neutral partial state
     for (int i = tid; i < G * (kD + 2); i += kTcThreads) {

@@ -167,10 +167,15 @@ size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, 
   return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits).total_bytes;
 }
 
-tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void *q,
-                              tq_dtype q_dtype, int h_q, const int32_t *len_dev, int max_len,
-                              float softmax_scale, float *out, void *workspace,
-                              size_t workspace_bytes, tq_stream_t stream) {
+namespace {
+
+// Shared by tq_decode_attention and tq_decode_attention_window (win_k null:
+// no window).
+tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq_dtype q_dtype,
+                        int h_q, const int32_t *len_dev, int max_len, const void *win_k,
+                        const void *win_v, tq_dtype win_dtype, const int32_t *win_len_dev,
+                        int win_cap, float softmax_scale, float *out, void *workspace,
+                        size_t workspace_bytes, tq_stream_t stream) {
   tq_status st = check_params(p);
   if (st != TQ_OK) return st;
   if ((st = check_cache(c)) != TQ_OK) return st;
@@ -181,6 +186,12 @@ tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void 
   if (max_len < 0 || max_len > c->capacity) return TQ_ERR_INVALID_ARGUMENT;
   if (!std::isfinite(softmax_scale)) return TQ_ERR_INVALID_ARGUMENT;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(len_dev, 4)) return TQ_ERR_INVALID_ARGUMENT;
+  if (win_k) {
+    if (!dtype_ok(win_dtype)) return TQ_ERR_UNSUPPORTED;
+    if (!win_v || !win_len_dev || win_cap < 1 || win_cap > kTile) return TQ_ERR_INVALID_ARGUMENT;
+    if (!aligned(win_k, 16) || !aligned(win_v, 16) || !aligned(win_len_dev, 4))
+      return TQ_ERR_INVALID_ARGUMENT;
+  }
   if (!workspace || !aligned(workspace, 256)) return TQ_ERR_WORKSPACE;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
@@ -192,11 +203,35 @@ tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void 
   a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q; a.ntiles = c->capacity / kTile;
   a.max_len = max_len; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
   a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
+  a.part_stride = win_k ? P.nsplit + 1 : P.nsplit;
+  a.win_k = win_k; a.win_v = win_v; a.win_dtype = win_dtype; a.win_len = win_len_dev;
+  a.win_cap = win_cap;
   a.num_sms = sms;
   tq::bind_workspace(a, P, workspace);
   a.out = out;
   if (tq::launch_decode(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
+}
+
+}  // namespace
+
+tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void *q,
+                              tq_dtype q_dtype, int h_q, const int32_t *len_dev, int max_len,
+                              float softmax_scale, float *out, void *workspace,
+                              size_t workspace_bytes, tq_stream_t stream) {
+  return decode_common(p, c, q, q_dtype, h_q, len_dev, max_len, nullptr, nullptr, TQ_BF16, nullptr, 0,
+                       softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+tq_status tq_decode_attention_window(const tq_params *p, const tq_cache *c, const void *q,
+                                     tq_dtype q_dtype, int h_q, const int32_t *len_dev,
+                                     int max_len, const void *win_k, const void *win_v,
+                                     tq_dtype win_dtype, const int32_t *win_len_dev, int win_cap,
+                                     float softmax_scale, float *out, void *workspace,
+                                     size_t workspace_bytes, tq_stream_t stream) {
+  if (!win_k) return TQ_ERR_INVALID_ARGUMENT;
+  return decode_common(p, c, q, q_dtype, h_q, len_dev, max_len, win_k, win_v, win_dtype, win_len_dev,
+                       win_cap, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
 tq_status tq_dequantize(const tq_params *p, const tq_cache *c, int b, int start, int count,

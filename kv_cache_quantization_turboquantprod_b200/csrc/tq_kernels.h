@@ -36,7 +36,8 @@ struct DecodePlan {
   int tiles_per_split; // 128-token tiles per split
   size_t status_bytes; // status word (nonzero: a kernel gave up on a bounded wait)
   size_t qrot_bytes;   // [B][H_q][2][d] fp32
-  size_t part_bytes;   // [B][H_q][nsplit][d + 2] fp32 (acc, m, l)
+  size_t part_bytes;   // [B][H_q][nsplit + 1][d + 2] fp32 (acc, m, l); the extra slot
+                       // holds the recent-token window's partial state
   size_t qblock_bytes; // per (b, h_kv) query block of the tensor-core kernel (0: SIMT path)
   size_t total_bytes;
 };
@@ -51,9 +52,15 @@ struct DecodeArgs {
   int key_bits, value_bits;
   float softmax_scale;
   int nsplit, tiles_per_split;
+  int part_stride;  // partial slots per (b, hq): nsplit, or nsplit + 1 with a window
+  // recent-token window kept exactly (win_k == nullptr: none)
+  const void *win_k, *win_v;
+  tq_dtype win_dtype;
+  const int32_t *win_len;
+  int win_cap;
   int *status;   // workspace: status word, cleared by qprep
   float *qrot;   // workspace: [B][H_q][2][d]
-  float *part;   // workspace: [B][H_q][nsplit][d+2]
+  float *part;   // workspace: [B][H_q][part_stride][d+2]
   uint8_t *qblocks;  // workspace: [B][H_kv] query blocks (tensor-core path)
   int num_sms;
   float *out;    // [B][H_q][d]

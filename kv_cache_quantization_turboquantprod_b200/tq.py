@@ -28,7 +28,7 @@ MAX_BATCH = 1024
 # Every function include/tq.h declares.
 EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_bytes",
            "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
-           "tq_dequantize", "tq_decode_attention_noalloc")
+           "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window")
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -82,6 +82,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_decode_attention.argtypes = [P, C, vp, ci, ci, vp, ci, ctypes.c_float, vp, vp, sz, vp]
     lib.tq_decode_attention_noalloc.restype = ci
     lib.tq_decode_attention_noalloc.argtypes = [P, C, vp, ci, ci, vp, ci, ctypes.c_float, vp, vp]
+    lib.tq_decode_attention_window.restype = ci
+    lib.tq_decode_attention_window.argtypes = [P, C, vp, ci, ci, vp, ci, vp, vp, ci, vp, ci,
+                                               ctypes.c_float, vp, vp, sz, vp]
     lib.tq_dequantize.restype = ci
     lib.tq_dequantize.argtypes = [P, C, ci, ci, ci, vp, vp, vp]
     if path is None:
@@ -215,6 +218,32 @@ def tq_decode_attention(layer: Layer, cache: CompressedCache, q: torch.Tensor,
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream))
     _check("tq_decode_attention", st)
+
+
+def tq_decode_attention_window(layer: Layer, cache: CompressedCache, q: torch.Tensor,
+                               len_dev: torch.Tensor, max_len: int, win_k: torch.Tensor,
+                               win_v: torch.Tensor, win_len_dev: torch.Tensor, out: torch.Tensor,
+                               workspace: torch.Tensor, softmax_scale: float | None = None,
+                               stream=None) -> None:
+    """Decode over the compressed cache plus a window of recent tokens kept
+    exactly: win_k, win_v [B, H_kv, win_cap, d] (fp32/bf16, contiguous),
+    win_len_dev [B] int32 device (valid slots per sequence)."""
+    if len_dev.dtype != torch.int32 or win_len_dev.dtype != torch.int32:
+        raise TypeError("len_dev and win_len_dev must be int32")
+    if win_k.dtype != win_v.dtype:
+        raise TypeError("win_k and win_v must share a dtype")
+    if not (win_k.is_contiguous() and win_v.is_contiguous()):
+        raise ValueError("win_k and win_v must be contiguous")
+    scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().tq_decode_attention_window(ctypes.byref(layer.params), ctypes.byref(cache.cache),
+                                           q.data_ptr(), _dtype_code(q), int(q.shape[1]),
+                                           len_dev.data_ptr(), int(max_len), win_k.data_ptr(),
+                                           win_v.data_ptr(), _dtype_code(win_k), win_len_dev.data_ptr(),
+                                           int(win_k.shape[2]), scale, out.data_ptr(),
+                                           workspace.data_ptr(),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream))
+    _check("tq_decode_attention_window", st)
 
 
 def tq_decode_attention_noalloc(layer: Layer, cache: CompressedCache, q: torch.Tensor,

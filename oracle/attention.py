@@ -91,6 +91,53 @@ def decode_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
     return out
 
 
+def decode_with_window(q: np.ndarray, rec: dict | None, win_k: np.ndarray, win_v: np.ndarray,
+                       pi, s, centroids, group: int,
+                       softmax_scale: float | None = None) -> np.ndarray:
+    """Decode attention over the compressed tokens of one sequence plus a
+    window of recent tokens kept exactly ("turboquant/audit_claims.py",
+    AUDIT 1: the store keeps the most recent 128 tokens uncompressed in
+    bf16 next to the compressed history).  One softmax over both sets:
+    compressed tokens score with the estimator (score_keys) and carry the
+    group-dequantized values; window tokens score q.k exactly and carry v.
+
+    q      [H_q, d]
+    rec    logical cache fields as in decode_one_sequence, or None / N = 0
+    win_k, win_v  [W, H_kv, d] exact window keys and values (W may be 0)
+    Returns out [H_q, d] float64 (zeros when there is no token at all).
+    """
+    q = np.asarray(q, np.float64)
+    hq, d = q.shape
+    win_k = np.asarray(win_k, np.float64)
+    win_v = np.asarray(win_v, np.float64)
+    w, hkv = win_k.shape[0], win_k.shape[1]
+    n = 0 if rec is None else rec["nk16"].shape[0]
+    g = hq // hkv
+    scale = 1.0 / np.sqrt(d) if softmax_scale is None else softmax_scale
+    out = np.zeros((hq, d))
+    if n + w == 0:
+        return out
+    for h in range(hkv):
+        vparts = []
+        if n:
+            vparts.append(dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
+                                            rec["zero16"][:, h], group))
+        if w:
+            vparts.append(win_v[:, h])
+        values = np.concatenate(vparts, axis=0)
+        for j in range(g):
+            qh = h * g + j
+            lparts = []
+            if n:
+                lparts.append(score_keys(q[qh], rec["idx"][:, h], rec["sign"][:, h],
+                                         rec["nk16"][:, h], rec["rn16"][:, h], pi, s,
+                                         centroids) * scale)
+            if w:
+                lparts.append((win_k[:, h] @ q[qh]) * scale)
+            out[qh] = softmax_average(np.concatenate(lparts), values)
+    return out
+
+
 def brute_force_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids,
                              group: int, softmax_scale: float | None = None) -> np.ndarray:
     """softmax(K_hat q / sqrt d) V_hat over explicitly dequantized K and V

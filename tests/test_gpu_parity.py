@@ -385,3 +385,58 @@ def test_decode_asymmetric_codebook(kb):
         kes, ves = encs[b]
         ref = pu.oracle_decode(olayer, q[b].float().numpy(), kes, ves, lengths[b])
         assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (kb, b)
+
+
+@pytest.mark.parametrize("name,kb,vb,h_kv,h_q", [
+    ("llama8b", 3, 2, 2, 8),     # tensor-core kernel, GQA 4
+    ("qwen15b_512", 3, 3, 1, 6),  # tensor-core kernel, 3-bit values, GQA 6
+    ("llama8b", 3, 4, 2, 4),     # SIMT split-K kernel
+])
+def test_decode_with_recent_window(name, kb, vb, h_kv, h_q):
+    """Compressed history plus an exact window of the next tokens of each
+    sequence, one softmax: lengths 0, 1, a tile plus one, 300; window
+    lengths 5, 0, 128, 64 (capacity 128), and a sequence with neither."""
+    import dataclasses
+    lengths = (0, 1, 129, 300, 0)
+    wlens = (5, 0, 128, 64, 0)
+    base = workloads.by_name(name)
+    wl = dataclasses.replace(base, batch=5, h_kv=h_kv, h_q=h_q, key_bits=kb, value_bits=vb,
+                             lengths=lengths, capacity=384, name=f"win_{name}_{kb}{vb}")
+    glayer, olayer, spec = _setup(wl)
+    buf, encs = _oracle_cache(wl, olayer, spec, lengths)
+    cap = 128
+    dt = torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32
+    wk = torch.zeros((wl.batch, h_kv, cap, 128), dtype=dt)
+    wv = torch.zeros_like(wk)
+    for b in range(wl.batch):
+        if wlens[b]:
+            k, v = workloads.kv_tokens(wl, b, lengths[b], lengths[b] + wlens[b])
+            wk[b, :, :wlens[b]] = k.transpose(0, 1).to(dt)
+            wv[b, :, :wlens[b]] = v.transpose(0, 1).to(dt)
+    q = workloads.queries(wl, 0)
+    cache = tq.CompressedCache(glayer, wl.batch, wl.h_kv, wl.capacity)
+    cache.buffer.copy_(torch.from_numpy(buf))
+    len_dev = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    wlen_dev = torch.tensor(wlens, dtype=torch.int32, device=DEV)
+    ml = max(lengths)
+    ws = tq.workspace_for(glayer, cache, wl.h_q, ml)
+    out = torch.empty((wl.batch, wl.h_q, 128), device=DEV)
+    tq.tq_decode_attention_window(glayer, cache, q.to(DEV).contiguous(), len_dev, ml,
+                                  wk.to(DEV).contiguous(), wv.to(DEV).contiguous(), wlen_dev, out, ws)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    from oracle import attention
+    for b in range(wl.batch):
+        n, w = lengths[b], wlens[b]
+        rec = None
+        if n:
+            kes, ves = encs[b]
+            rec = attention.stack_heads([pu.logical(ke, ve) for ke, ve in zip(kes, ves)])
+        wkb = wk[b, :, :w].transpose(0, 1).float().numpy()
+        wvb = wv[b, :, :w].transpose(0, 1).float().numpy()
+        ref = attention.decode_with_window(q[b].float().numpy(), rec, wkb, wvb, olayer.pi, olayer.s,
+                                           olayer.cent, 32)
+        if n + w == 0:
+            assert np.all(got[b] == 0.0)
+            continue
+        assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (name, b)

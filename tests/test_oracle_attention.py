@@ -131,3 +131,66 @@ def test_large_logits_stay_finite():
     assert np.all(np.isfinite(out))
     b = attention.brute_force_one_sequence(q, rec, pi, s, cent, 32)
     assert np.allclose(out, b, rtol=1e-9, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# recent-token window (exact) merged into the same softmax
+# ---------------------------------------------------------------------------
+
+def test_window_empty_equals_compressed_decode():
+    rec, pi, s, cent = _random_cache(40, 2, 128, 3, 2, 32, seed=11)
+    q = np.random.default_rng(12).standard_normal((4, 128))
+    empty = np.zeros((0, 2, 128))
+    a = attention.decode_with_window(q, rec, empty, empty, pi, s, cent, 32)
+    b = attention.decode_one_sequence(q, rec, pi, s, cent, 32)
+    assert np.array_equal(a, b)
+
+
+def test_window_alone_is_textbook_attention():
+    """No compressed tokens: exactly softmax(K q / sqrt d) V over the window,
+    written out here with explicit sums."""
+    rng = np.random.default_rng(13)
+    wk = rng.standard_normal((7, 1, 128))
+    wv = rng.standard_normal((7, 1, 128))
+    q = rng.standard_normal((3, 128))
+    out = attention.decode_with_window(q, None, wk, wv, None, None, None, 32)
+    for j in range(3):
+        logits = [float(np.dot(wk[t, 0], q[j])) / math.sqrt(128) for t in range(7)]
+        top = max(logits)
+        w = [math.exp(x - top) for x in logits]
+        ref = sum(w[t] * wv[t, 0] for t in range(7)) / sum(w)
+        assert np.allclose(out[j], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_window_merge_matches_log_sum_exp_of_the_parts():
+    """The one softmax over compressed + window tokens equals the log-sum-exp
+    merge of the two parts computed separately (a different route: split-K
+    combine of two partial states)."""
+    rec, pi, s, cent = _random_cache(33, 2, 128, 4, 2, 32, seed=14)
+    rng = np.random.default_rng(15)
+    wk = rng.standard_normal((5, 2, 128)) * 3
+    wv = rng.standard_normal((5, 2, 128))
+    q = rng.standard_normal((4, 128))
+    out = attention.decode_with_window(q, rec, wk, wv, pi, s, cent, 32)
+    for qh in range(4):
+        h = qh // 2
+        sc = attention.score_keys(q[qh], rec["idx"][:, h], rec["sign"][:, h], rec["nk16"][:, h],
+                                  rec["rn16"][:, h], pi, s, cent) / math.sqrt(128)
+        vh = quant.dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
+                                     rec["zero16"][:, h], 32)
+        lw = (wk[:, h] @ q[qh]) / math.sqrt(128)
+        parts = []
+        for logits, vals in ((sc, vh), (lw, wv[:, h])):
+            m = logits.max()
+            e = np.exp(logits - m)
+            parts.append((m, e.sum(), e @ vals / e.sum()))
+        M = max(p[0] for p in parts)
+        num = sum(np.exp(m - M) * l * o for m, l, o in parts)
+        den = sum(np.exp(m - M) * l for m, l, o in parts)
+        assert np.allclose(out[qh], num / den, rtol=1e-11, atol=1e-12)
+
+
+def test_window_nothing_cached_gives_zeros():
+    empty = np.zeros((0, 2, 128))
+    out = attention.decode_with_window(np.ones((2, 128)), None, empty, empty, None, None, None, 32)
+    assert not out.any()
