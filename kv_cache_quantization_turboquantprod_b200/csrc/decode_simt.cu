@@ -215,10 +215,33 @@ __global__ void __launch_bounds__(128) window_kernel(DecodeArgs a) {
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = 0.f;
-    for (int j = 0; j < kD; ++j) {
-      const float k = load_elem(a.win_k, a.win_dtype, (row0 + t) * kD + j);
+    // the slot's key row with 16-byte loads (8 bf16 or 4 fp32 at a time)
+    if (a.win_dtype == TQ_BF16) {
+      const uint4 *kr = reinterpret_cast<const uint4 *>(
+          reinterpret_cast<const __nv_bfloat16 *>(a.win_k) + (row0 + t) * kD);
+#pragma unroll 4
+      for (int c = 0; c < kD / 8; ++c) {
+        const uint4 w = kr[c];
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = fmaf(qs[g][j], k, acc[g]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            acc[g] = fmaf(qs[g][8 * c + 2 * e + 1], f.y, fmaf(qs[g][8 * c + 2 * e], f.x, acc[g]));
+        }
+      }
+    } else {
+      const float4 *kr = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.win_k) +
+                                                          (row0 + t) * kD);
+#pragma unroll 4
+      for (int c = 0; c < kD / 4; ++c) {
+        const float4 f = kr[c];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          acc[g] = fmaf(qs[g][4 * c + 3], f.w, fmaf(qs[g][4 * c + 2], f.z,
+                   fmaf(qs[g][4 * c + 1], f.y, fmaf(qs[g][4 * c], f.x, acc[g]))));
+      }
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) lg[g] = acc[g] * scale2;
