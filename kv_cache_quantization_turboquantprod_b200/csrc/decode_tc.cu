@@ -33,18 +33,20 @@
 // Per 128-token tile the record bytes arrive by one 1-D bulk copy (TMA
 // engine) into a ring of shared-memory stages.
 //
-// Warp roles (576 threads; each SM sub-partition gets one warp of each
-// worker group):
+// Warp roles (576 threads):
 //   warp 0        bulk-copy producer; allocates / frees tensor memory
 //   warp 1        MMA issuer (one elected lane issues), polling the score
 //                 and PV queues so neither blocks the other
-//   warps 2-5     key group: code-bit / sign planes -> u8 operands in tensor memory
-//   warps 6-9     value group: codes -> A_v (MN-major, shared memory); PV
-//                 epilogue and the per-channel accumulators
-//   warps 10-17   two softmax groups taking alternate tiles, each with its
-//                 own running max / sum (merged at the end like two splits):
-//                 score epilogue, tile max by warp redux + an mbarrier
-//                 exchange, the P' operand, running l and zero-point sums
+//   warps 2-17    four worker groups of four warps (one per TMEM lane
+//                 quarter); group g takes tiles g, g + 4, ... through every
+//                 SIMT step: plane operands -> tensor memory, value codes ->
+//                 A_v (MN-major, shared memory), score epilogue, tile max by
+//                 warp redux + an mbarrier exchange inside the group, online
+//                 softmax with the group's own running max / sum, the P'
+//                 operand, and the P.V read-back into per-channel
+//                 accumulators.  The four states are merged at the end like
+//                 four splits.  Every SM sub-partition runs one warp of each
+//                 group, so the per-tile work is spread evenly.
 // Every mbarrier wait is bounded (2 s); on timeout the CTA sets the status word in
 // the workspace, stops, waits for its own copies and MMAs and frees TMEM.
 #include <math.h>
@@ -63,6 +65,7 @@ constexpr int kTcThreads = 576;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTmemCols = 512;
 constexpr int kPlaneCols = 32;  // one u8 operand plane: 128 coordinates per row = 32 TMEM columns
+constexpr int kWorkGroups = 4;  // worker groups of 4 warps; group g takes tiles g, g + 4, ...
 
 // 2^n for n in [-126, 127]
 __device__ __forceinline__ float exp2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
@@ -77,12 +80,12 @@ __host__ __device__ constexpr int max_planes(int MB) { return (1 << MB); }
 // Score constants that follow B_q in a query block.
 constexpr int kQConstBytes = 256;
 struct QConst {
-  float cm[8];         // (a_0 - sum of the active a_S) * sum_j q~_j
-  float csum[8];       // sum_j s^_j
-  float coef_m[8][2];  // limb weights of the MSE term: 2^-F, 2^(14-F)
-  float coef_s[8][2];  // limb weights of the QJL term
-  int n_mse;           // active subset planes (1 .. 2^m - 1)
-  int subset[7];       // their code-bit masks
+  float cm[8];     // (a_0 - sum of the active a_S) * sum_j q~_j
+  float ncsum[8];  // -sum_j s^_j
+  float fm[8];     // limb weight 2^-F of the MSE term (the upper limb pair carries 2^14 more)
+  float fs[8];     // limb weight of the QJL term
+  int n_mse;       // active subset planes (1 .. 2^m - 1)
+  int subset[7];   // their code-bit masks
 };
 static_assert(sizeof(QConst) <= kQConstBytes, "query constants");
 
@@ -98,14 +101,16 @@ struct Cfg {
   static constexpr int NS = score_n(G);                 // score N per accumulator
   static constexpr int NPV = 16 * G;                    // PV N: 4 groups x G heads x 4 bytes
   static constexpr int NPL = max_planes(MB);            // operand planes, upper bound
+  static constexpr int SYM_COLS = (NSYM + 1) * kPlaneCols;  // A_k of one tile, symmetric codebook
   // tensor memory: A_k planes | D_s (2 buffers x (mse, qjl)) | D_pv (NR buffers).
-  // The P.V ring (A_v, B_p, D_pv) is 3 deep when three A_k buffers of a
-  // symmetric codebook's planes still fit, else 2; A_k takes what is left.
-  static constexpr int NR =
-      (4 * NS + 3 * NPV + 3 * (NSYM + 1) * kPlaneCols <= kTmemCols) ? 3 : 2;
+  // The P.V ring (A_v, B_p, D_pv) gets one slot per worker group when two
+  // symmetric A_k buffers still fit (each group then owns its slot), else
+  // as many as fit, at least 2.
+  static constexpr int NR_FIT = (kTmemCols - 4 * NS - 2 * SYM_COLS) / NPV;
+  static constexpr int NR = NR_FIT >= kWorkGroups ? kWorkGroups : (NR_FIT >= 2 ? NR_FIT : 2);
+  static constexpr bool OWN_SLOT = NR == kWorkGroups;
   static constexpr int AK_COLS = kTmemCols - 4 * NS - NR * NPV;
-  // A_k ring depth for a codebook with npl planes (1 or 2; a third buffer
-  // measured slower: it lets the key group run ahead of the other roles)
+  // A_k ring depth for a codebook with npl planes (2 when two buffers fit)
   __host__ __device__ static constexpr int ak_ring(int npl) {
     return AK_COLS / (npl * kPlaneCols) >= 2 ? 2 : 1;
   }
@@ -126,11 +131,12 @@ struct Cfg {
   static constexpr int AV_BYTES = 128 * 128;            // [128 channel slots] x [128 tokens]
   static constexpr int BP_BYTES = 128 * NPV;            // [128 tokens] x [NPV]
   static constexpr int SBO_V = 2048;                    // MN-major stride of 16-byte chunks
-  static constexpr int FIXED = NR * AV_BYTES + NR * BP_BYTES + QBLOCK + 4096;
-  static constexpr int STAGES_FIT = (220 * 1024 - FIXED) / TILE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int MERGE_BYTES = (kWorkGroups - 1) * 128 * G * 4 + kWorkGroups * 4 * G * 4 * 5 + 1024;
+  static constexpr int FIXED = NR * AV_BYTES + NR * BP_BYTES + QBLOCK + MERGE_BYTES + 2048;
+  static constexpr int STAGES_FIT = (224 * 1024 - FIXED) / TILE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static_assert(NPL * kPlaneCols <= AK_COLS, "tensor memory budget");
-  static_assert(STAGES >= 2, "shared memory budget");
+  static_assert(STAGES >= 4, "shared memory budget");
   static_assert(TILE_BYTES % 16 == 0, "bulk copy size");
   static_assert(QBLOCK == (int)qblock_bytes_for(MB, G), "query block size");
 };
@@ -145,16 +151,16 @@ struct TcSmem {
   uint64_t empty[C::STAGES];
   uint64_t ak_ready[2], s_ready[2], s_free[2];
   uint64_t av_ready[C::NR], p_ready[C::NR], pv_done[C::NR], pv_free[C::NR];
-  uint64_t red_bar[2];
+  uint64_t red_bar[kWorkGroups];
   uint64_t q_full;
   uint32_t tmem_base;
   volatile int abort_flag;
-  alignas(16) float red[2][2][C::G + 1][4];  // [softmax group][slot][head | value scale][warp]
-  float alpha[C::NR][C::G];
-  float pscale[C::NR];
-  float fin_m[2][C::G];
-  float lsum[2][4][C::G];
-  float zsum[2][4][C::G][4];
+  alignas(16) float red[kWorkGroups][2][C::G + 1][4];  // [group][slot][head | value scale][warp]
+  float fin_m[kWorkGroups][C::G];
+  float lsum[kWorkGroups][4][C::G];
+  float zsum[kWorkGroups][4][C::G][4];
+  float accx[kWorkGroups - 1][128][C::G];  // groups 1.. hand their accumulators to group 0
+  float dal[kWorkGroups][4][C::G + 1];     // per warp: alpha of its last tile, fixed-point scale
 };
 
 // Bounded wait (2 s of wall time) that also gives up when another role has
@@ -183,6 +189,10 @@ __device__ __forceinline__ uint32_t subset_word(int S, uint32_t b0, uint32_t b1,
   uint32_t x = ((S & 1) ? b0 : 0u) ^ ((S & 2) ? b1 : 0u) ^ ((S & 4) ? b2 : 0u);
   return (__popc(S) & 1) ? x : ~x;
 }
+
+// The odd code-bit subsets in increasing order: the planes of a symmetric
+// codebook (1 | 1, 2 | 1, 2, 4, 7 at m = 1, 2, 3).
+__host__ __device__ constexpr int odd_subset(int p) { return p < 2 ? p + 1 : (p == 2 ? 4 : 7); }
 
 // Eight u8 operand words of one 32-coordinate bit word w: word k, byte i is
 // coordinate 8i + k with weight 2^(k mod 4) (bits 4..7 are taken from w >> 4
@@ -275,14 +285,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 12);
+      mbar_init(&S.empty[s], 4);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&S.ak_ready[i], 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1);
       mbar_init(&S.s_free[i], 4);
-      mbar_init(&S.red_bar[i], 4);
     }
+    for (int i = 0; i < kWorkGroups; ++i) mbar_init(&S.red_bar[i], 4);
     for (int i = 0; i < C::NR; ++i) {
       mbar_init(&S.av_ready[i], 4);
       mbar_init(&S.p_ready[i], 4);
@@ -416,107 +426,168 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // never leave with an MMA in flight
     if (is > 0) mbar_wait(&S.s_ready[(is - 1) & 1], ((is - 1) >> 1) & 1);
     if (ip > 0) mbar_wait(&S.pv_done[(ip - 1) % C::NR], ((ip - 1) / C::NR) & 1);
-  } else if (warp < 6) {
-    // ---------------- key group: plane operands -> tensor memory ----------
-    // The next tile's plane words are fetched while this tile's tensor-memory
-    // stores drain.
+  } else {
+    // ---------------- worker groups ----------------------------------------
+    // Group grp (warps 2 + 4 grp .. 5 + 4 grp, one per TMEM lane quarter)
+    // takes tiles grp, grp + 4, ... through every SIMT step: plane operands
+    // to tensor memory, value operand, score epilogue, online softmax with
+    // its own running max / sum, P' operand and the P.V read-back.  The four
+    // groups' states are merged at the end like four splits.
+    const int grp = (warp - 2) >> 2;
     const int q4 = warp & 3;
-    const int t = 32 * q4 + lane;  // token slot == TMEM lane
+    const int t = 32 * q4 + lane;  // token slot (score, operands) == TMEM lane == M slot of P.V
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+    // value channel of this M slot and the 4^m weight its operand bytes carry
+    const int kk = C::PACKED_V ? 2 * ((t >> 2) & 3) : 0;
+    const int chan = C::PACKED_V ? 16 * (t >> 4) + 4 * (t & 3) + ((t >> 2) & 3)
+                                 : 32 * (t >> 5) + 8 * (t & 3) + 4 * ((t >> 4) & 1) + ((t >> 2) & 3);
+    const float kappa = qjl_kappa();
+    const float scale2 = a.softmax_scale * kLog2e;
     const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
     const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
     const int akb = C::ak_ring(npl);
-    int subs[7];
+    // symmetric codebook: the planes are the odd subsets, known at compile
+    // time, so the spin words need no selects
+    bool sym = nm == C::NSYM;
 #pragma unroll
-    for (int p = 0; p < 7; ++p) subs[p] = (qok && p < nm) ? Q.subset[p] : 0;
-    uint32_t bw[3][4], sw[4];
-    auto fetch = [&](int i) -> bool {
-      const int s = i % C::STAGES;
-      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) return false;
-      const uint8_t *st = S.stage[s];
+    for (int p = 0; p < C::NSYM; ++p) sym = sym && Q.subset[p] == odd_subset(p);
+
+    float mrun[G], lsum[G], zs[G][4], acc[G];
 #pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        if (p < MB) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(st + p * kPlaneBytes + t * kRowBytes);
-          bw[p][0] = v.x; bw[p][1] = v.y; bw[p][2] = v.z; bw[p][3] = v.w;
-        } else {
-          bw[p][0] = bw[p][1] = bw[p][2] = bw[p][3] = 0u;
-        }
-      }
-      const uint4 sv = *reinterpret_cast<const uint4 *>(st + C::OFF_SIGNS + t * kRowBytes);
-      sw[0] = sv.x; sw[1] = sv.y; sw[2] = sv.z; sw[3] = sv.w;
+    for (int g = 0; g < G; ++g) {
+      mrun[g] = -INFINITY;
+      lsum[g] = 0.f;
+      acc[g] = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) zs[g][gg] = 0.f;
+    }
+    // P.V read-back of tile jt in slot rb: acc = acc * alpha + D * sc, with
+    // alpha[0..G-1] and sc = alpha[G] as this warp left them in shared memory
+    float *dal = S.dal[grp][q4];
+    auto readback = [&](int jt, int rb) -> bool {
+      if (!wait_bar(&S.pv_done[rb], (jt / C::NR) & 1, &S.abort_flag, status)) return false;
+      tc_fence_after();
+      uint32_t d[4 * G];
+      tmem_ld_cols<4 * G>(tbase + lane_off + C::COL_DPV + rb * C::NPV + q4 * 4 * G, d);
+      tmem_wait_ld();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[s]);
+      if (lane == 0) mbar_arrive(&S.pv_free[rb]);
+      const float sc = dal[G] * exp2i(-kk);  // this M slot carries code * 4^m
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float v = fmaf(16777216.f, (float)d[4 * g + 3],
+                             fmaf(65536.f, (float)d[4 * g + 2], fmaf(256.f, (float)d[4 * g + 1], (float)d[4 * g])));
+        acc[g] = fmaf(acc[g], dal[g], v * sc);
+      }
       return true;
     };
-    bool ok = qok && fetch(0);
-    for (int i = 0; ok && i < ntile; ++i) {
-      // the A_k buffer of tile i was last read by the score MMA of tile i - akb
+    // with its own P.V slot a group reads tile jt's result back at its next
+    // tile (jt + 4), when the MMA has long finished
+    int prev = -1;
+
+    constexpr int NVW = C::PACKED_V ? 8 : 4 * VB;
+    bool ok = qok;
+    for (int i = grp; ok && i < ntile; i += kWorkGroups) {
+      const int n = i / kWorkGroups, s = i % C::STAGES, rb = i % C::NR;
+      ok = false;
+      // 1. code / sign plane words of the tile
+      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
+      const uint8_t *st = S.stage[s];
+      uint32_t bw[3][4], sw[4];
+      {
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          if (p < MB) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(st + p * kPlaneBytes + t * kRowBytes);
+            bw[p][0] = v.x; bw[p][1] = v.y; bw[p][2] = v.z; bw[p][3] = v.w;
+          } else {
+            bw[p][0] = bw[p][1] = bw[p][2] = bw[p][3] = 0u;
+          }
+        }
+        const uint4 sv = *reinterpret_cast<const uint4 *>(st + C::OFF_SIGNS + t * kRowBytes);
+        sw[0] = sv.x; sw[1] = sv.y; sw[2] = sv.z; sw[3] = sv.w;
+      }
+
+      // 2. plane operands -> A_k buffer of tile i, free once the score MMA
+      //    of tile i - akb has finished
       if (i >= akb) {
-        const int prev = i - akb;
-        if (!wait_bar(&S.s_ready[prev & 1], (prev >> 1) & 1, &S.abort_flag, status)) break;
+        const int pt = i - akb;
+        if (!wait_bar(&S.s_ready[pt & 1], (pt >> 1) & 1, &S.abort_flag, status)) break;
       }
       const int ab = akb == 2 ? (i & 1) : 0;
-      const uint32_t a_base = tbase + lane_off + ab * npl * kPlaneCols;
+      {
+        const uint32_t a_base = tbase + lane_off + ab * npl * kPlaneCols;
+        if (sym) {
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        if (p > nm) break;
-        uint32_t r[32];
+          for (int p = 0; p <= C::NSYM; ++p) {
 #pragma unroll
-        for (int wd = 0; wd < 4; ++wd)
-          plane_operands((p < nm) ? subset_word(subs[p < 7 ? p : 6], bw[0][wd], bw[1][wd], bw[2][wd]) : sw[wd],
-                         r + 8 * wd);
-        tmem_st32(a_base + p * kPlaneCols, r);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              uint32_t r[16];
+#pragma unroll
+              for (int wd = 0; wd < 2; ++wd)
+                plane_operands(p < C::NSYM ? subset_word(odd_subset(p), bw[0][2 * h2 + wd], bw[1][2 * h2 + wd],
+                                                         bw[2][2 * h2 + wd])
+                                           : sw[2 * h2 + wd],
+                               r + 8 * wd);
+              tmem_st16(a_base + p * kPlaneCols + 16 * h2, r);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            if (p > nm) break;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              uint32_t r[16];
+#pragma unroll
+              for (int wd = 0; wd < 2; ++wd)
+                plane_operands((p < nm) ? subset_word(Q.subset[p < 7 ? p : 6], bw[0][2 * h2 + wd], bw[1][2 * h2 + wd],
+                                                      bw[2][2 * h2 + wd])
+                                        : sw[2 * h2 + wd],
+                               r + 8 * wd);
+              tmem_st16(a_base + p * kPlaneCols + 16 * h2, r);
+            }
+          }
+        }
       }
-      const bool next = (i + 1 < ntile) ? fetch(i + 1) : true;
+
+      // 3. the P.V slot: its last tile's operands must have been consumed
+      if constexpr (C::OWN_SLOT) {
+        if (prev >= 0 && !readback(prev, rb)) break;
+      } else {
+        if (i >= C::NR && !wait_bar(&S.pv_done[rb], ((i - C::NR) / C::NR) & 1, &S.abort_flag, status)) break;
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.ak_ready[ab]);
-      ok = next;
-    }
-  } else if (warp < 10) {
-    // ---------------- value group ------------------------------------------
-    const int q4 = warp & 3;
-    const int t = 32 * q4 + lane;  // token slot for expansion; M slot for PV
-    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    // channel of this M slot and the 4^m weight its operand bytes carry
-    const int kk = C::PACKED_V ? 2 * ((t >> 2) & 3) : 0;
-    const int chan = C::PACKED_V ? 16 * (t >> 4) + 4 * (t & 3) + ((t >> 2) & 3)
-                                 : 32 * (t >> 5) + 8 * (t & 3) + 4 * ((t >> 4) & 1) + ((t >> 2) & 3);
-    float acc[2][G];
+
+      // 4. value codes, norms and value scales; the stage is then released
+      uint32_t vw[NVW];
+      uint32_t nrw;
+      uint4 szr;
+      {
+        if constexpr (C::PACKED_V) {
+          const uint4 v0 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes);
+          const uint4 v1 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes + 16);
+          vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
+          vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
+        } else {
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[0][g] = acc[1][g] = 0.f;
-    // value words of the next tile are fetched before this tile's PV result
-    // is waited for
-    constexpr int NVW = C::PACKED_V ? 8 : 4 * VB;
-    uint32_t vw[NVW];
-    auto fetch = [&](int i) -> bool {
-      const int s = i % C::STAGES;
-      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) return false;
-      const uint8_t *st = S.stage[s];
-      if constexpr (C::PACKED_V) {
-        const uint4 v0 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes);
-        const uint4 v1 = *reinterpret_cast<const uint4 *>(st + C::OFF_V + t * kPackedRowBytes + 16);
-        vw[0] = v0.x; vw[1] = v0.y; vw[2] = v0.z; vw[3] = v0.w;
-        vw[4] = v1.x; vw[5] = v1.y; vw[6] = v1.z; vw[7] = v1.w;
-      } else {
-#pragma unroll
-        for (int p = 0; p < VB; ++p) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
-          vw[4 * p] = v.x; vw[4 * p + 1] = v.y; vw[4 * p + 2] = v.z; vw[4 * p + 3] = v.w;
+          for (int p = 0; p < VB; ++p) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(st + C::OFF_V + p * kPlaneBytes + t * kRowBytes);
+            vw[4 * p] = v.x; vw[4 * p + 1] = v.y; vw[4 * p + 2] = v.z; vw[4 * p + 3] = v.w;
+          }
         }
+        nrw = *reinterpret_cast<const uint32_t *>(st + C::OFF_NORMS + t * 4);
+        szr = *reinterpret_cast<const uint4 *>(st + C::OFF_VSZ + t * 16);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[s]);
-      return true;
-    };
-    bool have = ntile > 0 && fetch(0);
-    for (int i = 0; i <= ntile; ++i) {
-      if (i < ntile) {
-        if (!have) break;
-        const int vb = i % C::NR;
-        uint8_t *row = S.av[vb] + (t >> 3) * 128 + (t & 7) * 16;
+      // value codes -> A_v (MN-major, shared memory)
+      {
+        uint8_t *row = S.av[rb] + (t >> 3) * 128 + (t & 7) * 16;
         if constexpr (C::PACKED_V) {
           // packed row: word w holds channels 16w .. 16w+15; mask m keeps
           // channel 16w + 4i + m in byte i as code * 4^m (M slot 16w + 4m + i)
@@ -542,99 +613,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             *reinterpret_cast<uint4 *>(row + m16 * C::SBO_V) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.av_ready[vb]);
-        have = (i + 1 < ntile) ? fetch(i + 1) : true;
       }
-      if (i >= 1) {
-        const int jt = i - 1, pb = jt % C::NR, sg = jt & 1;
-        const uint32_t rph = (jt / C::NR) & 1;
-        if (!wait_bar(&S.pv_done[pb], rph, &S.abort_flag, status)) break;
-        if (!wait_bar(&S.p_ready[pb], rph, &S.abort_flag, status)) break;
-        tc_fence_after();
-        uint32_t d[4 * G];
-        tmem_ld_cols<4 * G>(tbase + lane_off + C::COL_DPV + pb * C::NPV + q4 * 4 * G, d);
-        tmem_wait_ld();
-        tc_fence_before();
-        float alpha[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) alpha[g] = S.alpha[pb][g];
-        const float sc = S.pscale[pb] * exp2i(-kk);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.pv_free[pb]);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float v = fmaf(16777216.f, (float)d[4 * g + 3],
-                               fmaf(65536.f, (float)d[4 * g + 2],
-                                    fmaf(256.f, (float)d[4 * g + 1], (float)d[4 * g])));
-          acc[sg][g] = fmaf(acc[sg][g], alpha[g], v * sc);
-        }
-      }
-    }
-    named_bar_sync(3, 384);  // the softmax groups' states are in shared memory
-    // merge the two softmax states; unnormalised partial output
-    // sum_t p_t (code * scale + zero)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float m0 = S.fin_m[0][g], m1 = S.fin_m[1][g];
-      const float mm = fmaxf(m0, m1);
-      const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mm);
-      const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mm);
-      float z0 = 0.f, z1 = 0.f, l0 = 0.f, l1 = 0.f;
-#pragma unroll
-      for (int wq = 0; wq < 4; ++wq) {
-        z0 += S.zsum[0][wq][g][q4];
-        z1 += S.zsum[1][wq][g][q4];
-        l0 += S.lsum[0][wq][g];
-        l1 += S.lsum[1][wq][g];
-      }
-      float *pr = part_row(g);
-      pr[chan] = (acc[0][g] + z0) * f0 + (acc[1][g] + z1) * f1;
-      if (t == 0) {
-        // m (log2 units, as the SIMT path) and l of the split
-        pr[kD] = mm;
-        pr[kD + 1] = l0 * f0 + l1 * f1;
-      }
-    }
-  } else {
-    // ---------------- softmax groups ---------------------------------------
-    const int grp = (warp - 10) >> 2;  // takes tiles grp, grp + 2, ...
-    const int q4 = warp & 3;
-    const int t = 32 * q4 + lane;  // token slot == TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    const float kappa = qjl_kappa();
-    const float scale2 = a.softmax_scale * kLog2e;
-    float mrun[G], lsum[G], zs[G][4];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      mrun[g] = -INFINITY;
-      lsum[g] = 0.f;
-#pragma unroll
-      for (int gg = 0; gg < 4; ++gg) zs[g][gg] = 0.f;
-    }
-    const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
-    // score constants of this (sequence, KV head): in registers up to GQA 4
-    constexpr bool kRegConst = G <= 4;
-    float qcm[G], qcs[G], qfm[G], qfs[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      if (kRegConst) {
-        qcm[g] = Q.cm[g];
-        qcs[g] = -Q.csum[g];
-        qfm[g] = Q.coef_m[g][0];
-        qfs[g] = Q.coef_s[g][0];
-      }
-    }
-    for (int jt = grp; qok && jt < ntile; jt += 2) {
-      const int kb = grp, pb = jt % C::NR, s = jt % C::STAGES, n = jt >> 1;
-      if (!wait_bar(&S.full[s], (jt / C::STAGES) & 1, &S.abort_flag, status)) break;
-      if (!wait_bar(&S.s_ready[kb], n & 1, &S.abort_flag, status)) break;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.av_ready[rb]);
+
+      // 5. score epilogue; limbs combine as (D0 + 128 D1) 2^-F + (D2 + 128 D3) 2^(14-F)
+      if (!wait_bar(&S.s_ready[i & 1], (i >> 1) & 1, &S.abort_flag, status)) break;
       tc_fence_after();
       float mse[G], qjl[G];
       {
-        // limbs combine as (D0 + 128 D1) 2^-F + (D2 + 128 D3) 2^(14-F)
-        const uint32_t base = tbase + lane_off + C::COL_DS + kb * 2 * C::NS;
+        const uint32_t base = tbase + lane_off + C::COL_DS + (i & 1) * 2 * C::NS;
         uint32_t d[4 * G];
         tmem_ld_cols<4 * G>(base, d);
         tmem_wait_ld();
@@ -642,8 +631,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         for (int g = 0; g < G; ++g) {
           const int am = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
           const int bm = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
-          const float fm = kRegConst ? qfm[g] : Q.coef_m[g][0];
-          mse[g] = fmaf(fm * 16384.f, (float)bm, fmaf(fm, (float)am, kRegConst ? qcm[g] : Q.cm[g]));
+          const float fm = Q.fm[g];
+          mse[g] = fmaf(fm * 16384.f, (float)bm, fmaf(fm, (float)am, Q.cm[g]));
         }
         tmem_ld_cols<4 * G>(base + C::NS, d);
         tmem_wait_ld();
@@ -651,21 +640,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         for (int g = 0; g < G; ++g) {
           const int as = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
           const int bs = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
-          const float fs = kRegConst ? qfs[g] : Q.coef_s[g][0];
-          qjl[g] = fmaf(fs * 16384.f, (float)bs, fmaf(fs, (float)as, kRegConst ? qcs[g] : -Q.csum[g]));
+          const float fs = Q.fs[g];
+          qjl[g] = fmaf(fs * 16384.f, (float)bs, fmaf(fs, (float)as, Q.ncsum[g]));
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.s_free[kb]);
+      if (lane == 0) mbar_arrive(&S.s_free[i & 1]);
 
-      const uint8_t *st = S.stage[s];
-      const bool valid = t_begin + jt * kTile + t < t_end;
-      const __half2 nr = *reinterpret_cast<const __half2 *>(st + C::OFF_NORMS + t * 4);
+      // 6. logits, tile maxima over the group's 128 tokens, online softmax
+      const bool valid = t_begin + i * kTile + t < t_end;
+      const __half2 nr = *reinterpret_cast<const __half2 *>(&nrw);
       const float nk = __low2float(nr), rn = __high2float(nr);
-      const uint4 szr = *reinterpret_cast<const uint4 *>(st + C::OFF_VSZ + t * 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[s]);
       const __half2 *szh = reinterpret_cast<const __half2 *>(&szr);
       float vsc[4], vze[4];
       float msc = 0.f;
@@ -682,7 +668,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         const float score = nk * fmaf(krn, qjl[g], mse[g]);
         lg[g] = valid ? score * scale2 : -INFINITY;
       }
-      // tile maxima (logits per head, value scale) over the 128 tokens
       float(&red)[G + 1][4] = S.red[grp][n & 1];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -730,31 +715,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
         for (int gg = 0; gg < 4; ++gg) zs[g][gg] = fmaf(p[g], vze[gg], zs[g][gg]);
       }
-      // P' operand of tile jt: wait until the PV of tile jt - NR has been read
-      if (jt >= C::NR && !wait_bar(&S.pv_free[pb], ((jt / C::NR) & 1) ^ 1, &S.abort_flag, status)) break;
-      // column n = group * 4G + head * 4 + byte: one u32 per (group, head),
-      // 22-bit fixed point p * scale * 2^F
-      uint8_t *row = S.bp[pb] + (t >> 3) * 128 + (t & 7) * 16;
+
+      // 7. P' operand: column n = group * 4G + head * 4 + byte, one u32 per
+      //    (group, head) holding p * scale * 2^F as 22-bit fixed point
+      {
+        uint8_t *row = S.bp[rb] + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
-      for (int c = 0; c < G; ++c) {
-        uint32_t w4[4];
+        for (int c = 0; c < G; ++c) {
+          uint32_t w4[4];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
-          w4[x] = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
+          for (int x = 0; x < 4; ++x) {
+            const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
+            w4[x] = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
+          }
+          *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      if (t == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) S.alpha[pb][g] = alpha[g];
-        S.pscale[pb] = mscale > 0.f ? exp2i(-F) : 0.f;
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.p_ready[pb]);
+      if (lane == 0) mbar_arrive(&S.p_ready[rb]);
+
+      // 8. P.V read-back (now, or at this group's next tile)
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) dal[g] = alpha[g];
+        dal[G] = mscale > 0.f ? exp2i(-F) : 0.f;
+      }
+      __syncwarp();
+      if constexpr (C::OWN_SLOT) {
+        prev = i;
+      } else {
+        if (!readback(i, rb)) break;
+      }
+      ok = true;
     }
-    // l and the zero-point sums over this group's tokens, and its max
+    if constexpr (C::OWN_SLOT) {
+      if (ok && prev >= 0) ok = readback(prev, prev % C::NR);
+    }
+
+    // merge the four groups' states; unnormalised partial output
+    // sum_t p_t (code * scale + zero) of the split
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float l = warp_sum(lsum[g]);
@@ -765,8 +765,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         if (lane == 0) S.zsum[grp][q4][g][gg] = z;
       }
       if (t == 0) S.fin_m[grp][g] = mrun[g];
+      if (grp > 0) S.accx[grp - 1][t][g] = acc[g];
     }
-    named_bar_sync(3, 384);  // publish to the value group
+    named_bar_sync(1, 32 * 4 * kWorkGroups);
+    if (grp == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float mm = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kWorkGroups; ++k) mm = fmaxf(mm, S.fin_m[k][g]);
+        float o = 0.f, lt = 0.f;
+#pragma unroll
+        for (int k = 0; k < kWorkGroups; ++k) {
+          const float mk = S.fin_m[k][g];
+          const float f = (mk == -INFINITY) ? 0.f : exp2f(mk - mm);
+          float z = 0.f, l = 0.f;
+#pragma unroll
+          for (int wq = 0; wq < 4; ++wq) {
+            z += S.zsum[k][wq][g][q4];
+            l += S.lsum[k][wq][g];
+          }
+          const float ak = k == 0 ? acc[g] : S.accx[k - 1][t][g];
+          o = fmaf(ak + z, f, o);
+          lt = fmaf(l, f, lt);
+        }
+        float *pr = part_row(g);
+        pr[chan] = o;
+        if (t == 0) {
+          // m (log2 units, as the SIMT path) and l of the split
+          pr[kD] = mm;
+          pr[kD + 1] = lt;
+        }
+      }
+    }
   }
 
   tc_fence_before();
@@ -894,11 +925,9 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
       if (tid == 0) {
         // spins are 2 bit - 1: the -1 halves are constants per head
         qc->cm[g] = (wal[0] - wsum) * sq;
-        qc->csum[g] = ss;
-        qc->coef_m[g][0] = ldexpf(1.f, -fm[g]);
-        qc->coef_m[g][1] = ldexpf(1.f, 14 - fm[g]);
-        qc->coef_s[g][0] = ldexpf(1.f, -fs[g]);
-        qc->coef_s[g][1] = ldexpf(1.f, 14 - fs[g]);
+        qc->ncsum[g] = -ss;
+        qc->fm[g] = ldexpf(1.f, -fm[g]);
+        qc->fs[g] = ldexpf(1.f, -fs[g]);
       }
     }
     if (tid == 0) {
