@@ -180,7 +180,9 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
   float num = 0.f, den = 0.f;
   if (M != -INFINITY) {
     for (int s = 0; s < a.part_stride; ++s) {
-      const float f = exp2f(src[s * (kD + 2) + kD] - M);
+      const float ms = src[s * (kD + 2) + kD];
+      if (ms == -INFINITY) continue;  // empty split
+      const float f = exp2f(ms - M);
       num = fmaf(src[s * (kD + 2) + j], f, num);
       den = fmaf(src[s * (kD + 2) + kD + 1], f, den);
     }
@@ -306,7 +308,8 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   DecodePlan P;
   const int ntile = (max_len + kTile - 1) / kTile;
   const long long units = (long long)batch * h_kv;
-  const long long target = 4LL * num_sms;
+  // about two CTAs per SM: fewer, longer CTAs amortise each CTA's pipeline fill
+  const long long target = 2LL * num_sms;
   long long ns = (target + units - 1) / units;
   ns = std::max(1LL, std::min(ns, (long long)std::max(ntile, 1)));
   int tps = ntile > 0 ? (int)((ntile + ns - 1) / ns) : 0;

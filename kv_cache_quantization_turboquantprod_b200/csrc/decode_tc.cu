@@ -263,7 +263,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   TcSmem<C> &S = *reinterpret_cast<TcSmem<C> *>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // split-major grid: every unit's first splits are scheduled before any
+  // last (ragged, shorter) split, so the short CTAs fill the tail
+  const int split = blockIdx.z, h = blockIdx.x, b = blockIdx.y;
 
   int len = a.len[b];
   len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
@@ -992,7 +994,7 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
   qblock_kernel<MB, VB, G><<<qgrid, 256, qsmem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 grid(a.nsplit, a.h_kv, a.batch);
+  dim3 grid(a.h_kv, a.batch, a.nsplit);
   decode_tc_kernel<MB, VB, G><<<grid, kTcThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
