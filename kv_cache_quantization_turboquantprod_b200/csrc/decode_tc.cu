@@ -20,7 +20,7 @@
 //   m = 1, 2, 3).  A spin is 2 bit - 1, so each subset plane and the QJL sign
 //   plane enter as 0/1 bits (the -1 halves are per-head constants).  One LOP3
 //   (w & (0x01010101 << k)) turns a 32-bit plane word into four u8 operands
-//   of weight 2^k; the key group stores them straight into tensor memory, so
+//   of weight 2^k; the worker groups store them straight into tensor memory, so
 //   the score operands never touch shared memory.  The query side B holds
 //   2 a_S Pi q / 2^k (and 2 S q / 2^k) in four signed base-128 limbs; the s32
 //   accumulation is exact and the limbs are combined per (token, head).
