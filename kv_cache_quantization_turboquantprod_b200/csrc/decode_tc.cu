@@ -33,10 +33,10 @@
 // Per 128-token tile the record bytes arrive by one 1-D bulk copy (TMA
 // engine) into a ring of shared-memory stages.
 //
-// Warp roles (576 threads):
+// Warp roles (608 threads):
 //   warp 0        bulk-copy producer; allocates / frees tensor memory
-//   warp 1        MMA issuer (one elected lane issues), polling the score
-//                 and PV queues so neither blocks the other
+//   warp 1        score MMA issuer, warp 18 P.V MMA issuer (one elected lane
+//                 issues); each sleeps in blocking waits on its own queue
 //   warps 2-17    four worker groups of four warps (one per TMEM lane
 //                 quarter); group g takes tiles g, g + 4, ... through every
 //                 SIMT step: plane operands -> tensor memory, value codes ->
@@ -61,11 +61,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 576;
+constexpr int kTcThreads = 608;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTmemCols = 512;
 constexpr int kPlaneCols = 32;  // one u8 operand plane: 128 coordinates per row = 32 TMEM columns
 constexpr int kWorkGroups = 4;  // worker groups of 4 warps; group g takes tiles g, g + 4, ...
+constexpr int kPvWarp = 18;     // the P.V MMA issuer (warps 2 .. 17 are the worker groups)
 
 // 2^n for n in [-126, 127]
 __device__ __forceinline__ float exp2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
@@ -337,31 +338,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       for (int i = max(0, issued - C::STAGES); i < issued; ++i)
         mbar_wait(&S.full[i % C::STAGES], (i / C::STAGES) & 1);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ------------------------------------------
-    // The whole warp runs the loop, so queue tests and descriptor arithmetic
-    // stay warp-uniform; one elected lane issues each tcgen05 instruction.
-    // It polls both queues (score of tile is, PV of tile ip) with
-    // non-blocking tests and issues whichever is ready.
+  } else if (warp == 1 || warp == kPvWarp) {
+    // ---------------- MMA issuers -----------------------------------------
+    // Warp 1 issues the score MMAs of tiles 0, 1, ..., warp kPvWarp the P.V
+    // MMAs; each sleeps in blocking mbarrier waits for its own queue, so
+    // neither spends issue slots of the sub-partitions it shares with the
+    // worker groups, and neither waits behind the other.  The whole warp
+    // runs the loop (descriptors stay warp-uniform); one elected lane issues.
     const bool leader = elect_one();
-    const uint32_t id_s = idesc_i8(128, C::NS, false, true, false, false);
-    const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
-    const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
-    const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
-    const int akb = C::ak_ring(npl);
-    const uint64_t dbq = smem_desc(S.bq, C::LBO_Q, 128);
-    const uint64_t dav0 = smem_desc(S.av[0], 128, C::SBO_V), dbp0 = smem_desc(S.bp[0], 128, C::SBO_V);
-    int is = 0, ip = 0;
-    uint32_t idle = 0;
-    uint64_t t_idle = 0;
-    while (qok && ip < ntile) {
-      bool progress = false;
-      const int ab = akb == 2 ? (is & 1) : 0;
-      const uint32_t aph = akb == 2 ? ((is >> 1) & 1) : (is & 1);
-      bool rs = is < ntile && mbar_test(&S.ak_ready[ab], aph) &&
-                (is < 2 || mbar_test(&S.s_free[is & 1], ((is - 2) >> 1) & 1));
-      rs = __shfl_sync(0xffffffffu, rs, 0);
-      if (rs) {
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, &S.abort_flag, status));
+    };
+    const bool qok = wait_all(&S.q_full, 0);
+    int last = -1;  // last tile whose MMAs were committed
+    if (warp == 1) {
+      const uint32_t id_s = idesc_i8(128, C::NS, false, true, false, false);
+      const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
+      const int akb = C::ak_ring(npl);
+      const uint64_t dbq = smem_desc(S.bq, C::LBO_Q, 128);
+      for (int is = 0; qok && is < ntile; ++is) {
+        const int ab = akb == 2 ? (is & 1) : 0;
+        const uint32_t aph = akb == 2 ? ((is >> 1) & 1) : (is & 1);
+        if (!wait_all(&S.ak_ready[ab], aph)) break;
+        if (is >= 2 && !wait_all(&S.s_free[is & 1], ((is - 2) >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t d_mse = tbase + C::COL_DS + (is & 1) * 2 * C::NS;
         const uint32_t d_qjl = d_mse + C::NS;
@@ -384,17 +383,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         }
         if (leader) mma_commit(&S.s_ready[is & 1]);
         __syncwarp();
-        ++is;
-        progress = true;
+        last = is;
       }
-      const int rb = ip % C::NR;
-      const uint32_t rph = (ip / C::NR) & 1;
-      bool rp = ip < is && mbar_test(&S.p_ready[rb], rph) && mbar_test(&S.av_ready[rb], rph) &&
-                (ip < C::NR || mbar_test(&S.pv_free[rb], rph ^ 1));
-      rp = __shfl_sync(0xffffffffu, rp, 0);
-      if (rp) {
+      // never leave with an MMA in flight
+      if (last >= 0) mbar_wait(&S.s_ready[last & 1], (last >> 1) & 1);
+    } else {
+      const uint32_t id_p = idesc_i8(128, C::NPV, false, false, true, true);
+      const uint64_t dav0 = smem_desc(S.av[0], 128, C::SBO_V), dbp0 = smem_desc(S.bp[0], 128, C::SBO_V);
+      for (int ip = 0; qok && ip < ntile; ++ip) {
+        const int pb = ip % C::NR;
+        const uint32_t rph = (ip / C::NR) & 1;
+        if (!wait_all(&S.p_ready[pb], rph)) break;
+        if (!wait_all(&S.av_ready[pb], rph)) break;
+        if (ip >= C::NR && !wait_all(&S.pv_free[pb], rph ^ 1)) break;
         tc_fence_after();
-        const int pb = rb;
         const uint32_t d_pv = tbase + C::COL_DPV + pb * C::NPV;
         const uint64_t da = dav0 + (uint64_t)((pb * C::AV_BYTES) >> 4);
         const uint64_t db = dbp0 + (uint64_t)((pb * C::BP_BYTES) >> 4);
@@ -403,31 +405,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           if (leader) mma_i8_ss(d_pv, da + (uint64_t)(32 * ins), db + (uint64_t)(32 * ins), id_p, ins ? 1u : 0u);
         if (leader) mma_commit(&S.pv_done[pb]);
         __syncwarp();
-        ++ip;
-        progress = true;
+        last = ip;
       }
-      if (progress) {
-        idle = 0;
-        t_idle = 0;
-      } else if ((++idle & 15u) != 0) {
-        __nanosleep(32);  // yield the issue slots of this sub-partition
-      } else {  // the clock is read rarely
-        if (S.abort_flag) break;
-        const uint64_t now = globaltimer_ns();
-        if (t_idle == 0) {
-          t_idle = now;
-        } else if (now - t_idle > 2000000000ull) {
-          if (leader) {
-            S.abort_flag = 1;
-            atomicOr(status, 1);
-          }
-          break;
-        }
-      }
+      if (last >= 0) mbar_wait(&S.pv_done[last % C::NR], (last / C::NR) & 1);
     }
-    // never leave with an MMA in flight
-    if (is > 0) mbar_wait(&S.s_ready[(is - 1) & 1], ((is - 1) >> 1) & 1);
-    if (ip > 0) mbar_wait(&S.pv_done[(ip - 1) % C::NR], ((ip - 1) / C::NR) & 1);
   } else {
     // ---------------- worker groups ----------------------------------------
     // Group grp (warps 2 + 4 grp .. 5 + 4 grp, one per TMEM lane quarter)
