@@ -535,16 +535,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         }
       }
 
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.ak_ready[ab]);
+
       // 3. the P.V slot: its last tile's operands must have been consumed
+      //    (after the planes are handed over, so the score MMA starts first)
       if constexpr (C::OWN_SLOT) {
         if (prev >= 0 && !readback(prev, rb)) break;
       } else {
         if (i >= C::NR && !wait_bar(&S.pv_done[rb], ((i - C::NR) / C::NR) & 1, &S.abort_flag, status)) break;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.ak_ready[ab]);
 
       // 4. value codes, norms and value scales; the stage is then released
       uint32_t vw[NVW];
@@ -607,24 +609,42 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       float mse[G], qjl[G];
       {
         const uint32_t base = tbase + lane_off + C::COL_DS + (i & 1) * 2 * C::NS;
-        uint32_t d[4 * G];
-        tmem_ld_cols<4 * G>(base, d);
-        tmem_wait_ld();
+        if constexpr (4 * G == C::NS && G <= 4) {
+          // the MSE and QJL accumulators are adjacent: one load for both
+          uint32_t d[8 * G];
+          tmem_ld_cols<8 * G>(base, d);
+          tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const int am = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
-          const int bm = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
-          const float fm = Q.fm[g];
-          mse[g] = fmaf(fm * 16384.f, (float)bm, fmaf(fm, (float)am, Q.cm[g]));
-        }
-        tmem_ld_cols<4 * G>(base + C::NS, d);
-        tmem_wait_ld();
+          for (int g = 0; g < G; ++g) {
+            const int am = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
+            const int bm = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
+            const float fm = Q.fm[g];
+            mse[g] = fmaf(fm * 16384.f, (float)bm, fmaf(fm, (float)am, Q.cm[g]));
+            const int as = (int)d[4 * G + 4 * g] + 128 * (int)d[4 * G + 4 * g + 1];
+            const int bs = (int)d[4 * G + 4 * g + 2] + 128 * (int)d[4 * G + 4 * g + 3];
+            const float fs = Q.fs[g];
+            qjl[g] = fmaf(fs * 16384.f, (float)bs, fmaf(fs, (float)as, Q.ncsum[g]));
+          }
+        } else {
+          uint32_t d[4 * G];
+          tmem_ld_cols<4 * G>(base, d);
+          tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const int as = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
-          const int bs = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
-          const float fs = Q.fs[g];
-          qjl[g] = fmaf(fs * 16384.f, (float)bs, fmaf(fs, (float)as, Q.ncsum[g]));
+          for (int g = 0; g < G; ++g) {
+            const int am = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
+            const int bm = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
+            const float fm = Q.fm[g];
+            mse[g] = fmaf(fm * 16384.f, (float)bm, fmaf(fm, (float)am, Q.cm[g]));
+          }
+          tmem_ld_cols<4 * G>(base + C::NS, d);
+          tmem_wait_ld();
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const int as = (int)d[4 * g] + 128 * (int)d[4 * g + 1];
+            const int bs = (int)d[4 * g + 2] + 128 * (int)d[4 * g + 3];
+            const float fs = Q.fs[g];
+            qjl[g] = fmaf(fs * 16384.f, (float)bs, fmaf(fs, (float)as, Q.ncsum[g]));
+          }
         }
       }
       tc_fence_before();
