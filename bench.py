@@ -332,6 +332,7 @@ def run_ours(args, rank, world, device):
     if world == 1:
         line["window"] = bench_window(layer, cache, q, len_after, max_len, out, ws, wl, device,
                                       dec_bytes_all, dec_ms)
+        line["prefill"] = bench_prefill(layer, cache, len_after, max_len, wl, device, dec_bytes_all)
     if args.quantize and world == 1:
         line["quantize"] = bench_quantize(args, device)
     return line
@@ -361,6 +362,42 @@ def bench_window(layer, cache, q, len_dev, max_len, out, ws, wl, device, dec_byt
     return {"win_cap": 128, "decode_ms": ms, "decode_ms_without_window": dec_ms,
             "gbs": (dec_bytes + win_bytes) / (ms / 1e3) / 1e9,
             "window_bytes": win_bytes}
+
+
+def bench_prefill(layer, cache, len_dev, max_len, wl, device, dec_bytes, t_chunk=8):
+    """Causal prefill of an 8-token chunk per sequence over the same cache (the
+    chunk taken as the cache's last 8 tokens): each pass of the library's
+    tokens-per-pass streams the records once.  Reports query tokens/s and the
+    record bytes streamed per second."""
+    B, HQ, D = wl.batch, wl.h_q, wl.d
+    gen = torch.Generator(device=device)
+    gen.manual_seed(777)
+    qp = torch.randn((B, t_chunk, HQ, D), generator=gen, device=device).to(torch.bfloat16)
+    out = torch.empty((B, t_chunk, HQ, D), dtype=torch.float32, device=device)
+    ws = tq.prefill_workspace_for(layer, cache, HQ, t_chunk, max_len, device=device)
+    for _ in range(3):
+        tq.tq_prefill_attention(layer, cache, qp, len_dev, max_len, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 10
+    e0.record()
+    for _ in range(n):
+        tq.tq_prefill_attention(layer, cache, qp, len_dev, max_len, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    per_pass = tq.tq_prefill_tokens_per_pass(layer, HQ, wl.h_kv, t_chunk)
+    passes = 0
+    left = t_chunk
+    while left > 0:  # passes of per_pass tokens, the last of the largest power of two left
+        n = per_pass
+        while n > left:
+            n //= 2
+        left -= n
+        passes += 1
+    return {"t_chunk": t_chunk, "tokens_per_pass": per_pass, "passes": passes, "ms": ms,
+            "query_tokens_s": B * t_chunk / (ms / 1e3),
+            "record_gbs": passes * dec_bytes / (ms / 1e3) / 1e9}
 
 
 def bench_quantize(args, device):

@@ -235,6 +235,49 @@ TQ_API tq_status tq_decode_attention_window(const tq_params *p, const tq_cache *
                                      void *workspace, size_t workspace_bytes,
                                      tq_stream_t stream);
 
+/*
+ * Workspace bytes tq_prefill_attention needs for these shapes.  0 for bad
+ * arguments.
+ */
+TQ_API size_t tq_prefill_workspace_size(const tq_params *p, const tq_cache *c,
+                                 int h_q, int t_chunk, int max_len);
+
+/*
+ * Query tokens one pass of tq_prefill_attention takes together for these
+ * shapes (each pass streams the compressed records once): a power of two,
+ * 1 when no wider tensor-core shape is built.  0 for bad arguments.
+ */
+TQ_API int tq_prefill_tokens_per_pass(const tq_params *p, int h_q, int h_kv, int t_chunk);
+
+/*
+ * tq_prefill_attention -- causal attention of a chunk of t_chunk query
+ * tokens per sequence over the compressed cache, after the chunk's own keys
+ * and values were appended ("turboquant/audit_claims.py", AUDIT 7 and 8:
+ * long-context prefill as scaled-dot-product attention with a causal mask
+ * over the stored cache; here the stored cache is the compressed one, read
+ * in place).  Query token t of the chunk (0-based) of sequence b attends to
+ * the first len_dev[b] - (t_chunk - 1 - t) cached tokens, with the decode
+ * estimator of tq_decode_attention.  Passes of up to 8 / (h_q / h_kv) query
+ * tokens (a power of two the tensor-core kernel is built for) share every
+ * streamed KV tile: the chunk's tokens join the query heads of a KV head.
+ *
+ *   q              device, [batch][t_chunk][h_q][d], q_dtype (F32 or BF16)
+ *   t_chunk        query tokens per sequence, 1 <= t_chunk <= max_len
+ *   len_dev        device, [batch] int32: cached tokens of each sequence,
+ *                  the chunk included (len_dev[b] >= t_chunk expected; a
+ *                  query token that sees no token gets a zero row)
+ *   max_len        host: an upper bound of every len_dev[b]
+ *   out            device, [batch][t_chunk][h_q][d] fp32
+ *   workspace      device, >= tq_prefill_workspace_size(p, c, h_q,
+ *                  t_chunk, max_len) bytes, 256-byte aligned
+ * The other arguments and the errors are tq_decode_attention's.
+ */
+TQ_API tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c,
+                               const void *q, tq_dtype q_dtype, int h_q, int t_chunk,
+                               const int32_t *len_dev, int max_len, float softmax_scale,
+                               float *out, void *workspace, size_t workspace_bytes,
+                               tq_stream_t stream);
+
 /* Size of the fixed device scratch tq_decode_attention_noalloc uses. */
 #define TQ_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 

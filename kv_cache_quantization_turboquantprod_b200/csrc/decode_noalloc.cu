@@ -94,6 +94,7 @@ extern "C" tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_ca
   a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
   a.part_stride = P.nsplit;
   a.win_k = nullptr; a.win_v = nullptr; a.win_dtype = TQ_BF16; a.win_len = nullptr; a.win_cap = 0;
+  a.qt = 1; a.q_tstride = 1; a.q_t0 = 0; a.len_sub = 0;
   a.num_sms = sms;
   tq::bind_workspace(a, P, scratch);
   a.out = out;

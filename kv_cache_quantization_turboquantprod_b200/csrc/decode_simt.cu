@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(256) qprep_kernel(DecodeArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float qv[4];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) qv[m] = load_elem(a.q, a.q_dtype, (size_t)bh * kD + lane + 32 * m);
+  for (int m = 0; m < 4; ++m) qv[m] = load_elem(a.q, a.q_dtype, qrow_offset(a, bh / a.h_q, bh % a.h_q) + lane + 32 * m);
   float *dst = a.qrot + (size_t)bh * 2 * kD;
   for (int o = warp; o < 2 * kD; o += 8) {
     const float *row = (o < kD) ? (a.pi + (size_t)o * kD) : (a.s + (size_t)(o - kD) * kD);
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
   }
   __syncthreads();
 
-  int len = a.len[b];
+  int len = a.len[b] - a.len_sub;
   len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
   const int t0 = s * a.tiles_per_split * kTile;
   const int t1 = min(len, (s + 1) * a.tiles_per_split * kTile);
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
       den = fmaf(src[s * (kD + 2) + kD + 1], f, den);
     }
   }
-  a.out[(size_t)bh * kD + j] = den > 0.f ? num / den : 0.f;
+  a.out[qrow_offset(a, bh / a.h_q, bh % a.h_q) + j] = den > 0.f ? num / den : 0.f;
 }
 
 // ---------------------------------------------------------------------------

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   // last (ragged, shorter) split, so the short CTAs fill the tail
   const int split = blockIdx.z, h = blockIdx.x, b = blockIdx.y;
 
-  int len = a.len[b];
+  int len = a.len[b] - a.len_sub;
   len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
   const int tile0 = split * a.tiles_per_split;
   const int t_begin = tile0 * kTile;
@@ -358,8 +358,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       const uint64_t dbq = smem_desc(S.bq, C::LBO_Q, 128);
       for (int is = 0; qok && is < ntile; ++is) {
         const int ab = akb == 2 ? (is & 1) : 0;
-        const uint32_t aph = akb == 2 ? ((is >> 1) & 1) : (is & 1);
-        if (!wait_all(&S.ak_ready[ab], aph)) break;
+        // one hand-over barrier per tile parity, also with a single A_k
+        // buffer (one barrier completing every tile stalled at GQA 8)
+        if (!wait_all(&S.ak_ready[is & 1], (is >> 1) & 1)) break;
         if (is >= 2 && !wait_all(&S.s_free[is & 1], ((is - 2) >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t d_mse = tbase + C::COL_DS + (is & 1) * 2 * C::NS;
@@ -435,6 +436,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
     for (int p = 0; p < C::NSYM; ++p) sym = sym && Q.subset[p] == odd_subset(p);
 
+    const int qt1 = a.qt - 1, gshift = 31 - __clz(G / a.qt);
     float mrun[G], lsum[G], zs[G][4], acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -497,6 +499,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       if (i >= akb) {
         const int pt = i - akb;
         if (!wait_bar(&S.s_ready[pt & 1], (pt >> 1) & 1, &S.abort_flag, status)) break;
+        // the stores below must follow the MMA's reads of the buffer
+        tc_fence_after();
       }
       const int ab = akb == 2 ? (i & 1) : 0;
       {
@@ -538,7 +542,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.ak_ready[ab]);
+      if (lane == 0) mbar_arrive(&S.ak_ready[i & 1]);
 
       // 3. the P.V slot: its last tile's operands must have been consumed
       //    (after the planes are handed over, so the score MMA starts first)
@@ -652,7 +656,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       if (lane == 0) mbar_arrive(&S.s_free[i & 1]);
 
       // 6. logits, tile maxima over the group's 128 tokens, online softmax
-      const bool valid = t_begin + i * kTile + t < t_end;
+      const int tpos = t_begin + i * kTile + t;
+      const bool valid = tpos < t_end;
       const __half2 nr = *reinterpret_cast<const __half2 *>(&nrw);
       const float nk = __low2float(nr), rn = __high2float(nr);
       const __half2 *szh = reinterpret_cast<const __half2 *>(&szr);
@@ -669,7 +674,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float score = nk * fmaf(krn, qjl[g], mse[g]);
-        lg[g] = valid ? score * scale2 : -INFINITY;
+        // prefill: query token g >> gshift of the chunk sees len - (qt - 1 - that) tokens
+        lg[g] = (valid && tpos + qt1 - (g >> gshift) < len) ? score * scale2 : -INFINITY;
       }
       float(&red)[G + 1][4] = S.red[grp][n & 1];
 #pragma unroll
@@ -713,7 +719,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       float p[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        p[g] = valid ? exp2f(lg[g] - mrun[g]) : 0.f;
+        p[g] = lg[g] != -INFINITY ? exp2f(lg[g] - mrun[g]) : 0.f;
         lsum[g] += p[g];
 #pragma unroll
         for (int gg = 0; gg < 4; ++gg) zs[g][gg] = fmaf(p[g], vze[gg], zs[g][gg]);
@@ -884,7 +890,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int b = u / a.h_kv, h = u % a.h_kv;
     for (int i = tid; i < G * kD; i += 256)
-      qv[i] = load_elem(a.q, a.q_dtype, ((size_t)b * a.h_q + (size_t)h * G) * kD + i);
+      qv[i] = load_elem(a.q, a.q_dtype, qrow_offset(a, b, h * G + i / kD) + i % kD);
     __syncthreads();
     {  // thread o rotates row o of [Pi; S] against the G queries
       const int o = tid;
@@ -1006,6 +1012,9 @@ size_t decode_tc_qblock_bytes(int key_bits, int G) { return qblock_bytes_for(key
 
 bool decode_tc_supported(int key_bits, int value_bits, int G) {
   const int mb = key_bits - 1;
+  // 2-bit codes at GQA 8 leave room for one A_k buffer only; that schedule
+  // stalled or raced on long splits, so the shape runs on the SIMT kernel
+  if (value_bits == 2 && mb == 2 && G == 8) return false;
   if (value_bits == 2 && (G == 1 || G == 2 || G == 4 || G == 8) && (mb == 1 || mb == 2)) return true;
   if (value_bits == 2 && mb == 3 && G == 4) return true;
   if (value_bits == 3 && mb == 2 && G == 6) return true;

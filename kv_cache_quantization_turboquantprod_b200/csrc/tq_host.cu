@@ -169,6 +169,86 @@ size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, 
 
 namespace {
 
+// Query tokens of a prefill chunk that one decode pass takes together: the
+// largest power of two ts <= t_chunk with G * ts <= 8 that the tensor-core
+// kernel builds (so the pass reads every KV tile once for ts tokens), else 1.
+int prefill_tokens_per_pass(const tq_params *p, int gqa, int t_chunk) {
+  int ts = 1;
+  while (2 * ts <= t_chunk && gqa * 2 * ts <= 8 &&
+         tq::decode_tc_supported(p->key_bits, p->value_bits, gqa * 2 * ts))
+    ts *= 2;
+  return ts;
+}
+
+}  // namespace
+
+int tq_prefill_tokens_per_pass(const tq_params *p, int h_q, int h_kv, int t_chunk) {
+  if (check_params(p) != TQ_OK || h_kv < 1 || h_q < h_kv || h_q % h_kv || t_chunk < 1) return 0;
+  return prefill_tokens_per_pass(p, h_q / h_kv, t_chunk);
+}
+
+size_t tq_prefill_workspace_size(const tq_params *p, const tq_cache *c, int h_q, int t_chunk,
+                                 int max_len) {
+  if (check_params(p) != TQ_OK || check_cache(c) != TQ_OK) return 0;
+  if (h_q < c->h_kv || h_q % c->h_kv || t_chunk < 1 || max_len < t_chunk || max_len > c->capacity)
+    return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != cudaSuccess) return 0;
+  const int ts = prefill_tokens_per_pass(p, h_q / c->h_kv, t_chunk);
+  return tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits, p->value_bits)
+      .total_bytes;
+}
+
+tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void *q, tq_dtype q_dtype,
+                               int h_q, int t_chunk, const int32_t *len_dev, int max_len,
+                               float softmax_scale, float *out, void *workspace, size_t workspace_bytes,
+                               tq_stream_t stream) {
+  tq_status st = check_params(p);
+  if (st != TQ_OK) return st;
+  if ((st = check_cache(c)) != TQ_OK) return st;
+  if (!dtype_ok(q_dtype)) return TQ_ERR_UNSUPPORTED;
+  if (!q || !len_dev || !out) return TQ_ERR_INVALID_ARGUMENT;
+  if (h_q < c->h_kv || h_q % c->h_kv) return TQ_ERR_INVALID_ARGUMENT;
+  if (h_q / c->h_kv > 8) return TQ_ERR_UNSUPPORTED;
+  if (t_chunk < 1 || max_len < t_chunk || max_len > c->capacity) return TQ_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(softmax_scale)) return TQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(len_dev, 4)) return TQ_ERR_INVALID_ARGUMENT;
+  if (!workspace || !aligned(workspace, 256)) return TQ_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
+  const int G = h_q / c->h_kv;
+  const int ts = prefill_tokens_per_pass(p, G, t_chunk);
+  if (workspace_bytes < tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits,
+                                             p->value_bits).total_bytes)
+    return TQ_ERR_WORKSPACE;
+  // passes of ts tokens (the last one of the largest power of two that is
+  // left); pass tokens t0 .. t0 + n - 1 see len - (t_chunk - 1 - t) tokens
+  for (int t0 = 0; t0 < t_chunk;) {
+    int n = ts;
+    while (n > t_chunk - t0) n >>= 1;
+    const int len_sub = t_chunk - t0 - n;
+    const int ml = max_len - len_sub;
+    const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q * n, ml, sms, p->key_bits, p->value_bits);
+    tq::DecodeArgs a;
+    a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
+    a.data = c->data; a.q = q; a.q_dtype = q_dtype; a.len = len_dev;
+    a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q * n; a.ntiles = c->capacity / kTile;
+    a.max_len = ml; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
+    a.softmax_scale = softmax_scale; a.nsplit = P.nsplit; a.tiles_per_split = P.tiles_per_split;
+    a.part_stride = P.nsplit;
+    a.win_k = nullptr; a.win_v = nullptr; a.win_dtype = TQ_BF16; a.win_len = nullptr; a.win_cap = 0;
+    a.qt = n; a.q_tstride = t_chunk; a.q_t0 = t0; a.len_sub = len_sub;
+    a.num_sms = sms;
+    tq::bind_workspace(a, P, workspace);
+    a.out = out;
+    if (tq::launch_decode(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+    t0 += n;
+  }
+  return TQ_OK;
+}
+
+namespace {
+
 // Shared by tq_decode_attention and tq_decode_attention_window (win_k null:
 // no window).
 tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq_dtype q_dtype,
@@ -206,6 +286,7 @@ tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq
   a.part_stride = win_k ? P.nsplit + 1 : P.nsplit;
   a.win_k = win_k; a.win_v = win_v; a.win_dtype = win_dtype; a.win_len = win_len_dev;
   a.win_cap = win_cap;
+  a.qt = 1; a.q_tstride = 1; a.q_t0 = 0; a.len_sub = 0;
   a.num_sms = sms;
   tq::bind_workspace(a, P, workspace);
   a.out = out;

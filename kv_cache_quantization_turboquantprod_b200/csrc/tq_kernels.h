@@ -64,7 +64,25 @@ struct DecodeArgs {
   uint8_t *qblocks;  // workspace: [B][H_kv] query blocks (tensor-core path)
   int num_sms;
   float *out;    // [B][H_q][d]
+  // Chunked prefill (qt > 1 or q_tstride > 1): the h_q heads of a sequence
+  // are qt query tokens x (h_q / qt) heads; q and out are [B][q_tstride][H][d]
+  // blocks (H = h_q / qt) of which this call covers tokens q_t0 .. q_t0 + qt
+  // - 1.  The call attends over len[b] - len_sub cache tokens; query token t
+  // of it sees the first len[b] - len_sub - (qt - 1 - t).  Decode: qt = 1,
+  // q_tstride = 1, q_t0 = 0, len_sub = 0.
+  int qt, q_tstride, q_t0, len_sub;
 };
+
+constexpr int kQRowElems = 128;  // elements per query / output row (d)
+
+// Element offset of virtual head hv's row of sequence b in q / out.  Virtual
+// heads of KV head h are h * G' + t * (G' / qt) + g (G' = h_q / h_kv).
+__host__ __device__ inline size_t qrow_offset(const DecodeArgs &a, int b, int hv) {
+  if (a.qt == 1 && a.q_tstride == 1) return ((size_t)b * a.h_q + hv) * kQRowElems;
+  const int gv = a.h_q / a.h_kv, greal = gv / a.qt, hreal = a.h_q / a.qt;
+  const int h = hv / gv, r = hv % gv, t = r / greal, g = r % greal;
+  return (((size_t)b * a.q_tstride + a.q_t0 + t) * hreal + (size_t)h * greal + g) * kQRowElems;
+}
 
 struct DequantArgs {
   const float *pi, *s, *centroids;

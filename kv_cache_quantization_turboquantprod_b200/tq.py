@@ -28,7 +28,8 @@ MAX_BATCH = 1024
 # Every function include/tq.h declares.
 EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_bytes",
            "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
-           "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window")
+           "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window",
+           "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass")
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -85,6 +86,12 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_decode_attention_window.restype = ci
     lib.tq_decode_attention_window.argtypes = [P, C, vp, ci, ci, vp, ci, vp, vp, ci, vp, ci,
                                                ctypes.c_float, vp, vp, sz, vp]
+    lib.tq_prefill_workspace_size.restype = sz
+    lib.tq_prefill_workspace_size.argtypes = [P, C, ci, ci, ci]
+    lib.tq_prefill_tokens_per_pass.restype = ci
+    lib.tq_prefill_tokens_per_pass.argtypes = [P, ci, ci, ci]
+    lib.tq_prefill_attention.restype = ci
+    lib.tq_prefill_attention.argtypes = [P, C, vp, ci, ci, ci, vp, ci, ctypes.c_float, vp, vp, sz, vp]
     lib.tq_dequantize.restype = ci
     lib.tq_dequantize.argtypes = [P, C, ci, ci, ci, vp, vp, vp]
     if path is None:
@@ -259,6 +266,44 @@ def tq_decode_attention_noalloc(layer: Layer, cache: CompressedCache, q: torch.T
                                             len_dev.data_ptr(), int(max_len), scale,
                                             out.data_ptr(), _stream(stream))
     _check("tq_decode_attention_noalloc", st)
+
+
+def tq_prefill_workspace_size(layer: Layer, cache: CompressedCache, h_q: int, t_chunk: int,
+                              max_len: int) -> int:
+    return int(load().tq_prefill_workspace_size(ctypes.byref(layer.params), ctypes.byref(cache.cache),
+                                                h_q, t_chunk, max_len))
+
+
+def tq_prefill_attention(layer: Layer, cache: CompressedCache, q: torch.Tensor,
+                         len_dev: torch.Tensor, max_len: int, out: torch.Tensor,
+                         workspace: torch.Tensor, softmax_scale: float | None = None,
+                         stream=None) -> None:
+    """Causal attention of a chunk over the compressed cache (the chunk already
+    appended): q [B, T, H_q, d] (fp32/bf16, contiguous), len_dev [B] int32
+    device (cached tokens, the chunk included), out [B, T, H_q, d] fp32."""
+    if len_dev.dtype != torch.int32:
+        raise TypeError("len_dev must be int32")
+    if not q.is_contiguous() or q.dim() != 4:
+        raise ValueError("q must be a contiguous [B, T, H_q, d] tensor")
+    scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().tq_prefill_attention(ctypes.byref(layer.params), ctypes.byref(cache.cache),
+                                     q.data_ptr(), _dtype_code(q), int(q.shape[2]), int(q.shape[1]),
+                                     len_dev.data_ptr(), int(max_len), scale, out.data_ptr(),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream(stream))
+    _check("tq_prefill_attention", st)
+
+
+def tq_prefill_tokens_per_pass(layer: Layer, h_q: int, h_kv: int, t_chunk: int) -> int:
+    return int(load().tq_prefill_tokens_per_pass(ctypes.byref(layer.params), h_q, h_kv, t_chunk))
+
+
+def prefill_workspace_for(layer: Layer, cache: CompressedCache, h_q: int, t_chunk: int,
+                          max_len: int, device="cuda") -> torch.Tensor:
+    n = tq_prefill_workspace_size(layer, cache, h_q, t_chunk, max_len)
+    if n == 0:
+        raise TQError("tq_prefill_workspace_size", 1)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def tq_dequantize(layer: Layer, cache: CompressedCache, b: int, start: int, count: int,

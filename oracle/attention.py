@@ -138,6 +138,33 @@ def decode_with_window(q: np.ndarray, rec: dict | None, win_k: np.ndarray, win_v
     return out
 
 
+def prefill_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
+                         softmax_scale: float | None = None) -> np.ndarray:
+    """Causal attention of a chunk of T query tokens over the compressed cache
+    of one sequence whose last T tokens are the chunk itself
+    ("turboquant/audit_claims.py", AUDIT 7 and 8: long-context prefill as
+    scaled-dot-product attention with a causal mask over the stored cache).
+    Query token t (0-based) sees the first N - (T - 1 - t) cached tokens and
+    is scored exactly as decode_one_sequence scores a decode query.
+
+    q   [T, H_q, d]
+    rec logical cache fields with a leading [N, H_kv] (N >= T)
+    Returns out [T, H_q, d] float64; a token that sees no cached token gets
+    zeros.
+    """
+    q = np.asarray(q, np.float64)
+    t_chunk = q.shape[0]
+    n = rec["nk16"].shape[0]
+    out = np.zeros(q.shape)
+    for t in range(t_chunk):
+        m = n - (t_chunk - 1 - t)
+        if m <= 0:
+            continue
+        sub = {k: v[:m] for k, v in rec.items()}
+        out[t] = decode_one_sequence(q[t], sub, pi, s, centroids, group, softmax_scale)
+    return out
+
+
 def brute_force_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids,
                              group: int, softmax_scale: float | None = None) -> np.ndarray:
     """softmax(K_hat q / sqrt d) V_hat over explicitly dequantized K and V

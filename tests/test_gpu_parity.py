@@ -440,3 +440,80 @@ def test_decode_with_recent_window(name, kb, vb, h_kv, h_q):
             assert np.all(got[b] == 0.0)
             continue
         assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, (name, b)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("h_kv,h_q,kb,t_chunk", [(2, 8, 3, 3), (2, 4, 3, 5), (2, 2, 3, 8), (2, 8, 4, 3), (1, 1, 3, 11)])
+def test_prefill_parity(h_kv, h_q, kb, t_chunk):
+    """Causal chunked prefill over the compressed cache: passes of 8 / G
+    query tokens (GQA 4 -> 2 tokens, GQA 2 -> 4, GQA 1 -> 8) plus a smaller
+    last pass, and single-token passes where the wider kernel is not built
+    (4-bit keys at GQA 8); ragged lengths, a sequence holding exactly the
+    chunk."""
+    import dataclasses
+    lengths = (t_chunk, 127, 129, 300)
+    wl = dataclasses.replace(workloads.llama8b(), batch=4, h_kv=h_kv, h_q=h_q, key_bits=kb,
+                             lengths=lengths, capacity=384, name=f"prefill_{h_kv}_{h_q}_{kb}_{t_chunk}")
+    glayer, olayer, spec = _setup(wl)
+    buf, encs = _oracle_cache(wl, olayer, spec, lengths)
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn((wl.batch, t_chunk, h_q, wl.d), generator=g).to(torch.bfloat16)
+    cache = tq.CompressedCache(glayer, wl.batch, wl.h_kv, wl.capacity)
+    cache.buffer.copy_(torch.from_numpy(buf))
+    len_dev = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    ml = max(lengths)
+    ws = tq.prefill_workspace_for(glayer, cache, h_q, t_chunk, ml)
+    out = torch.full((wl.batch, t_chunk, h_q, wl.d), float("nan"), dtype=torch.float32, device=DEV)
+    tq.tq_prefill_attention(glayer, cache, q.to(DEV).contiguous(), len_dev, ml, out, ws)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    for b in range(wl.batch):
+        kes, ves = encs[b]
+        for t in range(t_chunk):
+            m = lengths[b] - (t_chunk - 1 - t)
+            ref = pu.oracle_decode(olayer, q[b, t].float().numpy(), kes, ves, m)
+            assert pu.row_rel_err(got[b, t], ref) <= pu.REL_TOL, (b, t)
+
+
+@pytest.mark.parametrize("kb,vb,h_q", [(3, 2, 64), (2, 2, 64), (4, 2, 32), (3, 3, 48), (3, 2, 32)])
+def test_decode_long_splits_every_kernel_shape(kb, vb, h_q):
+    """Every tensor-core decode shape with many tiles per CTA (32 sequences x
+    8 KV heads x 4096 tokens: the split plan gives each CTA 16 tiles, four per
+    worker group): the call finishes well inside the kernels' 2 s wait
+    bound, and sampled rows match the oracle run on the device's own records."""
+    import dataclasses
+    import time
+    from oracle import attention
+    n, B, hkv = 4096, 32, 8
+    wl = dataclasses.replace(workloads.batched(), batch=B, h_kv=hkv, h_q=h_q, key_bits=kb,
+                             value_bits=vb, lengths=(n,) * B, capacity=n, name=f"long{kb}{vb}{h_q}")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, B, hkv, n)
+    g = torch.Generator(device=DEV).manual_seed(9)
+    for b0 in range(0, B, 8):
+        k = torch.randn((8, n, hkv, 128), generator=g, device=DEV).to(torch.bfloat16)
+        v = torch.randn((8, n, hkv, 128), generator=g, device=DEV).to(torch.bfloat16)
+        # sequences b0 .. b0 + 7 take n tokens, the others none
+        ks = torch.zeros((B, n, hkv, 128), dtype=torch.bfloat16, device=DEV)
+        vs = torch.zeros_like(ks)
+        ks[b0:b0 + 8], vs[b0:b0 + 8] = k, v
+        nnew = [n if b0 <= b < b0 + 8 else 0 for b in range(B)]
+        tq.tq_quantize_append(glayer, cache, ks, vs, [0] * B, nnew)
+        del ks, vs, k, v
+    q = torch.randn((B, h_q, 128), generator=g, device=DEV).to(torch.bfloat16)
+    len_dev = torch.full((B,), n, dtype=torch.int32, device=DEV)
+    ws = tq.workspace_for(glayer, cache, h_q, n)
+    out = torch.empty((B, h_q, 128), dtype=torch.float32, device=DEV)
+    tq.tq_decode_attention(glayer, cache, q, len_dev, n, out, ws)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    tq.tq_decode_attention(glayer, cache, q, len_dev, n, out, ws)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 0.5
+    buf = cache.buffer.cpu().numpy()
+    got = out.cpu().numpy()
+    for b in (0, B - 1):
+        rec = attention.stack_heads([spec.read(buf, b, h, 0, n) for h in range(hkv)])
+        ref = attention.decode_one_sequence(q[b].float().cpu().numpy(), rec, olayer.pi, olayer.s,
+                                            olayer.cent, olayer.group)
+        assert pu.row_rel_err(got[b], ref) <= pu.REL_TOL, b

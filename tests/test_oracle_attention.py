@@ -194,3 +194,57 @@ def test_window_nothing_cached_gives_zeros():
     empty = np.zeros((0, 2, 128))
     out = attention.decode_with_window(np.ones((2, 128)), None, empty, empty, None, None, None, 32)
     assert not out.any()
+
+
+# ---- chunked prefill over the compressed cache (causal) ----------------------
+
+def test_prefill_single_token_is_decode():
+    rec, pi, s, cent = _random_cache(40, 2, 128, 3, 2, 32, seed=7)
+    q = np.random.default_rng(8).standard_normal((1, 8, 128))
+    a = attention.prefill_one_sequence(q, rec, pi, s, cent, 32)
+    b = attention.decode_one_sequence(q[0], rec, pi, s, cent, 32)
+    assert np.array_equal(a[0], b)
+
+
+def test_prefill_equals_causal_brute_force():
+    # causal softmax over explicitly dequantized K/V, query t sees the first
+    # N - (T - 1 - t) tokens
+    n, hkv, hq, t_chunk = 30, 2, 4, 5
+    rec, pi, s, cent = _random_cache(n, hkv, 128, 3, 2, 32, seed=11)
+    q = np.random.default_rng(12).standard_normal((t_chunk, hq, 128))
+    got = attention.prefill_one_sequence(q, rec, pi, s, cent, 32)
+    g = hq // hkv
+    for t in range(t_chunk):
+        m = n - (t_chunk - 1 - t)
+        for h in range(hkv):
+            khat = attention.dequantize_keys(rec["idx"][:m, h], rec["sign"][:m, h], rec["nk16"][:m, h],
+                                             rec["rn16"][:m, h], pi, s, cent)
+            vhat = attention.dequantize_values(rec["codes"][:m, h], rec["scale16"][:m, h],
+                                               rec["zero16"][:m, h], 32)
+            for j in range(g):
+                logits = khat @ q[t, h * g + j] / math.sqrt(128)
+                w = np.exp(logits - logits.max())
+                ref = (w / w.sum()) @ vhat
+                assert np.max(np.abs(got[t, h * g + j] - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_prefill_is_causal():
+    n, t_chunk = 24, 4
+    rec, pi, s, cent = _random_cache(n, 1, 128, 3, 2, 32, seed=13)
+    q = np.random.default_rng(14).standard_normal((t_chunk, 2, 128))
+    a = attention.prefill_one_sequence(q, rec, pi, s, cent, 32)
+    # change the last cached token (the chunk's last one): only the last query sees it
+    rec2 = {k: v.copy() for k, v in rec.items()}
+    rec2["nk16"][-1] = rec2["nk16"][-1] * 2
+    rec2["codes"][-1] = (rec2["codes"][-1] + 1) % 4
+    b = attention.prefill_one_sequence(q, rec2, pi, s, cent, 32)
+    assert np.array_equal(a[:-1], b[:-1])
+    assert not np.array_equal(a[-1], b[-1])
+
+
+def test_prefill_token_seeing_nothing_is_zero():
+    rec, pi, s, cent = _random_cache(2, 1, 128, 3, 2, 32, seed=15)
+    q = np.random.default_rng(16).standard_normal((4, 1, 128))
+    out = attention.prefill_one_sequence(q, rec, pi, s, cent, 32)
+    assert np.all(out[:2] == 0.0)
+    assert np.all(np.isfinite(out)) and np.any(out[3] != 0.0)
