@@ -257,9 +257,10 @@ TQ_API int tq_prefill_tokens_per_pass(const tq_params *p, int h_q, int h_kv, int
  * over the stored cache; here the stored cache is the compressed one, read
  * in place).  Query token t of the chunk (0-based) of sequence b attends to
  * the first len_dev[b] - (t_chunk - 1 - t) cached tokens, with the decode
- * estimator of tq_decode_attention.  Passes of up to 8 / (h_q / h_kv) query
- * tokens (a power of two the tensor-core kernel is built for) share every
- * streamed KV tile: the chunk's tokens join the query heads of a KV head.
+ * estimator of tq_decode_attention.  Passes of up to 4 / (h_q / h_kv) query
+ * tokens (a power of two the tensor-core kernel is built for; one token at
+ * GQA 4 and above) share every streamed KV tile: the chunk's tokens join the
+ * query heads of a KV head.
  *
  *   q              device, [batch][t_chunk][h_q][d], q_dtype (F32 or BF16)
  *   t_chunk        query tokens per sequence, 1 <= t_chunk <= max_len

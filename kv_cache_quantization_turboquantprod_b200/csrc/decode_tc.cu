@@ -100,7 +100,10 @@ struct Cfg {
   // MSE planes of a symmetric codebook (the odd code-bit subsets)
   static constexpr int NSYM = MB == 1 ? 1 : (MB == 2 ? 2 : 4);
   static constexpr int NS = score_n(G);                 // score N per accumulator
-  static constexpr int NPV = 16 * G;                    // PV N: 4 groups x G heads x 4 bytes
+  // P' bytes per (value group, head): the 22-bit fixed point needs 3; at
+  // GQA 8 only 3 are stored, so two A_k buffers still fit in tensor memory
+  static constexpr int PB = (G == 8) ? 3 : 4;
+  static constexpr int NPV = 4 * G * PB;                // PV N: 4 groups x G heads x PB bytes
   static constexpr int NPL = max_planes(MB);            // operand planes, upper bound
   static constexpr int SYM_COLS = (NSYM + 1) * kPlaneCols;  // A_k of one tile, symmetric codebook
   // tensor memory: A_k planes | D_s (2 buffers x (mse, qjl)) | D_pv (NR buffers).
@@ -452,8 +455,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     auto readback = [&](int jt, int rb) -> bool {
       if (!wait_bar(&S.pv_done[rb], (jt / C::NR) & 1, &S.abort_flag, status)) return false;
       tc_fence_after();
-      uint32_t d[4 * G];
-      tmem_ld_cols<4 * G>(tbase + lane_off + C::COL_DPV + rb * C::NPV + q4 * 4 * G, d);
+      constexpr int PB = C::PB;
+      uint32_t d[PB * G];
+      tmem_ld_cols<PB * G>(tbase + lane_off + C::COL_DPV + rb * C::NPV + q4 * PB * G, d);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -461,8 +465,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       const float sc = dal[G] * exp2i(-kk);  // this M slot carries code * 4^m
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float v = fmaf(16777216.f, (float)d[4 * g + 3],
-                             fmaf(65536.f, (float)d[4 * g + 2], fmaf(256.f, (float)d[4 * g + 1], (float)d[4 * g])));
+        float v = fmaf(65536.f, (float)d[PB * g + 2], fmaf(256.f, (float)d[PB * g + 1], (float)d[PB * g]));
+        if constexpr (PB == 4) v = fmaf(16777216.f, (float)d[PB * g + 3], v);
         acc[g] = fmaf(acc[g], dal[g], v * sc);
       }
       return true;
@@ -725,19 +729,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         for (int gg = 0; gg < 4; ++gg) zs[g][gg] = fmaf(p[g], vze[gg], zs[g][gg]);
       }
 
-      // 7. P' operand: column n = group * 4G + head * 4 + byte, one u32 per
-      //    (group, head) holding p * scale * 2^F as 22-bit fixed point
+      // 7. P' operand: column n = (group * G + head) * PB + byte, the PB
+      //    low bytes of p * scale * 2^F as 22-bit fixed point
       {
         uint8_t *row = S.bp[rb] + (t >> 3) * 128 + (t & 7) * 16;
+        if constexpr (C::PB == 4) {
 #pragma unroll
-        for (int c = 0; c < G; ++c) {
-          uint32_t w4[4];
+          for (int c = 0; c < G; ++c) {
+            uint32_t w4[4];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
-            w4[x] = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
+            for (int x = 0; x < 4; ++x) {
+              const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
+              w4[x] = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
+            }
+            *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-          *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        } else {
+          // 3 bytes per value, packed back to back: 4G values -> 3G words
+          uint32_t w[3 * G];
+#pragma unroll
+          for (int k = 0; k < 3 * G; ++k) w[k] = 0u;
+#pragma unroll
+          for (int j = 0; j < 4 * G; ++j) {
+            const int gg = j / G, g = j % G;
+            const uint32_t v = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
+            const int pos = 3 * j, wi = pos >> 2, off = pos & 3;
+            w[wi] |= v << (8 * off);
+            if (off > 1) w[wi + 1] |= v >> (8 * (4 - off));
+          }
+#pragma unroll
+          for (int c = 0; c < 3 * G / 4; ++c)
+            *reinterpret_cast<uint4 *>(row + c * C::SBO_V) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
         }
       }
       fence_proxy_async_smem();
@@ -1012,9 +1035,6 @@ size_t decode_tc_qblock_bytes(int key_bits, int G) { return qblock_bytes_for(key
 
 bool decode_tc_supported(int key_bits, int value_bits, int G) {
   const int mb = key_bits - 1;
-  // 2-bit codes at GQA 8 leave room for one A_k buffer only; that schedule
-  // stalled or raced on long splits, so the shape runs on the SIMT kernel
-  if (value_bits == 2 && mb == 2 && G == 8) return false;
   if (value_bits == 2 && (G == 1 || G == 2 || G == 4 || G == 8) && (mb == 1 || mb == 2)) return true;
   if (value_bits == 2 && mb == 3 && G == 4) return true;
   if (value_bits == 3 && mb == 2 && G == 6) return true;

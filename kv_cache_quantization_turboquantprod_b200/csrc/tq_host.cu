@@ -170,11 +170,13 @@ size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, 
 namespace {
 
 // Query tokens of a prefill chunk that one decode pass takes together: the
-// largest power of two ts <= t_chunk with G * ts <= 8 that the tensor-core
+// largest power of two ts <= t_chunk with G * ts <= 4 that the tensor-core
 // kernel builds (so the pass reads every KV tile once for ts tokens), else 1.
+// Wider passes (8 heads per worker thread) measured slower per token than
+// single-token passes at GQA 4.
 int prefill_tokens_per_pass(const tq_params *p, int gqa, int t_chunk) {
   int ts = 1;
-  while (2 * ts <= t_chunk && gqa * 2 * ts <= 8 &&
+  while (2 * ts <= t_chunk && gqa * 2 * ts <= 4 &&
          tq::decode_tc_supported(p->key_bits, p->value_bits, gqa * 2 * ts))
     ts *= 2;
   return ts;

@@ -445,11 +445,10 @@ def test_decode_with_recent_window(name, kb, vb, h_kv, h_q):
 @pytest.mark.gpu
 @pytest.mark.parametrize("h_kv,h_q,kb,t_chunk", [(2, 8, 3, 3), (2, 4, 3, 5), (2, 2, 3, 8), (2, 8, 4, 3), (1, 1, 3, 11)])
 def test_prefill_parity(h_kv, h_q, kb, t_chunk):
-    """Causal chunked prefill over the compressed cache: passes of 8 / G
-    query tokens (GQA 4 -> 2 tokens, GQA 2 -> 4, GQA 1 -> 8) plus a smaller
-    last pass, and single-token passes where the wider kernel is not built
-    (4-bit keys at GQA 8); ragged lengths, a sequence holding exactly the
-    chunk."""
+    """Causal chunked prefill over the compressed cache: passes of 4 / G
+    query tokens (GQA 1 -> 4 tokens, GQA 2 -> 2) plus smaller last passes,
+    single-token passes at GQA 4; ragged lengths, a sequence holding exactly
+    the chunk."""
     import dataclasses
     lengths = (t_chunk, 127, 129, 300)
     wl = dataclasses.replace(workloads.llama8b(), batch=4, h_kv=h_kv, h_q=h_q, key_bits=kb,
