@@ -18,8 +18,9 @@
 // Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
 // record section a tile writes is one contiguous run of the cache.
 //
-// Warp roles (416 threads):
-//   warp 0        MMA issuer (one elected lane), polling both epilogue groups
+// Warp roles (448 threads):
+//   warps 0, 13   MMA issuers of epilogue groups 0 and 1 (one elected lane),
+//                 each sleeping in blocking waits on its group's barriers
 //   warps 1-4     loader: K rows -> scaled fp16 A operand + norms in shared
 //                 memory; V rows -> codes, scales, zeros straight to the cache
 //   warps 5-8     epilogue group 0 (even tiles)   | thread = tile row = TMEM
@@ -38,7 +39,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQtThreads = 416;
+constexpr int kQtThreads = 448;
+constexpr int kIssuer1Warp = 13;  // MMA issuer of epilogue group 1 (warp 0 issues for group 0)
 constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
 constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
 constexpr float kSScale = 256.f;       // S parts x 2^8
@@ -192,97 +194,73 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
 
-  if (warp == 0) {
-    // ---------------- MMA issuer ------------------------------------------
+  if (warp == 0 || warp == kIssuer1Warp) {
+    // ---------------- MMA issuers -----------------------------------------
+    // Warp 0 issues the three GEMMs of epilogue group 0's tiles, warp 13
+    // those of group 1, each in order and sleeping in blocking waits on its
+    // group's operand barriers (a polling issuer shares its sub-partition's
+    // issue slots with the loader and epilogue warps).
+    const int g = warp == 0 ? 0 : 1;
     const bool leader = elect_one();
     const uint32_t id1 = idesc_f16(128, 128, false, false);
     const uint32_t id2 = idesc_f16(128, 128, false, true);
     const uint64_t dpk[2] = {smem_desc(S.pi[0], 2048, 128), smem_desc(S.pi[1], 2048, 128)};
     const uint64_t dpm[2] = {smem_desc(S.pi[0], 128, 2048), smem_desc(S.pi[1], 128, 2048)};
     const uint64_t dsk[2] = {smem_desc(S.s[0], 2048, 128), smem_desc(S.s[1], 2048, 128)};
-    const uint64_t da1[2] = {smem_desc(S.a1[0], 2048, 128), smem_desc(S.a1[1], 2048, 128)};
-    int tile[2] = {0, 1}, stage[2] = {0, 0};
-    uint64_t *last_bar[2] = {nullptr, nullptr};
-    uint32_t last_ph[2] = {0u, 0u};
-    uint32_t idle = 0;
-    uint64_t t_idle = 0;
-    while (tile[0] < nlocal || tile[1] < nlocal) {
-      bool progress = false;
+    const uint64_t da1 = smem_desc(S.a1[g], 2048, 128);
+    const uint32_t d = tbase + g * 256, aop = d + 128;
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, qwait(bar, parity, &S.abort_flag));
+    };
+    uint64_t *last_bar = nullptr;
+    uint32_t last_ph = 0u;
+    for (int i = g; i < nlocal; i += 2) {
+      const uint32_t ph = (i >> 1) & 1;
+      // Y = K Pi^T: (K)(Pi_hi + Pi_lo), once K is in and the group has read
+      // its previous tile's accumulators
+      if (!wait_all(&S.a1_full[g], ph)) break;
+      if (i >= 2 && !wait_all(&S.d_free[g], ph ^ 1)) break;
+      tc_fence_after();
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const int i = tile[g];
-        if (i >= nlocal) continue;
-        const uint32_t ph = (i >> 1) & 1;
-        const uint32_t d = tbase + g * 256, aop = d + 128;
-        bool ready;
-        if (stage[g] == 0)
-          ready = mbar_test(&S.a1_full[g], ph) && (i < 2 || mbar_test(&S.d_free[g], ph ^ 1));
-        else if (stage[g] == 1)
-          ready = mbar_test(&S.a2_full[g], ph);
-        else
-          ready = mbar_test(&S.a3_full[g], ph);
-        ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (!ready) continue;
-        tc_fence_after();
-        if (stage[g] == 0) {  // Y = K Pi^T: (K)(Pi_hi + Pi_lo)
+      for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
-          for (int pr = 0; pr < 2; ++pr)
+        for (int ks = 0; ks < 8; ++ks)
+          if (leader)
+            mma_f16_ss(d, da1 + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4), id1,
+                       (pr | ks) ? 1u : 0u);
+      if (leader) mma_commit(&S.d1_full[g]);
+      __syncwarp();
+      last_bar = &S.d1_full[g];
+      last_ph = ph;
+      // P = C Pi: C_hi Pi_hi + C_hi Pi_lo + C_lo Pi_hi
+      if (!wait_all(&S.a2_full[g], ph)) break;
+      tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              if (leader)
-                mma_f16_ss(d, da1[g] + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4),
-                           id1, (pr | ks) ? 1u : 0u);
-          if (leader) mma_commit(&S.d1_full[g]);
-          last_bar[g] = &S.d1_full[g];
-        } else if (stage[g] == 1) {  // P = C Pi: C_hi Pi_hi + C_hi Pi_lo + C_lo Pi_hi
+      for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
-          for (int pr = 0; pr < 3; ++pr)
+        for (int ks = 0; ks < 8; ++ks)
+          if (leader)
+            mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks, dpm[pr == 1 ? 1 : 0] + (uint64_t)(16 * ks), id2,
+                       (pr | ks) ? 1u : 0u);
+      if (leader) mma_commit(&S.d2_full[g]);
+      __syncwarp();
+      last_bar = &S.d2_full[g];
+      // Z = R S^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
+      if (!wait_all(&S.a3_full[g], ph)) break;
+      tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              if (leader)
-                mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks, dpm[pr == 1 ? 1 : 0] + (uint64_t)(16 * ks), id2,
-                           (pr | ks) ? 1u : 0u);
-          if (leader) mma_commit(&S.d2_full[g]);
-          last_bar[g] = &S.d2_full[g];
-        } else {  // Z = R S^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
+      for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
-          for (int pr = 0; pr < 3; ++pr)
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              if (leader)
-                mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks,
-                           dsk[pr == 1 ? 1 : 0] + (uint64_t)((ks * 4096) >> 4), id1, (pr | ks) ? 1u : 0u);
-          if (leader) mma_commit(&S.d3_full[g]);
-          last_bar[g] = &S.d3_full[g];
-        }
-        last_ph[g] = ph;
-        __syncwarp();
-        if (++stage[g] == 3) {
-          stage[g] = 0;
-          tile[g] += 2;
-        }
-        progress = true;
-      }
-      if (progress) {
-        idle = 0;
-        t_idle = 0;
-      } else if ((++idle & 15u) != 0) {
-        __nanosleep(64);
-      } else {
-        if (S.abort_flag) break;
-        const uint64_t now = globaltimer_ns();
-        if (t_idle == 0) {
-          t_idle = now;
-        } else if (now - t_idle > 2000000000ull) {
-          S.abort_flag = 1;
-          break;
-        }
-      }
+        for (int ks = 0; ks < 8; ++ks)
+          if (leader)
+            mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks, dsk[pr == 1 ? 1 : 0] + (uint64_t)((ks * 4096) >> 4),
+                       id1, (pr | ks) ? 1u : 0u);
+      if (leader) mma_commit(&S.d3_full[g]);
+      __syncwarp();
+      last_bar = &S.d3_full[g];
     }
-    // never leave with an MMA in flight: the last commit of each group
-#pragma unroll
-    for (int g = 0; g < 2; ++g)
-      if (last_bar[g]) mbar_wait(last_bar[g], last_ph[g]);
+    // never leave with an MMA in flight: the group's last commit
+    if (last_bar) mbar_wait(last_bar, last_ph);
   } else if (warp <= 4) {
     // ---------------- loader -----------------------------------------------
     // A warp takes 8 rows at a time (one 8-row group of the operand): lane
