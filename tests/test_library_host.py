@@ -152,3 +152,44 @@ def test_dequantize_validation_before_launch():
     assert f(ctypes.byref(P), ctypes.byref(C), 0, -1, 1, o, o, None) == 1
     assert f(ctypes.byref(P), ctypes.byref(C), 0, 0, 1, None, o, None) == 1
     assert f(ctypes.byref(P), ctypes.byref(C), 0, 0, 0, None, None, None) == 0
+
+
+def test_prefill_validation_before_launch():
+    lib = tq.load()
+    P = _params()
+    C = tq.Cache(2, 8, 256, 1 << 20)
+    f = lib.tq_prefill_attention
+    q, ln, out, ws = 1 << 22, 1 << 23, 1 << 24, 1 << 25
+    args = lambda **kw: [kw.get("p", ctypes.byref(P)), kw.get("c", ctypes.byref(C)),
+                         kw.get("q", q), kw.get("dt", 1), kw.get("hq", 32), kw.get("t", 4),
+                         kw.get("ln", ln), kw.get("ml", 256), kw.get("sc", 0.088), kw.get("out", out),
+                         kw.get("ws", ws), kw.get("wsb", 1 << 20), None]
+    assert f(*args(p=None)) == 1
+    assert f(*args(q=None)) == 1
+    assert f(*args(out=None)) == 1
+    assert f(*args(hq=12)) == 1           # not a multiple of h_kv
+    assert f(*args(hq=80)) == 2           # G = 10 not built
+    assert f(*args(t=0)) == 1             # empty chunk
+    assert f(*args(t=300)) == 1           # chunk longer than max_len
+    assert f(*args(ml=257)) == 1          # beyond capacity
+    assert f(*args(sc=float("nan"))) == 1
+    assert f(*args(ws=None)) == 4
+    assert f(*args(ws=ws + 8)) == 4
+    assert f(*args(dt=3)) == 2
+
+
+def test_prefill_tokens_per_pass():
+    """Passes take the largest power of two of query tokens with G x tokens <= 4
+    that the tensor-core kernel is built for (one token from GQA 4 up)."""
+    lib = tq.load()
+    P = _params()
+    g = lib.tq_prefill_tokens_per_pass
+    assert g(ctypes.byref(P), 32, 8, 8) == 1     # GQA 4
+    assert g(ctypes.byref(P), 16, 8, 8) == 2     # GQA 2
+    assert g(ctypes.byref(P), 8, 8, 8) == 4      # GQA 1
+    assert g(ctypes.byref(P), 8, 8, 3) == 2      # capped by the chunk
+    assert g(ctypes.byref(P), 8, 8, 1) == 1
+    assert g(ctypes.byref(P), 64, 8, 8) == 1     # GQA 8
+    assert g(ctypes.byref(P), 12, 8, 8) == 0     # not a multiple of h_kv
+    assert g(ctypes.byref(P), 32, 8, 0) == 0
+    assert g(None, 32, 8, 8) == 0
