@@ -109,7 +109,12 @@ typedef struct {
   int group;      /* value quantization group; 32 */
   const float *pi;         /* [d][d] row-major: Pi, y = Pi u; 16-byte aligned */
   const float *s;          /* [d][d] row-major: S, QJL sketch of r is S r; 16-byte aligned */
-  const float *centroids;  /* [2^(key_bits-1)] ascending */
+  const float *centroids;  /* [2^(key_bits-1)] ascending; tq_make_codebook's
+                              (symmetric) codebook is the one validated at every
+                              length.  A caller-made asymmetric codebook works
+                              (its even Walsh terms get their own operand
+                              planes) but with 3-4-bit keys it is validated at
+                              short lengths only (fewer than 8 tiles per split) */
   const float *boundaries; /* [2^(key_bits-1) - 1] ascending decision boundaries */
 } tq_params;
 
