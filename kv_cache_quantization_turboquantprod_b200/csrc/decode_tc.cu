@@ -32,6 +32,9 @@
 //   channel.
 // Per 128-token tile the record bytes arrive by one 1-D bulk copy (TMA
 // engine) into a ring of shared-memory stages.
+// Chunked prefill runs through the same kernel: the query heads of a unit
+// are then several query tokens of a chunk, each with its causal limit on
+// the tokens it sees (applied per head in the softmax).
 //
 // Warp roles (608 threads):
 //   warp 0        bulk-copy producer; allocates / frees tensor memory
