@@ -20,15 +20,18 @@ hoạt động"; "turboquant/audit_claims.py", AUDIT 1, AUDIT 5, AUDIT 6):
 Values ("turboquant/audit_claims.py", AUDIT 1: ``value_bits``,
 ``value_group_size``): asymmetric min/max quantization per group of
 ``group`` contiguous channels of one token's head vector, no rotation.
-Reading: fp16 scale and zero per group, codes by round-half-even then clamp.
-Because these floating-point steps decide integers (the codes), the oracle
-takes them in float32, the precision the kernel uses, step by step:
+Reading: fp16 scale and zero per group (the audit's record accounting), and
+each code is the nearest of the 2^vb levels zero16 + k scale16, found by
+rounding the exact quotient half-to-even and clamping.  In float64:
   mn, mx      = min, max of the group (exact)
   zero16      = fp16(mn)
-  scale16     = fp16( f32( f32(mx - mn) / f32(2^vb - 1) ) )
-  code        = clamp( rint( f32( f32(v - zero16) / scale16 ) ), 0, 2^vb - 1 ),
+  scale16     = fp16((mx - mn) / (2^vb - 1))
+  code        = clamp(rint((v - zero16) / scale16), 0, 2^vb - 1),
                 0 when scale16 == 0
   dequantized = code * scale16 + zero16
+For inputs of at most float32 precision, mx - mn and v - zero16 are exact in
+float64 and each quotient is within one float64 rounding of the exact one,
+so a float64 tie is an exact tie.
 """
 
 from __future__ import annotations
@@ -107,10 +110,12 @@ def residual_sketch(u: np.ndarray, idx: np.ndarray, pi: np.ndarray, s: np.ndarra
 
 
 def encode_values(values: np.ndarray, value_bits: int, group: int) -> dict:
-    """Group-quantize value vectors [n, d].  Returns codes [n, d] int,
-    scale16 / zero16 [n, d/group] (float64 holding fp16 values) and the
-    float32 code coordinate t [n, d] (for half-integer bands)."""
-    v = np.asarray(values, dtype=np.float32)
+    """Group-quantize value vectors [n, d] in float64.  Returns codes [n, d]
+    int, scale16 / zero16 [n, d/group] (float64 holding fp16 values), the
+    code coordinate t = (v - zero16) / scale16 [n, d] (0 where scale16 == 0)
+    and the unrounded scale quotient (mx - mn) / (2^vb - 1) [n, d/group], the
+    last two for the parity bands."""
+    v = np.asarray(values, dtype=np.float64)
     n, d = v.shape
     if d % group:
         raise ValueError("d must be a multiple of the group size")
@@ -118,23 +123,16 @@ def encode_values(values: np.ndarray, value_bits: int, group: int) -> dict:
     vg = v.reshape(n, ng, group)
     mn = vg.min(axis=2)
     mx = vg.max(axis=2)
-    levels = np.float32(2 ** value_bits - 1)
-    zero16 = mn.astype(np.float16)
-    diff = (mx - mn).astype(np.float32)              # f32 subtraction
-    s32 = (diff / levels).astype(np.float32)         # f32 division
-    scale16 = s32.astype(np.float16)
-    z32 = zero16.astype(np.float32)[:, :, None]
-    sc32 = scale16.astype(np.float32)[:, :, None]
-    num = (vg - z32).astype(np.float32)              # f32 subtraction
+    levels = float(2 ** value_bits - 1)
+    zero16 = fp16(mn)
+    scale_q = (mx - mn) / levels
+    scale16 = fp16(scale_q)
+    sc = scale16[:, :, None]
     with np.errstate(divide="ignore", invalid="ignore"):
-        t = (num / sc32).astype(np.float32)          # f32 division
-    codes = np.clip(np.rint(t), 0, 2 ** value_bits - 1)
-    codes = np.where(sc32 == 0, 0, codes).astype(np.int64)
-    t = np.where(sc32 == 0, 0.0, t)
-    return {"codes": codes.reshape(n, d),
-            "scale16": scale16.astype(np.float64),
-            "zero16": zero16.astype(np.float64),
-            "t": t.reshape(n, d).astype(np.float64)}
+        t = np.where(sc == 0.0, 0.0, (vg - zero16[:, :, None]) / np.where(sc == 0.0, 1.0, sc))
+    codes = np.clip(np.rint(t), 0, levels).astype(np.int64)
+    return {"codes": codes.reshape(n, d), "scale16": scale16, "zero16": zero16,
+            "t": t.reshape(n, d), "scale_q": scale_q}
 
 
 def dequantize_values(codes: np.ndarray, scale16: np.ndarray,

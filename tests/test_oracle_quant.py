@@ -8,6 +8,7 @@ S r), not from oracle helpers.
 """
 
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -150,16 +151,78 @@ def test_constant_group_has_zero_scale():
     assert np.all(vh == float(np.float16(np.float32(0.3))))
 
 
-def test_value_scale_is_computed_in_float32_then_rounded():
-    """scale16 = fp16(f32(f32(mx - mn) / 3)) -- the float32 steps, not fp64."""
-    rng = np.random.default_rng(5)
-    v = rng.standard_normal((200, 32)).astype(np.float32) * 7
-    enc = quant.encode_values(v, 2, 32)
-    for i in range(200):
-        mn, mx = np.float32(v[i].min()), np.float32(v[i].max())
-        s32 = np.float32(np.float32(mx - mn) / np.float32(3.0))
-        assert enc["scale16"][i, 0] == float(np.float16(s32))
-        assert enc["zero16"][i, 0] == float(np.float16(mn))
+def _fp16_exact(x: Fraction) -> Fraction:
+    """Round a rational to the nearest fp16 value, ties to an even
+    significand, by exact arithmetic (normal range and subnormals)."""
+    if x == 0:
+        return Fraction(0)
+    sgn = -1 if x < 0 else 1
+    a = abs(x)
+    e = -14
+    while e < 15 and a >= Fraction(2) ** (e + 1):
+        e += 1
+    ulp = Fraction(2) ** (e - 10)
+    k = a / ulp
+    lo = k.numerator // k.denominator
+    rem = k - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return sgn * lo * ulp
+
+
+def test_fp16_exact_helper_against_known_values():
+    assert _fp16_exact(Fraction(1, 3)) == Fraction(1365, 4096)          # 0x3555
+    assert _fp16_exact(Fraction(1) + Fraction(1, 2048)) == 1             # tie -> even
+    assert _fp16_exact(Fraction(1) + Fraction(3, 2048)) == Fraction(1) + Fraction(1, 512)
+    assert _fp16_exact(Fraction(-2, 3)) == -Fraction(1365, 2048)
+    assert _fp16_exact(Fraction(1, 2 ** 25)) == 0                       # half the least subnormal -> 0
+    assert _fp16_exact(Fraction(3, 2 ** 25)) == Fraction(1, 2 ** 23)    # 1.5 subnormal ulps -> 2
+    assert _fp16_exact(Fraction(65504)) == 65504                        # largest finite
+
+
+@pytest.mark.parametrize("vb", [2, 3, 4])
+def test_value_scale_and_zero_are_nearest_fp16_of_exact_values(vb):
+    """scale16 is the fp16 nearest to the exact rational (mx - mn)/(2^vb - 1)
+    and zero16 the fp16 nearest to mn, by exact arithmetic on the inputs."""
+    rng = np.random.default_rng(50 + vb)
+    v = (rng.standard_normal((60, 64)) * 7).astype(np.float32)
+    v[0, :32] = np.float32(0.1)                      # a constant group
+    enc = quant.encode_values(v, vb, 32)
+    for i in range(v.shape[0]):
+        for gi in range(2):
+            grp = [Fraction(float(x)) for x in v[i, 32 * gi:32 * gi + 32]]
+            mn, mx = min(grp), max(grp)
+            assert Fraction(enc["zero16"][i, gi]) == _fp16_exact(mn)
+            assert Fraction(enc["scale16"][i, gi]) == _fp16_exact((mx - mn) / (2 ** vb - 1))
+
+
+@pytest.mark.parametrize("vb", [2, 3])
+def test_value_codes_are_nearest_levels_by_brute_force(vb):
+    """Each code is the index of the nearest level zero16 + k scale16
+    (k = 0 .. 2^vb - 1), ties to the even k, searched over every level with
+    exact arithmetic; includes values exactly halfway between two levels."""
+    rng = np.random.default_rng(70 + vb)
+    v = (rng.standard_normal((40, 32)) * 3).astype(np.float32)
+    # a group with exact half-level values: zero 0, scale 1 after rounding
+    lv = 2 ** vb - 1
+    v[0] = 0.0
+    v[0, 1] = lv
+    v[0, 2:2 + lv] = np.arange(lv, dtype=np.float32) + 0.5
+    enc = quant.encode_values(v, vb, 32)
+    assert enc["scale16"][0, 0] == 1.0 and enc["zero16"][0, 0] == 0.0
+    for i in range(v.shape[0]):
+        z = Fraction(enc["zero16"][i, 0])
+        s = Fraction(enc["scale16"][i, 0])
+        for j in range(32):
+            x = Fraction(float(v[i, j]))
+            if s == 0:
+                assert enc["codes"][i, j] == 0
+                continue
+            dist = [abs(x - (z + k * s)) for k in range(lv + 1)]
+            best = min(dist)
+            cands = [k for k in range(lv + 1) if dist[k] == best]
+            want = cands[0] if len(cands) == 1 else [k for k in cands if k % 2 == 0][0]
+            assert enc["codes"][i, j] == want, (i, j)
 
 
 @pytest.mark.parametrize("vb", [2, 3, 4])
