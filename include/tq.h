@@ -24,8 +24,10 @@
  *
  * Conventions for every call:
  *  - Ownership: the caller owns every buffer and the stream.  The library
- *    allocates no memory, never synchronises, and keeps no state beyond a
- *    cached per-device SM count.
+ *    allocates no memory and never synchronises (except tq_device_errors);
+ *    its state is a cached per-device SM count, the wait limit, and one
+ *    4-byte error word per device (plus the no-allocation entry point's
+ *    fixed scratch).
  *  - Pointers documented as "device" must be device (or managed) memory of
  *    the current CUDA device; "host" pointers are read before the call
  *    returns.
@@ -33,6 +35,15 @@
  *    argument returns a status and launches nothing.  A launch failure
  *    returns TQ_ERR_CUDA (from cudaGetLastError).  Kernels never trap; an
  *    asynchronous fault surfaces at the caller's next synchronisation.
+ *  - Bounded waits: the pipelined tensor-core kernels hand work between warp
+ *    roles through shared-memory barriers, and every such wait gives up after
+ *    a time limit (2 s; tq_set_wait_limit_ns).  A kernel that gives up stops,
+ *    lets its own copies and tensor-core operations finish, frees its tensor
+ *    memory and returns, so the GPU stays usable; it records the failure in
+ *    the device's sticky error word (tq_device_errors) and in the call's own
+ *    result: decode calls write NaN output rows (and set the workspace status
+ *    word, see tq_decode_attention), quantize-append writes NaN norms into
+ *    the records it owns, so decode over them returns NaN.
  *  - Calls are asynchronous on `stream` and re-entrant.  Calls that write
  *    the same cache region (or the same workspace) must be ordered by the
  *    caller.
@@ -69,6 +80,10 @@ typedef enum {
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* Bits of the sticky per-device error word (tq_device_errors). */
+#define TQ_ERRF_DECODE_WAIT 1u   /* a decode kernel gave up on a bounded wait */
+#define TQ_ERRF_QUANTIZE_WAIT 2u /* a quantize-append kernel gave up on one */
 
 /* Tokens per cache tile; capacity must be a multiple of it. */
 #define TQ_TILE_TOKENS 128
@@ -109,12 +124,16 @@ typedef struct {
   int group;      /* value quantization group; 32 */
   const float *pi;         /* [d][d] row-major: Pi, y = Pi u; 16-byte aligned */
   const float *s;          /* [d][d] row-major: S, QJL sketch of r is S r; 16-byte aligned */
-  const float *centroids;  /* [2^(key_bits-1)] ascending; tq_make_codebook's
-                              (symmetric) codebook is the one validated at every
-                              length.  A caller-made asymmetric codebook works
-                              (its even Walsh terms get their own operand
-                              planes) but with 3-4-bit keys it is validated at
-                              short lengths only (fewer than 8 tiles per split) */
+  const float *centroids;  /* [2^(key_bits-1)] ascending; any codebook works.
+                              Decode expands it in the code bits (its Walsh
+                              expansion): tq_make_codebook's symmetric
+                              codebooks need only the odd terms; a caller-made
+                              asymmetric one also needs the even terms, and in
+                              the shapes where those planes fit in tensor
+                              memory only once (3-bit keys at GQA 4 and 8 with
+                              2-bit values, 4-bit keys at GQA 4, 3-bit keys and
+                              values at GQA 6) decode runs the SIMT split-K
+                              kernel for it (decided on the device per call) */
   const float *boundaries; /* [2^(key_bits-1) - 1] ascending decision boundaries */
 } tq_params;
 
@@ -203,7 +222,10 @@ TQ_API size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c,
  *                  standard choice); must be finite
  *   out            device, [batch][h_q][d] fp32
  *   workspace      device, >= tq_decode_workspace_size(p, c, h_q, max_len)
- *                  bytes, 256-byte aligned; contents need no initialisation
+ *                  bytes, 256-byte aligned; contents need no initialisation.
+ *                  Its first int32 is the call's status word once the call
+ *                  has run: 0, or nonzero if a kernel of the call gave up on a
+ *                  bounded wait, in which case every output row is NaN.
  * Errors: TQ_ERR_WORKSPACE if the workspace is missing or too small;
  * TQ_ERR_INVALID_ARGUMENT / TQ_ERR_UNSUPPORTED as for the other calls.
  */
@@ -307,7 +329,9 @@ TQ_API tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c,
  *    launches nothing.
  *  - The first call on a device looks up the array's device address with
  *    that device current and caches it; make that first call before any
- *    stream capture.
+ *    stream capture.  The cached address does not survive a device reset
+ *    (cudaDeviceReset): calling this entry point again after one is not
+ *    supported.
  *  - All calls share the one array and it keeps the previous call's contents
  *    (nothing in it needs clearing: every byte the kernels read is written
  *    earlier in the same call).  Calls that overlap on the GPU -- on
@@ -320,6 +344,28 @@ TQ_API tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_cache 
                                              const int32_t *len_dev, int max_len,
                                              float softmax_scale, float *out,
                                              tq_stream_t stream);
+
+/*
+ * tq_set_wait_limit_ns -- set the time limit of the kernels' bounded waits
+ * for calls made afterwards from any host thread (0 restores the default,
+ * 2 s); the kernels' suspend hint per wait test is min(limit, 1 ms).  For
+ * tests of the timeout path: a limit shorter than a call needs makes its
+ * kernels give up (NaN results, the error word set) and return.  Always
+ * TQ_OK.
+ */
+TQ_API tq_status tq_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * tq_device_errors -- synchronise the current device, then read (and, if
+ * `clear` is nonzero, reset) its sticky error word: an OR of TQ_ERRF_* bits
+ * set by kernels that gave up on a bounded wait since the last clear.
+ *   flags  host, written.
+ * The first call on a device looks the word's device address up (once per
+ * device); launches made by the library's other calls do the same.
+ * Errors: TQ_ERR_INVALID_ARGUMENT for a null pointer, TQ_ERR_CUDA if the
+ * device reports an error.
+ */
+TQ_API tq_status tq_device_errors(uint32_t *flags, int clear);
 
 /*
  * tq_dequantize -- explicit reconstruction of cached tokens [start,

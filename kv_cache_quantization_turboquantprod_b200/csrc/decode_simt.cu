@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(256) qprep_kernel(DecodeArgs a) {
 // tokens; a lane owns 4 consecutive dims (one nibble of every plane row).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
+  // behind the tensor-core kernel: only for a codebook that kernel left to us
+  if (a.fallback_gate && a.status[1] == 0) return;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = a.h_q / a.h_kv;
@@ -170,10 +172,16 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
 
 // ---------------------------------------------------------------------------
 // combine: out[b][hq][:] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
+// A call whose kernels gave up on a bounded wait (status word nonzero) gets
+// NaN rows, so a timeout never comes back as a plausible result.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
   const int bh = blockIdx.x;
   const int j = threadIdx.x;
+  if (a.status[0] != 0) {
+    a.out[qrow_offset(a, bh / a.h_q, bh % a.h_q) + j] = __int_as_float(0x7fc00000);
+    return;
+  }
   const float *src = a.part + (size_t)bh * a.part_stride * (kD + 2);
   float M = -INFINITY;
   for (int s = 0; s < a.part_stride; ++s) M = fmaxf(M, src[s * (kD + 2) + kD]);
@@ -338,11 +346,18 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   if (!decode_tc_supported(a.key_bits, a.value_bits, a.h_q / a.h_kv))
     return launch_decode_simt(a, stream);
   const int bhq = a.batch * a.h_q;
-  // the status word is cleared here; the query blocks are built inside
-  cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int), stream);
+  // the query-block kernel (first in launch_decode_tc) clears the status word
+  cudaError_t e = launch_decode_tc(a, stream);
   if (e != cudaSuccess) return e;
-  e = launch_decode_tc(a, stream);
-  if (e != cudaSuccess) return e;
+  if (decode_tc_needs_fallback(a.key_bits, a.value_bits, a.h_q / a.h_kv)) {
+    // returns at once unless the codebook needs it (status[1], set on the device)
+    DecodeArgs f = a;
+    f.fallback_gate = 1;
+    dim3 grid(a.nsplit, a.h_kv, a.batch);
+    decode_splitk_simt_kernel<<<grid, 128, 0, stream>>>(f);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (a.win_k) {
     e = launch_window(a, stream);
     if (e != cudaSuccess) return e;

@@ -50,8 +50,10 @@
 //                 accumulators.  The four states are merged at the end like
 //                 four splits.  Every SM sub-partition runs one warp of each
 //                 group, so the per-tile work is spread evenly.
-// Every mbarrier wait is bounded (2 s); on timeout the CTA sets the status word in
-// the workspace, stops, waits for its own copies and MMAs and frees TMEM.
+// Every mbarrier wait between roles is bounded (2 s unless the host set another
+// limit) and answers warp-uniformly; on timeout the CTA sets the call's status
+// word in the workspace (the combine then writes NaN rows) and the device's
+// sticky error word, stops, waits for its own copies and MMAs and frees TMEM.
 #include <math.h>
 
 #include "sm100.cuh"
@@ -170,24 +172,26 @@ struct TcSmem {
   float dal[kWorkGroups][4][C::G + 1];     // per warp: alpha of its last tile, fixed-point scale
 };
 
-// Bounded wait (2 s of wall time) that also gives up when another role has
-// aborted; a timeout raises the CTA's abort flag and the status word.
+// Bounded pipeline wait of one thread (limit a.wait_ns, 2 s by default) that
+// also gives up when another role has aborted; a timeout raises the CTA's
+// abort flag, the call's status word and the device's sticky error word.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         int *status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    // the abort flag and the clock are checked every 16 tries: a waiting
-    // warp then costs its sub-partition almost no issue slots
-#pragma unroll 1
-    for (int r = 0; r < 16; ++r)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > 2000000000ull) break;
+                                         const DecodeArgs &a) {
+  bool timed_out = false;
+  if (pipe_wait(bar, parity, abort_flag, a.wait_ns, a.wait_hint_ns, &timed_out)) return true;
+  if (timed_out) {
+    atomicOr(a.status, 1);
+    if (a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_DECODE_WAIT);
   }
-  *abort_flag = 1;
-  if (status) atomicOr(status, 1);
   return false;
+}
+
+// The same, with one answer for the whole (converged) warp, so that a warp
+// never splits between lanes that go on to warp-collective tensor-memory
+// instructions and lanes that gave up.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          const DecodeArgs &a) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, a));
 }
 
 // Spin word of code-bit subset S over 32 coordinates: bit set <=> the
@@ -273,6 +277,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   // split-major grid: every unit's first splits are scheduled before any
   // last (ragged, shorter) split, so the short CTAs fill the tail
   const int split = blockIdx.z, h = blockIdx.x, b = blockIdx.y;
+  // a codebook that needs the SIMT split-K kernel (the query-block kernel
+  // decided it): that kernel, launched next, writes every partial state
+  if (a.status[1] != 0) return;
 
   int len = a.len[b] - a.len_sub;
   len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
@@ -322,7 +329,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
-  int *status = a.status;
 
   if (warp == 0) {
     // ---------------- producer --------------------------------------------
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       for (int i = 0; i < ntile; ++i) {
         const int s = i % C::STAGES;
         if (i >= C::STAGES &&
-            !wait_bar(&S.empty[s], ((i / C::STAGES) - 1) & 1, &S.abort_flag, status))
+            !wait_bar(&S.empty[s], ((i / C::STAGES) - 1) & 1, &S.abort_flag, a))
           break;
         mbar_arrive_expect_tx(&S.full[s], C::TILE_BYTES);
         bulk_g2s(S.stage[s], tiles + (size_t)i * C::TILE_BYTES, C::TILE_BYTES, &S.full[s]);
@@ -352,9 +358,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // worker groups, and neither waits behind the other.  The whole warp
     // runs the loop (descriptors stay warp-uniform); one elected lane issues.
     const bool leader = elect_one();
-    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, &S.abort_flag, status));
-    };
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) { return wait_warp(bar, parity, &S.abort_flag, a); };
     const bool qok = wait_all(&S.q_full, 0);
     int last = -1;  // last tile whose MMAs were committed
     if (warp == 1) {
@@ -433,7 +437,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
                                  : 32 * (t >> 5) + 8 * (t & 3) + 4 * ((t >> 4) & 1) + ((t >> 2) & 3);
     const float kappa = qjl_kappa();
     const float scale2 = a.softmax_scale * kLog2e;
-    const bool qok = wait_bar(&S.q_full, 0, &S.abort_flag, status);
+    const bool qok = wait_warp(&S.q_full, 0, &S.abort_flag, a);
     const int nm = qok ? Q.n_mse : 0, npl = nm + 1;
     const int akb = C::ak_ring(npl);
     // symmetric codebook: the planes are the odd subsets, known at compile
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // alpha[0..G-1] and sc = alpha[G] as this warp left them in shared memory
     float *dal = S.dal[grp][q4];
     auto readback = [&](int jt, int rb) -> bool {
-      if (!wait_bar(&S.pv_done[rb], (jt / C::NR) & 1, &S.abort_flag, status)) return false;
+      if (!wait_warp(&S.pv_done[rb], (jt / C::NR) & 1, &S.abort_flag, a)) return false;
       tc_fence_after();
       constexpr int PB = C::PB;
       uint32_t d[PB * G];
@@ -484,7 +488,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       const int n = i / kWorkGroups, s = i % C::STAGES, rb = i % C::NR;
       ok = false;
       // 1. code / sign plane words of the tile
-      if (!wait_bar(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, status)) break;
+      if (!wait_warp(&S.full[s], (i / C::STAGES) & 1, &S.abort_flag, a)) break;
       const uint8_t *st = S.stage[s];
       uint32_t bw[3][4], sw[4];
       {
@@ -505,7 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       //    of tile i - akb has finished
       if (i >= akb) {
         const int pt = i - akb;
-        if (!wait_bar(&S.s_ready[pt & 1], (pt >> 1) & 1, &S.abort_flag, status)) break;
+        if (!wait_warp(&S.s_ready[pt & 1], (pt >> 1) & 1, &S.abort_flag, a)) break;
         // the stores below must follow the MMA's reads of the buffer
         tc_fence_after();
       }
@@ -556,7 +560,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       if constexpr (C::OWN_SLOT) {
         if (prev >= 0 && !readback(prev, rb)) break;
       } else {
-        if (i >= C::NR && !wait_bar(&S.pv_done[rb], ((i - C::NR) / C::NR) & 1, &S.abort_flag, status)) break;
+        if (i >= C::NR && !wait_warp(&S.pv_done[rb], ((i - C::NR) / C::NR) & 1, &S.abort_flag, a)) break;
       }
 
       // 4. value codes, norms and value scales; the stage is then released
@@ -615,7 +619,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       if (lane == 0) mbar_arrive(&S.av_ready[rb]);
 
       // 5. score epilogue; limbs combine as (D0 + 128 D1) 2^-F + (D2 + 128 D3) 2^(14-F)
-      if (!wait_bar(&S.s_ready[i & 1], (i >> 1) & 1, &S.abort_flag, status)) break;
+      if (!wait_warp(&S.s_ready[i & 1], (i >> 1) & 1, &S.abort_flag, a)) break;
       tc_fence_after();
       float mse[G], qjl[G];
       {
@@ -696,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.red_bar[grp]);
-      if (!wait_bar(&S.red_bar[grp], n & 1, &S.abort_flag, status)) break;
+      if (!wait_warp(&S.red_bar[grp], n & 1, &S.abort_flag, a)) break;
       float alpha[G];
       bool changed = false;
 #pragma unroll
@@ -909,6 +913,15 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     wts[0] = 0.f;
     nm = 1;
   }
+  // A codebook whose planes fit in tensor memory only once (an asymmetric
+  // codebook in a shape with little room) goes to the SIMT split-K kernel,
+  // which reads the rotated queries written below.  This kernel runs first
+  // in every tensor-core call, so it also clears the call's status word.
+  const bool fallback = C::ak_ring(nm + 1) < 2;
+  if (blockIdx.x == 0 && tid == 0) {
+    a.status[0] = 0;
+    a.status[1] = fallback ? 1 : 0;
+  }
   QConst *qc = reinterpret_cast<QConst *>(blk + C::BQ_BYTES);
   __syncthreads();
 
@@ -929,7 +942,10 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
         for (int g = 0; g < G; ++g) acc[g] = fmaf(m, qv[g * kD + i], acc[g]);
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) rot[g * 2 * kD + o] = acc[g];
+      for (int g = 0; g < G; ++g) {
+        rot[g * 2 * kD + o] = acc[g];
+        if (fallback) a.qrot[((size_t)b * a.h_q + h * G + g) * 2 * kD + o] = acc[g];
+      }
     }
     __syncthreads();
     // per head: sum and max |.| of q~ (warps 0-3) and s^ (warps 4-7)
@@ -1035,6 +1051,18 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 size_t decode_tc_qblock_bytes(int key_bits, int G) { return qblock_bytes_for(key_bits - 1, G); }
+
+bool decode_tc_needs_fallback(int key_bits, int value_bits, int G) {
+  if (!decode_tc_supported(key_bits, value_bits, G)) return false;
+  const int mb = key_bits - 1;
+#define TQ_TC(MB_, VB_, G_) \
+  if (mb == MB_ && value_bits == VB_ && G == G_) return Cfg<MB_, VB_, G_>::ak_ring(1 << MB_) < 2;
+  TQ_TC(1, 2, 1) TQ_TC(1, 2, 2) TQ_TC(1, 2, 4) TQ_TC(1, 2, 8)
+  TQ_TC(2, 2, 1) TQ_TC(2, 2, 2) TQ_TC(2, 2, 4) TQ_TC(2, 2, 8)
+  TQ_TC(3, 2, 4) TQ_TC(2, 3, 6)
+#undef TQ_TC
+  return false;
+}
 
 bool decode_tc_supported(int key_bits, int value_bits, int G) {
   const int mb = key_bits - 1;

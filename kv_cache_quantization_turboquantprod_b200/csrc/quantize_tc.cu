@@ -25,8 +25,10 @@
 //                 memory; V rows -> codes, scales, zeros straight to the cache
 //   warps 5-8     epilogue group 0 (even tiles)   | thread = tile row = TMEM
 //   warps 9-12    epilogue group 1 (odd tiles)    | lane; 256 TMEM columns each
-// Every mbarrier wait is bounded (2 s); on timeout the CTA raises its abort
-// flag, stops, lets its own MMAs finish and frees TMEM.
+// Every mbarrier wait between roles is bounded (2 s unless the host set another
+// limit) and answers warp-uniformly; on timeout the CTA raises its abort flag
+// and the device's sticky error word, stops, lets its own MMAs finish, frees
+// TMEM and marks the records it owns with NaN norms.
 #include <math.h>
 
 #include "sm100.cuh"
@@ -93,19 +95,15 @@ __device__ __forceinline__ TileInfo tile_info(const AppendArgs &a, int gt) {
   return ti;
 }
 
-__device__ __forceinline__ bool qwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    // abort flag and clock every 16 tries: a waiting warp costs few issue slots
-#pragma unroll 1
-    for (int r = 0; r < 16; ++r)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > 2000000000ull) break;
-  }
-  *abort_flag = 1;
-  return false;
+// Bounded pipeline wait (limit a.wait_ns, 2 s by default) with one answer for
+// the whole converged warp; a timeout raises the CTA's abort flag and the
+// device's sticky error word.
+__device__ __forceinline__ bool qwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                      const AppendArgs &a) {
+  bool timed_out = false;
+  const bool ok = pipe_wait(bar, parity, abort_flag, a.wait_ns, a.wait_hint_ns, &timed_out);
+  if (timed_out && a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_QUANTIZE_WAIT);
+  return __all_sync(0xffffffffu, ok);
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo_elem, float hi_elem) {
@@ -209,9 +207,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     const uint64_t dsk[2] = {smem_desc(S.s[0], 2048, 128), smem_desc(S.s[1], 2048, 128)};
     const uint64_t da1 = smem_desc(S.a1[g], 2048, 128);
     const uint32_t d = tbase + g * 256, aop = d + 128;
-    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, qwait(bar, parity, &S.abort_flag));
-    };
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) { return qwait(bar, parity, &S.abort_flag, a); };
     uint64_t *last_bar = nullptr;
     uint32_t last_ph = 0u;
     for (int i = g; i < nlocal; i += 2) {
@@ -300,7 +296,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       for (int pass = 0; pass < 4; ++pass) {
         uint4 kn[4], vn[4];
         fetch(4 * i + pass + 1, kn, vn);
-        if (pass == 0 && i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag)) {
+        if (pass == 0 && i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag, a)) {
           stop = true;
           break;
         }
@@ -448,7 +444,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       const int pos = a.lens[ti.b] + ti.t0 + r;
       uint8_t *tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
       const int slot = pos % kTile;
-      if (!qwait(&S.d1_full[g], ph, &S.abort_flag)) break;
+      if (!qwait(&S.d1_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
       const float nk = S.nk[g][r];
       const int sh = S.sh[g][r];
@@ -514,7 +510,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           *reinterpret_cast<uint4 *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes) =
               make_uint4(planes[p][0], planes[p][1], planes[p][2], planes[p][3]);
       // ---- E2: r = u - Pi^T c, ||r||, residual operand R ----
-      if (!qwait(&S.d2_full[g], ph, &S.abort_flag)) break;
+      if (!qwait(&S.d2_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
       float rr = 0.f;  // ||r||^2 x 2^26
       const float inv2r = inv2 * kRScale;
@@ -557,7 +553,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         mbar_arrive(&S.a1_free[g]);
       }
       // ---- E3: signs of z = S r, norms ----
-      if (!qwait(&S.d3_full[g], ph, &S.abort_flag)) break;
+      if (!qwait(&S.d3_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
       uint32_t sw[4] = {0u, 0u, 0u, 0u};
       tmem_ld16(dcol, dA);
@@ -590,6 +586,20 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     tc_fence_after();
     tmem_dealloc(tbase, 512);
     tmem_relinquish();
+  }
+  // A CTA that gave up on a wait leaves its tiles' records incomplete: mark
+  // every record it owns with NaN norms, so that decode over them returns
+  // NaN instead of a plausible result.
+  if (S.abort_flag) {
+    const uint32_t nan2 = 0x7E007E00u;  // two fp16 quiet NaNs (||k||, ||r||)
+    for (int i = 0; i < nlocal; ++i) {
+      const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
+      for (int r = tid; r < ti.nrow; r += kQtThreads) {
+        const int pos = a.lens[ti.b] + ti.t0 + r;
+        uint8_t *tp = tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile);
+        *reinterpret_cast<uint32_t *>(tp + L.norms + (pos % kTile) * 4) = nan2;
+      }
+    }
   }
 }
 

@@ -37,16 +37,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
       : "memory");
 }
 // One potentially blocking test of a phase: the thread may be suspended
-// until the phase completes or a time limit passes (hint: 1 ms), so a
-// waiting warp issues few instructions.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+// until the phase completes or a time limit passes (hint_ns), so a waiting
+// warp issues few instructions.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity,
+                                              uint32_t hint_ns = 1000000u) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -69,7 +70,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Bounded wait for the phase with the given parity to complete: gives up
-// (returns false) once `limit_ns` of wall time has passed.
+// (returns false) once `limit_ns` of wall time has passed.  Used where the
+// phase is completed by the hardware (a bulk copy landing, an MMA commit), so
+// it always ends well inside the limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -78,6 +81,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Bounded pipeline wait between the roles of one CTA.  Returns true once the
+// phase has completed; false when another role raised *abort_flag or when
+// limit_ns of wall time passed, in which case this call raises
+// *abort_flag and sets *timed_out.  The abort flag and the clock are checked
+// every 16 tests, so a waiting warp costs its sub-partition few issue slots.
+// Each test may suspend the thread for up to hint_ns.
+__device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned long long limit_ns, unsigned int hint_ns,
+                                          bool *timed_out) {
+  if (mbar_try_wait(bar, parity, hint_ns)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int r = 0; r < 16; ++r)
+      if (mbar_try_wait(bar, parity, hint_ns)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+  *abort_flag = 1;
+  *timed_out = true;
+  return false;
 }
 
 // ---------------------------------------------------------------------------

@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 #include "tq_common.cuh"
@@ -38,6 +39,46 @@ cudaError_t current_sm_count(int *out) {
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Bound of the kernels' pipeline waits (tq_set_wait_limit_ns).
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+
+// Sticky per-device error word (TQ_ERRF_* bits) that kernels set when they
+// give up on a bounded wait; its device address is looked up once per device.
+__device__ unsigned int g_error_word;
+std::atomic<unsigned int *> g_error_addr[kMaxDevices];
+std::mutex g_error_mutex;
+
+cudaError_t error_word_address(unsigned int **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  unsigned int *p = g_error_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_error_mutex);
+    p = g_error_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      void *v = nullptr;
+      e = cudaGetSymbolAddress(&v, g_error_word);
+      if (e != cudaSuccess) return e;
+      p = static_cast<unsigned int *>(v);
+      g_error_addr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
+// Wait limits and error word of a launch on the current device.
+template <class Args>
+cudaError_t set_wait_fields(Args &a) {
+  const unsigned long long ns = g_wait_ns.load(std::memory_order_relaxed);
+  a.wait_ns = ns;
+  a.wait_hint_ns = (unsigned int)(ns < 1000000ull ? ns : 1000000ull);
+  return error_word_address(&a.errors);
+}
 
 tq_status check_params(const tq_params *p) {
   if (!p) return TQ_ERR_INVALID_ARGUMENT;
@@ -153,6 +194,7 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
   a.key_bits = p->key_bits; a.value_bits = p->value_bits; a.dtype = dtype;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
+  if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
   const cudaError_t e = tq::quantize_tc_supported(a) ? tq::launch_quantize_tc(a, sms, (cudaStream_t)stream)
                                                     : tq::launch_quantize_simt(a, sms, (cudaStream_t)stream);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
@@ -241,6 +283,8 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
     a.win_k = nullptr; a.win_v = nullptr; a.win_dtype = TQ_BF16; a.win_len = nullptr; a.win_cap = 0;
     a.qt = n; a.q_tstride = t_chunk; a.q_t0 = t0; a.len_sub = len_sub;
     a.num_sms = sms;
+    a.fallback_gate = 0;
+    if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
     tq::bind_workspace(a, P, workspace);
     a.out = out;
     if (tq::launch_decode(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
@@ -249,15 +293,17 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
   return TQ_OK;
 }
 
-namespace {
+}  // extern "C"
 
-// Shared by tq_decode_attention and tq_decode_attention_window (win_k null:
-// no window).
+namespace tq {
+
+// Shared by tq_decode_attention, tq_decode_attention_window (win_k null: no
+// window) and tq_decode_attention_noalloc (the library's scratch as workspace).
 tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq_dtype q_dtype,
                         int h_q, const int32_t *len_dev, int max_len, const void *win_k,
                         const void *win_v, tq_dtype win_dtype, const int32_t *win_len_dev,
                         int win_cap, float softmax_scale, float *out, void *workspace,
-                        size_t workspace_bytes, tq_stream_t stream) {
+                        size_t workspace_bytes, cudaStream_t stream, bool validate_only) {
   tq_status st = check_params(p);
   if (st != TQ_OK) return st;
   if ((st = check_cache(c)) != TQ_OK) return st;
@@ -274,6 +320,7 @@ tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq
     if (!aligned(win_k, 16) || !aligned(win_v, 16) || !aligned(win_len_dev, 4))
       return TQ_ERR_INVALID_ARGUMENT;
   }
+  if (validate_only) return TQ_OK;
   if (!workspace || !aligned(workspace, 256)) return TQ_ERR_WORKSPACE;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
@@ -290,20 +337,24 @@ tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq
   a.win_cap = win_cap;
   a.qt = 1; a.q_tstride = 1; a.q_t0 = 0; a.len_sub = 0;
   a.num_sms = sms;
+  a.fallback_gate = 0;
+  if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
   tq::bind_workspace(a, P, workspace);
   a.out = out;
-  if (tq::launch_decode(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (tq::launch_decode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }
 
-}  // namespace
+}  // namespace tq
+
+extern "C" {
 
 tq_status tq_decode_attention(const tq_params *p, const tq_cache *c, const void *q,
                               tq_dtype q_dtype, int h_q, const int32_t *len_dev, int max_len,
                               float softmax_scale, float *out, void *workspace,
                               size_t workspace_bytes, tq_stream_t stream) {
-  return decode_common(p, c, q, q_dtype, h_q, len_dev, max_len, nullptr, nullptr, TQ_BF16, nullptr, 0,
-                       softmax_scale, out, workspace, workspace_bytes, stream);
+  return tq::decode_common(p, c, q, q_dtype, h_q, len_dev, max_len, nullptr, nullptr, TQ_BF16, nullptr,
+                           0, softmax_scale, out, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 tq_status tq_decode_attention_window(const tq_params *p, const tq_cache *c, const void *q,
@@ -313,8 +364,27 @@ tq_status tq_decode_attention_window(const tq_params *p, const tq_cache *c, cons
                                      float softmax_scale, float *out, void *workspace,
                                      size_t workspace_bytes, tq_stream_t stream) {
   if (!win_k) return TQ_ERR_INVALID_ARGUMENT;
-  return decode_common(p, c, q, q_dtype, h_q, len_dev, max_len, win_k, win_v, win_dtype, win_len_dev,
-                       win_cap, softmax_scale, out, workspace, workspace_bytes, stream);
+  return tq::decode_common(p, c, q, q_dtype, h_q, len_dev, max_len, win_k, win_v, win_dtype,
+                           win_len_dev, win_cap, softmax_scale, out, workspace, workspace_bytes,
+                           (cudaStream_t)stream);
+}
+
+tq_status tq_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
+tq_status tq_device_errors(uint32_t *flags, int clear) {
+  if (!flags) return TQ_ERR_INVALID_ARGUMENT;
+  unsigned int *p = nullptr;
+  if (error_word_address(&p) != cudaSuccess) return TQ_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return TQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TQ_ERR_CUDA;
+  *flags = v;
+  if (clear && cudaMemset(p, 0, sizeof(v)) != cudaSuccess) return TQ_ERR_CUDA;
+  if (clear && cudaDeviceSynchronize() != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
 }
 
 tq_status tq_dequantize(const tq_params *p, const tq_cache *c, int b, int start, int count,

@@ -27,6 +27,11 @@ struct AppendArgs {
   // tiles [tstart[b], tstart[b + 1])
   int tstart[TQ_MAX_BATCH + 1];
   int total_tiles;
+  // bounded pipeline waits (tensor-core path): limit, suspend hint, and the
+  // sticky per-device error word a timeout sets (TQ_ERRF_QUANTIZE_WAIT)
+  unsigned long long wait_ns;
+  unsigned int wait_hint_ns;
+  unsigned int *errors;
 };
 
 // Split-K plan of one decode call (host-computed, identical in the
@@ -58,7 +63,10 @@ struct DecodeArgs {
   tq_dtype win_dtype;
   const int32_t *win_len;
   int win_cap;
-  int *status;   // workspace: status word, cleared by qprep
+  // workspace words: status[0] nonzero once a kernel of this call gave up on a
+  // bounded wait (combine then writes NaN rows); status[1] nonzero when the
+  // codebook needs the SIMT split-K kernel (set by the query-block kernel)
+  int *status;
   float *qrot;   // workspace: [B][H_q][2][d]
   float *part;   // workspace: [B][H_q][part_stride][d+2]
   uint8_t *qblocks;  // workspace: [B][H_kv] query blocks (tensor-core path)
@@ -71,6 +79,14 @@ struct DecodeArgs {
   // of it sees the first len[b] - len_sub - (qt - 1 - t).  Decode: qt = 1,
   // q_tstride = 1, q_t0 = 0, len_sub = 0.
   int qt, q_tstride, q_t0, len_sub;
+  // bounded pipeline waits: limit, suspend hint, sticky per-device error word
+  // a timeout sets (TQ_ERRF_DECODE_WAIT)
+  unsigned long long wait_ns;
+  unsigned int wait_hint_ns;
+  unsigned int *errors;
+  // SIMT split-K launched behind the tensor-core kernel: runs only when
+  // status[1] says the codebook needs it
+  int fallback_gate;
 };
 
 constexpr int kQRowElems = 128;  // elements per query / output row (d)
@@ -102,12 +118,26 @@ cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 // Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
 bool decode_tc_supported(int key_bits, int value_bits, int gqa);
+// True when a codebook whose Walsh expansion has every subset plane (an
+// asymmetric codebook) leaves room for only one plane buffer of the
+// tensor-core kernel in tensor memory; such codebooks run the SIMT split-K
+// kernel instead (decided on the device per call).
+bool decode_tc_needs_fallback(int key_bits, int value_bits, int gqa);
 size_t decode_tc_qblock_bytes(int key_bits, int gqa);
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
 // qprep -> split-K (tensor-core kernel where built, SIMT otherwise) -> combine
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 // Fill DecodeArgs' workspace pointers from a plan.
 void bind_workspace(DecodeArgs &a, const DecodePlan &P, void *workspace);
+// Validate one decode call (tq_decode_attention's contract) and launch it
+// with the given scratch; shared by the workspace and no-allocation entry
+// points.  win_k == nullptr: no recent window.  validate_only: return after
+// the argument checks that need no device (before the workspace checks).
+tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq_dtype q_dtype,
+                        int h_q, const int32_t *len_dev, int max_len, const void *win_k,
+                        const void *win_v, tq_dtype win_dtype, const int32_t *win_len_dev,
+                        int win_cap, float softmax_scale, float *out, void *workspace,
+                        size_t workspace_bytes, cudaStream_t stream, bool validate_only = false);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t stream);
 
 }  // namespace tq

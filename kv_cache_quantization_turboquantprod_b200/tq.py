@@ -29,7 +29,9 @@ MAX_BATCH = 1024
 EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_bytes",
            "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
            "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window",
-           "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass")
+           "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass",
+           "tq_set_wait_limit_ns", "tq_device_errors")
+ERRF_DECODE_WAIT, ERRF_QUANTIZE_WAIT = 1, 2
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -94,6 +96,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_prefill_attention.argtypes = [P, C, vp, ci, ci, ci, vp, ci, ctypes.c_float, vp, vp, sz, vp]
     lib.tq_dequantize.restype = ci
     lib.tq_dequantize.argtypes = [P, C, ci, ci, ci, vp, vp, vp]
+    lib.tq_set_wait_limit_ns.restype = ci
+    lib.tq_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.tq_device_errors.restype = ci
+    lib.tq_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ci]
     if path is None:
         _lib = lib
     return lib
@@ -116,6 +122,32 @@ def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return TQ_BF16
     raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check_rows(name: str, t: torch.Tensor, shape, dtypes, device=None) -> None:
+    """Shape, dtype, contiguity and device of a tensor handed to the C ABI,
+    which cannot check buffer sizes itself."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be one of {dtypes}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda or (device is not None and t.device != device):
+        raise ValueError(f"{name} must be a CUDA tensor on the cache's device")
+
+
+def _check_decode_io(cache, q: torch.Tensor, len_dev: torch.Tensor, out: torch.Tensor) -> int:
+    """q [B, H_q, d] fp32/bf16, len_dev [B] int32, out [B, H_q, d] fp32, all
+    contiguous on the cache's device; returns H_q."""
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H_q, d]")
+    dev = cache.buffer.device
+    B, hq, d = cache.batch, int(q.shape[1]), int(q.shape[2])
+    _check_rows("q", q, (B, hq, d), (torch.float32, torch.bfloat16), dev)
+    _check_rows("len_dev", len_dev, (B,), (torch.int32,), dev)
+    _check_rows("out", out, (B, hq, d), (torch.float32,), dev)
+    return hq
 
 
 def _i32_array(xs):
@@ -216,11 +248,12 @@ def tq_decode_attention(layer: Layer, cache: CompressedCache, q: torch.Tensor,
                         stream=None) -> None:
     """q [B, H_q, d] (fp32/bf16), len_dev [B] int32 device, out [B, H_q, d]
     fp32, workspace a uint8 device tensor."""
-    if len_dev.dtype != torch.int32:
-        raise TypeError("len_dev must be int32")
+    hq = _check_decode_io(cache, q, len_dev, out)
     scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor")
     st = load().tq_decode_attention(ctypes.byref(layer.params), ctypes.byref(cache.cache),
-                                    q.data_ptr(), _dtype_code(q), int(q.shape[1]),
+                                    q.data_ptr(), _dtype_code(q), hq,
                                     len_dev.data_ptr(), int(max_len), scale, out.data_ptr(),
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream))
@@ -235,15 +268,16 @@ def tq_decode_attention_window(layer: Layer, cache: CompressedCache, q: torch.Te
     """Decode over the compressed cache plus a window of recent tokens kept
     exactly: win_k, win_v [B, H_kv, win_cap, d] (fp32/bf16, contiguous),
     win_len_dev [B] int32 device (valid slots per sequence)."""
-    if len_dev.dtype != torch.int32 or win_len_dev.dtype != torch.int32:
-        raise TypeError("len_dev and win_len_dev must be int32")
-    if win_k.dtype != win_v.dtype:
-        raise TypeError("win_k and win_v must share a dtype")
-    if not (win_k.is_contiguous() and win_v.is_contiguous()):
-        raise ValueError("win_k and win_v must be contiguous")
+    hq = _check_decode_io(cache, q, len_dev, out)
+    if win_k.dim() != 4:
+        raise ValueError("win_k must be [B, H_kv, win_cap, d]")
+    wshape = (cache.batch, cache.h_kv, int(win_k.shape[2]), int(q.shape[2]))
+    _check_rows("win_k", win_k, wshape, (torch.float32, torch.bfloat16), cache.buffer.device)
+    _check_rows("win_v", win_v, wshape, (win_k.dtype,), cache.buffer.device)
+    _check_rows("win_len_dev", win_len_dev, (cache.batch,), (torch.int32,), cache.buffer.device)
     scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
     st = load().tq_decode_attention_window(ctypes.byref(layer.params), ctypes.byref(cache.cache),
-                                           q.data_ptr(), _dtype_code(q), int(q.shape[1]),
+                                           q.data_ptr(), _dtype_code(q), hq,
                                            len_dev.data_ptr(), int(max_len), win_k.data_ptr(),
                                            win_v.data_ptr(), _dtype_code(win_k), win_len_dev.data_ptr(),
                                            int(win_k.shape[2]), scale, out.data_ptr(),
@@ -258,11 +292,10 @@ def tq_decode_attention_noalloc(layer: Layer, cache: CompressedCache, q: torch.T
                                 softmax_scale: float | None = None, stream=None) -> None:
     """Decode attention for callers that cannot allocate a workspace: the
     scratch is the library's fixed 8 MiB device array (see include/tq.h)."""
-    if len_dev.dtype != torch.int32:
-        raise TypeError("len_dev must be int32")
+    hq = _check_decode_io(cache, q, len_dev, out)
     scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
     st = load().tq_decode_attention_noalloc(ctypes.byref(layer.params), ctypes.byref(cache.cache),
-                                            q.data_ptr(), _dtype_code(q), int(q.shape[1]),
+                                            q.data_ptr(), _dtype_code(q), hq,
                                             len_dev.data_ptr(), int(max_len), scale,
                                             out.data_ptr(), _stream(stream))
     _check("tq_decode_attention_noalloc", st)
@@ -281,10 +314,12 @@ def tq_prefill_attention(layer: Layer, cache: CompressedCache, q: torch.Tensor,
     """Causal attention of a chunk over the compressed cache (the chunk already
     appended): q [B, T, H_q, d] (fp32/bf16, contiguous), len_dev [B] int32
     device (cached tokens, the chunk included), out [B, T, H_q, d] fp32."""
-    if len_dev.dtype != torch.int32:
-        raise TypeError("len_dev must be int32")
-    if not q.is_contiguous() or q.dim() != 4:
+    if q.dim() != 4:
         raise ValueError("q must be a contiguous [B, T, H_q, d] tensor")
+    dev = cache.buffer.device
+    _check_rows("q", q, (cache.batch,) + tuple(q.shape[1:]), (torch.float32, torch.bfloat16), dev)
+    _check_rows("len_dev", len_dev, (cache.batch,), (torch.int32,), dev)
+    _check_rows("out", out, tuple(q.shape), (torch.float32,), dev)
     scale = (1.0 / layer.d ** 0.5) if softmax_scale is None else float(softmax_scale)
     st = load().tq_prefill_attention(ctypes.byref(layer.params), ctypes.byref(cache.cache),
                                      q.data_ptr(), _dtype_code(q), int(q.shape[2]), int(q.shape[1]),
@@ -304,6 +339,27 @@ def prefill_workspace_for(layer: Layer, cache: CompressedCache, h_q: int, t_chun
     if n == 0:
         raise TQError("tq_prefill_workspace_size", 1)
     return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def tq_set_wait_limit_ns(ns: int) -> None:
+    """Time limit of the kernels' bounded waits for later calls (0: the
+    default, 2 s).  For tests of the timeout path."""
+    _check("tq_set_wait_limit_ns", load().tq_set_wait_limit_ns(int(ns)))
+
+
+def tq_device_errors(clear: bool = False) -> int:
+    """Synchronise the current device and return its sticky error word
+    (ERRF_* bits of kernels that gave up on a bounded wait); optionally
+    reset it."""
+    v = ctypes.c_uint32(0)
+    _check("tq_device_errors", load().tq_device_errors(ctypes.byref(v), int(bool(clear))))
+    return int(v.value)
+
+
+def decode_status(workspace: torch.Tensor) -> int:
+    """The status word a decode call left in its workspace (first int32):
+    nonzero if a kernel of that call gave up on a bounded wait."""
+    return int(workspace[:4].view(torch.int32).item())
 
 
 def tq_dequantize(layer: Layer, cache: CompressedCache, b: int, start: int, count: int,

@@ -170,3 +170,36 @@ def oracle_decode(layer: OracleLayer, q: np.ndarray, kes: list, ves: list, lengt
         recs.append({k2: v2[start:start + length] for k2, v2 in r.items()})
     rec = attention.stack_heads(recs)
     return attention.decode_one_sequence(q, rec, layer.pi, layer.s, layer.cent, layer.group)
+
+
+def fill_cache_gpu(glayer, cache, wl, lengths, device="cuda") -> None:
+    """Quantize-append every sequence's synthetic K/V (the workload's 8192-token
+    chunks drawn on the device) up to lengths[b] tokens, one call per chunk."""
+    chunk = workloads.TOKEN_CHUNK
+    lens = [0] * wl.batch
+    for c in range((max(lengths) + chunk - 1) // chunk):
+        t0 = c * chunk
+        nnew = [max(0, min(lengths[b] - t0, chunk)) for b in range(wl.batch)]
+        if max(nnew) == 0:
+            break
+        T = max(nnew)
+        ks, vs = [], []
+        for b in range(wl.batch):
+            k, v = workloads.kv_chunk(wl, b, c, device)
+            ks.append(k[:T])
+            vs.append(v[:T])
+        k = torch.stack(ks).contiguous()
+        v = torch.stack(vs).contiguous()
+        tq.tq_quantize_append(glayer, cache, k, v, lens, nnew)
+        lens = [lens[b] + nnew[b] for b in range(wl.batch)]
+        del k, v, ks, vs
+    torch.cuda.synchronize()
+
+
+def oracle_decode_head(layer: OracleLayer, spec, buf: np.ndarray, b: int, h: int, n: int,
+                       q_heads: np.ndarray) -> np.ndarray:
+    """Oracle decode of the G query heads of KV head h of sequence b over the
+    first n records of the library's cache bytes (read with the oracle's own
+    layout reader): [G, d]."""
+    rec = attention.stack_heads([spec.read(buf, b, h, 0, n)])
+    return attention.decode_one_sequence(q_heads, rec, layer.pi, layer.s, layer.cent, layer.group)

@@ -1,8 +1,9 @@
 """GPU parity: the CUDA path, called through the C ABI, against the oracle on
 the same seeded inputs.
 
-Quantize-append: codes and signs bit-exact outside the 1e-6 bands (band
-count <= 1e-4), value codes/scales/zeros exact, norms within 1e-3 relative.
+Quantize-append: codes and signs bit-exact outside the 1e-6 bands, value
+codes and scales outside the value band (band counts <= 1e-4 of the
+coordinates), zeros exact, norms within 1e-3 relative.
 Decode: the oracle's own encoding is packed (by the oracle's layout writer)
 into the device cache, so the CUDA decode and the oracle decode read the same
 records; outputs within 1e-3 relative per (b, h_q) row.
@@ -13,7 +14,7 @@ import pytest
 import torch
 
 from kv_cache_quantization_turboquantprod_b200 import tq, workloads
-from oracle import layout
+from oracle import attention, layout
 
 import parity_util as pu
 
@@ -203,7 +204,8 @@ def _run_decode(glayer, wl, buf, lengths, q, max_len=None):
     return out.cpu().numpy()
 
 
-@pytest.mark.parametrize("name", ["tiny", "llama8b", "qwen15b_512", "qwen15b_4096"])
+@pytest.mark.parametrize("name", ["tiny", "llama8b", "qwen15b_512", "qwen15b_4096", "qwen15b_8192",
+                                  "qwen15b_16384"])
 def test_decode_parity(name):
     wl = workloads.by_name(name)
     glayer, olayer, spec = _setup(wl)
@@ -299,10 +301,12 @@ def test_dequantize_parity():
 
 @pytest.mark.parametrize("name", ["tiny", "llama8b"])
 def test_end_to_end_quantize_then_decode(name):
-    """GPU quantize -> GPU decode against oracle quantize -> oracle decode.
-    The two caches can differ in band coordinates and in the last fp16 bit
-    of a norm, so the bar here is 5e-3; the 1e-3 bar is held by the
-    component tests above."""
+    """GPU quantize -> GPU decode, held to 1e-3 in two steps: the GPU's records
+    equal the oracle's encoding outside the bands (checked here), and the GPU
+    decode of those records equals the oracle's decode of the same records.
+    When no record differs at all (no banded code took the other cell, no norm
+    differs in its last fp16 bit), the GPU result is also held to 1e-3 against
+    the oracle's own quantize -> decode chain."""
     wl = workloads.by_name(name)
     glayer, olayer, spec = _setup(wl)
     cache = tq.CompressedCache(glayer, wl.batch, wl.h_kv, wl.capacity)
@@ -316,11 +320,26 @@ def test_end_to_end_quantize_then_decode(name):
     out = torch.empty((1, wl.h_q, 128), device=DEV)
     tq.tq_decode_attention(glayer, cache, q.to(DEV), len_dev, n, out, ws)
     torch.cuda.synchronize()
-    kes, ves = pu.oracle_records_for(olayer, k.float().numpy(), v.float().numpy())
+    got = out[0].cpu().numpy()
+    buf = cache.buffer.cpu().numpy()
+    kf, vf = k.float().numpy(), v.float().numpy()
+    kes, ves = pu.oracle_records_for(olayer, kf, vf)
+    stats = None
+    identical = True
+    for h in range(wl.h_kv):
+        stats = pu.compare_records(spec, buf, 0, h, 0, kes[h], ves[h], stats, olayer, kf[:, h])
+        rec = spec.read(buf, 0, h, 0, n)
+        identical &= all(np.array_equal(rec[f], pu.logical(kes[h], ves[h])[f]) for f in rec)
+    pu.check_band_fraction(stats)
+    rec = attention.stack_heads([spec.read(buf, 0, h, 0, n) for h in range(wl.h_kv)])
+    ref_dev = attention.decode_one_sequence(q[0].float().numpy(), rec, olayer.pi, olayer.s,
+                                            olayer.cent, olayer.group)
+    assert pu.row_rel_err(got, ref_dev) <= pu.REL_TOL
     ref = pu.oracle_decode(olayer, q[0].float().numpy(), kes, ves, n)
-    err = pu.row_rel_err(out[0].cpu().numpy(), ref)
-    print(name, "end-to-end row rel err", err)
-    assert err <= 5e-3
+    err = pu.row_rel_err(got, ref)
+    print(name, "records identical:", identical, "end-to-end row rel err", err, stats)
+    if identical:
+        assert err <= pu.REL_TOL
 
 
 @pytest.mark.parametrize("kb,vb", [(2, 2), (4, 2), (3, 4), (4, 3)])

@@ -1,0 +1,150 @@
+"""GPU checks of the failure paths and of the codebook fallback.
+
+* Bounded waits: with the library's wait limit set to one nanosecond, a
+  normal-sized decode call and a normal-sized tensor-core quantize-append give
+  up on their waits.  Each call still returns, the device still answers, the
+  failure shows (decode: the workspace status word is nonzero and every
+  output row is NaN; quantize-append: the appended records carry NaN norms;
+  both: the device's sticky error word), and with the default limit restored
+  the very next calls pass parity, so the kernels freed their tensor memory.
+  No fault is injected: the waits simply run out of time.
+* Asymmetric codebooks in the shapes where their operand planes fit in tensor
+  memory only once run the SIMT split-K kernel (chosen on the device); parity
+  at 16 tiles per CTA in every such shape.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_quantization_turboquantprod_b200 import tq, workloads
+from oracle import attention, layout
+
+import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from kv_cache_quantization_turboquantprod_b200 import build
+    build.build()
+    tq.load()
+
+
+def _setup(wl):
+    _, pi32, s32 = workloads.layer_matrices(wl)
+    glayer = pu.gpu_layer(pi32, s32, wl.key_bits, wl.value_bits)
+    olayer = pu.OracleLayer(pi32, s32, wl.key_bits, wl.value_bits)
+    spec = layout.CacheSpec(wl.batch, wl.h_kv, wl.capacity, wl.d, wl.key_bits,
+                            wl.value_bits, wl.group)
+    return glayer, olayer, spec
+
+
+def _decode(glayer, cache, q, lengths, max_len):
+    len_dev = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    ws = tq.workspace_for(glayer, cache, q.shape[1], max_len)
+    out = torch.zeros((q.shape[0], q.shape[1], 128), dtype=torch.float32, device=DEV)
+    tq.tq_decode_attention(glayer, cache, q, len_dev, max_len, out, ws)
+    return out, ws
+
+
+def test_decode_wait_timeout_reports_and_recovers():
+    wl = workloads.scaled(workloads.batched(), batch=8, lengths=(8192,) * 8, capacity=8192,
+                          name="timeout")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, wl.batch, wl.h_kv, wl.capacity)
+    pu.fill_cache_gpu(glayer, cache, wl, list(wl.lengths))
+    q = workloads.queries(wl, 0, device=DEV)
+    tq.tq_device_errors(clear=True)
+    try:
+        tq.tq_set_wait_limit_ns(1)
+        out, ws = _decode(glayer, cache, q, list(wl.lengths), 8192)
+        torch.cuda.synchronize()
+    finally:
+        tq.tq_set_wait_limit_ns(0)
+    assert tq.decode_status(ws) != 0
+    assert torch.isnan(out).all()
+    assert tq.tq_device_errors(clear=True) & tq.ERRF_DECODE_WAIT
+    # the device answers and the same call passes with the default limit
+    out, ws = _decode(glayer, cache, q, list(wl.lengths), 8192)
+    torch.cuda.synchronize()
+    assert tq.decode_status(ws) == 0
+    assert tq.tq_device_errors() == 0
+    got = out.cpu().numpy()
+    buf = cache.buffer.cpu().numpy()
+    qf = q.float().cpu().numpy()
+    G = wl.gqa
+    for b, h in [(0, 0), (5, 3), (7, 7)]:
+        ref = pu.oracle_decode_head(olayer, spec, buf, b, h, 8192, qf[b, h * G:(h + 1) * G])
+        assert pu.row_rel_err(got[b, h * G:(h + 1) * G], ref) <= pu.REL_TOL
+
+
+def test_quantize_wait_timeout_reports_and_recovers():
+    n = workloads.TOKEN_CHUNK
+    wl = workloads.scaled(workloads.longctx(), lengths=(n,) * 4, capacity=n, name="qtimeout")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, wl.batch, wl.h_kv, n, zero=True)
+    kv = [workloads.kv_chunk(wl, b, 0, DEV) for b in range(wl.batch)]
+    k = torch.stack([x[0] for x in kv]).contiguous()
+    v = torch.stack([x[1] for x in kv]).contiguous()
+    tq.tq_device_errors(clear=True)
+    try:
+        tq.tq_set_wait_limit_ns(1)
+        tq.tq_quantize_append(glayer, cache, k, v, [0] * wl.batch)
+        torch.cuda.synchronize()
+    finally:
+        tq.tq_set_wait_limit_ns(0)
+    assert tq.tq_device_errors(clear=True) & tq.ERRF_QUANTIZE_WAIT
+    buf = cache.buffer.cpu().numpy()
+    nk = np.concatenate([spec.read(buf, b, h, 0, n)["nk16"] for b in range(wl.batch)
+                         for h in range(wl.h_kv)])
+    assert np.isnan(nk).any()
+    # the same append with the default limit: every record of two heads exact
+    tq.tq_quantize_append(glayer, cache, k, v, [0] * wl.batch)
+    torch.cuda.synchronize()
+    assert tq.tq_device_errors() == 0
+    buf = cache.buffer.cpu().numpy()
+    stats = None
+    for b, h in [(0, 0), (3, 7)]:
+        kk = k[b, :, h].float().cpu().numpy()
+        ke, ve = olayer.encode(kk, v[b, :, h].float().cpu().numpy())
+        stats = pu.compare_records(spec, buf, b, h, 0, ke, ve, stats, olayer, kk)
+    pu.check_band_fraction(stats)
+
+
+@pytest.mark.parametrize("kb,vb,h_q", [(3, 2, 32), (3, 2, 64), (4, 2, 32), (3, 3, 48)])
+def test_asymmetric_codebook_long_splits(kb, vb, h_q):
+    """32 sequences x 8 KV heads x 4096 tokens (16 tiles per CTA), a shifted
+    and stretched codebook: the shapes whose asymmetric planes fit in tensor
+    memory once route to the SIMT split-K kernel; sampled rows match the
+    oracle run on the device's records with the same codebook."""
+    n, B, hkv = 4096, 32, 8
+    assert tq.load() is not None
+    wl = dataclasses.replace(workloads.batched(), batch=B, h_kv=hkv, h_q=h_q, key_bits=kb,
+                             value_bits=vb, lengths=(n,) * B, capacity=n, name=f"asym_long{kb}{vb}{h_q}")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, B, hkv, n)
+    pu.fill_cache_gpu(glayer, cache, wl, [n] * B)
+    m = len(olayer.cent)
+    cent = np.asarray(olayer.cent, np.float64) * (1.0 + 0.1 * np.arange(m) / m) + 0.02
+    cent = np.asarray(cent.astype(np.float32), np.float64)
+    olayer.cent = cent
+    glayer.centroids.copy_(torch.tensor(cent, dtype=torch.float32))
+    q = workloads.queries(wl, 0, device=DEV)
+    out, ws = _decode(glayer, cache, q, [n] * B, n)
+    torch.cuda.synchronize()
+    assert tq.decode_status(ws) == 0
+    got = out.cpu().numpy()
+    buf = cache.buffer.cpu().numpy()
+    qf = q.float().cpu().numpy()
+    G = h_q // hkv
+    for b, h in [(0, 0), (13, 4), (31, 7)]:
+        rec = attention.stack_heads([spec.read(buf, b, h, 0, n)])
+        ref = attention.decode_one_sequence(qf[b, h * G:(h + 1) * G], rec, olayer.pi, olayer.s,
+                                            olayer.cent, olayer.group)
+        assert pu.row_rel_err(got[b, h * G:(h + 1) * G], ref) <= pu.REL_TOL, (b, h)

@@ -193,3 +193,35 @@ def test_prefill_tokens_per_pass():
     assert g(ctypes.byref(P), 12, 8, 8) == 0     # not a multiple of h_kv
     assert g(ctypes.byref(P), 32, 8, 0) == 0
     assert g(None, 32, 8, 8) == 0
+
+
+def test_noalloc_validation_before_launch():
+    """The no-allocation entry point runs the same host checks as
+    tq_decode_attention before it looks up its scratch or launches anything:
+    a misaligned Pi or S (read with 16-byte loads) is rejected here rather
+    than faulting on the device."""
+    lib = tq.load()
+    C = tq.Cache(2, 8, 256, 1 << 20)
+    f = lib.tq_decode_attention_noalloc
+    q, ln, out = 1 << 22, 1 << 23, 1 << 24
+
+    def call(P, **kw):
+        return f(ctypes.byref(P) if P is not None else None, ctypes.byref(C), kw.get("q", q), 1,
+                 kw.get("hq", 32), ln, kw.get("ml", 256), 0.088, kw.get("out", out), None)
+
+    assert call(tq.Params(128, 3, 2, 32, 264, 256, 256, 256)) == 1   # Pi not 16-byte aligned
+    assert call(tq.Params(128, 3, 2, 32, 256, 260, 256, 256)) == 1   # S not 16-byte aligned
+    assert call(None) == 1
+    assert call(_params(d=64)) == 2
+    assert call(_params(), q=None) == 1
+    assert call(_params(), q=q + 4) == 1      # q alignment
+    assert call(_params(), out=out + 4) == 1  # out alignment
+    assert call(_params(), hq=12) == 1
+    assert call(_params(), ml=257) == 1
+
+
+def test_wait_limit_and_error_word_entry_points():
+    lib = tq.load()
+    assert lib.tq_set_wait_limit_ns(5000) == 0
+    assert lib.tq_set_wait_limit_ns(0) == 0       # back to the default
+    assert lib.tq_device_errors(None, 0) == 1     # null pointer, checked before the device
