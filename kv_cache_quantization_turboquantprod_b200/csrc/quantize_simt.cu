@@ -11,7 +11,8 @@
 // A persistent CTA keeps Pi and S in shared memory (rows padded to 129
 // floats so both row- and column-direction walks are bank-conflict free) and
 // encodes 16 vectors per pass: three 128x128 mat-vecs per vector (Pi u,
-// Pi^T c, S r) in fp32 with exact fp32 accumulation order per output.
+// Pi^T c, S r) in fp32 with exact fp32 accumulation order per output.  A
+// sketch component within 1e-5 of zero has its sign decided again in float64.
 #include "tq_common.cuh"
 #include "tq_kernels.h"
 
@@ -36,6 +37,7 @@ struct QuantSmem {
   float nk[kNV];
   float cent[16];
   float bnd[16];
+  uint32_t nearw[kNV][4];  // sketch components to re-decide in float64
 };
 
 __device__ __forceinline__ void vec_coords(const AppendArgs &a, long long id, int &b,
@@ -75,6 +77,7 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
   for (long long chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
     const long long id0 = chunk * kNV;
 
+    if (tid < kNV * 4) S.nearw[tid >> 2][tid & 3] = 0u;
     // ---- phase 0: load, normalise keys; quantize values ----------------
     for (int vi = warp; vi < kNV; vi += kThreads / 32) {
       int b, t, h;
@@ -243,6 +246,8 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
         const bool zero = !(S.nk[vi] > 0.f);
         const int bit = (!zero && acc[v] >= 0.f) ? 1 : 0;
         const unsigned word = __ballot_sync(0xffffffffu, bit);
+        const unsigned nearb = __ballot_sync(0xffffffffu, valid && !zero && fabsf(acc[v]) < kSignRefineZ);
+        if (lane == 0 && nearb) S.nearw[vi][i >> 5] = nearb;
         if (valid) {
           const int pos = a.lens[b] + t;
           uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
@@ -257,6 +262,35 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
           }
         }
       }
+    }
+    __syncthreads();
+
+    // ---- phase 4: sketch components next to zero, signs again in float64 --
+    for (int vi = warp; vi < kNV; vi += kThreads / 32) {
+      uint32_t nw[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) nw[w] = S.nearw[vi][w];
+      if (!(nw[0] | nw[1] | nw[2] | nw[3])) continue;
+      int b, t, h;
+      bool valid;
+      vec_coords(a, id0 + vi, b, t, h, valid);  // flagged vectors are valid
+      const int pos = a.lens[b] + t;
+      uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
+      const int slot = pos % kTile;
+      uint32_t planes[3][4], sw[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+          planes[p][w] = p < L.mb ? *reinterpret_cast<const uint32_t *>(tile + L.kplanes + p * kPlaneBytes +
+                                                                        slot * kRowBytes + 4 * w)
+                                  : 0u;
+        sw[w] = *reinterpret_cast<const uint32_t *>(tile + L.signs + slot * kRowBytes + 4 * w);
+      }
+      const size_t kbase = (((size_t)b * a.T + t) * a.h_kv + h) * kD;
+      refine_signs_f64(a.pi, a.s, S.cent, a.k, a.dtype, kbase, planes, nw, sw, 0);
+      if (lane == 0)
+        *reinterpret_cast<uint4 *>(tile + L.signs + slot * kRowBytes) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
     }
     __syncthreads();
   }

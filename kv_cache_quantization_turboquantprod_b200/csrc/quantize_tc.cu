@@ -556,21 +556,39 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       if (!qwait(&S.d3_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
       uint32_t sw[4] = {0u, 0u, 0u, 0u};
+      uint32_t nearw[4] = {0u, 0u, 0u, 0u};  // |S r| below the refinement threshold
+      // D = (S r) x 2^21 (R x 2^13 times S x 2^8)
+      constexpr float kNearZ = kSignRefineZ * 2097152.f;
       tmem_ld16(dcol, dA);
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t(&d)[16] = (c & 1) ? dB : dA;
         if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
-        uint32_t wv = 0u;
+        uint32_t wv = 0u, nv = 0u;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) wv |= (__uint_as_float(d[e]) >= 0.f ? 1u : 0u) << e;
+        for (int e = 0; e < 16; ++e) {
+          const float z = __uint_as_float(d[e]);
+          wv |= (z >= 0.f ? 1u : 0u) << e;
+          nv |= (fabsf(z) < kNearZ ? 1u : 0u) << e;
+        }
         sw[c >> 1] |= (zero ? 0u : wv) << (16 * (c & 1));
+        nearw[c >> 1] |= (zero || !valid ? 0u : nv) << (16 * (c & 1));
         if (c < 7) tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.d_free[g]);
+      // sketch components next to zero: the sign again in float64 (rare)
+      unsigned need = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1] | nearw[2] | nearw[3]) != 0u);
+      if (need) {
+        const size_t kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;
+        while (need) {
+          const int src = __ffs(need) - 1;
+          need &= need - 1;
+          refine_signs_f64(a.pi, a.s, S.cent, a.k, a.dtype, kbase, planes, nearw, sw, src);
+        }
+      }
       if (valid) {
         *reinterpret_cast<uint4 *>(tp + L.signs + slot * kRowBytes) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
         const float rn = zero ? 0.f : sqrtf(rr) * (1.f / kRScale);

@@ -124,4 +124,85 @@ __device__ __forceinline__ void stage_matrix(float *dst, int pad, const float *s
 // QJL constant sqrt(pi/2) / d.
 __host__ __device__ constexpr float qjl_kappa() { return 1.2533141373155003f / kD; }
 
+// Sketch components |(S r)_j| below this are re-decided in float64: the
+// single-precision paths (tensor-core hi/lo products, fp32 norms) can be off
+// by up to ~1e-6 there, and the sign of such a component is the key's stored
+// QJL bit.
+constexpr float kSignRefineZ = 1e-5f;
+
+__device__ __forceinline__ double warp_sum_f64(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Warp-cooperative float64 re-decision of QJL sign bits for the key row of
+// lane `src` (all 32 lanes call it together).  Lane src passes its row's key
+// (element offset kbase into k), its Lloyd-Max code bit-planes (three planes
+// of four 32-coordinate words, planes beyond the code width zero), the mask of coordinates to re-decide (near) and
+// its sign words (sw), which it gets back corrected.  In float64: ||k||,
+// u = k / ||k||, r = u - Pi^T c (c = centroids of the stored codes) and, for
+// every masked j, (S r)_j; the stored bit is [(S r)_j >= 0].  Pi and S are
+// read row-major from global memory (four coordinates per lane).
+__device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s, const float *cent,
+                                                 const void *k, tq_dtype dt, size_t kbase,
+                                                 const uint32_t (&planes)[3][4], const uint32_t (&near)[4],
+                                                 uint32_t (&sw)[4], int src) {
+  const int lane = threadIdx.x & 31;
+  uint32_t pl[3][4], nw[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int p = 0; p < 3; ++p) pl[p][w] = __shfl_sync(0xffffffffu, planes[p][w], src);
+    nw[w] = __shfl_sync(0xffffffffu, near[w], src);
+  }
+  const unsigned long long kb = __shfl_sync(0xffffffffu, (unsigned long long)kbase, src);
+  double x[4], ss = 0.0;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    x[m] = (double)load_elem(k, dt, kb + 4 * lane + m);
+    ss = fma(x[m], x[m], ss);
+  }
+  const double nk = sqrt(warp_sum_f64(ss));
+  double pc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t b0 = pl[0][w], b1 = pl[1][w], b2 = pl[2][w];
+#pragma unroll 4
+    for (int q = 0; q < 32; ++q) {
+      const int idx = (int)((b0 & 1u) | ((b1 & 1u) << 1) | ((b2 & 1u) << 2));
+      b0 >>= 1;
+      b1 >>= 1;
+      b2 >>= 1;
+      const double c = (double)cent[idx];
+      const float4 row = *reinterpret_cast<const float4 *>(pi + (size_t)(32 * w + q) * kD + 4 * lane);
+      pc[0] = fma((double)row.x, c, pc[0]);
+      pc[1] = fma((double)row.y, c, pc[1]);
+      pc[2] = fma((double)row.z, c, pc[2]);
+      pc[3] = fma((double)row.w, c, pc[3]);
+    }
+  }
+  double r[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) r[m] = x[m] / nk - pc[m];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t bits = nw[w];
+    while (bits) {
+      const int j = 32 * w + __ffs(bits) - 1;
+      bits &= bits - 1;
+      const float4 srow = *reinterpret_cast<const float4 *>(s + (size_t)j * kD + 4 * lane);
+      double part = (double)srow.x * r[0];
+      part = fma((double)srow.y, r[1], part);
+      part = fma((double)srow.z, r[2], part);
+      part = fma((double)srow.w, r[3], part);
+      const double z = warp_sum_f64(part);
+      if (lane == src) {
+        const uint32_t bit = 1u << (j & 31);
+        sw[w] = z >= 0.0 ? (sw[w] | bit) : (sw[w] & ~bit);
+      }
+    }
+  }
+}
+
 }  // namespace tq
