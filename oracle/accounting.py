@@ -11,6 +11,11 @@ Reading for the record size: fp16 norms and fp16 scale+zero per value group
 (the only layout that gives the audit's printed ratios, see
 tests/test_oracle_accounting.py); codebook = centroids + decision boundaries
 (a few dozen bytes, below the printed precision).
+
+TurboQuant-MSE values ("03. Results & Benchmarks", "At a Glance ->
+Compression": 3 bits per coordinate for keys and values, 1,288 KB -> 257 KB,
+5.02x): 3-bit value cells plus one fp16 value norm, 102 bytes per (token,
+head) at 3-bit keys, so the data-only ratio is 512 / 102.
 """
 
 from __future__ import annotations
@@ -18,8 +23,8 @@ from __future__ import annotations
 from .layout import record_bytes
 
 
-def data_bytes(n_tokens, h_kv, d, key_bits, value_bits, group) -> int:
-    return n_tokens * h_kv * record_bytes(d, key_bits, value_bits, group)
+def data_bytes(n_tokens, h_kv, d, key_bits, value_bits, group, value_mode="group") -> int:
+    return n_tokens * h_kv * record_bytes(d, key_bits, value_bits, group, value_mode)
 
 
 def fp16_kv_bytes(n_tokens, h_kv, d) -> int:
@@ -35,9 +40,9 @@ def ring_bytes(h_kv, d, ring_tokens=128) -> int:
     return ring_tokens * h_kv * d * 2
 
 
-def ratios(n_tokens, h_kv, d, key_bits, value_bits, group) -> dict:
+def ratios(n_tokens, h_kv, d, key_bits, value_bits, group, value_mode="group") -> dict:
     fp16 = fp16_kv_bytes(n_tokens, h_kv, d)
-    data = data_bytes(n_tokens, h_kv, d, key_bits, value_bits, group)
+    data = data_bytes(n_tokens, h_kv, d, key_bits, value_bits, group, value_mode)
     over = per_layer_overhead(d, key_bits)
     ring = ring_bytes(h_kv, d)
     return {"data_only": fp16 / data,

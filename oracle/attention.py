@@ -28,7 +28,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .quant import dequantize_keys, dequantize_values, kappa
+from .quant import dequantize_keys, dequantize_values, dequantize_values_mse, kappa
 
 
 def rotate_query(q: np.ndarray, pi: np.ndarray, s: np.ndarray):
@@ -54,6 +54,14 @@ def score_keys(q: np.ndarray, idx, sign, nk16, rn16, pi, s, centroids) -> np.nda
     return np.asarray(nk16, np.float64) * (mse + qjl_term(sh, sign, rn16, d))
 
 
+def value_rows(rec: dict, h: int, pi, group: int, value_centroids=None) -> np.ndarray:
+    """Explicitly dequantized values of KV head h: group-quantized records
+    (codes, scale16, zero16) or TurboQuant-MSE records (vidx, nv16)."""
+    if "vidx" in rec:
+        return dequantize_values_mse(rec["vidx"][:, h], rec["nv16"][:, h], pi, value_centroids)
+    return dequantize_values(rec["codes"][:, h], rec["scale16"][:, h], rec["zero16"][:, h], group)
+
+
 def softmax_average(logits: np.ndarray, vhat: np.ndarray) -> np.ndarray:
     """sum_n softmax(logits)_n vhat_n, max-subtracted, float64."""
     m = np.max(logits)
@@ -63,14 +71,23 @@ def softmax_average(logits: np.ndarray, vhat: np.ndarray) -> np.ndarray:
 
 
 def decode_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
-                        softmax_scale: float | None = None) -> np.ndarray:
+                        softmax_scale: float | None = None,
+                        value_centroids=None) -> np.ndarray:
     """Decode attention for one sequence.
 
     q   [H_q, d] query
     rec logical cache fields of the sequence's cached tokens, each with a
-        leading [N, H_kv] (idx, sign, codes: [N, H_kv, d]; nk16, rn16:
-        [N, H_kv]; scale16, zero16: [N, H_kv, d/group])
+        leading [N, H_kv] (idx, sign: [N, H_kv, d]; nk16, rn16: [N, H_kv];
+        group-quantized values: codes [N, H_kv, d], scale16, zero16
+        [N, H_kv, d/group]; TurboQuant-MSE values: vidx [N, H_kv, d], nv16
+        [N, H_kv], with value_centroids the values' codebook)
     Returns out [H_q, d] float64.
+
+    TurboQuant-MSE values are accumulated in the rotated space,
+    acc = sum_n p_n nv16_n c[vidx_n], and rotated back once per head,
+    out = Pi^T acc (the value half of the fused one-pass decode of
+    "03. Results & Benchmarks", "Latency Benchmarks", with the value
+    reconstruction of the key encoder's MSE stage).
     """
     q = np.asarray(q, np.float64)
     hq, d = q.shape
@@ -79,21 +96,31 @@ def decode_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
         raise ValueError("decode needs at least one cached token")
     g = hq // hkv
     scale = 1.0 / np.sqrt(d) if softmax_scale is None else softmax_scale
+    mse_values = "vidx" in rec
     out = np.zeros((hq, d))
     for h in range(hkv):
-        vhat = dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
-                                 rec["zero16"][:, h], group)
+        if mse_values:
+            vrot = (np.asarray(rec["nv16"][:, h], np.float64)[:, None]
+                    * np.asarray(value_centroids, np.float64)[rec["vidx"][:, h]])
+        else:
+            vhat = dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
+                                     rec["zero16"][:, h], group)
         for j in range(g):
             qh = h * g + j
             sc = score_keys(q[qh], rec["idx"][:, h], rec["sign"][:, h],
                             rec["nk16"][:, h], rec["rn16"][:, h], pi, s, centroids)
-            out[qh] = softmax_average(sc * scale, vhat)
+            if mse_values:
+                acc = softmax_average(sc * scale, vrot)          # rotated space
+                out[qh] = acc @ np.asarray(pi, np.float64)       # Pi^T acc, as a row
+            else:
+                out[qh] = softmax_average(sc * scale, vhat)
     return out
 
 
 def decode_with_window(q: np.ndarray, rec: dict | None, win_k: np.ndarray, win_v: np.ndarray,
                        pi, s, centroids, group: int,
-                       softmax_scale: float | None = None) -> np.ndarray:
+                       softmax_scale: float | None = None,
+                       value_centroids=None) -> np.ndarray:
     """Decode attention over the compressed tokens of one sequence plus a
     window of recent tokens kept exactly ("turboquant/audit_claims.py",
     AUDIT 1: the store keeps the most recent 128 tokens uncompressed in
@@ -120,8 +147,7 @@ def decode_with_window(q: np.ndarray, rec: dict | None, win_k: np.ndarray, win_v
     for h in range(hkv):
         vparts = []
         if n:
-            vparts.append(dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
-                                            rec["zero16"][:, h], group))
+            vparts.append(value_rows(rec, h, pi, group, value_centroids))
         if w:
             vparts.append(win_v[:, h])
         values = np.concatenate(vparts, axis=0)
@@ -139,7 +165,8 @@ def decode_with_window(q: np.ndarray, rec: dict | None, win_k: np.ndarray, win_v
 
 
 def prefill_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
-                         softmax_scale: float | None = None) -> np.ndarray:
+                         softmax_scale: float | None = None,
+                         value_centroids=None) -> np.ndarray:
     """Causal attention of a chunk of T query tokens over the compressed cache
     of one sequence whose last T tokens are the chunk itself
     ("turboquant/audit_claims.py", AUDIT 7 and 8: long-context prefill as
@@ -161,12 +188,14 @@ def prefill_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids, group: int,
         if m <= 0:
             continue
         sub = {k: v[:m] for k, v in rec.items()}
-        out[t] = decode_one_sequence(q[t], sub, pi, s, centroids, group, softmax_scale)
+        out[t] = decode_one_sequence(q[t], sub, pi, s, centroids, group, softmax_scale,
+                                     value_centroids)
     return out
 
 
 def brute_force_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids,
-                             group: int, softmax_scale: float | None = None) -> np.ndarray:
+                             group: int, softmax_scale: float | None = None,
+                             value_centroids=None) -> np.ndarray:
     """softmax(K_hat q / sqrt d) V_hat over explicitly dequantized K and V
     (the dequantize-then-matmul pattern of the audit's hybrid path, AUDIT 4)."""
     q = np.asarray(q, np.float64)
@@ -178,8 +207,7 @@ def brute_force_one_sequence(q: np.ndarray, rec: dict, pi, s, centroids,
     for h in range(hkv):
         khat = dequantize_keys(rec["idx"][:, h], rec["sign"][:, h], rec["nk16"][:, h],
                                rec["rn16"][:, h], pi, s, centroids)
-        vhat = dequantize_values(rec["codes"][:, h], rec["scale16"][:, h],
-                                 rec["zero16"][:, h], group)
+        vhat = value_rows(rec, h, pi, group, value_centroids)
         for j in range(g):
             qh = h * g + j
             logits = (khat @ q[qh]) * scale

@@ -22,6 +22,10 @@ The pages do not fix a layout (reading).  The spec:
 * Inside a plane row, byte i, bit k (LSB = 0) holds coordinate 8 i + k.
 * Record bytes per (token, KV head): R = (mb + 1 + vb) d/8 + 4 + 4 d/group,
   tile_bytes = 128 R.
+* TurboQuant-MSE values (value_mode "mse"): section 3 holds vb bit-planes of
+  the values' Lloyd-Max cell indices at every vb, and section 5 holds the
+  value norms [128] x fp16 (2 bytes a token) instead of scale/zero pairs:
+  R = (mb + 1 + vb) d/8 + 4 + 2 (102 bytes at 3-bit keys and values).
 """
 
 from __future__ import annotations
@@ -31,16 +35,18 @@ import numpy as np
 TILE = 128
 
 
-def record_bytes(d: int, key_bits: int, value_bits: int, group: int) -> int:
+def record_bytes(d: int, key_bits: int, value_bits: int, group: int,
+                 value_mode: str = "group") -> int:
     mb = key_bits - 1
-    return (mb + 1 + value_bits) * d // 8 + 4 + 4 * (d // group)
+    tail = 2 if value_mode == "mse" else 4 * (d // group)
+    return (mb + 1 + value_bits) * d // 8 + 4 + tail
 
 
-def tile_bytes(d, key_bits, value_bits, group) -> int:
-    return TILE * record_bytes(d, key_bits, value_bits, group)
+def tile_bytes(d, key_bits, value_bits, group, value_mode="group") -> int:
+    return TILE * record_bytes(d, key_bits, value_bits, group, value_mode)
 
 
-def section_offsets(d, key_bits, value_bits, group) -> dict:
+def section_offsets(d, key_bits, value_bits, group, value_mode="group") -> dict:
     mb = key_bits - 1
     plane = TILE * d // 8
     off = {}
@@ -54,14 +60,14 @@ def section_offsets(d, key_bits, value_bits, group) -> dict:
     off["norms"] = o
     o += TILE * 4
     off["vsz"] = o
-    o += TILE * 4 * (d // group)
+    o += TILE * 2 if value_mode == "mse" else TILE * 4 * (d // group)
     off["end"] = o
     return off
 
 
-def cache_bytes(batch, h_kv, capacity, d, key_bits, value_bits, group) -> int:
+def cache_bytes(batch, h_kv, capacity, d, key_bits, value_bits, group, value_mode="group") -> int:
     assert capacity % TILE == 0
-    return batch * h_kv * (capacity // TILE) * tile_bytes(d, key_bits, value_bits, group)
+    return batch * h_kv * (capacity // TILE) * tile_bytes(d, key_bits, value_bits, group, value_mode)
 
 
 def _bits_to_plane_row(bits: np.ndarray) -> np.ndarray:
@@ -93,14 +99,16 @@ def _plane_row_to_bits(rows: np.ndarray, d: int) -> np.ndarray:
 
 
 class CacheSpec:
-    def __init__(self, batch, h_kv, capacity, d, key_bits, value_bits, group):
+    def __init__(self, batch, h_kv, capacity, d, key_bits, value_bits, group, value_mode="group"):
         self.batch, self.h_kv, self.capacity = batch, h_kv, capacity
         self.d, self.key_bits, self.value_bits, self.group = d, key_bits, value_bits, group
+        self.value_mode = value_mode
+        self.mse = value_mode == "mse"
         self.mb = key_bits - 1
         self.ntiles = capacity // TILE
-        self.tile_bytes = tile_bytes(d, key_bits, value_bits, group)
-        self.off = section_offsets(d, key_bits, value_bits, group)
-        self.nbytes = cache_bytes(batch, h_kv, capacity, d, key_bits, value_bits, group)
+        self.tile_bytes = tile_bytes(d, key_bits, value_bits, group, value_mode)
+        self.off = section_offsets(d, key_bits, value_bits, group, value_mode)
+        self.nbytes = cache_bytes(batch, h_kv, capacity, d, key_bits, value_bits, group, value_mode)
 
     def tile_base(self, b, h, t) -> int:
         return ((b * self.h_kv + h) * self.ntiles + t) * self.tile_bytes
@@ -124,8 +132,8 @@ class CacheSpec:
             buf[o:o + rowb] = _bits_to_plane_row((idx >> p) & 1)
         o = base + self.off["signs"] + slot * rowb
         buf[o:o + rowb] = _bits_to_plane_row(keyrec["sign"][i])
-        codes = valrec["codes"][i]
-        if self.value_bits == 2:
+        codes = valrec["vidx"][i] if self.mse else valrec["codes"][i]
+        if self.value_bits == 2 and not self.mse:
             o = base + self.off["vplanes"] + slot * (d // 4)
             buf[o:o + d // 4] = _codes_to_packed2_row(codes)
         else:
@@ -135,6 +143,10 @@ class CacheSpec:
         o = base + self.off["norms"] + slot * 4
         buf[o:o + 4] = np.array([keyrec["nk16"][i], keyrec["rn16"][i]],
                                 np.float16).view(np.uint8)
+        if self.mse:
+            o = base + self.off["vsz"] + slot * 2
+            buf[o:o + 2] = np.array([valrec["nv16"][i]], np.float16).view(np.uint8)
+            return
         ng = d // self.group
         o = base + self.off["vsz"] + slot * 4 * ng
         sz = np.stack([valrec["scale16"][i], valrec["zero16"][i]], axis=1)
@@ -160,8 +172,8 @@ class CacheSpec:
             put(base + self.off["kplanes"] + p * plane + slot * rowb,
                 _bits_to_plane_row((idx >> p) & 1))
         put(base + self.off["signs"] + slot * rowb, _bits_to_plane_row(keyrec["sign"]))
-        codes = np.asarray(valrec["codes"])
-        if self.value_bits == 2:
+        codes = np.asarray(valrec["vidx"] if self.mse else valrec["codes"])
+        if self.value_bits == 2 and not self.mse:
             put(base + self.off["vplanes"] + slot * (d // 4), _codes_to_packed2_row(codes))
         else:
             for p in range(self.value_bits):
@@ -169,6 +181,10 @@ class CacheSpec:
                     _bits_to_plane_row((codes >> p) & 1))
         nr = np.stack([keyrec["nk16"], keyrec["rn16"]], axis=1).astype(np.float16)
         put(base + self.off["norms"] + slot * 4, nr.view(np.uint8).reshape(n, 4))
+        if self.mse:
+            nv = np.asarray(valrec["nv16"]).astype(np.float16)
+            put(base + self.off["vsz"] + slot * 2, nv.view(np.uint8).reshape(n, 2))
+            return
         sz = np.stack([valrec["scale16"], valrec["zero16"]], axis=2).astype(np.float16)
         put(base + self.off["vsz"] + slot * 4 * ng, sz.reshape(n, 2 * ng).view(np.uint8))
 
@@ -194,7 +210,7 @@ class CacheSpec:
             idx |= _plane_row_to_bits(rows, d).astype(np.int64) << p
         sign = _plane_row_to_bits(get(base + self.off["signs"] + slot * rowb, rowb), d)
         codes = np.zeros((count, d), np.int64)
-        if self.value_bits == 2:
+        if self.value_bits == 2 and not self.mse:
             rows = get(base + self.off["vplanes"] + slot * (d // 4), d // 4)
             codes = _packed2_row_to_codes(rows, d).astype(np.int64)
         else:
@@ -203,6 +219,10 @@ class CacheSpec:
                 codes |= _plane_row_to_bits(rows, d).astype(np.int64) << p
         nr = get(base + self.off["norms"] + slot * 4, 4).copy().view(np.float16)
         nr = nr.astype(np.float64).reshape(count, 2)
+        if self.mse:
+            nv = get(base + self.off["vsz"] + slot * 2, 2).copy().view(np.float16)
+            return {"idx": idx, "sign": sign.astype(np.uint8), "nk16": nr[:, 0],
+                    "rn16": nr[:, 1], "vidx": codes, "nv16": nv.astype(np.float64).reshape(count)}
         sz = get(base + self.off["vsz"] + slot * 4 * ng, 4 * ng).copy().view(np.float16)
         sz = sz.astype(np.float64).reshape(count, ng, 2)
         return {"idx": idx, "sign": sign.astype(np.uint8), "nk16": nr[:, 0],
@@ -232,7 +252,7 @@ class CacheSpec:
                 idx[i] |= _plane_row_to_bits(buf[o:o + rowb], d).astype(np.int64) << p
             o = base + self.off["signs"] + slot * rowb
             sign[i] = _plane_row_to_bits(buf[o:o + rowb], d)
-            if self.value_bits == 2:
+            if self.value_bits == 2 and not self.mse:
                 o = base + self.off["vplanes"] + slot * (d // 4)
                 codes[i] = _packed2_row_to_codes(buf[o:o + d // 4], d)
             else:
@@ -242,8 +262,15 @@ class CacheSpec:
             o = base + self.off["norms"] + slot * 4
             nr = buf[o:o + 4].copy().view(np.float16).astype(np.float64)
             nk[i], rn[i] = nr[0], nr[1]
+            if self.mse:
+                o = base + self.off["vsz"] + slot * 2
+                sc[i, 0] = buf[o:o + 2].copy().view(np.float16).astype(np.float64)[0]
+                continue
             o = base + self.off["vsz"] + slot * 4 * ng
             sz = buf[o:o + 4 * ng].copy().view(np.float16).astype(np.float64).reshape(ng, 2)
             sc[i], ze[i] = sz[:, 0], sz[:, 1]
+        if self.mse:
+            return {"idx": idx, "sign": sign, "nk16": nk, "rn16": rn, "vidx": codes,
+                    "nv16": sc[:, 0].copy()}
         return {"idx": idx, "sign": sign, "nk16": nk, "rn16": rn,
                 "codes": codes, "scale16": sc, "zero16": ze}

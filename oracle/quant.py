@@ -32,6 +32,15 @@ rounding the exact quotient half-to-even and clamping.  In float64:
 For inputs of at most float32 precision, mx - mn and v - zero16 are exact in
 float64 and each quotient is within one float64 rounding of the exact one,
 so a float64 tie is an exact tie.
+
+TurboQuant-MSE values ("03. Results & Benchmarks", turboquant_cutile, "At a
+Glance -> Compression": 3 bits per coordinate for keys and values, a 5.02x
+smaller cache; "Live Generation": the value cache replaced by the 3-bit
+TurboQuant version): the MSE stage of the key encoder applied to values,
+with no QJL bit.  nv = ||v||; w = v / nv; y = Pi w; idx_j = #{t_i < y_j}
+against the vb-bit Lloyd-Max boundaries; nv stored as fp16.  The value is
+reconstructed as nv16 * Pi^T c[idx].  A zero vector stores nv = 0 and all-zero
+codes.
 """
 
 from __future__ import annotations
@@ -158,3 +167,26 @@ def dequantize_keys(idx: np.ndarray, sign: np.ndarray, nk16: np.ndarray,
     mse = c @ pi                          # Pi^T c, row by row
     qjl = sigma @ s                       # S^T sigma, row by row
     return nk16[:, None] * (mse + kappa(d) * rn16[:, None] * qjl)
+
+
+def encode_values_mse(values: np.ndarray, pi: np.ndarray, centroids: np.ndarray,
+                      boundaries: np.ndarray) -> dict:
+    """TurboQuant-MSE encoding of value vectors [n, d]: Lloyd-Max cells of the
+    rotated unit vector and the fp16 norm.  Returns vidx [n, d] int, nv16 [n]
+    (float64 holding fp16 values), vy [n, d] = Pi v / ||v|| (for boundary
+    bands) and the unrounded norm nv [n]."""
+    x = np.asarray(values, dtype=np.float64)
+    nv = np.sqrt(np.sum(x * x, axis=1))
+    zero = nv == 0.0
+    w = np.where(zero[:, None], 0.0, x / np.where(zero, 1.0, nv)[:, None])
+    y = w @ np.asarray(pi, np.float64).T          # y = Pi w, row by row
+    idx = bucketize(y, boundaries)
+    idx[zero] = 0
+    return {"vidx": idx, "nv16": fp16(nv), "vy": y, "nv": nv}
+
+
+def dequantize_values_mse(vidx: np.ndarray, nv16: np.ndarray, pi: np.ndarray,
+                          centroids: np.ndarray) -> np.ndarray:
+    """v_hat = nv16 * Pi^T c[vidx], float64 [n, d]."""
+    c = np.asarray(centroids, np.float64)[vidx]
+    return np.asarray(nv16, np.float64)[:, None] * (c @ np.asarray(pi, np.float64))
