@@ -335,6 +335,8 @@ def run_ours(args, rank, world, device):
         line["prefill"] = bench_prefill(layer, cache, len_after, max_len, wl, device, dec_bytes_all)
     if args.quantize and world == 1:
         line["quantize"] = bench_quantize(args, device)
+    if args.configs and world == 1:
+        line["configs"] = bench_configs(device, peak)
     return line
 
 
@@ -398,6 +400,83 @@ def bench_prefill(layer, cache, len_dev, max_len, wl, device, dec_bytes, t_chunk
     return {"t_chunk": t_chunk, "tokens_per_pass": per_pass, "passes": passes, "ms": ms,
             "query_tokens_s": B * t_chunk / (ms / 1e3),
             "record_gbs": passes * dec_bytes / (ms / 1e3) / 1e9}
+
+
+def _time_ms(fn, n=20, warmup=3):
+    """Median CUDA-event time of fn() over n runs after warm-up (ms)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return float(np.median(times))
+
+
+def _decode_line(wl, layer, cache, lengths, device, peak):
+    """Decode-call latency of a workload (median of 20) and its record bandwidth."""
+    q = workloads.queries(wl, 0, device=device)
+    len_dev = torch.tensor(lengths, dtype=torch.int32, device=device)
+    ml = max(lengths)
+    ws = tq.workspace_for(layer, cache, wl.h_q, ml, device=device)
+    out = torch.empty((wl.batch, wl.h_q, wl.d), dtype=torch.float32, device=device)
+    ms = _time_ms(lambda: tq.tq_decode_attention(layer, cache, q, len_dev, ml, out, ws))
+    rec = layer.record_bytes()
+    nbytes = float(sum(lengths)) * wl.h_kv * rec
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"decode_us": ms * 1e3, "ctx_tokens_s": sum(lengths) / (ms / 1e3),
+            "record_bytes_per_call": nbytes, "gbs": gbs, "frac_of_8tbs": gbs / 8000.0,
+            "frac_of_peak": gbs / peak}
+
+
+def bench_configs(device, peak):
+    """Every configuration of the measurement table at N = 1: tiny and
+    Llama-shaped decode (latency-bound, records L2-resident), the
+    Qwen-shaped context sweep 512 .. 16K, and the long-context decode at
+    131,072 tokens (the cache filled by 16 quantize-append chunks)."""
+    res = {}
+    for name in ("tiny", "llama8b"):
+        wl = workloads.by_name(name)
+        _, pi32, s32 = workloads.layer_matrices(wl)
+        layer = tq.Layer(pi32, s32, wl.key_bits, wl.value_bits, device=device)
+        cache = tq.CompressedCache(layer, wl.batch, wl.h_kv, wl.capacity, device=device)
+        k, v = workloads.kv_tokens(wl, 0, 0, wl.lengths[0], device=device)
+        k, v = k[None].contiguous(), v[None].contiguous()
+        q_ms = _time_ms(lambda: tq.tq_quantize_append(layer, cache, k, v, [0]))
+        line = _decode_line(wl, layer, cache, list(wl.lengths), device, peak)
+        line["quantize_us"] = q_ms * 1e3
+        line["quantize_mvec_s"] = wl.lengths[0] * wl.h_kv / (q_ms / 1e3) / 1e6
+        res[name] = line
+    sweep = {}
+    for n in workloads.QWEN_SWEEP:
+        wl = workloads.qwen15b(n)
+        _, pi32, s32 = workloads.layer_matrices(wl)
+        layer = tq.Layer(pi32, s32, wl.key_bits, wl.value_bits, device=device)
+        cache = tq.CompressedCache(layer, wl.batch, wl.h_kv, wl.capacity, device=device)
+        _fill_cache(wl, layer, cache, device)
+        sweep[str(n)] = _decode_line(wl, layer, cache, list(wl.lengths), device, peak)
+    res["qwen15b"] = sweep
+    wl = workloads.longctx()
+    _, pi32, s32 = workloads.layer_matrices(wl)
+    layer = tq.Layer(pi32, s32, wl.key_bits, wl.value_bits, device=device)
+    cache = tq.CompressedCache(layer, wl.batch, wl.h_kv, wl.capacity, device=device)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    _fill_cache(wl, layer, cache, device)
+    e1.record()
+    torch.cuda.synchronize()
+    line = _decode_line(wl, layer, cache, list(wl.lengths), device, peak)
+    line["fill_ms_16_chunks_with_input_generation"] = e0.elapsed_time(e1)
+    res["longctx"] = line
+    del cache
+    torch.cuda.empty_cache()
+    return res
 
 
 def bench_quantize(args, device):
@@ -494,11 +573,29 @@ def cpu_baseline(wl, pi32, s32, args, budget_s=10.0):
     dt = time.perf_counter() - t0
     # a ctx-token covers all H_kv heads: a (b, h) pair's n tokens are n / H_kv ctx-tokens
     value = done_tokens / wl.h_kv / dt
+    # the same sample on one thread (BLAS limited to one thread in-process)
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t1 = time.perf_counter()
+            j, tok1 = 0, 0.0
+            while True:
+                _oracle_decode_samples(samples, consts, wl.group)
+                tok1 += sum(n for _, _, n in samples)
+                j += 1
+                if time.perf_counter() - t1 > budget_s / 2 or j >= 20:
+                    break
+            one = {"value": tok1 / wl.h_kv / (time.perf_counter() - t1), "cores": 1,
+                   "repeats": j}
+    except Exception as e:  # threadpoolctl missing: report why
+        one = {"unavailable": str(e)}
     return {"value": value, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
             "blas_threads": _blas_threads(), "kind": "oracle",
             "sample": f"oracle decode of 2 (sequence, KV head) pairs x {max_tokens} tokens "
                       f"x {wl.gqa} query heads, repeated {i}x ({dt:.1f} s); "
-                      f"ctx-tokens counted as tokens / H_kv"}
+                      f"ctx-tokens counted as tokens / H_kv",
+            "single_thread": one}
 
 
 def run_reference(args, rank, world):
@@ -545,6 +642,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-quantize", dest="quantize", action="store_false",
                     help="skip the quantize-append Mvec/s measurement")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the per-configuration latency table")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

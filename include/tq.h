@@ -48,7 +48,10 @@
  *    the same cache region (or the same workspace) must be ordered by the
  *    caller.
  *  - Only d = 128 and group = 32 are built; other values return
- *    TQ_ERR_UNSUPPORTED.
+ *    TQ_ERR_UNSUPPORTED.  TurboQuant-MSE values (tq_value_mode) are encoded
+ *    by the SIMT quantize-append kernel and decoded by the SIMT split-K
+ *    kernel, accumulated in the rotated space and rotated back once per
+ *    head in the combine step.
  */
 #ifndef TQ_H_
 #define TQ_H_
@@ -80,6 +83,18 @@ typedef enum {
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* How values are stored. */
+typedef enum {
+  TQ_VALUES_GROUP = 0, /* asymmetric min/max quantization per group of 32
+                          channels, fp16 scale and zero ("turboquant/
+                          audit_claims.py", AUDIT 1: value_bits,
+                          value_group_size) */
+  TQ_VALUES_MSE = 1    /* TurboQuant-MSE: Lloyd-Max cells of the rotated unit
+                          value Pi v / ||v|| plus the fp16 norm ("03. Results &
+                          Benchmarks", "At a Glance -> Compression": 3 bits
+                          per coordinate for keys and values, 5.02x) */
+} tq_value_mode;
 
 /* Bits of the sticky per-device error word (tq_device_errors). */
 #define TQ_ERRF_DECODE_WAIT 1u   /* a decode kernel gave up on a bounded wait */
@@ -135,6 +150,11 @@ typedef struct {
                               values at GQA 6) decode runs the SIMT split-K
                               kernel for it (decided on the device per call) */
   const float *boundaries; /* [2^(key_bits-1) - 1] ascending decision boundaries */
+  int value_mode;          /* tq_value_mode */
+  const float *v_centroids;  /* TQ_VALUES_MSE: the values' codebook, [2^value_bits]
+                                ascending (tq_make_codebook(value_bits, d));
+                                NULL for TQ_VALUES_GROUP */
+  const float *v_boundaries; /* TQ_VALUES_MSE: [2^value_bits - 1] ascending */
 } tq_params;
 
 /*
@@ -155,6 +175,10 @@ typedef struct {
  *      4. norms [128] x {||k||, ||r||}, two little-endian fp16 per token;
  *      5. value groups [128][d/group] x {scale, zero}, two fp16 each.
  *    In a plane row, byte i bit k (LSB first) is coordinate 8 i + k.
+ *  - With TQ_VALUES_MSE, section 3 holds value_bits bit-planes of the
+ *    values' cell indices (at every value_bits, plane p = bit p) and section
+ *    5 holds the value norms [128] x fp16; R = (key_bits + value_bits) d/8 +
+ *    4 + 2 (102 bytes for 3-bit keys and values).
  *  - Record bytes per (token, KV head) R = (key_bits + value_bits) d/8 + 4
  *    + 4 d/group (100 bytes for 3-bit keys and 2-bit values at d = 128);
  *    tile_bytes = 128 R.
@@ -354,6 +378,17 @@ TQ_API tq_status tq_decode_attention_noalloc(const tq_params *p, const tq_cache 
  * TQ_OK.
  */
 TQ_API tq_status tq_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * tq_test_withhold_handoffs -- for tests of the timeout path only: while on
+ * (nonzero), the tensor-core kernels of later calls withhold one hand-off
+ * that their other roles wait for (decode: the tile copies; quantize-append:
+ * the loaded key operand), so those bounded waits run out after the wait
+ * limit and the failure reporting above can be observed.  Nothing faults:
+ * every wait is bounded and each kernel returns.  Off by default.  Always
+ * TQ_OK.
+ */
+TQ_API tq_status tq_test_withhold_handoffs(int on);
 
 /*
  * tq_device_errors -- synchronise the current device, then read (and, if

@@ -51,14 +51,15 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = a.h_q / a.h_kv;
-  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode);
   const float kappa = qjl_kappa();
   const float scale2 = a.softmax_scale * kLog2e;
 
-  __shared__ float cent[16];
+  __shared__ float cent[16], vcent[16];
   __shared__ float sm_m[4][kMaxG], sm_l[4][kMaxG];
   __shared__ float sm_acc[4][kMaxG][kD];
   if (threadIdx.x < (1 << L.mb)) cent[threadIdx.x] = a.centroids[threadIdx.x];
+  if (L.mse && threadIdx.x < (1 << L.vb)) vcent[threadIdx.x] = a.v_centroids[threadIdx.x];
 
   float qt[kMaxG][4], sh[kMaxG][4], acc[kMaxG][4], mrun[kMaxG], lrun[kMaxG];
 #pragma unroll
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
     }
     const int snib = (tp[L.signs + slot * kRowBytes + byte] >> shift) & 0xF;
     int code[4] = {0, 0, 0, 0};
-    if (L.vb == 2) {
+    if (L.vb == 2 && !L.mse) {
       const int pk = tp[L.vplanes + slot * kPackedRowBytes + lane];  // channels 4 lane .. 4 lane + 3
 #pragma unroll
       for (int k = 0; k < 4; ++k) code[k] = (pk >> (2 * k)) & 3;
@@ -110,14 +111,22 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
     }
     const __half2 nr = *reinterpret_cast<const __half2 *>(tp + L.norms + slot * 4);
     const float nk = __low2float(nr), rn = __high2float(nr);
-    const __half2 sz = *reinterpret_cast<const __half2 *>(tp + L.vsz + (slot * kGroups + grp) * 4);
-    const float vs = __low2float(sz), vz = __high2float(sz);
     float c[4], sg[4], vh[4];
+    if (L.mse) {
+      // TurboQuant-MSE values, kept in the rotated space: ||v|| c[cell]
+      const float nv = __half2float(*reinterpret_cast<const __half *>(tp + L.vsz + slot * 2));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) vh[k] = nv * vcent[code[k]];
+    } else {
+      const __half2 sz = *reinterpret_cast<const __half2 *>(tp + L.vsz + (slot * kGroups + grp) * 4);
+      const float vs = __low2float(sz), vz = __high2float(sz);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) vh[k] = fmaf((float)code[k], vs, vz);
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       c[k] = cent[idx[k]];
       sg[k] = ((snib >> k) & 1) ? 1.f : -1.f;
-      vh[k] = fmaf((float)code[k], vs, vz);
     }
     const float krn = kappa * rn;
 #pragma unroll
@@ -172,7 +181,8 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
 
 // ---------------------------------------------------------------------------
 // combine: out[b][hq][:] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
-// A call whose kernels gave up on a bounded wait (status word nonzero) gets
+// (TurboQuant-MSE values: the partials are in the rotated space and the
+// merged accumulator is rotated back once, Pi^T acc).  A call whose kernels gave up on a bounded wait (status word nonzero) gets
 // NaN rows, so a timeout never comes back as a plausible result.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
@@ -194,6 +204,15 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
       num = fmaf(src[s * (kD + 2) + j], f, num);
       den = fmaf(src[s * (kD + 2) + kD + 1], f, den);
     }
+  }
+  if (a.value_mode == TQ_VALUES_MSE) {
+    // the merged accumulator is in the rotated space: out_j = (Pi^T acc)_j
+    __shared__ float acc[kD];
+    acc[j] = num;
+    __syncthreads();
+    float o = 0.f;
+    for (int i = 0; i < kD; ++i) o = fmaf(a.pi[(size_t)i * kD + j], acc[i], o);
+    num = o;
   }
   a.out[qrow_offset(a, bh / a.h_q, bh % a.h_q) + j] = den > 0.f ? num / den : 0.f;
 }
@@ -282,6 +301,19 @@ __global__ void __launch_bounds__(128) window_kernel(DecodeArgs a) {
       den[g] += ps[g][i];
     }
   }
+  if (a.value_mode == TQ_VALUES_MSE) {
+    // the compressed splits accumulate in the rotated space: rotate this
+    // partial too, (Pi num)_t
+#pragma unroll
+    for (int g = 0; g < G; ++g) qs[g][t] = num[g];
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float o = 0.f;
+      for (int j = 0; j < kD; ++j) o = fmaf(a.pi[(size_t)t * kD + j], qs[g][j], o);
+      num[g] = o;
+    }
+  }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     float *dst = a.part + (((size_t)b * a.h_q + (size_t)h * G + g) * a.part_stride + a.nsplit) * (kD + 2);
@@ -312,12 +344,15 @@ cudaError_t launch_window(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms,
-                            int key_bits, int value_bits) {
+                            int key_bits, int value_bits, int value_mode) {
   DecodePlan P;
   const int ntile = (max_len + kTile - 1) / kTile;
   const long long units = (long long)batch * h_kv;
   // about two CTAs per SM: fewer, longer CTAs amortise each CTA's pipeline fill
-  const long long target = 2LL * num_sms;
+#ifndef TQ_DECODE_CTAS_PER_SM
+#define TQ_DECODE_CTAS_PER_SM 2
+#endif
+  const long long target = (long long)TQ_DECODE_CTAS_PER_SM * num_sms;
   long long ns = (target + units - 1) / units;
   ns = std::max(1LL, std::min(ns, (long long)std::max(ntile, 1)));
   int tps = ntile > 0 ? (int)((ntile + ns - 1) / ns) : 0;
@@ -329,7 +364,8 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   P.qrot_bytes = al((size_t)batch * h_q * 2 * kD * sizeof(float));
   P.part_bytes = al((size_t)batch * h_q * (nsplit + 1) * (kD + 2) * sizeof(float));
   const int G = h_q / h_kv;
-  P.qblock_bytes = decode_tc_supported(key_bits, value_bits, G) ? decode_tc_qblock_bytes(key_bits, G) : 0;
+  P.qblock_bytes =
+      decode_tc_supported(key_bits, value_bits, G, value_mode) ? decode_tc_qblock_bytes(key_bits, G) : 0;
   P.total_bytes = P.status_bytes + P.qrot_bytes + P.part_bytes + al((size_t)batch * h_kv * P.qblock_bytes);
   return P;
 }
@@ -343,7 +379,7 @@ void bind_workspace(DecodeArgs &a, const DecodePlan &P, void *workspace) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
-  if (!decode_tc_supported(a.key_bits, a.value_bits, a.h_q / a.h_kv))
+  if (!decode_tc_supported(a.key_bits, a.value_bits, a.h_q / a.h_kv, a.value_mode))
     return launch_decode_simt(a, stream);
   const int bhq = a.batch * a.h_q;
   // the query-block kernel (first in launch_decode_tc) clears the status word

@@ -66,12 +66,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 608;
+// Worker groups of 4 warps; group g takes tiles g, g + kWorkGroups, ...
+#ifndef TQ_DECODE_WORKER_GROUPS
+#define TQ_DECODE_WORKER_GROUPS 4
+#endif
+constexpr int kWorkGroups = TQ_DECODE_WORKER_GROUPS;
+constexpr int kPvWarp = 2 + 4 * kWorkGroups;      // the P.V MMA issuer, after the worker warps
+constexpr int kTcThreads = 32 * (3 + 4 * kWorkGroups);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTmemCols = 512;
 constexpr int kPlaneCols = 32;  // one u8 operand plane: 128 coordinates per row = 32 TMEM columns
-constexpr int kWorkGroups = 4;  // worker groups of 4 warps; group g takes tiles g, g + 4, ...
-constexpr int kPvWarp = 18;     // the P.V MMA issuer (warps 2 .. 17 are the worker groups)
 
 // 2^n for n in [-126, 127]
 __device__ __forceinline__ float exp2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
@@ -336,7 +340,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       mbar_arrive_expect_tx(&S.q_full, C::QBLOCK);
       bulk_g2s(S.bq, a.qblocks + ((size_t)b * a.h_kv + h) * C::QBLOCK, C::QBLOCK, &S.q_full);
       int issued = 0;
-      for (int i = 0; i < ntile; ++i) {
+      // (a test of the timeout path withholds every tile copy: the workers'
+      // bounded waits on them then run out)
+      for (int i = 0; i < (a.test_withhold ? 0 : ntile); ++i) {
         const int s = i % C::STAGES;
         if (i >= C::STAGES &&
             !wait_bar(&S.empty[s], ((i / C::STAGES) - 1) & 1, &S.abort_flag, a))
@@ -1064,7 +1070,8 @@ bool decode_tc_needs_fallback(int key_bits, int value_bits, int G) {
   return false;
 }
 
-bool decode_tc_supported(int key_bits, int value_bits, int G) {
+bool decode_tc_supported(int key_bits, int value_bits, int G, int value_mode) {
+  if (value_mode != TQ_VALUES_GROUP) return false;  // MSE values: the SIMT split-K kernel
   const int mb = key_bits - 1;
   if (value_bits == 2 && (G == 1 || G == 2 || G == 4 || G == 8) && (mb == 1 || mb == 2)) return true;
   if (value_bits == 2 && mb == 3 && G == 4) return true;

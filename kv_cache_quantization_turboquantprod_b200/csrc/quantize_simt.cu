@@ -5,14 +5,17 @@
 // "turboquant/audit_claims.py", AUDIT 1 / AUDIT 5): u = k/||k||, y = Pi u,
 // idx = #{boundaries < y}, r = u - Pi^T c, signs = [S r >= 0], ||r||.
 // Values (AUDIT 1, value_bits / value_group_size): per 32-channel group
-// min/max, fp16 zero = min, fp16 scale = (max-min)/(2^vb - 1) computed in
-// fp32, code = clamp(rint((v - zero)/scale)).
+// min/max, fp16 zero = min, fp16 scale = (max-min)/(2^vb - 1) rounded once
+// from the exact quotient, code = clamp(rint((v - zero)/scale)) of the exact
+// quotient (float64 where single precision could round it the other way).
 //
 // A persistent CTA keeps Pi and S in shared memory (rows padded to 129
 // floats so both row- and column-direction walks are bank-conflict free) and
 // encodes 16 vectors per pass: three 128x128 mat-vecs per vector (Pi u,
 // Pi^T c, S r) in fp32 with exact fp32 accumulation order per output.  A
 // sketch component within 1e-5 of zero has its sign decided again in float64.
+// TurboQuant-MSE values ("03. Results & Benchmarks", "At a Glance ->
+// Compression"): the value's norm and the Lloyd-Max cells of Pi v / ||v||.
 #include "tq_common.cuh"
 #include "tq_kernels.h"
 
@@ -38,6 +41,11 @@ struct QuantSmem {
   float cent[16];
   float bnd[16];
   uint32_t nearw[kNV][4];  // sketch components to re-decide in float64
+  // TurboQuant-MSE values: unit value vectors, norms, the values' codebook
+  float w[kNV][kD];
+  float nv[kNV];
+  float vcent[16];
+  float vbnd[16];
 };
 
 __device__ __forceinline__ void vec_coords(const AppendArgs &a, long long id, int &b,
@@ -61,13 +69,16 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode);
   const int ncent = 1 << L.mb;
+  const int nvcent = 1 << L.vb;
 
   stage_matrix(S.pi, kPad, a.pi, tid, kThreads);
   stage_matrix(S.s, kPad, a.s, tid, kThreads);
   if (tid < ncent) S.cent[tid] = a.centroids[tid];
   if (tid < ncent - 1) S.bnd[tid] = a.boundaries[tid];
+  if (L.mse && tid < nvcent) S.vcent[tid] = a.v_centroids[tid];
+  if (L.mse && tid < nvcent - 1) S.vbnd[tid] = a.v_boundaries[tid];
   __syncthreads();
 
   const long long total = (long long)a.batch * a.T * a.h_kv;
@@ -97,7 +108,20 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
       for (int m = 0; m < 4; ++m) S.u[vi][lane + 32 * m] = nk > 0.f ? __fdiv_rn(x[m], nk) : 0.f;
       if (lane == 0) S.nk[vi] = nk;
 
-      if (valid) {
+      if (L.mse) {
+        // TurboQuant-MSE values: the unit vector (rotated and bucketized in
+        // phase 1) and its norm
+        float y[4], sv = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          y[m] = valid ? load_elem(a.v, a.dtype, base + lane + 32 * m) : 0.f;
+          sv = fmaf(y[m], y[m], sv);
+        }
+        const float nv = sqrtf(warp_sum(sv));
+#pragma unroll
+        for (int m = 0; m < 4; ++m) S.w[vi][lane + 32 * m] = nv > 0.f ? __fdiv_rn(y[m], nv) : 0.f;
+        if (lane == 0) S.nv[vi] = nv;
+      } else if (valid) {
         const int pos = a.lens[b] + t;
         uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
         const int slot = pos % kTile;
@@ -107,13 +131,17 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
           const float mn = warp_min(vv);
           const float mx = warp_max(vv);
           const __half zero16 = __float2half_rn(mn);
-          const float s32 = __fdiv_rn(__fsub_rn(mx, mn), vlevels);
-          const __half scale16 = __float2half_rn(s32);
+          // the scale from the exact quotient (float64, one rounding to fp16)
+          const __half scale16 = __double2half(((double)mx - (double)mn) / (double)vlevels);
           const float z32 = __half2float(zero16);
           const float sc32 = __half2float(scale16);
           int code = 0;
           if (sc32 != 0.f) {
-            float tq = rintf(__fdiv_rn(__fsub_rn(vv, z32), sc32));
+            // rint of the exact quotient: single precision decides unless the
+            // quotient is next to a half-integer, then float64 does
+            const float t32 = __fdiv_rn(__fsub_rn(vv, z32), sc32);
+            float tq = rintf(t32);
+            if (fabsf(t32 - tq) > 0.5f - 1e-5f) tq = (float)rint(((double)vv - (double)z32) / (double)sc32);
             tq = fminf(fmaxf(tq, 0.f), vlevels);
             code = (int)tq;
           }
@@ -183,6 +211,48 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
               *reinterpret_cast<uint32_t *>(tile + L.kplanes + p * kPlaneBytes +
                                             slot * kRowBytes + 4 * (i >> 5)) = word;
           }
+        }
+      }
+    }
+    // ---- phase 1b (MSE values): y = Pi w, value cells, value norm ---------
+    if (L.mse) {
+      const int i = tid & (kD - 1);
+      const int v0 = (tid >> 7) * (kNV / 2);
+      float acc[kNV / 2];
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) acc[v] = 0.f;
+      for (int j = 0; j < kD; j += 4) {
+        const float w0 = S.pi[i * kPad + j], w1 = S.pi[i * kPad + j + 1];
+        const float w2 = S.pi[i * kPad + j + 2], w3 = S.pi[i * kPad + j + 3];
+#pragma unroll
+        for (int v = 0; v < kNV / 2; ++v) {
+          const float4 ww = *reinterpret_cast<const float4 *>(&S.w[v0 + v][j]);
+          acc[v] = fmaf(w0, ww.x, acc[v]);
+          acc[v] = fmaf(w1, ww.y, acc[v]);
+          acc[v] = fmaf(w2, ww.z, acc[v]);
+          acc[v] = fmaf(w3, ww.w, acc[v]);
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < kNV / 2; ++v) {
+        const int vi = v0 + v;
+        int b, t, h;
+        bool valid;
+        vec_coords(a, id0 + vi, b, t, h, valid);
+        int idx = 0;
+        for (int q = 0; q < nvcent - 1; ++q) idx += (S.vbnd[q] < acc[v]) ? 1 : 0;
+        if (!(S.nv[vi] > 0.f)) idx = 0;
+        if (valid) {
+          const int pos = a.lens[b] + t;
+          uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
+          const int slot = pos % kTile;
+          for (int p = 0; p < L.vb; ++p) {
+            const unsigned word = __ballot_sync(0xffffffffu, (idx >> p) & 1);
+            if (lane == 0)
+              *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * kPlaneBytes + slot * kRowBytes +
+                                            4 * (i >> 5)) = word;
+          }
+          if (i == 0) *reinterpret_cast<__half *>(tile + L.vsz + slot * 2) = __float2half_rn(S.nv[vi]);
         }
       }
     }

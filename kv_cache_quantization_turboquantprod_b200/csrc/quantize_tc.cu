@@ -6,8 +6,9 @@
 //   GEMM1  Y = K Pi^T            y = Y / ||k||, bucketize -> codes, c = c[idx]
 //   GEMM2  P = C Pi              r = u - P (= u - Pi^T c), ||r||
 //   GEMM3  Z = R S^T             signs = [z >= 0]
-// Values are group-quantized (per 32 channels, fp16 scale/zero) by the
-// loader warps on the way in.
+// Values are group-quantized (per 32 channels, fp16 scale/zero) by a
+// separate bandwidth-bound kernel launched just before this one
+// (quantize_values.cu).
 //
 // Precision.  A bf16 key is exact in fp16 once scaled per vector by 2^s
 // (largest |k| 2^s in [2^14, 2^15)); Pi, S, the centroids and the residual
@@ -22,7 +23,7 @@
 //   warps 0, 13   MMA issuers of epilogue groups 0 and 1 (one elected lane),
 //                 each sleeping in blocking waits on its group's barriers
 //   warps 1-4     loader: K rows -> scaled fp16 A operand + norms in shared
-//                 memory; V rows -> codes, scales, zeros straight to the cache
+//                 memory
 //   warps 5-8     epilogue group 0 (even tiles)   | thread = tile row = TMEM
 //   warps 9-12    epilogue group 1 (odd tiles)    | lane; 256 TMEM columns each
 // Every mbarrier wait between roles is bounded (2 s unless the host set another
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   QtSmem &S = *reinterpret_cast<QtSmem *>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits);
+  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode);
   constexpr int ncent = 1 << MB;
   const int nlocal = a.total_tiles > (int)blockIdx.x
                          ? (a.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
@@ -261,13 +262,12 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     // ---------------- loader -----------------------------------------------
     // A warp takes 8 rows at a time (one 8-row group of the operand): lane
     // (row rr = lane / 4, channel quarter q = lane % 4) holds channels
-    // 32q .. 32q + 31 -- one value group.  Both rows are fetched before
-    // either is used.
+    // 32q .. 32q + 31.  Values are quantized by their own kernel, so the
+    // loader reads keys only; the rows of the next two steps are in flight
+    // while this step's are converted.
     const int w = warp - 1, rr = lane >> 2, q = lane & 3;
-    const float vlevels = (float)((1 << a.value_bits) - 1);
-    // rows of step u = 4 i + pass; the next step's rows are fetched while
-    // this step's are converted
-    auto fetch = [&](int u, uint4 (&kr)[4], uint4 (&vr)[4]) {
+    // rows of step u = 4 i + pass
+    auto fetch = [&](int u, uint4 (&kr)[4]) {
       const int i = u >> 2, pass = u & 3;
       bool valid = i < nlocal;
       size_t base = 0;
@@ -278,15 +278,12 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         base = ((((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD + 32 * q);
       }
       const uint4 *ks = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + base);
-      const uint4 *vs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v) + base);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        kr[c] = valid ? ks[c] : make_uint4(0u, 0u, 0u, 0u);
-        vr[c] = valid ? vs[c] : make_uint4(0u, 0u, 0u, 0u);
-      }
+      for (int c = 0; c < 4; ++c) kr[c] = valid ? ks[c] : make_uint4(0u, 0u, 0u, 0u);
     };
-    uint4 kr[4], vr[4];
-    fetch(0, kr, vr);
+    uint4 kr[4], k1[4];
+    fetch(0, kr);
+    fetch(1, k1);
     for (int i = 0; i < nlocal; ++i) {
       const int g = i & 1;
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
@@ -294,15 +291,13 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       bool stop = false;
 #pragma unroll 1
       for (int pass = 0; pass < 4; ++pass) {
-        uint4 kn[4], vn[4];
-        fetch(4 * i + pass + 1, kn, vn);
+        uint4 k2[4];
+        fetch(4 * i + pass + 2, k2);
         if (pass == 0 && i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag, a)) {
           stop = true;
           break;
         }
         const int r = 32 * pass + 8 * w + rr;
-        const bool valid = r < ti.nrow;
-        const int t = ti.t0 + r;
         // ---- key: norm, per-vector scale, fp16 operand ----
         float ss = 0.f, mx = 0.f;
 #pragma unroll
@@ -338,87 +333,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           S.nk[g][r] = nk;
           S.sh[g][r] = sh;
         }
-        // ---- values: this lane's 32 channels are one group ----
-        if (valid) {
-          float mn = INFINITY, mxv = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&vr[c]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(p2[e]);
-              mn = fminf(mn, fminf(f.x, f.y));
-              mxv = fmaxf(mxv, fmaxf(f.x, f.y));
-            }
-          }
-          const __half zero16 = __float2half_rn(mn);
-          const __half scale16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxv, mn), vlevels));
-          const float z32 = __half2float(zero16), sc32 = __half2float(scale16);
-          const float rsc = sc32 != 0.f ? 1.f / sc32 : 0.f;
-          const int pos = a.lens[ti.b] + t;
-          uint8_t *tp = tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile);
-          const int slot = pos % kTile;
-          // code = clamp(rint((v - zero) / scale)) with an exactly rounded
-          // quotient.  The reciprocal product is within 2 ulp of it, so it
-          // decides the code unless it sits next to a half-integer; those
-          // (rare) elements are redone with the exact division afterwards.
-          uint32_t codes[4] = {0u, 0u, 0u, 0u};  // 4 bits per element, 8 per word
-          uint32_t fix = 0u;
-          if (sc32 != 0.f) {
-            const int ilev = (int)vlevels;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t *w2v = reinterpret_cast<const uint32_t *>(&vr[c]);
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2) {
-                const uint32_t wb = w2v[e2 >> 1];  // two bf16
-                const float x = __uint_as_float((e2 & 1) ? (wb & 0xFFFF0000u) : (wb << 16));
-                // t stays within [-1, levels + 1] (fp16 zero/scale rounding);
-                // rint by the 1.5 * 2^23 magic add, integer clamp
-                const float tq = fminf(fmaxf(__fsub_rn(x, z32) * rsc, -1.f), vlevels + 1.f);
-                const float r = tq + 12582912.f;
-                const float rq = r - 12582912.f;
-                fix |= (fabsf(tq - rq) > 0.5f - 1e-5f ? 1u : 0u) << (8 * c + e2);
-                const int code = min(max(__float_as_int(r) - 0x4B400000, 0), ilev);
-                codes[c] |= (uint32_t)code << (4 * e2);
-              }
-            }
-            const __nv_bfloat16 *vrow = reinterpret_cast<const __nv_bfloat16 *>(a.v) +
-                                        ((((size_t)ti.b * a.T + t) * a.h_kv + ti.h) * kD + 32 * q);
-            while (fix) {
-              const int e = __ffs(fix) - 1;
-              fix &= fix - 1;
-              const float tq = __fdiv_rn(__fsub_rn(__bfloat162float(vrow[e]), z32), sc32);
-              const uint32_t code = (uint32_t)fminf(fmaxf(rintf(tq), 0.f), vlevels);
-              codes[e >> 3] = (codes[e >> 3] & ~(15u << (4 * (e & 7)))) | (code << (4 * (e & 7)));
-            }
-          }
-          if (L.vb == 2) {
-            // channel 4i + m of the group in bits 2m, 2m+1 of byte i
-            uint32_t w2[2] = {0u, 0u};
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w2[e >> 4] |= ((codes[e >> 3] >> (4 * (e & 7))) & 3u) << (2 * (e & 15));
-            *reinterpret_cast<uint2 *>(tp + L.vplanes + slot * kPackedRowBytes + 8 * q) = make_uint2(w2[0], w2[1]);
-          } else {
-            for (int p = 0; p < L.vb; ++p) {
-              uint32_t wp = 0u;
-#pragma unroll
-              for (int e = 0; e < 32; ++e) wp |= ((codes[e >> 3] >> (4 * (e & 7) + p)) & 1u) << e;
-              *reinterpret_cast<uint32_t *>(tp + L.vplanes + p * kPlaneBytes + slot * kRowBytes + 4 * q) = wp;
-            }
-          }
-          *reinterpret_cast<__half2 *>(tp + L.vsz + (slot * kGroups + q) * 4) = __halves2half2(scale16, zero16);
-        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          kr[c] = kn[c];
-          vr[c] = vn[c];
+          kr[c] = k1[c];
+          k1[c] = k2[c];
         }
       }
       if (stop) break;
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a1_full[g]);
+      // (a test of the timeout path withholds the hand-off: the MMA issuer's
+      // bounded wait on it then runs out)
+      if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full[g]);
     }
   } else {
     // ---------------- epilogue groups --------------------------------------
@@ -634,7 +560,7 @@ cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
 }  // namespace
 
 bool quantize_tc_supported(const AppendArgs &a) {
-  return a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 && a.value_bits >= 2 &&
+  return a.value_mode == TQ_VALUES_GROUP && a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 && a.value_bits >= 2 &&
          a.value_bits <= 4 && a.T >= 64;
 }
 
@@ -648,6 +574,8 @@ cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream) 
   a.total_tiles = total;
   if (total == 0) return cudaSuccess;
   const int grid = total < num_sms ? total : num_sms;
+  const cudaError_t ev = launch_value_quant(a, num_sms, stream);
+  if (ev != cudaSuccess) return ev;
   switch (a.key_bits - 1) {
     case 1: return launch_qt<1>(a, grid, stream);
     case 2: return launch_qt<2>(a, grid, stream);

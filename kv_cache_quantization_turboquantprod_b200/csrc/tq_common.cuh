@@ -27,19 +27,21 @@ struct TileLayout {
   int signs;       // offset of the sign plane
   int vplanes;     // offset of value planes
   int norms;       // offset of {||k||, ||r||} fp16 pairs
-  int vsz;         // offset of {scale, zero} fp16 pairs
+  int vsz;         // offset of {scale, zero} fp16 pairs (MSE values: fp16 norms)
   int tile_bytes;  // bytes of one tile
+  bool mse;        // TurboQuant-MSE values: value cells as bit-planes + one fp16 norm
 
-  __host__ __device__ static TileLayout make(int key_bits, int value_bits) {
+  __host__ __device__ static TileLayout make(int key_bits, int value_bits, int value_mode = 0) {
     TileLayout L;
     L.mb = key_bits - 1;
     L.vb = value_bits;
+    L.mse = value_mode == TQ_VALUES_MSE;
     L.kplanes = 0;
     L.signs = L.mb * kPlaneBytes;
     L.vplanes = L.signs + kPlaneBytes;
     L.norms = L.vplanes + L.vb * kPlaneBytes;
     L.vsz = L.norms + kTile * 4;
-    L.tile_bytes = L.vsz + kTile * 4 * kGroups;
+    L.tile_bytes = L.vsz + (L.mse ? kTile * 2 : kTile * 4 * kGroups);
     return L;
   }
   __host__ __device__ int record_bytes() const { return tile_bytes / kTile; }
@@ -54,9 +56,10 @@ __device__ __forceinline__ uint8_t *tile_ptr(void *data, const TileLayout &L,
 }
 
 // Value code of channel j of token slot `slot`: packed 2-bit codes (channel
-// 4i + m in bits 2m, 2m+1 of byte i) for 2-bit values, bit-planes otherwise.
+// 4i + m in bits 2m, 2m+1 of byte i) for 2-bit group-quantized values,
+// bit-planes otherwise (MSE values: the cell of rotated coordinate j).
 __device__ __forceinline__ int value_code(const uint8_t *tile, const TileLayout &L, int slot, int j) {
-  if (L.vb == 2) return (tile[L.vplanes + slot * kPackedRowBytes + (j >> 2)] >> (2 * (j & 3))) & 3;
+  if (L.vb == 2 && !L.mse) return (tile[L.vplanes + slot * kPackedRowBytes + (j >> 2)] >> (2 * (j & 3))) & 3;
   int code = 0;
   for (int p = 0; p < L.vb; ++p)
     code |= ((tile[L.vplanes + p * kPlaneBytes + slot * kRowBytes + (j >> 3)] >> (j & 7)) & 1) << p;

@@ -43,6 +43,8 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Bound of the kernels' pipeline waits (tq_set_wait_limit_ns).
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+// Tests of the timeout path (tq_test_withhold_handoffs).
+std::atomic<int> g_withhold{0};
 
 // Sticky per-device error word (TQ_ERRF_* bits) that kernels set when they
 // give up on a bounded wait; its device address is looked up once per device.
@@ -77,6 +79,7 @@ cudaError_t set_wait_fields(Args &a) {
   const unsigned long long ns = g_wait_ns.load(std::memory_order_relaxed);
   a.wait_ns = ns;
   a.wait_hint_ns = (unsigned int)(ns < 1000000ull ? ns : 1000000ull);
+  a.test_withhold = g_withhold.load(std::memory_order_relaxed);
   return error_word_address(&a.errors);
 }
 
@@ -87,6 +90,8 @@ tq_status check_params(const tq_params *p) {
   if (p->value_bits < 2 || p->value_bits > 4) return TQ_ERR_UNSUPPORTED;
   if (!p->pi || !p->s || !p->centroids || !p->boundaries) return TQ_ERR_INVALID_ARGUMENT;
   if (!aligned(p->pi, 16) || !aligned(p->s, 16)) return TQ_ERR_INVALID_ARGUMENT;
+  if (p->value_mode != TQ_VALUES_GROUP && p->value_mode != TQ_VALUES_MSE) return TQ_ERR_UNSUPPORTED;
+  if (p->value_mode == TQ_VALUES_MSE && (!p->v_centroids || !p->v_boundaries)) return TQ_ERR_INVALID_ARGUMENT;
   return TQ_OK;
 }
 
@@ -157,13 +162,13 @@ tq_status tq_make_codebook(int mse_bits, int d, double *centroids, double *bound
 
 size_t tq_record_bytes(const tq_params *p) {
   if (check_params(p) != TQ_OK) return 0;
-  return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits).record_bytes();
+  return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode).record_bytes();
 }
 
 size_t tq_cache_bytes(const tq_params *p, int batch, int h_kv, int capacity) {
   if (check_params(p) != TQ_OK) return 0;
   if (batch < 1 || h_kv < 1 || capacity < kTile || capacity % kTile) return 0;
-  const tq::TileLayout L = tq::TileLayout::make(p->key_bits, p->value_bits);
+  const tq::TileLayout L = tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode);
   return (size_t)batch * h_kv * (size_t)(capacity / kTile) * (size_t)L.tile_bytes;
 }
 
@@ -189,6 +194,7 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
     a.nnew[b] = nn;
   }
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids; a.boundaries = p->boundaries;
+  a.value_mode = p->value_mode; a.v_centroids = p->v_centroids; a.v_boundaries = p->v_boundaries;
   a.data = c->data; a.k = k; a.v = v;
   a.batch = c->batch; a.h_kv = c->h_kv; a.ntiles = c->capacity / kTile; a.T = T;
   a.key_bits = p->key_bits; a.value_bits = p->value_bits; a.dtype = dtype;
@@ -206,7 +212,8 @@ size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, 
   if (h_q < c->h_kv || h_q % c->h_kv || max_len < 0 || max_len > c->capacity) return 0;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return 0;
-  return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits).total_bytes;
+  return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits,
+                              p->value_mode).total_bytes;
 }
 
 namespace {
@@ -219,7 +226,7 @@ namespace {
 int prefill_tokens_per_pass(const tq_params *p, int gqa, int t_chunk) {
   int ts = 1;
   while (2 * ts <= t_chunk && gqa * 2 * ts <= 4 &&
-         tq::decode_tc_supported(p->key_bits, p->value_bits, gqa * 2 * ts))
+         tq::decode_tc_supported(p->key_bits, p->value_bits, gqa * 2 * ts, p->value_mode))
     ts *= 2;
   return ts;
 }
@@ -239,7 +246,8 @@ size_t tq_prefill_workspace_size(const tq_params *p, const tq_cache *c, int h_q,
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return 0;
   const int ts = prefill_tokens_per_pass(p, h_q / c->h_kv, t_chunk);
-  return tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits, p->value_bits)
+  return tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits, p->value_bits,
+                              p->value_mode)
       .total_bytes;
 }
 
@@ -263,7 +271,7 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
   const int G = h_q / c->h_kv;
   const int ts = prefill_tokens_per_pass(p, G, t_chunk);
   if (workspace_bytes < tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits,
-                                             p->value_bits).total_bytes)
+                                             p->value_bits, p->value_mode).total_bytes)
     return TQ_ERR_WORKSPACE;
   // passes of ts tokens (the last one of the largest power of two that is
   // left); pass tokens t0 .. t0 + n - 1 see len - (t_chunk - 1 - t) tokens
@@ -272,9 +280,11 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
     while (n > t_chunk - t0) n >>= 1;
     const int len_sub = t_chunk - t0 - n;
     const int ml = max_len - len_sub;
-    const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q * n, ml, sms, p->key_bits, p->value_bits);
+    const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q * n, ml, sms, p->key_bits, p->value_bits,
+                                                  p->value_mode);
     tq::DecodeArgs a;
     a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
+    a.value_mode = p->value_mode; a.v_centroids = p->v_centroids;
     a.data = c->data; a.q = q; a.q_dtype = q_dtype; a.len = len_dev;
     a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q * n; a.ntiles = c->capacity / kTile;
     a.max_len = ml; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
@@ -324,10 +334,12 @@ tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq
   if (!workspace || !aligned(workspace, 256)) return TQ_ERR_WORKSPACE;
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
-  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits);
+  const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits,
+                                                p->value_mode);
   if (workspace_bytes < P.total_bytes) return TQ_ERR_WORKSPACE;
   tq::DecodeArgs a;
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
+  a.value_mode = p->value_mode; a.v_centroids = p->v_centroids;
   a.data = c->data; a.q = q; a.q_dtype = q_dtype; a.len = len_dev;
   a.batch = c->batch; a.h_kv = c->h_kv; a.h_q = h_q; a.ntiles = c->capacity / kTile;
   a.max_len = max_len; a.key_bits = p->key_bits; a.value_bits = p->value_bits;
@@ -374,6 +386,11 @@ tq_status tq_set_wait_limit_ns(unsigned long long ns) {
   return TQ_OK;
 }
 
+tq_status tq_test_withhold_handoffs(int on) {
+  g_withhold.store(on ? 1 : 0, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
 tq_status tq_device_errors(uint32_t *flags, int clear) {
   if (!flags) return TQ_ERR_INVALID_ARGUMENT;
   unsigned int *p = nullptr;
@@ -398,6 +415,7 @@ tq_status tq_dequantize(const tq_params *p, const tq_cache *c, int b, int start,
   if (!k_out || !v_out || !aligned(k_out, 4) || !aligned(v_out, 4)) return TQ_ERR_INVALID_ARGUMENT;
   tq::DequantArgs a;
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids; a.data = c->data;
+  a.value_mode = p->value_mode; a.v_centroids = p->v_centroids;
   a.h_kv = c->h_kv; a.ntiles = c->capacity / kTile; a.b = b; a.start = start; a.count = count;
   a.key_bits = p->key_bits; a.value_bits = p->value_bits; a.k_out = k_out; a.v_out = v_out;
   if (tq::launch_dequantize(a, (cudaStream_t)stream) != cudaSuccess) return TQ_ERR_CUDA;

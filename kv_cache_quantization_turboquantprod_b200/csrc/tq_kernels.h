@@ -16,6 +16,8 @@ namespace tq {
 // offsets; CUDA 12.1+ allows kernel parameters up to 32764 bytes).
 struct AppendArgs {
   const float *pi, *s, *centroids, *boundaries;
+  int value_mode;                        // tq_value_mode
+  const float *v_centroids, *v_boundaries;  // MSE values' codebook
   void *data;
   const void *k, *v;
   int batch, h_kv, ntiles, T;
@@ -32,6 +34,8 @@ struct AppendArgs {
   unsigned long long wait_ns;
   unsigned int wait_hint_ns;
   unsigned int *errors;
+  // tests of the timeout path: the loader withholds its operand hand-offs
+  int test_withhold;
 };
 
 // Split-K plan of one decode call (host-computed, identical in the
@@ -49,6 +53,8 @@ struct DecodePlan {
 
 struct DecodeArgs {
   const float *pi, *s, *centroids;
+  int value_mode;              // tq_value_mode (MSE: partials in the rotated space)
+  const float *v_centroids;    // MSE values' codebook
   const void *data;
   const void *q;
   tq_dtype q_dtype;
@@ -84,6 +90,8 @@ struct DecodeArgs {
   unsigned long long wait_ns;
   unsigned int wait_hint_ns;
   unsigned int *errors;
+  // tests of the timeout path: the producer withholds the tile copies
+  int test_withhold;
   // SIMT split-K launched behind the tensor-core kernel: runs only when
   // status[1] says the codebook needs it
   int fallback_gate;
@@ -102,6 +110,8 @@ __host__ __device__ inline size_t qrow_offset(const DecodeArgs &a, int b, int hv
 
 struct DequantArgs {
   const float *pi, *s, *centroids;
+  int value_mode;
+  const float *v_centroids;
   const void *data;
   int h_kv, ntiles, b, start, count;
   int key_bits, value_bits;
@@ -109,15 +119,18 @@ struct DequantArgs {
 };
 
 DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms,
-                            int key_bits, int value_bits);
+                            int key_bits, int value_bits, int value_mode = 0);
 
 cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream);
 // Tensor-core quantize-append (bf16 K/V, appends of 64+ tokens).
 bool quantize_tc_supported(const AppendArgs &a);
 cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream);
+// Group quantization of values alone (bandwidth-bound), run by the
+// tensor-core append path before its key kernel.
+cudaError_t launch_value_quant(const AppendArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 // Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
-bool decode_tc_supported(int key_bits, int value_bits, int gqa);
+bool decode_tc_supported(int key_bits, int value_bits, int gqa, int value_mode = 0);
 // True when a codebook whose Walsh expansion has every subset plane (an
 // asymmetric codebook) leaves room for only one plane buffer of the
 // tensor-core kernel in tensor memory; such codebooks run the SIMT split-K

@@ -22,6 +22,7 @@ STATUS = {0: "TQ_OK", 1: "TQ_ERR_INVALID_ARGUMENT", 2: "TQ_ERR_UNSUPPORTED",
           3: "TQ_ERR_CAPACITY", 4: "TQ_ERR_WORKSPACE", 5: "TQ_ERR_CUDA",
           6: "TQ_ERR_INTERNAL"}
 TQ_F32, TQ_BF16 = 0, 1
+TQ_VALUES_GROUP, TQ_VALUES_MSE = 0, 1
 TILE_TOKENS = 128
 MAX_BATCH = 1024
 
@@ -30,7 +31,7 @@ EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_
            "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
            "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window",
            "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass",
-           "tq_set_wait_limit_ns", "tq_device_errors")
+           "tq_set_wait_limit_ns", "tq_device_errors", "tq_test_withhold_handoffs")
 ERRF_DECODE_WAIT, ERRF_QUANTIZE_WAIT = 1, 2
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -45,7 +46,9 @@ class Params(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("key_bits", ctypes.c_int),
                 ("value_bits", ctypes.c_int), ("group", ctypes.c_int),
                 ("pi", ctypes.c_void_p), ("s", ctypes.c_void_p),
-                ("centroids", ctypes.c_void_p), ("boundaries", ctypes.c_void_p)]
+                ("centroids", ctypes.c_void_p), ("boundaries", ctypes.c_void_p),
+                ("value_mode", ctypes.c_int), ("v_centroids", ctypes.c_void_p),
+                ("v_boundaries", ctypes.c_void_p)]
 
 
 class Cache(ctypes.Structure):
@@ -98,6 +101,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_dequantize.argtypes = [P, C, ci, ci, ci, vp, vp, vp]
     lib.tq_set_wait_limit_ns.restype = ci
     lib.tq_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.tq_test_withhold_handoffs.restype = ci
+    lib.tq_test_withhold_handoffs.argtypes = [ci]
     lib.tq_device_errors.restype = ci
     lib.tq_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ci]
     if path is None:
@@ -174,11 +179,13 @@ def tq_make_codebook(mse_bits: int, d: int):
 
 
 class Layer:
-    """Device-resident constants of one layer (Pi, S, codebook) packaged as
-    the C struct tq_params.  Holds references to the tensors it points to."""
+    """Device-resident constants of one layer (Pi, S, codebooks) packaged as
+    the C struct tq_params.  Holds references to the tensors it points to.
+    value_mode "group" (min/max groups of 32) or "mse" (TurboQuant-MSE values
+    with the value_bits Lloyd-Max codebook)."""
 
     def __init__(self, pi, s, key_bits: int, value_bits: int, group: int = 32,
-                 device="cuda"):
+                 device="cuda", value_mode: str = "group"):
         d = int(pi.shape[0])
         cent, bnd = tq_make_codebook(key_bits - 1, d)
         self.pi = torch.as_tensor(pi, dtype=torch.float32).contiguous().to(device)
@@ -186,9 +193,18 @@ class Layer:
         self.centroids = torch.tensor(cent, dtype=torch.float32, device=device)
         self.boundaries = torch.tensor(bnd if bnd else [0.0], dtype=torch.float32, device=device)
         self.codebook = (cent, bnd)
+        self.value_mode = value_mode
+        mode = {"group": TQ_VALUES_GROUP, "mse": TQ_VALUES_MSE}[value_mode]
+        vc_ptr = vb_ptr = None
+        if mode == TQ_VALUES_MSE:
+            vcent, vbnd = tq_make_codebook(value_bits, d)
+            self.v_centroids = torch.tensor(vcent, dtype=torch.float32, device=device)
+            self.v_boundaries = torch.tensor(vbnd, dtype=torch.float32, device=device)
+            self.value_codebook = (vcent, vbnd)
+            vc_ptr, vb_ptr = self.v_centroids.data_ptr(), self.v_boundaries.data_ptr()
         self.params = Params(d, key_bits, value_bits, group, self.pi.data_ptr(),
                              self.s.data_ptr(), self.centroids.data_ptr(),
-                             self.boundaries.data_ptr())
+                             self.boundaries.data_ptr(), mode, vc_ptr, vb_ptr)
 
     @property
     def d(self):
@@ -345,6 +361,12 @@ def tq_set_wait_limit_ns(ns: int) -> None:
     """Time limit of the kernels' bounded waits for later calls (0: the
     default, 2 s).  For tests of the timeout path."""
     _check("tq_set_wait_limit_ns", load().tq_set_wait_limit_ns(int(ns)))
+
+
+def tq_test_withhold_handoffs(on: bool) -> None:
+    """Tests of the timeout path: make later calls' tensor-core kernels
+    withhold one hand-off so that their bounded waits run out."""
+    _check("tq_test_withhold_handoffs", load().tq_test_withhold_handoffs(int(bool(on))))
 
 
 def tq_device_errors(clear: bool = False) -> int:

@@ -6,13 +6,10 @@ Parity bar:
 * key codes and sign bits bit-exact except coordinates within 1e-6 of a
   decision boundary (|y - t| < 1e-6, oracle y) or of zero (|S r| < 1e-6);
   the band count is reported and must be <= 1e-4 of all coordinates;
-* value codes, scales and zeros bit-exact except in the value band: a code
-  whose exact quotient t = (v - zero16) / scale16 lies within 1e-6 of a
-  half-integer without being one (an exact half-integer is a tie that both
-  sides resolve half-to-even), and every code and the scale of a group whose
-  scale quotient (mx - mn) / (2^vb - 1) lies within 1e-6 (relative) of an fp16
-  rounding midpoint; the band count is reported and must be <= 1e-4 of all
-  coordinates;
+* value codes bit-exact except in the value band (a code whose exact quotient
+  t = (v - zero16) / scale16 lies within 1e-6 of a half-integer without being
+  one; an exact half-integer is a tie that both sides resolve half-to-even),
+  counted, <= 1e-4 of all coordinates; scales and zeros bit-exact;
 * norms and attention outputs within 1e-3 relative: per row,
   max |gpu - oracle| / max |oracle|.
 """
@@ -31,24 +28,32 @@ REL_TOL = 1e-3
 
 
 class OracleLayer:
-    """The oracle's view of one layer: the same Pi (float32 values), S and a
-    codebook from the oracle's own Lloyd-Max."""
+    """The oracle's view of one layer: the same Pi (float32 values), S and
+    codebooks from the oracle's own Lloyd-Max (keys: key_bits - 1 bits;
+    TurboQuant-MSE values: value_bits bits)."""
 
     def __init__(self, pi32: np.ndarray, s32: np.ndarray, key_bits: int, value_bits: int,
-                 group: int = 32):
+                 group: int = 32, value_mode: str = "group"):
         self.pi = np.asarray(pi32, np.float64)
         self.s = np.asarray(s32, np.float64)
         self.key_bits, self.value_bits, self.group = key_bits, value_bits, group
+        self.value_mode = value_mode
         self.cent, self.bnd, _ = codebook.lloyd_max_gaussian(key_bits - 1, self.pi.shape[0])
+        self.vcent = self.vbnd = None
+        if value_mode == "mse":
+            self.vcent, self.vbnd, _ = codebook.lloyd_max_gaussian(value_bits, self.pi.shape[0])
 
     def encode(self, k: np.ndarray, v: np.ndarray):
         ke = quant.encode_keys(k, self.pi, self.s, self.cent, self.bnd)
-        ve = quant.encode_values(v, self.value_bits, self.group)
+        if self.value_mode == "mse":
+            ve = quant.encode_values_mse(v, self.pi, self.vcent, self.vbnd)
+        else:
+            ve = quant.encode_values(v, self.value_bits, self.group)
         return ke, ve
 
 
-def gpu_layer(pi32, s32, key_bits, value_bits, device="cuda"):
-    return tq.Layer(pi32, s32, key_bits, value_bits, device=device)
+def gpu_layer(pi32, s32, key_bits, value_bits, device="cuda", value_mode="group"):
+    return tq.Layer(pi32, s32, key_bits, value_bits, device=device, value_mode=value_mode)
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -95,12 +100,25 @@ def compare_records(spec: layout.CacheSpec, buf: np.ndarray, b: int, h: int, pos
     bad = (got["sign"] != sign_ref) & ~snear
     assert not bad.any(), f"sign mismatch outside band at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
     stats["alt_cell_vectors"] = stats.get("alt_cell_vectors", 0) + int(alt.size)
-    vnear, gband = value_band(ve)
-    bad = (got["codes"] != ve["codes"]) & ~vnear
-    assert not bad.any(), f"value code mismatch at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
-    bad = (got["scale16"] != ve["scale16"]) & ~gband
-    assert not bad.any(), f"value scale mismatch at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
-    assert np.array_equal(got["zero16"], ve["zero16"]), "value zero mismatch"
+    if "vidx" in ve:
+        # TurboQuant-MSE values: cells exact outside |y - t| < 1e-6 of the
+        # values' boundaries (oracle y), the norm within the norm tolerance
+        vb = codebook.lloyd_max_gaussian(spec.value_bits, spec.d)[1]
+        vnear = np.zeros_like(ve["vy"], dtype=bool)
+        for tb in vb:
+            vnear |= np.abs(ve["vy"] - tb) < BAND
+        vnear[ve["nv"] == 0] = False
+        bad = (got["vidx"] != ve["vidx"]) & ~vnear
+        assert not bad.any(), f"value cell mismatch at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
+        rel = np.abs(got["nv16"] - ve["nv16"]) / np.maximum(np.abs(ve["nv16"]), 1e-30)
+        rel[(ve["nv16"] == 0) & (got["nv16"] == 0)] = 0.0
+        assert rel.max(initial=0.0) <= REL_TOL, f"nv16 rel err {rel.max()}"
+    else:
+        vnear = value_band(ve)
+        bad = (got["codes"] != ve["codes"]) & ~vnear
+        assert not bad.any(), f"value code mismatch at (b={b}, h={h}): {np.argwhere(bad)[:5]}"
+        assert np.array_equal(got["scale16"], ve["scale16"]), "value scale mismatch"
+        assert np.array_equal(got["zero16"], ve["zero16"]), "value zero mismatch"
     for key in ("nk16", "rn16"):
         ref = ke[key] if key == "nk16" else rn16_ref
         rel = np.abs(got[key] - ref) / np.maximum(np.abs(ref), 1e-30)
@@ -111,22 +129,18 @@ def compare_records(spec: layout.CacheSpec, buf: np.ndarray, b: int, h: int, pos
     stats["code_band"] += int(near.sum())
     stats["sign_band"] += int(snear.sum())
     stats["value_band"] += int(vnear.sum())
+    vkey = "vidx" if "vidx" in ve else "codes"
     stats["value_mismatch_in_band"] = stats.get("value_mismatch_in_band", 0) + int(
-        (got["codes"] != ve["codes"]).sum())
+        (got[vkey] != ve[vkey]).sum())
     return stats
 
 
 def value_band(ve: dict):
-    """(per-element value band mask [n, d], per-group scale band mask
-    [n, d/group]) of the oracle's value encoding ``ve``."""
+    """Per-element value band mask [n, d] of the oracle's value encoding
+    ``ve``: quotients within 1e-6 of a half-integer, exact ties excluded."""
     t = ve["t"]
     half = np.floor(t) + 0.5
-    near = (np.abs(t - half) < BAND) & (t != half)
-    q = ve["scale_q"]
-    gband = quant.fp16(q * (1.0 - BAND)) != quant.fp16(q * (1.0 + BAND))
-    group = t.shape[1] // q.shape[1]
-    near |= np.repeat(gband, group, axis=1)
-    return near, gband
+    return (np.abs(t - half) < BAND) & (t != half)
 
 
 def check_band_fraction(stats: dict) -> None:
@@ -156,6 +170,9 @@ def oracle_records_for(layer: OracleLayer, k: np.ndarray, v: np.ndarray):
 
 
 def logical(ke: dict, ve: dict) -> dict:
+    if "vidx" in ve:
+        return {"idx": ke["idx"], "sign": ke["sign"], "nk16": ke["nk16"], "rn16": ke["rn16"],
+                "vidx": ve["vidx"], "nv16": ve["nv16"]}
     return {"idx": ke["idx"], "sign": ke["sign"], "nk16": ke["nk16"], "rn16": ke["rn16"],
             "codes": ve["codes"], "scale16": ve["scale16"], "zero16": ve["zero16"]}
 
@@ -169,7 +186,8 @@ def oracle_decode(layer: OracleLayer, q: np.ndarray, kes: list, ves: list, lengt
         r = logical(ke, ve)
         recs.append({k2: v2[start:start + length] for k2, v2 in r.items()})
     rec = attention.stack_heads(recs)
-    return attention.decode_one_sequence(q, rec, layer.pi, layer.s, layer.cent, layer.group)
+    return attention.decode_one_sequence(q, rec, layer.pi, layer.s, layer.cent, layer.group,
+                                         value_centroids=layer.vcent)
 
 
 def fill_cache_gpu(glayer, cache, wl, lengths, device="cuda") -> None:
@@ -202,4 +220,5 @@ def oracle_decode_head(layer: OracleLayer, spec, buf: np.ndarray, b: int, h: int
     first n records of the library's cache bytes (read with the oracle's own
     layout reader): [G, d]."""
     rec = attention.stack_heads([spec.read(buf, b, h, 0, n)])
-    return attention.decode_one_sequence(q_heads, rec, layer.pi, layer.s, layer.cent, layer.group)
+    return attention.decode_one_sequence(q_heads, rec, layer.pi, layer.s, layer.cent, layer.group,
+                                         value_centroids=layer.vcent)

@@ -1,13 +1,15 @@
 """GPU checks of the failure paths and of the codebook fallback.
 
-* Bounded waits: with the library's wait limit set to one nanosecond, a
-  normal-sized decode call and a normal-sized tensor-core quantize-append give
-  up on their waits.  Each call still returns, the device still answers, the
+* Bounded waits: with the library's wait limit set to 2 ms and one hand-off
+  withheld (the decode producer's tile copies; the quantize loader's key
+  operand), a normal-sized decode call and a normal-sized tensor-core
+  quantize-append give up on the waits that nothing completes.  Each call
+  still returns, the device still answers, the
   failure shows (decode: the workspace status word is nonzero and every
   output row is NaN; quantize-append: the appended records carry NaN norms;
   both: the device's sticky error word), and with the default limit restored
   the very next calls pass parity, so the kernels freed their tensor memory.
-  No fault is injected: the waits simply run out of time.
+  No fault is injected: every wait is bounded and simply runs out of time.
 * Asymmetric codebooks in the shapes where their operand planes fit in tensor
   memory only once run the SIMT split-K kernel (chosen on the device); parity
   at 16 tiles per CTA in every such shape.
@@ -62,10 +64,12 @@ def test_decode_wait_timeout_reports_and_recovers():
     q = workloads.queries(wl, 0, device=DEV)
     tq.tq_device_errors(clear=True)
     try:
-        tq.tq_set_wait_limit_ns(1)
+        tq.tq_set_wait_limit_ns(2_000_000)
+        tq.tq_test_withhold_handoffs(True)
         out, ws = _decode(glayer, cache, q, list(wl.lengths), 8192)
         torch.cuda.synchronize()
     finally:
+        tq.tq_test_withhold_handoffs(False)
         tq.tq_set_wait_limit_ns(0)
     assert tq.decode_status(ws) != 0
     assert torch.isnan(out).all()
@@ -94,10 +98,12 @@ def test_quantize_wait_timeout_reports_and_recovers():
     v = torch.stack([x[1] for x in kv]).contiguous()
     tq.tq_device_errors(clear=True)
     try:
-        tq.tq_set_wait_limit_ns(1)
+        tq.tq_set_wait_limit_ns(2_000_000)
+        tq.tq_test_withhold_handoffs(True)
         tq.tq_quantize_append(glayer, cache, k, v, [0] * wl.batch)
         torch.cuda.synchronize()
     finally:
+        tq.tq_test_withhold_handoffs(False)
         tq.tq_set_wait_limit_ns(0)
     assert tq.tq_device_errors(clear=True) & tq.ERRF_QUANTIZE_WAIT
     buf = cache.buffer.cpu().numpy()

@@ -62,8 +62,8 @@ def test_status_strings():
         assert tq.tq_status_string(code) == name
 
 
-def _params(d=128, kb=3, vb=2, g=32, ptr=256):
-    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr)
+def _params(d=128, kb=3, vb=2, g=32, ptr=256, mode=0, vptr=None):
+    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr, mode, vptr, vptr)
 
 
 def test_record_and_cache_bytes():
@@ -82,6 +82,11 @@ def test_record_and_cache_bytes():
     assert lib.tq_record_bytes(ctypes.byref(misaligned)) == 0
     misaligned = tq.Params(128, 3, 2, 32, 256, 260, 256, 256)
     assert lib.tq_record_bytes(ctypes.byref(misaligned)) == 0
+    # TurboQuant-MSE values: 102-byte records, the values' codebook required
+    assert lib.tq_record_bytes(ctypes.byref(_params(vb=3, mode=1, vptr=256))) == 102
+    assert lib.tq_record_bytes(ctypes.byref(_params(vb=3, mode=1))) == 0
+    assert lib.tq_record_bytes(ctypes.byref(_params(vb=3, mode=2, vptr=256))) == 0
+    assert lib.tq_cache_bytes(ctypes.byref(_params(vb=3, mode=1, vptr=256)), 1, 2, 256) == 2 * 2 * 13056
 
 
 def test_append_validation_before_launch():
@@ -209,8 +214,8 @@ def test_noalloc_validation_before_launch():
         return f(ctypes.byref(P) if P is not None else None, ctypes.byref(C), kw.get("q", q), 1,
                  kw.get("hq", 32), ln, kw.get("ml", 256), 0.088, kw.get("out", out), None)
 
-    assert call(tq.Params(128, 3, 2, 32, 264, 256, 256, 256)) == 1   # Pi not 16-byte aligned
-    assert call(tq.Params(128, 3, 2, 32, 256, 260, 256, 256)) == 1   # S not 16-byte aligned
+    assert call(tq.Params(128, 3, 2, 32, 264, 256, 256, 256, 0, None, None)) == 1   # Pi misaligned
+    assert call(tq.Params(128, 3, 2, 32, 256, 260, 256, 256, 0, None, None)) == 1   # S misaligned
     assert call(None) == 1
     assert call(_params(d=64)) == 2
     assert call(_params(), q=None) == 1
