@@ -56,6 +56,7 @@
 // sticky error word, stops, waits for its own copies and MMAs and frees TMEM.
 #include <math.h>
 
+#include "decode_splitk.cuh"
 #include "sm100.cuh"
 #include "tq_common.cuh"
 #include "tq_kernels.h"
@@ -281,9 +282,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   // split-major grid: every unit's first splits are scheduled before any
   // last (ragged, shorter) split, so the short CTAs fill the tail
   const int split = blockIdx.z, h = blockIdx.x, b = blockIdx.y;
-  // a codebook that needs the SIMT split-K kernel (the query-block kernel
-  // decided it): that kernel, launched next, writes every partial state
-  if (a.status[1] != 0) return;
+  // the query blocks (and the status words) come from the preceding kernel
+  pdl_wait();
+  pdl_trigger();
+  // A codebook whose operand planes fit in tensor memory only once (the
+  // query-block kernel decided it): this split runs the SIMT split-K body
+  // on 128 threads instead.
+  if (a.status[1] != 0) {
+    if (tid < 128) splitk_simt_body<G>(a, split, h, b, tid, smem_raw, 1);
+    return;
+  }
 
   int len = a.len[b] - a.len_sub;
   len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
@@ -879,6 +887,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   float *red = rot + G * 2 * kD;            // [8 warps][G][4]
   uint8_t *blk = reinterpret_cast<uint8_t *>(red + 8 * G * 4);  // QBLOCK staging
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();  // the decode kernel may launch now; it waits for this grid
 
   stage_matrix(mat, kPadQ, a.pi, tid, 256);
   stage_matrix(mat + kD * kPadQ, kPadQ, a.s, tid, 256);
@@ -920,8 +929,8 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     nm = 1;
   }
   // A codebook whose planes fit in tensor memory only once (an asymmetric
-  // codebook in a shape with little room) goes to the SIMT split-K kernel,
-  // which reads the rotated queries written below.  This kernel runs first
+  // codebook in a shape with little room) goes to the SIMT split-K body in
+  // the decode kernel, which reads the rotated queries written below.  This kernel runs first
   // in every tensor-core call, so it also clears the call's status word.
   const bool fallback = C::ak_ring(nm + 1) < 2;
   if (blockIdx.x == 0 && tid == 0) {
@@ -1037,6 +1046,7 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
   using C = Cfg<MB, VB, G>;
   const size_t smem = sizeof(TcSmem<C>);
   static_assert(sizeof(TcSmem<C>) <= 227 * 1024, "shared memory per CTA");
+  static_assert(sizeof(TcSmem<C>) >= (size_t)SplitkSmem<G>::kBytes, "fallback body scratch");
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<MB, VB, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1049,29 +1059,17 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
   qblock_kernel<MB, VB, G><<<qgrid, 256, qsmem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 grid(a.h_kv, a.batch, a.nsplit);
-  decode_tc_kernel<MB, VB, G><<<grid, kTcThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(decode_tc_kernel<MB, VB, G>, dim3(a.h_kv, a.batch, a.nsplit), dim3(kTcThreads), smem,
+                    stream, a);
 }
 
 }  // namespace
 
 size_t decode_tc_qblock_bytes(int key_bits, int G) { return qblock_bytes_for(key_bits - 1, G); }
 
-bool decode_tc_needs_fallback(int key_bits, int value_bits, int G) {
-  if (!decode_tc_supported(key_bits, value_bits, G)) return false;
-  const int mb = key_bits - 1;
-#define TQ_TC(MB_, VB_, G_) \
-  if (mb == MB_ && value_bits == VB_ && G == G_) return Cfg<MB_, VB_, G_>::ak_ring(1 << MB_) < 2;
-  TQ_TC(1, 2, 1) TQ_TC(1, 2, 2) TQ_TC(1, 2, 4) TQ_TC(1, 2, 8)
-  TQ_TC(2, 2, 1) TQ_TC(2, 2, 2) TQ_TC(2, 2, 4) TQ_TC(2, 2, 8)
-  TQ_TC(3, 2, 4) TQ_TC(2, 3, 6)
-#undef TQ_TC
-  return false;
-}
-
-bool decode_tc_supported(int key_bits, int value_bits, int G, int value_mode) {
-  if (value_mode != TQ_VALUES_GROUP) return false;  // MSE values: the SIMT split-K kernel
+bool decode_tc_supported(int key_bits, int value_bits, int G, int value_mode, int d) {
+  // MSE values and head dims other than 128: the SIMT split-K kernel
+  if (value_mode != TQ_VALUES_GROUP || d != kD) return false;
   const int mb = key_bits - 1;
   if (value_bits == 2 && (G == 1 || G == 2 || G == 4 || G == 8) && (mb == 1 || mb == 2)) return true;
   if (value_bits == 2 && mb == 3 && G == 4) return true;

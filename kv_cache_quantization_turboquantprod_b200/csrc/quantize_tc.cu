@@ -560,7 +560,7 @@ cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
 }  // namespace
 
 bool quantize_tc_supported(const AppendArgs &a) {
-  return a.value_mode == TQ_VALUES_GROUP && a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 && a.value_bits >= 2 &&
+  return a.d == kD && a.value_mode == TQ_VALUES_GROUP && a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 && a.value_bits >= 2 &&
          a.value_bits <= 4 && a.T >= 64;
 }
 

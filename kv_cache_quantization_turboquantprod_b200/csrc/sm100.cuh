@@ -107,6 +107,16 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor in the stream has finished;
+// pdl_wait() blocks until that predecessor has completed and its memory is
+// visible (a no-op for a normal launch).  pdl_trigger() lets this grid's
+// dependents be scheduled once every CTA of it has triggered or exited.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // 1-D bulk copy global -> shared, completing on an mbarrier (TMA engine).
 // dst and src 16-byte aligned, bytes a multiple of 16.
 // ---------------------------------------------------------------------------

@@ -19,10 +19,17 @@ constexpr int kRowBytes = kD / 8;  // one bit-plane row of a token
 constexpr int kPlaneBytes = kTile * kRowBytes;  // 2048
 constexpr int kPackedRowBytes = kD / 4;         // packed 2-bit value codes of a token
 
-// Byte offsets of the sections inside one tile.
+// Byte offsets of the sections inside one tile (head dim d: 64, 128 or 256;
+// the tensor-core kernels are built for d = kD = 128 and use the constants
+// above).
 struct TileLayout {
   int mb;          // Lloyd-Max bits (key_bits - 1)
   int vb;          // value bits
+  int d;           // head dim
+  int row_bytes;   // one bit-plane row of a token (d / 8)
+  int plane_bytes; // one bit-plane of a tile (128 rows)
+  int packed_row_bytes;  // packed 2-bit value codes of a token (d / 4)
+  int groups;      // value groups of a token (d / 32)
   int kplanes;     // offset of key planes
   int signs;       // offset of the sign plane
   int vplanes;     // offset of value planes
@@ -31,17 +38,23 @@ struct TileLayout {
   int tile_bytes;  // bytes of one tile
   bool mse;        // TurboQuant-MSE values: value cells as bit-planes + one fp16 norm
 
-  __host__ __device__ static TileLayout make(int key_bits, int value_bits, int value_mode = 0) {
+  __host__ __device__ static TileLayout make(int key_bits, int value_bits, int value_mode = 0,
+                                             int d = kD) {
     TileLayout L;
     L.mb = key_bits - 1;
     L.vb = value_bits;
+    L.d = d;
+    L.row_bytes = d / 8;
+    L.plane_bytes = kTile * L.row_bytes;
+    L.packed_row_bytes = d / 4;
+    L.groups = d / kGroup;
     L.mse = value_mode == TQ_VALUES_MSE;
     L.kplanes = 0;
-    L.signs = L.mb * kPlaneBytes;
-    L.vplanes = L.signs + kPlaneBytes;
-    L.norms = L.vplanes + L.vb * kPlaneBytes;
+    L.signs = L.mb * L.plane_bytes;
+    L.vplanes = L.signs + L.plane_bytes;
+    L.norms = L.vplanes + L.vb * L.plane_bytes;
     L.vsz = L.norms + kTile * 4;
-    L.tile_bytes = L.vsz + (L.mse ? kTile * 2 : kTile * 4 * kGroups);
+    L.tile_bytes = L.vsz + (L.mse ? kTile * 2 : kTile * 4 * L.groups);
     return L;
   }
   __host__ __device__ int record_bytes() const { return tile_bytes / kTile; }
@@ -59,10 +72,10 @@ __device__ __forceinline__ uint8_t *tile_ptr(void *data, const TileLayout &L,
 // 4i + m in bits 2m, 2m+1 of byte i) for 2-bit group-quantized values,
 // bit-planes otherwise (MSE values: the cell of rotated coordinate j).
 __device__ __forceinline__ int value_code(const uint8_t *tile, const TileLayout &L, int slot, int j) {
-  if (L.vb == 2 && !L.mse) return (tile[L.vplanes + slot * kPackedRowBytes + (j >> 2)] >> (2 * (j & 3))) & 3;
+  if (L.vb == 2 && !L.mse) return (tile[L.vplanes + slot * L.packed_row_bytes + (j >> 2)] >> (2 * (j & 3))) & 3;
   int code = 0;
   for (int p = 0; p < L.vb; ++p)
-    code |= ((tile[L.vplanes + p * kPlaneBytes + slot * kRowBytes + (j >> 3)] >> (j & 7)) & 1) << p;
+    code |= ((tile[L.vplanes + p * L.plane_bytes + slot * L.row_bytes + (j >> 3)] >> (j & 7)) & 1) << p;
   return code;
 }
 
@@ -97,12 +110,13 @@ __device__ __forceinline__ float warp_min(float x) {
   return x;
 }
 
-// Copy a row-major kD x kD fp32 matrix (16-byte aligned) into shared memory
+// Copy a row-major D x D fp32 matrix (16-byte aligned) into shared memory
 // with a row stride of `pad` floats.  Eight 16-byte loads per thread are in
 // flight at a time, so staging is bandwidth- rather than latency-bound.
+template <int D = kD>
 __device__ __forceinline__ void stage_matrix(float *dst, int pad, const float *src, int tid, int nthr) {
   const float4 *s4 = reinterpret_cast<const float4 *>(src);
-  constexpr int kN4 = kD * kD / 4;
+  constexpr int kN4 = D * D / 4;
   for (int base = tid; base < kN4; base += 8 * nthr) {
     float4 v[8];
 #pragma unroll
@@ -114,7 +128,7 @@ __device__ __forceinline__ void stage_matrix(float *dst, int pad, const float *s
     for (int u = 0; u < 8; ++u) {
       const int i = base + u * nthr;
       if (i < kN4) {
-        float *d = dst + ((4 * i) / kD) * pad + (4 * i) % kD;
+        float *d = dst + ((4 * i) / D) * pad + (4 * i) % D;
         d[0] = v[u].x;
         d[1] = v[u].y;
         d[2] = v[u].z;
@@ -125,7 +139,7 @@ __device__ __forceinline__ void stage_matrix(float *dst, int pad, const float *s
 }
 
 // QJL constant sqrt(pi/2) / d.
-__host__ __device__ constexpr float qjl_kappa() { return 1.2533141373155003f / kD; }
+__host__ __device__ constexpr float qjl_kappa(int d = kD) { return 1.2533141373155003f / d; }
 
 // Sketch components |(S r)_j| below this are re-decided in float64: the
 // single-precision paths (tensor-core hi/lo products, fp32 norms) can be off
@@ -140,36 +154,43 @@ __device__ __forceinline__ double warp_sum_f64(double x) {
 }
 
 // Warp-cooperative float64 re-decision of QJL sign bits for the key row of
-// lane `src` (all 32 lanes call it together).  Lane src passes its row's key
-// (element offset kbase into k), its Lloyd-Max code bit-planes (three planes
-// of four 32-coordinate words, planes beyond the code width zero), the mask of coordinates to re-decide (near) and
-// its sign words (sw), which it gets back corrected.  In float64: ||k||,
-// u = k / ||k||, r = u - Pi^T c (c = centroids of the stored codes) and, for
-// every masked j, (S r)_j; the stored bit is [(S r)_j >= 0].  Pi and S are
-// read row-major from global memory (four coordinates per lane).
+// lane `src` (all 32 lanes call it together), head dim D.  Lane src passes its
+// row's key (element offset kbase into k), its Lloyd-Max code bit-planes
+// (three planes of D/32 32-coordinate words, planes beyond the code width
+// zero), the mask of coordinates to re-decide (near) and its sign words (sw),
+// which it gets back corrected.  In float64: ||k||, u = k / ||k||,
+// r = u - Pi^T c (c = centroids of the stored codes) and, for every masked j,
+// (S r)_j; the stored bit is [(S r)_j >= 0].  Pi and S are read row-major
+// from global memory (D/32 coordinates per lane).
+template <int D = kD>
 __device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s, const float *cent,
                                                  const void *k, tq_dtype dt, size_t kbase,
-                                                 const uint32_t (&planes)[3][4], const uint32_t (&near)[4],
-                                                 uint32_t (&sw)[4], int src) {
+                                                 const uint32_t (&planes)[3][D / 32],
+                                                 const uint32_t (&near)[D / 32], uint32_t (&sw)[D / 32],
+                                                 int src) {
+  constexpr int W = D / 32;   // 32-coordinate words of a row
+  constexpr int C = D / 32;   // coordinates per lane
   const int lane = threadIdx.x & 31;
-  uint32_t pl[3][4], nw[4];
+  uint32_t pl[3][W], nw[W];
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = 0; w < W; ++w) {
 #pragma unroll
     for (int p = 0; p < 3; ++p) pl[p][w] = __shfl_sync(0xffffffffu, planes[p][w], src);
     nw[w] = __shfl_sync(0xffffffffu, near[w], src);
   }
   const unsigned long long kb = __shfl_sync(0xffffffffu, (unsigned long long)kbase, src);
-  double x[4], ss = 0.0;
+  double x[C], ss = 0.0;
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    x[m] = (double)load_elem(k, dt, kb + 4 * lane + m);
+  for (int m = 0; m < C; ++m) {
+    x[m] = (double)load_elem(k, dt, kb + C * lane + m);
     ss = fma(x[m], x[m], ss);
   }
   const double nk = sqrt(warp_sum_f64(ss));
-  double pc[4] = {0.0, 0.0, 0.0, 0.0};
+  double pc[C];
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int m = 0; m < C; ++m) pc[m] = 0.0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
     uint32_t b0 = pl[0][w], b1 = pl[1][w], b2 = pl[2][w];
 #pragma unroll 4
     for (int q = 0; q < 32; ++q) {
@@ -178,27 +199,24 @@ __device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s
       b1 >>= 1;
       b2 >>= 1;
       const double c = (double)cent[idx];
-      const float4 row = *reinterpret_cast<const float4 *>(pi + (size_t)(32 * w + q) * kD + 4 * lane);
-      pc[0] = fma((double)row.x, c, pc[0]);
-      pc[1] = fma((double)row.y, c, pc[1]);
-      pc[2] = fma((double)row.z, c, pc[2]);
-      pc[3] = fma((double)row.w, c, pc[3]);
+      const float *row = pi + (size_t)(32 * w + q) * D + C * lane;
+#pragma unroll
+      for (int m = 0; m < C; ++m) pc[m] = fma((double)row[m], c, pc[m]);
     }
   }
-  double r[4];
+  double r[C];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) r[m] = x[m] / nk - pc[m];
+  for (int m = 0; m < C; ++m) r[m] = x[m] / nk - pc[m];
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = 0; w < W; ++w) {
     uint32_t bits = nw[w];
     while (bits) {
       const int j = 32 * w + __ffs(bits) - 1;
       bits &= bits - 1;
-      const float4 srow = *reinterpret_cast<const float4 *>(s + (size_t)j * kD + 4 * lane);
-      double part = (double)srow.x * r[0];
-      part = fma((double)srow.y, r[1], part);
-      part = fma((double)srow.z, r[2], part);
-      part = fma((double)srow.w, r[3], part);
+      const float *srow = s + (size_t)j * D + C * lane;
+      double part = 0.0;
+#pragma unroll
+      for (int m = 0; m < C; ++m) part = fma((double)srow[m], r[m], part);
       const double z = warp_sum_f64(part);
       if (lane == src) {
         const uint32_t bit = 1u << (j & 31);

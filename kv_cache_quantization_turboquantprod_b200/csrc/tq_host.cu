@@ -85,7 +85,7 @@ cudaError_t set_wait_fields(Args &a) {
 
 tq_status check_params(const tq_params *p) {
   if (!p) return TQ_ERR_INVALID_ARGUMENT;
-  if (p->d != kD || p->group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if ((p->d != 64 && p->d != 128 && p->d != 256) || p->group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (p->key_bits < 2 || p->key_bits > 4) return TQ_ERR_UNSUPPORTED;
   if (p->value_bits < 2 || p->value_bits > 4) return TQ_ERR_UNSUPPORTED;
   if (!p->pi || !p->s || !p->centroids || !p->boundaries) return TQ_ERR_INVALID_ARGUMENT;
@@ -162,13 +162,13 @@ tq_status tq_make_codebook(int mse_bits, int d, double *centroids, double *bound
 
 size_t tq_record_bytes(const tq_params *p) {
   if (check_params(p) != TQ_OK) return 0;
-  return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode).record_bytes();
+  return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode, p->d).record_bytes();
 }
 
 size_t tq_cache_bytes(const tq_params *p, int batch, int h_kv, int capacity) {
   if (check_params(p) != TQ_OK) return 0;
   if (batch < 1 || h_kv < 1 || capacity < kTile || capacity % kTile) return 0;
-  const tq::TileLayout L = tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode);
+  const tq::TileLayout L = tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode, p->d);
   return (size_t)batch * h_kv * (size_t)(capacity / kTile) * (size_t)L.tile_bytes;
 }
 
@@ -193,6 +193,7 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
     a.lens[b] = len;
     a.nnew[b] = nn;
   }
+  a.d = p->d;
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids; a.boundaries = p->boundaries;
   a.value_mode = p->value_mode; a.v_centroids = p->v_centroids; a.v_boundaries = p->v_boundaries;
   a.data = c->data; a.k = k; a.v = v;
@@ -213,7 +214,7 @@ size_t tq_decode_workspace_size(const tq_params *p, const tq_cache *c, int h_q, 
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return 0;
   return tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits,
-                              p->value_mode).total_bytes;
+                              p->value_mode, p->d).total_bytes;
 }
 
 namespace {
@@ -226,7 +227,7 @@ namespace {
 int prefill_tokens_per_pass(const tq_params *p, int gqa, int t_chunk) {
   int ts = 1;
   while (2 * ts <= t_chunk && gqa * 2 * ts <= 4 &&
-         tq::decode_tc_supported(p->key_bits, p->value_bits, gqa * 2 * ts, p->value_mode))
+         tq::decode_tc_supported(p->key_bits, p->value_bits, gqa * 2 * ts, p->value_mode, p->d))
     ts *= 2;
   return ts;
 }
@@ -247,7 +248,7 @@ size_t tq_prefill_workspace_size(const tq_params *p, const tq_cache *c, int h_q,
   if (current_sm_count(&sms) != cudaSuccess) return 0;
   const int ts = prefill_tokens_per_pass(p, h_q / c->h_kv, t_chunk);
   return tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits, p->value_bits,
-                              p->value_mode)
+                              p->value_mode, p->d)
       .total_bytes;
 }
 
@@ -271,7 +272,7 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
   const int G = h_q / c->h_kv;
   const int ts = prefill_tokens_per_pass(p, G, t_chunk);
   if (workspace_bytes < tq::make_decode_plan(c->batch, c->h_kv, h_q * ts, max_len, sms, p->key_bits,
-                                             p->value_bits, p->value_mode).total_bytes)
+                                             p->value_bits, p->value_mode, p->d).total_bytes)
     return TQ_ERR_WORKSPACE;
   // passes of ts tokens (the last one of the largest power of two that is
   // left); pass tokens t0 .. t0 + n - 1 see len - (t_chunk - 1 - t) tokens
@@ -281,8 +282,9 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
     const int len_sub = t_chunk - t0 - n;
     const int ml = max_len - len_sub;
     const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q * n, ml, sms, p->key_bits, p->value_bits,
-                                                  p->value_mode);
+                                                  p->value_mode, p->d);
     tq::DecodeArgs a;
+    a.d = p->d;
     a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
     a.value_mode = p->value_mode; a.v_centroids = p->v_centroids;
     a.data = c->data; a.q = q; a.q_dtype = q_dtype; a.len = len_dev;
@@ -293,7 +295,6 @@ tq_status tq_prefill_attention(const tq_params *p, const tq_cache *c, const void
     a.win_k = nullptr; a.win_v = nullptr; a.win_dtype = TQ_BF16; a.win_len = nullptr; a.win_cap = 0;
     a.qt = n; a.q_tstride = t_chunk; a.q_t0 = t0; a.len_sub = len_sub;
     a.num_sms = sms;
-    a.fallback_gate = 0;
     if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
     tq::bind_workspace(a, P, workspace);
     a.out = out;
@@ -335,9 +336,10 @@ tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
   const tq::DecodePlan P = tq::make_decode_plan(c->batch, c->h_kv, h_q, max_len, sms, p->key_bits, p->value_bits,
-                                                p->value_mode);
+                                                p->value_mode, p->d);
   if (workspace_bytes < P.total_bytes) return TQ_ERR_WORKSPACE;
   tq::DecodeArgs a;
+  a.d = p->d;
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids;
   a.value_mode = p->value_mode; a.v_centroids = p->v_centroids;
   a.data = c->data; a.q = q; a.q_dtype = q_dtype; a.len = len_dev;
@@ -349,7 +351,6 @@ tq_status decode_common(const tq_params *p, const tq_cache *c, const void *q, tq
   a.win_cap = win_cap;
   a.qt = 1; a.q_tstride = 1; a.q_t0 = 0; a.len_sub = 0;
   a.num_sms = sms;
-  a.fallback_gate = 0;
   if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
   tq::bind_workspace(a, P, workspace);
   a.out = out;
@@ -414,6 +415,7 @@ tq_status tq_dequantize(const tq_params *p, const tq_cache *c, int b, int start,
   if (count == 0) return TQ_OK;
   if (!k_out || !v_out || !aligned(k_out, 4) || !aligned(v_out, 4)) return TQ_ERR_INVALID_ARGUMENT;
   tq::DequantArgs a;
+  a.d = p->d;
   a.pi = p->pi; a.s = p->s; a.centroids = p->centroids; a.data = c->data;
   a.value_mode = p->value_mode; a.v_centroids = p->v_centroids;
   a.h_kv = c->h_kv; a.ntiles = c->capacity / kTile; a.b = b; a.start = start; a.count = count;

@@ -6,15 +6,36 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "tq.h"
 
 namespace tq {
 
+// Launch `kernel` on `stream` with programmatic stream serialization: it may
+// start while its predecessor in the stream is still running and must call
+// pdl_wait() (sm100.cuh) before it reads that predecessor's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Arguments of one quantize_append launch.  Passed by value as a
 // __grid_constant__ kernel parameter (12 KB of per-sequence lengths and tile
 // offsets; CUDA 12.1+ allows kernel parameters up to 32764 bytes).
 struct AppendArgs {
+  int d;                                 // head dim (64, 128 or 256)
   const float *pi, *s, *centroids, *boundaries;
   int value_mode;                        // tq_value_mode
   const float *v_centroids, *v_boundaries;  // MSE values' codebook
@@ -52,6 +73,7 @@ struct DecodePlan {
 };
 
 struct DecodeArgs {
+  int d;                       // head dim (64, 128 or 256)
   const float *pi, *s, *centroids;
   int value_mode;              // tq_value_mode (MSE: partials in the rotated space)
   const float *v_centroids;    // MSE values' codebook
@@ -92,23 +114,20 @@ struct DecodeArgs {
   unsigned int *errors;
   // tests of the timeout path: the producer withholds the tile copies
   int test_withhold;
-  // SIMT split-K launched behind the tensor-core kernel: runs only when
-  // status[1] says the codebook needs it
-  int fallback_gate;
 };
 
-constexpr int kQRowElems = 128;  // elements per query / output row (d)
-
-// Element offset of virtual head hv's row of sequence b in q / out.  Virtual
-// heads of KV head h are h * G' + t * (G' / qt) + g (G' = h_q / h_kv).
+// Element offset of virtual head hv's row of sequence b in q / out (rows of
+// a.d elements).  Virtual heads of KV head h are h * G' + t * (G' / qt) + g
+// (G' = h_q / h_kv).
 __host__ __device__ inline size_t qrow_offset(const DecodeArgs &a, int b, int hv) {
-  if (a.qt == 1 && a.q_tstride == 1) return ((size_t)b * a.h_q + hv) * kQRowElems;
+  if (a.qt == 1 && a.q_tstride == 1) return ((size_t)b * a.h_q + hv) * a.d;
   const int gv = a.h_q / a.h_kv, greal = gv / a.qt, hreal = a.h_q / a.qt;
   const int h = hv / gv, r = hv % gv, t = r / greal, g = r % greal;
-  return (((size_t)b * a.q_tstride + a.q_t0 + t) * hreal + (size_t)h * greal + g) * kQRowElems;
+  return (((size_t)b * a.q_tstride + a.q_t0 + t) * hreal + (size_t)h * greal + g) * a.d;
 }
 
 struct DequantArgs {
+  int d;
   const float *pi, *s, *centroids;
   int value_mode;
   const float *v_centroids;
@@ -119,7 +138,7 @@ struct DequantArgs {
 };
 
 DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_sms,
-                            int key_bits, int value_bits, int value_mode = 0);
+                            int key_bits, int value_bits, int value_mode = 0, int d = 128);
 
 cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream);
 // Tensor-core quantize-append (bf16 K/V, appends of 64+ tokens).
@@ -130,12 +149,8 @@ cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_value_quant(const AppendArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 // Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
-bool decode_tc_supported(int key_bits, int value_bits, int gqa, int value_mode = 0);
-// True when a codebook whose Walsh expansion has every subset plane (an
-// asymmetric codebook) leaves room for only one plane buffer of the
-// tensor-core kernel in tensor memory; such codebooks run the SIMT split-K
-// kernel instead (decided on the device per call).
-bool decode_tc_needs_fallback(int key_bits, int value_bits, int gqa);
+bool decode_tc_supported(int key_bits, int value_bits, int gqa, int value_mode = 0, int d = 128);
+
 size_t decode_tc_qblock_bytes(int key_bits, int gqa);
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
 // qprep -> split-K (tensor-core kernel where built, SIMT otherwise) -> combine

@@ -74,7 +74,9 @@ def test_record_and_cache_bytes():
     assert lib.tq_record_bytes(ctypes.byref(_params(vb=3))) == 116
     assert lib.tq_cache_bytes(ctypes.byref(P), 2, 8, 256) == 2 * 8 * 2 * 12800
     assert lib.tq_cache_bytes(ctypes.byref(P), 2, 8, 200) == 0     # not a tile multiple
-    assert lib.tq_record_bytes(ctypes.byref(_params(d=64))) == 0
+    assert lib.tq_record_bytes(ctypes.byref(_params(d=64))) == 52       # head dims 64 and 256
+    assert lib.tq_record_bytes(ctypes.byref(_params(d=256))) == 196
+    assert lib.tq_record_bytes(ctypes.byref(_params(d=96))) == 0
     assert lib.tq_record_bytes(ctypes.byref(_params(g=16))) == 0
     assert lib.tq_record_bytes(ctypes.byref(_params(kb=5))) == 0
     # Pi and S must be 16-byte aligned (the kernels stage them with 16-byte loads)
@@ -98,7 +100,7 @@ def test_append_validation_before_launch():
     k = v = 1 << 21
     f = lib.tq_quantize_append
     assert f(None, ctypes.byref(C), k, v, 1, 4, lens, None, None) == 1
-    assert f(ctypes.byref(_params(d=64)), ctypes.byref(C), k, v, 1, 4, lens, None, None) == 2
+    assert f(ctypes.byref(_params(d=96)), ctypes.byref(C), k, v, 1, 4, lens, None, None) == 2
     assert f(ctypes.byref(P), None, k, v, 1, 4, lens, None, None) == 1
     assert f(ctypes.byref(P), ctypes.byref(C), k, v, 7, 4, lens, None, None) == 2   # dtype
     assert f(ctypes.byref(P), ctypes.byref(C), k, v, 1, -1, lens, None, None) == 1
@@ -217,7 +219,7 @@ def test_noalloc_validation_before_launch():
     assert call(tq.Params(128, 3, 2, 32, 264, 256, 256, 256, 0, None, None)) == 1   # Pi misaligned
     assert call(tq.Params(128, 3, 2, 32, 256, 260, 256, 256, 0, None, None)) == 1   # S misaligned
     assert call(None) == 1
-    assert call(_params(d=64)) == 2
+    assert call(_params(d=96)) == 2
     assert call(_params(), q=None) == 1
     assert call(_params(), q=q + 4) == 1      # q alignment
     assert call(_params(), out=out + 4) == 1  # out alignment
