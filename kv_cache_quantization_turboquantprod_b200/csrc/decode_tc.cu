@@ -191,10 +191,17 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   return false;
 }
 
-// The same, with one answer for the whole (converged) warp, so that a warp
-// never splits between lanes that go on to warp-collective tensor-memory
-// instructions and lanes that gave up.
+// The wait of a converged worker warp.  Every input of the decision -- the
+// barrier phase, the abort flag, the clock -- is read by one warp-wide
+// instruction, so the lanes of a converged warp decide alike and leave
+// together (no vote needed; a vote per wait measured 3.5% on decode).
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          const DecodeArgs &a) {
+  return wait_bar(bar, parity, abort_flag, a);
+}
+
+// The same with an explicit vote, for the MMA issuer warps (off the hot path).
+__device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           const DecodeArgs &a) {
   return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, a));
 }
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // worker groups, and neither waits behind the other.  The whole warp
     // runs the loop (descriptors stay warp-uniform); one elected lane issues.
     const bool leader = elect_one();
-    auto wait_all = [&](uint64_t *bar, uint32_t parity) { return wait_warp(bar, parity, &S.abort_flag, a); };
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) { return wait_vote(bar, parity, &S.abort_flag, a); };
     const bool qok = wait_all(&S.q_full, 0);
     int last = -1;  // last tile whose MMAs were committed
     if (warp == 1) {
