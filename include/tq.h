@@ -25,9 +25,9 @@
  * Conventions for every call:
  *  - Ownership: the caller owns every buffer and the stream.  The library
  *    allocates no memory and never synchronises (except tq_device_errors);
- *    its state is a cached per-device SM count, the wait limit, and one
- *    4-byte error word per device (plus the no-allocation entry point's
- *    fixed scratch).
+ *    its state is a cached per-device SM count, the wait limit, one 4-byte
+ *    error word and one 8-byte refinement counter per device (plus the
+ *    no-allocation entry point's fixed scratch).
  *  - Pointers documented as "device" must be device (or managed) memory of
  *    the current CUDA device; "host" pointers are read before the call
  *    returns.
@@ -47,8 +47,9 @@
  *  - Calls are asynchronous on `stream` and re-entrant.  Calls that write
  *    the same cache region (or the same workspace) must be ordered by the
  *    caller.
- *  - Only d = 128 and group = 32 are built; other values return
- *    TQ_ERR_UNSUPPORTED.  TurboQuant-MSE values (tq_value_mode) are encoded
+ *  - Head dims d = 64, 128 and 256 with group = 32 are built (the
+ *    tensor-core kernels at d = 128, the SIMT kernels at all three); other
+ *    values return TQ_ERR_UNSUPPORTED.  TurboQuant-MSE values (tq_value_mode) are encoded
  *    by the SIMT quantize-append kernel and decoded by the SIMT split-K
  *    kernel, accumulated in the rotated space and rotated back once per
  *    head in the combine step.
@@ -389,6 +390,25 @@ TQ_API tq_status tq_set_wait_limit_ns(unsigned long long ns);
  * TQ_OK.
  */
 TQ_API tq_status tq_test_withhold_handoffs(int on);
+
+/*
+ * tq_test_sign_refine_threshold -- for tests of the float64 sign refinement
+ * only: quantize-append calls made afterwards re-decide in float64 every QJL
+ * sign whose single-precision sketch component has |(S r)_j| < z (0 restores
+ * the default, 1e-5; negative: TQ_ERR_INVALID_ARGUMENT).  A larger z sends
+ * many more keys through the refinement (slower, same stored bits outside
+ * float64 rounding).
+ */
+TQ_API tq_status tq_test_sign_refine_threshold(double z);
+
+/*
+ * tq_test_refine_count -- synchronise the current device, then read (and, if
+ * `clear` is nonzero, reset) the number of QJL sign bits that quantize-append
+ * kernels on it have re-decided in float64 since the last reset.  count: host
+ * pointer.  TQ_ERR_INVALID_ARGUMENT for a null pointer, TQ_ERR_CUDA if the
+ * device reports an error.
+ */
+TQ_API tq_status tq_test_refine_count(unsigned long long *count, int clear);
 
 /*
  * tq_device_errors -- synchronise the current device, then read (and, if

@@ -332,7 +332,7 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
         const bool zero = !(S.nk[vi] > 0.f);
         const int bit = (!zero && acc[v] >= 0.f) ? 1 : 0;
         const unsigned word = __ballot_sync(0xffffffffu, bit);
-        const unsigned nearb = __ballot_sync(0xffffffffu, valid && !zero && fabsf(acc[v]) < kSignRefineZ);
+        const unsigned nearb = __ballot_sync(0xffffffffu, valid && !zero && fabsf(acc[v]) < a.refine_z);
         if (lane == 0 && nearb) S.nearw[vi][i >> 5] = nearb;
         if (valid) {
           const int pos = a.lens[b] + t;
@@ -380,10 +380,15 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
       }
       const size_t kbase = (((size_t)b * a.T + t) * a.h_kv + h) * D;
       refine_signs_f64<D>(a.pi, a.s, S.cent, a.k, a.dtype, kbase, planes, nw, sw, 0);
-      if (lane == 0)
+      if (lane == 0) {
+        int nbits = 0;
 #pragma unroll
-        for (int w = 0; w < C; ++w)
+        for (int w = 0; w < C; ++w) {
           *reinterpret_cast<uint32_t *>(tile + L.signs + slot * L.row_bytes + 4 * w) = sw[w];
+          nbits += __popc(nw[w]);
+        }
+        if (a.refine_count) atomicAdd(a.refine_count, (unsigned long long)nbits);
+      }
     }
     __syncthreads();
   }

@@ -19,13 +19,18 @@
 // Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
 // record section a tile writes is one contiguous run of the cache.
 //
-// Warp roles (448 threads):
+// Warp roles (480 threads):
 //   warps 0, 13   MMA issuers of epilogue groups 0 and 1 (one elected lane),
 //                 each sleeping in blocking waits on its group's barriers
 //   warps 1-4     loader: K rows -> scaled fp16 A operand + norms in shared
 //                 memory
 //   warps 5-8     epilogue group 0 (even tiles)   | thread = tile row = TMEM
 //   warps 9-12    epilogue group 1 (odd tiles)    | lane; 256 TMEM columns each
+//   warp 14       sign refiner: sketch components the epilogue found next to
+//                 zero (|S r| < 1e-5, about one key in 300) get their sign
+//                 again in float64, off the pipeline's critical path; each
+//                 epilogue warp hands such rows over through its own ring in
+//                 shared memory and the refiner patches the stored sign words
 // Every mbarrier wait between roles is bounded (2 s unless the host set another
 // limit) and answers warp-uniformly; on timeout the CTA raises its abort flag
 // and the device's sticky error word, stops, lets its own MMAs finish, frees
@@ -42,8 +47,10 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQtThreads = 448;
+constexpr int kQtThreads = 480;
 constexpr int kIssuer1Warp = 13;  // MMA issuer of epilogue group 1 (warp 0 issues for group 0)
+constexpr int kRefineWarp = 14;   // float64 sign refiner
+constexpr int kRingCap = 16;      // refinement requests per epilogue warp in flight
 constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
 constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
 constexpr float kSScale = 256.f;       // S parts x 2^8
@@ -57,6 +64,16 @@ constexpr float kRScale = 8192.f;      // residual parts x 2^13
 __host__ __device__ constexpr int blk_off(int row, int col) {
   return (col >> 3) * 2048 + (row >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2;
 }
+
+// A key row whose sketch has components next to zero: its code planes, the
+// mask of components to re-decide, its key's element offset and the address
+// of its stored sign row.
+struct RefineReq {
+  uint32_t planes[3][4];
+  uint32_t near[4];
+  unsigned long long kbase;
+  unsigned long long signs;
+};
 
 struct QtSmem {
   alignas(1024) uint8_t pi[2][kMat16];  // Pi x 2^10: hi, lo
@@ -72,6 +89,12 @@ struct QtSmem {
       d_free[2];
   uint32_t tmem_base;
   volatile int abort_flag;
+  // refinement rings, one per epilogue warp (single producer, the refiner
+  // the single consumer): requests [head, tail) are pending
+  RefineReq ring[8][kRingCap];
+  volatile int ring_head[8], ring_tail[8];
+  volatile int epi_done;  // epilogue warps past their last tile
+  volatile int progress;  // changes whenever an epilogue warp finishes a tile
 };
 
 struct TileInfo {
@@ -104,6 +127,30 @@ __device__ __forceinline__ bool qwait(uint64_t *bar, uint32_t parity, volatile i
   bool timed_out = false;
   const bool ok = pipe_wait(bar, parity, abort_flag, a.wait_ns, a.wait_hint_ns, &timed_out);
   if (timed_out && a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_QUANTIZE_WAIT);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait until epilogue warp ew's refinement ring has room for the
+// requests before index `upto` (upto - head <= kRingCap); one answer for the
+// whole warp.
+__device__ __forceinline__ bool ring_room(QtSmem &S, int ew, int upto, const AppendArgs &a) {
+  bool ok = true;
+  if (upto - S.ring_head[ew] > kRingCap) {
+    const uint64_t t0 = globaltimer_ns();
+    while (upto - S.ring_head[ew] > kRingCap) {
+      if (S.abort_flag) {
+        ok = false;
+        break;
+      }
+      if (globaltimer_ns() - t0 > a.wait_ns) {
+        S.abort_flag = 1;
+        if (a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_QUANTIZE_WAIT);
+        ok = false;
+        break;
+      }
+      __nanosleep(128);
+    }
+  }
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -184,6 +231,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       mbar_init(&S.d_free[g], 4);
     }
     S.abort_flag = 0;
+    for (int w = 0; w < 8; ++w) S.ring_head[w] = S.ring_tail[w] = 0;
+    S.epi_done = 0;
+    S.progress = 0;
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&S.tmem_base, 512);
@@ -346,7 +396,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       // bounded wait on it then runs out)
       if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full[g]);
     }
-  } else {
+  } else if (warp <= 12) {
     // ---------------- epilogue groups --------------------------------------
     const int g = (warp - 5) >> 2;
     const int q4 = warp & 3;
@@ -484,7 +534,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       uint32_t sw[4] = {0u, 0u, 0u, 0u};
       uint32_t nearw[4] = {0u, 0u, 0u, 0u};  // |S r| below the refinement threshold
       // D = (S r) x 2^21 (R x 2^13 times S x 2^8)
-      constexpr float kNearZ = kSignRefineZ * 2097152.f;
+      const float kNearZ = a.refine_z * 2097152.f;
       tmem_ld16(dcol, dA);
       tmem_wait_ld();
 #pragma unroll
@@ -505,22 +555,125 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.d_free[g]);
-      // sketch components next to zero: the sign again in float64 (rare)
-      unsigned need = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1] | nearw[2] | nearw[3]) != 0u);
-      if (need) {
-        const size_t kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;
-        while (need) {
-          const int src = __ffs(need) - 1;
-          need &= need - 1;
-          refine_signs_f64(a.pi, a.s, S.cent, a.k, a.dtype, kbase, planes, nearw, sw, src);
-        }
-      }
       if (valid) {
         *reinterpret_cast<uint4 *>(tp + L.signs + slot * kRowBytes) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
         const float rn = zero ? 0.f : sqrtf(rr) * (1.f / kRScale);
         *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) =
             __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
       }
+      // sketch components next to zero: handed to the float64 refiner, which
+      // patches the sign words stored above (at most kRingCap rows at a time)
+      unsigned rest = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1] | nearw[2] | nearw[3]) != 0u);
+      bool stop = false;
+      while (rest) {
+        const int ew = warp - 5;
+        const int tail = S.ring_tail[ew];
+        const int rank = __popc(rest & ((1u << lane) - 1u));
+        const unsigned chunk = __ballot_sync(0xffffffffu, ((rest >> lane) & 1u) && rank < kRingCap);
+        const int n = __popc(chunk);
+        if (!ring_room(S, ew, tail + n, a)) {
+          stop = true;
+          break;
+        }
+        if ((chunk >> lane) & 1u) {
+          RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int p = 0; p < 3; ++p) q.planes[p][w] = p < MB ? planes[p][w] : 0u;
+            q.near[w] = nearw[w];
+          }
+          q.kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;
+          q.signs = (unsigned long long)(tp + L.signs + slot * kRowBytes);
+        }
+        // the sign rows and the requests, then the new tail
+        __threadfence_block();
+        __syncwarp();
+        if (lane == 0) S.ring_tail[ew] = tail + n;
+        __syncwarp();
+        rest &= ~chunk;
+      }
+      if (stop) break;
+      if (lane == 0) S.progress = S.progress + 1;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      atomicAdd(const_cast<int *>(&S.epi_done), 1);
+    }
+  } else if (warp == kRefineWarp) {
+    // ---------------- sign refiner -----------------------------------------
+    // Serves the eight rings in turn until every epilogue warp is done and
+    // the rings are empty.  Its waits are on the epilogue warps, whose own
+    // waits are bounded; it is bounded too (same limit, measured from the
+    // last request or finished tile it saw) and gives up by raising the
+    // abort flag.
+    unsigned long long t_last = globaltimer_ns();
+    int seen = S.progress;
+    while (true) {
+      // shared words are read by lane 0 and broadcast, so the warp stays converged
+      const int done = __shfl_sync(0xffffffffu, S.epi_done, 0);  // before the rings: no request after it is missed
+      bool any = false;
+#pragma unroll 1
+      for (int ew = 0; ew < 8; ++ew) {
+        int h = __shfl_sync(0xffffffffu, S.ring_head[ew], 0);
+        const int t = __shfl_sync(0xffffffffu, S.ring_tail[ew], 0);
+        if (h == t) continue;
+        __threadfence_block();
+        for (; h != t; ++h) {
+          const RefineReq &q = S.ring[ew][h % kRingCap];
+          uint32_t pl[3][4], nw[4], res[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int p = 0; p < 3; ++p) pl[p][w] = q.planes[p][w];
+            nw[w] = q.near[w];
+          }
+          const unsigned long long kb = q.kbase;
+          uint32_t *words = reinterpret_cast<uint32_t *>(q.signs);
+          refine_row_f64<kD, 32>(a.pi, a.s, S.cent, a.k, a.dtype, kb, pl, nw, res);
+          uint32_t mn = 0u, mr = 0u;  // lane w < 4 patches word w
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            if (lane == w) {
+              mn = nw[w];
+              mr = res[w];
+            }
+          if (mn != 0u) {
+            atomicAnd(words + lane, ~mn);
+            atomicOr(words + lane, mr);
+          }
+          if (lane == 0 && a.refine_count)
+            atomicAdd(a.refine_count,
+                      (unsigned long long)(__popc(nw[0]) + __popc(nw[1]) + __popc(nw[2]) + __popc(nw[3])));
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence_block();
+            S.ring_head[ew] = h + 1;  // the slot may be reused
+          }
+          __syncwarp();
+        }
+        any = true;
+      }
+      if (any) {
+        t_last = globaltimer_ns();
+        continue;
+      }
+      if (done == 8) break;
+      if (__shfl_sync(0xffffffffu, S.abort_flag, 0)) break;
+      const int prog = __shfl_sync(0xffffffffu, S.progress, 0);
+      if (prog != seen) {
+        seen = prog;
+        t_last = globaltimer_ns();
+      } else if (globaltimer_ns() - t_last > a.wait_ns) {
+        if (lane == 0) {
+          S.abort_flag = 1;
+          if (a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_QUANTIZE_WAIT);
+        }
+        __syncwarp();
+        break;
+      }
+      __nanosleep(256);
     }
   }
 

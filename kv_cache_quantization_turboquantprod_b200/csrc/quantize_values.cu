@@ -3,19 +3,25 @@
 // value_bits, value_group_size): per group of 32 channels of one token's
 // head vector, zero = fp16(min), scale = fp16((max - min) / (2^vb - 1))
 // rounded once from the exact quotient, code = clamp(rint((v - zero) /
-// scale)) of the exact quotient.
+// scale)) of the exact quotient (half to even).
 //
-// Memory-level parallelism decides the speed of this streaming kernel: a
-// half-warp takes one vector (16 lanes x 8 channels, one 16-byte load of
-// bf16 per lane), a warp two, and every iteration issues the loads of four
-// such pairs (eight vectors) before it quantizes any.  A group of 32
-// channels is 4 lanes (min and max by two shuffles).  Codes use the
-// reciprocal of the fp16 scale and are redone in float64 where the product
-// sits next to a half-integer, so every code is the rounded exact quotient.
-// The records' value sections (codes, scale, zero) are written in place;
-// the key sections are the tensor-core kernel's.  Grid-stride over all
-// B x T x H_kv vector slots; head dim 128, bf16 input (the tensor-core append
-// path).
+// A quarter-warp takes one vector: lane ql of the quarter holds channels
+// 16 ql .. 16 ql + 15 (two 16-byte loads of bf16), so a group of 32 channels
+// is a lane pair (min and max by one shuffle) and a warp streams four
+// consecutive vectors (1 KB) per round; two rounds' loads are issued before
+// either is quantized.  The vector slot id = (b T + t) H_kv + h gives the
+// input offset directly; the division into (b, t, h) and the record address
+// are computed by one lane per vector and handed to its quarter by shuffles.
+//
+// Codes.  For 2-bit values the code is the number of the group's three
+// rounding thresholds z + (k + 1/2) s below v, with the thresholds formed in
+// float64 (exact: z and s are fp16) and rounded down to float32; a threshold
+// that is exactly representable and belongs to an odd k (a tie that rounds
+// up to even) also counts v equal to it.  That is the rounded exact quotient
+// by comparisons alone.  For 3 and 4 bits the code is rint of the float32
+// quotient, redone in float64 where it sits within 1e-5 of a half-integer.
+// The records' value sections (codes, scale, zero) are written in place; the
+// key sections are the tensor-core kernel's.  Head dim 128, bf16 input.
 #include "tq_common.cuh"
 #include "tq_kernels.h"
 
@@ -24,100 +30,140 @@ namespace tq {
 namespace {
 
 constexpr int kVqThreads = 256;
-constexpr int kVqUnroll = 4;  // vector pairs in flight per warp
+constexpr int kVqRounds = 2;  // rounds of 4 vectors per warp iteration
 
-__global__ void __launch_bounds__(kVqThreads) value_quant_kernel(const __grid_constant__ AppendArgs a) {
-  const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode, kD);
-  const int lane = threadIdx.x & 31;
-  const int half = lane >> 4, hl = lane & 15;  // vector of the pair, lane within it
-  const long long per_b = (long long)a.T * a.h_kv;
-  const long long total = (long long)a.batch * per_b;
-  const long long npairs = (total + 1) / 2;
-  const long long nwarps = (long long)gridDim.x * (kVqThreads / 32);
-  const float vlevels = (float)((1 << a.value_bits) - 1);
-  const int ilev = (1 << a.value_bits) - 1;
-  for (long long p0 = ((long long)blockIdx.x * (kVqThreads / 32) + (threadIdx.x >> 5)) * kVqUnroll;
-       p0 < npairs; p0 += nwarps * kVqUnroll) {
-    // issue every load of the iteration first
-    uint4 raw[kVqUnroll];
-    int vb_[kVqUnroll], vt_[kVqUnroll], vh_[kVqUnroll];
-    bool ok[kVqUnroll];
+// fp16 scale of a group: the float64 difference and quotient, rounded once
+// to fp16 (the same operations as the float64 definition).
+__device__ __forceinline__ __half group_scale(float mn, float mx, int levels) {
+  return __double2half(((double)mx - (double)mn) / (double)levels);
+}
+
+// The largest float below a finite float f.
+__device__ __forceinline__ float float_below(float f) {
+  if (f == 0.f) return -__uint_as_float(1u);  // the negative of the least subnormal
+  const uint32_t u = __float_as_uint(f);
+  return __uint_as_float(f > 0.f ? u - 1u : u + 1u);
+}
+
+// Packed 2-bit codes of 16 channels (channel 4i + m in bits 2m, 2m+1 of
+// byte i) by threshold counts.
+__device__ __forceinline__ uint32_t codes2_packed(const float (&x)[16], __half zero16, __half scale16) {
+  float thr[3];
+  const double z = (double)__half2float(zero16), s = (double)__half2float(scale16);
 #pragma unroll
-    for (int u = 0; u < kVqUnroll; ++u) {
-      const long long id = 2 * (p0 + u) + half;
-      ok[u] = id < total;
-      int b = 0, t = 0, h = 0;
-      if (ok[u]) {
-        b = (int)(id / per_b);
-        const long long rem = id - (long long)b * per_b;
-        t = (int)(rem / a.h_kv);
-        h = (int)(rem - (long long)t * a.h_kv);
-        ok[u] = t < a.nnew[b];
+  for (int k = 0; k < 3; ++k) {
+    if (s == 0.0) {
+      thr[k] = INFINITY;  // zero scale: every code 0
+      continue;
+    }
+    const double t = fma((double)k + 0.5, s, z);  // exact
+    float tf = __double2float_rd(t);
+    // odd k: a value equal to the threshold rounds up (to the even code)
+    if ((k & 1) && (double)tf == t) tf = float_below(tf);
+    thr[k] = tf;
+  }
+  uint32_t w = 0u;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const uint32_t c = (x[e] > thr[0] ? 1u : 0u) + (x[e] > thr[1] ? 1u : 0u) + (x[e] > thr[2] ? 1u : 0u);
+    w |= c << (2 * e);
+  }
+  return w;
+}
+
+template <int VB>
+__global__ void __launch_bounds__(kVqThreads) value_quant_kernel(const __grid_constant__ AppendArgs a) {
+  const TileLayout L = TileLayout::make(a.key_bits, VB, a.value_mode, kD);
+  const int lane = threadIdx.x & 31;
+  const int qv = lane >> 3, ql = lane & 7;  // vector of the round, lane within it
+  const long long total = (long long)a.batch * a.T * a.h_kv;
+  const long long per_b = (long long)a.T * a.h_kv;
+  const long long nwarps = (long long)gridDim.x * (kVqThreads / 32);
+  constexpr int kLevels = (1 << VB) - 1;
+  constexpr int kVecs = 4 * kVqRounds;  // vectors per warp iteration
+  for (long long id0 = ((long long)blockIdx.x * (kVqThreads / 32) + (threadIdx.x >> 5)) * kVecs; id0 < total;
+       id0 += nwarps * kVecs) {
+    // lane j < kVecs: where vector id0 + j goes (record offset, slot; -1: none)
+    long long roff = -1;
+    int rslot = 0;
+    if (lane < kVecs && id0 + lane < total) {
+      const long long id = id0 + lane;
+      const int b = (int)(id / per_b);
+      const long long rem = id - (long long)b * per_b;
+      const int t = (int)(rem / a.h_kv);
+      const int h = (int)(rem - (long long)t * a.h_kv);
+      if (t < a.nnew[b]) {
+        const int pos = a.lens[b] + t;
+        roff = (long long)((((size_t)b * a.h_kv + h) * (size_t)a.ntiles + (size_t)(pos / kTile)) *
+                           (size_t)L.tile_bytes);
+        rslot = pos % kTile;
       }
-      vb_[u] = b; vt_[u] = t; vh_[u] = h;
-      const size_t base = (((size_t)b * a.T + t) * a.h_kv + h) * kD + 8 * hl;
-      raw[u] = ok[u] ? *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v) + base)
-                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // issue every load of the iteration first
+    uint4 raw[kVqRounds][2];
+#pragma unroll
+    for (int u = 0; u < kVqRounds; ++u) {
+      const long long id = id0 + 4 * u + qv;
+      const bool in = id < total;
+      const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v) +
+                                                         (size_t)(in ? id : 0) * kD + 16 * ql);
+      raw[u][0] = in ? src[0] : make_uint4(0u, 0u, 0u, 0u);
+      raw[u][1] = in ? src[1] : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int u = 0; u < kVqUnroll; ++u) {
-      float x[8];
-      const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u]);
+    for (int u = 0; u < kVqRounds; ++u) {
+      const long long off = __shfl_sync(0xffffffffu, roff, 4 * u + qv);
+      const int slot = __shfl_sync(0xffffffffu, rslot, 4 * u + qv);
+      float x[16];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(p2[e]);
-        x[2 * e] = f.x;
-        x[2 * e + 1] = f.y;
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t *wv = reinterpret_cast<const uint32_t *>(&raw[u][c]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[8 * c + 2 * e] = __uint_as_float(wv[e] << 16);
+          x[8 * c + 2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
+        }
       }
       float mn = x[0], mx = x[0];
 #pragma unroll
-      for (int e = 1; e < 8; ++e) {
+      for (int e = 1; e < 16; ++e) {
         mn = fminf(mn, x[e]);
         mx = fmaxf(mx, x[e]);
       }
-      // a group of 32 channels = 4 consecutive lanes
+      // a group of 32 channels = lanes 2i, 2i + 1 of the quarter
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const __half zero16 = __float2half_rn(mn);
-      const __half scale16 = __double2half(((double)mx - (double)mn) / (double)vlevels);
-      const float z32 = __half2float(zero16), sc32 = __half2float(scale16);
-      int code[8];
+      const __half scale16 = group_scale(mn, mx, kLevels);
+      if (off < 0) continue;  // uniform within each quarter; no collectives follow
+      uint8_t *tile = reinterpret_cast<uint8_t *>(a.data) + off;
+      if constexpr (VB == 2) {
+        // packed: this lane's 16 channels are bytes 4 ql .. 4 ql + 3 of the row
+        *reinterpret_cast<uint32_t *>(tile + L.vplanes + slot * L.packed_row_bytes + 4 * ql) =
+            codes2_packed(x, zero16, scale16);
+      } else {
+        const float z32 = __half2float(zero16), sc32 = __half2float(scale16);
+        const float rsc = sc32 != 0.f ? 1.f / sc32 : 0.f;
+        uint32_t pw[VB];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) code[e] = 0;
-      if (sc32 != 0.f) {
-        const float rsc = 1.f / sc32;
+        for (int p = 0; p < VB; ++p) pw[p] = 0u;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 16; ++e) {
           const float tq = (x[e] - z32) * rsc;
           float r = rintf(tq);
           if (fabsf(tq - r) > 0.5f - 1e-5f) r = (float)rint(((double)x[e] - (double)z32) / (double)sc32);
-          code[e] = min(max((int)r, 0), ilev);
-        }
-      }
-      if (!ok[u]) continue;  // uniform within each half-warp; no collectives follow
-      const int pos = a.lens[vb_[u]] + vt_[u];
-      uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, vb_[u], vh_[u], pos / kTile);
-      const int slot = pos % kTile;
-      if (L.vb == 2) {
-        // packed: channel 4i + m in bits 2m, 2m+1 of byte i; this lane's 8
-        // channels are bytes 2 hl and 2 hl + 1
-        uint32_t w = 0u;
+          const uint32_t code = sc32 != 0.f ? (uint32_t)min(max((int)r, 0), kLevels) : 0u;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w |= (uint32_t)code[e] << (2 * e);
-        *reinterpret_cast<uint16_t *>(tile + L.vplanes + slot * L.packed_row_bytes + 2 * hl) = (uint16_t)w;
-      } else {
-        // plane p: byte hl of the row holds bit p of this lane's 8 channels
-        for (int p = 0; p < L.vb; ++p) {
-          uint32_t byte = 0u;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) byte |= (uint32_t)((code[e] >> p) & 1) << e;
-          tile[L.vplanes + p * L.plane_bytes + slot * L.row_bytes + hl] = (uint8_t)byte;
+          for (int p = 0; p < VB; ++p) pw[p] |= ((code >> p) & 1u) << e;
         }
+        // plane p: bytes 2 ql, 2 ql + 1 of the row hold bit p of this lane's channels
+#pragma unroll
+        for (int p = 0; p < VB; ++p)
+          *reinterpret_cast<uint16_t *>(tile + L.vplanes + p * L.plane_bytes + slot * L.row_bytes + 2 * ql) =
+              (uint16_t)pw[p];
       }
-      if ((hl & 3) == 0)
-        *reinterpret_cast<__half2 *>(tile + L.vsz + (slot * L.groups + (hl >> 2)) * 4) =
+      if ((ql & 1) == 0)
+        *reinterpret_cast<__half2 *>(tile + L.vsz + (slot * L.groups + (ql >> 1)) * 4) =
             __halves2half2(scale16, zero16);
     }
   }
@@ -128,10 +174,15 @@ __global__ void __launch_bounds__(kVqThreads) value_quant_kernel(const __grid_co
 cudaError_t launch_value_quant(const AppendArgs &a, int num_sms, cudaStream_t stream) {
   const long long total = (long long)a.batch * a.T * a.h_kv;
   if (total == 0) return cudaSuccess;
-  const long long per_block = 2LL * kVqUnroll * (kVqThreads / 32);  // vectors per block iteration
+  const long long per_block = 4LL * kVqRounds * (kVqThreads / 32);  // vectors per block iteration
   const long long blocks = (total + per_block - 1) / per_block;
   const int grid = (int)std::min<long long>(blocks, 8LL * num_sms);
-  value_quant_kernel<<<grid, kVqThreads, 0, stream>>>(a);
+  switch (a.value_bits) {
+    case 2: value_quant_kernel<2><<<grid, kVqThreads, 0, stream>>>(a); break;
+    case 3: value_quant_kernel<3><<<grid, kVqThreads, 0, stream>>>(a); break;
+    case 4: value_quant_kernel<4><<<grid, kVqThreads, 0, stream>>>(a); break;
+    default: return cudaErrorNotSupported;
+  }
   return cudaGetLastError();
 }
 

@@ -153,36 +153,29 @@ __device__ __forceinline__ double warp_sum_f64(double x) {
   return x;
 }
 
-// Warp-cooperative float64 re-decision of QJL sign bits for the key row of
-// lane `src` (all 32 lanes call it together), head dim D.  Lane src passes its
-// row's key (element offset kbase into k), its Lloyd-Max code bit-planes
+// Warp-cooperative float64 re-decision of QJL sign bits of one key row, head
+// dim D (all 32 lanes call it together with the same arguments).  The row's
+// key starts at element kbase of k; pl holds its Lloyd-Max code bit-planes
 // (three planes of D/32 32-coordinate words, planes beyond the code width
-// zero), the mask of coordinates to re-decide (near) and its sign words (sw),
-// which it gets back corrected.  In float64: ||k||, u = k / ||k||,
-// r = u - Pi^T c (c = centroids of the stored codes) and, for every masked j,
-// (S r)_j; the stored bit is [(S r)_j >= 0].  Pi and S are read row-major
-// from global memory (D/32 coordinates per lane).
-template <int D = kD>
-__device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s, const float *cent,
-                                                 const void *k, tq_dtype dt, size_t kbase,
-                                                 const uint32_t (&planes)[3][D / 32],
-                                                 const uint32_t (&near)[D / 32], uint32_t (&sw)[D / 32],
-                                                 int src) {
+// zero) and near the mask of coordinates to re-decide.  In float64: ||k||,
+// u = k / ||k||, r = u - Pi^T c (c = centroids of the stored codes) and, for
+// every masked j, (S r)_j; bit j of the returned words is [(S r)_j >= 0]
+// (zero outside the mask).  Pi and S are read row-major from global memory
+// (D/32 coordinates per lane), Pi in batches of rows whose loads (a lane's
+// kFloatsInFlight floats) are all in flight before any is used.
+template <int D = kD, int kFloatsInFlight = 64>
+__device__ __forceinline__ void refine_row_f64(const float *pi, const float *s, const float *cent,
+                                               const void *k, tq_dtype dt, size_t kbase,
+                                               const uint32_t (&pl)[3][D / 32], const uint32_t (&nw)[D / 32],
+                                               uint32_t (&res)[D / 32]) {
   constexpr int W = D / 32;   // 32-coordinate words of a row
   constexpr int C = D / 32;   // coordinates per lane
+  constexpr int kBatch = kFloatsInFlight / C;  // rows of Pi per batch (<= 32)
   const int lane = threadIdx.x & 31;
-  uint32_t pl[3][W], nw[W];
-#pragma unroll
-  for (int w = 0; w < W; ++w) {
-#pragma unroll
-    for (int p = 0; p < 3; ++p) pl[p][w] = __shfl_sync(0xffffffffu, planes[p][w], src);
-    nw[w] = __shfl_sync(0xffffffffu, near[w], src);
-  }
-  const unsigned long long kb = __shfl_sync(0xffffffffu, (unsigned long long)kbase, src);
   double x[C], ss = 0.0;
 #pragma unroll
   for (int m = 0; m < C; ++m) {
-    x[m] = (double)load_elem(k, dt, kb + C * lane + m);
+    x[m] = (double)load_elem(k, dt, kbase + C * lane + m);
     ss = fma(x[m], x[m], ss);
   }
   const double nk = sqrt(warp_sum_f64(ss));
@@ -191,17 +184,22 @@ __device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s
   for (int m = 0; m < C; ++m) pc[m] = 0.0;
 #pragma unroll
   for (int w = 0; w < W; ++w) {
-    uint32_t b0 = pl[0][w], b1 = pl[1][w], b2 = pl[2][w];
-#pragma unroll 4
-    for (int q = 0; q < 32; ++q) {
-      const int idx = (int)((b0 & 1u) | ((b1 & 1u) << 1) | ((b2 & 1u) << 2));
-      b0 >>= 1;
-      b1 >>= 1;
-      b2 >>= 1;
-      const double c = (double)cent[idx];
-      const float *row = pi + (size_t)(32 * w + q) * D + C * lane;
+#pragma unroll 1
+    for (int q0 = 0; q0 < 32; q0 += kBatch) {
+      const int i0 = 32 * w + q0;
+      float row[kBatch][C];
 #pragma unroll
-      for (int m = 0; m < C; ++m) pc[m] = fma((double)row[m], c, pc[m]);
+      for (int e = 0; e < kBatch; ++e)
+#pragma unroll
+        for (int m = 0; m < C; ++m) row[e][m] = pi[(size_t)(i0 + e) * D + C * lane + m];
+      const uint32_t b0 = pl[0][w] >> q0, b1 = pl[1][w] >> q0, b2 = pl[2][w] >> q0;
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e) {
+        const int idx = (int)(((b0 >> e) & 1u) | (((b1 >> e) & 1u) << 1) | (((b2 >> e) & 1u) << 2));
+        const double c = (double)cent[idx];
+#pragma unroll
+        for (int m = 0; m < C; ++m) pc[m] = fma((double)row[e][m], c, pc[m]);
+      }
     }
   }
   double r[C];
@@ -209,6 +207,7 @@ __device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s
   for (int m = 0; m < C; ++m) r[m] = x[m] / nk - pc[m];
 #pragma unroll
   for (int w = 0; w < W; ++w) {
+    res[w] = 0u;
     uint32_t bits = nw[w];
     while (bits) {
       const int j = 32 * w + __ffs(bits) - 1;
@@ -217,13 +216,33 @@ __device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s
       double part = 0.0;
 #pragma unroll
       for (int m = 0; m < C; ++m) part = fma((double)srow[m], r[m], part);
-      const double z = warp_sum_f64(part);
-      if (lane == src) {
-        const uint32_t bit = 1u << (j & 31);
-        sw[w] = z >= 0.0 ? (sw[w] | bit) : (sw[w] & ~bit);
-      }
+      if (warp_sum_f64(part) >= 0.0) res[w] |= 1u << (j & 31);
     }
   }
+}
+
+// The same for the key row of lane `src`: lane src passes its planes, mask,
+// key offset and sign words (sw), and gets the sign words back corrected.
+template <int D = kD>
+__device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s, const float *cent,
+                                                 const void *k, tq_dtype dt, size_t kbase,
+                                                 const uint32_t (&planes)[3][D / 32],
+                                                 const uint32_t (&near)[D / 32], uint32_t (&sw)[D / 32],
+                                                 int src) {
+  constexpr int W = D / 32;
+  const int lane = threadIdx.x & 31;
+  uint32_t pl[3][W], nw[W], res[W];
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+#pragma unroll
+    for (int p = 0; p < 3; ++p) pl[p][w] = __shfl_sync(0xffffffffu, planes[p][w], src);
+    nw[w] = __shfl_sync(0xffffffffu, near[w], src);
+  }
+  const unsigned long long kb = __shfl_sync(0xffffffffu, (unsigned long long)kbase, src);
+  refine_row_f64<D>(pi, s, cent, k, dt, kb, pl, nw, res);
+  if (lane == src)
+#pragma unroll
+    for (int w = 0; w < W; ++w) sw[w] = (sw[w] & ~nw[w]) | res[w];
 }
 
 }  // namespace tq

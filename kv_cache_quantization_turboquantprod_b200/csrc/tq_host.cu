@@ -45,32 +45,47 @@ constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
 // Tests of the timeout path (tq_test_withhold_handoffs).
 std::atomic<int> g_withhold{0};
+// Tests of the sign refinement (tq_test_sign_refine_threshold).
+std::atomic<float> g_refine_z{tq::kSignRefineZ};
 
 // Sticky per-device error word (TQ_ERRF_* bits) that kernels set when they
-// give up on a bounded wait; its device address is looked up once per device.
+// give up on a bounded wait, and the per-device count of QJL sign bits the
+// append kernels re-decided in float64 (tq_test_refine_count); their device
+// addresses are looked up once per device.
 __device__ unsigned int g_error_word;
+__device__ unsigned long long g_refine_count;
 std::atomic<unsigned int *> g_error_addr[kMaxDevices];
-std::mutex g_error_mutex;
+std::atomic<unsigned long long *> g_refine_addr[kMaxDevices];
+std::mutex g_symbol_mutex;
 
-cudaError_t error_word_address(unsigned int **out) {
+template <class T>
+cudaError_t cached_symbol_address(const T &symbol, std::atomic<T *> (&cache)[kMaxDevices], T **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  unsigned int *p = g_error_addr[dev].load(std::memory_order_acquire);
+  T *p = cache[dev].load(std::memory_order_acquire);
   if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(g_error_mutex);
-    p = g_error_addr[dev].load(std::memory_order_acquire);
+    std::lock_guard<std::mutex> lock(g_symbol_mutex);
+    p = cache[dev].load(std::memory_order_acquire);
     if (p == nullptr) {
       void *v = nullptr;
-      e = cudaGetSymbolAddress(&v, g_error_word);
+      e = cudaGetSymbolAddress(&v, symbol);
       if (e != cudaSuccess) return e;
-      p = static_cast<unsigned int *>(v);
-      g_error_addr[dev].store(p, std::memory_order_release);
+      p = static_cast<T *>(v);
+      cache[dev].store(p, std::memory_order_release);
     }
   }
   *out = p;
   return cudaSuccess;
+}
+
+cudaError_t error_word_address(unsigned int **out) {
+  return cached_symbol_address(g_error_word, g_error_addr, out);
+}
+
+cudaError_t refine_count_address(unsigned long long **out) {
+  return cached_symbol_address(g_refine_count, g_refine_addr, out);
 }
 
 // Wait limits and error word of a launch on the current device.
@@ -202,6 +217,8 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
   int sms = 0;
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
   if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
+  a.refine_z = g_refine_z.load(std::memory_order_relaxed);
+  if (refine_count_address(&a.refine_count) != cudaSuccess) return TQ_ERR_CUDA;
   const cudaError_t e = tq::quantize_tc_supported(a) ? tq::launch_quantize_tc(a, sms, (cudaStream_t)stream)
                                                     : tq::launch_quantize_simt(a, sms, (cudaStream_t)stream);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
@@ -389,6 +406,25 @@ tq_status tq_set_wait_limit_ns(unsigned long long ns) {
 
 tq_status tq_test_withhold_handoffs(int on) {
   g_withhold.store(on ? 1 : 0, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
+tq_status tq_test_sign_refine_threshold(double z) {
+  if (!(z >= 0.0)) return TQ_ERR_INVALID_ARGUMENT;
+  g_refine_z.store(z == 0.0 ? tq::kSignRefineZ : (float)z, std::memory_order_relaxed);
+  return TQ_OK;
+}
+
+tq_status tq_test_refine_count(unsigned long long *count, int clear) {
+  if (!count) return TQ_ERR_INVALID_ARGUMENT;
+  unsigned long long *p = nullptr;
+  if (refine_count_address(&p) != cudaSuccess) return TQ_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return TQ_ERR_CUDA;
+  unsigned long long v = 0;
+  if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TQ_ERR_CUDA;
+  *count = v;
+  if (clear && cudaMemset(p, 0, sizeof(v)) != cudaSuccess) return TQ_ERR_CUDA;
+  if (clear && cudaDeviceSynchronize() != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }
 

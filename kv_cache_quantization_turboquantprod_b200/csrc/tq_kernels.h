@@ -57,6 +57,10 @@ struct AppendArgs {
   unsigned int *errors;
   // tests of the timeout path: the loader withholds its operand hand-offs
   int test_withhold;
+  // QJL signs with |(S r)_j| below this are re-decided in float64; the
+  // number re-decided is added to *refine_count
+  float refine_z;
+  unsigned long long *refine_count;
 };
 
 // Split-K plan of one decode call (host-computed, identical in the

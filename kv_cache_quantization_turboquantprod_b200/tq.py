@@ -31,7 +31,8 @@ EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_
            "tq_quantize_append", "tq_decode_workspace_size", "tq_decode_attention",
            "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window",
            "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass",
-           "tq_set_wait_limit_ns", "tq_device_errors", "tq_test_withhold_handoffs")
+           "tq_set_wait_limit_ns", "tq_device_errors", "tq_test_withhold_handoffs",
+           "tq_test_sign_refine_threshold", "tq_test_refine_count")
 ERRF_DECODE_WAIT, ERRF_QUANTIZE_WAIT = 1, 2
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -103,6 +104,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.tq_test_withhold_handoffs.restype = ci
     lib.tq_test_withhold_handoffs.argtypes = [ci]
+    lib.tq_test_sign_refine_threshold.restype = ci
+    lib.tq_test_sign_refine_threshold.argtypes = [ctypes.c_double]
+    lib.tq_test_refine_count.restype = ci
+    lib.tq_test_refine_count.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ci]
     lib.tq_device_errors.restype = ci
     lib.tq_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ci]
     if path is None:
@@ -367,6 +372,20 @@ def tq_test_withhold_handoffs(on: bool) -> None:
     """Tests of the timeout path: make later calls' tensor-core kernels
     withhold one hand-off so that their bounded waits run out."""
     _check("tq_test_withhold_handoffs", load().tq_test_withhold_handoffs(int(bool(on))))
+
+
+def tq_test_sign_refine_threshold(z: float) -> None:
+    """Tests of the float64 sign refinement: later appends re-decide every
+    QJL sign with |(S r)_j| < z in float64 (0: the default, 1e-5)."""
+    _check("tq_test_sign_refine_threshold", load().tq_test_sign_refine_threshold(float(z)))
+
+
+def tq_test_refine_count(clear: bool = False) -> int:
+    """Synchronise the device; QJL sign bits re-decided in float64 by the
+    append kernels since the last reset (reset it when ``clear``)."""
+    n = ctypes.c_ulonglong(0)
+    _check("tq_test_refine_count", load().tq_test_refine_count(ctypes.byref(n), int(bool(clear))))
+    return int(n.value)
 
 
 def tq_device_errors(clear: bool = False) -> int:

@@ -170,6 +170,60 @@ def test_quantize_append_bit_widths_bf16_tiles(kb, vb):
     print(kb, vb, stats)
 
 
+def _tie_values(n_tok, h_kv, d, vb, seed):
+    """bf16 values whose groups put many channels exactly on rounding
+    thresholds z + (k + 1/2) s (ties) and on the levels z + k s: per group
+    the minimum o = m 2^e (m a small integer), the maximum o + L 2^e
+    (L = 2^vb - 1), so zero = o and scale = 2^e exactly, and the other
+    channels drawn from o + 2^e {k + 1/2, k, k + 1/2 +- 1/8}: at most 8
+    significant bits, exact in bf16."""
+    rng = np.random.default_rng(seed)
+    L = (1 << vb) - 1
+    v = np.empty((n_tok, h_kv, d), dtype=np.float64)
+    ks = np.arange(L, dtype=np.float64)
+    cands = np.concatenate([ks + 0.5, ks, ks + 0.5 + 0.125, ks + 0.5 - 0.125, [L]])
+    for t in range(n_tok):
+        for h in range(h_kv):
+            for g in range(d // 32):
+                e = 2.0 ** int(rng.integers(-4, 3))
+                o = e * int(rng.integers(-3, 4))
+                grp = o + e * rng.choice(cands, size=32)
+                grp[rng.integers(0, 32)] = o
+                grp[rng.integers(0, 32)] = o + e * L
+                grp[:] = np.where(grp < o, o, grp)
+                v[t, h, 32 * g:32 * g + 32] = grp
+    vt = torch.from_numpy(v).to(torch.bfloat16)
+    assert np.array_equal(vt.double().numpy(), v), "tie values must be exact in bf16"
+    return vt
+
+
+@pytest.mark.parametrize("vb", [2, 3, 4])
+@pytest.mark.parametrize("T", [128, 8])  # the tensor-core path and the SIMT path
+def test_value_codes_exact_ties(vb, T):
+    """Group-quantized value codes on exact rounding ties (half to even) and
+    exact levels: bit-exact against the oracle with no band, on both append
+    kernels."""
+    import dataclasses
+    wl = dataclasses.replace(workloads.llama8b(), batch=1, key_bits=3, value_bits=vb, capacity=256,
+                             lengths=(T,), name=f"ties{vb}")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, 1, wl.h_kv, 256, zero=True)
+    k = workloads.kv_tokens(wl, 0, 0, T)[0]
+    v = _tie_values(T, wl.h_kv, 128, vb, seed=vb * 100 + T)
+    tq.tq_quantize_append(glayer, cache, k[None].to(DEV).contiguous(), v[None].to(DEV).contiguous(), [0])
+    torch.cuda.synchronize()
+    buf = cache.buffer.cpu().numpy()
+    ties = 0
+    for h in range(wl.h_kv):
+        ke, ve = olayer.encode(k[:, h].float().numpy(), v[:, h].float().numpy())
+        got = spec.read(buf, 0, h, 0, T)
+        assert np.array_equal(got["scale16"], ve["scale16"])
+        assert np.array_equal(got["zero16"], ve["zero16"])
+        assert np.array_equal(got["codes"], ve["codes"]), np.argwhere(got["codes"] != ve["codes"])[:5]
+        ties += int(np.sum(ve["t"] == np.floor(ve["t"]) + 0.5))
+    assert ties > 100, ties
+
+
 # ---------------------------------------------------------------------------
 # decode parity (oracle-encoded cache uploaded to the device)
 # ---------------------------------------------------------------------------

@@ -13,6 +13,13 @@
 * Asymmetric codebooks in the shapes where their operand planes fit in tensor
   memory only once run the SIMT split-K kernel (chosen on the device); parity
   at 16 tiles per CTA in every such shape.
+* Float64 sign refinement under load: with the refinement threshold raised
+  (1e-2 / 1e-3 instead of 1e-5), a large share of the QJL signs is re-decided
+  in float64 -- by the tensor-core kernel's refiner warp (its hand-off rings
+  run full) or the SIMT kernel's last phase.  The library's count of
+  re-decided bits equals the oracle's count of components below the threshold
+  (up to those within 1e-6 of it), and every sign whose oracle component has
+  |z| >= 1e-12 is the oracle's.
 """
 
 import dataclasses
@@ -154,3 +161,46 @@ def test_asymmetric_codebook_long_splits(kb, vb, h_q):
         ref = attention.decode_one_sequence(qf[b, h * G:(h + 1) * G], rec, olayer.pi, olayer.s,
                                             olayer.cent, olayer.group)
         assert pu.row_rel_err(got[b, h * G:(h + 1) * G], ref) <= pu.REL_TOL, (b, h)
+
+
+@pytest.mark.parametrize("batch,T,dtype,thr", [
+    (3, 1024, "bf16", 1e-2),   # tensor-core kernel: 192 tiles, > 1 per CTA, rings full
+    (1, 20, "bf16", 1e-3),     # SIMT kernel
+    (1, 300, "f32", 1e-3),     # SIMT kernel, fp32 input
+])
+def test_sign_refinement_forced(batch, T, dtype, thr):
+    wl = dataclasses.replace(workloads.llama8b(), batch=batch, capacity=1024, lengths=(T,) * batch,
+                             kv_dtype=dtype, name=f"refine{T}")
+    glayer, olayer, spec = _setup(wl)
+    cache = tq.CompressedCache(glayer, batch, wl.h_kv, 1024, zero=True)
+    kv = [workloads.kv_tokens(wl, b, 0, T) for b in range(batch)]
+    k = torch.stack([x[0] for x in kv])
+    v = torch.stack([x[1] for x in kv])
+    tq.tq_test_refine_count(clear=True)
+    tq.tq_test_sign_refine_threshold(thr)
+    try:
+        tq.tq_quantize_append(glayer, cache, k.to(DEV).contiguous(), v.to(DEV).contiguous(), [0] * batch)
+        n = tq.tq_test_refine_count(clear=True)
+    finally:
+        tq.tq_test_sign_refine_threshold(0)
+    assert tq.tq_device_errors() == 0
+    buf = cache.buffer.cpu().numpy()
+    lo = hi = refined_checked = 0
+    slack = 0
+    for b in range(batch):
+        for h in range(wl.h_kv):
+            kk = k[b, :, h].float().numpy()
+            ke, _ = olayer.encode(kk, v[b, :, h].float().numpy())
+            got = spec.read(buf, b, h, 0, T)
+            live = ke["nk"] > 0
+            same = (got["idx"] == ke["idx"]).all(axis=1) & live
+            slack += 128 * int(np.sum(live & ~same))
+            az = np.abs(ke["z"])
+            bad = (got["sign"] != ke["sign"]) & (az >= 1e-12) & same[:, None]
+            assert not bad.any(), (b, h, np.argwhere(bad)[:5], az[bad][:5])
+            refined_checked += int(np.sum((az < thr) & same[:, None]))
+            lo += int(np.sum((az < thr - 1e-6) & live[:, None]))
+            hi += int(np.sum((az < thr + 1e-6) & live[:, None]))
+    assert lo - slack <= n <= hi + slack, (n, lo, hi, slack)
+    assert n > 1000 if thr >= 1e-2 else n > 20, n
+    print(batch, T, dtype, thr, "refined", n, "checked", refined_checked)

@@ -232,3 +232,12 @@ def test_wait_limit_and_error_word_entry_points():
     assert lib.tq_set_wait_limit_ns(5000) == 0
     assert lib.tq_set_wait_limit_ns(0) == 0       # back to the default
     assert lib.tq_device_errors(None, 0) == 1     # null pointer, checked before the device
+
+
+def test_refinement_test_hooks_validate():
+    lib = tq.load()
+    assert lib.tq_test_sign_refine_threshold(-1.0) == 1          # negative: invalid
+    assert lib.tq_test_sign_refine_threshold(float("nan")) == 1
+    assert lib.tq_test_sign_refine_threshold(1e-3) == 0
+    assert lib.tq_test_sign_refine_threshold(0.0) == 0           # back to the default
+    assert lib.tq_test_refine_count(None, 0) == 1                # null pointer, before the device
