@@ -134,7 +134,7 @@ TQ_API tq_status tq_make_codebook(int mse_bits, int d, double *centroids,
 /* Constants of one layer.  All pointers: device, fp32, read-only, owned by
  * the caller, alive for the duration of every call that uses them. */
 typedef struct {
-  int d;          /* head dimension; 128 */
+  int d;          /* head dimension: 64, 128 or 256 */
   int key_bits;   /* 2..4 total key bits: key_bits - 1 Lloyd-Max bits + 1 QJL bit */
   int value_bits; /* 2..4 */
   int group;      /* value quantization group; 32 */
@@ -156,6 +156,15 @@ typedef struct {
                                 ascending (tq_make_codebook(value_bits, d));
                                 NULL for TQ_VALUES_GROUP */
   const float *v_boundaries; /* TQ_VALUES_MSE: [2^value_bits - 1] ascending */
+  const double *s_pit;       /* device, [d][d] row-major float64: W = S Pi^T,
+                                W[j][m] = sum_i S[j][i] Pi[m][i], as
+                                tq_sketch_product writes it from pi and s;
+                                16-byte aligned.  tq_quantize_append re-decides
+                                a QJL sign whose single-precision sketch
+                                component is next to zero (|(S r)_j| < 1e-5) in
+                                float64 as z_j = S_j . u - sum_m c_m W[j][m]
+                                (= S_j . (u - Pi^T c)); required there, unused
+                                by the other calls (may be NULL) */
 } tq_params;
 
 /*
@@ -193,6 +202,15 @@ typedef struct {
   void *data;   /* device, tq_cache_bytes() bytes */
 } tq_cache;
 
+/*
+ * tq_sketch_product -- write W = S Pi^T in float64 (the d x d products of the
+ * float32 Pi and S, each summed in float64 in index order) into s_pit,
+ * device, d * d doubles, 16-byte aligned.  Only p->d, p->pi and p->s are
+ * read.  Asynchronous on `stream`.  TQ_ERR_INVALID_ARGUMENT for null or
+ * misaligned pointers, TQ_ERR_UNSUPPORTED for d.
+ */
+TQ_API tq_status tq_sketch_product(const tq_params *p, double *s_pit, tq_stream_t stream);
+
 /* Bytes per (token, KV head) record R, or 0 for unsupported params. */
 TQ_API size_t tq_record_bytes(const tq_params *p);
 
@@ -213,8 +231,8 @@ TQ_API size_t tq_cache_bytes(const tq_params *p, int batch, int h_kv, int capaci
  *               (<= T); NULL takes all T for every sequence
  * The caller advances its lengths afterwards; the library keeps none.
  * Errors: TQ_ERR_CAPACITY if len + n_new > capacity for any sequence or
- * batch > TQ_MAX_BATCH; TQ_ERR_INVALID_ARGUMENT for null pointers,
- * negative sizes or misalignment; TQ_ERR_UNSUPPORTED for params.
+ * batch > TQ_MAX_BATCH; TQ_ERR_INVALID_ARGUMENT for null pointers (p->s_pit
+ * included), negative sizes or misalignment; TQ_ERR_UNSUPPORTED for params.
  * A zero key stores ||k|| = ||r|| = 0 with all-zero codes and signs.
  * Norms above the fp16 range (65504) are not representable (unsupported).
  */

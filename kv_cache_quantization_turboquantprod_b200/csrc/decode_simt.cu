@@ -49,6 +49,10 @@ __global__ void __launch_bounds__(256) qprep_kernel(DecodeArgs a) {
     acc = warp_sum(acc);
     if (lane == 0) dst[o] = acc;
   }
+  // launched as a dependent of the call's predecessor (reads only the
+  // queries and Pi, S; writes only the workspace): wait for it before
+  // finishing, so the split-K kernel's wait covers both
+  pdl_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -275,8 +279,7 @@ cudaError_t launch_window(const DecodeArgs &a, cudaStream_t stream) {
 template <int D>
 cudaError_t launch_decode_simt_d(const DecodeArgs &a, cudaStream_t stream) {
   const int bhq = a.batch * a.h_q;
-  qprep_kernel<D><<<bhq, 256, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(qprep_kernel<D>, dim3(bhq), dim3(256), 0, stream, a);
   if (e != cudaSuccess) return e;
   e = launch_pdl(decode_splitk_simt_kernel<D>, dim3(a.nsplit, a.h_kv, a.batch), dim3(128), 0, stream, a);
   if (e != cudaSuccess) return e;

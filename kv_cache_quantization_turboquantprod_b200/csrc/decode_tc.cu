@@ -873,9 +873,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // Query blocks: for every (sequence, KV head) the score MMA's B operand
 // (s8, in its shared-memory byte layout) and the score constants, built once
-// per decode call.  A persistent CTA keeps Pi and S in shared memory (rows
-// padded to 129 floats) and rotates the G query heads of each unit:
-// q~ = Pi q, s^ = S q (fp32).  Plane P < n_mse holds 2 a_S q~ for the P-th
+// per decode call.  One CTA per unit rotates its G query heads,
+// q~ = Pi q, s^ = S q (fp32): warp w takes rows 32 w .. 32 w + 31 of [Pi; S],
+// reads each row once (coalesced, from L1/L2) against all G queries and
+// reduces the lanes' partial sums by recursive halving, so lane l ends with
+// row 32 w + l.  Plane P < n_mse holds 2 a_S q~ for the P-th
 // active code-bit subset S (Walsh coefficient a_S of the codebook), the last
 // plane holds 2 s^.  K byte kappa of a plane is operand byte i of TMEM column
 // c = kappa / 4, i.e. coordinate j = 32 (c / 8) + 8 i + (c % 8) with weight
@@ -885,19 +887,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 template <int MB, int VB, int G>
 __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ DecodeArgs a) {
   using C = Cfg<MB, VB, G>;
-  constexpr int kPadQ = kD + 1;
   constexpr int NC = 1 << MB;
   extern __shared__ __align__(16) float qsm[];
-  float *mat = qsm;                         // [256][129]: rows of Pi then S
-  float *qv = mat + 2 * kD * kPadQ;         // [G][128]
-  float *rot = qv + G * kD;                 // [G][2][128]
+  float *rot = qsm;                         // [G][2][128]
   float *red = rot + G * 2 * kD;            // [8 warps][G][4]
   uint8_t *blk = reinterpret_cast<uint8_t *>(red + 8 * G * 4);  // QBLOCK staging
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_trigger();  // the decode kernel may launch now; it waits for this grid
+  // The decode kernel may launch now (it waits for this grid).  This grid
+  // itself is launched as a dependent of the call's predecessor (typically
+  // the quantize-append of the new token): it reads only the queries and the
+  // layer constants, writes only the workspace, and waits for the
+  // predecessor before it finishes, so the decode kernel's wait covers both.
+  pdl_trigger();
 
-  stage_matrix(mat, kPadQ, a.pi, tid, 256);
-  stage_matrix(mat + kD * kPadQ, kPadQ, a.s, tid, 256);
   for (int i = tid; i < C::QBLOCK / 4; i += 256) reinterpret_cast<uint32_t *>(blk)[i] = 0u;
   // Walsh coefficients of the codebook, idx paired with its complement so
   // that a symmetric codebook gives exact zeros for the even subsets
@@ -950,23 +952,49 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   const int units = a.batch * a.h_kv;
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int b = u / a.h_kv, h = u % a.h_kv;
-    for (int i = tid; i < G * kD; i += 256)
-      qv[i] = load_elem(a.q, a.q_dtype, qrow_offset(a, b, h * G + i / kD) + i % kD);
-    __syncthreads();
-    {  // thread o rotates row o of [Pi; S] against the G queries
-      const int o = tid;
-      float acc[G];
+    {  // warp w: rows 32 w .. 32 w + 31 of [Pi; S] against the G queries
+      const float *mrows = (warp < 4 ? a.pi : a.s) + (size_t)(32 * (warp & 3)) * kD + 4 * lane;
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = 0.f;
-      for (int i = 0; i < kD; ++i) {
-        const float m = mat[o * kPadQ + i];
+      for (int g0 = 0; g0 < G; g0 += 4) {
+        constexpr int GB = G < 4 ? G : 4;  // heads per pass (register budget)
+        float qx[GB][4];
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = fmaf(m, qv[g * kD + i], acc[g]);
-      }
+        for (int gi = 0; gi < GB; ++gi)
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        rot[g * 2 * kD + o] = acc[g];
-        if (fallback) a.qrot[((size_t)b * a.h_q + h * G + g) * 2 * kD + o] = acc[g];
+          for (int e = 0; e < 4; ++e)
+            qx[gi][e] = load_elem(a.q, a.q_dtype, qrow_offset(a, b, h * G + g0 + gi) + 4 * lane + e);
+        float p[GB][32];
+#pragma unroll
+        for (int r0 = 0; r0 < 32; r0 += 8) {
+          float4 w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = *reinterpret_cast<const float4 *>(mrows + (size_t)(r0 + e) * kD);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int gi = 0; gi < GB; ++gi)
+              p[gi][r0 + e] = fmaf(w[e].w, qx[gi][3], fmaf(w[e].z, qx[gi][2],
+                                   fmaf(w[e].y, qx[gi][1], w[e].x * qx[gi][0])));
+        }
+        // recursive halving: lane l ends with row 32 w + l
+#pragma unroll
+        for (int sft = 16; sft >= 1; sft >>= 1) {
+          const bool upper = (lane & sft) != 0;
+#pragma unroll
+          for (int q = 0; q < sft; ++q)
+#pragma unroll
+            for (int gi = 0; gi < GB; ++gi) {
+              const float send = upper ? p[gi][q] : p[gi][q + sft];
+              const float keep = upper ? p[gi][q + sft] : p[gi][q];
+              p[gi][q] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+            }
+        }
+        const int o = 32 * warp + lane;  // row of [Pi; S]
+#pragma unroll
+        for (int gi = 0; gi < GB; ++gi) {
+          rot[(g0 + gi) * 2 * kD + o] = p[gi][0];
+          if (fallback) a.qrot[((size_t)b * a.h_q + h * G + g0 + gi) * 2 * kD + o] = p[gi][0];
+        }
       }
     }
     __syncthreads();
@@ -1040,12 +1068,13 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     for (int i = tid; i < C::QBLOCK / 16; i += 256) dst[i] = src[i];
     __syncthreads();
   }
+  pdl_wait();
 }
 
 template <int MB, int VB, int G>
 size_t qblock_smem_bytes() {
   using C = Cfg<MB, VB, G>;
-  return sizeof(float) * (2 * kD * (kD + 1) + G * kD + G * 2 * kD + 8 * G * 4) + C::QBLOCK;
+  return sizeof(float) * (G * 2 * kD + 8 * G * 4) + C::QBLOCK;
 }
 
 template <int MB, int VB, int G>
@@ -1062,9 +1091,8 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
                            (int)qsmem);
   if (e != cudaSuccess) return e;
   const int units = a.batch * a.h_kv;
-  const int qgrid = units < a.num_sms ? units : a.num_sms;
-  qblock_kernel<MB, VB, G><<<qgrid, 256, qsmem, stream>>>(a);
-  e = cudaGetLastError();
+  const int qgrid = units;  // one unit per CTA
+  e = launch_pdl(qblock_kernel<MB, VB, G>, dim3(qgrid), dim3(256), qsmem, stream, a);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_tc_kernel<MB, VB, G>, dim3(a.h_kv, a.batch, a.nsplit), dim3(kTcThreads), smem,
                     stream, a);

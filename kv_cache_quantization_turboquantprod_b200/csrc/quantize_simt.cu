@@ -12,6 +12,7 @@
 // TurboQuant-MSE values ("03. Results & Benchmarks", "At a Glance ->
 // Compression"): the value's norm and the Lloyd-Max cells of Pi v / ||v||.
 //
+// This form serves large appends (small ones take quantize_warp.cu).
 // A persistent CTA encodes kNV vectors per pass: three D x D mat-vecs per
 // vector (Pi u, Pi^T c, S r; and Pi w for MSE values) in fp32 with a fixed
 // accumulation order per output.  Up to D = 128, Pi and S sit in shared
@@ -20,6 +21,8 @@
 // sketch component within 1e-5 of zero has its sign decided again in float64.
 #include <stddef.h>
 
+#include "quantize_common.cuh"
+#include "sm100.cuh"
 #include "tq_common.cuh"
 #include "tq_kernels.h"
 
@@ -52,19 +55,6 @@ struct QuantSmem {
   float vbnd[16];
 };
 
-__device__ __forceinline__ void vec_coords(const AppendArgs &a, long long id, int &b,
-                                           int &t, int &h, bool &valid) {
-  const long long per_b = (long long)a.T * a.h_kv;
-  const long long total = (long long)a.batch * per_b;
-  valid = id < total;
-  if (!valid) { b = t = h = 0; return; }
-  b = (int)(id / per_b);
-  long long rem = id - (long long)b * per_b;
-  t = (int)(rem / a.h_kv);
-  h = (int)(rem - (long long)t * a.h_kv);
-  valid = t < a.nnew[b];
-}
-
 // Element (i, j) of a row-major D x D matrix: shared memory (padded rows) up
 // to D = 128, global memory above.
 template <int kNV, int D>
@@ -89,6 +79,9 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
   const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode, D);
   const int ncent = 1 << L.mb;
   const int nvcent = 1 << L.vb;
+  // a decode call's query kernel may start now: it reads none of this
+  // kernel's output and waits for this grid before it finishes
+  sm100::pdl_trigger();
 
   if constexpr (SM::kMatsInSmem) {
     stage_matrix<D>(S.pi, SM::kPad, a.pi, tid, kThreads);
@@ -145,51 +138,8 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
         if (lane == 0) S.nv[vi] = nv;
       } else if (valid) {
         const int pos = a.lens[b] + t;
-        uint8_t *tile = tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile);
-        const int slot = pos % kTile;
-        // group m = channels 32m .. 32m + 31: one element per lane
-#pragma unroll
-        for (int m = 0; m < C; ++m) {
-          const float vv = load_elem(a.v, a.dtype, base + lane + 32 * m);
-          const float mn = warp_min(vv);
-          const float mx = warp_max(vv);
-          const __half zero16 = __float2half_rn(mn);
-          // the scale from the exact quotient (float64, one rounding to fp16)
-          const __half scale16 = __double2half(((double)mx - (double)mn) / (double)vlevels);
-          const float z32 = __half2float(zero16);
-          const float sc32 = __half2float(scale16);
-          int code = 0;
-          if (sc32 != 0.f) {
-            // rint of the exact quotient: single precision decides unless the
-            // quotient is next to a half-integer, then float64 does
-            const float t32 = __fdiv_rn(__fsub_rn(vv, z32), sc32);
-            float tq = rintf(t32);
-            if (fabsf(t32 - tq) > 0.5f - 1e-5f) tq = (float)rint(((double)vv - (double)z32) / (double)sc32);
-            tq = fminf(fmaxf(tq, 0.f), vlevels);
-            code = (int)tq;
-          }
-          if (L.vb == 2) {
-            // packed codes: channel 4i + m' of a row in bits 2m', 2m'+1 of byte i
-            const unsigned lo = __ballot_sync(0xffffffffu, code & 1);
-            const unsigned hi = __ballot_sync(0xffffffffu, (code >> 1) & 1);
-            if (lane == 0) {
-              uint32_t *dst = reinterpret_cast<uint32_t *>(tile + L.vplanes + slot * L.packed_row_bytes + 8 * m);
-              dst[0] = spread_bits16(lo & 0xFFFFu) | (spread_bits16(hi & 0xFFFFu) << 1);
-              dst[1] = spread_bits16(lo >> 16) | (spread_bits16(hi >> 16) << 1);
-            }
-          } else {
-            for (int p = 0; p < L.vb; ++p) {
-              const unsigned word = __ballot_sync(0xffffffffu, (code >> p) & 1);
-              if (lane == 0)
-                *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * L.plane_bytes + slot * L.row_bytes + 4 * m) =
-                    word;
-            }
-          }
-          if (lane == 0) {
-            __half2 sz = __halves2half2(scale16, zero16);
-            *reinterpret_cast<__half2 *>(tile + L.vsz + (slot * L.groups + m) * 4) = sz;
-          }
-        }
+        quantize_value_groups<D>(a, L, tile_ptr(a.data, L, a.h_kv, a.ntiles, b, h, pos / kTile), pos % kTile,
+                                 base, vlevels);
       }
     }
     __syncthreads();
@@ -379,7 +329,7 @@ quantize_append_simt_kernel(const __grid_constant__ AppendArgs a) {
         sw[w] = *reinterpret_cast<const uint32_t *>(tile + L.signs + slot * L.row_bytes + 4 * w);
       }
       const size_t kbase = (((size_t)b * a.T + t) * a.h_kv + h) * D;
-      refine_signs_f64<D>(a.pi, a.s, S.cent, a.k, a.dtype, kbase, planes, nw, sw, 0);
+      refine_signs_f64<D>(a.s, a.s_pit, S.cent, a.k, a.dtype, kbase, planes, nw, sw, 0);
       if (lane == 0) {
         int nbits = 0;
 #pragma unroll
@@ -411,20 +361,39 @@ cudaError_t launch_simt_nv(const AppendArgs &a, int num_sms, cudaStream_t stream
   return cudaGetLastError();
 }
 
-// vectors per pass: 16 for large appends; for small ones (decode steps) the
-// fewest one pass of 256 threads covers (kThreads / D), so a 1-token append
-// over B x H_kv heads still spreads over many SMs
+// 16 vectors per pass (small appends take the warp-per-vector kernel)
 template <int D>
 cudaError_t launch_simt_d(const AppendArgs &a, int num_sms, cudaStream_t stream) {
-  constexpr int kSmall = kThreads / D;
-  const long long total = (long long)a.batch * a.T * a.h_kv;
-  return total <= (long long)kSmall * num_sms ? launch_simt_nv<kSmall, D>(a, num_sms, stream)
-                                              : launch_simt_nv<16, D>(a, num_sms, stream);
+  return launch_simt_nv<16, D>(a, num_sms, stream);
 }
 
 }  // namespace
 
+// W = S Pi^T in float64: one thread per entry (j, m), the d products of the
+// float32 entries summed in float64 in index order.  A one-off per layer.
+__global__ void sketch_product_kernel(const float *__restrict__ pi, const float *__restrict__ s, int d,
+                                      double *__restrict__ out) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= d * d) return;
+  const int j = e / d, m = e - j * d;
+  const float *srow = s + (size_t)j * d, *prow = pi + (size_t)m * d;
+  double acc = 0.0;
+  for (int i = 0; i < d; ++i) acc = fma((double)srow[i], (double)prow[i], acc);
+  out[e] = acc;
+}
+
+cudaError_t launch_sketch_product(const float *pi, const float *s, int d, double *out, cudaStream_t stream) {
+  const int n = d * d;
+  sketch_product_kernel<<<(n + 255) / 256, 256, 0, stream>>>(pi, s, d, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_simt(const AppendArgs &a, int num_sms, cudaStream_t stream) {
+  // Up to eight vector slots per SM (a decode step appends one token per
+  // sequence and head) the warp-per-vector kernel, which stages nothing, is
+  // faster than staging Pi and S in every CTA.
+  const long long total = (long long)a.batch * a.T * a.h_kv;
+  if (total <= 8LL * num_sms) return launch_quantize_warp(a, num_sms, stream);
   switch (a.d) {
     case 64: return launch_simt_d<64>(a, num_sms, stream);
     case 128: return launch_simt_d<128>(a, num_sms, stream);

@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   QtSmem &S = *reinterpret_cast<QtSmem *>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode);
+  // a decode call's query kernel may start now: it reads none of this
+  // kernel's output and waits for this grid before it finishes
+  pdl_trigger();
   constexpr int ncent = 1 << MB;
   const int nlocal = a.total_tiles > (int)blockIdx.x
                          ? (a.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
@@ -631,7 +634,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           }
           const unsigned long long kb = q.kbase;
           uint32_t *words = reinterpret_cast<uint32_t *>(q.signs);
-          refine_row_f64<kD, 32>(a.pi, a.s, S.cent, a.k, a.dtype, kb, pl, nw, res);
+          refine_row_f64<kD>(a.s, a.s_pit, S.cent, a.k, a.dtype, kb, pl, nw, res);
           uint32_t mn = 0u, mr = 0u;  // lane w < 4 patches word w
 #pragma unroll
           for (int w = 0; w < 4; ++w)

@@ -22,6 +22,7 @@
 // quotient, redone in float64 where it sits within 1e-5 of a half-integer.
 // The records' value sections (codes, scale, zero) are written in place; the
 // key sections are the tensor-core kernel's.  Head dim 128, bf16 input.
+#include "sm100.cuh"
 #include "tq_common.cuh"
 #include "tq_kernels.h"
 
@@ -74,6 +75,7 @@ __device__ __forceinline__ uint32_t codes2_packed(const float (&x)[16], __half z
 template <int VB>
 __global__ void __launch_bounds__(kVqThreads) value_quant_kernel(const __grid_constant__ AppendArgs a) {
   const TileLayout L = TileLayout::make(a.key_bits, VB, a.value_mode, kD);
+  sm100::pdl_trigger();  // see the tensor-core append kernel
   const int lane = threadIdx.x & 31;
   const int qv = lane >> 3, ql = lane & 7;  // vector of the round, lane within it
   const long long total = (long long)a.batch * a.T * a.h_kv;

@@ -157,20 +157,19 @@ __device__ __forceinline__ double warp_sum_f64(double x) {
 // dim D (all 32 lanes call it together with the same arguments).  The row's
 // key starts at element kbase of k; pl holds its Lloyd-Max code bit-planes
 // (three planes of D/32 32-coordinate words, planes beyond the code width
-// zero) and near the mask of coordinates to re-decide.  In float64: ||k||,
-// u = k / ||k||, r = u - Pi^T c (c = centroids of the stored codes) and, for
-// every masked j, (S r)_j; bit j of the returned words is [(S r)_j >= 0]
-// (zero outside the mask).  Pi and S are read row-major from global memory
-// (D/32 coordinates per lane), Pi in batches of rows whose loads (a lane's
-// kFloatsInFlight floats) are all in flight before any is used.
-template <int D = kD, int kFloatsInFlight = 64>
-__device__ __forceinline__ void refine_row_f64(const float *pi, const float *s, const float *cent,
+// zero) and nw the mask of coordinates to re-decide.  In float64: ||k||,
+// u = k / ||k|| and, for every masked j,
+//   z_j = S_j . u - sum_m c_m W[j][m]     (W = S Pi^T, c = centroids of the codes)
+// which is (S (u - Pi^T c))_j; bit j of the returned words is [z_j >= 0]
+// (zero outside the mask).  A lane holds D/32 consecutive coordinates; S and
+// W rows are read from global memory.
+template <int D = kD>
+__device__ __forceinline__ void refine_row_f64(const float *s, const double *s_pit, const float *cent,
                                                const void *k, tq_dtype dt, size_t kbase,
                                                const uint32_t (&pl)[3][D / 32], const uint32_t (&nw)[D / 32],
                                                uint32_t (&res)[D / 32]) {
   constexpr int W = D / 32;   // 32-coordinate words of a row
   constexpr int C = D / 32;   // coordinates per lane
-  constexpr int kBatch = kFloatsInFlight / C;  // rows of Pi per batch (<= 32)
   const int lane = threadIdx.x & 31;
   double x[C], ss = 0.0;
 #pragma unroll
@@ -179,32 +178,22 @@ __device__ __forceinline__ void refine_row_f64(const float *pi, const float *s, 
     ss = fma(x[m], x[m], ss);
   }
   const double nk = sqrt(warp_sum_f64(ss));
-  double pc[C];
+  // centroids of this lane's coordinates C lane .. C lane + C - 1
+  const int wi = (C * lane) >> 5, sh = (C * lane) & 31;
+  uint32_t b0 = 0u, b1 = 0u, b2 = 0u;
 #pragma unroll
-  for (int m = 0; m < C; ++m) pc[m] = 0.0;
-#pragma unroll
-  for (int w = 0; w < W; ++w) {
-#pragma unroll 1
-    for (int q0 = 0; q0 < 32; q0 += kBatch) {
-      const int i0 = 32 * w + q0;
-      float row[kBatch][C];
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e)
-#pragma unroll
-        for (int m = 0; m < C; ++m) row[e][m] = pi[(size_t)(i0 + e) * D + C * lane + m];
-      const uint32_t b0 = pl[0][w] >> q0, b1 = pl[1][w] >> q0, b2 = pl[2][w] >> q0;
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e) {
-        const int idx = (int)(((b0 >> e) & 1u) | (((b1 >> e) & 1u) << 1) | (((b2 >> e) & 1u) << 2));
-        const double c = (double)cent[idx];
-#pragma unroll
-        for (int m = 0; m < C; ++m) pc[m] = fma((double)row[e][m], c, pc[m]);
-      }
+  for (int w = 0; w < W; ++w)
+    if (w == wi) {
+      b0 = pl[0][w] >> sh;
+      b1 = pl[1][w] >> sh;
+      b2 = pl[2][w] >> sh;
     }
-  }
-  double r[C];
+  double u[C], c[C];
 #pragma unroll
-  for (int m = 0; m < C; ++m) r[m] = x[m] / nk - pc[m];
+  for (int m = 0; m < C; ++m) {
+    u[m] = x[m] / nk;
+    c[m] = (double)cent[((b0 >> m) & 1u) | (((b1 >> m) & 1u) << 1) | (((b2 >> m) & 1u) << 2)];
+  }
 #pragma unroll
   for (int w = 0; w < W; ++w) {
     res[w] = 0u;
@@ -213,9 +202,12 @@ __device__ __forceinline__ void refine_row_f64(const float *pi, const float *s, 
       const int j = 32 * w + __ffs(bits) - 1;
       bits &= bits - 1;
       const float *srow = s + (size_t)j * D + C * lane;
+      const double *wrow = s_pit + (size_t)j * D + C * lane;
       double part = 0.0;
 #pragma unroll
-      for (int m = 0; m < C; ++m) part = fma((double)srow[m], r[m], part);
+      for (int m = 0; m < C; ++m) part = fma((double)srow[m], u[m], part);
+#pragma unroll
+      for (int m = 0; m < C; ++m) part = fma(-wrow[m], c[m], part);
       if (warp_sum_f64(part) >= 0.0) res[w] |= 1u << (j & 31);
     }
   }
@@ -224,7 +216,7 @@ __device__ __forceinline__ void refine_row_f64(const float *pi, const float *s, 
 // The same for the key row of lane `src`: lane src passes its planes, mask,
 // key offset and sign words (sw), and gets the sign words back corrected.
 template <int D = kD>
-__device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s, const float *cent,
+__device__ __forceinline__ void refine_signs_f64(const float *s, const double *s_pit, const float *cent,
                                                  const void *k, tq_dtype dt, size_t kbase,
                                                  const uint32_t (&planes)[3][D / 32],
                                                  const uint32_t (&near)[D / 32], uint32_t (&sw)[D / 32],
@@ -239,7 +231,7 @@ __device__ __forceinline__ void refine_signs_f64(const float *pi, const float *s
     nw[w] = __shfl_sync(0xffffffffu, near[w], src);
   }
   const unsigned long long kb = __shfl_sync(0xffffffffu, (unsigned long long)kbase, src);
-  refine_row_f64<D>(pi, s, cent, k, dt, kb, pl, nw, res);
+  refine_row_f64<D>(s, s_pit, cent, k, dt, kb, pl, nw, res);
   if (lane == src)
 #pragma unroll
     for (int w = 0; w < W; ++w) sw[w] = (sw[w] & ~nw[w]) | res[w];

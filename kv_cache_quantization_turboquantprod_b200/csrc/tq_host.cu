@@ -175,6 +175,14 @@ tq_status tq_make_codebook(int mse_bits, int d, double *centroids, double *bound
   return TQ_OK;
 }
 
+tq_status tq_sketch_product(const tq_params *p, double *s_pit, tq_stream_t stream) {
+  if (!p || !s_pit || !aligned(s_pit, 16)) return TQ_ERR_INVALID_ARGUMENT;
+  if (p->d != 64 && p->d != 128 && p->d != 256) return TQ_ERR_UNSUPPORTED;
+  if (!p->pi || !p->s || !aligned(p->pi, 16) || !aligned(p->s, 16)) return TQ_ERR_INVALID_ARGUMENT;
+  return tq::launch_sketch_product(p->pi, p->s, p->d, s_pit, (cudaStream_t)stream) == cudaSuccess ? TQ_OK
+                                                                                               : TQ_ERR_CUDA;
+}
+
 size_t tq_record_bytes(const tq_params *p) {
   if (check_params(p) != TQ_OK) return 0;
   return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode, p->d).record_bytes();
@@ -198,6 +206,7 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
   if (c->batch > TQ_MAX_BATCH) return TQ_ERR_CAPACITY;
   if (T == 0) return TQ_OK;
   if (!k || !v || !aligned(k, 16) || !aligned(v, 16)) return TQ_ERR_INVALID_ARGUMENT;
+  if (!p->s_pit || !aligned(p->s_pit, 16)) return TQ_ERR_INVALID_ARGUMENT;
   tq::AppendArgs a;
   memset(&a, 0, sizeof(a));
   for (int b = 0; b < c->batch; ++b) {
@@ -218,6 +227,7 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
   if (current_sm_count(&sms) != cudaSuccess) return TQ_ERR_CUDA;
   if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
   a.refine_z = g_refine_z.load(std::memory_order_relaxed);
+  a.s_pit = p->s_pit;
   if (refine_count_address(&a.refine_count) != cudaSuccess) return TQ_ERR_CUDA;
   const cudaError_t e = tq::quantize_tc_supported(a) ? tq::launch_quantize_tc(a, sms, (cudaStream_t)stream)
                                                     : tq::launch_quantize_simt(a, sms, (cudaStream_t)stream);

@@ -57,9 +57,11 @@ struct AppendArgs {
   unsigned int *errors;
   // tests of the timeout path: the loader withholds its operand hand-offs
   int test_withhold;
-  // QJL signs with |(S r)_j| below this are re-decided in float64; the
-  // number re-decided is added to *refine_count
+  // QJL signs with |(S r)_j| below this are re-decided in float64 (with
+  // s_pit = S Pi^T in float64); the number re-decided is added to
+  // *refine_count
   float refine_z;
+  const double *s_pit;
   unsigned long long *refine_count;
 };
 
@@ -151,6 +153,10 @@ cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream);
 // Group quantization of values alone (bandwidth-bound), run by the
 // tensor-core append path before its key kernel.
 cudaError_t launch_value_quant(const AppendArgs &a, int num_sms, cudaStream_t stream);
+// Warp-per-vector append for small appends (decode steps).
+cudaError_t launch_quantize_warp(const AppendArgs &a, int num_sms, cudaStream_t stream);
+// W = S Pi^T in float64 (d x d, row-major by sketch row j).
+cudaError_t launch_sketch_product(const float *pi, const float *s, int d, double *out, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 // Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
 bool decode_tc_supported(int key_bits, int value_bits, int gqa, int value_mode = 0, int d = 128);

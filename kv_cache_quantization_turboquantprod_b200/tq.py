@@ -32,7 +32,7 @@ EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_
            "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window",
            "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass",
            "tq_set_wait_limit_ns", "tq_device_errors", "tq_test_withhold_handoffs",
-           "tq_test_sign_refine_threshold", "tq_test_refine_count")
+           "tq_test_sign_refine_threshold", "tq_test_refine_count", "tq_sketch_product")
 ERRF_DECODE_WAIT, ERRF_QUANTIZE_WAIT = 1, 2
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -49,7 +49,7 @@ class Params(ctypes.Structure):
                 ("pi", ctypes.c_void_p), ("s", ctypes.c_void_p),
                 ("centroids", ctypes.c_void_p), ("boundaries", ctypes.c_void_p),
                 ("value_mode", ctypes.c_int), ("v_centroids", ctypes.c_void_p),
-                ("v_boundaries", ctypes.c_void_p)]
+                ("v_boundaries", ctypes.c_void_p), ("s_pit", ctypes.c_void_p)]
 
 
 class Cache(ctypes.Structure):
@@ -79,6 +79,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
                                      ctypes.POINTER(ctypes.c_double)]
     lib.tq_record_bytes.restype = sz
     lib.tq_record_bytes.argtypes = [P]
+    lib.tq_sketch_product.restype = ci
+    lib.tq_sketch_product.argtypes = [P, vp, vp]
     lib.tq_cache_bytes.restype = sz
     lib.tq_cache_bytes.argtypes = [P, ci, ci, ci]
     lib.tq_quantize_append.restype = ci
@@ -207,9 +209,14 @@ class Layer:
             self.v_boundaries = torch.tensor(vbnd, dtype=torch.float32, device=device)
             self.value_codebook = (vcent, vbnd)
             vc_ptr, vb_ptr = self.v_centroids.data_ptr(), self.v_boundaries.data_ptr()
+        # W = S Pi^T in float64, for the append kernels' sign refinement
+        self.s_pit = torch.empty((d, d), dtype=torch.float64, device=device)
         self.params = Params(d, key_bits, value_bits, group, self.pi.data_ptr(),
                              self.s.data_ptr(), self.centroids.data_ptr(),
-                             self.boundaries.data_ptr(), mode, vc_ptr, vb_ptr)
+                             self.boundaries.data_ptr(), mode, vc_ptr, vb_ptr,
+                             self.s_pit.data_ptr())
+        if self.s_pit.is_cuda:
+            tq_sketch_product(self)
 
     @property
     def d(self):
@@ -232,6 +239,12 @@ class CompressedCache:
         self.buffer = alloc(n, dtype=torch.uint8, device=device)
         self.cache = Cache(batch, h_kv, capacity, self.buffer.data_ptr())
         self.batch, self.h_kv, self.capacity = batch, h_kv, capacity
+
+
+def tq_sketch_product(layer: Layer, stream=None) -> None:
+    """Write W = S Pi^T (float64) into layer.s_pit from the layer's Pi and S."""
+    st = load().tq_sketch_product(ctypes.byref(layer.params), layer.s_pit.data_ptr(), _stream(stream))
+    _check("tq_sketch_product", st)
 
 
 def tq_record_bytes(layer: Layer) -> int:

@@ -170,6 +170,20 @@ def test_quantize_append_bit_widths_bf16_tiles(kb, vb):
     print(kb, vb, stats)
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_sketch_product_is_float64_s_pi_t(d):
+    """W = S Pi^T (the append kernels' float64 refinement reads it) equals
+    the float64 product of the float32 matrices to a few ulps."""
+    pi, s = workloads.rotation_and_sketch(d, 77)
+    pi32, s32 = pi.astype(np.float32), s.astype(np.float32)
+    layer = pu.gpu_layer(pi32, s32, 3, 2)
+    torch.cuda.synchronize()
+    got = layer.s_pit.cpu().numpy()
+    ref = s32.astype(np.float64) @ pi32.astype(np.float64).T
+    assert got.shape == (d, d)
+    assert np.max(np.abs(got - ref)) <= 1e-13 * max(1.0, np.max(np.abs(ref)))
+
+
 def _tie_values(n_tok, h_kv, d, vb, seed):
     """bf16 values whose groups put many channels exactly on rounding
     thresholds z + (k + 1/2) s (ties) and on the levels z + k s: per group

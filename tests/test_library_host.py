@@ -62,8 +62,8 @@ def test_status_strings():
         assert tq.tq_status_string(code) == name
 
 
-def _params(d=128, kb=3, vb=2, g=32, ptr=256, mode=0, vptr=None):
-    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr, mode, vptr, vptr)
+def _params(d=128, kb=3, vb=2, g=32, ptr=256, mode=0, vptr=None, wptr=256):
+    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr, mode, vptr, vptr, wptr)
 
 
 def test_record_and_cache_bytes():
@@ -121,6 +121,19 @@ def test_append_validation_before_launch():
     assert f(ctypes.byref(P), ctypes.byref(Cbig), k, v, 1, 4, big, None, None) == 3
     # T = 0 is a no-op that succeeds without launching
     assert f(ctypes.byref(P), ctypes.byref(C), None, None, 1, 0, lens, None, None) == 0
+    # the float64 product S Pi^T is required, 16-byte aligned
+    assert f(ctypes.byref(_params(wptr=None)), ctypes.byref(C), k, v, 1, 4, lens, None, None) == 1
+    assert f(ctypes.byref(_params(wptr=264)), ctypes.byref(C), k, v, 1, 4, lens, None, None) == 1
+
+
+def test_sketch_product_validation():
+    lib = tq.load()
+    f = lib.tq_sketch_product
+    assert f(None, 1 << 20, None) == 1
+    assert f(ctypes.byref(_params()), None, None) == 1
+    assert f(ctypes.byref(_params()), (1 << 20) + 8, None) == 1         # output alignment
+    assert f(ctypes.byref(_params(d=96)), 1 << 20, None) == 2
+    assert f(ctypes.byref(_params(ptr=260)), 1 << 20, None) == 1        # Pi / S alignment
 
 
 def test_decode_validation_before_launch():
