@@ -873,11 +873,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // Query blocks: for every (sequence, KV head) the score MMA's B operand
 // (s8, in its shared-memory byte layout) and the score constants, built once
-// per decode call.  One CTA per unit rotates its G query heads,
-// q~ = Pi q, s^ = S q (fp32): warp w takes rows 32 w .. 32 w + 31 of [Pi; S],
-// reads each row once (coalesced, from L1/L2) against all G queries and
-// reduces the lanes' partial sums by recursive halving, so lane l ends with
-// row 32 w + l.  Plane P < n_mse holds 2 a_S q~ for the P-th
+// per decode call.  A CTA copies Pi and S into shared memory (16-byte
+// asynchronous copies, all in flight at once) and rotates the G query heads
+// of each of its units, q~ = Pi q, s^ = S q (fp32): warp w takes rows
+// 32 w .. 32 w + 31 of [Pi; S], reads each row once against all G queries
+// and reduces the lanes' partial sums by recursive halving, so lane l ends
+// with row 32 w + l.  Plane P < n_mse holds 2 a_S q~ for the P-th
 // active code-bit subset S (Walsh coefficient a_S of the codebook), the last
 // plane holds 2 s^.  K byte kappa of a plane is operand byte i of TMEM column
 // c = kappa / 4, i.e. coordinate j = 32 (c / 8) + 8 i + (c % 8) with weight
@@ -889,7 +890,8 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   using C = Cfg<MB, VB, G>;
   constexpr int NC = 1 << MB;
   extern __shared__ __align__(16) float qsm[];
-  float *rot = qsm;                         // [G][2][128]
+  float *mats = qsm;                        // [2][128][128]: Pi, S
+  float *rot = mats + 2 * kD * kD;          // [G][2][128]
   float *red = rot + G * 2 * kD;            // [8 warps][G][4]
   uint8_t *blk = reinterpret_cast<uint8_t *>(red + 8 * G * 4);  // QBLOCK staging
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -900,6 +902,10 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   // predecessor before it finishes, so the decode kernel's wait covers both.
   pdl_trigger();
 
+  for (int i = tid; i < kD * kD / 4; i += 256) {
+    cp_async16(mats + 4 * i, a.pi + 4 * i);
+    cp_async16(mats + kD * kD + 4 * i, a.s + 4 * i);
+  }
   for (int i = tid; i < C::QBLOCK / 4; i += 256) reinterpret_cast<uint32_t *>(blk)[i] = 0u;
   // Walsh coefficients of the codebook, idx paired with its complement so
   // that a symmetric codebook gives exact zeros for the even subsets
@@ -947,13 +953,14 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     a.status[1] = fallback ? 1 : 0;
   }
   QConst *qc = reinterpret_cast<QConst *>(blk + C::BQ_BYTES);
+  cp_async_wait_all();
   __syncthreads();
 
   const int units = a.batch * a.h_kv;
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int b = u / a.h_kv, h = u % a.h_kv;
     {  // warp w: rows 32 w .. 32 w + 31 of [Pi; S] against the G queries
-      const float *mrows = (warp < 4 ? a.pi : a.s) + (size_t)(32 * (warp & 3)) * kD + 4 * lane;
+      const float *mrows = mats + (warp < 4 ? 0 : kD * kD) + 32 * (warp & 3) * kD + 4 * lane;
 #pragma unroll
       for (int g0 = 0; g0 < G; g0 += 4) {
         constexpr int GB = G < 4 ? G : 4;  // heads per pass (register budget)
@@ -1074,7 +1081,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
 template <int MB, int VB, int G>
 size_t qblock_smem_bytes() {
   using C = Cfg<MB, VB, G>;
-  return sizeof(float) * (G * 2 * kD + 8 * G * 4) + C::QBLOCK;
+  return sizeof(float) * (2 * kD * kD + G * 2 * kD + 8 * G * 4) + C::QBLOCK;
 }
 
 template <int MB, int VB, int G>
@@ -1091,7 +1098,7 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
                            (int)qsmem);
   if (e != cudaSuccess) return e;
   const int units = a.batch * a.h_kv;
-  const int qgrid = units;  // one unit per CTA
+  const int qgrid = units < a.num_sms ? units : a.num_sms;
   e = launch_pdl(qblock_kernel<MB, VB, G>, dim3(qgrid), dim3(256), qsmem, stream, a);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_tc_kernel<MB, VB, G>, dim3(a.h_kv, a.batch, a.nsplit), dim3(kTcThreads), smem,

@@ -31,13 +31,14 @@ __device__ __forceinline__ void vec_coords(const AppendArgs &a, long long id, in
 // (single precision decides unless the quotient is next to a half-integer,
 // then float64 does).  Writes the record's value codes and (scale, zero) at
 // token slot `slot` of `tile`; the value starts at element `base` of a.v.
+// Groups m0, m0 + mstep, ... (all of them by default).
 template <int D>
 __device__ __forceinline__ void quantize_value_groups(const AppendArgs &a, const TileLayout &L, uint8_t *tile,
-                                                      int slot, size_t base, float vlevels) {
+                                                      int slot, size_t base, float vlevels, int m0 = 0,
+                                                      int mstep = 1) {
   constexpr int C = D / 32;
   const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int m = 0; m < C; ++m) {
+  for (int m = m0; m < C; m += mstep) {
     const float vv = load_elem(a.v, a.dtype, base + lane + 32 * m);
     const float mn = warp_min(vv);
     const float mx = warp_max(vv);

@@ -65,13 +65,14 @@ __host__ __device__ constexpr int blk_off(int row, int col) {
   return (col >> 3) * 2048 + (row >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2;
 }
 
-// A key row whose sketch has components next to zero: its code planes, the
-// mask of components to re-decide, its key's element offset and the address
-// of its stored sign row.
+// A key row whose sketch has components next to zero: the mask of
+// components to re-decide, its key's element offset, and the addresses of
+// its stored code-plane rows (plane p at planes + p * plane bytes) and sign
+// row.  The requesting thread stored those rows itself before the hand-off.
 struct RefineReq {
-  uint32_t planes[3][4];
   uint32_t near[4];
   unsigned long long kbase;
+  unsigned long long planes;
   unsigned long long signs;
 };
 
@@ -456,10 +457,10 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
               for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
               idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
-            } else {  // binary search
+            } else {  // any codebook: count the boundaries below y
               idx = 0;
 #pragma unroll
-              for (int step = NC / 2; step >= 1; step >>= 1) idx += (S.bnd[idx + step - 1] < y) ? step : 0;
+              for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
             }
             idx = zero ? 0 : idx;
 #pragma unroll
@@ -581,12 +582,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         if ((chunk >> lane) & 1u) {
           RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-#pragma unroll
-            for (int p = 0; p < 3; ++p) q.planes[p][w] = p < MB ? planes[p][w] : 0u;
-            q.near[w] = nearw[w];
-          }
+          for (int w = 0; w < 4; ++w) q.near[w] = nearw[w];
           q.kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;
+          q.planes = (unsigned long long)(tp + L.kplanes + slot * kRowBytes);
           q.signs = (unsigned long long)(tp + L.signs + slot * kRowBytes);
         }
         // the sign rows and the requests, then the new tail
@@ -626,12 +624,17 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         for (; h != t; ++h) {
           const RefineReq &q = S.ring[ew][h % kRingCap];
           uint32_t pl[3][4], nw[4], res[4];
+          const uint8_t *prow = reinterpret_cast<const uint8_t *>(q.planes);
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-#pragma unroll
-            for (int p = 0; p < 3; ++p) pl[p][w] = q.planes[p][w];
-            nw[w] = q.near[w];
+          for (int p = 0; p < 3; ++p) {
+            const uint4 v = p < MB ? *reinterpret_cast<const uint4 *>(prow + p * kPlaneBytes) : make_uint4(0u, 0u, 0u, 0u);
+            pl[p][0] = v.x;
+            pl[p][1] = v.y;
+            pl[p][2] = v.z;
+            pl[p][3] = v.w;
           }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) nw[w] = q.near[w];
           const unsigned long long kb = q.kbase;
           uint32_t *words = reinterpret_cast<uint32_t *>(q.signs);
           refine_row_f64<kD>(a.s, a.s_pit, S.cent, a.k, a.dtype, kb, pl, nw, res);

@@ -1,5 +1,5 @@
 // quantize_append for small appends (a decode step's one token per sequence
-// and head): one warp per vector.  Up to d = 128 the CTA first copies Pi and
+// and head): four warps per vector, each taking a quarter of every mat-vec.  Up to d = 128 the CTA first copies Pi and
 // S into shared memory as they are (row-major, 16-byte asynchronous copies,
 // all in flight at once); at d = 256 they are read from global memory
 // (L1/L2).  Same encoding as the other append kernels ("TurboQuant"
@@ -9,14 +9,16 @@
 // TurboQuant-MSE values ("03. Results & Benchmarks", "At a Glance ->
 // Compression": the Lloyd-Max cells of Pi v/||v|| and ||v||).
 //
-// Layout in the warp.  A vector (u, r, the unit value) is held as lane l ->
+// Layout in a warp.  A vector (u, r, the unit value) is held as lane l ->
 // coordinates C l .. C l + C - 1 (C = D/32), so every row of Pi or S is one
-// coalesced read.  M x for 32 rows at a time is the lanes' partial dot
+// coalesced read.  M x for a block of 32 rows is the lanes' partial dot
 // products reduced by recursive halving (31 shuffles for 32 rows), which
 // leaves row r0 + l in lane l: exactly the order of a code-plane word, so
-// one ballot per plane packs it.  Pi^T c streams the rows of Pi with c_i
-// broadcast from its lane.  Sketch components within 1e-5 of zero have
-// their sign decided again in float64 (with W = S Pi^T).
+// one ballot per plane packs it.  The four warps of a quad take the 32-row
+// blocks of Pi u and S r in turn, a quarter of the rows of Pi^T c each (the
+// c_i and the partial sums meet in shared memory), and the value groups in
+// turn.  Sketch components within 1e-5 of zero have their sign decided
+// again in float64 (with W = S Pi^T).
 #include "quantize_common.cuh"
 #include "sm100.cuh"
 #include "tq_common.cuh"
@@ -28,15 +30,8 @@ namespace {
 
 constexpr int kWarpsPerCta = 8;
 
-// Asynchronous 16-byte global -> shared copies (the copy engine's
-// LDGSTS path); the waits below always complete.
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
+using sm100::cp_async16;
+using sm100::cp_async_wait_all;
 
 // C consecutive floats of row `row` of a row-major D x D matrix, this lane's
 // coordinates C lane .. C lane + C - 1.
@@ -108,31 +103,41 @@ __device__ __forceinline__ int bucketize(const float (&bnd)[NB], float y) {
 template <int D>
 __host__ __device__ constexpr bool stage_mats() { return D <= 128; }
 
-// Per-warp scratch: the centroids c_i of the key's codes, and the 32-bit
-// words of its code planes, signs and refinement mask.
+// Scratch of a group of four warps that encodes one vector together: the
+// centroids c_i of the key's codes, the four warps' partial sums of Pi^T c,
+// and the 32-bit words of the code planes, signs and refinement mask.
 template <int D>
-struct WarpScratch {
+struct QuadScratch {
   float c[D];
+  float part[4][D];
   uint32_t planes[3][D / 32];
   uint32_t sw[D / 32], nw[D / 32];
 };
 
+constexpr int kQuads = kWarpsPerCta / 4;  // vectors in flight per CTA
+
 template <int D>
 __host__ __device__ constexpr size_t warp_kernel_smem() {
-  return (stage_mats<D>() ? 2 * D * D * sizeof(float) : 0) + kWarpsPerCta * sizeof(WarpScratch<D>);
+  return (stage_mats<D>() ? 2 * D * D * sizeof(float) : 0) + kQuads * sizeof(QuadScratch<D>);
 }
 
-// One vector, by one converged warp; Pi and S at pim and sm (shared or
-// global memory), W its scratch.
+// Named barrier of the 128 threads of quad q (id 1 + q; id 0 is the CTA's).
+__device__ __forceinline__ void quad_sync(int q) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
+}
+
+// One vector, by the four converged warps of quad `quad` (qw = 0..3 within
+// it); Pi and S at pim and sm (shared or global memory), Q its scratch.
+// The 32-row blocks of every mat-vec are spread over the four warps.
 template <int D>
 __device__ __forceinline__ void encode_vector(const AppendArgs &a, long long id, const float *__restrict__ pim,
-                                              const float *__restrict__ sm, WarpScratch<D> &W) {
+                                              const float *__restrict__ sm, QuadScratch<D> &Q, int quad, int qw) {
   constexpr int C = D / 32;  // coordinates per lane; also 32-coordinate words per row
   const int lane = threadIdx.x & 31;
   int b, t, h;
   bool valid;
   vec_coords(a, id, b, t, h, valid);
-  if (!valid) return;  // warp-uniform
+  if (!valid) return;  // uniform over the quad
   const TileLayout L = TileLayout::make(a.key_bits, a.value_bits, a.value_mode, D);
   const size_t base = (((size_t)b * a.T + t) * a.h_kv + h) * D;
   const int pos = a.lens[b] + t;
@@ -146,7 +151,7 @@ __device__ __forceinline__ void encode_vector(const AppendArgs &a, long long id,
     if (q < 7) bnd[q] = q < ncent - 1 ? a.boundaries[q] : INFINITY;
   }
 
-  // ---- key: u = k / ||k|| ---------------------------------------------------
+  // ---- key: u = k / ||k|| (every warp of the quad) ---------------------------
   float u[C], ss = 0.f;
 #pragma unroll
   for (int m = 0; m < C; ++m) {
@@ -158,131 +163,135 @@ __device__ __forceinline__ void encode_vector(const AppendArgs &a, long long id,
 #pragma unroll
   for (int m = 0; m < C; ++m) u[m] = zero ? 0.f : __fdiv_rn(u[m], nk);
 
-  // ---- y = Pi u, codes: round k leaves coordinate 32 k + l in lane l -------
-#pragma unroll 1
-  for (int k = 0; k < C; ++k) {
+  // ---- y = Pi u, codes: block k leaves coordinate 32 k + l in lane l -------
+  for (int k = qw; k < C; k += 4) {
     const float y = rows32_dot<D>(pim, 32 * k, u);
     const int idx = zero ? 0 : bucketize(bnd, y);
     float c = 0.f;
 #pragma unroll
     for (int q = 0; q < 8; ++q) c = (q == idx) ? cent[q] : c;
-    W.c[32 * k + lane] = zero ? 0.f : c;
+    Q.c[32 * k + lane] = zero ? 0.f : c;
 #pragma unroll
     for (int p = 0; p < 3; ++p) {
       const uint32_t word = p < L.mb ? __ballot_sync(0xffffffffu, (idx >> p) & 1) : 0u;
-      if (lane == 0) W.planes[p][k] = word;
+      if (lane == 0) Q.planes[p][k] = word;
     }
   }
-  __syncwarp();
+  quad_sync(quad);
 
-  // ---- r = u - Pi^T c, ||r|| ---------------------------------------------------
+  // ---- r = u - Pi^T c (rows split over the warps), ||r|| ----------------------
   float r[C];
   {
     float acc[C];
 #pragma unroll
     for (int m = 0; m < C; ++m) acc[m] = 0.f;
 #pragma unroll 8
-    for (int i = 0; i < D; ++i) {
-      const float ci = W.c[i];
+    for (int i = qw * (D / 4); i < (qw + 1) * (D / 4); ++i) {
+      const float ci = Q.c[i];
       float w[C];
       load_row_chunk<D>(pim, i, w);
 #pragma unroll
       for (int m = 0; m < C; ++m) acc[m] = fmaf(w[m], ci, acc[m]);
     }
+#pragma unroll
+    for (int m = 0; m < C; ++m) Q.part[qw][C * lane + m] = acc[m];
+    quad_sync(quad);
     float rr = 0.f;
 #pragma unroll
     for (int m = 0; m < C; ++m) {
-      r[m] = u[m] - acc[m];
+      const int j = C * lane + m;
+      r[m] = u[m] - (((Q.part[0][j] + Q.part[1][j]) + Q.part[2][j]) + Q.part[3][j]);
       rr = fmaf(r[m], r[m], rr);
     }
     rr = warp_sum(rr);
-    if (lane == 0)
+    if (qw == 0 && lane == 0)
       *reinterpret_cast<__half2 *>(tile + L.norms + slot * 4) =
           __halves2half2(__float2half_rn(nk), __float2half_rn(zero ? 0.f : sqrtf(rr)));
   }
 
   // ---- z = S r: signs, and the components to re-decide in float64 ----------
-#pragma unroll 1
-  for (int k = 0; k < C; ++k) {
+  for (int k = qw; k < C; k += 4) {
     const float z = rows32_dot<D>(sm, 32 * k, r);
     const uint32_t sw = __ballot_sync(0xffffffffu, !zero && z >= 0.f);
     const uint32_t nw = __ballot_sync(0xffffffffu, !zero && fabsf(z) < a.refine_z);
     if (lane == 0) {
-      W.sw[k] = sw;
-      W.nw[k] = nw;
+      Q.sw[k] = sw;
+      Q.nw[k] = nw;
     }
   }
-  __syncwarp();
-  uint32_t planes[3][C], sw[C], nw[C];
-  uint32_t anynear = 0u;
-#pragma unroll
-  for (int k = 0; k < C; ++k) {
-#pragma unroll
-    for (int p = 0; p < 3; ++p) planes[p][k] = W.planes[p][k];
-    sw[k] = W.sw[k];
-    nw[k] = W.nw[k];
-    anynear |= nw[k];
-  }
-  if (anynear) {
-    uint32_t res[C];
-    refine_row_f64<D>(a.s, a.s_pit, a.centroids, a.k, a.dtype, base, planes, nw, res);
-    int nbits = 0;
+  quad_sync(quad);
+  if (qw == 0) {
+    uint32_t planes[3][C], sw[C], nw[C];
+    uint32_t anynear = 0u;
 #pragma unroll
     for (int k = 0; k < C; ++k) {
-      sw[k] = (sw[k] & ~nw[k]) | res[k];
-      nbits += __popc(nw[k]);
-    }
-    if (lane == 0 && a.refine_count) atomicAdd(a.refine_count, (unsigned long long)nbits);
-  }
-  if (lane < C) {  // lane k writes word k of every plane and of the signs
-    uint32_t pw[3] = {0u, 0u, 0u}, sk = 0u;
 #pragma unroll
-    for (int k = 0; k < C; ++k)
-      if (lane == k) {
-        pw[0] = planes[0][k];
-        pw[1] = planes[1][k];
-        pw[2] = planes[2][k];
-        sk = sw[k];
+      for (int p = 0; p < 3; ++p) planes[p][k] = Q.planes[p][k];
+      sw[k] = Q.sw[k];
+      nw[k] = Q.nw[k];
+      anynear |= nw[k];
+    }
+    if (anynear) {
+      uint32_t res[C];
+      refine_row_f64<D>(a.s, a.s_pit, a.centroids, a.k, a.dtype, base, planes, nw, res);
+      int nbits = 0;
+#pragma unroll
+      for (int k = 0; k < C; ++k) {
+        sw[k] = (sw[k] & ~nw[k]) | res[k];
+        nbits += __popc(nw[k]);
       }
+      if (lane == 0 && a.refine_count) atomicAdd(a.refine_count, (unsigned long long)nbits);
+    }
+    if (lane < C) {  // lane k writes word k of every plane and of the signs
+      uint32_t pw[3] = {0u, 0u, 0u}, sk = 0u;
 #pragma unroll
-    for (int p = 0; p < 3; ++p)
-      if (p < L.mb)
-        *reinterpret_cast<uint32_t *>(tile + L.kplanes + p * L.plane_bytes + slot * L.row_bytes + 4 * lane) = pw[p];
-    *reinterpret_cast<uint32_t *>(tile + L.signs + slot * L.row_bytes + 4 * lane) = sk;
-  }
-  __syncwarp();  // the scratch is reused by this warp's next vector
-
-  // ---- values ---------------------------------------------------------------
-  if (!L.mse) {
-    quantize_value_groups<D>(a, L, tile, slot, base, (float)((1 << a.value_bits) - 1));
-    return;
-  }
-  // TurboQuant-MSE: the cells of Pi w, w = v / ||v||, and ||v||
-  const int nvc = 1 << L.vb;
-  float vbnd[15];
+      for (int k = 0; k < C; ++k)
+        if (lane == k) {
+          pw[0] = planes[0][k];
+          pw[1] = planes[1][k];
+          pw[2] = planes[2][k];
+          sk = sw[k];
+        }
 #pragma unroll
-  for (int q = 0; q < 15; ++q) vbnd[q] = q < nvc - 1 ? a.v_boundaries[q] : INFINITY;
-  float w[C], sv = 0.f;
-#pragma unroll
-  for (int m = 0; m < C; ++m) {
-    w[m] = load_elem(a.v, a.dtype, base + C * lane + m);
-    sv = fmaf(w[m], w[m], sv);
-  }
-  const float nv = sqrtf(warp_sum(sv));
-  const bool vzero = !(nv > 0.f);
-#pragma unroll
-  for (int m = 0; m < C; ++m) w[m] = vzero ? 0.f : __fdiv_rn(w[m], nv);
-#pragma unroll 1
-  for (int k = 0; k < C; ++k) {
-    const float y = rows32_dot<D>(pim, 32 * k, w);
-    const int idx = vzero ? 0 : bucketize(vbnd, y);
-    for (int p = 0; p < L.vb; ++p) {
-      const uint32_t word = __ballot_sync(0xffffffffu, (idx >> p) & 1);
-      if (lane == 0)
-        *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * L.plane_bytes + slot * L.row_bytes + 4 * k) = word;
+      for (int p = 0; p < 3; ++p)
+        if (p < L.mb)
+          *reinterpret_cast<uint32_t *>(tile + L.kplanes + p * L.plane_bytes + slot * L.row_bytes + 4 * lane) =
+              pw[p];
+      *reinterpret_cast<uint32_t *>(tile + L.signs + slot * L.row_bytes + 4 * lane) = sk;
     }
   }
-  if (lane == 0) *reinterpret_cast<__half *>(tile + L.vsz + slot * 2) = __float2half_rn(nv);
+
+  // ---- values (the groups / 32-row blocks spread over the warps) -------------
+  if (!L.mse) {
+    quantize_value_groups<D>(a, L, tile, slot, base, (float)((1 << a.value_bits) - 1), qw, 4);
+  } else {
+    // TurboQuant-MSE: the cells of Pi w, w = v / ||v||, and ||v||
+    const int nvc = 1 << L.vb;
+    float vbnd[15];
+#pragma unroll
+    for (int q = 0; q < 15; ++q) vbnd[q] = q < nvc - 1 ? a.v_boundaries[q] : INFINITY;
+    float w[C], sv = 0.f;
+#pragma unroll
+    for (int m = 0; m < C; ++m) {
+      w[m] = load_elem(a.v, a.dtype, base + C * lane + m);
+      sv = fmaf(w[m], w[m], sv);
+    }
+    const float nv = sqrtf(warp_sum(sv));
+    const bool vzero = !(nv > 0.f);
+#pragma unroll
+    for (int m = 0; m < C; ++m) w[m] = vzero ? 0.f : __fdiv_rn(w[m], nv);
+    for (int k = qw; k < C; k += 4) {
+      const float y = rows32_dot<D>(pim, 32 * k, w);
+      const int idx = vzero ? 0 : bucketize(vbnd, y);
+      for (int p = 0; p < L.vb; ++p) {
+        const uint32_t word = __ballot_sync(0xffffffffu, (idx >> p) & 1);
+        if (lane == 0)
+          *reinterpret_cast<uint32_t *>(tile + L.vplanes + p * L.plane_bytes + slot * L.row_bytes + 4 * k) = word;
+      }
+    }
+    if (qw == 0 && lane == 0) *reinterpret_cast<__half *>(tile + L.vsz + slot * 2) = __float2half_rn(nv);
+  }
+  quad_sync(quad);  // the scratch is reused by the quad's next vector
 }
 
 template <int D>
@@ -304,17 +313,17 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta, 1) quantize_append_warp_ker
     pim = mats;
     sm = mats + D * D;
   }
-  WarpScratch<D> &W = reinterpret_cast<WarpScratch<D> *>(mats + kMatFloats)[threadIdx.x >> 5];
+  const int warp = threadIdx.x >> 5, quad = warp >> 2, qw = warp & 3;
+  QuadScratch<D> &Q = reinterpret_cast<QuadScratch<D> *>(mats + kMatFloats)[quad];
   const long long total = (long long)a.batch * a.T * a.h_kv;
-  for (long long id = (long long)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); id < total;
-       id += (long long)gridDim.x * kWarpsPerCta)
-    encode_vector<D>(a, id, pim, sm, W);
+  for (long long id = (long long)blockIdx.x * kQuads + quad; id < total; id += (long long)gridDim.x * kQuads)
+    encode_vector<D>(a, id, pim, sm, Q, quad, qw);
 }
 
 template <int D>
 cudaError_t launch_warp_d(const AppendArgs &a, int num_sms, cudaStream_t stream) {
   const long long total = (long long)a.batch * a.T * a.h_kv;
-  const long long blocks = std::min<long long>((total + kWarpsPerCta - 1) / kWarpsPerCta, num_sms);
+  const long long blocks = std::min<long long>((total + kQuads - 1) / kQuads, num_sms);
   if (blocks == 0) return cudaSuccess;
   const int smem = (int)warp_kernel_smem<D>();
   cudaError_t e = cudaFuncSetAttribute(quantize_append_warp_kernel<D>,

@@ -107,6 +107,18 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Asynchronous 16-byte global -> shared copies (cp.async, L2 only); the
+// wait always completes (no barrier, no other role involved).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start before its predecessor in the stream has finished;
 // pdl_wait() blocks until that predecessor has completed and its memory is

@@ -169,6 +169,13 @@ tq_status tq_make_codebook(int mse_bits, int d, double *centroids, double *bound
     c.swap(cn);
     if (delta < 1e-14 * sigma) break;
   }
+  // the law is symmetric: make the fixed point exactly antisymmetric (the
+  // iteration leaves last-bit differences), c_i = -c_{n-1-i}
+  for (int i = 0; i < levels / 2; ++i) {
+    const double m = 0.5 * (c[levels - 1 - i] - c[i]);
+    c[i] = -m;
+    c[levels - 1 - i] = m;
+  }
   for (int i = 0; i + 1 < levels; ++i) t[i] = 0.5 * (c[i] + c[i + 1]);
   for (int i = 0; i < levels; ++i) centroids[i] = c[i];
   for (int i = 0; i + 1 < levels; ++i) boundaries[i] = t[i];

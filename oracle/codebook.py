@@ -13,6 +13,10 @@ boundaries ("turboquant/audit_claims.py", AUDIT 1).
 Reading: the codebook is fitted to the Gaussian N(0, sigma^2 = 1/d), not to
 the exact Beta law, so that the Gaussian Lloyd-Max constants
 (+-0.7979 sigma at 1 bit; +-0.4528 sigma, +-1.510 sigma at 2 bits) hold.
+The law is symmetric, so its Lloyd-Max quantizer is: the iteration's
+floating-point result is made exactly antisymmetric (c_i = -c_{n-1-i}, the
+mean of the two magnitudes) and the boundaries are the midpoints of that,
+the middle one exactly 0.
 
 Algorithm (Lloyd's two optimality conditions, iterated to a fixed point):
   t_i = (c_i + c_{i+1}) / 2                       (nearest-neighbour boundary)
@@ -69,6 +73,9 @@ def lloyd_max_gaussian(mse_bits: int, d: int, tol: float = 1e-14,
         c = c_new
         if delta < tol * sigma:
             break
+    # exact antisymmetry (the iteration leaves last-bit differences)
+    mag = 0.5 * (c[::-1] - c)
+    c = -mag
     t = 0.5 * (c[:-1] + c[1:])
     return c, t, it
 

@@ -46,6 +46,12 @@ def test_host_codebook_matches_oracle(bits, d):
     oc, ob, _ = codebook.lloyd_max_gaussian(bits, d)
     assert np.allclose(c, oc, rtol=0, atol=1e-13)
     assert np.allclose(b, ob, rtol=0, atol=1e-13)
+    # exactly antisymmetric in float64 and in the float32 the kernels read
+    # (the kernels' symmetric fast paths test exactly that)
+    c, b = np.asarray(c), np.asarray(b)
+    assert np.array_equal(c, -c[::-1]) and np.array_equal(b, -b[::-1])
+    c32, b32 = c.astype(np.float32), b.astype(np.float32)
+    assert np.array_equal(c32, -c32[::-1]) and np.array_equal(b32, -b32[::-1])
 
 
 def test_codebook_argument_errors():

@@ -51,7 +51,10 @@ def test_fixed_point_and_symmetry(bits):
     assert len(c) == 2 ** bits and len(t) == 2 ** bits - 1
     assert np.all(np.diff(c) > 0) and np.all(np.diff(t) > 0)
     assert codebook.fixed_point_residual(c, t, d) < 1e-12
-    assert np.allclose(c, -c[::-1], atol=1e-15)
+    # the symmetric law's quantizer is exactly antisymmetric, the middle
+    # boundary (even level count) exactly 0
+    assert np.array_equal(c, -c[::-1]) and np.array_equal(t, -t[::-1])
+    assert t[len(t) // 2] == 0.0
     # boundaries lie between neighbouring centroids
     assert np.all(c[:-1] < t) and np.all(t < c[1:])
 
