@@ -892,8 +892,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
   extern __shared__ __align__(16) float qsm[];
   float *mats = qsm;                        // [2][128][128]: Pi, S
   float *rot = mats + 2 * kD * kD;          // [G][2][128]
-  float *red = rot + G * 2 * kD;            // [8 warps][G][4]
-  uint8_t *blk = reinterpret_cast<uint8_t *>(red + 8 * G * 4);  // QBLOCK staging
+  float *red = rot + G * 2 * kD;            // [8 warps][G][2]: sum, max |.|
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // The decode kernel may launch now (it waits for this grid).  This grid
   // itself is launched as a dependent of the call's predecessor (typically
@@ -906,7 +905,6 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     cp_async16(mats + 4 * i, a.pi + 4 * i);
     cp_async16(mats + kD * kD + 4 * i, a.s + 4 * i);
   }
-  for (int i = tid; i < C::QBLOCK / 4; i += 256) reinterpret_cast<uint32_t *>(blk)[i] = 0u;
   // Walsh coefficients of the codebook, idx paired with its complement so
   // that a symmetric codebook gives exact zeros for the even subsets
   float cent[NC];
@@ -952,7 +950,6 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     a.status[0] = 0;
     a.status[1] = fallback ? 1 : 0;
   }
-  QConst *qc = reinterpret_cast<QConst *>(blk + C::BQ_BYTES);
   cp_async_wait_all();
   __syncthreads();
 
@@ -961,9 +958,11 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     const int b = u / a.h_kv, h = u % a.h_kv;
     {  // warp w: rows 32 w .. 32 w + 31 of [Pi; S] against the G queries
       const float *mrows = mats + (warp < 4 ? 0 : kD * kD) + 32 * (warp & 3) * kD + 4 * lane;
+      // heads per pass (register budget): a divisor of G, at most 4
+      constexpr int GB = G <= 4 ? G : (G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1)));
+      static_assert(G % GB == 0, "heads per pass must divide G");
 #pragma unroll
-      for (int g0 = 0; g0 < G; g0 += 4) {
-        constexpr int GB = G < 4 ? G : 4;  // heads per pass (register budget)
+      for (int g0 = 0; g0 < G; g0 += GB) {
         float qx[GB][4];
 #pragma unroll
         for (int gi = 0; gi < GB; ++gi)
@@ -1001,31 +1000,27 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
         for (int gi = 0; gi < GB; ++gi) {
           rot[(g0 + gi) * 2 * kD + o] = p[gi][0];
           if (fallback) a.qrot[((size_t)b * a.h_q + h * G + g0 + gi) * 2 * kD + o] = p[gi][0];
+          // per head: this warp's sum and max |.| of q~ (warps 0-3) or s^ (4-7)
+          const float sm = warp_sum(p[gi][0]), mx = warp_max(fabsf(p[gi][0]));
+          if (lane == 0) {
+            red[(warp * G + g0 + gi) * 2 + 0] = sm;
+            red[(warp * G + g0 + gi) * 2 + 1] = mx;
+          }
         }
       }
     }
     __syncthreads();
-    // per head: sum and max |.| of q~ (warps 0-3) and s^ (warps 4-7)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int j = tid & (kD - 1);
-      const float x = rot[g * 2 * kD + (tid < kD ? 0 : kD) + j];
-      const float sm = warp_sum(x), mx = warp_max(fabsf(x));
-      if (lane == 0) {
-        red[(warp * G + g) * 4 + 0] = sm;
-        red[(warp * G + g) * 4 + 1] = mx;
-      }
-    }
-    __syncthreads();
+    uint8_t *qb = a.qblocks + (size_t)u * C::QBLOCK;
+    QConst *qc = reinterpret_cast<QConst *>(qb + C::BQ_BYTES);
     int fm[G], fs[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float sq = 0.f, mq = 0.f, ss = 0.f, ms = 0.f;
       for (int wq = 0; wq < 4; ++wq) {
-        sq += red[(wq * G + g) * 4 + 0];
-        mq = fmaxf(mq, red[(wq * G + g) * 4 + 1]);
-        ss += red[((wq + 4) * G + g) * 4 + 0];
-        ms = fmaxf(ms, red[((wq + 4) * G + g) * 4 + 1]);
+        sq += red[(wq * G + g) * 2 + 0];
+        mq = fmaxf(mq, red[(wq * G + g) * 2 + 1]);
+        ss += red[((wq + 4) * G + g) * 2 + 0];
+        ms = fmaxf(ms, red[((wq + 4) * G + g) * 2 + 1]);
       }
       const float bm = 2.f * wmax * mq, bs = 2.f * ms;
       fm[g] = bm > 0.f ? 25 - ilogbf(bm) : 0;
@@ -1042,12 +1037,16 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
       qc->n_mse = nm;
       for (int p = 0; p < 7; ++p) qc->subset[p] = p < nm ? subs[p] : 0;
     }
+    // the B_q bytes, written straight to the unit's query block (columns
+    // beyond the 4 G limbs are zero)
     for (int kappa = tid; kappa < (nm + 1) * 128; kappa += 256) {
       const int P = kappa >> 7, rem = kappa & 127;
       const int col = rem >> 2, bi = rem & 3;
       const int wd = col >> 3, k = col & 7, kw = k & 3;
       const int coord = 32 * wd + 8 * bi + k;
-      uint8_t *dst0 = blk + P * C::BQ_PLANE + (rem >> 4) * C::LBO_Q + (rem & 15);
+      uint8_t *dst0 = qb + P * C::BQ_PLANE + (rem >> 4) * C::LBO_Q + (rem & 15);
+#pragma unroll
+      for (int n = 4 * G; n < C::NS; ++n) dst0[(n >> 3) * 128 + (n & 7) * 16] = 0;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float x;
@@ -1069,11 +1068,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
         }
       }
     }
-    __syncthreads();
-    uint4 *dst = reinterpret_cast<uint4 *>(a.qblocks + (size_t)u * C::QBLOCK);
-    const uint4 *src = reinterpret_cast<const uint4 *>(blk);
-    for (int i = tid; i < C::QBLOCK / 16; i += 256) dst[i] = src[i];
-    __syncthreads();
+    __syncthreads();  // rot and red are reused by the next unit
   }
   pdl_wait();
 }
@@ -1081,7 +1076,7 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
 template <int MB, int VB, int G>
 size_t qblock_smem_bytes() {
   using C = Cfg<MB, VB, G>;
-  return sizeof(float) * (2 * kD * kD + G * 2 * kD + 8 * G * 4) + C::QBLOCK;
+  return sizeof(float) * (2 * kD * kD + G * 2 * kD + 8 * G * 2);
 }
 
 template <int MB, int VB, int G>

@@ -37,6 +37,8 @@
 // TMEM and marks the records it owns with NaN norms.
 #include <math.h>
 
+#include <type_traits>
+
 #include "sm100.cuh"
 #include "tq_common.cuh"
 #include "tq_kernels.h"
@@ -436,50 +438,58 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       // the next chunk's TMEM load in flight while this one is processed) ----
       uint32_t planes[3][4];
       uint32_t dA[16], dB[16];
-      tmem_ld16(dcol, dA);
-      tmem_wait_ld();
+      // The codebook's shape is decided once per tile, outside the element
+      // loop: a branch per element would keep the compiler from interleaving
+      // the elements' dependent chains (measured: 3x the E1 time).
+      auto e1 = [&](auto sym_c) {
+        constexpr bool SYM = decltype(sym_c)::value;
+        tmem_ld16(dcol, dA);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t(&d)[16] = (c & 1) ? dB : dA;
-        if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
-        uint32_t hw[8], lw[8];
-        uint32_t pw[3] = {0u, 0u, 0u};
+        for (int c = 0; c < 8; ++c) {
+          uint32_t(&d)[16] = (c & 1) ? dB : dA;
+          if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
+          uint32_t hw[8], lw[8];
+          uint32_t pw[3] = {0u, 0u, 0u};
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          int ix[2];
+          for (int e = 0; e < 16; e += 2) {
+            int ix[2];
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const float y = __uint_as_float(d[e + x]) * inv1;
-            int idx;  // #{boundaries < y}
-            if (sym) {
-              const float ay = fabsf(y);
-              int cnt = 0;
+            for (int x = 0; x < 2; ++x) {
+              const float y = __uint_as_float(d[e + x]) * inv1;
+              int idx;  // #{boundaries < y}
+              if constexpr (SYM) {
+                const float ay = fabsf(y);
+                int cnt = 0;
 #pragma unroll
-              for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
-              idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
-            } else {  // any codebook: count the boundaries below y
-              idx = 0;
+                for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
+                idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
+              } else {  // any codebook: count the boundaries below y
+                idx = 0;
 #pragma unroll
-              for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
+                for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
+              }
+              idx = zero ? 0 : idx;
+#pragma unroll
+              for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
+              ix[x] = idx;
             }
-            idx = zero ? 0 : idx;
-#pragma unroll
-            for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
-            ix[x] = idx;
+            const int pi2 = ix[0] | (ix[1] << 3);
+            hw[e >> 1] = zero ? 0u : S.cpair[0][pi2];
+            lw[e >> 1] = zero ? 0u : S.cpair[1][pi2];
           }
-          const int pi2 = ix[0] | (ix[1] << 3);
-          hw[e >> 1] = zero ? 0u : S.cpair[0][pi2];
-          lw[e >> 1] = zero ? 0u : S.cpair[1][pi2];
-        }
-        tmem_st8(acol + 8 * c, hw);
-        tmem_st8(acol + 64 + 8 * c, lw);
+          tmem_st8(acol + 8 * c, hw);
+          tmem_st8(acol + 64 + 8 * c, lw);
 #pragma unroll
-        for (int p = 0; p < 3; ++p) {
-          if (c & 1) planes[p][c >> 1] |= pw[p] << 16;
-          else planes[p][c >> 1] = pw[p];
+          for (int p = 0; p < 3; ++p) {
+            if (c & 1) planes[p][c >> 1] |= pw[p] << 16;
+            else planes[p][c >> 1] = pw[p];
+          }
+          if (c < 7) tmem_wait_ld();
         }
-        if (c < 7) tmem_wait_ld();
-      }
+      };
+      if (sym) e1(std::true_type{});
+      else e1(std::false_type{});
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
