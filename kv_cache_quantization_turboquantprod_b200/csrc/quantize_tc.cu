@@ -19,18 +19,21 @@
 // Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
 // record section a tile writes is one contiguous run of the cache.
 //
-// Warp roles (480 threads):
-//   warps 0, 13   MMA issuers of epilogue groups 0 and 1 (one elected lane),
-//                 each sleeping in blocking waits on its group's barriers
-//   warps 1-4     loader: K rows -> scaled fp16 A operand + norms in shared
-//                 memory
-//   warps 5-8     epilogue group 0 (even tiles)   | thread = tile row = TMEM
-//   warps 9-12    epilogue group 1 (odd tiles)    | lane; 256 TMEM columns each
-//   warp 14       sign refiner: sketch components the epilogue found next to
-//                 zero (|S r| < 1e-5, about one key in 300) get their sign
-//                 again in float64, off the pipeline's critical path; each
-//                 epilogue warp hands such rows over through its own ring in
-//                 shared memory and the refiner patches the stored sign words
+// Warp roles (512 threads, by warpgroup):
+//   WG0  warps 0, 1   MMA issuers of epilogue groups 0 and 1 (one elected
+//                     lane), each sleeping in blocking waits on its group's
+//                     barriers
+//        warps 2, 3   sign refiners: sketch components the epilogue found next
+//                     to zero (|S r| < 1e-5, about one key in 300) get their
+//                     sign again in float64, off the pipeline's critical path;
+//                     each epilogue warp hands such rows over through its own
+//                     ring in shared memory and a refiner patches the stored
+//                     sign words
+//   WG1  warps 4-7    loader: K rows -> scaled fp16 A operand + norms in
+//                     shared memory
+//   WG2  warps 8-11   epilogue group 0 (even tiles) | thread = tile row = TMEM
+//   WG3  warps 12-15  epilogue group 1 (odd tiles)  | lane; 256 columns each
+// setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
 // Every mbarrier wait between roles is bounded (2 s unless the host set another
 // limit) and answers warp-uniformly; on timeout the CTA raises its abort flag
 // and the device's sticky error word, stops, lets its own MMAs finish, frees
@@ -49,9 +52,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQtThreads = 480;
-constexpr int kIssuer1Warp = 13;  // MMA issuer of epilogue group 1 (warp 0 issues for group 0)
-constexpr int kRefineWarp = 14;   // float64 sign refiner
+constexpr int kQtThreads = 512;
+constexpr int kQtRegs = 128;  // registers a thread at launch: 65536 / kQtThreads
 constexpr int kRingCap = 16;      // refinement requests per epilogue warp in flight
 constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
 constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
@@ -249,13 +251,19 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
 
-  if (warp == 0 || warp == kIssuer1Warp) {
+  // Registers move from the warpgroups that need few (issuers and refiners,
+  // loader) to the epilogue warpgroups: (64 + 96) x 128 + 176 x 256 = 65536,
+  // exactly the 128 x 512 the CTA is launched with (checked on the host).
+  const int wg = warp >> 2;
+  if (wg == 0) {
+    reg_dealloc<64>();
+    if (warp < 2) {
     // ---------------- MMA issuers -----------------------------------------
-    // Warp 0 issues the three GEMMs of epilogue group 0's tiles, warp 13
+    // Warp 0 issues the three GEMMs of epilogue group 0's tiles, warp 1
     // those of group 1, each in order and sleeping in blocking waits on its
     // group's operand barriers (a polling issuer shares its sub-partition's
     // issue slots with the loader and epilogue warps).
-    const int g = warp == 0 ? 0 : 1;
+    const int g = warp;
     const bool leader = elect_one();
     const uint32_t id1 = idesc_f16(128, 128, false, false);
     const uint32_t id2 = idesc_f16(128, 128, false, true);
@@ -314,14 +322,95 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     }
     // never leave with an MMA in flight: the group's last commit
     if (last_bar) mbar_wait(last_bar, last_ph);
-  } else if (warp <= 4) {
+    } else {
+    // ---------------- sign refiners ----------------------------------------
+    // Warp 2 serves the rings of epilogue warps 0-3, warp 3 those of 4-7, in
+    // turn, until every epilogue warp is done and its rings are empty.  Its waits are on the epilogue warps, whose own
+    // waits are bounded; it is bounded too (same limit, measured from the
+    // last request or finished tile it saw) and gives up by raising the
+    // abort flag.
+    unsigned long long t_last = globaltimer_ns();
+    int seen = S.progress;
+    while (true) {
+      // shared words are read by lane 0 and broadcast, so the warp stays converged
+      const int done = __shfl_sync(0xffffffffu, S.epi_done, 0);  // before the rings: no request after it is missed
+      bool any = false;
+#pragma unroll 1
+      for (int ew = 4 * (warp - 2); ew < 4 * (warp - 2) + 4; ++ew) {
+        int h = __shfl_sync(0xffffffffu, S.ring_head[ew], 0);
+        const int t = __shfl_sync(0xffffffffu, S.ring_tail[ew], 0);
+        if (h == t) continue;
+        __threadfence_block();
+        for (; h != t; ++h) {
+          const RefineReq &q = S.ring[ew][h % kRingCap];
+          uint32_t pl[3][4], nw[4], res[4];
+          const uint8_t *prow = reinterpret_cast<const uint8_t *>(q.planes);
+#pragma unroll
+          for (int p = 0; p < 3; ++p) {
+            const uint4 v = p < MB ? *reinterpret_cast<const uint4 *>(prow + p * kPlaneBytes) : make_uint4(0u, 0u, 0u, 0u);
+            pl[p][0] = v.x;
+            pl[p][1] = v.y;
+            pl[p][2] = v.z;
+            pl[p][3] = v.w;
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) nw[w] = q.near[w];
+          const unsigned long long kb = q.kbase;
+          uint32_t *words = reinterpret_cast<uint32_t *>(q.signs);
+          refine_row_f64<kD>(a.s, a.s_pit, S.cent, a.k, a.dtype, kb, pl, nw, res);
+          uint32_t mn = 0u, mr = 0u;  // lane w < 4 patches word w
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            if (lane == w) {
+              mn = nw[w];
+              mr = res[w];
+            }
+          if (mn != 0u) {
+            atomicAnd(words + lane, ~mn);
+            atomicOr(words + lane, mr);
+          }
+          if (lane == 0 && a.refine_count)
+            atomicAdd(a.refine_count,
+                      (unsigned long long)(__popc(nw[0]) + __popc(nw[1]) + __popc(nw[2]) + __popc(nw[3])));
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence_block();
+            S.ring_head[ew] = h + 1;  // the slot may be reused
+          }
+          __syncwarp();
+        }
+        any = true;
+      }
+      if (any) {
+        t_last = globaltimer_ns();
+        continue;
+      }
+      if (done == 8) break;
+      if (__shfl_sync(0xffffffffu, S.abort_flag, 0)) break;
+      const int prog = __shfl_sync(0xffffffffu, S.progress, 0);
+      if (prog != seen) {
+        seen = prog;
+        t_last = globaltimer_ns();
+      } else if (globaltimer_ns() - t_last > a.wait_ns) {
+        if (lane == 0) {
+          S.abort_flag = 1;
+          if (a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_QUANTIZE_WAIT);
+        }
+        __syncwarp();
+        break;
+      }
+      __nanosleep(256);
+    }
+    }
+  } else if (wg == 1) {
+    reg_dealloc<96>();
     // ---------------- loader -----------------------------------------------
     // A warp takes 8 rows at a time (one 8-row group of the operand): lane
     // (row rr = lane / 4, channel quarter q = lane % 4) holds channels
     // 32q .. 32q + 31.  Values are quantized by their own kernel, so the
     // loader reads keys only; the rows of the next two steps are in flight
     // while this step's are converted.
-    const int w = warp - 1, rr = lane >> 2, q = lane & 3;
+    const int w = warp - 4, rr = lane >> 2, q = lane & 3;
     // rows of step u = 4 i + pass
     auto fetch = [&](int u, uint4 (&kr)[4]) {
       const int i = u >> 2, pass = u & 3;
@@ -402,9 +491,10 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       // bounded wait on it then runs out)
       if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full[g]);
     }
-  } else if (warp <= 12) {
+  } else {
+    reg_alloc<176>();
     // ---------------- epilogue groups --------------------------------------
-    const int g = (warp - 5) >> 2;
+    const int g = (warp - 8) >> 2;
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;  // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
@@ -580,7 +670,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       unsigned rest = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1] | nearw[2] | nearw[3]) != 0u);
       bool stop = false;
       while (rest) {
-        const int ew = warp - 5;
+        const int ew = warp - 8;
         const int tail = S.ring_tail[ew];
         const int rank = __popc(rest & ((1u << lane) - 1u));
         const unsigned chunk = __ballot_sync(0xffffffffu, ((rest >> lane) & 1u) && rank < kRingCap);
@@ -612,85 +702,6 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       __threadfence_block();
       atomicAdd(const_cast<int *>(&S.epi_done), 1);
     }
-  } else if (warp == kRefineWarp) {
-    // ---------------- sign refiner -----------------------------------------
-    // Serves the eight rings in turn until every epilogue warp is done and
-    // the rings are empty.  Its waits are on the epilogue warps, whose own
-    // waits are bounded; it is bounded too (same limit, measured from the
-    // last request or finished tile it saw) and gives up by raising the
-    // abort flag.
-    unsigned long long t_last = globaltimer_ns();
-    int seen = S.progress;
-    while (true) {
-      // shared words are read by lane 0 and broadcast, so the warp stays converged
-      const int done = __shfl_sync(0xffffffffu, S.epi_done, 0);  // before the rings: no request after it is missed
-      bool any = false;
-#pragma unroll 1
-      for (int ew = 0; ew < 8; ++ew) {
-        int h = __shfl_sync(0xffffffffu, S.ring_head[ew], 0);
-        const int t = __shfl_sync(0xffffffffu, S.ring_tail[ew], 0);
-        if (h == t) continue;
-        __threadfence_block();
-        for (; h != t; ++h) {
-          const RefineReq &q = S.ring[ew][h % kRingCap];
-          uint32_t pl[3][4], nw[4], res[4];
-          const uint8_t *prow = reinterpret_cast<const uint8_t *>(q.planes);
-#pragma unroll
-          for (int p = 0; p < 3; ++p) {
-            const uint4 v = p < MB ? *reinterpret_cast<const uint4 *>(prow + p * kPlaneBytes) : make_uint4(0u, 0u, 0u, 0u);
-            pl[p][0] = v.x;
-            pl[p][1] = v.y;
-            pl[p][2] = v.z;
-            pl[p][3] = v.w;
-          }
-#pragma unroll
-          for (int w = 0; w < 4; ++w) nw[w] = q.near[w];
-          const unsigned long long kb = q.kbase;
-          uint32_t *words = reinterpret_cast<uint32_t *>(q.signs);
-          refine_row_f64<kD>(a.s, a.s_pit, S.cent, a.k, a.dtype, kb, pl, nw, res);
-          uint32_t mn = 0u, mr = 0u;  // lane w < 4 patches word w
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            if (lane == w) {
-              mn = nw[w];
-              mr = res[w];
-            }
-          if (mn != 0u) {
-            atomicAnd(words + lane, ~mn);
-            atomicOr(words + lane, mr);
-          }
-          if (lane == 0 && a.refine_count)
-            atomicAdd(a.refine_count,
-                      (unsigned long long)(__popc(nw[0]) + __popc(nw[1]) + __popc(nw[2]) + __popc(nw[3])));
-          __syncwarp();
-          if (lane == 0) {
-            __threadfence_block();
-            S.ring_head[ew] = h + 1;  // the slot may be reused
-          }
-          __syncwarp();
-        }
-        any = true;
-      }
-      if (any) {
-        t_last = globaltimer_ns();
-        continue;
-      }
-      if (done == 8) break;
-      if (__shfl_sync(0xffffffffu, S.abort_flag, 0)) break;
-      const int prog = __shfl_sync(0xffffffffu, S.progress, 0);
-      if (prog != seen) {
-        seen = prog;
-        t_last = globaltimer_ns();
-      } else if (globaltimer_ns() - t_last > a.wait_ns) {
-        if (lane == 0) {
-          S.abort_flag = 1;
-          if (a.errors) atomicOr(a.errors, (unsigned int)TQ_ERRF_QUANTIZE_WAIT);
-        }
-        __syncwarp();
-        break;
-      }
-      __nanosleep(256);
-    }
   }
 
   tc_fence_before();
@@ -720,8 +731,17 @@ template <int MB>
 cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
   const size_t smem = sizeof(QtSmem);
   static_assert(sizeof(QtSmem) <= 227 * 1024, "shared memory per CTA");
+  static_assert(kQtRegs * kQtThreads == 65536 && (64 + 96) * 128 + 176 * 256 == kQtRegs * kQtThreads,
+                "warpgroup register targets must add up to the launch pool");
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // The register targets assume the build gave the kernel exactly kQtRegs
+  // registers a thread; refuse to launch otherwise (an increase beyond the
+  // pool would wait forever).
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, quantize_tc_kernel<MB>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kQtRegs) return cudaErrorInvalidConfiguration;
   quantize_tc_kernel<MB><<<grid, kQtThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

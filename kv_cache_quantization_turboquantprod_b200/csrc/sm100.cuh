@@ -119,6 +119,21 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // ---------------------------------------------------------------------------
+// Warpgroup register reallocation (setmaxnreg): all four warps of a
+// warpgroup execute the same call.  An increase waits until the CTA's pool
+// (threads x registers at launch) has the registers, so the warpgroups'
+// targets must add up to at most that pool.
+// ---------------------------------------------------------------------------
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------------------
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start before its predecessor in the stream has finished;
 // pdl_wait() blocks until that predecessor has completed and its memory is
