@@ -30,7 +30,8 @@
 //                     ring in shared memory and a refiner patches the stored
 //                     sign words
 //   WG1  warps 4-7    loader: K rows -> scaled fp16 A operand + norms in
-//                     shared memory
+//                     shared memory; a group releases its buffer as soon as
+//                     GEMM1 has read it (its E2 reads the bf16 key rows again)
 //   WG2  warps 8-11   epilogue group 0 (even tiles) | thread = tile row = TMEM
 //   WG3  warps 12-15  epilogue group 1 (odd tiles)  | lane; 256 columns each
 // setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
@@ -499,7 +500,6 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     const int r = 32 * q4 + lane;  // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const uint32_t dcol = tbase + lane_off + g * 256, acol = dcol + 128;
-    const uint8_t *a1 = S.a1[g];
     constexpr int NC = 1 << MB;
     // upper half of a symmetric codebook's boundaries, for the compare-count
     // bucketize: idx = NC/2 + #{ub < |y|} (y > 0) or NC/2 - 1 - #{ub < |y|}
@@ -516,14 +516,20 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       const int pos = a.lens[ti.b] + ti.t0 + r;
       uint8_t *tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
       const int slot = pos % kTile;
+      const size_t kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;  // this row's key
       if (!qwait(&S.d1_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
       const float nk = S.nk[g][r];
       const int sh = S.sh[g][r];
+      // GEMM1 has read the K operand and the norms are in registers: the
+      // loader may refill this group's buffer now (E2 reads the bf16 key
+      // rows from global memory instead), which keeps the loader off the
+      // group's critical path
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a1_free[g]);
       const bool zero = !(nk > 0.f);
       const float rnk = zero ? 0.f : 1.f / nk;
       const float inv1 = ldexpf(rnk, -(sh + 10));  // y = Y 2^-(s+10) / ||k||
-      const float inv2 = ldexpf(rnk, -sh);         // u = K 2^-s / ||k||
       // ---- E1: y = Pi u, codes, centroid operand C (16 columns at a time,
       // the next chunk's TMEM load in flight while this one is processed) ----
       uint32_t planes[3][4];
@@ -590,10 +596,17 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           *reinterpret_cast<uint4 *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes) =
               make_uint4(planes[p][0], planes[p][1], planes[p][2], planes[p][3]);
       // ---- E2: r = u - Pi^T c, ||r||, residual operand R ----
+      // the key row (bf16, 16-byte loads) is fetched while GEMM2 runs
+      uint4 krow[16];
+      {
+        const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + kbase);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) krow[j] = valid ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+      }
       if (!qwait(&S.d2_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
       float rr = 0.f;  // ||r||^2 x 2^26
-      const float inv2r = inv2 * kRScale;
+      const float inv2r = rnk * kRScale;  // u x 2^13 = k ||k||^-1 2^13
       tmem_ld16(dcol, dA);
       tmem_wait_ld();
 #pragma unroll
@@ -603,11 +616,10 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         uint32_t hw[8], lw[8];
 #pragma unroll
         for (int c8 = 0; c8 < 2; ++c8) {
-          const uint4 kv = *reinterpret_cast<const uint4 *>(a1 + blk_off(r, 16 * c + 8 * c8));
-          const __half2 *kh = reinterpret_cast<const __half2 *>(&kv);
+          const __nv_bfloat162 *kh = reinterpret_cast<const __nv_bfloat162 *>(&krow[2 * c + c8]);
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 kf = __half22float2(kh[e2]);
+            const float2 kf = __bfloat1622float2(kh[e2]);
             const int e = 8 * c8 + 2 * e2;
             // r x 2^13 = u 2^13 - (Pi^T c) 2^13, with D = (Pi^T c) 2^26
             const float s0 = zero ? 0.f : fmaf(__uint_as_float(d[e]), -1.220703125e-04f, kf.x * inv2r);
@@ -628,10 +640,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&S.a3_full[g]);
-        mbar_arrive(&S.a1_free[g]);
-      }
+      if (lane == 0) mbar_arrive(&S.a3_full[g]);
       // ---- E3: signs of z = S r, norms ----
       if (!qwait(&S.d3_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
@@ -683,7 +692,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
 #pragma unroll
           for (int w = 0; w < 4; ++w) q.near[w] = nearw[w];
-          q.kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;
+          q.kbase = kbase;
           q.planes = (unsigned long long)(tp + L.kplanes + slot * kRowBytes);
           q.signs = (unsigned long long)(tp + L.signs + slot * kRowBytes);
         }
