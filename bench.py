@@ -223,10 +223,14 @@ def run_ours(args, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    if args.profile_steps:
+        torch.cuda.profiler.start()  # ncu --profile-from-start off captures the timed steps only
     t_start.record(stream)
     for i in range(args.steps):
         step(dec_events[i])
     t_end.record(stream)
+    if args.profile_steps:
+        torch.cuda.profiler.stop()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -642,6 +646,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-quantize", dest="quantize", action="store_false",
                     help="skip the quantize-append Mvec/s measurement")
+    ap.add_argument("--profile-steps", action="store_true",
+                    help="bracket the timed steps with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the per-configuration latency table")
     args = ap.parse_args()

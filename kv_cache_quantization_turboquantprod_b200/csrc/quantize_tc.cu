@@ -332,6 +332,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     // abort flag.
     unsigned long long t_last = globaltimer_ns();
     int seen = S.progress;
+    // idle polls back off from 256 ns to 2 us (a poll costs its
+    // sub-partition ~40 issue slots; requests are rare)
+    unsigned int nap = 256;
     while (true) {
       // shared words are read by lane 0 and broadcast, so the warp stays converged
       const int done = __shfl_sync(0xffffffffu, S.epi_done, 0);  // before the rings: no request after it is missed
@@ -384,6 +387,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       }
       if (any) {
         t_last = globaltimer_ns();
+        nap = 256;
         continue;
       }
       if (done == 8) break;
@@ -400,7 +404,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         __syncwarp();
         break;
       }
-      __nanosleep(256);
+      __nanosleep(nap);
+      nap = nap < 2048 ? 2 * nap : 2048;
     }
     }
   } else if (wg == 1) {
