@@ -19,7 +19,7 @@
 // Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
 // record section a tile writes is one contiguous run of the cache.
 //
-// Warp roles (512 threads, by warpgroup):
+// Warp roles (768 threads, by warpgroup):
 //   WG0  warps 0, 1   MMA issuers of epilogue groups 0 and 1 (one elected
 //                     lane), each sleeping in blocking waits on its group's
 //                     barriers
@@ -32,8 +32,10 @@
 //   WG1  warps 4-7    loader: K rows -> scaled fp16 A operand + norms in
 //                     shared memory; a group releases its buffer as soon as
 //                     GEMM1 has read it (its E2 reads the bf16 key rows again)
-//   WG2  warps 8-11   epilogue group 0 (even tiles) | thread = tile row = TMEM
-//   WG3  warps 12-15  epilogue group 1 (odd tiles)  | lane; 256 columns each
+//   WG2, WG3          epilogue group 0 (even tiles): thread = tile row = TMEM
+//   WG4, WG5          epilogue group 1 (odd tiles)   lane, 256 columns a group;
+//                     the first warpgroup of a group takes columns 0-63 of its
+//                     rows, the second columns 64-127
 // setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
 // Every mbarrier wait between roles is bounded (2 s unless the host set another
 // limit) and answers warp-uniformly; on timeout the CTA raises its abort flag
@@ -53,9 +55,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQtThreads = 512;
-constexpr int kQtRegs = 128;  // registers a thread at launch: 65536 / kQtThreads
-constexpr int kRingCap = 16;      // refinement requests per epilogue warp in flight
+constexpr int kQtThreads = 768;  // 6 warpgroups
+constexpr int kQtRegs = 80;      // registers a thread at launch (65536 / 768, rounded down to 8)
+// setmaxnreg shares: WG0 (issuers, refiners), WG1 (loader), WG2-5 (epilogue)
+constexpr int kIssRegs = 56, kLoadRegs = 72, kEpiRegs = 88;
+constexpr int kRingCap = 8;      // refinement requests per epilogue warp in flight
 constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
 constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
 constexpr float kSScale = 256.f;       // S parts x 2^8
@@ -97,9 +101,14 @@ struct QtSmem {
   volatile int abort_flag;
   // refinement rings, one per epilogue warp (single producer, the refiner
   // the single consumer): requests [head, tail) are pending
-  RefineReq ring[8][kRingCap];
-  volatile int ring_head[8], ring_tail[8];
+  RefineReq ring[16][kRingCap];
+  volatile int ring_head[16], ring_tail[16];
   volatile int epi_done;  // epilogue warps past their last tile
+  // [group][tile parity][half][row]: ||r||^2 x 2^26 over each half of a row
+  // (by parity, so a half that runs a tile ahead cannot overwrite a value
+  // its partner has yet to read: that would take the partner's next arrival)
+  float rrpart[2][2][2][128];
+  uint64_t pair[2][4];      // [group][lane quarter]: the two halves of a row block meet
   volatile int progress;  // changes whenever an epilogue warp finishes a tile
 };
 
@@ -231,16 +240,20 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   if (tid == 0) {
     for (int g = 0; g < 2; ++g) {
       mbar_init(&S.a1_full[g], 4);
-      mbar_init(&S.a1_free[g], 4);
+      mbar_init(&S.a1_free[g], 8);
       mbar_init(&S.d1_full[g], 1);
-      mbar_init(&S.a2_full[g], 4);
+      mbar_init(&S.a2_full[g], 8);
       mbar_init(&S.d2_full[g], 1);
-      mbar_init(&S.a3_full[g], 4);
+      mbar_init(&S.a3_full[g], 8);
       mbar_init(&S.d3_full[g], 1);
-      mbar_init(&S.d_free[g], 4);
+      mbar_init(&S.d_free[g], 8);
     }
     S.abort_flag = 0;
-    for (int w = 0; w < 8; ++w) S.ring_head[w] = S.ring_tail[w] = 0;
+    for (int w = 0; w < 16; ++w) S.ring_head[w] = S.ring_tail[w] = 0;
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&S.pair[0][q], 2);
+      mbar_init(&S.pair[1][q], 2);
+    }
     S.epi_done = 0;
     S.progress = 0;
     fence_mbar_init();
@@ -253,11 +266,12 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   const uint32_t tbase = S.tmem_base;
 
   // Registers move from the warpgroups that need few (issuers and refiners,
-  // loader) to the epilogue warpgroups: (64 + 96) x 128 + 176 x 256 = 65536,
-  // exactly the 128 x 512 the CTA is launched with (checked on the host).
+  // loader) to the four epilogue warpgroups: (56 + 72) x 128 + 88 x 512 =
+  // 61440, exactly the 80 x 768 the CTA is launched with (the kernel's
+  // register count is checked on the host before launch).
   const int wg = warp >> 2;
   if (wg == 0) {
-    reg_dealloc<64>();
+    reg_dealloc<kIssRegs>();
     if (warp < 2) {
     // ---------------- MMA issuers -----------------------------------------
     // Warp 0 issues the three GEMMs of epilogue group 0's tiles, warp 1
@@ -340,7 +354,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       const int done = __shfl_sync(0xffffffffu, S.epi_done, 0);  // before the rings: no request after it is missed
       bool any = false;
 #pragma unroll 1
-      for (int ew = 4 * (warp - 2); ew < 4 * (warp - 2) + 4; ++ew) {
+      for (int ew = 8 * (warp - 2); ew < 8 * (warp - 2) + 8; ++ew) {
         int h = __shfl_sync(0xffffffffu, S.ring_head[ew], 0);
         const int t = __shfl_sync(0xffffffffu, S.ring_tail[ew], 0);
         if (h == t) continue;
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         nap = 256;
         continue;
       }
-      if (done == 8) break;
+      if (done == 16) break;
       if (__shfl_sync(0xffffffffu, S.abort_flag, 0)) break;
       const int prog = __shfl_sync(0xffffffffu, S.progress, 0);
       if (prog != seen) {
@@ -409,7 +423,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     }
     }
   } else if (wg == 1) {
-    reg_dealloc<96>();
+    reg_dealloc<kLoadRegs>();
     // ---------------- loader -----------------------------------------------
     // A warp takes 8 rows at a time (one 8-row group of the operand): lane
     // (row rr = lane / 4, channel quarter q = lane % 4) holds channels
@@ -498,9 +512,14 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full[g]);
     }
   } else {
-    reg_alloc<176>();
+    reg_alloc<kEpiRegs>();
     // ---------------- epilogue groups --------------------------------------
-    const int g = (warp - 8) >> 2;
+    // Group g's warps: WG(2 + 2g) takes columns 0-63 of its rows, WG(3 + 2g)
+    // columns 64-127 (half h); the two warps of a TMEM lane quarter share a
+    // row block and meet once per tile (the ||r||^2 halves and the plane
+    // words of the row) through their pair barrier.
+    const int ew = warp - 8;  // epilogue warp 0 .. 15 (its refinement ring)
+    const int g = ew >> 3, half = (ew >> 2) & 1;
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;  // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
@@ -535,21 +554,25 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       const bool zero = !(nk > 0.f);
       const float rnk = zero ? 0.f : 1.f / nk;
       const float inv1 = ldexpf(rnk, -(sh + 10));  // y = Y 2^-(s+10) / ||k||
+      // a zero key gets y = -inf everywhere, which every bucketize below
+      // maps to code 0 (its C operand is never used: E2 zeroes its residual)
+      const float ybias = zero ? -INFINITY : 0.f;
       // ---- E1: y = Pi u, codes, centroid operand C (16 columns at a time,
       // the next chunk's TMEM load in flight while this one is processed) ----
-      uint32_t planes[3][4];
+      uint32_t planes[3][2];
       uint32_t dA[16], dB[16];
       // The codebook's shape is decided once per tile, outside the element
       // loop: a branch per element would keep the compiler from interleaving
-      // the elements' dependent chains (measured: 3x the E1 time).
+      // the elements' dependent chains.
       auto e1 = [&](auto sym_c) {
         constexpr bool SYM = decltype(sym_c)::value;
-        tmem_ld16(dcol, dA);
+        tmem_ld16(dcol + 64 * half, dA);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t(&d)[16] = (c & 1) ? dB : dA;
-          if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = 4 * half + cc;
+          uint32_t(&d)[16] = (cc & 1) ? dB : dA;
+          if (cc < 3) tmem_ld16(dcol + 16 * (c + 1), (cc & 1) ? dA : dB);
           uint32_t hw[8], lw[8];
           uint32_t pw[3] = {0u, 0u, 0u};
 #pragma unroll
@@ -557,7 +580,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
             int ix[2];
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
-              const float y = __uint_as_float(d[e + x]) * inv1;
+              const float y = fmaf(__uint_as_float(d[e + x]), inv1, ybias);
               int idx;  // #{boundaries < y}
               if constexpr (SYM) {
                 const float ay = fabsf(y);
@@ -570,23 +593,22 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
                 for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
               }
-              idx = zero ? 0 : idx;
 #pragma unroll
               for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
               ix[x] = idx;
             }
-            const int pi2 = ix[0] | (ix[1] << 3);
-            hw[e >> 1] = zero ? 0u : S.cpair[0][pi2];
-            lw[e >> 1] = zero ? 0u : S.cpair[1][pi2];
+            const int pi2 = ix[0] + 8 * ix[1];
+            hw[e >> 1] = S.cpair[0][pi2];
+            lw[e >> 1] = S.cpair[1][pi2];
           }
           tmem_st8(acol + 8 * c, hw);
           tmem_st8(acol + 64 + 8 * c, lw);
 #pragma unroll
           for (int p = 0; p < 3; ++p) {
-            if (c & 1) planes[p][c >> 1] |= pw[p] << 16;
-            else planes[p][c >> 1] = pw[p];
+            if (cc & 1) planes[p][cc >> 1] |= pw[p] << 16;
+            else planes[p][cc >> 1] = pw[p];
           }
-          if (c < 7) tmem_wait_ld();
+          if (cc < 3) tmem_wait_ld();
         }
       };
       if (sym) e1(std::true_type{});
@@ -595,40 +617,40 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.a2_full[g]);
-      if (valid)
+      if (valid)  // this half's two words of every code plane row
 #pragma unroll
         for (int p = 0; p < MB; ++p)
-          *reinterpret_cast<uint4 *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes) =
-              make_uint4(planes[p][0], planes[p][1], planes[p][2], planes[p][3]);
+          *reinterpret_cast<uint2 *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 8 * half) =
+              make_uint2(planes[p][0], planes[p][1]);
       // ---- E2: r = u - Pi^T c, ||r||, residual operand R ----
-      // the key row (bf16, 16-byte loads) is fetched while GEMM2 runs
-      uint4 krow[16];
+      // this half of the key row (bf16, 16-byte loads), fetched while GEMM2 runs
+      uint4 krow[8];
       {
-        const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + kbase);
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + kbase) + 8 * half;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) krow[j] = valid ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+        for (int j = 0; j < 8; ++j) krow[j] = valid ? src[j] : make_uint4(0u, 0u, 0u, 0u);
       }
       if (!qwait(&S.d2_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
-      float rr = 0.f;  // ||r||^2 x 2^26
+      float rr = 0.f;  // ||r||^2 x 2^26 over this half
       const float inv2r = rnk * kRScale;  // u x 2^13 = k ||k||^-1 2^13
-      tmem_ld16(dcol, dA);
-      tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t(&d)[16] = (c & 1) ? dB : dA;
-        if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * half + cc;
+        tmem_ld16(dcol + 16 * c, dA);
+        tmem_wait_ld();
         uint32_t hw[8], lw[8];
 #pragma unroll
         for (int c8 = 0; c8 < 2; ++c8) {
-          const __nv_bfloat162 *kh = reinterpret_cast<const __nv_bfloat162 *>(&krow[2 * c + c8]);
+          const __nv_bfloat162 *kh = reinterpret_cast<const __nv_bfloat162 *>(&krow[2 * cc + c8]);
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const float2 kf = __bfloat1622float2(kh[e2]);
             const int e = 8 * c8 + 2 * e2;
             // r x 2^13 = u 2^13 - (Pi^T c) 2^13, with D = (Pi^T c) 2^26
-            const float s0 = zero ? 0.f : fmaf(__uint_as_float(d[e]), -1.220703125e-04f, kf.x * inv2r);
-            const float s1 = zero ? 0.f : fmaf(__uint_as_float(d[e + 1]), -1.220703125e-04f, kf.y * inv2r);
+            const float s0 = zero ? 0.f : fmaf(__uint_as_float(dA[e]), -1.220703125e-04f, kf.x * inv2r);
+            const float s1 = zero ? 0.f : fmaf(__uint_as_float(dA[e + 1]), -1.220703125e-04f, kf.y * inv2r);
             rr = fmaf(s0, s0, rr);
             rr = fmaf(s1, s1, rr);
             const __half2 hh = __floats2half2_rn(s0, s1);
@@ -640,25 +662,29 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         }
         tmem_st8(acol + 8 * c, hw);
         tmem_st8(acol + 64 + 8 * c, lw);
-        if (c < 7) tmem_wait_ld();
       }
       tmem_wait_st();
       tc_fence_before();
+      S.rrpart[g][ph][half][r] = rr;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a3_full[g]);
+      if (lane == 0) {
+        mbar_arrive(&S.a3_full[g]);
+        mbar_arrive(&S.pair[g][q4]);  // this half's planes and ||r||^2 are written
+      }
       // ---- E3: signs of z = S r, norms ----
       if (!qwait(&S.d3_full[g], ph, &S.abort_flag, a)) break;
       tc_fence_after();
-      uint32_t sw[4] = {0u, 0u, 0u, 0u};
-      uint32_t nearw[4] = {0u, 0u, 0u, 0u};  // |S r| below the refinement threshold
+      uint32_t sw[2] = {0u, 0u};
+      uint32_t nearw[2] = {0u, 0u};  // |S r| below the refinement threshold
       // D = (S r) x 2^21 (R x 2^13 times S x 2^8)
       const float kNearZ = a.refine_z * 2097152.f;
-      tmem_ld16(dcol, dA);
+      tmem_ld16(dcol + 64 * half, dA);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t(&d)[16] = (c & 1) ? dB : dA;
-        if (c < 7) tmem_ld16(dcol + 16 * (c + 1), (c & 1) ? dA : dB);
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * half + cc;
+        uint32_t(&d)[16] = (cc & 1) ? dB : dA;
+        if (cc < 3) tmem_ld16(dcol + 16 * (c + 1), (cc & 1) ? dA : dB);
         uint32_t wv = 0u, nv = 0u;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -666,25 +692,29 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           wv |= (z >= 0.f ? 1u : 0u) << e;
           nv |= (fabsf(z) < kNearZ ? 1u : 0u) << e;
         }
-        sw[c >> 1] |= (zero ? 0u : wv) << (16 * (c & 1));
-        nearw[c >> 1] |= (zero || !valid ? 0u : nv) << (16 * (c & 1));
-        if (c < 7) tmem_wait_ld();
+        sw[cc >> 1] |= (zero ? 0u : wv) << (16 * (cc & 1));
+        nearw[cc >> 1] |= (zero || !valid ? 0u : nv) << (16 * (cc & 1));
+        if (cc < 3) tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.d_free[g]);
+      // the other half's plane words and ||r||^2 half
+      if (!qwait(&S.pair[g][q4], ph, &S.abort_flag, a)) break;
       if (valid) {
-        *reinterpret_cast<uint4 *>(tp + L.signs + slot * kRowBytes) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-        const float rn = zero ? 0.f : sqrtf(rr) * (1.f / kRScale);
-        *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) =
-            __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
+        *reinterpret_cast<uint2 *>(tp + L.signs + slot * kRowBytes + 8 * half) = make_uint2(sw[0], sw[1]);
+        if (half == 0) {
+          const float rr2 = rr + S.rrpart[g][ph][1][r];
+          const float rn = zero ? 0.f : sqrtf(rr2) * (1.f / kRScale);
+          *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) =
+              __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
+        }
       }
       // sketch components next to zero: handed to the float64 refiner, which
       // patches the sign words stored above (at most kRingCap rows at a time)
-      unsigned rest = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1] | nearw[2] | nearw[3]) != 0u);
+      unsigned rest = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1]) != 0u);
       bool stop = false;
       while (rest) {
-        const int ew = warp - 8;
         const int tail = S.ring_tail[ew];
         const int rank = __popc(rest & ((1u << lane) - 1u));
         const unsigned chunk = __ballot_sync(0xffffffffu, ((rest >> lane) & 1u) && rank < kRingCap);
@@ -696,7 +726,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         if ((chunk >> lane) & 1u) {
           RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) q.near[w] = nearw[w];
+          for (int w = 0; w < 4; ++w) q.near[w] = (w >> 1) == half ? nearw[w & 1] : 0u;
           q.kbase = kbase;
           q.planes = (unsigned long long)(tp + L.kplanes + slot * kRowBytes);
           q.signs = (unsigned long long)(tp + L.signs + slot * kRowBytes);
@@ -745,8 +775,9 @@ template <int MB>
 cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
   const size_t smem = sizeof(QtSmem);
   static_assert(sizeof(QtSmem) <= 227 * 1024, "shared memory per CTA");
-  static_assert(kQtRegs * kQtThreads == 65536 && (64 + 96) * 128 + 176 * 256 == kQtRegs * kQtThreads,
-                "warpgroup register targets must add up to the launch pool");
+  static_assert((kIssRegs + kLoadRegs) * 128 + kEpiRegs * 512 <= kQtRegs * kQtThreads &&
+                    kQtRegs * kQtThreads <= 65536 && kIssRegs % 8 == 0 && kLoadRegs % 8 == 0 && kEpiRegs % 8 == 0,
+                "warpgroup register targets must add up to at most the launch pool");
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // The register targets assume the build gave the kernel exactly kQtRegs
