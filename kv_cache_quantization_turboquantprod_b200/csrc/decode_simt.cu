@@ -70,58 +70,81 @@ __global__ void __launch_bounds__(128) decode_splitk_simt_kernel(DecodeArgs a) {
 // (TurboQuant-MSE values: the partials are in the rotated space and the
 // merged accumulator is rotated back once, Pi^T acc).  A call whose kernels
 // gave up on a bounded wait (status word nonzero) gets NaN rows, so a
-// timeout never comes back as a plausible result.  128 threads; thread j
-// takes dims j, j + 128, ...
+// timeout never comes back as a plausible result.
+// 256 threads: M from one split per thread, then warp w sums splits w,
+// w + 8, ... (lane l holding dims 64u + 2l, 64u + 2l + 1), so the loads of
+// every split are in flight at once; the eight warp sums meet in shared
+// memory and thread j finishes dim j.
 // ---------------------------------------------------------------------------
+constexpr int kCombThreads = 256;
+constexpr int kCombWarps = kCombThreads / 32;
+
 template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
-  constexpr int J = (D + 127) / 128;
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
+  static_assert(D % 64 == 0 && D <= kCombThreads, "combine layout");
+  constexpr int U = D / 64;  // float2 loads per lane and split
+  __shared__ float smax[kCombWarps], sden[kCombWarps];
+  __shared__ __align__(8) float snum[kCombWarps][D];
+  __shared__ float acc[D];
   pdl_wait();
   const int bh = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t orow = qrow_offset(a, bh / a.h_q, bh % a.h_q);
   if (a.status[0] != 0) {
-    for (int j = tid; j < D; j += 128) a.out[orow + j] = __int_as_float(0x7fc00000);
+    if (tid < D) a.out[orow + tid] = __int_as_float(0x7fc00000);
     return;
   }
-  const float *src = a.part + (size_t)bh * a.part_stride * (D + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < a.part_stride; ++s) M = fmaxf(M, src[s * (D + 2) + D]);
-  float num[J], den = 0.f;
+  const int ns = a.part_stride;
+  const float *src = a.part + (size_t)bh * ns * (D + 2);
+  float m = -INFINITY;
+  for (int s = tid; s < ns; s += kCombThreads) m = fmaxf(m, src[(size_t)s * (D + 2) + D]);
+  m = warp_max(m);
+  if (lane == 0) smax[warp] = m;
+  __syncthreads();
+  float M = smax[0];
 #pragma unroll
-  for (int u = 0; u < J; ++u) num[u] = 0.f;
+  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, smax[w]);
+  float2 num[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) num[u] = make_float2(0.f, 0.f);
+  float den = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < a.part_stride; ++s) {
-      const float ms = src[s * (D + 2) + D];
-      if (ms == -INFINITY) continue;  // empty split
-      const float f = exp2f(ms - M);
+#pragma unroll 4
+    for (int s = warp; s < ns; s += kCombWarps) {
+      const float *row = src + (size_t)s * (D + 2);
+      const float2 ml = *reinterpret_cast<const float2 *>(row + D);  // (m_s, l_s)
+      if (ml.x == -INFINITY) continue;  // empty split
+      const float f = exp2f(ml.x - M);
 #pragma unroll
-      for (int u = 0; u < J; ++u)
-        if (tid + 128 * u < D) num[u] = fmaf(src[s * (D + 2) + tid + 128 * u], f, num[u]);
-      den = fmaf(src[s * (D + 2) + D + 1], f, den);
+      for (int u = 0; u < U; ++u) {
+        const float2 v = *reinterpret_cast<const float2 *>(row + 64 * u + 2 * lane);
+        num[u].x = fmaf(v.x, f, num[u].x);
+        num[u].y = fmaf(v.y, f, num[u].y);
+      }
+      den = fmaf(ml.y, f, den);
     }
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) *reinterpret_cast<float2 *>(&snum[warp][64 * u + 2 * lane]) = num[u];
+  if (lane == 0) sden[warp] = den;
+  __syncthreads();
+  float o = 0.f, dsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombWarps; ++w) dsum += sden[w];
+  if (tid < D) {
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) o += snum[w][tid];
   }
   if (a.value_mode == TQ_VALUES_MSE) {
     // the merged accumulator is in the rotated space: out_j = (Pi^T acc)_j
-    __shared__ float acc[D];
-#pragma unroll
-    for (int u = 0; u < J; ++u)
-      if (tid + 128 * u < D) acc[tid + 128 * u] = num[u];
+    if (tid < D) acc[tid] = o;
     __syncthreads();
-#pragma unroll
-    for (int u = 0; u < J; ++u) {
-      const int j = tid + 128 * u;
-      if (j >= D) continue;
-      float o = 0.f;
-      for (int i = 0; i < D; ++i) o = fmaf(a.pi[(size_t)i * D + j], acc[i], o);
-      num[u] = o;
+    if (tid < D) {
+      o = 0.f;
+      for (int i = 0; i < D; ++i) o = fmaf(a.pi[(size_t)i * D + tid], acc[i], o);
     }
   }
-#pragma unroll
-  for (int u = 0; u < J; ++u) {
-    const int j = tid + 128 * u;
-    if (j < D) a.out[orow + j] = den > 0.f ? num[u] / den : 0.f;
-  }
+  if (tid < D) a.out[orow + tid] = dsum > 0.f ? o / dsum : 0.f;
 }
 
 // ---------------------------------------------------------------------------
@@ -287,7 +310,7 @@ cudaError_t launch_decode_simt_d(const DecodeArgs &a, cudaStream_t stream) {
     e = launch_window(a, stream);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(combine_kernel<D>, dim3(bhq), dim3(128), 0, stream, a);
+  return launch_pdl(combine_kernel<D>, dim3(bhq), dim3(kCombThreads), 0, stream, a);
 }
 
 }  // namespace
@@ -347,7 +370,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     e = launch_window(a, stream);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(combine_kernel<kD>, dim3(bhq), dim3(128), 0, stream, a);
+  return launch_pdl(combine_kernel<kD>, dim3(bhq), dim3(kCombThreads), 0, stream, a);
 }
 
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream) {

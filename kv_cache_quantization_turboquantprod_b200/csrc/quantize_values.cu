@@ -14,11 +14,10 @@
 // are computed by one lane per vector and handed to its quarter by shuffles.
 //
 // Codes.  For 2-bit values the code is the number of the group's three
-// rounding thresholds z + (k + 1/2) s below v, with the thresholds formed in
-// float64 (exact: z and s are fp16) and rounded down to float32; a threshold
-// that is exactly representable and belongs to an odd k (a tie that rounds
-// up to even) also counts v equal to it.  That is the rounded exact quotient
-// by comparisons alone.  For 3 and 4 bits the code is rint of the float32
+// rounding thresholds z + (k + 1/2) s below v, compared on bf16 pairs: each
+// threshold rounded down to bf16, or for an odd k (a tie rounds up to the
+// even code) whose threshold is a bf16, the bf16 just below it.  That is the
+// rounded exact quotient by comparisons alone.  For 3 and 4 bits the code is rint of the float32
 // quotient, redone in float64 where it sits within 1e-5 of a half-integer.
 // The records' value sections (codes, scale, zero) are written in place; the
 // key sections are the tensor-core kernel's.  Head dim 128, bf16 input.
@@ -39,35 +38,45 @@ __device__ __forceinline__ __half group_scale(float mn, float mx, int levels) {
   return __double2half(((double)mx - (double)mn) / (double)levels);
 }
 
-// The largest float below a finite float f.
-__device__ __forceinline__ float float_below(float f) {
-  if (f == 0.f) return -__uint_as_float(1u);  // the negative of the least subnormal
-  const uint32_t u = __float_as_uint(f);
-  return __uint_as_float(f > 0.f ? u - 1u : u + 1u);
+// The largest bf16 below a finite bf16 b (as raw bits).
+__device__ __forceinline__ unsigned short bf16_below(unsigned short b) {
+  if ((b & 0x7fffu) == 0u) return 0x8001u;  // below +-0: the negative of the least subnormal
+  return (b & 0x8000u) ? (unsigned short)(b + 1u) : (unsigned short)(b - 1u);
 }
 
-// Packed 2-bit codes of 16 channels (channel 4i + m in bits 2m, 2m+1 of
-// byte i) by threshold counts.
-__device__ __forceinline__ uint32_t codes2_packed(const float (&x)[16], __half zero16, __half scale16) {
-  float thr[3];
-  const double z = (double)__half2float(zero16), s = (double)__half2float(scale16);
+// Packed 2-bit codes of 16 bf16 channels (channel 4i + m in bits 2m, 2m+1 of
+// byte i) by threshold counts, two channels per comparison.  Threshold k is
+// t = z + (k + 1/2) s; one FMA rounded down and one rounded up bracket it
+// and agree exactly when t is a float.  A bf16 value v is above t iff it is
+// above t rounded down to bf16; for odd k, where a tie rounds up to the even
+// code, v counts when it equals t, i.e. when it is above the bf16 below t.
+__device__ __forceinline__ uint32_t codes2_packed(const uint32_t (&xw)[8], __half zero16, __half scale16) {
+  const float z = __half2float(zero16), s = __half2float(scale16);
+  __nv_bfloat162 thr[3];
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
-    if (s == 0.0) {
-      thr[k] = INFINITY;  // zero scale: every code 0
-      continue;
+    unsigned short tb;
+    if (s == 0.f) {
+      tb = 0x7f80u;  // +inf: zero scale, every code 0
+    } else {
+      const float tlo = __fmaf_rd((float)k + 0.5f, s, z), thi = __fmaf_ru((float)k + 0.5f, s, z);
+      const __nv_bfloat16 b = __float2bfloat16_rd(tlo);
+      tb = __bfloat16_as_ushort(b);
+      // odd k: a value equal to the threshold rounds up (to the even code)
+      if ((k & 1) && tlo == thi && __bfloat162float(b) == tlo) tb = bf16_below(tb);
     }
-    const double t = fma((double)k + 0.5, s, z);  // exact
-    float tf = __double2float_rd(t);
-    // odd k: a value equal to the threshold rounds up (to the even code)
-    if ((k & 1) && (double)tf == t) tf = float_below(tf);
-    thr[k] = tf;
+    const __nv_bfloat16 bt = __ushort_as_bfloat16(tb);
+    thr[k] = __halves2bfloat162(bt, bt);
   }
   uint32_t w = 0u;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const uint32_t c = (x[e] > thr[0] ? 1u : 0u) + (x[e] > thr[1] ? 1u : 0u) + (x[e] > thr[2] ? 1u : 0u);
-    w |= c << (2 * e);
+  for (int j = 0; j < 8; ++j) {
+    const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162 *>(&xw[j]);
+    // per 16-bit half: 0xffff where the channel is above the threshold
+    const uint32_t c = (__hgt2_mask(x2, thr[0]) & 0x00010001u) + (__hgt2_mask(x2, thr[1]) & 0x00010001u) +
+                       (__hgt2_mask(x2, thr[2]) & 0x00010001u);
+    // channels 2j (low half) and 2j + 1 (high half): bits 4j and 4j + 2
+    w |= ((c & 3u) | ((c >> 14) & 0xcu)) << (4 * j);
   }
   return w;
 }
@@ -116,21 +125,26 @@ __global__ void __launch_bounds__(kVqThreads) value_quant_kernel(const __grid_co
     for (int u = 0; u < kVqRounds; ++u) {
       const long long off = __shfl_sync(0xffffffffu, roff, 4 * u + qv);
       const int slot = __shfl_sync(0xffffffffu, rslot, 4 * u + qv);
-      float x[16];
+      // this lane's 16 channels as 8 bf16 pairs
+      uint32_t xw[8];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const uint32_t *wv = reinterpret_cast<const uint32_t *>(&raw[u][c]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[8 * c + 2 * e] = __uint_as_float(wv[e] << 16);
-          x[8 * c + 2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
-        }
+        xw[4 * c] = raw[u][c].x;
+        xw[4 * c + 1] = raw[u][c].y;
+        xw[4 * c + 2] = raw[u][c].z;
+        xw[4 * c + 3] = raw[u][c].w;
       }
-      float mn = x[0], mx = x[0];
+      float mn, mx;
+      {
+        __nv_bfloat162 lo2 = *reinterpret_cast<const __nv_bfloat162 *>(&xw[0]), hi2 = lo2;
 #pragma unroll
-      for (int e = 1; e < 16; ++e) {
-        mn = fminf(mn, x[e]);
-        mx = fmaxf(mx, x[e]);
+        for (int j = 1; j < 8; ++j) {
+          const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162 *>(&xw[j]);
+          lo2 = __hmin2(lo2, x2);
+          hi2 = __hmax2(hi2, x2);
+        }
+        mn = fminf(__low2float(lo2), __high2float(lo2));
+        mx = fmaxf(__low2float(hi2), __high2float(hi2));
       }
       // a group of 32 channels = lanes 2i, 2i + 1 of the quarter
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
@@ -142,13 +156,19 @@ __global__ void __launch_bounds__(kVqThreads) value_quant_kernel(const __grid_co
       if constexpr (VB == 2) {
         // packed: this lane's 16 channels are bytes 4 ql .. 4 ql + 3 of the row
         *reinterpret_cast<uint32_t *>(tile + L.vplanes + slot * L.packed_row_bytes + 4 * ql) =
-            codes2_packed(x, zero16, scale16);
+            codes2_packed(xw, zero16, scale16);
       } else {
         const float z32 = __half2float(zero16), sc32 = __half2float(scale16);
         const float rsc = sc32 != 0.f ? 1.f / sc32 : 0.f;
         uint32_t pw[VB];
 #pragma unroll
         for (int p = 0; p < VB; ++p) pw[p] = 0u;
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          x[2 * j] = __uint_as_float(xw[j] << 16);
+          x[2 * j + 1] = __uint_as_float(xw[j] & 0xffff0000u);
+        }
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float tq = (x[e] - z32) * rsc;
