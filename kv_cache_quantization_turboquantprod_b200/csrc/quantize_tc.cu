@@ -1,28 +1,38 @@
 // quantize_append on the 5th-generation tensor cores (tcgen05 kind::f16):
 // the TurboQuant-prod key encoding of "TurboQuant" explainer (troisinh.com,
 // "Ý tưởng cốt lõi") and "turboquant/audit_claims.py" (AUDIT 1 / AUDIT 5),
-// with the three d x d products of every key vector as tensor-core GEMMs
-// over 128-vector tiles and everything else fused in their epilogues:
-//   GEMM1  Y = K Pi^T            y = Y / ||k||, bucketize -> codes, c = c[idx]
-//   GEMM2  P = C Pi              r = u - P (= u - Pi^T c), ||r||
-//   GEMM3  Z = R S^T             signs = [z >= 0]
+// with the d x d products of every key vector as tensor-core GEMMs over
+// 128-vector tiles and everything else fused in their epilogues:
+//   GEMM1  Y = K Pi^T            y = Y / ||k||, bucketize -> codes, c = c[idx],
+//                                E = y - c, ||r|| = ||E||
+//   GEMM2  Z = E W^T             signs = [z >= 0]
+// with W = S Pi^T (float64, formed once per layer).  Pi is orthogonal, so
+// the residual r = u - Pi^T c equals Pi^T (y - c): its norm is that of
+// E = y - c and its sketch is S r = S Pi^T E = W E.  No r is formed and no
+// key row is read twice.
 // Values are group-quantized (per 32 channels, fp16 scale/zero) by a
 // separate bandwidth-bound kernel launched just before this one
 // (quantize_values.cu).
 //
 // Precision.  A bf16 key is exact in fp16 once scaled per vector by 2^s
-// (largest |k| 2^s in [2^14, 2^15)); Pi, S, the centroids and the residual
-// are split into fp16 hi + lo parts (scaled so no part is subnormal where it
-// matters), and each product takes the three significant hi/lo terms with
-// f32 accumulation: about 22 bits per operand, the error of an fp32 mat-vec.
+// (largest |k| 2^s in [2^14, 2^15)); Pi, W and E are split into fp16 hi +
+// lo parts (scaled so no part is subnormal where it matters), and each
+// product takes the significant hi/lo terms with f32 accumulation: about 22
+// bits per operand, the error of an fp32 mat-vec.  E is formed from the
+// accumulator in one rounding (fma(Y, 2^13 / (2^(s+10) ||k||), -c 2^13)).
 //
 // Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
 // record section a tile writes is one contiguous run of the cache.
 //
+// Pipeline.  Tensor memory holds the accumulators D1 (columns 0-127) and D2
+// (128-255) and GEMM2's A operand E (256-383: fp16 hi and lo parts, 16
+// columns a K-step).  The epilogue hands E to the issuer a K-step at a time
+// (one barrier per K-step), so GEMM2 runs under E1, and the next tile's
+// GEMM1 runs while this tile's signs are read.
+//
 // Warp roles (768 threads, by warpgroup):
-//   WG0  warps 0, 1   MMA issuers of epilogue groups 0 and 1 (one elected
-//                     lane), each sleeping in blocking waits on its group's
-//                     barriers
+//   WG0  warp 0       MMA issuer (one elected lane), sleeping in blocking
+//                     waits on the operand barriers; warp 1 idles
 //        warps 2, 3   sign refiners: sketch components the epilogue found next
 //                     to zero (|S r| < 1e-5, about one key in 300) get their
 //                     sign again in float64, off the pipeline's critical path;
@@ -30,12 +40,10 @@
 //                     ring in shared memory and a refiner patches the stored
 //                     sign words
 //   WG1  warps 4-7    loader: K rows -> scaled fp16 A operand + norms in
-//                     shared memory; a group releases its buffer as soon as
-//                     GEMM1 has read it (its E2 reads the bf16 key rows again)
-//   WG2, WG3          epilogue group 0 (even tiles): thread = tile row = TMEM
-//   WG4, WG5          epilogue group 1 (odd tiles)   lane, 256 columns a group;
-//                     the first warpgroup of a group takes columns 0-63 of its
-//                     rows, the second columns 64-127
+//                     shared memory (two buffers); the epilogue releases a
+//                     buffer as soon as GEMM1 has read it
+//   WG2-WG5           epilogue: thread = tile row = TMEM lane; warp w takes
+//                     lane quarter w % 4 and one quarter of the columns
 // setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
 // Every mbarrier wait between roles is bounded (2 s unless the host set another
 // limit) and answers warp-uniformly; on timeout the CTA raises its abort flag
@@ -62,9 +70,8 @@ constexpr int kIssRegs = 56, kLoadRegs = 72, kEpiRegs = 88;
 constexpr int kRingCap = 8;      // refinement requests per epilogue warp in flight
 constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
 constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
-constexpr float kSScale = 256.f;       // S parts x 2^8
-constexpr float kCScale = 65536.f;     // centroid parts x 2^16
-constexpr float kRScale = 8192.f;      // residual parts x 2^13
+constexpr double kWScale = 256.0;     // W = S Pi^T parts x 2^8
+constexpr float kEScale = 8192.f;      // E = y - c parts x 2^13
 
 // byte offset of element (row, col) of a 128 x 128 fp16 matrix in the
 // canonical no-swizzle layout: 8 x 8 blocks, block (row / 8, col / 8) at
@@ -87,16 +94,20 @@ struct RefineReq {
 
 struct QtSmem {
   alignas(1024) uint8_t pi[2][kMat16];  // Pi x 2^10: hi, lo
-  alignas(1024) uint8_t s[2][kMat16];   // S x 2^8: hi, lo
-  alignas(1024) uint8_t a1[2][kMat16];  // K rows x 2^s (fp16), one per epilogue group
+  alignas(1024) uint8_t w[2][kMat16];   // W = S Pi^T x 2^8: hi, lo
+  alignas(1024) uint8_t a1[2][kMat16];  // K rows x 2^s (fp16), double-buffered by tile
   float nk[2][128];
   int sh[2][128];
   float cent[8];
+  float cent13[8];               // centroids x 2^13
   float bnd[8];                  // ascending, padded with +inf
-  uint32_t cpair[2][64];         // packed fp16 (hi, lo) parts of c[i0], c[i1] x 2^16, index i0 | i1 << 3
   int sym;                       // boundaries exactly antisymmetric (b[i] == -b[nb - 1 - i])
-  uint64_t a1_full[2], a1_free[2], d1_full[2], a2_full[2], d2_full[2], a3_full[2], d3_full[2],
-      d_free[2];
+  // a1_full / a1_free: a K operand buffer is loaded / read by GEMM1 and its
+  // norms taken; d1_full / d2_full: a tile's GEMM1 / GEMM2 is complete;
+  // d_free: the epilogue has read D2; kc[c]: K-step c of the tile's E
+  // operand is in tensor memory; fin: the issuer's last commit (every MMA
+  // it issued is done)
+  uint64_t a1_full[2], a1_free[2], d1_full, d2_full, d_free, kc[8], fin;
   uint32_t tmem_base;
   volatile int abort_flag;
   // refinement rings, one per epilogue warp (single producer, the refiner
@@ -104,11 +115,11 @@ struct QtSmem {
   RefineReq ring[16][kRingCap];
   volatile int ring_head[16], ring_tail[16];
   volatile int epi_done;  // epilogue warps past their last tile
-  // [group][tile parity][half][row]: ||r||^2 x 2^26 over each half of a row
-  // (by parity, so a half that runs a tile ahead cannot overwrite a value
-  // its partner has yet to read: that would take the partner's next arrival)
-  float rrpart[2][2][2][128];
-  uint64_t pair[2][4];      // [group][lane quarter]: the two halves of a row block meet
+  // [tile parity][column quarter][row]: ||r||^2 x 2^26 over a quarter of a
+  // row (by parity, so a warp that runs a tile ahead cannot overwrite a value
+  // that is yet to be read: that would take the reader's next hand-over)
+  float rrq[2][4][128];
+  uint64_t pair[4];         // [lane quarter]: the four column quarters of a row block meet
   volatile int progress;  // changes whenever an epilogue warp finishes a tile
 };
 
@@ -194,17 +205,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                          ? (a.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
                          : 0;
 
-  // ---- setup: split Pi and S into fp16 parts, barriers, TMEM -------------
+  // ---- setup: split Pi and W = S Pi^T into fp16 parts, barriers, TMEM ---
   // eight elements (one 16-byte block row) per item, both matrices' loads
-  // issued before any is used
+  // issued before any is used; W is split from its float64 values
   for (int it = tid; it < 128 * 16; it += kQtThreads) {
     const int i = it >> 4, j0 = (it & 15) * 8;
     const float4 *pp = reinterpret_cast<const float4 *>(a.pi + i * 128 + j0);
-    const float4 *sp = reinterpret_cast<const float4 *>(a.s + i * 128 + j0);
-    const float4 p0 = pp[0], p1 = pp[1], s0 = sp[0], s1 = sp[1];
+    const double2 *wp = reinterpret_cast<const double2 *>(a.s_pit + i * 128 + j0);
+    const float4 p0 = pp[0], p1 = pp[1];
+    const double2 w0 = wp[0], w1 = wp[1], w2 = wp[2], w3 = wp[3];
     const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    uint32_t ph[4], pl[4], sh2[4], sl[4];
+    const double wv[8] = {w0.x, w0.y, w1.x, w1.y, w2.x, w2.y, w3.x, w3.y};
+    uint32_t ph[4], pl[4], wh[4], wl[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float h0, l0, h1, l1;
@@ -212,48 +224,42 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       split16(pv[2 * e + 1] * kPiScale, h1, l1);
       ph[e] = pack_h2(h0, h1);
       pl[e] = pack_h2(l0, l1);
-      split16(sv[2 * e] * kSScale, h0, l0);
-      split16(sv[2 * e + 1] * kSScale, h1, l1);
-      sh2[e] = pack_h2(h0, h1);
-      sl[e] = pack_h2(l0, l1);
+      const double x0 = wv[2 * e] * kWScale, x1 = wv[2 * e + 1] * kWScale;
+      const __half hh0 = __double2half(x0), hh1 = __double2half(x1);
+      const __half ll0 = __double2half(x0 - (double)__half2float(hh0));
+      const __half ll1 = __double2half(x1 - (double)__half2float(hh1));
+      const __half2 hw2 = __halves2half2(hh0, hh1), lw2 = __halves2half2(ll0, ll1);
+      wh[e] = *reinterpret_cast<const uint32_t *>(&hw2);
+      wl[e] = *reinterpret_cast<const uint32_t *>(&lw2);
     }
     *reinterpret_cast<uint4 *>(S.pi[0] + blk_off(i, j0)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
     *reinterpret_cast<uint4 *>(S.pi[1] + blk_off(i, j0)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-    *reinterpret_cast<uint4 *>(S.s[0] + blk_off(i, j0)) = make_uint4(sh2[0], sh2[1], sh2[2], sh2[3]);
-    *reinterpret_cast<uint4 *>(S.s[1] + blk_off(i, j0)) = make_uint4(sl[0], sl[1], sl[2], sl[3]);
+    *reinterpret_cast<uint4 *>(S.w[0] + blk_off(i, j0)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4 *>(S.w[1] + blk_off(i, j0)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
   }
-  if (tid < ncent) S.cent[tid] = a.centroids[tid];
+  if (tid < ncent) {
+    S.cent[tid] = a.centroids[tid];
+    S.cent13[tid] = a.centroids[tid] * kEScale;
+  }
   if (tid < 8) S.bnd[tid] = tid < ncent - 1 ? a.boundaries[tid] : INFINITY;
   if (tid == 0) {
     int sym = 1;
     for (int i = 0; i < ncent - 1; ++i) sym &= (a.boundaries[i] == -a.boundaries[ncent - 2 - i]) ? 1 : 0;
     S.sym = sym;
   }
-  if (tid < 64) {
-    const int i0 = tid & 7, i1 = tid >> 3;
-    float h0 = 0.f, l0 = 0.f, h1 = 0.f, l1 = 0.f;
-    if (i0 < ncent) split16(a.centroids[i0] * kCScale, h0, l0);
-    if (i1 < ncent) split16(a.centroids[i1] * kCScale, h1, l1);
-    S.cpair[0][tid] = pack_h2(h0, h1);
-    S.cpair[1][tid] = pack_h2(l0, l1);
-  }
   if (tid == 0) {
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&S.a1_full[g], 4);
-      mbar_init(&S.a1_free[g], 8);
-      mbar_init(&S.d1_full[g], 1);
-      mbar_init(&S.a2_full[g], 8);
-      mbar_init(&S.d2_full[g], 1);
-      mbar_init(&S.a3_full[g], 8);
-      mbar_init(&S.d3_full[g], 1);
-      mbar_init(&S.d_free[g], 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.a1_full[b], 4);
+      mbar_init(&S.a1_free[b], 16);
     }
+    mbar_init(&S.d1_full, 1);
+    mbar_init(&S.d2_full, 1);
+    mbar_init(&S.d_free, 16);
+    for (int c = 0; c < 8; ++c) mbar_init(&S.kc[c], 4);
+    mbar_init(&S.fin, 1);
     S.abort_flag = 0;
     for (int w = 0; w < 16; ++w) S.ring_head[w] = S.ring_tail[w] = 0;
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(&S.pair[0][q], 2);
-      mbar_init(&S.pair[1][q], 2);
-    }
+    for (int q = 0; q < 4; ++q) mbar_init(&S.pair[q], 4);
     S.epi_done = 0;
     S.progress = 0;
     fence_mbar_init();
@@ -272,76 +278,73 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   const int wg = warp >> 2;
   if (wg == 0) {
     reg_dealloc<kIssRegs>();
-    if (warp < 2) {
-    // ---------------- MMA issuers -----------------------------------------
-    // Warp 0 issues the three GEMMs of epilogue group 0's tiles, warp 1
-    // those of group 1, each in order and sleeping in blocking waits on its
-    // group's operand barriers (a polling issuer shares its sub-partition's
-    // issue slots with the loader and epilogue warps).
-    const int g = warp;
+    if (warp == 0) {
+    // ---------------- MMA issuer -------------------------------------------
+    // One warp issues every product, in order, sleeping in blocking waits on
+    // the operand barriers (a polling issuer shares its sub-partition's
+    // issue slots with the loader and epilogue warps).  GEMM2 goes out
+    // K-step by K-step as the epilogue hands over the chunks of its A
+    // operand, so it runs under the epilogue step that produces it.
     const bool leader = elect_one();
     const uint32_t id1 = idesc_f16(128, 128, false, false);
-    const uint32_t id2 = idesc_f16(128, 128, false, true);
     const uint64_t dpk[2] = {smem_desc(S.pi[0], 2048, 128), smem_desc(S.pi[1], 2048, 128)};
-    const uint64_t dpm[2] = {smem_desc(S.pi[0], 128, 2048), smem_desc(S.pi[1], 128, 2048)};
-    const uint64_t dsk[2] = {smem_desc(S.s[0], 2048, 128), smem_desc(S.s[1], 2048, 128)};
-    const uint64_t da1 = smem_desc(S.a1[g], 2048, 128);
-    const uint32_t d = tbase + g * 256, aop = d + 128;
+    const uint64_t dwk[2] = {smem_desc(S.w[0], 2048, 128), smem_desc(S.w[1], 2048, 128)};
+    const uint64_t da1[2] = {smem_desc(S.a1[0], 2048, 128), smem_desc(S.a1[1], 2048, 128)};
+    const uint32_t d1col = tbase, d2col = tbase + 128;
+    const uint32_t eop = tbase + 256;  // E operand: K-step c hi at 16 c, lo at 16 c + 8
     auto wait_all = [&](uint64_t *bar, uint32_t parity) { return qwait(bar, parity, &S.abort_flag, a); };
-    uint64_t *last_bar = nullptr;
-    uint32_t last_ph = 0u;
-    for (int i = g; i < nlocal; i += 2) {
-      const uint32_t ph = (i >> 1) & 1;
-      // Y = K Pi^T: (K)(Pi_hi + Pi_lo), once K is in and the group has read
-      // its previous tile's accumulators
-      if (!wait_all(&S.a1_full[g], ph)) break;
-      if (i >= 2 && !wait_all(&S.d_free[g], ph ^ 1)) break;
+    for (int j = 0; j < nlocal; ++j) {
+      const int buf = j & 1;
+      const uint32_t ph = j & 1;
+      // Y = K Pi^T: (K)(Pi_hi + Pi_lo), once K is in.  D1 of the previous
+      // tile has been read: every warp loads its D1 columns before handing
+      // over its first E chunk, and all were handed over.
+      if (!wait_all(&S.a1_full[buf], (j >> 1) & 1)) break;
       tc_fence_after();
 #pragma unroll
       for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           if (leader)
-            mma_f16_ss(d, da1 + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4), id1,
+            mma_f16_ss(d1col, da1[buf] + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4), id1,
                        (pr | ks) ? 1u : 0u);
-      if (leader) mma_commit(&S.d1_full[g]);
+      if (leader) mma_commit(&S.d1_full);
       __syncwarp();
-      last_bar = &S.d1_full[g];
-      last_ph = ph;
-      // P = C Pi: C_hi Pi_hi + C_hi Pi_lo + C_lo Pi_hi
-      if (!wait_all(&S.a2_full[g], ph)) break;
-      tc_fence_after();
+      // Z = E W^T: E_hi W_hi + E_hi W_lo + E_lo W_hi, once the previous
+      // tile's D2 has been read; K-steps in the order the chunks are done
+      // (every column quarter's first chunk, then every second one)
+      if (j > 0 && !wait_all(&S.d_free, ph ^ 1u)) break;
+      bool ok = true;
+#pragma unroll 1
+      for (int o = 0; o < 8; ++o) {
+        const int ks = 2 * (o & 3) + (o >> 2);
+        if (!wait_all(&S.kc[ks], ph)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int pr = 0; pr < 3; ++pr)
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
+        for (int pr = 0; pr < 3; ++pr)
           if (leader)
-            mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks, dpm[pr == 1 ? 1 : 0] + (uint64_t)(16 * ks), id2,
-                       (pr | ks) ? 1u : 0u);
-      if (leader) mma_commit(&S.d2_full[g]);
+            mma_f16_ts(d2col, eop + 16 * ks + (pr == 2 ? 8 : 0), dwk[pr == 1 ? 1 : 0] + (uint64_t)((ks * 4096) >> 4),
+                       id1, (o | pr) ? 1u : 0u);
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (leader) mma_commit(&S.d2_full);
       __syncwarp();
-      last_bar = &S.d2_full[g];
-      // Z = R S^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
-      if (!wait_all(&S.a3_full[g], ph)) break;
-      tc_fence_after();
-#pragma unroll
-      for (int pr = 0; pr < 3; ++pr)
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          if (leader)
-            mma_f16_ts(d, aop + (pr == 2 ? 64 : 0) + 8 * ks, dsk[pr == 1 ? 1 : 0] + (uint64_t)((ks * 4096) >> 4),
-                       id1, (pr | ks) ? 1u : 0u);
-      if (leader) mma_commit(&S.d3_full[g]);
-      __syncwarp();
-      last_bar = &S.d3_full[g];
     }
-    // never leave with an MMA in flight: the group's last commit
-    if (last_bar) mbar_wait(last_bar, last_ph);
-    } else {
+    // never leave with an MMA in flight (also after a wait that gave up
+    // between two K-steps): one more commit covers all of them
+    if (leader) mma_commit(&S.fin);
+    __syncwarp();
+    mbar_wait(&S.fin, 0u);
+    } else if (warp >= 2) {
     // ---------------- sign refiners ----------------------------------------
-    // Warp 2 serves the rings of epilogue warps 0-3, warp 3 those of 4-7, in
-    // turn, until every epilogue warp is done and its rings are empty.  Its waits are on the epilogue warps, whose own
-    // waits are bounded; it is bounded too (same limit, measured from the
+    // Warp 2 serves the rings of epilogue warps 0-7, warp 3 those of 8-15, in
+    // turn, until every epilogue warp is done and its rings are empty.  Its
+    // waits are on the epilogue warps, whose own waits are bounded; it is
+    // bounded too (same limit, measured from the
     // last request or finished tile it saw) and gives up by raising the
     // abort flag.
     unsigned long long t_last = globaltimer_ns();
@@ -513,17 +516,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     }
   } else {
     reg_alloc<kEpiRegs>();
-    // ---------------- epilogue groups --------------------------------------
-    // Group g's warps: WG(2 + 2g) takes columns 0-63 of its rows, WG(3 + 2g)
-    // columns 64-127 (half h); the two warps of a TMEM lane quarter share a
-    // row block and meet once per tile (the ||r||^2 halves and the plane
-    // words of the row) through their pair barrier.
+    // ---------------- epilogue ---------------------------------------------
+    // Warp w of WG2-WG5 takes TMEM lane quarter w % 4 (tile rows 32 (w % 4)
+    // .. + 31, a row per thread) and column quarter cq (coordinates 32 cq ..
+    // 32 cq + 31, the K-steps 2 cq and 2 cq + 1 of GEMM2).  The four warps
+    // of a lane quarter meet once per tile for ||r||^2.
     const int ew = warp - 8;  // epilogue warp 0 .. 15 (its refinement ring)
-    const int g = ew >> 3, half = (ew >> 2) & 1;
+    const int cq = ew >> 2;
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;  // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    const uint32_t dcol = tbase + lane_off + g * 256, acol = dcol + 128;
+    const uint32_t d1col = tbase + lane_off + 32 * cq, d2col = d1col + 128;
+    const uint32_t ecol = tbase + lane_off + 256;  // E operand
     constexpr int NC = 1 << MB;
     // upper half of a symmetric codebook's boundaries, for the compare-count
     // bucketize: idx = NC/2 + #{ub < |y|} (y > 0) or NC/2 - 1 - #{ub < |y|}
@@ -533,54 +537,56 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
     for (int k = 0; k < NU; ++k) ub[k] = (k < NC / 2 - 1) ? S.bnd[NC / 2 + k] : INFINITY;
     const bool sym = S.sym != 0;
-    for (int i = g; i < nlocal; i += 2) {
-      const uint32_t ph = (i >> 1) & 1;
-      const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
+    const float kNearZ = a.refine_z * 2097152.f;  // D2 = (S r) x 2^21 (E x 2^13 times W x 2^8)
+    for (int j = 0; j < nlocal; ++j) {
+      const int buf = j & 1;
+      const uint32_t ph = j & 1;
+      const TileInfo ti = tile_info(a, blockIdx.x + j * gridDim.x);
       const bool valid = r < ti.nrow;
       const int pos = a.lens[ti.b] + ti.t0 + r;
       uint8_t *tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
       const int slot = pos % kTile;
       const size_t kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;  // this row's key
-      if (!qwait(&S.d1_full[g], ph, &S.abort_flag, a)) break;
+      if (!qwait(&S.d1_full, ph, &S.abort_flag, a)) break;
       tc_fence_after();
-      const float nk = S.nk[g][r];
-      const int sh = S.sh[g][r];
+      const float nk = S.nk[buf][r];
+      const int sh = S.sh[buf][r];
       // GEMM1 has read the K operand and the norms are in registers: the
-      // loader may refill this group's buffer now (E2 reads the bf16 key
-      // rows from global memory instead), which keeps the loader off the
-      // group's critical path
+      // loader may refill the buffer now
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a1_free[g]);
+      if (lane == 0) mbar_arrive(&S.a1_free[buf]);
       const bool zero = !(nk > 0.f);
       const float rnk = zero ? 0.f : 1.f / nk;
       const float inv1 = ldexpf(rnk, -(sh + 10));  // y = Y 2^-(s+10) / ||k||
+      const float inv13 = inv1 * kEScale;
       // a zero key gets y = -inf everywhere, which every bucketize below
-      // maps to code 0 (its C operand is never used: E2 zeroes its residual)
+      // maps to code 0; its E row is finite garbage (D1 = 0, scale 0) whose
+      // products stay in its own row, and its signs and ||r|| are zeroed
       const float ybias = zero ? -INFINITY : 0.f;
-      // ---- E1: y = Pi u, codes, centroid operand C (16 columns at a time,
-      // the next chunk's TMEM load in flight while this one is processed) ----
-      uint32_t planes[3][2];
+      // ---- E1: y = Pi u, codes, E = (y - c) x 2^13 handed to GEMM2 a K-step
+      // (16 coordinates) at a time, ||r||^2 = ||E||^2 ----
+      uint32_t pw[3] = {0u, 0u, 0u};
+      float rr = 0.f;  // ||r||^2 x 2^26 over this quarter
       uint32_t dA[16], dB[16];
       // The codebook's shape is decided once per tile, outside the element
       // loop: a branch per element would keep the compiler from interleaving
       // the elements' dependent chains.
       auto e1 = [&](auto sym_c) {
         constexpr bool SYM = decltype(sym_c)::value;
-        tmem_ld16(dcol + 64 * half, dA);
+        tmem_ld16(d1col, dA);
+        tmem_ld16(d1col + 16, dB);
         tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = 4 * half + cc;
-          uint32_t(&d)[16] = (cc & 1) ? dB : dA;
-          if (cc < 3) tmem_ld16(dcol + 16 * (c + 1), (cc & 1) ? dA : dB);
-          uint32_t hw[8], lw[8];
-          uint32_t pw[3] = {0u, 0u, 0u};
+        for (int cc = 0; cc < 2; ++cc) {
+          const uint32_t(&d)[16] = cc ? dB : dA;
+          uint32_t hl[16];  // hi parts (columns 0-7), lo parts (8-15)
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
-            int ix[2];
+            float ev[2];
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
-              const float y = fmaf(__uint_as_float(d[e + x]), inv1, ybias);
+              const float dv = __uint_as_float(d[e + x]);
+              const float y = fmaf(dv, inv1, ybias);
               int idx;  // #{boundaries < y}
               if constexpr (SYM) {
                 const float ay = fabsf(y);
@@ -594,125 +600,69 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                 for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
               }
 #pragma unroll
-              for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (e + x);
-              ix[x] = idx;
+              for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (16 * cc + e + x);
+              // E = (y - c) 2^13 from D1 in one rounding
+              ev[x] = fmaf(dv, inv13, -S.cent13[idx]);
+              rr = fmaf(ev[x], ev[x], rr);
             }
-            const int pi2 = ix[0] + 8 * ix[1];
-            hw[e >> 1] = S.cpair[0][pi2];
-            lw[e >> 1] = S.cpair[1][pi2];
+            const __half2 hh = __floats2half2_rn(ev[0], ev[1]);
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(ev[0] - hf.x, ev[1] - hf.y);
+            hl[e >> 1] = *reinterpret_cast<const uint32_t *>(&hh);
+            hl[8 + (e >> 1)] = *reinterpret_cast<const uint32_t *>(&ll);
           }
-          tmem_st8(acol + 8 * c, hw);
-          tmem_st8(acol + 64 + 8 * c, lw);
-#pragma unroll
-          for (int p = 0; p < 3; ++p) {
-            if (cc & 1) planes[p][cc >> 1] |= pw[p] << 16;
-            else planes[p][cc >> 1] = pw[p];
-          }
-          if (cc < 3) tmem_wait_ld();
+          tmem_st16(ecol + 16 * (2 * cq + cc), hl);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.kc[2 * cq + cc]);
         }
       };
       if (sym) e1(std::true_type{});
       else e1(std::false_type{});
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a2_full[g]);
-      if (valid)  // this half's two words of every code plane row
+      if (valid)  // this warp's word of every code plane row
 #pragma unroll
         for (int p = 0; p < MB; ++p)
-          *reinterpret_cast<uint2 *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 8 * half) =
-              make_uint2(planes[p][0], planes[p][1]);
-      // ---- E2: r = u - Pi^T c, ||r||, residual operand R ----
-      // this half of the key row (bf16, 16-byte loads), fetched while GEMM2 runs
-      uint4 krow[8];
-      {
-        const uint4 *src =
-            reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + kbase) + 8 * half;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) krow[j] = valid ? src[j] : make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (!qwait(&S.d2_full[g], ph, &S.abort_flag, a)) break;
-      tc_fence_after();
-      float rr = 0.f;  // ||r||^2 x 2^26 over this half
-      const float inv2r = rnk * kRScale;  // u x 2^13 = k ||k||^-1 2^13
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * half + cc;
-        tmem_ld16(dcol + 16 * c, dA);
-        tmem_wait_ld();
-        uint32_t hw[8], lw[8];
-#pragma unroll
-        for (int c8 = 0; c8 < 2; ++c8) {
-          const __nv_bfloat162 *kh = reinterpret_cast<const __nv_bfloat162 *>(&krow[2 * cc + c8]);
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 kf = __bfloat1622float2(kh[e2]);
-            const int e = 8 * c8 + 2 * e2;
-            // r x 2^13 = u 2^13 - (Pi^T c) 2^13, with D = (Pi^T c) 2^26
-            const float s0 = zero ? 0.f : fmaf(__uint_as_float(dA[e]), -1.220703125e-04f, kf.x * inv2r);
-            const float s1 = zero ? 0.f : fmaf(__uint_as_float(dA[e + 1]), -1.220703125e-04f, kf.y * inv2r);
-            rr = fmaf(s0, s0, rr);
-            rr = fmaf(s1, s1, rr);
-            const __half2 hh = __floats2half2_rn(s0, s1);
-            const float2 hf = __half22float2(hh);
-            const __half2 ll = __floats2half2_rn(s0 - hf.x, s1 - hf.y);
-            hw[4 * c8 + e2] = *reinterpret_cast<const uint32_t *>(&hh);
-            lw[4 * c8 + e2] = *reinterpret_cast<const uint32_t *>(&ll);
-          }
-        }
-        tmem_st8(acol + 8 * c, hw);
-        tmem_st8(acol + 64 + 8 * c, lw);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      S.rrpart[g][ph][half][r] = rr;
+          *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = pw[p];
+      S.rrq[ph][cq][r] = rr;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&S.a3_full[g]);
-        mbar_arrive(&S.pair[g][q4]);  // this half's planes and ||r||^2 are written
-      }
-      // ---- E3: signs of z = S r, norms ----
-      if (!qwait(&S.d3_full[g], ph, &S.abort_flag, a)) break;
+      if (lane == 0) mbar_arrive(&S.pair[q4]);  // this quarter's ||r||^2 is written
+      // ---- E2: signs of z = S r = W (y - c), norms ----
+      if (!qwait(&S.d2_full, ph, &S.abort_flag, a)) break;
       tc_fence_after();
-      uint32_t sw[2] = {0u, 0u};
-      uint32_t nearw[2] = {0u, 0u};  // |S r| below the refinement threshold
-      // D = (S r) x 2^21 (R x 2^13 times S x 2^8)
-      const float kNearZ = a.refine_z * 2097152.f;
-      tmem_ld16(dcol + 64 * half, dA);
+      tmem_ld16(d2col, dA);
+      tmem_ld16(d2col + 16, dB);
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.d_free);  // D2 is in registers
+      uint32_t sw = 0u;
+      uint32_t nearw = 0u;  // |S r| below the refinement threshold
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * half + cc;
-        uint32_t(&d)[16] = (cc & 1) ? dB : dA;
-        if (cc < 3) tmem_ld16(dcol + 16 * (c + 1), (cc & 1) ? dA : dB);
-        uint32_t wv = 0u, nv = 0u;
+      for (int cc = 0; cc < 2; ++cc) {
+        const uint32_t(&d)[16] = cc ? dB : dA;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float z = __uint_as_float(d[e]);
-          wv |= (z >= 0.f ? 1u : 0u) << e;
-          nv |= (fabsf(z) < kNearZ ? 1u : 0u) << e;
+          sw |= (z >= 0.f ? 1u : 0u) << (16 * cc + e);
+          nearw |= (fabsf(z) < kNearZ ? 1u : 0u) << (16 * cc + e);
         }
-        sw[cc >> 1] |= (zero ? 0u : wv) << (16 * (cc & 1));
-        nearw[cc >> 1] |= (zero || !valid ? 0u : nv) << (16 * (cc & 1));
-        if (cc < 3) tmem_wait_ld();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.d_free[g]);
-      // the other half's plane words and ||r||^2 half
-      if (!qwait(&S.pair[g][q4], ph, &S.abort_flag, a)) break;
-      if (valid) {
-        *reinterpret_cast<uint2 *>(tp + L.signs + slot * kRowBytes + 8 * half) = make_uint2(sw[0], sw[1]);
-        if (half == 0) {
-          const float rr2 = rr + S.rrpart[g][ph][1][r];
-          const float rn = zero ? 0.f : sqrtf(rr2) * (1.f / kRScale);
-          *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) =
-              __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
+      if (zero) sw = 0u;
+      if (zero || !valid) nearw = 0u;
+      if (valid) *reinterpret_cast<uint32_t *>(tp + L.signs + slot * kRowBytes + 4 * cq) = sw;
+      if (cq == 0) {
+        // the other quarters' ||r||^2
+        if (!qwait(&S.pair[q4], ph, &S.abort_flag, a)) break;
+        if (valid) {
+          const float rr2 = (rr + S.rrq[ph][1][r]) + (S.rrq[ph][2][r] + S.rrq[ph][3][r]);
+          const float rn = zero ? 0.f : sqrtf(rr2) * (1.f / kEScale);
+          *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) = __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
         }
       }
       // sketch components next to zero: handed to the float64 refiner, which
       // patches the sign words stored above (at most kRingCap rows at a time)
-      unsigned rest = __ballot_sync(0xffffffffu, (nearw[0] | nearw[1]) != 0u);
+      unsigned rest = __ballot_sync(0xffffffffu, nearw != 0u);
       bool stop = false;
       while (rest) {
         const int tail = S.ring_tail[ew];
@@ -726,7 +676,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         if ((chunk >> lane) & 1u) {
           RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) q.near[w] = (w >> 1) == half ? nearw[w & 1] : 0u;
+          for (int w = 0; w < 4; ++w) q.near[w] = w == cq ? nearw : 0u;
           q.kbase = kbase;
           q.planes = (unsigned long long)(tp + L.kplanes + slot * kRowBytes);
           q.signs = (unsigned long long)(tp + L.signs + slot * kRowBytes);
