@@ -14,21 +14,24 @@
 // separate bandwidth-bound kernel launched just before this one
 // (quantize_values.cu).
 //
-// Precision.  A bf16 key is exact in fp16 once scaled per vector by 2^s
-// (largest |k| 2^s in [2^14, 2^15)); Pi, W and E are split into fp16 hi +
-// lo parts (scaled so no part is subnormal where it matters), and each
-// product takes the significant hi/lo terms with f32 accumulation: about 22
-// bits per operand, the error of an fp32 mat-vec.  E is formed from the
-// accumulator in one rounding (fma(Y, 2^13 / (2^(s+10) ||k||), -c 2^13)).
+// Precision.  GEMM1 multiplies the bf16 key rows by Pi split into three bf16
+// parts whose sum is Pi exactly, so every product is exact and only the f32
+// accumulation rounds.  W and E are split into fp16 hi + lo parts (scaled
+// so no part is subnormal where it matters) and GEMM2 takes the three
+// significant hi/lo terms with f32 accumulation: about 22 bits per operand,
+// the error of an fp32 mat-vec.  E is formed from the accumulator in one
+// rounding (fma(Y, 2^13 / ||k||, -c 2^13)).
 //
 // Tiles are 128 consecutive new tokens of one (sequence, KV head), so every
 // record section a tile writes is one contiguous run of the cache.
 //
-// Pipeline.  Tensor memory holds the accumulators D1 (columns 0-127) and D2
-// (128-255) and GEMM2's A operand E (256-383: fp16 hi and lo parts, 16
-// columns a K-step).  The epilogue hands E to the issuer a K-step at a time
-// (one barrier per K-step), so GEMM2 runs under E1, and the next tile's
-// GEMM1 runs while this tile's signs are read.
+// Pipeline.  Tensor memory holds the accumulator D1 (columns 0-127), two D2
+// buffers (128-255, 256-383) and GEMM2's A operand E (384-511: fp16 hi and
+// lo parts, 16 columns a K-step).  The epilogue hands E to the issuer a
+// K-step at a time (one barrier per K-step), so GEMM2 runs under E1; the
+// next tile's GEMM1 goes out as soon as every warp holds its D1 columns;
+// and tile j's signs are read after E1 of tile j + 1, so the end of GEMM2
+// runs while the epilogue works on the next tile.
 //
 // Warp roles (768 threads, by warpgroup):
 //   WG0  warp 0       MMA issuer (one elected lane), sleeping in blocking
@@ -39,9 +42,9 @@
 //                     each epilogue warp hands such rows over through its own
 //                     ring in shared memory and a refiner patches the stored
 //                     sign words
-//   WG1  warps 4-7    loader: K rows -> scaled fp16 A operand + norms in
-//                     shared memory (two buffers); the epilogue releases a
-//                     buffer as soon as GEMM1 has read it
+//   WG1  warps 4-7    loader: the next tile's bf16 K rows -> the A operand
+//                     buffer (cp.async) as soon as GEMM1 has read it, and
+//                     their norms
 //   WG2-WG5           epilogue: thread = tile row = TMEM lane; warp w takes
 //                     lane quarter w % 4 and one quarter of the columns
 // setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
@@ -68,8 +71,7 @@ constexpr int kQtRegs = 80;      // registers a thread at launch (65536 / 768, r
 // setmaxnreg shares: WG0 (issuers, refiners), WG1 (loader), WG2-5 (epilogue)
 constexpr int kIssRegs = 56, kLoadRegs = 72, kEpiRegs = 88;
 constexpr int kRingCap = 8;      // refinement requests per epilogue warp in flight
-constexpr int kMat16 = 128 * 128 * 2;  // one fp16 128 x 128 operand (32 KB)
-constexpr float kPiScale = 1024.f;     // Pi parts are stored x 2^10
+constexpr int kMat16 = 128 * 128 * 2;  // one 16-bit 128 x 128 operand (32 KB)
 constexpr double kWScale = 256.0;     // W = S Pi^T parts x 2^8
 constexpr float kEScale = 8192.f;      // E = y - c parts x 2^13
 
@@ -93,21 +95,21 @@ struct RefineReq {
 };
 
 struct QtSmem {
-  alignas(1024) uint8_t pi[2][kMat16];  // Pi x 2^10: hi, lo
-  alignas(1024) uint8_t w[2][kMat16];   // W = S Pi^T x 2^8: hi, lo
-  alignas(1024) uint8_t a1[2][kMat16];  // K rows x 2^s (fp16), double-buffered by tile
-  float nk[2][128];
-  int sh[2][128];
+  alignas(1024) uint8_t pi[3][kMat16];  // Pi as three bf16 parts (their sum is Pi exactly)
+  alignas(1024) uint8_t w[2][kMat16];   // W = S Pi^T x 2^8: fp16 hi, lo
+  alignas(1024) uint8_t a1[kMat16];     // the tile's bf16 K rows
+  float nk[2][128];                     // ||k|| by tile parity
   float cent[8];
   float cent13[8];               // centroids x 2^13
   float bnd[8];                  // ascending, padded with +inf
   int sym;                       // boundaries exactly antisymmetric (b[i] == -b[nb - 1 - i])
-  // a1_full / a1_free: a K operand buffer is loaded / read by GEMM1 and its
-  // norms taken; d1_full / d2_full: a tile's GEMM1 / GEMM2 is complete;
-  // d_free: the epilogue has read D2; kc[c]: K-step c of the tile's E
-  // operand is in tensor memory; fin: the issuer's last commit (every MMA
-  // it issued is done)
-  uint64_t a1_full[2], a1_free[2], d1_full, d2_full, d_free, kc[8], fin;
+  // a1_full / a1_free: the K operand is loaded / has been read by GEMM1;
+  // d1_full / d2_full[b]: a tile's GEMM1 / GEMM2 (into D2
+  // buffer b) is complete; d1_read: every epilogue warp holds its D1
+  // columns; d_free[b]: the epilogue has read D2 buffer b; kc[c]: K-step c
+  // of the tile's E operand is in tensor memory; fin: the issuer's last
+  // commit (every MMA it issued is done)
+  uint64_t a1_full, a1_free, d1_full, d2_full[2], d1_read, d_free[2], kc[8], fin;
   uint32_t tmem_base;
   volatile int abort_flag;
   // refinement rings, one per epilogue warp (single producer, the refiner
@@ -115,11 +117,10 @@ struct QtSmem {
   RefineReq ring[16][kRingCap];
   volatile int ring_head[16], ring_tail[16];
   volatile int epi_done;  // epilogue warps past their last tile
-  // [tile parity][column quarter][row]: ||r||^2 x 2^26 over a quarter of a
-  // row (by parity, so a warp that runs a tile ahead cannot overwrite a value
-  // that is yet to be read: that would take the reader's next hand-over)
-  float rrq[2][4][128];
-  uint64_t pair[4];         // [lane quarter]: the four column quarters of a row block meet
+  // [tile mod 4][column quarter][row]: ||r||^2 x 2^26 over a quarter of a
+  // row (the reader takes tile t's values while the others write t + 1's)
+  float rrq[4][4][128];
+  uint64_t pair[2][4];      // [tile parity][lane quarter]: the four column quarters of a row block meet
   volatile int progress;  // changes whenever an epilogue warp finishes a tile
 };
 
@@ -180,16 +181,6 @@ __device__ __forceinline__ bool ring_room(QtSmem &S, int ew, int upto, const App
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ uint32_t pack_h2(float lo_elem, float hi_elem) {
-  const __half2 h = __floats2half2_rn(lo_elem, hi_elem);
-  return *reinterpret_cast<const uint32_t *>(&h);
-}
-
-// hi + lo fp16 parts of x (already scaled)
-__device__ __forceinline__ void split16(float x, float &hi, float &lo) {
-  hi = __half2float(__float2half_rn(x));
-  lo = x - hi;
-}
 
 template <int MB>
 __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid_constant__ AppendArgs a) {
@@ -216,14 +207,19 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     const double2 w0 = wp[0], w1 = wp[1], w2 = wp[2], w3 = wp[3];
     const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     const double wv[8] = {w0.x, w0.y, w1.x, w1.y, w2.x, w2.y, w3.x, w3.y};
-    uint32_t ph[4], pl[4], wh[4], wl[4];
+    uint32_t pp3[3][4], wh[4], wl[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float h0, l0, h1, l1;
-      split16(pv[2 * e] * kPiScale, h0, l0);
-      split16(pv[2 * e + 1] * kPiScale, h1, l1);
-      ph[e] = pack_h2(h0, h1);
-      pl[e] = pack_h2(l0, l1);
+      // x = p1 + p2 + p3 exactly: each remainder is exact in fp32 and the
+      // last has at most 8 significant bits
+      float r0 = pv[2 * e], r1 = pv[2 * e + 1];
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(r0, r1);
+        pp3[q][e] = *reinterpret_cast<const uint32_t *>(&b2);
+        r0 -= __low2float(b2);
+        r1 -= __high2float(b2);
+      }
       const double x0 = wv[2 * e] * kWScale, x1 = wv[2 * e + 1] * kWScale;
       const __half hh0 = __double2half(x0), hh1 = __double2half(x1);
       const __half ll0 = __double2half(x0 - (double)__half2float(hh0));
@@ -232,8 +228,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       wh[e] = *reinterpret_cast<const uint32_t *>(&hw2);
       wl[e] = *reinterpret_cast<const uint32_t *>(&lw2);
     }
-    *reinterpret_cast<uint4 *>(S.pi[0] + blk_off(i, j0)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-    *reinterpret_cast<uint4 *>(S.pi[1] + blk_off(i, j0)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+      *reinterpret_cast<uint4 *>(S.pi[q] + blk_off(i, j0)) = make_uint4(pp3[q][0], pp3[q][1], pp3[q][2], pp3[q][3]);
     *reinterpret_cast<uint4 *>(S.w[0] + blk_off(i, j0)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
     *reinterpret_cast<uint4 *>(S.w[1] + blk_off(i, j0)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
   }
@@ -248,18 +245,22 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     S.sym = sym;
   }
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&S.a1_full[b], 4);
-      mbar_init(&S.a1_free[b], 16);
-    }
+    mbar_init(&S.a1_full, 4);
+    mbar_init(&S.a1_free, 1);
     mbar_init(&S.d1_full, 1);
-    mbar_init(&S.d2_full, 1);
-    mbar_init(&S.d_free, 16);
+    mbar_init(&S.d1_read, 16);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.d2_full[b], 1);
+      mbar_init(&S.d_free[b], 16);
+    }
     for (int c = 0; c < 8; ++c) mbar_init(&S.kc[c], 4);
     mbar_init(&S.fin, 1);
     S.abort_flag = 0;
     for (int w = 0; w < 16; ++w) S.ring_head[w] = S.ring_tail[w] = 0;
-    for (int q = 0; q < 4; ++q) mbar_init(&S.pair[q], 4);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&S.pair[0][q], 4);
+      mbar_init(&S.pair[1][q], 4);
+    }
     S.epi_done = 0;
     S.progress = 0;
     fence_mbar_init();
@@ -287,33 +288,52 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     // operand, so it runs under the epilogue step that produces it.
     const bool leader = elect_one();
     const uint32_t id1 = idesc_f16(128, 128, false, false);
-    const uint64_t dpk[2] = {smem_desc(S.pi[0], 2048, 128), smem_desc(S.pi[1], 2048, 128)};
+    const uint32_t idb = idesc_f16(128, 128, false, false) | (1u << 7) | (1u << 10);  // bf16 A and B
+    const uint64_t dpk[3] = {smem_desc(S.pi[0], 2048, 128), smem_desc(S.pi[1], 2048, 128),
+                             smem_desc(S.pi[2], 2048, 128)};
     const uint64_t dwk[2] = {smem_desc(S.w[0], 2048, 128), smem_desc(S.w[1], 2048, 128)};
-    const uint64_t da1[2] = {smem_desc(S.a1[0], 2048, 128), smem_desc(S.a1[1], 2048, 128)};
-    const uint32_t d1col = tbase, d2col = tbase + 128;
-    const uint32_t eop = tbase + 256;  // E operand: K-step c hi at 16 c, lo at 16 c + 8
+    const uint64_t da1 = smem_desc(S.a1, 2048, 128);
+    const uint32_t d1col = tbase;      // D1; D2 buffers at 128, 256
+    const uint32_t eop = tbase + 384;  // E operand: K-step c hi at 16 c, lo at 16 c + 8
     auto wait_all = [&](uint64_t *bar, uint32_t parity) { return qwait(bar, parity, &S.abort_flag, a); };
-    for (int j = 0; j < nlocal; ++j) {
-      const int buf = j & 1;
-      const uint32_t ph = j & 1;
-      // Y = K Pi^T: (K)(Pi_hi + Pi_lo), once K is in.  D1 of the previous
-      // tile has been read: every warp loads its D1 columns before handing
-      // over its first E chunk, and all were handed over.
-      if (!wait_all(&S.a1_full[buf], (j >> 1) & 1)) break;
+    // non-blocking: has every lane seen the phase complete?
+    auto ready = [&](uint64_t *bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test(bar, parity)); };
+    // Y = K Pi^T of tile t into D1: K (Pi_1 + Pi_2 + Pi_3), bf16 products
+    // exact in the f32 accumulator; its commit also frees the K buffer
+    auto gemm1 = [&](int t) {
       tc_fence_after();
 #pragma unroll
-      for (int pr = 0; pr < 2; ++pr)
+      for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           if (leader)
-            mma_f16_ss(d1col, da1[buf] + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4), id1,
+            mma_f16_ss(d1col, da1 + (uint64_t)((ks * 4096) >> 4), dpk[pr] + (uint64_t)((ks * 4096) >> 4), idb,
                        (pr | ks) ? 1u : 0u);
-      if (leader) mma_commit(&S.d1_full);
+      if (leader) {
+        mma_commit(&S.d1_full);
+        mma_commit(&S.a1_free);
+      }
       __syncwarp();
-      // Z = E W^T: E_hi W_hi + E_hi W_lo + E_lo W_hi, once the previous
-      // tile's D2 has been read; K-steps in the order the chunks are done
-      // (every column quarter's first chunk, then every second one)
-      if (j > 0 && !wait_all(&S.d_free, ph ^ 1u)) break;
+    };
+    if (nlocal > 0 && wait_all(&S.a1_full, 0u)) gemm1(0);
+    for (int j = 0; j < nlocal; ++j) {
+      const int buf = j & 1;
+      const uint32_t ph = j & 1;
+      // GEMM1 of tile j + 1 goes out as soon as every warp holds its D1
+      // columns of tile j and that tile's K is in: before GEMM2 of tile j
+      // where it can, between its K-steps or after it otherwise
+      if (!wait_all(&S.d1_read, ph)) break;
+      bool g1 = j + 1 < nlocal;
+      const uint32_t nph = (j + 1) & 1;
+      if (g1 && ready(&S.a1_full, nph)) {
+        gemm1(j + 1);
+        g1 = false;
+      }
+      // Z = E W^T: E_hi W_hi + E_hi W_lo + E_lo W_hi into D2 buffer j % 2,
+      // once tile j - 2's D2 has been read; K-steps in the order the chunks
+      // are done (every column quarter's first chunk, then every second one)
+      const uint32_t d2col = tbase + 128 + 128 * buf;
+      if (j >= 2 && !wait_all(&S.d_free[buf], ((j - 2) >> 1) & 1)) break;
       bool ok = true;
 #pragma unroll 1
       for (int o = 0; o < 8; ++o) {
@@ -329,10 +349,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
             mma_f16_ts(d2col, eop + 16 * ks + (pr == 2 ? 8 : 0), dwk[pr == 1 ? 1 : 0] + (uint64_t)((ks * 4096) >> 4),
                        id1, (o | pr) ? 1u : 0u);
         __syncwarp();
+        if (g1 && ready(&S.a1_full, nph)) {
+          gemm1(j + 1);
+          g1 = false;
+        }
       }
       if (!ok) break;
-      if (leader) mma_commit(&S.d2_full);
+      if (leader) mma_commit(&S.d2_full[buf]);
       __syncwarp();
+      if (g1) {
+        if (!wait_all(&S.a1_full, nph)) break;
+        gemm1(j + 1);
+      }
     }
     // never leave with an MMA in flight (also after a wait that gave up
     // between two K-steps): one more commit covers all of them
@@ -428,106 +456,62 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   } else if (wg == 1) {
     reg_dealloc<kLoadRegs>();
     // ---------------- loader -----------------------------------------------
-    // A warp takes 8 rows at a time (one 8-row group of the operand): lane
-    // (row rr = lane / 4, channel quarter q = lane % 4) holds channels
-    // 32q .. 32q + 31.  Values are quantized by their own kernel, so the
-    // loader reads keys only; the rows of the next two steps are in flight
-    // while this step's are converted.
-    const int w = warp - 4, rr = lane >> 2, q = lane & 3;
-    // rows of step u = 4 i + pass
-    auto fetch = [&](int u, uint4 (&kr)[4]) {
-      const int i = u >> 2, pass = u & 3;
-      bool valid = i < nlocal;
-      size_t base = 0;
-      if (valid) {
-        const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
-        const int r = 32 * pass + 8 * w + rr;
-        valid = r < ti.nrow;
-        base = ((((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD + 32 * q);
-      }
-      const uint4 *ks = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k) + base);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) kr[c] = valid ? ks[c] : make_uint4(0u, 0u, 0u, 0u);
-    };
-    uint4 kr[4], k1[4];
-    fetch(0, kr);
-    fetch(1, k1);
+    // Warp w takes tile rows 32 w .. 32 w + 31.  Once GEMM1 has read the K
+    // buffer, the next tile's bf16 rows are copied by cp.async straight into
+    // it at their canonical places (an instruction covers 8 rows x 4 16-byte
+    // chunks), so all of a tile's loads are in flight together; then each
+    // lane takes its row's norm.  Rows past the tile's end are zero-filled.
+    const int w = warp - 4;
+    const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(a.k);
     for (int i = 0; i < nlocal; ++i) {
-      const int g = i & 1;
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
-      uint8_t *a1 = S.a1[g];
-      bool stop = false;
-#pragma unroll 1
-      for (int pass = 0; pass < 4; ++pass) {
-        uint4 k2[4];
-        fetch(4 * i + pass + 2, k2);
-        if (pass == 0 && i >= 2 && !qwait(&S.a1_free[g], ((i - 2) >> 1) & 1, &S.abort_flag, a)) {
-          stop = true;
-          break;
-        }
-        const int r = 32 * pass + 8 * w + rr;
-        // ---- key: norm, per-vector scale, fp16 operand ----
-        float ss = 0.f, mx = 0.f;
+      if (i >= 1 && !qwait(&S.a1_free, (i - 1) & 1, &S.abort_flag, a)) break;
+#pragma unroll 4
+      for (int it = 0; it < 16; ++it) {
+        const int row = 32 * w + 8 * (it >> 2) + (lane & 7);
+        const int ch = 4 * (it & 3) + (lane >> 3);  // channels 8 ch .. 8 ch + 7
+        const bool valid = row < ti.nrow;
+        const size_t off = valid ? (((size_t)ti.b * a.T + ti.t0 + row) * a.h_kv + ti.h) * kD + 8 * ch : 0;
+        cp_async16_zfill(S.a1 + blk_off(row, 8 * ch), kg + off, valid);
+      }
+      cp_async_wait_all();
+      __syncwarp();
+      const int row = 32 * w + lane;
+      float ss = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(S.a1 + blk_off(row, 8 * c));
+        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[c]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(p2[e]);
-            ss = fmaf(f.x, f.x, ss);
-            ss = fmaf(f.y, f.y, ss);
-            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-          }
-        }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float nk = sqrtf(ss);
-        const int sh = mx > 0.f ? min(14 - ilogbf(mx), 127) : 0;
-        const float f2 = __uint_as_float((uint32_t)(sh + 127) << 23);  // 2^sh
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[c]);
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(p2[e]);
-            o[e] = pack_h2(f.x * f2, f.y * f2);
-          }
-          *reinterpret_cast<uint4 *>(a1 + blk_off(r, 32 * q + 8 * c)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        if (q == 0) {
-          S.nk[g][r] = nk;
-          S.sh[g][r] = sh;
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          kr[c] = k1[c];
-          k1[c] = k2[c];
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(p2[e]);
+          ss = fmaf(f.x, f.x, ss);
+          ss = fmaf(f.y, f.y, ss);
         }
       }
-      if (stop) break;
+      S.nk[i & 1][row] = sqrtf(ss);
       fence_proxy_async_smem();
       __syncwarp();
       // (a test of the timeout path withholds the hand-off: the MMA issuer's
       // bounded wait on it then runs out)
-      if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full[g]);
+      if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full);
     }
   } else {
     reg_alloc<kEpiRegs>();
     // ---------------- epilogue ---------------------------------------------
     // Warp w of WG2-WG5 takes TMEM lane quarter w % 4 (tile rows 32 (w % 4)
     // .. + 31, a row per thread) and column quarter cq (coordinates 32 cq ..
-    // 32 cq + 31, the K-steps 2 cq and 2 cq + 1 of GEMM2).  The four warps
-    // of a lane quarter meet once per tile for ||r||^2.
+    // 32 cq + 31, the K-steps 2 cq and 2 cq + 1 of GEMM2).  Step j runs E1
+    // of tile j and then E2 of tile j - 1, whose GEMM2 ran under E1 and has
+    // finished by then.  The four warps of a lane quarter meet once per tile
+    // for ||r||^2.
     const int ew = warp - 8;  // epilogue warp 0 .. 15 (its refinement ring)
     const int cq = ew >> 2;
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;  // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    const uint32_t d1col = tbase + lane_off + 32 * cq, d2col = d1col + 128;
-    const uint32_t ecol = tbase + lane_off + 256;  // E operand
+    const uint32_t d1col = tbase + lane_off + 32 * cq;
+    const uint32_t ecol = tbase + lane_off + 384;  // E operand
     constexpr int NC = 1 << MB;
     // upper half of a symmetric codebook's boundaries, for the compare-count
     // bucketize: idx = NC/2 + #{ub < |y|} (y > 0) or NC/2 - 1 - #{ub < |y|}
@@ -538,158 +522,186 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     for (int k = 0; k < NU; ++k) ub[k] = (k < NC / 2 - 1) ? S.bnd[NC / 2 + k] : INFINITY;
     const bool sym = S.sym != 0;
     const float kNearZ = a.refine_z * 2097152.f;  // D2 = (S r) x 2^21 (E x 2^13 times W x 2^8)
-    for (int j = 0; j < nlocal; ++j) {
-      const int buf = j & 1;
-      const uint32_t ph = j & 1;
-      const TileInfo ti = tile_info(a, blockIdx.x + j * gridDim.x);
-      const bool valid = r < ti.nrow;
-      const int pos = a.lens[ti.b] + ti.t0 + r;
-      uint8_t *tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
-      const int slot = pos % kTile;
-      const size_t kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;  // this row's key
-      if (!qwait(&S.d1_full, ph, &S.abort_flag, a)) break;
-      tc_fence_after();
-      const float nk = S.nk[buf][r];
-      const int sh = S.sh[buf][r];
-      // GEMM1 has read the K operand and the norms are in registers: the
-      // loader may refill the buffer now
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a1_free[buf]);
-      const bool zero = !(nk > 0.f);
-      const float rnk = zero ? 0.f : 1.f / nk;
-      const float inv1 = ldexpf(rnk, -(sh + 10));  // y = Y 2^-(s+10) / ||k||
-      const float inv13 = inv1 * kEScale;
-      // a zero key gets y = -inf everywhere, which every bucketize below
-      // maps to code 0; its E row is finite garbage (D1 = 0, scale 0) whose
-      // products stay in its own row, and its signs and ||r|| are zeroed
-      const float ybias = zero ? -INFINITY : 0.f;
-      // ---- E1: y = Pi u, codes, E = (y - c) x 2^13 handed to GEMM2 a K-step
-      // (16 coordinates) at a time, ||r||^2 = ||E||^2 ----
-      uint32_t pw[3] = {0u, 0u, 0u};
-      float rr = 0.f;  // ||r||^2 x 2^26 over this quarter
-      uint32_t dA[16], dB[16];
-      // The codebook's shape is decided once per tile, outside the element
-      // loop: a branch per element would keep the compiler from interleaving
-      // the elements' dependent chains.
-      auto e1 = [&](auto sym_c) {
-        constexpr bool SYM = decltype(sym_c)::value;
-        tmem_ld16(d1col, dA);
-        tmem_ld16(d1col + 16, dB);
+    // the previous tile's row, for its E2
+    bool pv_valid = false, pv_zero = true;
+    uint8_t *pv_tp = nullptr;
+    int pv_slot = 0;
+    size_t pv_kbase = 0;
+    float pv_nk = 0.f;
+    for (int j = 0; j <= nlocal; ++j) {
+      bool valid = false, zero = true;
+      uint8_t *tp = nullptr;
+      int slot = 0;
+      size_t kbase = 0;
+      float nk = 0.f;
+      if (j < nlocal) {
+        const int buf = j & 1;
+        const TileInfo ti = tile_info(a, blockIdx.x + j * gridDim.x);
+        valid = r < ti.nrow;
+        const int pos = a.lens[ti.b] + ti.t0 + r;
+        tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
+        slot = pos % kTile;
+        kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;  // this row's key
+        if (!qwait(&S.d1_full, j & 1, &S.abort_flag, a)) break;
+        tc_fence_after();
+        nk = S.nk[buf][r];
+        zero = !(nk > 0.f);
+        const float inv1 = zero ? 0.f : 1.f / nk;  // y = Y / ||k||
+        const float inv13 = inv1 * kEScale;
+        // a zero key gets y = -inf everywhere, which every bucketize below
+        // maps to code 0; its E row is finite garbage (D1 = 0, scale 0) whose
+        // products stay in its own row, and its signs and ||r|| are zeroed
+        const float ybias = zero ? -INFINITY : 0.f;
+        // ---- E1: y = Pi u, codes, E = (y - c) x 2^13 handed to GEMM2 a
+        // K-step (16 coordinates) at a time, ||r||^2 = ||E||^2 ----
+        uint32_t pw[3] = {0u, 0u, 0u};
+        float rr = 0.f;  // ||r||^2 x 2^26 over this quarter
+        // The codebook's shape is decided once per tile, outside the element
+        // loop: a branch per element would keep the compiler from
+        // interleaving the elements' dependent chains.
+        // GEMM1 of the next tile may overwrite D1 once every warp holds its
+        // columns; E may be overwritten once the previous tile's GEMM2 is done
+        auto e1 = [&](auto sym_c) -> bool {
+          constexpr bool SYM = decltype(sym_c)::value;
+          uint32_t dA[16], dB[16];
+          tmem_ld16(d1col, dA);
+          tmem_ld16(d1col + 16, dB);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.d1_read);
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t(&d)[16] = cc ? dB : dA;
+            uint32_t hl[16];  // hi parts (columns 0-7), lo parts (8-15)
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              float ev[2];
+#pragma unroll
+              for (int x = 0; x < 2; ++x) {
+                const float dv = __uint_as_float(d[e + x]);
+                const float y = fmaf(dv, inv1, ybias);
+                int idx;  // #{boundaries < y}
+                if constexpr (SYM) {
+                  const float ay = fabsf(y);
+                  int cnt = 0;
+#pragma unroll
+                  for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
+                  idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
+                } else {  // any codebook: count the boundaries below y
+                  idx = 0;
+#pragma unroll
+                  for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
+                }
+#pragma unroll
+                for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (16 * cc + e + x);
+                // E = (y - c) 2^13 from D1 in one rounding
+                ev[x] = fmaf(dv, inv13, -S.cent13[idx]);
+                rr = fmaf(ev[x], ev[x], rr);
+              }
+              const __half2 hh = __floats2half2_rn(ev[0], ev[1]);
+              const float2 hf = __half22float2(hh);
+              const __half2 ll = __floats2half2_rn(ev[0] - hf.x, ev[1] - hf.y);
+              hl[e >> 1] = *reinterpret_cast<const uint32_t *>(&hh);
+              hl[8 + (e >> 1)] = *reinterpret_cast<const uint32_t *>(&ll);
+            }
+            if (cc == 0 && j >= 1) {
+              if (!qwait(&S.d2_full[(j - 1) & 1], ((j - 1) >> 1) & 1, &S.abort_flag, a)) return false;
+              tc_fence_after();
+            }
+            tmem_st16(ecol + 16 * (2 * cq + cc), hl);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.kc[2 * cq + cc]);
+          }
+          return true;
+        };
+        if (!(sym ? e1(std::true_type{}) : e1(std::false_type{}))) break;
+        if (valid)  // this warp's word of every code plane row
+#pragma unroll
+          for (int p = 0; p < MB; ++p)
+            *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = pw[p];
+        S.rrq[j & 3][cq][r] = rr;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.pair[j & 1][q4]);  // this quarter's ||r||^2 is written
+      }
+      if (j >= 1) {
+        // ---- E2 of tile t = j - 1: signs of z = S r = W (y - c), norms ----
+        const int t = j - 1, tb = t & 1;
+        const uint32_t tph = (t >> 1) & 1;
+        if (!qwait(&S.d2_full[tb], tph, &S.abort_flag, a)) break;
+        tc_fence_after();
+        uint32_t dA[16], dB[16];
+        tmem_ld16(d1col + 128 + 128 * tb, dA);
+        tmem_ld16(d1col + 128 + 128 * tb + 16, dB);
         tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.d_free[tb]);  // D2 is in registers
+        uint32_t sw = 0u;
+        uint32_t nearw = 0u;  // |S r| below the refinement threshold
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const uint32_t(&d)[16] = cc ? dB : dA;
-          uint32_t hl[16];  // hi parts (columns 0-7), lo parts (8-15)
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float ev[2];
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              const float dv = __uint_as_float(d[e + x]);
-              const float y = fmaf(dv, inv1, ybias);
-              int idx;  // #{boundaries < y}
-              if constexpr (SYM) {
-                const float ay = fabsf(y);
-                int cnt = 0;
-#pragma unroll
-                for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
-                idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
-              } else {  // any codebook: count the boundaries below y
-                idx = 0;
-#pragma unroll
-                for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
-              }
-#pragma unroll
-              for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (16 * cc + e + x);
-              // E = (y - c) 2^13 from D1 in one rounding
-              ev[x] = fmaf(dv, inv13, -S.cent13[idx]);
-              rr = fmaf(ev[x], ev[x], rr);
-            }
-            const __half2 hh = __floats2half2_rn(ev[0], ev[1]);
-            const float2 hf = __half22float2(hh);
-            const __half2 ll = __floats2half2_rn(ev[0] - hf.x, ev[1] - hf.y);
-            hl[e >> 1] = *reinterpret_cast<const uint32_t *>(&hh);
-            hl[8 + (e >> 1)] = *reinterpret_cast<const uint32_t *>(&ll);
+          for (int e = 0; e < 16; ++e) {
+            const float z = __uint_as_float(d[e]);
+            sw |= (z >= 0.f ? 1u : 0u) << (16 * cc + e);
+            nearw |= (fabsf(z) < kNearZ ? 1u : 0u) << (16 * cc + e);
           }
-          tmem_st16(ecol + 16 * (2 * cq + cc), hl);
-          tmem_wait_st();
-          tc_fence_before();
+        }
+        if (pv_zero) sw = 0u;
+        if (pv_zero || !pv_valid) nearw = 0u;
+        if (pv_valid) *reinterpret_cast<uint32_t *>(pv_tp + L.signs + pv_slot * kRowBytes + 4 * cq) = sw;
+        if (cq == 0) {
+          // the four quarters' ||r||^2
+          if (!qwait(&S.pair[tb][q4], tph, &S.abort_flag, a)) break;
+          if (pv_valid) {
+            const float rr2 = (S.rrq[t & 3][0][r] + S.rrq[t & 3][1][r]) + (S.rrq[t & 3][2][r] + S.rrq[t & 3][3][r]);
+            const float rn = pv_zero ? 0.f : sqrtf(rr2) * (1.f / kEScale);
+            *reinterpret_cast<__half2 *>(pv_tp + L.norms + pv_slot * 4) =
+                __halves2half2(__float2half_rn(pv_nk), __float2half_rn(rn));
+          }
+        }
+        // sketch components next to zero: handed to the float64 refiner,
+        // which patches the sign words stored above (at most kRingCap rows
+        // at a time)
+        unsigned rest = __ballot_sync(0xffffffffu, nearw != 0u);
+        bool stop = false;
+        while (rest) {
+          const int tail = S.ring_tail[ew];
+          const int rank = __popc(rest & ((1u << lane) - 1u));
+          const unsigned chunk = __ballot_sync(0xffffffffu, ((rest >> lane) & 1u) && rank < kRingCap);
+          const int n = __popc(chunk);
+          if (!ring_room(S, ew, tail + n, a)) {
+            stop = true;
+            break;
+          }
+          if ((chunk >> lane) & 1u) {
+            RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) q.near[w] = w == cq ? nearw : 0u;
+            q.kbase = pv_kbase;
+            q.planes = (unsigned long long)(pv_tp + L.kplanes + pv_slot * kRowBytes);
+            q.signs = (unsigned long long)(pv_tp + L.signs + pv_slot * kRowBytes);
+          }
+          // the sign rows and the requests, then the new tail
+          __threadfence_block();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S.kc[2 * cq + cc]);
+          if (lane == 0) S.ring_tail[ew] = tail + n;
+          __syncwarp();
+          rest &= ~chunk;
         }
-      };
-      if (sym) e1(std::true_type{});
-      else e1(std::false_type{});
-      if (valid)  // this warp's word of every code plane row
-#pragma unroll
-        for (int p = 0; p < MB; ++p)
-          *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = pw[p];
-      S.rrq[ph][cq][r] = rr;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.pair[q4]);  // this quarter's ||r||^2 is written
-      // ---- E2: signs of z = S r = W (y - c), norms ----
-      if (!qwait(&S.d2_full, ph, &S.abort_flag, a)) break;
-      tc_fence_after();
-      tmem_ld16(d2col, dA);
-      tmem_ld16(d2col + 16, dB);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.d_free);  // D2 is in registers
-      uint32_t sw = 0u;
-      uint32_t nearw = 0u;  // |S r| below the refinement threshold
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const uint32_t(&d)[16] = cc ? dB : dA;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float z = __uint_as_float(d[e]);
-          sw |= (z >= 0.f ? 1u : 0u) << (16 * cc + e);
-          nearw |= (fabsf(z) < kNearZ ? 1u : 0u) << (16 * cc + e);
-        }
+        if (stop) break;
+        if (lane == 0) S.progress = S.progress + 1;
       }
-      if (zero) sw = 0u;
-      if (zero || !valid) nearw = 0u;
-      if (valid) *reinterpret_cast<uint32_t *>(tp + L.signs + slot * kRowBytes + 4 * cq) = sw;
-      if (cq == 0) {
-        // the other quarters' ||r||^2
-        if (!qwait(&S.pair[q4], ph, &S.abort_flag, a)) break;
-        if (valid) {
-          const float rr2 = (rr + S.rrq[ph][1][r]) + (S.rrq[ph][2][r] + S.rrq[ph][3][r]);
-          const float rn = zero ? 0.f : sqrtf(rr2) * (1.f / kEScale);
-          *reinterpret_cast<__half2 *>(tp + L.norms + slot * 4) = __halves2half2(__float2half_rn(nk), __float2half_rn(rn));
-        }
-      }
-      // sketch components next to zero: handed to the float64 refiner, which
-      // patches the sign words stored above (at most kRingCap rows at a time)
-      unsigned rest = __ballot_sync(0xffffffffu, nearw != 0u);
-      bool stop = false;
-      while (rest) {
-        const int tail = S.ring_tail[ew];
-        const int rank = __popc(rest & ((1u << lane) - 1u));
-        const unsigned chunk = __ballot_sync(0xffffffffu, ((rest >> lane) & 1u) && rank < kRingCap);
-        const int n = __popc(chunk);
-        if (!ring_room(S, ew, tail + n, a)) {
-          stop = true;
-          break;
-        }
-        if ((chunk >> lane) & 1u) {
-          RefineReq &q = S.ring[ew][(tail + rank) % kRingCap];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) q.near[w] = w == cq ? nearw : 0u;
-          q.kbase = kbase;
-          q.planes = (unsigned long long)(tp + L.kplanes + slot * kRowBytes);
-          q.signs = (unsigned long long)(tp + L.signs + slot * kRowBytes);
-        }
-        // the sign rows and the requests, then the new tail
-        __threadfence_block();
-        __syncwarp();
-        if (lane == 0) S.ring_tail[ew] = tail + n;
-        __syncwarp();
-        rest &= ~chunk;
-      }
-      if (stop) break;
-      if (lane == 0) S.progress = S.progress + 1;
+      pv_valid = valid;
+      pv_zero = zero;
+      pv_tp = tp;
+      pv_slot = slot;
+      pv_kbase = kbase;
+      pv_nk = nk;
     }
     __syncwarp();
     if (lane == 0) {
