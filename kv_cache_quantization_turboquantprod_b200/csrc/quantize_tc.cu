@@ -43,8 +43,8 @@
 //                     ring in shared memory and a refiner patches the stored
 //                     sign words
 //   WG1  warps 4-7    loader: the next tile's bf16 K rows -> the A operand
-//                     buffer (cp.async) as soon as GEMM1 has read it, and
-//                     their norms
+//                     buffer (TMA tensor copies) as soon as GEMM1 has read
+//                     it, and their norms
 //   WG2-WG5           epilogue: thread = tile row = TMEM lane; warp w takes
 //                     lane quarter w % 4 and one quarter of the columns
 // setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
@@ -52,8 +52,11 @@
 // limit) and answers warp-uniformly; on timeout the CTA raises its abort flag
 // and the device's sticky error word, stops, lets its own MMAs finish, frees
 // TMEM and marks the records it owns with NaN norms.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 
+#include <mutex>
 #include <type_traits>
 
 #include "sm100.cuh"
@@ -103,13 +106,13 @@ struct QtSmem {
   float cent13[8];               // centroids x 2^13
   float bnd[8];                  // ascending, padded with +inf
   int sym;                       // boundaries exactly antisymmetric (b[i] == -b[nb - 1 - i])
-  // a1_full / a1_free: the K operand is loaded / has been read by GEMM1;
-  // d1_full / d2_full[b]: a tile's GEMM1 / GEMM2 (into D2
+  // k_full: the tile's K rows have landed (TMA); a1_full / a1_free: the K
+  // operand and its norms are in / it has been read by GEMM1; d1_full / d2_full[b]: a tile's GEMM1 / GEMM2 (into D2
   // buffer b) is complete; d1_read: every epilogue warp holds its D1
   // columns; d_free[b]: the epilogue has read D2 buffer b; kc[c]: K-step c
   // of the tile's E operand is in tensor memory; fin: the issuer's last
   // commit (every MMA it issued is done)
-  uint64_t a1_full, a1_free, d1_full, d2_full[2], d1_read, d_free[2], kc[8], fin;
+  uint64_t k_full, a1_full, a1_free, d1_full, d2_full[2], d1_read, d_free[2], kc[8], fin;
   uint32_t tmem_base;
   volatile int abort_flag;
   // refinement rings, one per epilogue warp (single producer, the refiner
@@ -183,7 +186,8 @@ __device__ __forceinline__ bool ring_room(QtSmem &S, int ew, int upto, const App
 
 
 template <int MB>
-__global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid_constant__ AppendArgs a) {
+__global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid_constant__ AppendArgs a,
+                                                                   const __grid_constant__ CUtensorMap kmap) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   QtSmem &S = *reinterpret_cast<QtSmem *>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -245,6 +249,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     S.sym = sym;
   }
   if (tid == 0) {
+    mbar_init(&S.k_full, 1);
     mbar_init(&S.a1_full, 4);
     mbar_init(&S.a1_free, 1);
     mbar_init(&S.d1_full, 1);
@@ -456,26 +461,26 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   } else if (wg == 1) {
     reg_dealloc<kLoadRegs>();
     // ---------------- loader -----------------------------------------------
-    // Warp w takes tile rows 32 w .. 32 w + 31.  Once GEMM1 has read the K
-    // buffer, the next tile's bf16 rows are copied by cp.async straight into
-    // it at their canonical places (an instruction covers 8 rows x 4 16-byte
-    // chunks), so all of a tile's loads are in flight together; then each
-    // lane takes its row's norm.  Rows past the tile's end are zero-filled.
+    // Once GEMM1 has read the K buffer, one lane has the TMA engine copy the
+    // next tile's bf16 rows into it: 16 boxes of 8 channels x 128 tokens of
+    // the (channel, head, token, sequence) tensor map, each landing as one
+    // 16-byte column of the canonical operand layout; tokens past the
+    // sequence's end read as zeros.  Then warp w takes the norms of tile
+    // rows 32 w .. 32 w + 31 (a row per lane).
     const int w = warp - 4;
-    const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(a.k);
+    int in_flight = -1;  // a tile whose copies were issued and not yet seen landing
     for (int i = 0; i < nlocal; ++i) {
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
       if (i >= 1 && !qwait(&S.a1_free, (i - 1) & 1, &S.abort_flag, a)) break;
-#pragma unroll 4
-      for (int it = 0; it < 16; ++it) {
-        const int row = 32 * w + 8 * (it >> 2) + (lane & 7);
-        const int ch = 4 * (it & 3) + (lane >> 3);  // channels 8 ch .. 8 ch + 7
-        const bool valid = row < ti.nrow;
-        const size_t off = valid ? (((size_t)ti.b * a.T + ti.t0 + row) * a.h_kv + ti.h) * kD + 8 * ch : 0;
-        cp_async16_zfill(S.a1 + blk_off(row, 8 * ch), kg + off, valid);
+      if (w == 0 && lane == 0) {
+        mbar_arrive_expect_tx(&S.k_full, 16 * 2048);
+#pragma unroll 1
+        for (int ch = 0; ch < 16; ++ch) tma_load_4d(S.a1 + ch * 2048, &kmap, 8 * ch, ti.h, ti.t0, ti.b, &S.k_full);
       }
-      cp_async_wait_all();
       __syncwarp();
+      in_flight = i;
+      if (!qwait(&S.k_full, i & 1, &S.abort_flag, a)) break;
+      in_flight = -1;
       const int row = 32 * w + lane;
       float ss = 0.f;
 #pragma unroll 4
@@ -490,12 +495,14 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         }
       }
       S.nk[i & 1][row] = sqrtf(ss);
-      fence_proxy_async_smem();
       __syncwarp();
       // (a test of the timeout path withholds the hand-off: the MMA issuer's
       // bounded wait on it then runs out)
       if (lane == 0 && !a.test_withhold) mbar_arrive(&S.a1_full);
     }
+    // never leave with a copy in flight (a role gave up while it ran): the
+    // copy engine completes it, so this wait ends
+    if (in_flight >= 0) mbar_wait(&S.k_full, in_flight & 1);
   } else {
     reg_alloc<kEpiRegs>();
     // ---------------- epilogue ---------------------------------------------
@@ -734,7 +741,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 }
 
 template <int MB>
-cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
+cudaError_t launch_qt(const AppendArgs &a, const CUtensorMap &kmap, int grid, cudaStream_t stream) {
   const size_t smem = sizeof(QtSmem);
   static_assert(sizeof(QtSmem) <= 227 * 1024, "shared memory per CTA");
   static_assert((kIssRegs + kLoadRegs) * 128 + kEpiRegs * 512 <= kQtRegs * kQtThreads &&
@@ -749,15 +756,45 @@ cudaError_t launch_qt(const AppendArgs &a, int grid, cudaStream_t stream) {
   e = cudaFuncGetAttributes(&fa, quantize_tc_kernel<MB>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kQtRegs) return cudaErrorInvalidConfiguration;
-  quantize_tc_kernel<MB><<<grid, kQtThreads, smem, stream>>>(a);
+  quantize_tc_kernel<MB><<<grid, kQtThreads, smem, stream>>>(a, kmap);
   return cudaGetLastError();
+}
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// K as a (channel, head, token, sequence) bf16 tensor, boxes of 8 channels
+// x 1 head x 128 tokens x 1 sequence, no swizzle, zero fill out of range.
+cudaError_t encode_k_map(const AppendArgs &a, CUtensorMap *map) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.h_kv, (cuuint64_t)a.T, (cuuint64_t)a.batch};
+  const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)a.h_kv * kD * 2, (cuuint64_t)a.T * a.h_kv * kD * 2};
+  const cuuint32_t box[4] = {8, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(a.k), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 bool quantize_tc_supported(const AppendArgs &a) {
-  return a.d == kD && a.value_mode == TQ_VALUES_GROUP && a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 && a.value_bits >= 2 &&
-         a.value_bits <= 4 && a.T >= 64;
+  // (the K tensor map wants a 16-byte aligned base)
+  return a.d == kD && a.value_mode == TQ_VALUES_GROUP && a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 &&
+         a.value_bits >= 2 && a.value_bits <= 4 && a.T >= 64 && (reinterpret_cast<uintptr_t>(a.k) & 15) == 0;
 }
 
 cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream) {
@@ -770,12 +807,15 @@ cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream) 
   a.total_tiles = total;
   if (total == 0) return cudaSuccess;
   const int grid = total < num_sms ? total : num_sms;
+  CUtensorMap kmap;
+  const cudaError_t em = encode_k_map(a, &kmap);
+  if (em != cudaSuccess) return em;
   const cudaError_t ev = launch_value_quant(a, num_sms, stream);
   if (ev != cudaSuccess) return ev;
   switch (a.key_bits - 1) {
-    case 1: return launch_qt<1>(a, grid, stream);
-    case 2: return launch_qt<2>(a, grid, stream);
-    case 3: return launch_qt<3>(a, grid, stream);
+    case 1: return launch_qt<1>(a, kmap, grid, stream);
+    case 2: return launch_qt<2>(a, kmap, grid, stream);
+    case 3: return launch_qt<3>(a, kmap, grid, stream);
     default: return cudaErrorNotSupported;
   }
 }
