@@ -792,9 +792,11 @@ cudaError_t encode_k_map(const AppendArgs &a, CUtensorMap *map) {
 }  // namespace
 
 bool quantize_tc_supported(const AppendArgs &a) {
-  // (the K tensor map wants a 16-byte aligned base)
+  // (the K tensor map wants a 16-byte aligned base; the value kernel splits
+  // vector slots with 32-bit arithmetic below a sequence)
   return a.d == kD && a.value_mode == TQ_VALUES_GROUP && a.dtype == TQ_BF16 && a.key_bits >= 2 && a.key_bits <= 4 &&
-         a.value_bits >= 2 && a.value_bits <= 4 && a.T >= 64 && (reinterpret_cast<uintptr_t>(a.k) & 15) == 0;
+         a.value_bits >= 2 && a.value_bits <= 4 && a.T >= 64 && (reinterpret_cast<uintptr_t>(a.k) & 15) == 0 &&
+         (long long)a.T * a.h_kv < (1LL << 31);
 }
 
 cudaError_t launch_quantize_tc(AppendArgs &a, int num_sms, cudaStream_t stream) {
