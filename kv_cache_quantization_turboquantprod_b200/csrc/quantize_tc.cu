@@ -738,6 +738,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       }
     }
   }
+  // launched as a dependent of the value kernel: this grid is not complete
+  // before that one is
+  pdl_wait();
 }
 
 template <int MB>
@@ -756,8 +759,10 @@ cudaError_t launch_qt(const AppendArgs &a, const CUtensorMap &kmap, int grid, cu
   e = cudaFuncGetAttributes(&fa, quantize_tc_kernel<MB>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kQtRegs) return cudaErrorInvalidConfiguration;
-  quantize_tc_kernel<MB><<<grid, kQtThreads, smem, stream>>>(a, kmap);
-  return cudaGetLastError();
+  // a programmatic dependent of the value kernel, whose record bytes it
+  // does not touch: it starts as that kernel's blocks drain and waits for
+  // it only before it finishes
+  return launch_pdl(quantize_tc_kernel<MB>, dim3(grid), dim3(kQtThreads), smem, stream, a, kmap);
 }
 
 // The driver's tensor-map encoder, looked up once through the runtime.
