@@ -325,16 +325,23 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   // fill, and the split-major grid runs every unit's first split before any
   // ragged last one); with fewer, longer units, about eight, so the last wave
   // of CTAs is a small part of the call (measured on 4 x 131,072-token
-  // sequences: 0.299 ms at two, 0.270 ms at eight)
+  // sequences: 0.299 ms at two, 0.270 ms at eight) -- but no split shorter
+  // than 32 tiles, whose pipeline fill and merge would dominate (measured on
+  // 8 sequences of 16K-32K tokens, 64 units: 123 us with 19 splits of ~10
+  // tiles, 110 us with 6)
 #ifndef TQ_DECODE_CTAS_PER_SM
 #define TQ_DECODE_CTAS_PER_SM 2
 #endif
 #ifndef TQ_DECODE_CTAS_PER_SM_FEW_UNITS
 #define TQ_DECODE_CTAS_PER_SM_FEW_UNITS 8
 #endif
+#ifndef TQ_DECODE_MIN_TILES_PER_SPLIT
+#define TQ_DECODE_MIN_TILES_PER_SPLIT 32
+#endif
   const long long cps = units >= num_sms ? TQ_DECODE_CTAS_PER_SM : TQ_DECODE_CTAS_PER_SM_FEW_UNITS;
   const long long target = cps * num_sms;
   long long ns = (target + units - 1) / units;
+  ns = std::min(ns, (long long)std::max(ntile / TQ_DECODE_MIN_TILES_PER_SPLIT, 1));
   ns = std::max(1LL, std::min(ns, (long long)std::max(ntile, 1)));
   int tps = ntile > 0 ? (int)((ntile + ns - 1) / ns) : 0;
   int nsplit = tps > 0 ? (ntile + tps - 1) / tps : 1;
