@@ -728,7 +728,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       for (int g = 0; g < G; ++g) {
         const float4 r4 = *reinterpret_cast<const float4 *>(red[g]);
         const float mnew = fmaxf(mrun[g], fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
-        alpha[g] = exp2f(mrun[g] - mnew);
+        // a head that has seen no token yet (causally masked prefill rows)
+        // keeps its empty state: its factor is 1, not exp2(-inf + inf)
+        alpha[g] = mnew == -INFINITY ? 1.f : exp2f(mrun[g] - mnew);
         changed |= (mnew != mrun[g]);
         mrun[g] = mnew;
       }
