@@ -561,7 +561,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         const float ybias = zero ? -INFINITY : 0.f;
         // ---- E1: y = Pi u, codes, E = (y - c) x 2^13 handed to GEMM2 a
         // K-step (16 coordinates) at a time, ||r||^2 = ||E||^2 ----
-        uint32_t pw[3] = {0u, 0u, 0u};
+        // code indices as nibbles (element e in bits 4 (e % 8) of word e / 8),
+        // split into bit-planes once the quarter is done
+        uint32_t nib[4] = {0u, 0u, 0u, 0u};
         float rr = 0.f;  // ||r||^2 x 2^26 over this quarter
         // The codebook's shape is decided once per tile, outside the element
         // loop: a branch per element would keep the compiler from
@@ -600,8 +602,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
                   for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
                 }
-#pragma unroll
-                for (int p = 0; p < MB; ++p) pw[p] |= (uint32_t)((idx >> p) & 1) << (16 * cc + e + x);
+                const int el = 16 * cc + e + x;
+                nib[el >> 3] |= (uint32_t)idx << (4 * (el & 7));
                 // E = (y - c) 2^13 from D1 in one rounding
                 ev[x] = fmaf(dv, inv13, -S.cent13[idx]);
                 rr = fmaf(ev[x], ev[x], rr);
@@ -627,8 +629,19 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         if (!(sym ? e1(std::true_type{}) : e1(std::false_type{}))) break;
         if (valid)  // this warp's word of every code plane row
 #pragma unroll
-          for (int p = 0; p < MB; ++p)
-            *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = pw[p];
+          for (int p = 0; p < MB; ++p) {
+            uint32_t w = 0u;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              // bit p of nibbles 0..7 (bits 4i + p) -> bits 0..7
+              uint32_t v = (nib[q] >> p) & 0x11111111u;
+              v = (v | (v >> 3)) & 0x03030303u;
+              v = (v | (v >> 6)) & 0x000F000Fu;
+              v = (v | (v >> 12)) & 0xFFu;
+              w |= v << (8 * q);
+            }
+            *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = w;
+          }
         S.rrq[j & 3][cq][r] = rr;
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.pair[j & 1][q4]);  // this quarter's ||r||^2 is written
