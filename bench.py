@@ -52,6 +52,16 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _bf16_peak():
+    """Dense bf16 tensor peak in TFLOP/s (burst): measured, else the recipe's fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def _source_hash(files):
     h = hashlib.sha256()
     for f in sorted(files):
@@ -548,11 +558,18 @@ def bench_quantize(args, device):
     vecs = wl.batch * workloads.TOKEN_CHUNK * wl.h_kv
     in_bytes = k.numel() * k.element_size() * 2
     out_bytes = vecs * layer.record_bytes()
+    peak, peak_kind = _bf16_peak()
+    # two d x d products a key vector: y = Pi u and the sketch S r = W (y - c)
+    useful = vecs * 2 * 2 * 128 * 128 / (ms / 1e3) / 1e12
+    # issued: 48 MMAs of 128 x 128 x 16 a 128-vector tile (GEMM1 three bf16
+    # parts of Pi, GEMM2 three hi/lo products), 16-bit operands
+    issued = vecs * (48 * 2 * 128 * 128 * 16 / 128) / (ms / 1e3) / 1e12
     return {"workload": "longctx chunk (4 x 8192 tokens x 8 heads, bf16)",
             "ms_per_chunk": ms, "mvec_s": vecs / (ms / 1e3) / 1e6,
             "gbs": (in_bytes + out_bytes) / (ms / 1e3) / 1e9,
-            # two d x d products a key vector: y = Pi u and the sketch S r = W (y - c)
-            "useful_tflops": vecs * 2 * 2 * 128 * 128 / (ms / 1e3) / 1e12}
+            "useful_tflops": useful, "mma_tflops": issued,
+            "tensor": {"peak_tflops": peak, "peak_kind": peak_kind, "useful_frac": useful / peak,
+                       "mma_frac": issued / peak}}
 
 
 # ---------------------------------------------------------------------------
