@@ -354,7 +354,9 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   const int G = h_q / h_kv;
   P.qblock_bytes =
       decode_tc_supported(key_bits, value_bits, G, value_mode, d) ? decode_tc_qblock_bytes(key_bits, G) : 0;
-  P.total_bytes = P.status_bytes + P.qrot_bytes + P.part_bytes + al((size_t)batch * h_kv * P.qblock_bytes);
+  P.order_bytes = P.qblock_bytes ? al((size_t)batch * h_kv * nsplit * sizeof(int2)) : 0;
+  P.total_bytes =
+      P.status_bytes + P.qrot_bytes + P.part_bytes + al((size_t)batch * h_kv * P.qblock_bytes) + P.order_bytes;
   return P;
 }
 
@@ -364,6 +366,8 @@ void bind_workspace(DecodeArgs &a, const DecodePlan &P, void *workspace) {
   a.qrot = reinterpret_cast<float *>(w + P.status_bytes);
   a.part = reinterpret_cast<float *>(w + P.status_bytes + P.qrot_bytes);
   a.qblocks = w + P.status_bytes + P.qrot_bytes + P.part_bytes;
+  // the work list is the last region
+  a.order = P.order_bytes ? reinterpret_cast<int2 *>(w + P.total_bytes - P.order_bytes) : nullptr;
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {

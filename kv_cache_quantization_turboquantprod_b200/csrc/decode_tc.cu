@@ -288,10 +288,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // split-major grid: every unit's first splits are scheduled before any
   // last (ragged, shorter) split, so the short CTAs fill the tail
-  const int split = blockIdx.z, h = blockIdx.x, b = blockIdx.y;
-  // the query blocks (and the status words) come from the preceding kernel
+  // the query blocks, the status words and the work list come from the
+  // preceding kernel
   pdl_wait();
   pdl_trigger();
+  // this CTA's (split, KV head, sequence): work items largest first, so the
+  // short ones fill the tail
+  int split, h, b, len;
+  {
+    const int units = a.batch * a.h_kv;
+    const int2 it = a.order ? a.order[blockIdx.x] : make_int2((int)blockIdx.x, -1);
+    split = it.x / units;
+    const int u = it.x - split * units;
+    b = u / a.h_kv;
+    h = u - b * a.h_kv;
+    len = it.y;
+  }
   // A codebook whose operand planes fit in tensor memory only once (the
   // query-block kernel decided it): this split runs the SIMT split-K body
   // on 128 threads instead.
@@ -300,8 +312,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     return;
   }
 
-  int len = a.len[b] - a.len_sub;
-  len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
+  if (len < 0) {
+    len = a.len[b] - a.len_sub;
+    len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
+  }
   const int tile0 = split * a.tiles_per_split;
   const int t_begin = tile0 * kTile;
   const int t_end = min(len, (split + 1) * a.tiles_per_split * kTile);
@@ -887,6 +901,77 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // 2^((c % 8) mod 4), so it holds X = round(x_j 2^(F - weight exponent)) as
 // four signed base-128 limbs; F per head keeps |X| < 2^26.
 // ---------------------------------------------------------------------------
+// The decode kernel's work list: items i = split * B * H_kv + b * H_kv + h
+// ordered by their tile count, largest first, equal counts in item order, so
+// the block scheduler hands the longest splits out first and the short ones
+// fill the tail, and equal splits keep the split-major order.  A stable
+// counting sort by one CTA of 256 threads: every item's count computed once
+// (in parallel, into shared memory), a histogram over kOrderBins counts and
+// its scan, then one warp places the items in item order.  Lists longer than
+// kSortMax keep the item order.
+constexpr int kOrderBins = 1024;
+constexpr int kSortMax = 4096;
+__device__ __forceinline__ void build_work_list(const DecodeArgs &a, int tid) {
+  __shared__ int bins[kOrderBins];
+  __shared__ unsigned short keys[kSortMax];
+  __shared__ int lens[kSortMax];
+  const int units = a.batch * a.h_kv, n = units * a.nsplit;
+  auto clamped_len = [&](int i) {
+    const int b = (i % units) / a.h_kv;
+    const int len = a.len[b] - a.len_sub;
+    return len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
+  };
+  if (n > kSortMax) {
+    for (int i = tid; i < n; i += 256) a.order[i] = make_int2(i, clamped_len(i));
+    return;
+  }
+  for (int i = tid; i < kOrderBins; i += 256) bins[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += 256) {
+    const int split = i / units;
+    const int len = clamped_len(i);
+    lens[i] = len;
+    const int t_begin = split * a.tiles_per_split * kTile;
+    const int t_end = min(len, (split + 1) * a.tiles_per_split * kTile);
+    const int nt = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
+    const int k = kOrderBins - 1 - min(nt, kOrderBins - 1);  // bin 0: the largest
+    keys[i] = (unsigned short)k;
+    atomicAdd(&bins[k], 1);
+  }
+  __syncthreads();
+  if (tid < 32) {  // exclusive scan: lane l takes bins 32 l .. 32 l + 31
+    int sum = 0;
+    for (int j = 0; j < 32; ++j) sum += bins[32 * tid + j];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += v;
+    }
+    int off = incl - sum;
+    for (int j = 0; j < 32; ++j) {
+      const int c = bins[32 * tid + j];
+      bins[32 * tid + j] = off;
+      off += c;
+    }
+    __syncwarp();
+    // stable placement: 32 items at a time in item order, equal keys ranked
+    // by lane
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + tid;
+      const int k = i < n ? (int)keys[i] : -1;  // past the end: a key of its own
+      const unsigned same = __match_any_sync(0xffffffffu, k);
+      const int leader = __ffs(same) - 1;
+      const int rank = __popc(same & ((1u << tid) - 1u));
+      int base = 0;
+      if (tid == leader && k >= 0) base = atomicAdd(&bins[k], __popc(same));
+      base = __shfl_sync(0xffffffffu, base, leader);
+      if (k >= 0) a.order[base + rank] = make_int2(i, lens[i]);
+    }
+  }
+  __syncthreads();
+}
+
 template <int MB, int VB, int G>
 __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ DecodeArgs a) {
   using C = Cfg<MB, VB, G>;
@@ -952,6 +1037,8 @@ __global__ void __launch_bounds__(256, 1) qblock_kernel(const __grid_constant__ 
     a.status[0] = 0;
     a.status[1] = fallback ? 1 : 0;
   }
+  // (the last CTA has the fewest units)
+  if (blockIdx.x == gridDim.x - 1 && a.order) build_work_list(a, tid);
   cp_async_wait_all();
   __syncthreads();
 
@@ -1098,7 +1185,7 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
   const int qgrid = units < a.num_sms ? units : a.num_sms;
   e = launch_pdl(qblock_kernel<MB, VB, G>, dim3(qgrid), dim3(256), qsmem, stream, a);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_tc_kernel<MB, VB, G>, dim3(a.h_kv, a.batch, a.nsplit), dim3(kTcThreads), smem,
+  return launch_pdl(decode_tc_kernel<MB, VB, G>, dim3(a.h_kv * a.batch * a.nsplit), dim3(kTcThreads), smem,
                     stream, a);
 }
 

@@ -75,6 +75,7 @@ struct DecodePlan {
   size_t part_bytes;   // [B][H_q][nsplit + 1][d + 2] fp32 (acc, m, l); the extra slot
                        // holds the recent-token window's partial state
   size_t qblock_bytes; // per (b, h_kv) query block of the tensor-core kernel (0: SIMT path)
+  size_t order_bytes;  // the tensor-core kernel's work items, largest first (0: SIMT path)
   size_t total_bytes;
 };
 
@@ -104,6 +105,11 @@ struct DecodeArgs {
   float *qrot;   // workspace: [B][H_q][2][d]
   float *part;   // workspace: [B][H_q][part_stride][d+2]
   uint8_t *qblocks;  // workspace: [B][H_kv] query blocks (tensor-core path)
+  // workspace: the tensor-core kernel's work items {split * B * H_kv + b *
+  // H_kv + h, the sequence's length clamped to [0, max_len]}, ordered by tile
+  // count, largest first (written by the query-block kernel; CTA i takes
+  // item order[i])
+  int2 *order;
   int num_sms;
   float *out;    // [B][H_q][d]
   // Chunked prefill (qt > 1 or q_tstride > 1): the h_q heads of a sequence
