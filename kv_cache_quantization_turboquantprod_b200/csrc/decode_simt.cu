@@ -328,7 +328,8 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   // sequences: 0.299 ms at two, 0.270 ms at eight) -- but no split shorter
   // than 32 tiles, whose pipeline fill and merge would dominate (measured on
   // 8 sequences of 16K-32K tokens, 64 units: 123 us with 19 splits of ~10
-  // tiles, 110 us with 6)
+  // tiles, 110 us with 6), unless that leaves SMs without a CTA (a few short
+  // sequences: there more, shorter splits are what keeps the call short)
 #ifndef TQ_DECODE_CTAS_PER_SM
 #define TQ_DECODE_CTAS_PER_SM 2
 #endif
@@ -341,7 +342,8 @@ DecodePlan make_decode_plan(int batch, int h_kv, int h_q, int max_len, int num_s
   const long long cps = units >= num_sms ? TQ_DECODE_CTAS_PER_SM : TQ_DECODE_CTAS_PER_SM_FEW_UNITS;
   const long long target = cps * num_sms;
   long long ns = (target + units - 1) / units;
-  ns = std::min(ns, (long long)std::max(ntile / TQ_DECODE_MIN_TILES_PER_SPLIT, 1));
+  ns = std::min(ns, std::max((long long)std::max(ntile / TQ_DECODE_MIN_TILES_PER_SPLIT, 1),
+                              ((long long)num_sms + units - 1) / units));
   ns = std::max(1LL, std::min(ns, (long long)std::max(ntile, 1)));
   int tps = ntile > 0 ? (int)((ntile + ns - 1) / ns) : 0;
   int nsplit = tps > 0 ? (ntile + tps - 1) / tps : 1;

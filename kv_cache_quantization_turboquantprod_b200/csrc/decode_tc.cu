@@ -482,10 +482,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     for (int p = 0; p < C::NSYM; ++p) sym = sym && Q.subset[p] == odd_subset(p);
 
     const int qt1 = a.qt - 1, gshift = 31 - __clz(G / a.qt);
+    // The running maxima start at -1e30, below any logit, not at -inf: a head
+    // whose tiles so far masked every token (causal prefill rows) then keeps
+    // the factor exp2(0) = 1 instead of exp2(-inf + inf) = NaN, with no
+    // select in the loop, and its -1e30 drops out of every merge below
+    // (exp2(-1e30 - m) = 0, or an all-empty state stays 0 / 0 -> 0).
     float mrun[G], lsum[G], zs[G][4], acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      mrun[g] = -INFINITY;
+      mrun[g] = -1e30f;
       lsum[g] = 0.f;
       acc[g] = 0.f;
 #pragma unroll
@@ -742,9 +747,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       for (int g = 0; g < G; ++g) {
         const float4 r4 = *reinterpret_cast<const float4 *>(red[g]);
         const float mnew = fmaxf(mrun[g], fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
-        // a head that has seen no token yet (causally masked prefill rows)
-        // keeps its empty state: its factor is 1, not exp2(-inf + inf)
-        alpha[g] = mnew == -INFINITY ? 1.f : exp2f(mrun[g] - mnew);
+        alpha[g] = exp2f(mrun[g] - mnew);
         changed |= (mnew != mrun[g]);
         mrun[g] = mnew;
       }
