@@ -103,7 +103,7 @@ struct QtSmem {
   alignas(1024) uint8_t a1[kMat16];     // the tile's bf16 K rows
   float nk[2][128];                     // ||k|| by tile parity
   float cent[8];
-  float cent13[8];               // centroids x 2^13
+  float ncent13[8];              // -(centroids x 2^13)
   float bnd[8];                  // ascending, padded with +inf
   int sym;                       // boundaries exactly antisymmetric (b[i] == -b[nb - 1 - i])
   // k_full: the tile's K rows have landed (TMA); a1_full / a1_free: the K
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   }
   if (tid < ncent) {
     S.cent[tid] = a.centroids[tid];
-    S.cent13[tid] = a.centroids[tid] * kEScale;
+    S.ncent13[tid] = -(a.centroids[tid] * kEScale);
   }
   if (tid < 8) S.bnd[tid] = tid < ncent - 1 ? a.boundaries[tid] : INFINITY;
   if (tid == 0) {
@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         // code indices as nibbles (element e in bits 4 (e % 8) of word e / 8),
         // split into bit-planes once the quarter is done
         uint32_t nib[4] = {0u, 0u, 0u, 0u};
-        float rr = 0.f;  // ||r||^2 x 2^26 over this quarter
+        float2 rr2 = make_float2(0.f, 0.f);  // ||r||^2 x 2^26 over this quarter, in two halves
         // The codebook's shape is decided once per tile, outside the element
         // loop: a branch per element would keep the compiler from
         // interleaving the elements' dependent chains.
@@ -585,11 +585,13 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
             uint32_t hl[16];  // hi parts (columns 0-7), lo parts (8-15)
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
-              float ev[2];
+              // two coordinates at a time, in paired f32 arithmetic
+              const float2 dv2 = make_float2(__uint_as_float(d[e]), __uint_as_float(d[e + 1]));
+              const float2 y2 = __ffma2_rn(dv2, make_float2(inv1, inv1), make_float2(ybias, ybias));
+              float nc[2];  // -c x 2^13
 #pragma unroll
               for (int x = 0; x < 2; ++x) {
-                const float dv = __uint_as_float(d[e + x]);
-                const float y = fmaf(dv, inv1, ybias);
+                const float y = x ? y2.y : y2.x;
                 int idx;  // #{boundaries < y}
                 if constexpr (SYM) {
                   const float ay = fabsf(y);
@@ -604,13 +606,15 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                 }
                 const int el = 16 * cc + e + x;
                 nib[el >> 3] |= (uint32_t)idx << (4 * (el & 7));
-                // E = (y - c) 2^13 from D1 in one rounding
-                ev[x] = fmaf(dv, inv13, -S.cent13[idx]);
-                rr = fmaf(ev[x], ev[x], rr);
+                nc[x] = S.ncent13[idx];
               }
-              const __half2 hh = __floats2half2_rn(ev[0], ev[1]);
-              const float2 hf = __half22float2(hh);
-              const __half2 ll = __floats2half2_rn(ev[0] - hf.x, ev[1] - hf.y);
+              // E = (y - c) 2^13 from D1 in one rounding
+              const float2 ev = __ffma2_rn(dv2, make_float2(inv13, inv13), make_float2(nc[0], nc[1]));
+              rr2 = __ffma2_rn(ev, ev, rr2);
+              const __half2 hh = __floats2half2_rn(ev.x, ev.y);
+              // lo = E - hi, exact
+              const float2 lo = __ffma2_rn(__half22float2(hh), make_float2(-1.f, -1.f), ev);
+              const __half2 ll = __floats2half2_rn(lo.x, lo.y);
               hl[e >> 1] = *reinterpret_cast<const uint32_t *>(&hh);
               hl[8 + (e >> 1)] = *reinterpret_cast<const uint32_t *>(&ll);
             }
@@ -642,7 +646,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
             }
             *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = w;
           }
-        S.rrq[j & 3][cq][r] = rr;
+        S.rrq[j & 3][cq][r] = rr2.x + rr2.y;
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.pair[j & 1][q4]);  // this quarter's ||r||^2 is written
       }
