@@ -487,14 +487,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // the factor exp2(0) = 1 instead of exp2(-inf + inf) = NaN, with no
     // select in the loop, and its -1e30 drops out of every merge below
     // (exp2(-1e30 - m) = 0, or an all-empty state stays 0 / 0 -> 0).
-    float mrun[G], lsum[G], zs[G][4], acc[G];
+    // zs: per head the zero-point sums of the four value groups, as pairs
+    // (updated two groups per paired f32 instruction)
+    float mrun[G], lsum[G], acc[G];
+    float2 zs[G][2];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       mrun[g] = -1e30f;
       lsum[g] = 0.f;
       acc[g] = 0.f;
 #pragma unroll
-      for (int gg = 0; gg < 4; ++gg) zs[g][gg] = 0.f;
+      for (int gh = 0; gh < 2; ++gh) zs[g][gh] = make_float2(0.f, 0.f);
     }
     // P.V read-back of tile jt in slot rb: acc = acc * alpha + D * sc, with
     // alpha[0..G-1] and sc = alpha[G] as this warp left them in shared memory
@@ -758,7 +761,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         for (int g = 0; g < G; ++g) {
           lsum[g] *= alpha[g];
 #pragma unroll
-          for (int gg = 0; gg < 4; ++gg) zs[g][gg] *= alpha[g];
+          for (int gh = 0; gh < 2; ++gh) zs[g][gh] = __fmul2_rn(zs[g][gh], make_float2(alpha[g], alpha[g]));
         }
       }
       // p * scale <= mscale < 2^(e+1); fixed point with values < 2^21
@@ -773,7 +776,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         p[g] = lg[g] != -INFINITY ? exp2f(lg[g] - mrun[g]) : 0.f;
         lsum[g] += p[g];
 #pragma unroll
-        for (int gg = 0; gg < 4; ++gg) zs[g][gg] = fmaf(p[g], vze[gg], zs[g][gg]);
+        for (int gh = 0; gh < 2; ++gh)
+          zs[g][gh] = __ffma2_rn(make_float2(p[g], p[g]), make_float2(vze[2 * gh], vze[2 * gh + 1]), zs[g][gh]);
       }
 
       // 7. P' operand: column n = (group * G + head) * PB + byte, the PB
@@ -785,9 +789,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
           for (int c = 0; c < G; ++c) {
             uint32_t w4[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const int gg = (4 * c + x) / G, g = (4 * c + x) % G;
-              w4[x] = __float_as_uint(fmaf(p[g], vscf[gg], 12582912.f)) & 0x3FFFFFu;
+            for (int x = 0; x < 4; x += 2) {
+              const int gg0 = (4 * c + x) / G, g0 = (4 * c + x) % G;
+              const int gg1 = (4 * c + x + 1) / G, g1 = (4 * c + x + 1) % G;
+              const float2 f = __ffma2_rn(make_float2(p[g0], p[g1]), make_float2(vscf[gg0], vscf[gg1]),
+                                          make_float2(12582912.f, 12582912.f));
+              w4[x] = __float_as_uint(f.x) & 0x3FFFFFu;
+              w4[x + 1] = __float_as_uint(f.y) & 0x3FFFFFu;
             }
             *reinterpret_cast<uint4 *>(row + c * C::SBO_V) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
@@ -840,7 +848,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       if (lane == 0) S.lsum[grp][q4][g] = l;
 #pragma unroll
       for (int gg = 0; gg < 4; ++gg) {
-        const float z = warp_sum(zs[g][gg]);
+        const float z = warp_sum((gg & 1) ? zs[g][gg >> 1].y : zs[g][gg >> 1].x);
         if (lane == 0) S.zsum[grp][q4][g][gg] = z;
       }
       if (t == 0) S.fin_m[grp][g] = mrun[g];
