@@ -165,7 +165,21 @@ typedef struct {
                                 float64 as z_j = S_j . u - sum_m c_m W[j][m]
                                 (= S_j . (u - Pi^T c)); required there, unused
                                 by the other calls (may be NULL) */
+  const void *tc_operands;   /* device, TQ_TC_OPERAND_BYTES bytes, 128-byte
+                                aligned, or NULL: the tensor-core append's
+                                shared-memory operand images of Pi (three
+                                bf16 parts whose sum is Pi) and of W (fp16 hi
+                                and lo parts of W x 2^8), as
+                                tq_prepare_operands writes them from pi and
+                                s_pit.  With NULL every CTA of every
+                                tq_quantize_append builds them itself (same
+                                bytes, ~10 us more a call); they must be
+                                rewritten when pi or s_pit change.  d = 128
+                                only (ignored otherwise) */
 } tq_params;
+
+/* Bytes of the tensor-core append's operand images (tq_prepare_operands). */
+#define TQ_TC_OPERAND_BYTES (5 * 128 * 128 * 2)
 
 /*
  * One layer's compressed cache: a single caller-owned device buffer.
@@ -210,6 +224,16 @@ typedef struct {
  * misaligned pointers, TQ_ERR_UNSUPPORTED for d.
  */
 TQ_API tq_status tq_sketch_product(const tq_params *p, double *s_pit, tq_stream_t stream);
+
+/*
+ * tq_prepare_operands -- write the tensor-core append's operand images into
+ * dst (device, TQ_TC_OPERAND_BYTES bytes, 128-byte aligned) from p->pi and
+ * p->s_pit (which tq_sketch_product must have written, earlier on the same
+ * stream), for p->tc_operands.  Once per layer.  Asynchronous on `stream`.
+ * TQ_ERR_INVALID_ARGUMENT for null or misaligned pointers,
+ * TQ_ERR_UNSUPPORTED for d != 128.
+ */
+TQ_API tq_status tq_prepare_operands(const tq_params *p, void *dst, tq_stream_t stream);
 
 /* Bytes per (token, KV head) record R, or 0 for unsupported params. */
 TQ_API size_t tq_record_bytes(const tq_params *p);

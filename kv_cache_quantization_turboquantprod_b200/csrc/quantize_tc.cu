@@ -75,6 +75,8 @@ constexpr int kQtRegs = 80;      // registers a thread at launch (65536 / 768, r
 constexpr int kIssRegs = 56, kLoadRegs = 72, kEpiRegs = 88;
 constexpr int kRingCap = 8;      // refinement requests per epilogue warp in flight
 constexpr int kMat16 = 128 * 128 * 2;  // one 16-bit 128 x 128 operand (32 KB)
+constexpr int kOperandBytes = 5 * kMat16;  // Pi's three bf16 parts, W's fp16 hi and lo
+static_assert(kOperandBytes == TQ_TC_OPERAND_BYTES, "operand image size");
 constexpr double kWScale = 256.0;     // W = S Pi^T parts x 2^8
 constexpr float kEScale = 8192.f;      // E = y - c parts x 2^13
 
@@ -113,6 +115,7 @@ struct QtSmem {
   // of the tile's E operand is in tensor memory; fin: the issuer's last
   // commit (every MMA it issued is done)
   uint64_t k_full, a1_full, a1_free, d1_full, d2_full[2], d1_read, d_free[2], kc[8], fin;
+  uint64_t ops_full;  // the prepared operand images have landed
   uint32_t tmem_base;
   volatile int abort_flag;
   // refinement rings, one per epilogue warp (single producer, the refiner
@@ -126,6 +129,8 @@ struct QtSmem {
   uint64_t pair[2][4];      // [tile parity][lane quarter]: the four column quarters of a row block meet
   volatile int progress;  // changes whenever an epilogue warp finishes a tile
 };
+
+static_assert(offsetof(QtSmem, w) == offsetof(QtSmem, pi) + 3 * kMat16, "operand images back to back");
 
 struct TileInfo {
   int b, h, t0, nrow;
@@ -185,6 +190,53 @@ __device__ __forceinline__ bool ring_room(QtSmem &S, int ew, int upto, const App
 }
 
 
+// The shared-memory operand images of Pi (three bf16 parts, their sum Pi
+// exactly) and W = S Pi^T (fp16 hi + lo of W x 2^8, split from its float64
+// values), 32 KB each, back to back at dst in the canonical no-swizzle
+// layout.  Item it (0 .. 2047) writes eight elements (one 16-byte block row)
+// of each, both matrices' loads issued before any is used.
+__device__ __forceinline__ void operand_item(const float *pi, const double *s_pit, int it, uint8_t *dst) {
+  const int i = it >> 4, j0 = (it & 15) * 8;
+  const float4 *pp = reinterpret_cast<const float4 *>(pi + i * 128 + j0);
+  const double2 *wp = reinterpret_cast<const double2 *>(s_pit + i * 128 + j0);
+  const float4 p0 = pp[0], p1 = pp[1];
+  const double2 w0 = wp[0], w1 = wp[1], w2 = wp[2], w3 = wp[3];
+  const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+  const double wv[8] = {w0.x, w0.y, w1.x, w1.y, w2.x, w2.y, w3.x, w3.y};
+  uint32_t pp3[3][4], wh[4], wl[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    // x = p1 + p2 + p3 exactly: each remainder is exact in fp32 and the
+    // last has at most 8 significant bits
+    float r0 = pv[2 * e], r1 = pv[2 * e + 1];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(r0, r1);
+      pp3[q][e] = *reinterpret_cast<const uint32_t *>(&b2);
+      r0 -= __low2float(b2);
+      r1 -= __high2float(b2);
+    }
+    const double x0 = wv[2 * e] * kWScale, x1 = wv[2 * e + 1] * kWScale;
+    const __half hh0 = __double2half(x0), hh1 = __double2half(x1);
+    const __half ll0 = __double2half(x0 - (double)__half2float(hh0));
+    const __half ll1 = __double2half(x1 - (double)__half2float(hh1));
+    const __half2 hw2 = __halves2half2(hh0, hh1), lw2 = __halves2half2(ll0, ll1);
+    wh[e] = *reinterpret_cast<const uint32_t *>(&hw2);
+    wl[e] = *reinterpret_cast<const uint32_t *>(&lw2);
+  }
+#pragma unroll
+  for (int q = 0; q < 3; ++q)
+    *reinterpret_cast<uint4 *>(dst + q * kMat16 + blk_off(i, j0)) = make_uint4(pp3[q][0], pp3[q][1], pp3[q][2], pp3[q][3]);
+  *reinterpret_cast<uint4 *>(dst + 3 * kMat16 + blk_off(i, j0)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+  *reinterpret_cast<uint4 *>(dst + 4 * kMat16 + blk_off(i, j0)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+}
+
+// The operand images written once per layer into global memory.
+__global__ void __launch_bounds__(256) prepare_operands_kernel(const float *pi, const double *s_pit, uint8_t *dst) {
+  const int it = blockIdx.x * 256 + threadIdx.x;
+  if (it < 128 * 16) operand_item(pi, s_pit, it, dst);
+}
+
 template <int MB>
 __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid_constant__ AppendArgs a,
                                                                    const __grid_constant__ CUtensorMap kmap) {
@@ -200,43 +252,20 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                          ? (a.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
                          : 0;
 
-  // ---- setup: split Pi and W = S Pi^T into fp16 parts, barriers, TMEM ---
-  // eight elements (one 16-byte block row) per item, both matrices' loads
-  // issued before any is used; W is split from its float64 values
-  for (int it = tid; it < 128 * 16; it += kQtThreads) {
-    const int i = it >> 4, j0 = (it & 15) * 8;
-    const float4 *pp = reinterpret_cast<const float4 *>(a.pi + i * 128 + j0);
-    const double2 *wp = reinterpret_cast<const double2 *>(a.s_pit + i * 128 + j0);
-    const float4 p0 = pp[0], p1 = pp[1];
-    const double2 w0 = wp[0], w1 = wp[1], w2 = wp[2], w3 = wp[3];
-    const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    const double wv[8] = {w0.x, w0.y, w1.x, w1.y, w2.x, w2.y, w3.x, w3.y};
-    uint32_t pp3[3][4], wh[4], wl[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      // x = p1 + p2 + p3 exactly: each remainder is exact in fp32 and the
-      // last has at most 8 significant bits
-      float r0 = pv[2 * e], r1 = pv[2 * e + 1];
-#pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(r0, r1);
-        pp3[q][e] = *reinterpret_cast<const uint32_t *>(&b2);
-        r0 -= __low2float(b2);
-        r1 -= __high2float(b2);
-      }
-      const double x0 = wv[2 * e] * kWScale, x1 = wv[2 * e + 1] * kWScale;
-      const __half hh0 = __double2half(x0), hh1 = __double2half(x1);
-      const __half ll0 = __double2half(x0 - (double)__half2float(hh0));
-      const __half ll1 = __double2half(x1 - (double)__half2float(hh1));
-      const __half2 hw2 = __halves2half2(hh0, hh1), lw2 = __halves2half2(ll0, ll1);
-      wh[e] = *reinterpret_cast<const uint32_t *>(&hw2);
-      wl[e] = *reinterpret_cast<const uint32_t *>(&lw2);
+  // ---- setup: the operand images of Pi and W, barriers, TMEM ------------
+  if (a.tc_ops) {
+    // prepared once per layer (tq_prepare_operands): one bulk copy
+    if (tid == 0) {
+      mbar_init(&S.ops_full, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(&S.ops_full, kOperandBytes);
+#pragma unroll 1
+      for (int c = 0; c < kOperandBytes / kMat16; ++c)
+        bulk_g2s(S.pi[0] + c * kMat16, reinterpret_cast<const uint8_t *>(a.tc_ops) + c * kMat16, kMat16,
+                 &S.ops_full);
     }
-#pragma unroll
-    for (int q = 0; q < 3; ++q)
-      *reinterpret_cast<uint4 *>(S.pi[q] + blk_off(i, j0)) = make_uint4(pp3[q][0], pp3[q][1], pp3[q][2], pp3[q][3]);
-    *reinterpret_cast<uint4 *>(S.w[0] + blk_off(i, j0)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-    *reinterpret_cast<uint4 *>(S.w[1] + blk_off(i, j0)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+  } else {
+    for (int it = tid; it < 128 * 16; it += kQtThreads) operand_item(a.pi, a.s_pit, it, S.pi[0]);
   }
   if (tid < ncent) {
     S.cent[tid] = a.centroids[tid];
@@ -271,6 +300,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&S.tmem_base, 512);
+  // the MMA issuer (warp 0) sees the prepared images land itself; the copy
+  // engine completes them, so the wait ends
+  if (a.tc_ops && warp == 0) mbar_wait(&S.ops_full, 0);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -812,6 +844,11 @@ cudaError_t encode_k_map(const AppendArgs &a, CUtensorMap *map) {
 }
 
 }  // namespace
+
+cudaError_t launch_prepare_operands(const float *pi, const double *s_pit, void *dst, cudaStream_t stream) {
+  prepare_operands_kernel<<<128 * 16 / 256, 256, 0, stream>>>(pi, s_pit, reinterpret_cast<uint8_t *>(dst));
+  return cudaGetLastError();
+}
 
 bool quantize_tc_supported(const AppendArgs &a) {
   // (the K tensor map wants a 16-byte aligned base; the value kernel splits

@@ -190,6 +190,14 @@ tq_status tq_sketch_product(const tq_params *p, double *s_pit, tq_stream_t strea
                                                                                                : TQ_ERR_CUDA;
 }
 
+tq_status tq_prepare_operands(const tq_params *p, void *dst, tq_stream_t stream) {
+  if (!p || !dst || !aligned(dst, 128)) return TQ_ERR_INVALID_ARGUMENT;
+  if (p->d != 128) return TQ_ERR_UNSUPPORTED;
+  if (!p->pi || !p->s_pit || !aligned(p->pi, 16) || !aligned(p->s_pit, 16)) return TQ_ERR_INVALID_ARGUMENT;
+  return tq::launch_prepare_operands(p->pi, p->s_pit, dst, (cudaStream_t)stream) == cudaSuccess ? TQ_OK
+                                                                                                : TQ_ERR_CUDA;
+}
+
 size_t tq_record_bytes(const tq_params *p) {
   if (check_params(p) != TQ_OK) return 0;
   return (size_t)tq::TileLayout::make(p->key_bits, p->value_bits, p->value_mode, p->d).record_bytes();
@@ -235,6 +243,7 @@ tq_status tq_quantize_append(const tq_params *p, const tq_cache *c, const void *
   if (set_wait_fields(a) != cudaSuccess) return TQ_ERR_CUDA;
   a.refine_z = g_refine_z.load(std::memory_order_relaxed);
   a.s_pit = p->s_pit;
+  a.tc_ops = p->d == 128 ? p->tc_operands : nullptr;
   if (refine_count_address(&a.refine_count) != cudaSuccess) return TQ_ERR_CUDA;
   const cudaError_t e = tq::quantize_tc_supported(a) ? tq::launch_quantize_tc(a, sms, (cudaStream_t)stream)
                                                     : tq::launch_quantize_simt(a, sms, (cudaStream_t)stream);

@@ -63,6 +63,9 @@ struct AppendArgs {
   float refine_z;
   const double *s_pit;
   unsigned long long *refine_count;
+  // the tensor-core append's prepared operand images (tq_prepare_operands),
+  // or nullptr: then every CTA builds them from pi and s_pit
+  const void *tc_ops;
 };
 
 // Split-K plan of one decode call (host-computed, identical in the
@@ -163,6 +166,7 @@ cudaError_t launch_value_quant(const AppendArgs &a, int num_sms, cudaStream_t st
 cudaError_t launch_quantize_warp(const AppendArgs &a, int num_sms, cudaStream_t stream);
 // W = S Pi^T in float64 (d x d, row-major by sketch row j).
 cudaError_t launch_sketch_product(const float *pi, const float *s, int d, double *out, cudaStream_t stream);
+cudaError_t launch_prepare_operands(const float *pi, const double *s_pit, void *dst, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
 // Tensor-core split-K kernel (qprep and combine are shared with the SIMT path).
 bool decode_tc_supported(int key_bits, int value_bits, int gqa, int value_mode = 0, int d = 128);

@@ -32,7 +32,7 @@ EXPORTS = ("tq_status_string", "tq_make_codebook", "tq_record_bytes", "tq_cache_
            "tq_dequantize", "tq_decode_attention_noalloc", "tq_decode_attention_window",
            "tq_prefill_workspace_size", "tq_prefill_attention", "tq_prefill_tokens_per_pass",
            "tq_set_wait_limit_ns", "tq_device_errors", "tq_test_withhold_handoffs",
-           "tq_test_sign_refine_threshold", "tq_test_refine_count", "tq_sketch_product")
+           "tq_test_sign_refine_threshold", "tq_test_refine_count", "tq_sketch_product", "tq_prepare_operands")
 ERRF_DECODE_WAIT, ERRF_QUANTIZE_WAIT = 1, 2
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -49,7 +49,10 @@ class Params(ctypes.Structure):
                 ("pi", ctypes.c_void_p), ("s", ctypes.c_void_p),
                 ("centroids", ctypes.c_void_p), ("boundaries", ctypes.c_void_p),
                 ("value_mode", ctypes.c_int), ("v_centroids", ctypes.c_void_p),
-                ("v_boundaries", ctypes.c_void_p), ("s_pit", ctypes.c_void_p)]
+                ("v_boundaries", ctypes.c_void_p), ("s_pit", ctypes.c_void_p),
+                ("tc_operands", ctypes.c_void_p)]
+
+TQ_TC_OPERAND_BYTES = 5 * 128 * 128 * 2
 
 
 class Cache(ctypes.Structure):
@@ -81,6 +84,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_record_bytes.argtypes = [P]
     lib.tq_sketch_product.restype = ci
     lib.tq_sketch_product.argtypes = [P, vp, vp]
+    lib.tq_prepare_operands.restype = ci
+    lib.tq_prepare_operands.argtypes = [P, vp, vp]
     lib.tq_cache_bytes.restype = sz
     lib.tq_cache_bytes.argtypes = [P, ci, ci, ci]
     lib.tq_quantize_append.restype = ci
@@ -209,14 +214,21 @@ class Layer:
             self.v_boundaries = torch.tensor(vbnd, dtype=torch.float32, device=device)
             self.value_codebook = (vcent, vbnd)
             vc_ptr, vb_ptr = self.v_centroids.data_ptr(), self.v_boundaries.data_ptr()
-        # W = S Pi^T in float64, for the append kernels' sign refinement
+        # W = S Pi^T in float64, for the append kernels' sign refinement and
+        # sketch; at d = 128 also the tensor-core append's operand images
         self.s_pit = torch.empty((d, d), dtype=torch.float64, device=device)
+        on_gpu = self.s_pit.is_cuda
+        self.tc_operands = (torch.empty(TQ_TC_OPERAND_BYTES, dtype=torch.uint8, device=device)
+                            if on_gpu and d == 128 else None)
         self.params = Params(d, key_bits, value_bits, group, self.pi.data_ptr(),
                              self.s.data_ptr(), self.centroids.data_ptr(),
                              self.boundaries.data_ptr(), mode, vc_ptr, vb_ptr,
-                             self.s_pit.data_ptr())
-        if self.s_pit.is_cuda:
+                             self.s_pit.data_ptr(),
+                             self.tc_operands.data_ptr() if self.tc_operands is not None else None)
+        if on_gpu:
             tq_sketch_product(self)
+            if self.tc_operands is not None:
+                tq_prepare_operands(self)
 
     @property
     def d(self):
@@ -245,6 +257,13 @@ def tq_sketch_product(layer: Layer, stream=None) -> None:
     """Write W = S Pi^T (float64) into layer.s_pit from the layer's Pi and S."""
     st = load().tq_sketch_product(ctypes.byref(layer.params), layer.s_pit.data_ptr(), _stream(stream))
     _check("tq_sketch_product", st)
+
+
+def tq_prepare_operands(layer: Layer, stream=None) -> None:
+    """Write the tensor-core append's operand images of the layer's Pi and
+    W into layer.tc_operands (after tq_sketch_product)."""
+    st = load().tq_prepare_operands(ctypes.byref(layer.params), layer.tc_operands.data_ptr(), _stream(stream))
+    _check("tq_prepare_operands", st)
 
 
 def tq_record_bytes(layer: Layer) -> int:

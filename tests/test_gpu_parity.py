@@ -144,6 +144,38 @@ def test_quantize_append_bit_widths(kb, vb):
     pu.check_band_fraction(stats)
 
 
+@pytest.mark.parametrize("kb", [3, 4])
+def test_prepared_operands_give_the_same_records(kb):
+    """The tensor-core append with operand images prepared once per layer
+    (tq_prepare_operands, the default of tq.Layer) writes the same bytes as
+    with tc_operands = NULL (every CTA building them itself), and the
+    prepared images match a second preparation; 20 tiles of bf16 keys per
+    sequence (several tiles per CTA)."""
+    import ctypes
+    import dataclasses
+    wl = dataclasses.replace(workloads.llama8b(), batch=2, key_bits=kb, value_bits=2,
+                             capacity=2560, lengths=(2560, 2560), name=f"ops{kb}")
+    glayer, olayer, spec = _setup(wl)
+    assert glayer.tc_operands is not None
+    again = torch.empty_like(glayer.tc_operands)
+    st = tq.load().tq_prepare_operands(ctypes.byref(glayer.params), again.data_ptr(), None)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(again, glayer.tc_operands)
+    T = 2560
+    k = torch.stack([workloads.kv_tokens(wl, b, 0, T)[0] for b in range(2)]).to(DEV).contiguous()
+    v = torch.stack([workloads.kv_tokens(wl, b, 0, T)[1] for b in range(2)]).to(DEV).contiguous()
+    bufs = []
+    for prepared in (True, False):
+        glayer.params.tc_operands = glayer.tc_operands.data_ptr() if prepared else None
+        cache = tq.CompressedCache(glayer, 2, wl.h_kv, T, zero=True)
+        tq.tq_quantize_append(glayer, cache, k, v, [0, 0], [T, T - 100])
+        torch.cuda.synchronize()
+        bufs.append(cache.buffer.cpu().numpy())
+    glayer.params.tc_operands = glayer.tc_operands.data_ptr()
+    assert np.array_equal(bufs[0], bufs[1])
+
+
 @pytest.mark.parametrize("kb,vb", [(2, 2), (4, 2), (3, 3), (4, 4)])
 def test_quantize_append_bit_widths_bf16_tiles(kb, vb):
     """bf16 appends of 300 tokens (the tensor-core kernel) at every key and

@@ -68,8 +68,8 @@ def test_status_strings():
         assert tq.tq_status_string(code) == name
 
 
-def _params(d=128, kb=3, vb=2, g=32, ptr=256, mode=0, vptr=None, wptr=256):
-    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr, mode, vptr, vptr, wptr)
+def _params(d=128, kb=3, vb=2, g=32, ptr=256, mode=0, vptr=None, wptr=256, optr=None):
+    return tq.Params(d, kb, vb, g, ptr, ptr, ptr, ptr, mode, vptr, vptr, wptr, optr)
 
 
 def test_record_and_cache_bytes():
@@ -140,6 +140,18 @@ def test_sketch_product_validation():
     assert f(ctypes.byref(_params()), (1 << 20) + 8, None) == 1         # output alignment
     assert f(ctypes.byref(_params(d=96)), 1 << 20, None) == 2
     assert f(ctypes.byref(_params(ptr=260)), 1 << 20, None) == 1        # Pi / S alignment
+
+
+def test_prepare_operands_validation():
+    lib = tq.load()
+    f = lib.tq_prepare_operands
+    assert f(None, 1 << 20, None) == 1
+    assert f(ctypes.byref(_params()), None, None) == 1
+    assert f(ctypes.byref(_params()), (1 << 20) + 64, None) == 1        # output alignment (128 bytes)
+    assert f(ctypes.byref(_params(d=64)), 1 << 20, None) == 2          # the tensor-core append is d = 128 only
+    assert f(ctypes.byref(_params(wptr=None)), 1 << 20, None) == 1     # needs W = S Pi^T
+    assert f(ctypes.byref(_params(ptr=260)), 1 << 20, None) == 1       # Pi alignment
+    assert tq.TQ_TC_OPERAND_BYTES == 5 * 128 * 128 * 2
 
 
 def test_decode_validation_before_launch():
