@@ -72,7 +72,7 @@ using namespace sm100;
 constexpr int kQtThreads = 768;  // 6 warpgroups
 constexpr int kQtRegs = 80;      // registers a thread at launch (65536 / 768, rounded down to 8)
 // setmaxnreg shares: WG0 (issuers, refiners), WG1 (loader), WG2-5 (epilogue)
-constexpr int kIssRegs = 56, kLoadRegs = 72, kEpiRegs = 88;
+constexpr int kIssRegs = 72, kLoadRegs = 56, kEpiRegs = 88;
 constexpr int kRingCap = 8;      // refinement requests per epilogue warp in flight
 constexpr int kMat16 = 128 * 128 * 2;  // one 16-bit 128 x 128 operand (32 KB)
 constexpr int kOperandBytes = 5 * kMat16;  // Pi's three bf16 parts, W's fp16 hi and lo
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
   const uint32_t tbase = S.tmem_base;
 
   // Registers move from the warpgroups that need few (issuers and refiners,
-  // loader) to the four epilogue warpgroups: (56 + 72) x 128 + 88 x 512 =
+  // loader) to the four epilogue warpgroups: (72 + 56) x 128 + 88 x 512 =
   // 61440, exactly the 80 x 768 the CTA is launched with (the kernel's
   // register count is checked on the host before launch).
   const int wg = warp >> 2;
@@ -626,11 +626,13 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                 const float y = x ? y2.y : y2.x;
                 int idx;  // #{boundaries < y}
                 if constexpr (SYM) {
+                  // NC/2 + cnt above zero, NC/2 - 1 - cnt = NC/2 + ~cnt at or
+                  // below it: one xor with the all-ones mask of y <= 0
                   const float ay = fabsf(y);
                   int cnt = 0;
 #pragma unroll
                   for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
-                  idx = y > 0.f ? NC / 2 + cnt : NC / 2 - 1 - cnt;
+                  idx = NC / 2 + (cnt ^ -(int)!(y > 0.f));
                 } else {  // any codebook: count the boundaries below y
                   idx = 0;
 #pragma unroll
@@ -695,17 +697,27 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.d_free[tb]);  // D2 is in registers
-        uint32_t sw = 0u;
+        // sign bits: element e's sign bit shifted in last-first, so it ends
+        // in bit e (one funnel shift an element); a set sign bit is z < 0
+        // except at z = -0, which like every |z| < the refinement threshold
+        // is re-decided by the refiner
+        uint32_t neg = 0u;
+#pragma unroll
+        for (int e = 31; e >= 0; --e) neg = __funnelshift_l(e < 16 ? dA[e] : dB[e - 16], neg, 1);
+        uint32_t sw = ~neg;
+        // the smallest |z| of the row (three-input minima); the mask of the
+        // components next to zero only where it is below the threshold
+        float zmin = fabsf(__uint_as_float(dA[0]));
+#pragma unroll
+        for (int e = 1; e < 31; e += 2)
+          zmin = min3f(zmin, fabsf(__uint_as_float(e < 16 ? dA[e] : dB[e - 16])),
+                       fabsf(__uint_as_float(e + 1 < 16 ? dA[e + 1] : dB[e - 15])));
+        zmin = fminf(zmin, fabsf(__uint_as_float(dB[15])));
         uint32_t nearw = 0u;  // |S r| below the refinement threshold
+        if (zmin < kNearZ) {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const uint32_t(&d)[16] = cc ? dB : dA;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float z = __uint_as_float(d[e]);
-            sw |= (z >= 0.f ? 1u : 0u) << (16 * cc + e);
-            nearw |= (fabsf(z) < kNearZ ? 1u : 0u) << (16 * cc + e);
-          }
+          for (int e = 0; e < 32; ++e)
+            nearw |= (fabsf(__uint_as_float(e < 16 ? dA[e] : dB[e - 16])) < kNearZ ? 1u : 0u) << e;
         }
         if (pv_zero) sw = 0u;
         if (pv_zero || !pv_valid) nearw = 0u;

@@ -298,6 +298,14 @@ __device__ __forceinline__ float redux_max_f32(float x) {
   return r;
 }
 
+// Minimum of three floats in one instruction (the three-input min.f32 of
+// sm_100; a NaN operand is ignored, as by fminf).
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Order-preserving map of floats to unsigned (for integer max reductions).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
   const uint32_t b = __float_as_uint(f);
