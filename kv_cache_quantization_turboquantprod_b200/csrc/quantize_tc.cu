@@ -593,8 +593,10 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         const float ybias = zero ? -INFINITY : 0.f;
         // ---- E1: y = Pi u, codes, E = (y - c) x 2^13 handed to GEMM2 a
         // K-step (16 coordinates) at a time, ||r||^2 = ||E||^2 ----
-        // code indices as nibbles (element e in bits 4 (e % 8) of word e / 8),
-        // split into bit-planes once the quarter is done
+        // code indices as nibbles, split into bit-planes once the quarter is
+        // done: element e goes to word e / 8, nibble 2 b (b = e % 8 < 4) or
+        // 2 (b - 4) + 1 (b >= 4), the order one multiply gathers bit p of
+        // the eight nibbles in
         uint32_t nib[4] = {0u, 0u, 0u, 0u};
         float2 rr2 = make_float2(0.f, 0.f);  // ||r||^2 x 2^26 over this quarter, in two halves
         // The codebook's shape is decided once per tile, outside the element
@@ -624,7 +626,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
 #pragma unroll
               for (int x = 0; x < 2; ++x) {
                 const float y = x ? y2.y : y2.x;
-                int idx;  // #{boundaries < y}
+                // the code is #{boundaries < y} = NC/2 + xi
+                int xi;
                 if constexpr (SYM) {
                   // NC/2 + cnt above zero, NC/2 - 1 - cnt = NC/2 + ~cnt at or
                   // below it: one xor with the all-ones mask of y <= 0
@@ -632,15 +635,18 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
                   int cnt = 0;
 #pragma unroll
                   for (int k = 0; k < NU; ++k) cnt += (ub[k] < ay) ? 1 : 0;
-                  idx = NC / 2 + (cnt ^ -(int)!(y > 0.f));
+                  xi = cnt ^ -(int)!(y > 0.f);
                 } else {  // any codebook: count the boundaries below y
-                  idx = 0;
+                  xi = -NC / 2;
 #pragma unroll
-                  for (int k = 0; k < NC - 1; ++k) idx += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
+                  for (int k = 0; k < NC - 1; ++k) xi += (S.bnd[k] < y) ? 1 : 0;  // independent broadcast reads
                 }
-                const int el = 16 * cc + e + x;
-                nib[el >> 3] |= (uint32_t)idx << (4 * (el & 7));
-                nc[x] = S.ncent13[idx];
+                // xi in [-NC/2, NC/2): the words hold sum xi 16^slot, and
+                // NC/2 in every nibble is added at the end (the sums are exact
+                // modulo 2^32, so the borrows cancel)
+                const int el = 16 * cc + e + x, b = el & 7;
+                nib[el >> 3] += (uint32_t)xi << (4 * (b < 4 ? 2 * b : 2 * b - 7));
+                nc[x] = S.ncent13[NC / 2 + xi];
               }
               // E = (y - c) 2^13 from D1 in one rounding
               const float2 ev = __ffma2_rn(dv2, make_float2(inv13, inv13), make_float2(nc[0], nc[1]));
@@ -665,19 +671,20 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           return true;
         };
         if (!(sym ? e1(std::true_type{}) : e1(std::false_type{}))) break;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) nib[q] += (uint32_t)(NC / 2) * 0x11111111u;
         if (valid)  // this warp's word of every code plane row
 #pragma unroll
           for (int p = 0; p < MB; ++p) {
-            uint32_t w = 0u;
+            // bit p of nibble i sits at 4 i + p; times sum_k 2^(7 k + 3 - p)
+            // it lands at 4 i + 7 k + 3, sixteen distinct positions for
+            // k < 4 (no carries), with nibbles 0, 2, 4, 6 at bits 24-27
+            // (k = 3 - i / 2) and 1, 3, 5, 7 at 28-31: byte 3 is elements
+            // 8q .. 8q + 7 of the quarter in order
+            uint32_t g[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              // bit p of nibbles 0..7 (bits 4i + p) -> bits 0..7
-              uint32_t v = (nib[q] >> p) & 0x11111111u;
-              v = (v | (v >> 3)) & 0x03030303u;
-              v = (v | (v >> 6)) & 0x000F000Fu;
-              v = (v | (v >> 12)) & 0xFFu;
-              w |= v << (8 * q);
-            }
+            for (int q = 0; q < 4; ++q) g[q] = (nib[q] & (0x11111111u << p)) * (0x00204081u << (3 - p));
+            const uint32_t w = __byte_perm(__byte_perm(g[0], g[1], 0x0073u), __byte_perm(g[2], g[3], 0x0073u), 0x5410u);
             *reinterpret_cast<uint32_t *>(tp + L.kplanes + p * kPlaneBytes + slot * kRowBytes + 4 * cq) = w;
           }
         S.rrq[j & 3][cq][r] = rr2.x + rr2.y;
