@@ -749,13 +749,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float4 r4 = *reinterpret_cast<const float4 *>(red[g]);
-        const float mnew = fmaxf(mrun[g], fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
-        alpha[g] = exp2f(mrun[g] - mnew);
+        const float mnew = max3f(max3f(mrun[g], r4.x, r4.y), r4.z, r4.w);
+        alpha[g] = ex2_approx(mrun[g] - mnew);
         changed |= (mnew != mrun[g]);
         mrun[g] = mnew;
       }
       const float4 rs = *reinterpret_cast<const float4 *>(red[G]);
-      const float mscale = fmaxf(fmaxf(rs.x, rs.y), fmaxf(rs.z, rs.w));
+      const float mscale = max3f(max3f(rs.x, rs.y, rs.z), rs.w, 0.f);
       if (changed) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -773,7 +773,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
       float p[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        p[g] = lg[g] != -INFINITY ? exp2f(lg[g] - mrun[g]) : 0.f;
+        p[g] = ex2_approx(lg[g] - mrun[g]);  // a masked token: 2^-inf = 0
         lsum[g] += p[g];
 #pragma unroll
         for (int gh = 0; gh < 2; ++gh)

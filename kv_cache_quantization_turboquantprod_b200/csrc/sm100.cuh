@@ -306,6 +306,22 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
   return r;
 }
 
+// Maximum of three floats in one instruction (the three-input max.f32 of
+// sm_100; a NaN operand is ignored, as by fmaxf).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x by the SFU's approximation (ex2.approx.ftz: relative error about
+// 2^-22, subnormal results flushed to zero, 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Order-preserving map of floats to unsigned (for integer max reductions).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
   const uint32_t b = __float_as_uint(f);
