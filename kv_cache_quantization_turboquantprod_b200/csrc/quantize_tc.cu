@@ -99,11 +99,21 @@ struct RefineReq {
   unsigned long long signs;
 };
 
+// Where a tile's rows go: rows below nrow are new tokens; row r is cache
+// slot pos0 + r of the (sequence, head) whose records start at byte offset
+// rec of the cache, its key at element kbase0 + r H_kv d of K.
+struct TileRec {
+  int nrow, pos0;
+  long long rec, kbase0;
+};
+
 struct QtSmem {
   alignas(1024) uint8_t pi[3][kMat16];  // Pi as three bf16 parts (their sum is Pi exactly)
   alignas(1024) uint8_t w[2][kMat16];   // W = S Pi^T x 2^8: fp16 hi, lo
   alignas(1024) uint8_t a1[kMat16];     // the tile's bf16 K rows
   float nk[2][128];                     // ||k|| by tile parity
+  float ninv[2][128];                   // 1 / ||k|| (0 for a zero key)
+  TileRec trec[2];                      // by tile parity, written with the norms
   float cent[8];
   float ncent13[8];              // -(centroids x 2^13)
   float bnd[8];                  // ascending, padded with +inf
@@ -504,6 +514,15 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
     for (int i = 0; i < nlocal; ++i) {
       const TileInfo ti = tile_info(a, blockIdx.x + i * gridDim.x);
       if (i >= 1 && !qwait(&S.a1_free, (i - 1) & 1, &S.abort_flag, a)) break;
+      // (GEMM1 of tile i - 1 is done, so every epilogue warp has read the
+      // record of tile i - 2 that this one replaces)
+      if (w == 1 && lane == 0) {
+        TileRec &tr = S.trec[i & 1];
+        tr.nrow = ti.nrow;
+        tr.pos0 = a.lens[ti.b] + ti.t0;
+        tr.rec = ((long long)ti.b * a.h_kv + ti.h) * a.ntiles * (long long)L.tile_bytes;
+        tr.kbase0 = (((long long)ti.b * a.T + ti.t0) * a.h_kv + ti.h) * kD;
+      }
       if (w == 0 && lane == 0) {
         mbar_arrive_expect_tx(&S.k_full, 16 * 2048);
 #pragma unroll 1
@@ -526,7 +545,9 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
           ss = fmaf(f.y, f.y, ss);
         }
       }
-      S.nk[i & 1][row] = sqrtf(ss);
+      const float nrm = sqrtf(ss);
+      S.nk[i & 1][row] = nrm;
+      S.ninv[i & 1][row] = nrm > 0.f ? 1.f / nrm : 0.f;
       __syncwarp();
       // (a test of the timeout path withholds the hand-off: the MMA issuer's
       // bounded wait on it then runs out)
@@ -575,17 +596,21 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
       float nk = 0.f;
       if (j < nlocal) {
         const int buf = j & 1;
-        const TileInfo ti = tile_info(a, blockIdx.x + j * gridDim.x);
-        valid = r < ti.nrow;
-        const int pos = a.lens[ti.b] + ti.t0 + r;
-        tp = valid ? tile_ptr(a.data, L, a.h_kv, a.ntiles, ti.b, ti.h, pos / kTile) : nullptr;
-        slot = pos % kTile;
-        kbase = (((size_t)ti.b * a.T + ti.t0 + r) * a.h_kv + ti.h) * kD;  // this row's key
         if (!qwait(&S.d1_full, j & 1, &S.abort_flag, a)) break;
         tc_fence_after();
+        // the tile's record and norms, written by the loader before GEMM1
+        {
+          const TileRec &tr = S.trec[buf];
+          valid = r < tr.nrow;
+          const int pos = tr.pos0 + r;
+          tp = valid ? reinterpret_cast<uint8_t *>(a.data) + tr.rec + (long long)((unsigned)pos / kTile) * L.tile_bytes
+                     : nullptr;
+          slot = (int)((unsigned)pos % kTile);
+          kbase = (size_t)(tr.kbase0 + (long long)r * a.h_kv * kD);  // this row's key
+        }
         nk = S.nk[buf][r];
         zero = !(nk > 0.f);
-        const float inv1 = zero ? 0.f : 1.f / nk;  // y = Y / ||k||
+        const float inv1 = S.ninv[buf][r];  // y = Y / ||k||
         const float inv13 = inv1 * kEScale;
         // a zero key gets y = -inf everywhere, which every bucketize below
         // maps to code 0; its E row is finite garbage (D1 = 0, scale 0) whose
