@@ -44,7 +44,8 @@
 //                     sign words
 //   WG1  warps 4-7    loader: the next tile's bf16 K rows -> the A operand
 //                     buffer (TMA tensor copies) as soon as GEMM1 has read
-//                     it, and their norms
+//                     it, their norms and inverse norms, and where the
+//                     tile's records go
 //   WG2-WG5           epilogue: thread = tile row = TMEM lane; warp w takes
 //                     lane quarter w % 4 and one quarter of the columns
 // setmaxnreg moves registers from WG0 and WG1 to the epilogue warpgroups.
