@@ -314,8 +314,8 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// 2^x by the SFU's approximation (ex2.approx.ftz: relative error about
-// 2^-22, subnormal results flushed to zero, 2^-inf = +0).
+// 2^x by the SFU's approximation (ex2.approx.ftz: a few ulp of relative
+// error, subnormal results flushed to zero, 2^-inf = +0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float r;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
