@@ -632,16 +632,15 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         // columns; E may be overwritten once the previous tile's GEMM2 is done
         auto e1 = [&](auto sym_c) -> bool {
           constexpr bool SYM = decltype(sym_c)::value;
-          uint32_t dA[16], dB[16];
-          tmem_ld16(d1col, dA);
-          tmem_ld16(d1col + 16, dB);
+          uint32_t d1[32];
+          tmem_ld32(d1col, d1);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.d1_read);
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
-            const uint32_t(&d)[16] = cc ? dB : dA;
+            const uint32_t *d = d1 + 16 * cc;
             uint32_t hl[16];  // hi parts (columns 0-7), lo parts (8-15)
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
@@ -723,9 +722,8 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         const uint32_t tph = (t >> 1) & 1;
         if (!qwait(&S.d2_full[tb], tph, &S.abort_flag, a)) break;
         tc_fence_after();
-        uint32_t dA[16], dB[16];
-        tmem_ld16(d1col + 128 + 128 * tb, dA);
-        tmem_ld16(d1col + 128 + 128 * tb + 16, dB);
+        uint32_t d2[32];
+        tmem_ld32(d1col + 128 + 128 * tb, d2);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -736,21 +734,21 @@ __global__ void __launch_bounds__(kQtThreads, 1) quantize_tc_kernel(const __grid
         // is re-decided by the refiner
         uint32_t neg = 0u;
 #pragma unroll
-        for (int e = 31; e >= 0; --e) neg = __funnelshift_l(e < 16 ? dA[e] : dB[e - 16], neg, 1);
+        for (int e = 31; e >= 0; --e) neg = __funnelshift_l(d2[e], neg, 1);
         uint32_t sw = ~neg;
         // the smallest |z| of the row (three-input minima); the mask of the
         // components next to zero only where it is below the threshold
-        float zmin = fabsf(__uint_as_float(dA[0]));
+        float zmin = fabsf(__uint_as_float(d2[0]));
 #pragma unroll
         for (int e = 1; e < 31; e += 2)
-          zmin = min3f(zmin, fabsf(__uint_as_float(e < 16 ? dA[e] : dB[e - 16])),
-                       fabsf(__uint_as_float(e + 1 < 16 ? dA[e + 1] : dB[e - 15])));
-        zmin = fminf(zmin, fabsf(__uint_as_float(dB[15])));
+          zmin = min3f(zmin, fabsf(__uint_as_float(d2[e])),
+                       fabsf(__uint_as_float(d2[e + 1])));
+        zmin = fminf(zmin, fabsf(__uint_as_float(d2[31])));
         uint32_t nearw = 0u;  // |S r| below the refinement threshold
         if (zmin < kNearZ) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            nearw |= (fabsf(__uint_as_float(e < 16 ? dA[e] : dB[e - 16])) < kNearZ ? 1u : 0u) << e;
+            nearw |= (fabsf(__uint_as_float(d2[e])) < kNearZ ? 1u : 0u) << e;
         }
         if (pv_zero) sw = 0u;
         if (pv_zero || !pv_valid) nearw = 0u;
