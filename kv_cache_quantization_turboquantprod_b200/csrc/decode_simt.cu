@@ -230,7 +230,28 @@ __global__ void __launch_bounds__(128) window_kernel(DecodeArgs a) {
 #pragma unroll
     for (int u = 0; u < J; ++u) num[g][u] = 0.f;
   }
-  for (int i = 0; i < wl; ++i) {
+  // kWinBatch slots at a time, every load of the batch issued before any
+  // is used (the slots' rows are independent), then the tail one by one
+  constexpr int kWinBatch = 16;
+  int i = 0;
+  for (; i + kWinBatch <= wl; i += kWinBatch) {
+    float v[kWinBatch][J];
+#pragma unroll
+    for (int k = 0; k < kWinBatch; ++k)
+#pragma unroll
+      for (int u = 0; u < J; ++u)
+        v[k][u] = (t + 128 * u < D) ? load_elem(a.win_v, a.win_dtype, (row0 + i + k) * D + t + 128 * u) : 0.f;
+#pragma unroll
+    for (int k = 0; k < kWinBatch; ++k) {
+#pragma unroll
+      for (int u = 0; u < J; ++u)
+#pragma unroll
+        for (int g = 0; g < G; ++g) num[g][u] = fmaf(ps[g][i + k], v[k][u], num[g][u]);
+#pragma unroll
+      for (int g = 0; g < G; ++g) den[g] += ps[g][i + k];
+    }
+  }
+  for (; i < wl; ++i) {
 #pragma unroll
     for (int u = 0; u < J; ++u) {
       if (t + 128 * u >= D) continue;
