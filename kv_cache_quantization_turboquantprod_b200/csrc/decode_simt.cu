@@ -154,11 +154,16 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
 // One CTA per (h_kv, b); thread t scores window slot t, then sums dims
 // t, t + 128, ... over the slots.  (TurboQuant-MSE values: the partial is
 // rotated like the compressed splits, Pi acc.)
+// Launched as a programmatic dependent of the split-K kernel, whose CTAs
+// signal only after their own wait on the call's predecessors (or which
+// signals by finishing), so the queries and the window rows are complete
+// when this grid starts; it reads nothing the split-K kernel writes, so it
+// runs beside that kernel's last CTAs and waits for it only before it
+// finishes (the combine's wait then covers both).
 // ---------------------------------------------------------------------------
 template <int G, int D>
 __global__ void __launch_bounds__(128) window_kernel(DecodeArgs a) {
   constexpr int J = (D + 127) / 128;
-  pdl_wait();
   const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
   __shared__ float qs[G][D];
   __shared__ float ps[G][kTile];
@@ -293,6 +298,7 @@ __global__ void __launch_bounds__(128) window_kernel(DecodeArgs a) {
       dst[D + 1] = den[g];
     }
   }
+  pdl_wait();
 }
 
 template <int D>
